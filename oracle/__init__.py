@@ -1,0 +1,253 @@
+"""The correctness oracle: a plain, slow, single-threaded CPU restatement of
+indexed 64-bit rANS coding (C core in rans_oracle.c, stream layout here in
+numpy).
+
+TEST INFRASTRUCTURE ONLY.  Only tests/, ``__graft_entry__.smoke()`` and the
+bench's ``cpu_baseline`` / ``--impl reference`` legs may import this package.
+It shares no code with ``rans_entropy_coding_b200`` and never imports it.
+
+Sources (page title, then section):
+  * "kompressor" README -- Why: the symbol array is cut into independent
+    chunks with no cross-chunk dependency (the rayon parallelism); Getting
+    Started: "chunks=24".
+  * "torch_ans 0.3.0" -- Low-level API (cdfs, cdfs_sizes, offsets, one index
+    per symbol); rans_stream_to_byte_strings (streams serialised as byte
+    strings).
+
+Readings where the pages are silent:
+  * contiguous chunking: stream k covers [k*ceil(N/S), min((k+1)*ceil(N/S), N));
+  * tiled chunking of an NCHW tensor: streams ordered (b, channel group,
+    tile row, tile column); symbols inside a stream in (channel, row, column)
+    order; edge tiles are partial;
+  * one index per ``index_block`` consecutive elements of the flattened
+    tensor: element p uses indexes[p // index_block];
+  * the container is the streams' bytes concatenated, with uint64 offsets
+    (S + 1 entries, offsets[0] = 0).
+
+Parity status: every function here is pinned (tests/test_oracle_*.py).
+Byte-exactness against CompressAI itself is unpinned: no CompressAI output is
+available to compare against.
+"""
+import ctypes
+import os
+
+import numpy as np
+
+from . import build as _build
+
+OK = 0
+ERR_ARG = -1
+ERR_INDEX = -2
+ERR_ZERO_FREQ = -3
+ERR_RANGE = -4
+ERR_CAPACITY = -5
+ERR_CORRUPT = -6
+
+_lib = None
+
+
+def lib():
+    global _lib
+    if _lib is None:
+        path = _build.build()
+        L = ctypes.CDLL(path)
+        P = ctypes.c_void_p
+        i32, i64, f64 = ctypes.c_int32, ctypes.c_int64, ctypes.c_double
+        L.orc_pmf_to_cdf.argtypes = [P, ctypes.c_int, P]
+        L.orc_pmf_to_cdf.restype = ctypes.c_int
+        L.orc_gaussian_multiplier.argtypes = [f64]
+        L.orc_gaussian_multiplier.restype = f64
+        L.orc_gaussian_center.argtypes = [ctypes.c_float, f64, P]
+        L.orc_gaussian_center.restype = ctypes.c_int
+        L.orc_build_cdfs_from_scales.argtypes = [P, ctypes.c_int, f64, P, ctypes.c_int, P, P]
+        L.orc_build_cdfs_from_scales.restype = ctypes.c_int
+        L.orc_build_cdfs_from_pmfs.argtypes = [P, ctypes.c_int, ctypes.c_int, P, P, P,
+                                               ctypes.c_int, P]
+        L.orc_build_cdfs_from_pmfs.restype = ctypes.c_int
+        L.orc_encode_stream.argtypes = [P, P, i64, P, ctypes.c_int, ctypes.c_int, P, P,
+                                        ctypes.c_int, P, i64]
+        L.orc_encode_stream.restype = i64
+        L.orc_decode_stream.argtypes = [P, i64, P, i64, P, ctypes.c_int, ctypes.c_int, P, P,
+                                        ctypes.c_int, P]
+        L.orc_decode_stream.restype = ctypes.c_int
+        del i32
+        _lib = L
+    return _lib
+
+
+class OracleError(RuntimeError):
+    def __init__(self, status, what=""):
+        super().__init__("oracle status %d %s" % (status, what))
+        self.status = status
+
+
+def _ptr(a):
+    return a.ctypes.data_as(ctypes.c_void_p) if a is not None else None
+
+
+# ------------------------------------------------------------------ tables --
+def pmf_to_cdf(pmf):
+    """pmf (tail mass last) -> quantised cdf row of len(pmf) + 1 entries."""
+    p = np.ascontiguousarray(pmf, dtype=np.float32)
+    out = np.zeros(p.size + 1, dtype=np.int32)
+    st = lib().orc_pmf_to_cdf(_ptr(p), p.size, _ptr(out))
+    if st:
+        raise OracleError(st, "pmf_to_cdf")
+    return out
+
+
+def gaussian_multiplier(tail_mass=1e-9):
+    return lib().orc_gaussian_multiplier(tail_mass)
+
+
+def gaussian_center(scale, tail_mass=1e-9):
+    c = np.zeros(1, dtype=np.int32)
+    st = lib().orc_gaussian_center(ctypes.c_float(scale), tail_mass, _ptr(c))
+    if st:
+        raise OracleError(st, "gaussian_center")
+    return int(c[0])
+
+
+def build_cdfs_from_scales(scales, tail_mass=1e-9, Lmax=None):
+    """Gaussian rows -> (cdfs[K, Lmax] int32, lengths[K], offsets[K])."""
+    s = np.ascontiguousarray(scales, dtype=np.float32)
+    K = s.size
+    if Lmax is None:
+        Lmax = max(2 * gaussian_center(float(v), tail_mass) + 3 for v in s)
+    cdfs = np.zeros((K, Lmax), dtype=np.int32)
+    lengths = np.zeros(K, dtype=np.int32)
+    offsets = np.zeros(K, dtype=np.int32)
+    st = lib().orc_build_cdfs_from_scales(_ptr(s), K, tail_mass, _ptr(cdfs), Lmax,
+                                          _ptr(lengths), _ptr(offsets))
+    if st:
+        raise OracleError(st, "build_cdfs_from_scales")
+    return cdfs, lengths, offsets
+
+
+def build_cdfs_from_pmfs(pmfs, pmf_lengths, tail_mass, Lmax=None):
+    """pmf rows -> (cdfs[K, Lmax] int32, lengths[K])."""
+    p = np.ascontiguousarray(pmfs, dtype=np.float32)
+    K, S = p.shape
+    pl = np.ascontiguousarray(pmf_lengths, dtype=np.int32)
+    tm = np.ascontiguousarray(tail_mass, dtype=np.float32)
+    if Lmax is None:
+        Lmax = int(pl.max()) + 2
+    cdfs = np.zeros((K, Lmax), dtype=np.int32)
+    lengths = np.zeros(K, dtype=np.int32)
+    st = lib().orc_build_cdfs_from_pmfs(_ptr(p), K, S, _ptr(pl), _ptr(tm), _ptr(cdfs),
+                                        Lmax, _ptr(lengths))
+    if st:
+        raise OracleError(st, "build_cdfs_from_pmfs")
+    return cdfs, lengths
+
+
+# ----------------------------------------------------------------- streams --
+def encode_stream(symbols, rows, cdfs, lengths, offsets, W=1):
+    """Codes one stream; returns its bytes as a uint8 array."""
+    s = np.ascontiguousarray(symbols, dtype=np.int64)
+    r = np.ascontiguousarray(rows, dtype=np.int32)
+    c = np.ascontiguousarray(cdfs, dtype=np.int32)
+    ln = np.ascontiguousarray(lengths, dtype=np.int32)
+    of = np.ascontiguousarray(offsets, dtype=np.int32)
+    K, Lmax = c.shape
+    cap = 8 * W + 16 + 8 * s.size + 64
+    out = np.zeros(cap, dtype=np.uint8)
+    n = lib().orc_encode_stream(_ptr(s), _ptr(r), s.size, _ptr(c), K, Lmax, _ptr(ln),
+                                _ptr(of), W, _ptr(out), cap)
+    if n < 0:
+        raise OracleError(int(n), "encode_stream")
+    return out[:n].copy()
+
+
+def decode_stream(data, rows, cdfs, lengths, offsets, W=1):
+    """Decodes len(rows) symbols of one stream; returns int64 symbols."""
+    d = np.ascontiguousarray(data, dtype=np.uint8)
+    r = np.ascontiguousarray(rows, dtype=np.int32)
+    c = np.ascontiguousarray(cdfs, dtype=np.int32)
+    ln = np.ascontiguousarray(lengths, dtype=np.int32)
+    of = np.ascontiguousarray(offsets, dtype=np.int32)
+    K, Lmax = c.shape
+    out = np.zeros(r.size, dtype=np.int64)
+    st = lib().orc_decode_stream(_ptr(d), d.size, _ptr(r), r.size, _ptr(c), K, Lmax,
+                                 _ptr(ln), _ptr(of), W, _ptr(out))
+    if st:
+        raise OracleError(st, "decode_stream")
+    return out
+
+
+# ---------------------------------------------------------------- chunking --
+def stream_positions(n, chunking):
+    """Flat element positions of every stream, in coding order.
+
+    ``chunking`` is a dict: {"kind": "contig", "n_streams": S} |
+    {"kind": "explicit", "starts": [S+1 offsets]} |
+    {"kind": "tiled", "shape": (B, C, H, W), "cg": g, "th": th, "tw": tw}.
+    """
+    kind = chunking["kind"]
+    if kind == "contig":
+        S = int(chunking["n_streams"])
+        per = -(-n // S) if S > 0 else 0
+        out = []
+        for k in range(S):
+            a = min(k * per, n)
+            b = min((k + 1) * per, n)
+            out.append(np.arange(a, b, dtype=np.int64))
+        return out
+    if kind == "explicit":
+        st = np.asarray(chunking["starts"], dtype=np.int64)
+        return [np.arange(st[k], st[k + 1], dtype=np.int64) for k in range(st.size - 1)]
+    if kind == "tiled":
+        B, C, H, Wd = (int(v) for v in chunking["shape"])
+        cg, th, tw = int(chunking["cg"]), int(chunking["th"]), int(chunking["tw"])
+        assert B * C * H * Wd == n
+        out = []
+        for b in range(B):
+            for c0 in range(0, C, cg):
+                for h0 in range(0, H, th):
+                    for w0 in range(0, Wd, tw):
+                        cs = np.arange(c0, min(c0 + cg, C), dtype=np.int64)
+                        hs = np.arange(h0, min(h0 + th, H), dtype=np.int64)
+                        ws = np.arange(w0, min(w0 + tw, Wd), dtype=np.int64)
+                        pos = ((b * C + cs[:, None, None]) * H + hs[None, :, None]) * Wd \
+                            + ws[None, None, :]
+                        out.append(pos.reshape(-1))
+        return out
+    raise ValueError("unknown chunking kind %r" % kind)
+
+
+def _rows_for(positions, indexes, index_block):
+    return np.asarray(indexes, dtype=np.int32)[positions // index_block]
+
+
+def encode_with_indexes(symbols, indexes, cdfs, lengths, offsets, chunking, W=1,
+                        index_block=1, streams=None):
+    """Container encode: returns (bytes uint8[total], offsets uint64[S+1]).
+
+    ``streams`` optionally restricts the work to a subset of stream ids; the
+    result then holds those streams only (offsets over the subset)."""
+    flat = np.asarray(symbols).reshape(-1)
+    pos = stream_positions(flat.size, chunking)
+    ids = range(len(pos)) if streams is None else streams
+    parts, offs = [], [0]
+    for k in ids:
+        p = pos[k]
+        b = encode_stream(flat[p].astype(np.int64), _rows_for(p, indexes, index_block),
+                          cdfs, lengths, offsets, W)
+        parts.append(b)
+        offs.append(offs[-1] + b.size)
+    data = np.concatenate(parts) if parts else np.zeros(0, dtype=np.uint8)
+    return data, np.asarray(offs, dtype=np.uint64)
+
+
+def decode_with_indexes(data, stream_offsets, indexes, cdfs, lengths, offsets, chunking,
+                        n, W=1, index_block=1, dtype=np.int32):
+    """Container decode of n elements; returns a flat array of ``dtype``."""
+    pos = stream_positions(n, chunking)
+    out = np.zeros(n, dtype=np.int64)
+    so = np.asarray(stream_offsets, dtype=np.uint64)
+    d = np.asarray(data, dtype=np.uint8)
+    for k, p in enumerate(pos):
+        a, b = int(so[k]), int(so[k + 1])
+        out[p] = decode_stream(d[a:b], _rows_for(p, indexes, index_block), cdfs, lengths,
+                               offsets, W)
+    return out.astype(dtype)

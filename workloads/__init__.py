@@ -1,0 +1,170 @@
+"""Seeded synthetic inputs for the five coding workloads.
+
+Shared by the oracle side and the CUDA side of every test and of the bench:
+both code exactly these arrays.  This module holds none of the coder's
+arithmetic (no CDF quantisation, no rANS step); it only draws symbols, row
+indexes and the model-side inputs the coder starts from (a scale table or
+float pmfs).
+
+The pages measure on the latents of one 1920x1080 image run through CompressAI's
+mbt2018_mean model ("kompressor" README, Getting Started and Benchmarks: the y
+latent has 1,566,720 symbols and 64 CDF rows, the z latent 65,280 symbols).
+Those latents need trained weights that are not available, so the generators
+below stand in for them with the same shapes and row structure:
+
+  tiny   4,096 int32; 8 Gaussian rows (scales log-spaced 0.11..8); uniform
+         row per symbol; symbol = round(N(0, row scale)); about 1% forced far
+         past every row's coded range (|s| >= 65, so the bypass path carries
+         1-8 raw nibbles) plus INT32_MIN / INT32_MAX; 1 stream, W = 1.
+  z      128 x 17 x 30 int32 (NCHW, batch 1); one Laplace pmf row per channel,
+         b ~ U[0.3, 3]; symbols drawn from the channel's pmf; 32 contiguous
+         streams, W = 1.
+  y      192 x 68 x 120 int32; 64-row Gaussian scale table
+         exp(linspace(ln 0.11, ln 256, 64)); per-element scale log-uniform on
+         [0.11, 256]; row = the nearest table entry in log space; symbol =
+         round(N(0, element scale)); 24 contiguous streams, W = 1 or 32.
+  batch  16 y latents (image b drawn with seed 3000 + b), NCHW
+         [16, 192, 68, 120]; one stream per 64 x 64 spatial tile per group of
+         4 channels (3,072 streams), W = 32.
+  sweep  2^28 uint8 symbols; 16 Zipf rows p(k) ~ (k+1)^-s, s in
+         linspace(0.8, 1.6, 16), over 256 symbols with no tail; one row per
+         4,096-symbol block; 8,192 contiguous streams, W = 32.
+
+Seeds: numpy Generator(PCG64(1000 * workload_number + image)).
+"""
+import math
+
+import numpy as np
+
+SCALE_MIN = 0.11
+SCALE_MAX_Y = 256.0
+N_ROWS_Y = 64
+Y_SHAPE = (192, 68, 120)
+Z_SHAPE = (128, 17, 30)
+
+
+def _rng(seed):
+    return np.random.Generator(np.random.PCG64(seed))
+
+
+def log_spaced_scales(lo, hi, k):
+    """k scales log-spaced from lo to hi, as float32."""
+    return np.exp(np.linspace(math.log(lo), math.log(hi), k)).astype(np.float32)
+
+
+def _sample_from_pmfs(rng, cum, rows):
+    """Draws one value per entry of ``rows`` from that row's distribution;
+    ``cum`` holds each row's running sum of probabilities (float64)."""
+    u = rng.random(rows.size)
+    out = np.empty(rows.size, dtype=np.int64)
+    for r in np.unique(rows):
+        sel = np.nonzero(rows == r)[0]
+        c = cum[r]
+        out[sel] = np.minimum(np.searchsorted(c, u[sel] * c[-1], side="right"), c.size - 1)
+    return out
+
+
+def tiny(seed=0, n=4096):
+    rng = _rng(seed)
+    scales = log_spaced_scales(SCALE_MIN, 8.0, 8)
+    idx = rng.integers(0, 8, size=n).astype(np.int32)
+    sym = np.rint(rng.standard_normal(n) * scales[idx].astype(np.float64))
+    force = rng.random(n) < 0.01
+    sign = np.where(rng.random(n) < 0.5, -1.0, 1.0)
+    k = np.floor(2.0 ** rng.uniform(0.0, 30.0, size=n))
+    sym = np.where(force, sign * (65.0 + k), sym)
+    sym = sym.astype(np.int64)
+    sym[1] = np.iinfo(np.int32).min
+    sym[2] = np.iinfo(np.int32).max
+    return dict(name="tiny", symbols=sym.astype(np.int32), indexes=idx, scales=scales,
+                tail_mass=1e-9, chunking=dict(kind="contig", n_streams=1), W=1,
+                index_block=1)
+
+
+def z_latent(seed=1000):
+    rng = _rng(seed)
+    C, H, Wd = Z_SHAPE
+    b = rng.uniform(0.3, 3.0, size=C)
+    centers = np.ceil(b * math.log(1e9) - 0.5).astype(np.int64)
+    S = int(2 * centers.max() + 1)
+    pmfs = np.zeros((C, S), dtype=np.float32)
+    pmf_lengths = (2 * centers + 1).astype(np.int32)
+    tails = np.zeros(C, dtype=np.float32)
+    cum = []
+    for c in range(C):
+        k = np.arange(-centers[c], centers[c] + 1, dtype=np.float64)
+        lap = lambda x: np.where(x < 0, 0.5 * np.exp(x / b[c]), 1.0 - 0.5 * np.exp(-x / b[c]))
+        p = lap(k + 0.5) - lap(k - 0.5)
+        pmfs[c, :p.size] = p.astype(np.float32)
+        tails[c] = np.float32(2.0 * lap(np.array(-centers[c] - 0.5)))
+        cum.append(np.cumsum(p))
+    rows = np.repeat(np.arange(C, dtype=np.int32), H * Wd)
+    v = _sample_from_pmfs(rng, cum, rows)
+    sym = (v - centers[rows]).astype(np.int32)
+    return dict(name="z", symbols=sym.reshape(1, C, H, Wd), indexes=rows, pmfs=pmfs,
+                pmf_lengths=pmf_lengths, tail=tails,
+                offsets=(-centers).astype(np.int32),
+                chunking=dict(kind="contig", n_streams=32), W=1, index_block=1)
+
+
+def _y_image(seed):
+    rng = _rng(seed)
+    n = int(np.prod(Y_SHAPE))
+    lo, hi = math.log(SCALE_MIN), math.log(SCALE_MAX_Y)
+    u = rng.uniform(lo, hi, size=n)
+    step = (hi - lo) / (N_ROWS_Y - 1)
+    idx = np.clip(np.rint((u - lo) / step), 0, N_ROWS_Y - 1).astype(np.int32)
+    sym = np.rint(rng.standard_normal(n) * np.exp(u))
+    sym = np.clip(sym, np.iinfo(np.int32).min, np.iinfo(np.int32).max).astype(np.int32)
+    return sym, idx
+
+
+def y_latent(seed=2000, W=1):
+    sym, idx = _y_image(seed)
+    return dict(name="y", symbols=sym.reshape((1,) + Y_SHAPE), indexes=idx,
+                scales=log_spaced_scales(SCALE_MIN, SCALE_MAX_Y, N_ROWS_Y), tail_mass=1e-9,
+                chunking=dict(kind="contig", n_streams=24), W=W, index_block=1)
+
+
+def y_batch(n_images=16, first_image=0, cg=4, th=64, tw=64):
+    """Images first_image .. first_image + n_images - 1 of the batch."""
+    syms, idxs = [], []
+    for b in range(first_image, first_image + n_images):
+        s, i = _y_image(3000 + b)
+        syms.append(s)
+        idxs.append(i)
+    C, H, Wd = Y_SHAPE
+    return dict(name="batch", symbols=np.concatenate(syms).reshape(n_images, C, H, Wd),
+                indexes=np.concatenate(idxs),
+                scales=log_spaced_scales(SCALE_MIN, SCALE_MAX_Y, N_ROWS_Y), tail_mass=1e-9,
+                chunking=dict(kind="tiled", shape=(n_images, C, H, Wd), cg=cg, th=th, tw=tw),
+                W=32, index_block=1)
+
+
+def sweep(log2_n=28, seed=4000, n_streams=None, block=4096, n_rows=16):
+    n = 1 << log2_n
+    rng = _rng(seed)
+    s = np.linspace(0.8, 1.6, n_rows)
+    k = np.arange(1, 257, dtype=np.float64)
+    pmfs = np.zeros((n_rows, 256), dtype=np.float32)
+    cum = []
+    for r in range(n_rows):
+        p = k ** (-s[r])
+        p /= p.sum()
+        pmfs[r] = p.astype(np.float32)
+        cum.append(np.cumsum(p))
+    nblk = -(-n // block)
+    idx = rng.integers(0, n_rows, size=nblk).astype(np.int32)
+    sym = np.empty(n, dtype=np.uint8)
+    chunk = 1 << 22
+    for a in range(0, n, chunk):
+        b = min(a + chunk, n)
+        rows = np.repeat(idx[a // block: -(-b // block)], block)[: b - a]
+        sym[a:b] = _sample_from_pmfs(rng, cum, rows).astype(np.uint8)
+    if n_streams is None:
+        n_streams = max(1, n // 32768)
+    return dict(name="sweep", symbols=sym, indexes=idx, pmfs=pmfs,
+                pmf_lengths=np.full(n_rows, 256, dtype=np.int32),
+                tail=np.zeros(n_rows, dtype=np.float32),
+                offsets=np.zeros(n_rows, dtype=np.int32),
+                chunking=dict(kind="contig", n_streams=n_streams), W=32, index_block=block)
