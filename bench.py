@@ -1,0 +1,391 @@
+#!/usr/bin/env python
+"""Throughput of librans_b200 on the 16-image 1080p latent batch.
+
+One step = the whole coding path over one batch: the 64 Gaussian CDF rows
+built from the scale table, the coder's tables prepared, every stream encoded
+(with compaction) and decoded, on one GPU per rank.  Workload: 16 synthetic
+y latents [16, 192, 68, 120] int32 (25,067,520 symbols), one stream per
+64 x 64 spatial tile per group of 4 channels (3,072 streams), 32 interleaved
+states per stream.  Ranks shard by image (weak scaling: every rank codes its
+own 16 images; no collective on the data path).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Prints one JSON line (rank 0).  Inputs (200 MB of symbols and indexes) are
+larger than the 126 MB L2, so no flush is needed between steps.
+"""
+import argparse
+import concurrent.futures as cf
+import json
+import os
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import workloads as WL  # noqa: E402
+
+METRIC = ("rANS encode & decode Gsymbol/s and HBM GB/s (fraction of B200 roofline), 1 GPU")
+UNIT = "Gsymbol/s"
+WORKLOAD = "batch16_y1080p: 16x192x68x120 int32, 64 Gaussian rows, tiles 64x64 x 4 channels, W=32"
+N_IMAGES = 16
+CLOCK_FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+                "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+                "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--group", type=int, default=4, help="channels per stream")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-clocks", action="store_true")
+    ap.add_argument("--traffic-json", default=os.path.join(ROOT, "profiles", "traffic.json"))
+    return ap.parse_args()
+
+
+def dist_setup(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+
+        import torch
+        import torch.distributed as dist
+        backend = "gloo" if args.impl == "reference" else "nccl"
+        if backend == "nccl":
+            torch.cuda.set_device(local)
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(v, world, device=None):
+    if world == 1:
+        return v
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([v], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+class ClockSampler:
+    """nvidia-smi samples of SM clock and throttle reasons while running."""
+
+    def __init__(self, gpu_index, enabled=True):
+        self.gpu = gpu_index
+        self.enabled = enabled
+        self.proc = None
+
+    def __enter__(self):
+        if self.enabled:
+            self.f = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+            try:
+                self.proc = subprocess.Popen(
+                    ["nvidia-smi", "-i", str(self.gpu), "--query-gpu=" + CLOCK_FIELDS,
+                     "--format=csv,noheader,nounits", "-lms", "100"], stdout=self.f,
+                    stderr=subprocess.DEVNULL)
+                time.sleep(0.3)
+            except OSError:
+                self.proc = None
+        return self
+
+    def __exit__(self, *a):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        if self.proc is None:
+            return None
+        self.f.flush()
+        rows = []
+        with open(self.f.name) as fh:
+            for line in fh:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) >= 9:
+                    rows.append(parts)
+        os.unlink(self.f.name)
+        if not rows:
+            return None
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i] == "Active"})
+        return {"sm_mhz": float(np.median(sm)) if sm else None,
+                "sm_max_mhz": max(mx) if mx else None, "reasons": reasons,
+                "samples": len(rows)}
+
+
+def load_inputs(rank, group):
+    w = WL.y_batch(n_images=N_IMAGES, first_image=N_IMAGES * rank, cg=group)
+    return w
+
+
+# --------------------------------------------------------- CPU oracle leg --
+def oracle_sample(w, max_streams, workers):
+    """Oracle encode + decode of the first max_streams streams of the batch,
+    one stream per call, spread over `workers` threads (the C oracle runs
+    without the GIL).  Returns (symbols coded, seconds)."""
+    import oracle as O
+    c, l, o = O.build_cdfs_from_scales(w["scales"], w["tail_mass"])
+    flat = np.asarray(w["symbols"]).reshape(-1)
+    pos = O.stream_positions(flat.size, w["chunking"])[:max_streams]
+    idx = np.asarray(w["indexes"], dtype=np.int32)
+
+    def one(p):
+        s = flat[p].astype(np.int64)
+        r = idx[p]
+        b = O.encode_stream(s, r, c, l, o, W=32)
+        back = O.decode_stream(b, r, c, l, o, W=32)
+        assert np.array_equal(back, s)
+        return p.size
+
+    t = time.perf_counter()
+    with cf.ThreadPoolExecutor(max_workers=workers) as ex:
+        n = sum(ex.map(one, pos))
+    return n, time.perf_counter() - t
+
+
+def run_reference(args, world, rank):
+    """--impl reference: the oracle as it stands on the host cores."""
+    if rank != 0:
+        return
+    w = load_inputs(0, args.group)
+    workers = os.cpu_count() or 1
+    max_streams = 768     # 4 of the 16 images per step: a bounded sample
+    for _ in range(args.warmup):
+        oracle_sample(w, 48, workers)
+    tot_n, tot_t = 0, 0.0
+    for _ in range(args.steps):
+        n, t = oracle_sample(w, max_streams, workers)
+        tot_n += n
+        tot_t += t
+    value = tot_n / tot_t / 1e9
+    sample = ("oracle encode+decode of streams 0..767 (images 0-3, %d symbols) per step, "
+              "one stream per call over %d threads" % (tot_n // max(args.steps, 1), workers))
+    print(json.dumps({
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": 1,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * tot_t / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "u64",
+        "data": "synthetic", "config": {"workload": WORKLOAD, "streams_per_step": max_streams},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": workers, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }), flush=True)
+
+
+# --------------------------------------------------------------- GPU leg --
+def run_ours(args, world, rank, local):
+    import torch
+
+    import rans_entropy_coding_b200 as rb
+
+    rb.lib()
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    w = load_inputs(rank, args.group)
+    sym_np = np.ascontiguousarray(np.asarray(w["symbols"]).reshape(-1))
+    idx_np = np.ascontiguousarray(w["indexes"], dtype=np.int32)
+    n = sym_np.size
+    sym = torch.from_numpy(sym_np).to(dev)
+    idx = torch.from_numpy(idx_np).to(dev)
+    scales = torch.from_numpy(w["scales"]).to(dev)
+    tail = w["tail_mass"]
+    ch = rb.Chunking.from_spec(w["chunking"], 32)
+    S = rb.rans_num_streams(ch, n)
+
+    # tables: sized once; rebuilt inside every step
+    cdfs, lengths, offsets = rb.Tables.build_from_scales(scales, tail)
+    K, Lmax = cdfs.shape
+    tables = rb.Tables(cdfs, lengths, offsets)
+    blob = tables.blob
+    ws = rb.Workspaces(ch, n, dev)
+    dec = torch.empty_like(sym)
+    stream = torch.cuda.current_stream()
+
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+
+    def step(e=None):
+        if e: e[0].record(stream)
+        rb.check(rb.rans_build_cdfs_from_scales(scales, tail, cdfs, lengths, offsets), "cdfs")
+        rb.check(rb.rans_tables_prepare(cdfs, lengths, offsets, blob, tables.c), "prepare")
+        if e: e[1].record(stream)
+        rb.check(rb.rans_encode_with_indexes(sym, idx, n, tables, ch, ws.out, ws.offsets,
+                                             ws.enc), "encode")
+        if e: e[2].record(stream)
+        rb.check(rb.rans_decode_with_indexes(ws.out, ws.offsets, idx, n, tables, ch, dec,
+                                             ws.dec), "decode")
+        if e: e[3].record(stream)
+
+    for _ in range(max(args.warmup, 0)):
+        step()
+    torch.cuda.synchronize()
+    rb.check(rb.rans_get_status(ws.enc), "encode status")
+    rb.check(rb.rans_get_status(ws.dec), "decode status")
+    assert torch.equal(dec, sym), "round trip failed"
+    barrier(world)
+
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local, enabled=not args.no_clocks) as clk:
+        torch.cuda.synchronize()
+        barrier(world)
+        t0.record(stream)
+        for i in range(args.steps):
+            step(ev[i])
+        t1.record(stream)
+        torch.cuda.synchronize()
+        barrier(world)
+    elapsed_ms = max_over_ranks(t0.elapsed_time(t1), world, dev)
+    clocks = clk.summary()
+    rb.check(rb.rans_get_status(ws.enc), "encode status")
+    rb.check(rb.rans_get_status(ws.dec), "decode status")
+    assert torch.equal(dec, sym), "round trip failed"
+
+    tab_ms = float(np.mean([e[0].elapsed_time(e[1]) for e in ev]))
+    enc_ms = float(np.mean([e[1].elapsed_time(e[2]) for e in ev]))
+    dec_ms = float(np.mean([e[2].elapsed_time(e[3]) for e in ev]))
+    comp = int(ws.offsets[-1].item())
+    sym_b = sym.element_size()
+    alg_enc = n * (sym_b + 4) + comp     # symbols + indexes read, bytes written
+    alg_dec = n * (sym_b + 4) + comp     # bytes + indexes read, symbols written
+    peaks = {}
+    pk_path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(pk_path):
+        peaks = json.load(open(pk_path))
+    peak = peaks.get("hbm_gbs")
+    peak_src = "measured" if peak else "fallback"
+    peak = peak or 6650.0
+    enc_gbs = alg_enc / (enc_ms * 1e-3) / 1e9
+    dec_gbs = alg_dec / (dec_ms * 1e-3) / 1e9
+    dominant = "decode" if dec_ms >= enc_ms else "encode"
+    traffic = None
+    if os.path.exists(args.traffic_json):
+        try:
+            tj = json.load(open(args.traffic_json))
+            traffic = tj.get(dominant, {}).get("bytes_per_launch")
+        except (OSError, ValueError):
+            traffic = None
+    ach = dec_gbs if dominant == "decode" else enc_gbs
+    total_syms = n * world
+    ms_per_step = elapsed_ms / args.steps
+    value = total_syms / (ms_per_step * 1e-3) / 1e9
+
+    # end to end through the public API with host buffers
+    e2e = None
+    if not args.no_e2e:
+        h_sym = torch.from_numpy(sym_np).pin_memory()
+        h_idx = torch.from_numpy(idx_np).pin_memory()
+        h_out = torch.empty(ws.out.numel(), dtype=torch.uint8).pin_memory()
+        h_dec = torch.empty(n, dtype=torch.int32).pin_memory()
+        d_sym = torch.empty_like(sym)
+        d_idx = torch.empty_like(idx)
+        h2d = d2h = 0
+
+        def e2e_step():
+            nonlocal h2d, d2h
+            d_sym.copy_(h_sym, non_blocking=True)
+            d_idx.copy_(h_idx, non_blocking=True)
+            rb.check(rb.rans_build_cdfs_from_scales(scales, tail, cdfs, lengths, offsets))
+            rb.check(rb.rans_tables_prepare(cdfs, lengths, offsets, blob, tables.c))
+            rb.check(rb.rans_encode_with_indexes(d_sym, d_idx, n, tables, ch, ws.out,
+                                                 ws.offsets, ws.enc))
+            total = int(ws.offsets[-1].item())
+            h_out[:total].copy_(ws.out[:total], non_blocking=True)
+            rb.check(rb.rans_decode_with_indexes(ws.out, ws.offsets, d_idx, n, tables, ch, dec,
+                                                 ws.dec))
+            h_dec.copy_(dec, non_blocking=True)
+            torch.cuda.synchronize()
+            h2d = n * sym_b + n * 4
+            d2h = total + 8 * (S + 1) + n * sym_b
+
+        for _ in range(2):
+            e2e_step()
+        torch.cuda.synchronize()
+        barrier(world)
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        ke = max(3, min(args.steps, 10))
+        a.record(stream)
+        for _ in range(ke):
+            e2e_step()
+        b.record(stream)
+        torch.cuda.synchronize()
+        e_ms = max_over_ranks(a.elapsed_time(b), world, dev) / ke
+        assert torch.equal(h_dec, torch.from_numpy(sym_np)), "e2e round trip failed"
+        e2e = {"value": total_syms / (e_ms * 1e-3) / 1e9, "unit": UNIT,
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        workers = os.cpu_count() or 1
+        ns, ts = oracle_sample(w, 768, workers)
+        cpu = {"value": ns / ts / 1e9, "unit": UNIT, "cores": workers, "kind": "oracle",
+               "sample": "oracle encode+decode of streams 0..767 (images 0-3, %d symbols), "
+                         "one stream per call over %d threads" % (ns, workers)}
+
+    launches_per_step = 1 + 2 + 3 + 1   # rows, prepare (pack, slots), enc+scan+copy, dec
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "u64",
+            "data": "synthetic",
+            "config": {"workload": WORKLOAD, "symbols_per_gpu": n, "streams_per_gpu": S,
+                       "channel_group": args.group, "interleave": 32, "rows": K,
+                       "lmax": Lmax, "parallelism": "shard-by-image x%d" % world,
+                       "l2": "inputs larger than L2 (%d MB read per encode)" %
+                             (n * (sym_b + 4) // 2**20)},
+            "encode": {"ms": enc_ms, "gsym_s": n / enc_ms / 1e6, "GBps": enc_gbs,
+                       "frac_hbm": enc_gbs / peak, "alg_bytes": alg_enc},
+            "decode": {"ms": dec_ms, "gsym_s": n / dec_ms / 1e6, "GBps": dec_gbs,
+                       "frac_hbm": dec_gbs / peak, "alg_bytes": alg_dec},
+            "tables": {"ms": tab_ms},
+            "compressed_bytes": comp, "bits_per_symbol": 8.0 * comp / n,
+            "roofline": {"bound": "hbm", "achieved": ach, "peak": peak, "unit": "GB/s",
+                         "frac": ach / peak, "traffic": traffic, "kernel": dominant,
+                         "peak_source": peak_src},
+            "cpu_baseline": cpu,
+            "e2e": e2e,
+            "clocks": clocks,
+            "gpu_launches": launches_per_step * args.steps,
+        }
+        print(json.dumps(line), flush=True)
+
+
+def main():
+    args = parse()
+    world, rank, local = dist_setup(args)
+    try:
+        if args.impl == "reference":
+            run_reference(args, world, rank)
+        else:
+            run_ours(args, world, rank, local)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,283 @@
+/*
+ * rans_b200.h -- C ABI of librans_b200: indexed 64-bit rANS entropy coding on
+ * one NVIDIA B200 (sm_100a).
+ *
+ * What is coded (sources are page title + section):
+ *   - rANS with a 64-bit state, 32-bit renormalisation words and 16-bit CDF
+ *     precision ("torch_ans 0.3.0", Usage, variants table, rans64 row;
+ *     "kompressor" README, Credits: CompressAI's ryg_rans-style coder).
+ *   - One CDF row per symbol, chosen through an index array; rows given as
+ *     cdfs / cdf_lengths / offsets ("torch_ans 0.3.0", Low-level API,
+ *     rans_push and rans_pop).
+ *   - Symbols outside a row's coded range [offset, offset + cdf_length - 2)
+ *     take the row's escape bucket and are then sent as a zig-zag raw value
+ *     in 4-bit bypass pieces (same section, "Range limit"; "kompressor"
+ *     README, Correctness: the bypass path).
+ *   - Many independent streams: contiguous chunks or spatial tiles ("kompressor"
+ *     README, Why: zero cross-chunk dependency), each coded with W = 1 state
+ *     or W = 32 interleaved states sharing one word stream, lane i mod 32
+ *     ("torch_ans 0.3.0", Usage legend and FAQ: interleaved states share one
+ *     bitstream; the 32-way form maps the states onto the lanes of a warp).
+ *   - pmf -> quantised CDF rows ("torch_ans 0.3.0", High-level API,
+ *     init_params) and Gaussian rows from a scale table ("kompressor" README,
+ *     Getting Started: 64 CDF rows for the y latent).
+ *
+ * Fixed format: state bound L = 2^31 (initial encoder state, final decoder
+ * state), symbol op renormalises when x >= 2^47 * freq, bypass op when
+ * x >= 2^59; the stream of one chunk is its W lane states (low word, high
+ * word; lane 0 first) followed by the renormalisation words in the order the
+ * decoder consumes them, all little-endian 32-bit words.  The escape raw value
+ * is 2(v - maxv) above the range and -2v - 1 below it; it is sent as a count
+ * of 4-bit pieces (in pieces of at most 15, where 15 means "more follows"),
+ * then the pieces, least significant first.
+ *
+ * Conventions for every entry point:
+ *   - All array pointers are DEVICE pointers unless a name says host_.
+ *   - The caller allocates every buffer; the library never allocates device
+ *     memory (sizes come from the *_bytes queries).
+ *   - `stream` is a cudaStream_t (NULL = the legacy default stream); all work
+ *     is enqueued on it.  Only rans_tables_prepare and rans_get_status
+ *     synchronise.
+ *   - Argument errors detectable on the host return immediately with a
+ *     negative status.  Errors found on the device (bad index, zero-width
+ *     bucket, raw value beyond 60 bits, a malformed or truncated stream, output
+ *     capacity) are recorded in the workspace's status word, first error wins,
+ *     and are returned by rans_get_status; the outputs are then undefined.
+ *     No kernel traps or asserts.
+ */
+#ifndef RANS_B200_H
+#define RANS_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define RANS_PRECISION 16
+#define RANS_BYPASS_BITS 4
+
+typedef enum rans_status {
+    RANS_OK = 0,
+    RANS_ERR_ARG = -1,        /* invalid argument (host-side or a bad chunking) */
+    RANS_ERR_INDEX = -2,      /* an index outside [0, K) */
+    RANS_ERR_ZERO_FREQ = -3,  /* a symbol maps to a bucket of width 0 */
+    RANS_ERR_RANGE = -4,      /* an escape raw value of 2^60 or more */
+    RANS_ERR_CAPACITY = -5,   /* an output or table buffer is too small */
+    RANS_ERR_CORRUPT = -6,    /* a stream is truncated, too long or inconsistent */
+    RANS_ERR_CUDA = -7,       /* a CUDA runtime call failed */
+    RANS_ERR_TABLE = -8,      /* a malformed CDF row or pmf */
+    RANS_ERR_TIMEOUT = -9     /* a bounded device wait gave up */
+} rans_status;
+
+/* Symbol element types. */
+enum { RANS_SYM_INT32 = 0, RANS_SYM_UINT8 = 1, RANS_SYM_INT16 = 2 };
+
+/* Chunking kinds. */
+enum { RANS_CHUNK_CONTIG = 0, RANS_CHUNK_EXPLICIT = 1, RANS_CHUNK_TILED = 2 };
+
+/*
+ * How the n symbols are cut into streams, and how indexes map to symbols.
+ *   CONTIG:   n_streams streams; stream k covers elements
+ *             [k*ceil(n/S), min((k+1)*ceil(n/S), n)) (trailing streams may be
+ *             empty).
+ *   EXPLICIT: n_streams streams; stream k covers [stream_starts[k],
+ *             stream_starts[k+1]) -- stream_starts is a device array of
+ *             n_streams + 1 non-decreasing element offsets within [0, n].
+ *   TILED:    the symbols are an NCHW tensor shape[0..3] = (B, C, H, W);
+ *             one stream per (image, group of `group` channels, tile of
+ *             tile_h x tile_w), ordered (b, g, tile row, tile column); inside a
+ *             stream the elements go (channel, row, column); edge tiles are
+ *             partial.  n must equal B*C*H*W.
+ *   interleave: 1 or 32 states per stream.
+ *   index_block: element p (flat position in the symbol array) uses row
+ *             indexes[p / index_block]; 1 = one index per symbol; must be a
+ *             power of two.
+ */
+typedef struct rans_chunking {
+    int32_t kind;
+    int32_t interleave;
+    int64_t n_streams;
+    const int64_t *stream_starts;
+    int64_t shape[4];
+    int64_t group, tile_h, tile_w;
+    int64_t index_block;
+} rans_chunking;
+
+/*
+ * A prepared table set, filled by rans_tables_prepare.  `blob` is the
+ * caller's device buffer; the other fields describe its layout and are read
+ * by the encoder and decoder.  One table set serves both directions and every
+ * chunking.  Treat the fields as opaque.
+ */
+typedef struct rans_tables {
+    void *blob;
+    uint64_t blob_bytes;
+    int32_t K;              /* rows */
+    int32_t max_buckets;    /* longest row's bucket count (cdf_length - 1) */
+    int64_t n_buckets;      /* all rows' buckets */
+    int64_t n_slots;        /* decode lookup slots */
+    uint32_t meta_bytes, bucket_bytes, slot_bytes;  /* section sizes (16-B padded) */
+    int32_t enc_in_smem;    /* 1: encode stages meta + buckets in shared memory */
+    int32_t dec_in_smem;    /* 1: decode stages all three sections */
+    int32_t device;         /* CUDA device the blob lives on */
+} rans_tables;
+
+/* ------------------------------------------------------------ status ---- */
+
+/* A short English description of a status code (static storage). */
+const char *rans_status_string(int status);
+
+/* Library version: major * 10000 + minor * 100 + patch. */
+int rans_version(void);
+
+/* ------------------------------------------------------- CDF tables ---- */
+
+/*
+ * Lengths and offsets of K Gaussian rows ("kompressor" README, Getting
+ * Started: the y latent's 64 rows; "Benchmark notes", section 4: 200512 table
+ * entries).  For tail mass t, m = -Phi^-1(t/2); row r has centre
+ * c = ceil(scales[r] * m), cdf_length 2c + 3 and offset -c.
+ *   scales:      device float[K], each > 0 and finite.
+ *   cdf_lengths: device int32[K] out; a row that cannot be built gets a
+ *                negative status instead of its length.
+ *   offsets:     device int32[K] out.
+ * Use it to size Lmax before rans_build_cdfs_from_scales.  Asynchronous.
+ */
+int rans_gaussian_lengths(const float *scales, int32_t K, double tail_mass,
+                          int32_t *cdf_lengths, int32_t *offsets, void *stream);
+
+/*
+ * K Gaussian CDF rows.  Row r's pmf is Phi((0.5-|k|)/s) - Phi((-0.5-|k|)/s)
+ * for k = -c..c (Phi in double, cast to float), followed by the tail mass
+ * 2 Phi((-0.5-c)/s); the pmf is quantised as in rans_build_cdfs_from_pmfs.
+ *   cdfs: device int32[K][Lmax] out; entries past a row's length are 0.
+ *   cdf_lengths, offsets: device int32[K] out (as rans_gaussian_lengths);
+ *   a row longer than Lmax, or one that cannot be quantised, gets a negative
+ *   status as its length.  Asynchronous.
+ */
+int rans_build_cdfs_from_scales(const float *scales, int32_t K, double tail_mass,
+                                int32_t *cdfs, int32_t Lmax, int32_t *cdf_lengths,
+                                int32_t *offsets, void *stream);
+
+/*
+ * K CDF rows from pmfs ("torch_ans 0.3.0", High-level API, init_params; FAQ:
+ * rows are increasing positive integers up to 2^precision).  Row r takes
+ * pmf_lengths[r] probabilities pmfs[r*pmf_stride ...] and then tail_mass[r];
+ * each is scaled by 2^16 and rounded half away from zero, the running sum is
+ * rescaled to floor(2^16 c / total), and every empty bucket then takes one
+ * unit from the narrowest bucket wider than 1 (the first such on ties) --
+ * scanning empty buckets in ascending order.
+ *   pmfs:        device float[K][pmf_stride].
+ *   pmf_lengths: device int32[K], each in [0, pmf_stride].
+ *   tail_mass:   device float[K].
+ *   cdfs:        device int32[K][Lmax] out (Lmax >= max pmf_length + 2).
+ *   cdf_lengths: device int32[K] out: pmf_length + 2, or a negative status for
+ *                a row that cannot be built (negative or non-finite
+ *                probability, total 0, nothing to steal from, too long).
+ * Offsets are the caller's (they come with the pmfs).  Asynchronous.
+ */
+int rans_build_cdfs_from_pmfs(const float *pmfs, int32_t K, int32_t pmf_stride,
+                              const int32_t *pmf_lengths, const float *tail_mass,
+                              int32_t *cdfs, int32_t Lmax, int32_t *cdf_lengths,
+                              void *stream);
+
+/* Upper bound on the blob size rans_tables_prepare needs for K rows of at
+ * most Lmax entries. */
+uint64_t rans_tables_bytes(int32_t K, int32_t Lmax);
+
+/*
+ * Validates CDF rows and lays out the coder's tables in `blob` (device,
+ * blob_bytes >= rans_tables_bytes(K, Lmax)): per-row metadata, every bucket's
+ * (start, width) packed in 32 bits, and a per-row lookup table mapping the
+ * top bits of a decoder state's low 16 bits to its bucket.  Each row must
+ * have 2 <= cdf_lengths[r] <= Lmax, cdf[0] = 0, cdf[len-1] = 65536 and
+ * strictly increasing entries; otherwise RANS_ERR_TABLE (or the negative
+ * length left by a builder).  Synchronous (reads back the K lengths and the
+ * validation status); fills *out.
+ *   cdfs: device int32[K][Lmax]; cdf_lengths, offsets: device int32[K].
+ */
+int rans_tables_prepare(const int32_t *cdfs, int32_t K, int32_t Lmax,
+                        const int32_t *cdf_lengths, const int32_t *offsets,
+                        void *blob, uint64_t blob_bytes, rans_tables *out, void *stream);
+
+/* ------------------------------------------------- sizes and queries ---- */
+
+/* Number of streams the chunking makes of n symbols (< 0: invalid chunking). */
+int64_t rans_num_streams(const rans_chunking *chunking, int64_t n);
+
+/* Bytes of workspace rans_encode_with_indexes needs (status word, per-stream
+ * lengths and a worst-case scratch slot per stream: 8 bytes per symbol plus
+ * 16 * interleave + 16 per stream). */
+uint64_t rans_encode_workspace_bytes(const rans_chunking *chunking, int64_t n);
+
+/* Bytes of workspace rans_decode_with_indexes needs. */
+uint64_t rans_decode_workspace_bytes(const rans_chunking *chunking, int64_t n);
+
+/* An output capacity that can never be too small for n symbols. */
+uint64_t rans_max_compressed_bytes(const rans_chunking *chunking, int64_t n);
+
+/* ---------------------------------------------------- encode / decode ---- */
+
+/*
+ * encode_with_indexes ("torch_ans 0.3.0", Low-level API rans_push and
+ * High-level API encode_with_indexes).  Codes the n symbols into one
+ * byte string per stream, packed back to back in `out`; stream_offsets
+ * receives S + 1 uint64 byte offsets (offsets[0] = 0, offsets[S] = total).
+ * Each stream is coded symbol by symbol in reverse order into a worst-case
+ * scratch slot of the workspace, then all streams are compacted into `out`
+ * with a device prefix scan.
+ *   symbols:   device array of n elements of sym_dtype (RANS_SYM_*).
+ *   indexes:   device int32[ceil(n / index_block)], each in [0, tables->K).
+ *   out:       device uint8[out_capacity].
+ *   stream_offsets: device uint64[S + 1].
+ *   workspace: device, >= rans_encode_workspace_bytes; 256-byte aligned.
+ * Asynchronous; device errors via rans_get_status(workspace).
+ */
+int rans_encode_with_indexes(const void *symbols, int32_t sym_dtype, const int32_t *indexes,
+                             int64_t n, const rans_tables *tables,
+                             const rans_chunking *chunking, uint8_t *out,
+                             uint64_t out_capacity, uint64_t *stream_offsets,
+                             void *workspace, uint64_t workspace_bytes, void *stream);
+
+/*
+ * decode_with_indexes ("torch_ans 0.3.0", Low-level API rans_pop; the decoded
+ * symbol is the row's last bucket whose CDF entry is <= the state's low 16
+ * bits, the rule of the linear scan in "Benchmark notes" section 4).
+ *   in:             device uint8[in_bytes]: the packed streams.
+ *   stream_offsets: device uint64[S + 1] from the encoder.
+ *   indexes:        as for encode; must equal the encoder's.
+ *   symbols_out:    device array of n elements of sym_dtype.
+ *   workspace:      device, >= rans_decode_workspace_bytes; 256-byte aligned.
+ * Every read is bounded by its stream's [offsets[k], offsets[k+1]); a stream
+ * that does not end exactly where its words end with every lane back at the
+ * initial state 2^31 is reported as RANS_ERR_CORRUPT.  Asynchronous.
+ */
+int rans_decode_with_indexes(const uint8_t *in, uint64_t in_bytes,
+                             const uint64_t *stream_offsets, const int32_t *indexes,
+                             int64_t n, const rans_tables *tables,
+                             const rans_chunking *chunking, void *symbols_out,
+                             int32_t sym_dtype, void *workspace, uint64_t workspace_bytes,
+                             void *stream);
+
+/* Synchronises `stream` and returns the first error recorded in `workspace`
+ * (RANS_OK if none), then clears it. */
+int rans_get_status(void *workspace, void *stream);
+
+/* ------------------------------------------------------- diagnostics ---- */
+
+/*
+ * The encoder's division step on its own: q[i] = x[i] / f[i] and
+ * r[i] = x[i] % f[i] for x < 2^47 f, 1 <= f <= 65536, computed the way the
+ * encoder does (a double-precision quotient estimate and an exact integer
+ * correction).  For tests.  Asynchronous.
+ */
+int rans_debug_divide(const uint64_t *x, const uint32_t *f, int64_t n, uint64_t *q,
+                      uint32_t *r, void *stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* RANS_B200_H */

@@ -1,0 +1,404 @@
+// decode.cu -- decode_with_indexes.
+//
+//  * symbol lookup: the decoded bucket is the row's last bucket whose CDF
+//    entry is <= cum = x mod 2^16 (the rule of CompressAI's linear scan,
+//    "Benchmark notes" section 4).  It is found through a per-row table of
+//    2^q slots keyed by the top q bits of cum ("torch_ans 0.3.0", Usage,
+//    inverse-CDF decoding): a slot either names the bucket, or holds one
+//    boundary to compare against, or bounds a short run of boundaries that
+//    the warp counts together (one ballot per 32 candidates);
+//  * state update x = freq (x >> 16) + cum - start and a refill of one
+//    32-bit word when x < 2^31 (64-bit state / 32-bit words / 16-bit
+//    precision: "torch_ans 0.3.0", Usage, rans64 row);
+//  * W = 32: one warp per stream, lane = symbol index mod 32; refills take
+//    the next words of the shared stream in lane order (ballot + popc),
+//    served from a two-window register buffer of 64 prefetched words
+//    ("torch_ans 0.3.0", Usage legend: warp renormalisation with one shared
+//    cursor);
+//  * escapes run off the fast path: lanes proceed one by one in ascending
+//    order, reading their bypass pieces, since how many words a lane takes
+//    depends on what it reads ("torch_ans 0.3.0", Performance Tuning, GPU
+//    item 5: the bypass phase is sequential across the lanes and skipped by a
+//    group ballot).
+//  Tables are staged into shared memory with bulk copies when they fit.
+#include "rans_common.cuh"
+#include "rans_internal.h"
+
+namespace rb {
+namespace {
+
+constexpr int kDecMaxThreads32 = 768;
+constexpr int kDecThreads1 = 128;
+
+struct DecCtx {
+  const uint8_t *in;
+  uint64_t in_bytes;
+  const uint64_t *offs;
+  const int32_t *idx;
+  int32_t K;
+  uint32_t meta_bytes, bucket_bytes, slot_bytes;
+  const char *blob;
+  Geom g;
+  void *out;
+  int32_t *status;
+};
+
+__device__ __forceinline__ bool stream_bounds(const DecCtx &c, int64_t s, int W,
+                                              const uint32_t *&words, uint64_t &nw) {
+  const uint64_t b0 = c.offs[s], b1 = c.offs[s + 1];
+  if (b1 < b0 || b1 > c.in_bytes || ((b0 | b1) & 3ull) != 0 || (b1 - b0) < 8ull * W)
+    return false;
+  words = reinterpret_cast<const uint32_t *>(c.in + b0);
+  nw = (b1 - b0) >> 2;
+  return true;
+}
+
+template <typename SymT>
+__device__ void decode_stream_w32(const DecCtx &c, const RowMeta *meta, const uint32_t *buckets,
+                                  const uint32_t *slots, int64_t s) {
+  const int lane = threadIdx.x & 31;
+  const StreamDesc d = stream_desc(c.g, s);
+  const uint32_t *words = nullptr;
+  uint64_t nw = 0;
+  if (!d.ok || !stream_bounds(c, s, 32, words, nw)) {
+    if (lane == 0) report(c.status, d.ok ? RANS_ERR_CORRUPT : RANS_ERR_ARG, s);
+    return;
+  }
+  const int ib = c.g.ib_shift;
+  uint64_t x = (uint64_t)__ldg(words + 2 * lane) | ((uint64_t)__ldg(words + 2 * lane + 1) << 32);
+  uint64_t cur = 64;  // absolute word index of the window start
+  uint32_t off = 0;   // words of the window already consumed
+  uint32_t w0 = cur + lane < nw ? __ldg(words + cur + lane) : 0u;
+  uint32_t w1 = cur + 32 + lane < nw ? __ldg(words + cur + 32 + lane) : 0u;
+  bool bad = false;
+
+  const int64_t n = d.n;
+  const int64_t G = (n + 31) >> 5;
+  Walker wk;
+  wk.init(d, lane);
+  int32_t nr = 0;
+  int64_t np = 0;
+  if (lane < n) {
+    np = wk.pos();
+    nr = __ldg(c.idx + (np >> ib));
+  }
+  for (int64_t g = 0; g < G; ++g) {
+    const bool active = g * 32 + lane < n;
+    const int32_t r = nr;
+    const int64_t p = np;
+    if (g + 1 < G) {
+      wk.fwd(32);
+      if ((g + 1) * 32 + lane < n) {
+        np = wk.pos();
+        nr = __ldg(c.idx + (np >> ib));
+      }
+    }
+    if (__any_sync(kFull, active && (uint32_t)r >= (uint32_t)c.K)) {
+      if (lane == 0) report(c.status, RANS_ERR_INDEX, s);
+      return;
+    }
+    const RowMeta m = meta[active ? r : 0];
+    const uint32_t cum = (uint32_t)x & (kTotal - 1);
+    const uint32_t sh = slot_shift(m.slot);
+    const uint32_t se = slots[slot_base(m.slot) + (cum >> sh)];
+    const uint32_t lo = se & 0xffffu;
+    const uint32_t code = se >> 16;
+    uint32_t sym = lo + ((cum & ((1u << sh) - 1u)) >= code ? 1u : 0u);
+    uint32_t mm = __ballot_sync(kFull, active && (code & 0x8000u));
+    while (mm) {
+      const int l = __ffs(mm) - 1;
+      mm &= mm - 1;
+      const uint32_t base_l = __shfl_sync(kFull, m.bucket_base + lo, l);
+      const uint32_t cnt_l = __shfl_sync(kFull, code & 0x7fffu, l);
+      const uint32_t cum_l = __shfl_sync(kFull, cum, l);
+      uint32_t cnt = 0;
+      for (uint32_t k0 = 0; k0 < cnt_l; k0 += 32) {
+        const uint32_t k = k0 + lane + 1;
+        const bool le = k <= cnt_l && bucket_start(buckets[base_l + k]) <= cum_l;
+        cnt += __popc(__ballot_sync(kFull, le));
+      }
+      if (lane == l) sym = lo + cnt;
+    }
+    const uint32_t e = buckets[m.bucket_base + sym];
+    if (active) x = (uint64_t)bucket_freq(e) * (x >> kPrec) + cum - bucket_start(e);
+    const bool esc = active && sym == m.maxv;
+    int64_t val = (int64_t)sym;
+    if (!__any_sync(kFull, esc)) {
+      const bool need = active && x < kL;
+      const uint32_t nm = __ballot_sync(kFull, need);
+      const uint32_t j = off + __popc(nm & lanemask_lt());
+      const uint32_t a = __shfl_sync(kFull, w0, j & 31);
+      const uint32_t b = __shfl_sync(kFull, w1, j & 31);
+      if (need) x = (x << 32) | (j < 32 ? a : b);
+      off += __popc(nm);
+      if (off >= 32) {
+        w0 = w1;
+        cur += 32;
+        off -= 32;
+        w1 = cur + 32 + lane < nw ? __ldg(words + cur + 32 + lane) : 0u;
+      }
+    } else {
+      // Lanes consume words in ascending lane order; an escaping lane's
+      // count is known only after it has read its pieces.
+      const uint64_t abs0 = cur + off;
+      const bool need_sym = active && x < kL;
+      uint32_t cons = need_sym ? 1u : 0u;
+      uint32_t rem = __ballot_sync(kFull, esc);
+      while (rem) {
+        const int el = __ffs(rem) - 1;
+        rem &= rem - 1;
+        uint32_t inc = cons;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+          const uint32_t t = __shfl_up_sync(kFull, inc, o);
+          if (lane >= o) inc += t;
+        }
+        const uint32_t pre = __shfl_sync(kFull, inc - cons, el);
+        if (lane == el) {
+          uint64_t pp = abs0 + pre;
+          auto rd = [&]() -> uint32_t {
+            uint32_t v = 0;
+            if (pp < nw) v = __ldg(words + pp); else bad = true;
+            ++pp;
+            return v;
+          };
+          if (x < kL) x = (x << 32) | rd();
+          auto getbits = [&]() -> uint32_t {
+            const uint32_t v = (uint32_t)x & kBypassMax;
+            x >>= kBypassBits;
+            if (x < kL) x = (x << 32) | rd();
+            return v;
+          };
+          uint32_t v4 = getbits();
+          uint32_t nb = v4;
+          while (v4 == kBypassMax && nb <= 15) {
+            v4 = getbits();
+            nb += v4;
+          }
+          if (nb > 15) {
+            bad = true;
+            nb = 0;
+          }
+          uint64_t raw = 0;
+          for (uint32_t k = 0; k < nb; ++k) raw |= (uint64_t)getbits() << (kBypassBits * k);
+          const int64_t half = (int64_t)(raw >> 1);
+          val = (raw & 1) ? (-half - 1) : ((int64_t)m.maxv + half);
+          cons = (uint32_t)(pp - (abs0 + pre));
+        }
+      }
+      uint32_t inc = cons;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const uint32_t t = __shfl_up_sync(kFull, inc, o);
+        if (lane >= o) inc += t;
+      }
+      if (need_sym && !esc) {
+        const uint64_t pp = abs0 + (inc - cons);
+        uint32_t v = 0;
+        if (pp < nw) v = __ldg(words + pp); else bad = true;
+        x = (x << 32) | v;
+      }
+      cur = abs0 + __shfl_sync(kFull, inc, 31);
+      off = 0;
+      w0 = cur + lane < nw ? __ldg(words + cur + lane) : 0u;
+      w1 = cur + 32 + lane < nw ? __ldg(words + cur + 32 + lane) : 0u;
+    }
+    if (active) SymIO<SymT>::store(c.out, p, val + (int64_t)m.offset);
+  }
+  const bool ok = !bad && x == kL && cur + off == nw;
+  if (!__all_sync(kFull, ok) && lane == 0) report(c.status, RANS_ERR_CORRUPT, s);
+}
+
+template <typename SymT>
+__device__ void decode_stream_w1(const DecCtx &c, const RowMeta *meta, const uint32_t *buckets,
+                                 const uint32_t *slots, int64_t s) {
+  const StreamDesc d = stream_desc(c.g, s);
+  const uint32_t *words = nullptr;
+  uint64_t nw = 0;
+  if (!d.ok || !stream_bounds(c, s, 1, words, nw)) {
+    report(c.status, d.ok ? RANS_ERR_CORRUPT : RANS_ERR_ARG, s);
+    return;
+  }
+  const int ib = c.g.ib_shift;
+  uint64_t x = (uint64_t)__ldg(words) | ((uint64_t)__ldg(words + 1) << 32);
+  uint64_t pp = 2;
+  bool bad = false;
+  auto rd = [&]() -> uint32_t {
+    uint32_t v = 0;
+    if (pp < nw) v = __ldg(words + pp); else bad = true;
+    ++pp;
+    return v;
+  };
+  Walker wk;
+  wk.init(d, 0);
+  for (int64_t i = 0; i < d.n; ++i) {
+    const int64_t p = wk.pos();
+    wk.fwd(1);
+    const int32_t r = __ldg(c.idx + (p >> ib));
+    if ((uint32_t)r >= (uint32_t)c.K) {
+      report(c.status, RANS_ERR_INDEX, s);
+      return;
+    }
+    const RowMeta m = meta[r];
+    const uint32_t cum = (uint32_t)x & (kTotal - 1);
+    const uint32_t sh = slot_shift(m.slot);
+    const uint32_t se = slots[slot_base(m.slot) + (cum >> sh)];
+    uint32_t sym = se & 0xffffu;
+    const uint32_t code = se >> 16;
+    if (code & 0x8000u) {
+      // last bucket in [sym, sym + count] whose start is <= cum
+      uint32_t lo = sym, hi = sym + (code & 0x7fffu);
+      while (lo < hi) {
+        const uint32_t mid = (lo + hi + 1) >> 1;
+        if (bucket_start(buckets[m.bucket_base + mid]) <= cum) lo = mid; else hi = mid - 1;
+      }
+      sym = lo;
+    } else {
+      sym += (cum & ((1u << sh) - 1u)) >= code ? 1u : 0u;
+    }
+    const uint32_t e = buckets[m.bucket_base + sym];
+    x = (uint64_t)bucket_freq(e) * (x >> kPrec) + cum - bucket_start(e);
+    if (x < kL) x = (x << 32) | rd();
+    int64_t val = (int64_t)sym;
+    if (sym == m.maxv) {
+      auto getbits = [&]() -> uint32_t {
+        const uint32_t v = (uint32_t)x & kBypassMax;
+        x >>= kBypassBits;
+        if (x < kL) x = (x << 32) | rd();
+        return v;
+      };
+      uint32_t v4 = getbits();
+      uint32_t nb = v4;
+      while (v4 == kBypassMax && nb <= 15) {
+        v4 = getbits();
+        nb += v4;
+      }
+      if (nb > 15) {
+        bad = true;
+        nb = 0;
+      }
+      uint64_t raw = 0;
+      for (uint32_t k = 0; k < nb; ++k) raw |= (uint64_t)getbits() << (kBypassBits * k);
+      const int64_t half = (int64_t)(raw >> 1);
+      val = (raw & 1) ? (-half - 1) : ((int64_t)m.maxv + half);
+    }
+    SymIO<SymT>::store(c.out, p, val + (int64_t)m.offset);
+  }
+  if (bad || x != kL || pp != nw) report(c.status, RANS_ERR_CORRUPT, s);
+}
+
+template <int W, typename SymT, bool SMEM>
+__global__ void __launch_bounds__(W == 32 ? kDecMaxThreads32 : kDecThreads1)
+    decode_kernel(DecCtx c) {
+  extern __shared__ __align__(16) unsigned char smem[];
+  __shared__ uint64_t bar;
+  const unsigned char *tb;
+  if (SMEM) {
+    if (!stage_to_smem(smem, c.blob + kHeaderBytes, c.meta_bytes + c.bucket_bytes + c.slot_bytes,
+                       &bar, c.status))
+      return;
+    tb = smem;
+  } else {
+    tb = reinterpret_cast<const unsigned char *>(c.blob + kHeaderBytes);
+  }
+  const RowMeta *meta = reinterpret_cast<const RowMeta *>(tb);
+  const uint32_t *buckets = reinterpret_cast<const uint32_t *>(tb + c.meta_bytes);
+  const uint32_t *slots = reinterpret_cast<const uint32_t *>(tb + c.meta_bytes + c.bucket_bytes);
+  if (W == 32) {
+    const int warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+    for (int64_t s = blockIdx.x + (int64_t)gridDim.x * warp; s < c.g.S;
+         s += (int64_t)gridDim.x * nw)
+      decode_stream_w32<SymT>(c, meta, buckets, slots, s);
+  } else {
+    for (int64_t s = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; s < c.g.S;
+         s += (int64_t)gridDim.x * blockDim.x)
+      decode_stream_w1<SymT>(c, meta, buckets, slots, s);
+  }
+}
+
+template <int W, typename SymT, bool SMEM>
+int launch_decode_t(const DecCtx &c, cudaStream_t st) {
+  auto kern = decode_kernel<W, SymT, SMEM>;
+  const uint32_t smem = SMEM ? c.meta_bytes + c.bucket_bytes + c.slot_bytes : 0;
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (SMEM && cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                   (int)smem) != cudaSuccess)
+    return RANS_ERR_CUDA;
+  const int sms = num_sms(dev);
+  int threads, blocks;
+  if (W == 32) {
+    // One or a few CTAs per SM (bounded by the staged tables); enough warps
+    // for one stream each when possible.
+    int per_sm = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, 32, smem) != cudaSuccess ||
+        per_sm < 1)
+      return RANS_ERR_CUDA;
+    int64_t nblk = (int64_t)sms * per_sm;
+    if (nblk > c.g.S) nblk = c.g.S < 1 ? 1 : c.g.S;
+    int64_t warps = (c.g.S + nblk - 1) / nblk;
+    const int max_warps = kDecMaxThreads32 / 32;
+    if (warps > max_warps) warps = max_warps;
+    if (warps < 1) warps = 1;
+    threads = (int)warps * 32;
+    int fit = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&fit, kern, threads, smem) != cudaSuccess ||
+        fit < 1)
+      return RANS_ERR_CUDA;
+    int64_t need = (c.g.S + warps - 1) / warps;
+    int64_t cap = (int64_t)fit * sms;
+    blocks = (int)(need < cap ? need : cap);
+  } else {
+    threads = kDecThreads1;
+    int fit = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&fit, kern, threads, smem) != cudaSuccess ||
+        fit < 1)
+      return RANS_ERR_CUDA;
+    int64_t need = (c.g.S + threads - 1) / threads;
+    int64_t cap = (int64_t)fit * sms;
+    blocks = (int)(need < cap ? need : cap);
+  }
+  if (blocks < 1) blocks = 1;
+  kern<<<blocks, threads, smem, st>>>(c);
+  return cudaGetLastError() == cudaSuccess ? RANS_OK : RANS_ERR_CUDA;
+}
+
+template <int W, typename SymT>
+int launch_decode_w(const DecCtx &c, bool smem, cudaStream_t st) {
+  return smem ? launch_decode_t<W, SymT, true>(c, st) : launch_decode_t<W, SymT, false>(c, st);
+}
+
+template <typename SymT>
+int launch_decode_s(const DecCtx &c, bool smem, cudaStream_t st) {
+  return c.g.W == 32 ? launch_decode_w<32, SymT>(c, smem, st)
+                     : launch_decode_w<1, SymT>(c, smem, st);
+}
+
+}  // namespace
+
+int launch_decode(const uint8_t *in, uint64_t in_bytes, const uint64_t *offsets,
+                  const int32_t *indexes, const rans_tables &t, const Geom &g, void *symbols,
+                  int sym_dtype, int32_t *status, cudaStream_t st) {
+  DecCtx c;
+  c.in = in;
+  c.in_bytes = in_bytes;
+  c.offs = offsets;
+  c.idx = indexes;
+  c.K = t.K;
+  c.meta_bytes = t.meta_bytes;
+  c.bucket_bytes = t.bucket_bytes;
+  c.slot_bytes = t.slot_bytes;
+  c.blob = reinterpret_cast<const char *>(t.blob);
+  c.g = g;
+  c.out = symbols;
+  c.status = status;
+  const bool smem = t.dec_in_smem != 0;
+  switch (sym_dtype) {
+    case RANS_SYM_INT32: return launch_decode_s<int32_t>(c, smem, st);
+    case RANS_SYM_UINT8: return launch_decode_s<uint8_t>(c, smem, st);
+    case RANS_SYM_INT16: return launch_decode_s<int16_t>(c, smem, st);
+    default: return RANS_ERR_ARG;
+  }
+}
+
+}  // namespace rb

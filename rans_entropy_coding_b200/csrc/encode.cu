@@ -1,0 +1,415 @@
+// encode.cu -- encode_with_indexes: every stream is coded in reverse symbol
+// order into a worst-case scratch slot (words written downward, the way a
+// ryg_rans encoder fills its buffer from the end), then the streams are
+// compacted behind a device prefix scan.
+//
+//  * value mapping and escape ("torch_ans 0.3.0", Low-level API, rans_push:
+//    coded range [offset, offset + cdf_size - 2), zig-zag raw value, bypass
+//    pieces; "kompressor" README, Correctness: the bypass path);
+//  * symbol op: renormalise when x >= 2^47 freq, then
+//    x = (x / freq) 2^16 + x mod freq + start (64-bit state, 32-bit words,
+//    16-bit precision: "torch_ans 0.3.0", Usage, rans64 row);
+//  * W = 32: one warp per stream, lane = symbol index mod 32, one shared word
+//    stream ("torch_ans 0.3.0", Usage legend: __ballot_sync-based warp
+//    renormalisation with one shared cursor; FAQ: interleaved states share
+//    one bitstream, processed sequentially).  In the serial order a group of
+//    32 symbols is coded lane 31 first, so lane l's words land below those of
+//    lanes > l: a ballot + popc places them.  A group holding an escape is
+//    coded off the fast path: each lane counts its words, a suffix sum over
+//    lanes places them, and the lane writes them.
+#include "rans_common.cuh"
+#include "rans_internal.h"
+
+namespace rb {
+namespace {
+
+constexpr int kEncThreads32 = 512;
+constexpr int kEncThreads1 = 128;
+
+struct EncCtx {
+  const void *sym;
+  const int32_t *idx;
+  int32_t K;
+  uint32_t meta_bytes, bucket_bytes;
+  const char *blob;
+  Geom g;
+  char *scratch;
+  uint64_t *lens;
+  int32_t *status;
+};
+
+// Maps symbol s through row m: bucket start / width, and the escape's raw
+// value (zig-zag: below the range 2|v| - 1, above it 2 (v - maxv)).
+__device__ __forceinline__ void map_symbol(int32_t s, const RowMeta &m, const uint32_t *buckets,
+                                           uint32_t &start, uint32_t &freq, uint64_t &raw,
+                                           bool &esc) {
+  int64_t v = (int64_t)s - (int64_t)m.offset;
+  const int64_t maxv = (int64_t)m.maxv;
+  raw = 0;
+  if (v < 0) {
+    raw = (uint64_t)(-2 * v - 1);
+    v = maxv;
+  } else if (v >= maxv) {
+    raw = (uint64_t)(2 * (v - maxv));
+    v = maxv;
+  }
+  esc = (v == maxv);
+  const uint32_t e = buckets[m.bucket_base + (uint32_t)v];
+  start = bucket_start(e);
+  freq = bucket_freq(e);
+}
+
+// Bypass op: renormalise when x >= 2^59, then append 4 bits.
+template <bool WRITE>
+__device__ __forceinline__ void bits_op(uint64_t &x, uint32_t val, uint32_t *end, uint32_t &k,
+                                        uint32_t pos0) {
+  if (x >= (1ull << 59)) {
+    if (WRITE) end[-1 - (int64_t)(pos0 + k)] = (uint32_t)x;
+    ++k;
+    x >>= 32;
+  }
+  x = (x << kBypassBits) | val;
+}
+
+// All ops of one symbol, in reverse op order (bypass pieces last to first,
+// then the count pieces last to first, then the symbol op).  Returns the
+// number of words pushed; with WRITE they go to end[-1 - (pos0 + j)].
+template <bool WRITE>
+__device__ __forceinline__ uint32_t symbol_ops(uint64_t &x, uint32_t start, uint32_t freq,
+                                               double rcp, uint64_t raw, bool esc,
+                                               uint32_t *end, uint32_t pos0) {
+  uint32_t k = 0;
+  if (esc) {
+    uint32_t nb = 0;
+    while (nb < 16 && (raw >> (kBypassBits * nb)) != 0) ++nb;
+    for (int j = (int)nb - 1; j >= 0; --j)
+      bits_op<WRITE>(x, (uint32_t)(raw >> (kBypassBits * j)) & kBypassMax, end, k, pos0);
+    bits_op<WRITE>(x, nb % kBypassMax, end, k, pos0);
+    for (uint32_t t = 0; t < nb / kBypassMax; ++t) bits_op<WRITE>(x, kBypassMax, end, k, pos0);
+  }
+  if (x >= ((uint64_t)freq << 47)) {
+    if (WRITE) end[-1 - (int64_t)(pos0 + k)] = (uint32_t)x;
+    ++k;
+    x >>= 32;
+  }
+  x = enc_sym_step(x, start, freq, rcp);
+  return k;
+}
+
+template <typename SymT>
+__device__ void encode_stream_w32(const EncCtx &c, const RowMeta *meta, const uint32_t *buckets,
+                                  int64_t s) {
+  const int lane = threadIdx.x & 31;
+  const StreamDesc d = stream_desc(c.g, s);
+  if (!d.ok) {
+    if (lane == 0) report(c.status, RANS_ERR_ARG, s);
+    return;
+  }
+  uint32_t *end = reinterpret_cast<uint32_t *>(c.scratch + slot_end(c.g, d, s));
+  const int64_t n = d.n;
+  const int64_t G = (n + 31) >> 5;
+  const int ib = c.g.ib_shift;
+  uint64_t x = kL;
+  uint32_t cursor = 0;
+
+  Walker wk;
+  int32_t nsv = 0, nr = 0;
+  if (G > 0) {
+    wk.init(d, (G - 1) * 32 + lane);
+    if ((G - 1) * 32 + lane < n) {
+      const int64_t p = wk.pos();
+      nsv = SymIO<SymT>::load(c.sym, p);
+      nr = __ldg(c.idx + (p >> ib));
+    }
+  }
+  for (int64_t g = G - 1; g >= 0; --g) {
+    const bool active = g * 32 + lane < n;
+    const int32_t sv = nsv, r = nr;
+    if (g > 0) {
+      wk.back(32);
+      const int64_t p = wk.pos();
+      nsv = SymIO<SymT>::load(c.sym, p);
+      nr = __ldg(c.idx + (p >> ib));
+    }
+    if (__any_sync(kFull, active && (uint32_t)r >= (uint32_t)c.K)) {
+      if (lane == 0) report(c.status, RANS_ERR_INDEX, s);
+      return;
+    }
+    const RowMeta m = meta[active ? r : 0];
+    uint32_t start, freq;
+    uint64_t raw;
+    bool esc;
+    map_symbol(sv, m, buckets, start, freq, raw, esc);
+    esc = esc && active;
+    const double rcp = freq_reciprocal(freq);
+    if (!__any_sync(kFull, esc)) {
+      const bool need = active && x >= ((uint64_t)freq << 47);
+      const uint32_t bm = __ballot_sync(kFull, need);
+      if (need) {
+        const uint32_t k = cursor + __popc(bm & (0xfffffffeu << lane));
+        end[-1 - (int64_t)k] = (uint32_t)x;
+        x >>= 32;
+      }
+      cursor += __popc(bm);
+      if (active) x = enc_sym_step(x, start, freq, rcp);
+    } else {
+      if (__any_sync(kFull, esc && (raw >> 60) != 0)) {
+        if (lane == 0) report(c.status, RANS_ERR_RANGE, s);
+        return;
+      }
+      uint32_t k = 0;
+      if (active) {
+        uint64_t y = x;
+        k = symbol_ops<false>(y, start, freq, rcp, raw, esc, end, 0);
+      }
+      uint32_t inc = k;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const uint32_t t = __shfl_down_sync(kFull, inc, o);
+        if (lane + o < 32) inc += t;
+      }
+      const uint32_t total = __shfl_sync(kFull, inc, 0);
+      if (active) symbol_ops<true>(x, start, freq, rcp, raw, esc, end, cursor + inc - k);
+      cursor += total;
+    }
+  }
+  // flush: lanes 31..0 push high then low, so lane 0's low word comes first
+  const uint32_t kk = cursor + 2u * (31u - (uint32_t)lane);
+  end[-1 - (int64_t)kk] = (uint32_t)(x >> 32);
+  end[-2 - (int64_t)kk] = (uint32_t)x;
+  cursor += 64;
+  if (lane == 0) c.lens[s] = 4ull * cursor;
+}
+
+template <typename SymT>
+__device__ void encode_stream_w1(const EncCtx &c, const RowMeta *meta, const uint32_t *buckets,
+                                 int64_t s) {
+  const StreamDesc d = stream_desc(c.g, s);
+  if (!d.ok) {
+    report(c.status, RANS_ERR_ARG, s);
+    return;
+  }
+  uint32_t *end = reinterpret_cast<uint32_t *>(c.scratch + slot_end(c.g, d, s));
+  const int ib = c.g.ib_shift;
+  uint64_t x = kL;
+  uint32_t cursor = 0;
+  Walker wk;
+  if (d.n > 0) wk.init(d, d.n - 1);
+  for (int64_t i = d.n - 1; i >= 0; --i) {
+    const int64_t p = wk.pos();
+    wk.back(1);
+    const int32_t sv = SymIO<SymT>::load(c.sym, p);
+    const int32_t r = __ldg(c.idx + (p >> ib));
+    if ((uint32_t)r >= (uint32_t)c.K) {
+      report(c.status, RANS_ERR_INDEX, s);
+      return;
+    }
+    uint32_t start, freq;
+    uint64_t raw;
+    bool esc;
+    map_symbol(sv, meta[r], buckets, start, freq, raw, esc);
+    if (esc && (raw >> 60) != 0) {
+      report(c.status, RANS_ERR_RANGE, s);
+      return;
+    }
+    cursor += symbol_ops<true>(x, start, freq, freq_reciprocal(freq), raw, esc, end, cursor);
+  }
+  end[-1 - (int64_t)cursor] = (uint32_t)(x >> 32);
+  end[-2 - (int64_t)cursor] = (uint32_t)x;
+  cursor += 2;
+  c.lens[s] = 4ull * cursor;
+}
+
+template <int W, typename SymT, bool SMEM>
+__global__ void __launch_bounds__(W == 32 ? kEncThreads32 : kEncThreads1)
+    encode_kernel(EncCtx c) {
+  extern __shared__ __align__(16) unsigned char smem[];
+  __shared__ uint64_t bar;
+  const RowMeta *meta;
+  const uint32_t *buckets;
+  if (SMEM) {
+    if (!stage_to_smem(smem, c.blob + kHeaderBytes, c.meta_bytes + c.bucket_bytes, &bar,
+                       c.status))
+      return;
+    meta = reinterpret_cast<const RowMeta *>(smem);
+    buckets = reinterpret_cast<const uint32_t *>(smem + c.meta_bytes);
+  } else {
+    meta = reinterpret_cast<const RowMeta *>(c.blob + kHeaderBytes);
+    buckets = reinterpret_cast<const uint32_t *>(c.blob + kHeaderBytes + c.meta_bytes);
+  }
+  if (W == 32) {
+    const int warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+    for (int64_t s = blockIdx.x + (int64_t)gridDim.x * warp; s < c.g.S;
+         s += (int64_t)gridDim.x * nw)
+      encode_stream_w32<SymT>(c, meta, buckets, s);
+  } else {
+    for (int64_t s = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; s < c.g.S;
+         s += (int64_t)gridDim.x * blockDim.x)
+      encode_stream_w1<SymT>(c, meta, buckets, s);
+  }
+}
+
+// ---- compaction -----------------------------------------------------------
+
+constexpr int kScanThreads = 1024;
+
+__global__ void __launch_bounds__(kScanThreads)
+    scan_lengths_kernel(const uint64_t *lens, int64_t S, uint64_t *offsets, uint64_t capacity,
+                        int32_t *status) {
+  __shared__ unsigned long long warp_tot[kScanThreads / 32];
+  __shared__ unsigned long long carry_sh;
+  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+  if (threadIdx.x == 0) {
+    carry_sh = 0;
+    offsets[0] = 0;
+  }
+  __syncthreads();
+  for (int64_t base = 0; base < S; base += kScanThreads) {
+    const int64_t i = base + threadIdx.x;
+    unsigned long long v = i < S ? lens[i] : 0ull;
+    unsigned long long inc = v;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      unsigned long long t = __shfl_up_sync(kFull, inc, o);
+      if (lane >= o) inc += t;
+    }
+    if (lane == 31) warp_tot[wid] = inc;
+    __syncthreads();
+    if (wid == 0) {
+      unsigned long long w = warp_tot[lane];
+      unsigned long long wi = w;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        unsigned long long t = __shfl_up_sync(kFull, wi, o);
+        if (lane >= o) wi += t;
+      }
+      warp_tot[lane] = wi - w;
+    }
+    __syncthreads();
+    const unsigned long long carry = carry_sh;
+    const unsigned long long out = carry + warp_tot[wid] + inc;
+    if (i < S) offsets[i + 1] = out;
+    __syncthreads();
+    if (threadIdx.x == kScanThreads - 1) carry_sh = out;
+    __syncthreads();
+  }
+  if (threadIdx.x == 0 && carry_sh > capacity) report(status, RANS_ERR_CAPACITY, -1);
+}
+
+__global__ void copy_streams_kernel(Geom g, const char *scratch, const uint64_t *lens,
+                                    const uint64_t *offsets, uint8_t *out, uint64_t capacity) {
+  const int lane = threadIdx.x & 31;
+  const int64_t nw = (int64_t)gridDim.x * (blockDim.x >> 5);
+  for (int64_t s = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); s < g.S;
+       s += nw) {
+    const StreamDesc d = stream_desc(g, s);
+    if (!d.ok) continue;
+    const uint64_t len = lens[s];
+    const uint64_t off = offsets[s];
+    if (off + len > capacity) continue;
+    const uint32_t *src =
+        reinterpret_cast<const uint32_t *>(scratch + slot_end(g, d, s) - len);
+    uint32_t *dst = reinterpret_cast<uint32_t *>(out + off);
+    const uint64_t words = len >> 2;
+    for (uint64_t k = lane; k < words; k += 32) dst[k] = __ldg(src + k);
+  }
+}
+
+__global__ void debug_divide_kernel(const uint64_t *x, const uint32_t *f, int64_t n, uint64_t *q,
+                                    uint32_t *r) {
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n;
+       i += (int64_t)gridDim.x * blockDim.x) {
+    uint64_t qq;
+    uint32_t rr;
+    divmod_freq(x[i], f[i], freq_reciprocal(f[i]), qq, rr);
+    q[i] = qq;
+    r[i] = rr;
+  }
+}
+
+template <int W, typename SymT, bool SMEM>
+int launch_encode_t(const EncCtx &c, cudaStream_t st) {
+  const int dev_threads = W == 32 ? kEncThreads32 : kEncThreads1;
+  auto kern = encode_kernel<W, SymT, SMEM>;
+  const uint32_t smem = SMEM ? c.meta_bytes + c.bucket_bytes : 0;
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (SMEM && cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                   (int)smem) != cudaSuccess)
+    return RANS_ERR_CUDA;
+  int per_sm = 0;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, dev_threads, smem) !=
+          cudaSuccess ||
+      per_sm < 1)
+    return RANS_ERR_CUDA;
+  const int64_t units_per_block = W == 32 ? dev_threads / 32 : dev_threads;
+  int64_t blocks = (c.g.S + units_per_block - 1) / units_per_block;
+  const int64_t cap = (int64_t)per_sm * num_sms(dev);
+  if (blocks > cap) blocks = cap;
+  if (blocks < 1) blocks = 1;
+  kern<<<(unsigned)blocks, dev_threads, smem, st>>>(c);
+  return cudaGetLastError() == cudaSuccess ? RANS_OK : RANS_ERR_CUDA;
+}
+
+template <int W, typename SymT>
+int launch_encode_w(const EncCtx &c, bool smem, cudaStream_t st) {
+  return smem ? launch_encode_t<W, SymT, true>(c, st) : launch_encode_t<W, SymT, false>(c, st);
+}
+
+template <typename SymT>
+int launch_encode_s(const EncCtx &c, bool smem, cudaStream_t st) {
+  return c.g.W == 32 ? launch_encode_w<32, SymT>(c, smem, st)
+                     : launch_encode_w<1, SymT>(c, smem, st);
+}
+
+}  // namespace
+
+int launch_encode(const void *symbols, int sym_dtype, const int32_t *indexes,
+                  const rans_tables &t, const Geom &g, char *scratch, uint64_t *lens,
+                  int32_t *status, cudaStream_t st) {
+  EncCtx c;
+  c.sym = symbols;
+  c.idx = indexes;
+  c.K = t.K;
+  c.meta_bytes = t.meta_bytes;
+  c.bucket_bytes = t.bucket_bytes;
+  c.blob = reinterpret_cast<const char *>(t.blob);
+  c.g = g;
+  c.scratch = scratch;
+  c.lens = lens;
+  c.status = status;
+  const bool smem = t.enc_in_smem != 0;
+  switch (sym_dtype) {
+    case RANS_SYM_INT32: return launch_encode_s<int32_t>(c, smem, st);
+    case RANS_SYM_UINT8: return launch_encode_s<uint8_t>(c, smem, st);
+    case RANS_SYM_INT16: return launch_encode_s<int16_t>(c, smem, st);
+    default: return RANS_ERR_ARG;
+  }
+}
+
+int launch_compact(const Geom &g, const char *scratch, const uint64_t *lens, uint8_t *out,
+                   uint64_t out_capacity, uint64_t *offsets, int32_t *status,
+                   cudaStream_t st) {
+  scan_lengths_kernel<<<1, kScanThreads, 0, st>>>(lens, g.S, offsets, out_capacity, status);
+  if (g.S > 0) {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    int64_t blocks = (g.S + 7) / 8;
+    const int64_t cap = 8LL * num_sms(dev);
+    if (blocks > cap) blocks = cap;
+    copy_streams_kernel<<<(unsigned)blocks, 256, 0, st>>>(g, scratch, lens, offsets, out,
+                                                          out_capacity);
+  }
+  return cudaGetLastError() == cudaSuccess ? RANS_OK : RANS_ERR_CUDA;
+}
+
+int launch_debug_divide(const uint64_t *x, const uint32_t *f, int64_t n, uint64_t *q,
+                        uint32_t *r, cudaStream_t st) {
+  if (n <= 0) return RANS_OK;
+  int64_t blocks = (n + 255) / 256;
+  if (blocks > 4096) blocks = 4096;
+  debug_divide_kernel<<<(unsigned)blocks, 256, 0, st>>>(x, f, n, q, r);
+  return cudaGetLastError() == cudaSuccess ? RANS_OK : RANS_ERR_CUDA;
+}
+
+}  // namespace rb

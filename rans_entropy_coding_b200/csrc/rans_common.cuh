@@ -1,0 +1,325 @@
+// rans_common.cuh -- device-side building blocks shared by the librans_b200
+// kernels: format constants, the prepared-table layout, stream geometry, the
+// encoder's division step and error reporting.
+//
+// Format (page title + section): 64-bit state, 32-bit words, 16-bit CDF
+// precision ("torch_ans 0.3.0", Usage, rans64 row); lower state bound 2^31;
+// bypass pieces of 4 bits ("torch_ans 0.3.0", Low-level API, rans_push).
+#pragma once
+
+#include <cstdint>
+#include <cuda_runtime.h>
+
+#include "rans_b200.h"
+
+namespace rb {
+
+constexpr uint32_t kPrec = 16;
+constexpr uint32_t kTotal = 1u << kPrec;
+constexpr uint64_t kL = 1ull << 31;            // state lower bound
+constexpr uint32_t kBypassBits = 4;
+constexpr uint32_t kBypassMax = 15;
+constexpr unsigned kFull = 0xffffffffu;
+
+// ------------------------------------------------------------ table blob --
+// [header 256 B][RowMeta K][bucket words][slot words], sections 16-B padded.
+// A bucket word packs start | (width - 1) << 16.  A slot word packs
+// lo | code << 16 where lo is the row-local bucket holding the slot's first
+// cumulative value and code says what lies inside the slot:
+//   code < 0x8000: one bucket boundary at offset `code` from the slot start
+//                  (code == slot width: no boundary inside);
+//   code & 0x8000: (code & 0x7fff) boundaries inside (a few, searched).
+struct RowMeta {
+  uint32_t bucket_base;  // index of the row's bucket 0 in the bucket words
+  uint32_t maxv;         // escape bucket = cdf_length - 2
+  int32_t offset;        // value of bucket 0
+  uint32_t slot;         // slot base | (16 - q) << 27, q = log2(slots in row)
+};
+static_assert(sizeof(RowMeta) == 16, "RowMeta is one 16-byte load");
+
+constexpr uint32_t kHeaderBytes = 256;
+constexpr int kMinQ = 2;
+constexpr int kMaxQ = 14;
+
+__host__ __device__ inline uint32_t pad16(uint64_t b) {
+  return (uint32_t)((b + 15) & ~uint64_t(15));
+}
+
+__device__ __forceinline__ uint32_t bucket_start(uint32_t e) { return e & 0xffffu; }
+__device__ __forceinline__ uint32_t bucket_freq(uint32_t e) { return (e >> 16) + 1u; }
+__device__ __forceinline__ uint32_t slot_base(uint32_t s) { return s & 0x07ffffffu; }
+__device__ __forceinline__ uint32_t slot_shift(uint32_t s) { return s >> 27; }
+
+// ---------------------------------------------------------------- status --
+// The first word of a workspace (and of a table blob's header) holds the
+// first error recorded on the device; the second a detail (stream id).
+struct StatusWord {
+  int32_t code;
+  int32_t pad;
+  int64_t detail;
+};
+
+__device__ __forceinline__ void report(int32_t *status, int code, int64_t detail = 0) {
+  if (atomicCAS(status, 0, code) == 0) {
+    reinterpret_cast<StatusWord *>(status)->detail = detail;
+  }
+}
+
+// ------------------------------------------------------------- geometry --
+// Host-computed description of a chunking, passed by value to kernels.
+struct Geom {
+  int32_t kind;          // RANS_CHUNK_*
+  int32_t W;             // 1 or 32
+  int64_t n;             // symbols
+  int64_t S;             // streams
+  int64_t per;           // CONTIG: ceil(n / S)
+  const int64_t *starts; // EXPLICIT
+  int64_t C, H, Wd;      // TILED tensor dims (batch is implied by S)
+  int64_t cg, th, tw;    // TILED group / tile sizes
+  int64_t ng, nty, ntx;  // TILED counts per image
+  int32_t ib_shift;      // log2(index_block)
+  int32_t pad;
+  uint64_t slot_bytes;   // CONTIG / TILED: uniform scratch slot per stream
+  uint64_t slot_extra;   // 16 W + 16: per-stream scratch beyond 8 B/symbol
+};
+
+// One stream's extent.  Element i of a stream (coding order) sits at flat
+// position base + i (contiguous) or base + c*plane + h*row + w with
+// i = (c * hh + h) * ww + w (tiled).
+struct StreamDesc {
+  int64_t n;
+  int64_t base;
+  int64_t plane, row;
+  int32_t hh, ww;
+  bool tiled;
+  bool ok;
+};
+
+__device__ __forceinline__ StreamDesc stream_desc(const Geom &g, int64_t s) {
+  StreamDesc d;
+  d.tiled = false;
+  d.ok = true;
+  d.plane = 0;
+  d.row = 0;
+  d.hh = 1;
+  d.ww = 1;
+  if (g.kind == RANS_CHUNK_CONTIG) {
+    int64_t a = s * g.per;
+    a = a < g.n ? a : g.n;
+    int64_t b = a + g.per;
+    b = b < g.n ? b : g.n;
+    d.base = a;
+    d.n = b - a;
+  } else if (g.kind == RANS_CHUNK_EXPLICIT) {
+    int64_t a = g.starts[s], b = g.starts[s + 1];
+    d.ok = (a >= 0) && (a <= b) && (b <= g.n);
+    d.base = a;
+    d.n = d.ok ? b - a : 0;
+  } else {
+    int64_t per_img = g.ng * g.nty * g.ntx;
+    int64_t b = s / per_img;
+    int64_t r = s - b * per_img;
+    int64_t gi = r / (g.nty * g.ntx);
+    int64_t r2 = r - gi * (g.nty * g.ntx);
+    int64_t ty = r2 / g.ntx;
+    int64_t tx = r2 - ty * g.ntx;
+    int64_t c0 = gi * g.cg, h0 = ty * g.th, w0 = tx * g.tw;
+    int64_t nc = g.C - c0 < g.cg ? g.C - c0 : g.cg;
+    int64_t hh = g.H - h0 < g.th ? g.H - h0 : g.th;
+    int64_t ww = g.Wd - w0 < g.tw ? g.Wd - w0 : g.tw;
+    d.tiled = true;
+    d.plane = g.H * g.Wd;
+    d.row = g.Wd;
+    d.hh = (int32_t)hh;
+    d.ww = (int32_t)ww;
+    d.base = ((b * g.C + c0) * g.H + h0) * g.Wd + w0;
+    d.n = nc * hh * ww;
+  }
+  return d;
+}
+
+// Byte offset of stream s's scratch slot end (words are written downward).
+__device__ __forceinline__ uint64_t slot_end(const Geom &g, const StreamDesc &d, int64_t s) {
+  if (g.kind == RANS_CHUNK_EXPLICIT) {
+    uint64_t before = (uint64_t)(d.base - g.starts[0]);
+    return 8ull * (before + (uint64_t)d.n) + g.slot_extra * (uint64_t)(s + 1);
+  }
+  return g.slot_bytes * (uint64_t)(s + 1);
+}
+
+// Position walker over a stream's elements, stepping by +-k.
+struct Walker {
+  int64_t base, plane, row;
+  int32_t c, h, w, hh, ww;
+  bool tiled;
+  __device__ __forceinline__ void init(const StreamDesc &d, int64_t i) {
+    base = d.base;
+    plane = d.plane;
+    row = d.row;
+    hh = d.hh;
+    ww = d.ww;
+    tiled = d.tiled;
+    if (tiled) {
+      int64_t per = (int64_t)hh * ww;
+      int64_t cc = i / per;
+      int64_t rem = i - cc * per;
+      c = (int32_t)cc;
+      h = (int32_t)(rem / ww);
+      w = (int32_t)(rem - (int64_t)h * ww);
+    } else {
+      c = 0;
+      h = 0;
+      w = 0;
+      base = d.base + i;
+    }
+  }
+  __device__ __forceinline__ int64_t pos() const {
+    return tiled ? base + (int64_t)c * plane + (int64_t)h * row + w : base;
+  }
+  __device__ __forceinline__ void fwd(int k) {
+    if (!tiled) { base += k; return; }
+    w += k;
+    while (w >= ww) {
+      w -= ww;
+      if (++h >= hh) { h = 0; ++c; }
+    }
+  }
+  __device__ __forceinline__ void back(int k) {
+    if (!tiled) { base -= k; return; }
+    w -= k;
+    while (w < 0) {
+      w += ww;
+      if (--h < 0) { h = hh - 1; --c; }
+    }
+  }
+};
+
+// ------------------------------------------------------------- symbols --
+template <typename T> struct SymIO;
+template <> struct SymIO<int32_t> {
+  static __device__ __forceinline__ int32_t load(const void *p, int64_t i) {
+    return __ldg(reinterpret_cast<const int32_t *>(p) + i);
+  }
+  static __device__ __forceinline__ void store(void *p, int64_t i, int64_t v) {
+    reinterpret_cast<int32_t *>(p)[i] = (int32_t)v;
+  }
+};
+template <> struct SymIO<int16_t> {
+  static __device__ __forceinline__ int32_t load(const void *p, int64_t i) {
+    return (int32_t)__ldg(reinterpret_cast<const short *>(p) + i);
+  }
+  static __device__ __forceinline__ void store(void *p, int64_t i, int64_t v) {
+    reinterpret_cast<int16_t *>(p)[i] = (int16_t)v;
+  }
+};
+template <> struct SymIO<uint8_t> {
+  static __device__ __forceinline__ int32_t load(const void *p, int64_t i) {
+    return (int32_t)__ldg(reinterpret_cast<const unsigned char *>(p) + i);
+  }
+  static __device__ __forceinline__ void store(void *p, int64_t i, int64_t v) {
+    reinterpret_cast<uint8_t *>(p)[i] = (uint8_t)v;
+  }
+};
+
+// ------------------------------------------------------------- division --
+// x / f and x % f for x < 2^47 f and 1 <= f <= 2^16 (so the quotient is
+// below 2^47).  The quotient is estimated in double precision -- x rounded to
+// 53 bits times the correctly rounded reciprocal of f, relative error at most
+// about 3 * 2^-53, i.e. an absolute error below 0.05 -- so its truncation is
+// within one of the true quotient; an exact integer remainder check fixes it.
+// (The "float divide + rarely taken exact integer fix-up" of "torch_ans
+// 0.3.0", Performance Tuning, CPU item 3.)
+__device__ __forceinline__ double freq_reciprocal(uint32_t f) {
+  return __drcp_rn((double)f);
+}
+
+__device__ __forceinline__ void divmod_freq(uint64_t x, uint32_t f, double rcp, uint64_t &q,
+                                            uint32_t &r) {
+  uint64_t qe = __double2ull_rz(__ull2double_rn(x) * rcp);
+  int64_t rem = (int64_t)(x - qe * (uint64_t)f);
+  if (rem < 0) {
+    qe -= 1;
+    rem += f;
+  } else if (rem >= (int64_t)f) {
+    qe += 1;
+    rem -= f;
+  }
+  q = qe;
+  r = (uint32_t)rem;
+}
+
+// One symbol op of the encoder: x -> (x / f) 2^16 + x mod f + start.
+__device__ __forceinline__ uint64_t enc_sym_step(uint64_t x, uint32_t start, uint32_t f,
+                                                 double rcp) {
+  uint64_t q;
+  uint32_t r;
+  divmod_freq(x, f, rcp, q, r);
+  return (q << kPrec) + r + start;
+}
+
+// ------------------------------------------------------- warp helpers --
+__device__ __forceinline__ uint32_t lanemask_lt() {
+  uint32_t m;
+  asm("mov.u32 %0, %%lanemask_lt;" : "=r"(m));
+  return m;
+}
+
+// ------------------------------------------------ bulk staging (TMA) ----
+// Copies `bytes` (multiple of 16, both addresses 16-B aligned) from global
+// into shared memory with one-dimensional bulk copies (cp.async.bulk, no
+// multicast) completing on an mbarrier.  The wait is bounded; on timeout the
+// status gets RANS_ERR_TIMEOUT and false is returned.
+__device__ __forceinline__ uint32_t smem_addr(const void *p) {
+  return (uint32_t)__cvta_generic_to_shared(p);
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity), "r"(1000u)
+      : "memory");
+  return ok != 0;
+}
+
+__device__ inline bool stage_to_smem(void *dst, const void *src, uint32_t bytes,
+                                     uint64_t *bar_storage, int32_t *status) {
+  const uint32_t bar = smem_addr(bar_storage);
+  if (threadIdx.x == 0) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(bar) : "memory");
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes)
+                 : "memory");
+    const uint32_t chunk = 32768;
+    const char *s = reinterpret_cast<const char *>(src);
+    uint32_t d = smem_addr(dst);
+    for (uint32_t off = 0; off < bytes; off += chunk) {
+      uint32_t sz = bytes - off < chunk ? bytes - off : chunk;
+      asm volatile(
+          "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, "
+          "[%3];" ::"r"(d + off),
+          "l"(s + off), "r"(sz), "r"(bar)
+          : "memory");
+    }
+  }
+  bool done = false;
+  for (uint32_t it = 0; it < (1u << 21); ++it) {
+    if (mbar_try_wait(bar, 0)) { done = true; break; }
+  }
+  if (!done) {
+    report(status, RANS_ERR_TIMEOUT, -1);
+    for (uint32_t it = 0; it < (1u << 21); ++it)
+      if (mbar_try_wait(bar, 0)) break;
+  }
+  __syncthreads();
+  return __syncthreads_and(done ? 1 : 0) != 0;
+}
+
+}  // namespace rb

@@ -1,0 +1,45 @@
+// rans_internal.h -- host-side launchers shared between the librans_b200
+// translation units (not part of the public ABI).
+#pragma once
+
+#include <cstdint>
+#include <cuda_runtime.h>
+
+#include "rans_b200.h"
+
+namespace rb {
+
+struct Geom;
+
+int launch_gaussian_lengths(const float *scales, int K, double tail, int32_t *lengths,
+                            int32_t *offsets, cudaStream_t st);
+int launch_gaussian_rows(const float *scales, int K, double tail, int32_t *cdfs, int Lmax,
+                         int32_t *lengths, int32_t *offsets, cudaStream_t st);
+int launch_pmf_rows(const float *pmfs, int K, int stride, const int32_t *pmf_lengths,
+                    const float *tail, int32_t *cdfs, int Lmax, int32_t *lengths,
+                    cudaStream_t st);
+uint64_t tables_bytes_bound(int K, int Lmax);
+int prepare_tables(const int32_t *cdfs, int K, int Lmax, const int32_t *lengths,
+                   const int32_t *offsets, void *blob, uint64_t blob_bytes, rans_tables *out,
+                   cudaStream_t st);
+
+// Encoder: codes every stream into its scratch slot and records its byte
+// length in lens[S].
+int launch_encode(const void *symbols, int sym_dtype, const int32_t *indexes,
+                  const rans_tables &t, const Geom &g, char *scratch, uint64_t *lens,
+                  int32_t *status, cudaStream_t st);
+// Compaction: exclusive scan of lens into offsets[S+1], then a copy of every
+// stream from the end of its scratch slot to out + offsets[k].
+int launch_compact(const Geom &g, const char *scratch, const uint64_t *lens, uint8_t *out,
+                   uint64_t out_capacity, uint64_t *offsets, int32_t *status, cudaStream_t st);
+int launch_decode(const uint8_t *in, uint64_t in_bytes, const uint64_t *offsets,
+                  const int32_t *indexes, const rans_tables &t, const Geom &g, void *symbols,
+                  int sym_dtype, int32_t *status, cudaStream_t st);
+int launch_debug_divide(const uint64_t *x, const uint32_t *f, int64_t n, uint64_t *q,
+                        uint32_t *r, cudaStream_t st);
+
+// Device properties cached per device.
+int num_sms(int device);
+int smem_optin(int device);
+
+}  // namespace rb

@@ -1,0 +1,462 @@
+// tables.cu -- CDF-table construction and the coder's prepared tables.
+//
+//  * Gaussian rows from a scale table ("kompressor" README, Getting Started:
+//    64 CDF rows for the y latent; "Benchmark notes", section 4: 200512 table
+//    entries = 64 rows x 3133).
+//  * pmf -> quantised CDF ("torch_ans 0.3.0", High-level API, init_params;
+//    FAQ: increasing positive integers up to 2^precision).
+//  * The decoder lookup table: the top q bits of the state's low 16 bits pick
+//    a slot that names the bucket directly or bounds a short search
+//    ("torch_ans 0.3.0", Usage: inverse-CDF decoding with a 2^q table and a
+//    bounded walk).
+//
+// One CUDA block quantises one row.  The steal step (every empty bucket takes
+// one unit from the narrowest bucket wider than 1, first on ties, in ascending
+// order of empty buckets) is computed in closed form: the units come from the
+// buckets in (width, index) order, each drained to width 1 before the next is
+// touched, so a threshold width t and a rank among the width-t buckets decide
+// every bucket's final width.
+#include <cmath>
+#include <cstring>
+#include <vector>
+
+#include "rans_common.cuh"
+#include "rans_internal.h"
+
+namespace rb {
+
+namespace {
+
+constexpr int kRowThreads = 256;
+
+// Block-wide sum / exclusive scan of a 64-bit value (kRowThreads threads).
+struct BlockScratch {
+  unsigned long long warp[kRowThreads / 32];
+  unsigned long long total;
+};
+
+__device__ unsigned long long block_sum(unsigned long long v, BlockScratch &sh) {
+  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(kFull, v, o);
+  __syncthreads();
+  if (lane == 0) sh.warp[wid] = v;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    unsigned long long t = 0;
+    for (int i = 0; i < kRowThreads / 32; ++i) t += sh.warp[i];
+    sh.total = t;
+  }
+  __syncthreads();
+  return sh.total;
+}
+
+// Returns the exclusive prefix of v over threads; *total gets the block sum.
+__device__ unsigned long long block_excl_scan(unsigned long long v, BlockScratch &sh,
+                                              unsigned long long *total) {
+  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+  unsigned long long inc = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    unsigned long long t = __shfl_up_sync(kFull, inc, o);
+    if (lane >= o) inc += t;
+  }
+  __syncthreads();
+  if (lane == 31) sh.warp[wid] = inc;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    unsigned long long run = 0;
+    for (int i = 0; i < kRowThreads / 32; ++i) {
+      unsigned long long w = sh.warp[i];
+      sh.warp[i] = run;
+      run += w;
+    }
+    sh.total = run;
+  }
+  __syncthreads();
+  *total = sh.total;
+  return sh.warp[wid] + inc - v;
+}
+
+// Scaled and rounded probability: round(p * 2^16) half away from zero, or
+// -1 when p is negative, not finite or too large.
+__device__ __forceinline__ long long scaled_freq(float p) {
+  float v = p * (float)kTotal;            // exact: times a power of two
+  float r = roundf(v);                    // half away from zero
+  if (!(r >= 0.0f) || (double)r > 4294967295.0) return -1;
+  return (long long)r;
+}
+
+// Quantises n probabilities (pf(i), the last one the tail mass) into row[0..n]
+// of a CDF row.  Returns RANS_OK or RANS_ERR_TABLE (same value on every
+// thread).  row[] is used as scratch for the widths.
+template <class PF>
+__device__ int quantise_row(const PF &pf, int n, int32_t *row, BlockScratch &sh) {
+  // pass 1: total of the rounded values
+  unsigned long long local = 0;
+  int bad = 0;
+  for (int i = threadIdx.x; i < n; i += kRowThreads) {
+    long long f = scaled_freq(pf(i));
+    if (f < 0) bad = 1; else local += (unsigned long long)f;
+  }
+  const unsigned long long T = block_sum(local, sh);
+  bad = __syncthreads_or(bad);
+  if (bad || T == 0) return RANS_ERR_TABLE;
+
+  // pass 2: widths of the rescaled running sum, floor(2^16 c / T)
+  unsigned long long carry = 0;
+  for (int base = 0; base < n; base += kRowThreads) {
+    int i = base + threadIdx.x;
+    unsigned long long f = 0;
+    if (i < n) f = (unsigned long long)scaled_freq(pf(i));
+    unsigned long long tot;
+    unsigned long long ex = block_excl_scan(f, sh, &tot) + carry;
+    if (i < n) {
+      unsigned long long c0 = ((unsigned long long)kTotal * ex) / T;
+      unsigned long long c1 = ((unsigned long long)kTotal * (ex + f)) / T;
+      row[i + 1] = (int32_t)(c1 - c0);
+    }
+    carry += tot;
+  }
+  __syncthreads();
+
+  // empty buckets
+  unsigned long long zl = 0;
+  for (int i = threadIdx.x; i < n; i += kRowThreads) zl += (row[i + 1] == 0);
+  const unsigned long long Z = block_sum(zl, sh);
+  if (Z > 0) {
+    // S(t) = sum over buckets with 1 < w <= t of (w - 1)
+    auto S = [&](long long t) -> unsigned long long {
+      unsigned long long s = 0;
+      for (int i = threadIdx.x; i < n; i += kRowThreads) {
+        long long w = row[i + 1];
+        if (w > 1 && w <= t) s += (unsigned long long)(w - 1);
+      }
+      return block_sum(s, sh);
+    };
+    if (S(kTotal) < Z) return RANS_ERR_TABLE;
+    long long lo = 2, hi = kTotal;
+    while (lo < hi) {
+      long long mid = (lo + hi) >> 1;
+      if (S(mid) >= Z) hi = mid; else lo = mid + 1;
+    }
+    const long long t = lo;
+    const unsigned long long R = Z - S(t - 1);
+    const unsigned long long full = R / (unsigned long long)(t - 1);
+    const unsigned long long part = R % (unsigned long long)(t - 1);
+    unsigned long long rank_carry = 0;
+    for (int base = 0; base < n; base += kRowThreads) {
+      int i = base + threadIdx.x;
+      long long w = i < n ? row[i + 1] : 0;
+      unsigned long long tot;
+      unsigned long long rk = block_excl_scan(w == t ? 1ull : 0ull, sh, &tot) + rank_carry;
+      if (i < n) {
+        if (w > 1 && w < t) w = 1;
+        else if (w == t) {
+          if (rk < full) w = 1;
+          else if (rk == full) w -= (long long)part;
+        }
+        if (w == 0) w = 1;
+        row[i + 1] = (int32_t)w;
+      }
+      rank_carry += tot;
+    }
+    __syncthreads();
+  }
+
+  // widths -> CDF in place
+  unsigned long long run = 0;
+  for (int base = 0; base < n; base += kRowThreads) {
+    int i = base + threadIdx.x;
+    unsigned long long w = i < n ? (unsigned long long)row[i + 1] : 0ull;
+    unsigned long long tot;
+    unsigned long long ex = block_excl_scan(w, sh, &tot) + run;
+    __syncthreads();
+    if (i < n) row[i + 1] = (int32_t)(ex + w);
+    run += tot;
+  }
+  if (threadIdx.x == 0) row[0] = 0;
+  __syncthreads();
+  return RANS_OK;
+}
+
+// Standard normal CDF as 0.5 erfc(-z / sqrt 2), in double.
+__device__ __forceinline__ double std_normal_cdf(double z) {
+  return 0.5 * erfc(-z / sqrt(2.0));
+}
+
+__device__ __forceinline__ int gaussian_center(float scale, double tail, int32_t *center) {
+  if (!(scale > 0.0f) || !isfinite(scale) || !(tail > 0.0) || !(tail < 1.0))
+    return RANS_ERR_ARG;
+  double m = -normcdfinv(tail / 2.0);
+  double c = ceil((double)scale * m);
+  if (!(c >= 0.0) || c > 32766.0) return RANS_ERR_ARG;
+  *center = (int32_t)c;
+  return RANS_OK;
+}
+
+__global__ void gaussian_lengths_kernel(const float *scales, int K, double tail,
+                                        int32_t *lengths, int32_t *offsets) {
+  int r = blockIdx.x * blockDim.x + threadIdx.x;
+  if (r >= K) return;
+  int32_t c = 0;
+  int st = gaussian_center(scales[r], tail, &c);
+  lengths[r] = st ? st : 2 * c + 3;
+  offsets[r] = st ? 0 : -c;
+}
+
+struct GaussPmf {
+  int center, npmf;
+  double s;
+  __device__ float operator()(int i) const {
+    if (i == npmf) return (float)(2.0 * std_normal_cdf((-0.5 - (double)center) / s));
+    double d = fabs((double)(i - center));
+    double upper = std_normal_cdf((0.5 - d) / s);
+    double lower = std_normal_cdf((-0.5 - d) / s);
+    return (float)(upper - lower);
+  }
+};
+
+struct GivenPmf {
+  const float *p;
+  int n;
+  float tail;
+  __device__ float operator()(int i) const { return i == n ? tail : p[i]; }
+};
+
+__global__ void __launch_bounds__(kRowThreads)
+    gaussian_rows_kernel(const float *scales, double tail, int32_t *cdfs, int Lmax,
+                         int32_t *lengths, int32_t *offsets) {
+  __shared__ BlockScratch sh;
+  const int r = blockIdx.x;
+  int32_t *row = cdfs + (size_t)r * (size_t)Lmax;
+  int32_t c = 0;
+  int st = gaussian_center(scales[r], tail, &c);
+  int len = 2 * c + 3;
+  if (st == RANS_OK && len > Lmax) st = RANS_ERR_CAPACITY;
+  if (st == RANS_OK) {
+    GaussPmf pf{c, 2 * c + 1, (double)scales[r]};
+    st = quantise_row(pf, 2 * c + 2, row, sh);
+  }
+  for (int j = (st == RANS_OK ? len : 0) + threadIdx.x; j < Lmax; j += kRowThreads) row[j] = 0;
+  if (threadIdx.x == 0) {
+    lengths[r] = st ? st : len;
+    offsets[r] = st ? 0 : -c;
+  }
+}
+
+__global__ void __launch_bounds__(kRowThreads)
+    pmf_rows_kernel(const float *pmfs, int stride, const int32_t *pmf_lengths,
+                    const float *tail, int32_t *cdfs, int Lmax, int32_t *lengths) {
+  __shared__ BlockScratch sh;
+  const int r = blockIdx.x;
+  int32_t *row = cdfs + (size_t)r * (size_t)Lmax;
+  int n = pmf_lengths[r];
+  int st = RANS_OK;
+  if (n < 0 || n > stride) st = RANS_ERR_ARG;
+  else if (n + 2 > Lmax) st = RANS_ERR_CAPACITY;
+  if (st == RANS_OK) {
+    GivenPmf pf{pmfs + (size_t)r * (size_t)stride, n, tail[r]};
+    st = quantise_row(pf, n + 1, row, sh);
+  }
+  for (int j = (st == RANS_OK ? n + 2 : 0) + threadIdx.x; j < Lmax; j += kRowThreads) row[j] = 0;
+  if (threadIdx.x == 0) lengths[r] = st ? st : n + 2;
+}
+
+// ---- prepared tables ----------------------------------------------------
+
+// Validates row r and writes its packed buckets.  One block per row.
+__global__ void pack_buckets_kernel(const int32_t *cdfs, int Lmax, const RowMeta *meta,
+                                    const int32_t *lengths, uint32_t *buckets,
+                                    int32_t *status) {
+  const int r = blockIdx.x;
+  const int32_t *row = cdfs + (size_t)r * (size_t)Lmax;
+  const int len = lengths[r];
+  const uint32_t base = meta[r].bucket_base;
+  if (threadIdx.x == 0 && (row[0] != 0 || row[len - 1] != (int32_t)kTotal))
+    report(status, RANS_ERR_TABLE, r);
+  for (int j = threadIdx.x; j < len - 1; j += blockDim.x) {
+    int32_t a = row[j], b = row[j + 1];
+    if (!(b > a) || a < 0 || b > (int32_t)kTotal) {
+      report(status, RANS_ERR_TABLE, r);
+      continue;
+    }
+    buckets[base + j] = (uint32_t)(a & 0xffff) | ((uint32_t)(b - a - 1) << 16);
+  }
+}
+
+// Largest j in [0, nb) with row[j] <= v (row strictly increasing, row[0]=0).
+__device__ __forceinline__ int bucket_of(const int32_t *row, int nb, int v) {
+  int lo = 0, hi = nb - 1;
+  while (lo < hi) {
+    int mid = (lo + hi + 1) >> 1;
+    if (row[mid] <= v) lo = mid; else hi = mid - 1;
+  }
+  return lo;
+}
+
+__global__ void fill_slots_kernel(const int32_t *cdfs, int Lmax, const RowMeta *meta,
+                                  const int32_t *lengths, uint32_t *slots) {
+  const int r = blockIdx.y;
+  const RowMeta m = meta[r];
+  const int shift = (int)slot_shift(m.slot);
+  const int nslots = 1 << (16 - shift);
+  const int t = blockIdx.x * blockDim.x + threadIdx.x;
+  if (t >= nslots) return;
+  const int32_t *row = cdfs + (size_t)r * (size_t)Lmax;
+  const int nb = lengths[r] - 1;
+  const int w = 1 << shift;
+  const int a = t * w, b = a + w - 1;
+  const int lo = bucket_of(row, nb, a);
+  const int hi = bucket_of(row, nb, b);
+  const int inside = hi - lo;
+  uint32_t code;
+  if (inside == 0) code = (uint32_t)w;
+  else if (inside == 1) code = (uint32_t)(row[lo + 1] - a);
+  else code = 0x8000u | (uint32_t)(inside < 0x7fff ? inside : 0x7fff);
+  slots[slot_base(m.slot) + t] = (uint32_t)lo | (code << 16);
+}
+
+int ceil_log2(int64_t v) {
+  int q = 0;
+  while ((int64_t(1) << q) < v) ++q;
+  return q;
+}
+
+}  // namespace
+
+// ---- host entry points (called from api.cu) ------------------------------
+
+int launch_gaussian_lengths(const float *scales, int K, double tail, int32_t *lengths,
+                            int32_t *offsets, cudaStream_t st) {
+  gaussian_lengths_kernel<<<(K + 127) / 128, 128, 0, st>>>(scales, K, tail, lengths, offsets);
+  return cudaGetLastError() == cudaSuccess ? RANS_OK : RANS_ERR_CUDA;
+}
+
+int launch_gaussian_rows(const float *scales, int K, double tail, int32_t *cdfs, int Lmax,
+                         int32_t *lengths, int32_t *offsets, cudaStream_t st) {
+  gaussian_rows_kernel<<<K, kRowThreads, 0, st>>>(scales, tail, cdfs, Lmax, lengths, offsets);
+  return cudaGetLastError() == cudaSuccess ? RANS_OK : RANS_ERR_CUDA;
+}
+
+int launch_pmf_rows(const float *pmfs, int K, int stride, const int32_t *pmf_lengths,
+                    const float *tail, int32_t *cdfs, int Lmax, int32_t *lengths,
+                    cudaStream_t st) {
+  pmf_rows_kernel<<<K, kRowThreads, 0, st>>>(pmfs, stride, pmf_lengths, tail, cdfs, Lmax,
+                                              lengths);
+  return cudaGetLastError() == cudaSuccess ? RANS_OK : RANS_ERR_CUDA;
+}
+
+uint64_t tables_bytes_bound(int K, int Lmax) {
+  if (K <= 0 || Lmax < 2) return 0;
+  const int64_t nb = (int64_t)Lmax - 1;
+  int q = ceil_log2(nb) + 1;
+  q = q < kMinQ ? kMinQ : (q > kMaxQ ? kMaxQ : q);
+  return (uint64_t)kHeaderBytes + pad16(16ull * K) + pad16(4ull * K * nb) +
+         pad16(4ull * K * (1ull << q));
+}
+
+int prepare_tables(const int32_t *cdfs, int K, int Lmax, const int32_t *lengths,
+                   const int32_t *offsets, void *blob, uint64_t blob_bytes, rans_tables *out,
+                   cudaStream_t st) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return RANS_ERR_CUDA;
+  if (K > 65535) return RANS_ERR_ARG;  // one grid row per table row below
+  std::vector<int32_t> len(K), off(K);
+  if (cudaMemcpyAsync(len.data(), lengths, sizeof(int32_t) * K, cudaMemcpyDeviceToHost, st) !=
+          cudaSuccess ||
+      cudaMemcpyAsync(off.data(), offsets, sizeof(int32_t) * K, cudaMemcpyDeviceToHost, st) !=
+          cudaSuccess ||
+      cudaStreamSynchronize(st) != cudaSuccess)
+    return RANS_ERR_CUDA;
+
+  std::vector<RowMeta> meta(K);
+  std::vector<int> q(K);
+  uint64_t nbuckets = 0;
+  int max_nb = 0;
+  for (int r = 0; r < K; ++r) {
+    if (len[r] < 0) return len[r];
+    if (len[r] < 2 || len[r] > Lmax) return RANS_ERR_TABLE;
+    const int nb = len[r] - 1;
+    meta[r].bucket_base = (uint32_t)nbuckets;
+    meta[r].maxv = (uint32_t)(len[r] - 2);
+    meta[r].offset = off[r];
+    nbuckets += (uint64_t)nb;
+    if (nb > max_nb) max_nb = nb;
+    int qq = ceil_log2(nb) + 1;
+    q[r] = qq < kMinQ ? kMinQ : (qq > kMaxQ ? kMaxQ : qq);
+  }
+  if (nbuckets > (1ull << 31)) return RANS_ERR_ARG;
+
+  const uint32_t meta_bytes = pad16(16ull * K);
+  const uint32_t bucket_bytes = pad16(4ull * nbuckets);
+  int optin = 0;
+  cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
+  const int64_t budget = (int64_t)optin - 1024;  // room for barriers and scratch
+  auto slot_total = [&]() {
+    uint64_t t = 0;
+    for (int r = 0; r < K; ++r) t += 1ull << q[r];
+    return t;
+  };
+  const bool enc_smem = (int64_t)meta_bytes + bucket_bytes <= budget;
+  bool dec_smem = false;
+  if (enc_smem) {
+    const int64_t room = budget - meta_bytes - bucket_bytes;
+    // Halve the largest row's lookup until the three sections fit.
+    while ((int64_t)pad16(4ull * slot_total()) > room) {
+      int best = -1;
+      for (int r = 0; r < K; ++r)
+        if (q[r] > kMinQ && (best < 0 || q[r] >= q[best])) best = r;
+      if (best < 0) break;
+      --q[best];
+    }
+    dec_smem = (int64_t)pad16(4ull * slot_total()) <= room;
+  }
+  uint64_t sbase = 0;
+  for (int r = 0; r < K; ++r) {
+    meta[r].slot = (uint32_t)sbase | ((uint32_t)(16 - q[r]) << 27);
+    sbase += 1ull << q[r];
+  }
+  if (sbase >= (1ull << 27)) return RANS_ERR_ARG;
+  const uint32_t slot_bytes = pad16(4ull * sbase);
+  const uint64_t need = (uint64_t)kHeaderBytes + meta_bytes + bucket_bytes + slot_bytes;
+  if (blob == nullptr || blob_bytes < need) return RANS_ERR_CAPACITY;
+  if ((reinterpret_cast<uintptr_t>(blob) & 255) != 0) return RANS_ERR_ARG;
+
+  char *b = reinterpret_cast<char *>(blob);
+  int32_t *status = reinterpret_cast<int32_t *>(b);
+  RowMeta *dmeta = reinterpret_cast<RowMeta *>(b + kHeaderBytes);
+  uint32_t *dbuckets = reinterpret_cast<uint32_t *>(b + kHeaderBytes + meta_bytes);
+  uint32_t *dslots = reinterpret_cast<uint32_t *>(b + kHeaderBytes + meta_bytes + bucket_bytes);
+  if (cudaMemsetAsync(b, 0, kHeaderBytes, st) != cudaSuccess) return RANS_ERR_CUDA;
+  if (cudaMemcpyAsync(dmeta, meta.data(), sizeof(RowMeta) * K, cudaMemcpyHostToDevice, st) !=
+      cudaSuccess)
+    return RANS_ERR_CUDA;
+  pack_buckets_kernel<<<K, 256, 0, st>>>(cdfs, Lmax, dmeta, lengths, dbuckets, status);
+  int maxslots = 0;
+  for (int r = 0; r < K; ++r) maxslots = maxslots > (1 << q[r]) ? maxslots : (1 << q[r]);
+  dim3 grid((maxslots + 255) / 256, K);
+  fill_slots_kernel<<<grid, 256, 0, st>>>(cdfs, Lmax, dmeta, lengths, dslots);
+  if (cudaGetLastError() != cudaSuccess) return RANS_ERR_CUDA;
+  StatusWord sw;
+  if (cudaMemcpyAsync(&sw, status, sizeof(sw), cudaMemcpyDeviceToHost, st) != cudaSuccess ||
+      cudaStreamSynchronize(st) != cudaSuccess)
+    return RANS_ERR_CUDA;
+  if (sw.code != 0) return sw.code;
+
+  out->blob = blob;
+  out->blob_bytes = need;
+  out->K = K;
+  out->max_buckets = max_nb;
+  out->n_buckets = (int64_t)nbuckets;
+  out->n_slots = (int64_t)sbase;
+  out->meta_bytes = meta_bytes;
+  out->bucket_bytes = bucket_bytes;
+  out->slot_bytes = slot_bytes;
+  out->enc_in_smem = enc_smem ? 1 : 0;
+  out->dec_in_smem = dec_smem ? 1 : 0;
+  out->device = dev;
+  return RANS_OK;
+}
+
+}  // namespace rb

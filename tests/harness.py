@@ -1,0 +1,64 @@
+"""Runs one workload through the oracle and through librans_b200 (C ABI) so
+tests can compare them.  Both sides code the same seeded arrays; the GPU
+side never feeds the oracle."""
+import numpy as np
+import torch
+
+import oracle as O
+import rans_entropy_coding_b200 as rb
+
+
+def oracle_tables(w):
+    if "scales" in w:
+        c, l, o = O.build_cdfs_from_scales(w["scales"], w["tail_mass"])
+    else:
+        c, l = O.build_cdfs_from_pmfs(w["pmfs"], w["pmf_lengths"], w["tail"])
+        o = np.asarray(w["offsets"], dtype=np.int32)
+    return c, l, o
+
+
+def gpu_rows(w, dev="cuda"):
+    """CDF rows built on the GPU: (cdfs, lengths, offsets) CUDA tensors."""
+    if "scales" in w:
+        return rb.Tables.build_from_scales(torch.from_numpy(np.asarray(w["scales"])).to(dev),
+                                           w["tail_mass"])
+    cdfs, lengths = rb.Tables.build_from_pmfs(
+        torch.from_numpy(np.ascontiguousarray(w["pmfs"])).to(dev),
+        torch.from_numpy(np.asarray(w["pmf_lengths"], np.int32)).to(dev),
+        torch.from_numpy(np.asarray(w["tail"], np.float32)).to(dev))
+    return cdfs, lengths, torch.from_numpy(np.asarray(w["offsets"], np.int32)).to(dev)
+
+
+def tables_from_numpy(c, l, o, dev="cuda"):
+    return rb.Tables(torch.from_numpy(np.ascontiguousarray(c)).to(dev),
+                     torch.from_numpy(np.ascontiguousarray(l)).to(dev),
+                     torch.from_numpy(np.ascontiguousarray(o)).to(dev))
+
+
+def chunking_of(w, dev="cuda"):
+    return rb.Chunking.from_spec(w["chunking"], w["W"], w["index_block"], device=dev)
+
+
+def gpu_encode_decode(w, tables, dev="cuda", expect_ok=True):
+    """Returns (bytes, offsets, decoded, enc_status, dec_status) as numpy."""
+    sym = torch.from_numpy(np.ascontiguousarray(w["symbols"]).reshape(-1)).to(dev)
+    idx = torch.from_numpy(np.ascontiguousarray(w["indexes"], dtype=np.int32)).to(dev)
+    ch = chunking_of(w, dev)
+    out, offs, ws = rb.encode_with_indexes(sym, idx, tables, ch)
+    est = rb.rans_get_status(ws.enc)
+    total = int(offs[-1].item()) if offs.numel() else 0
+    if expect_ok:
+        assert est == rb.OK, rb.RansError(est, "encode")
+    data = out[:total] if est == rb.OK else out[:0]
+    dec, wsd = rb.decode_with_indexes(data, offs, idx, tables, ch, sym.numel(), sym.dtype, ws=ws)
+    dst = rb.rans_get_status(wsd)
+    if expect_ok:
+        assert dst == rb.OK, rb.RansError(dst, "decode")
+    return (data.cpu().numpy(), offs.cpu().numpy().astype(np.uint64), dec.cpu().numpy(), est,
+            dst)
+
+
+def oracle_encode(w, c, l, o, streams=None):
+    sym = np.asarray(w["symbols"]).reshape(-1)
+    return O.encode_with_indexes(sym, w["indexes"], c, l, o, w["chunking"], W=w["W"],
+                                 index_block=w["index_block"], streams=streams)

@@ -1,0 +1,323 @@
+"""GPU parity: librans_b200 (through its C ABI) against the CPU oracle.
+
+Integer work, so the bar is exact: CDF tables identical, every stream's bytes
+and the offsets identical, decoded symbols identical, on the same seeded
+inputs."""
+import numpy as np
+import pytest
+import torch
+
+import oracle as O
+import rans_entropy_coding_b200 as rb
+import workloads as WL
+from harness import (chunking_of, gpu_encode_decode, gpu_rows, oracle_encode, oracle_tables,
+                     tables_from_numpy)
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _cuda():
+    if not torch.cuda.is_available():
+        pytest.fail("a CUDA device is required for the gpu tests")
+    from rans_entropy_coding_b200 import build
+    build.build()
+    rb.lib()
+    torch.cuda.set_device(0)
+
+
+def _edge_tiny(W=1, seed=0, dtype=np.int32):
+    """The tiny workload plus each row's range edges (centre, centre + 1 --
+    the escape with raw value 0 -- and -centre - 1)."""
+    w = WL.tiny(seed=seed)
+    w["W"] = W
+    c, l, o = oracle_tables(w)
+    sym = w["symbols"].astype(np.int64)
+    rng = np.random.Generator(np.random.PCG64(99))
+    for r in range(len(l)):
+        cen = -int(o[r])
+        for v in (cen, cen + 1, -cen - 1, -cen, 0):
+            pos = int(rng.integers(3, sym.size))
+            sym[pos] = v
+            w["indexes"][pos] = r
+    if dtype == np.int16:
+        sym = np.clip(sym, -32768, 32767)
+    w["symbols"] = sym.astype(dtype)
+    return w
+
+
+def _check_streams(w, exact_tables=True):
+    c, l, o = oracle_tables(w)
+    tables = tables_from_numpy(c, l, o)
+    data, offs, dec, _, _ = gpu_encode_decode(w, tables)
+    want, woffs = oracle_encode(w, c, l, o)
+    assert offs.tolist() == woffs.tolist()
+    assert data.size == want.size
+    if not np.array_equal(data, want):
+        bad = np.nonzero(data != want)[0][0]
+        s = int(np.searchsorted(woffs, bad, side="right")) - 1
+        raise AssertionError("stream %d differs at byte %d" % (s, bad - int(woffs[s])))
+    sym = np.asarray(w["symbols"]).reshape(-1)
+    assert np.array_equal(dec, sym)
+    return data, offs
+
+
+# ------------------------------------------------------------- division --
+def test_division_is_exact_for_every_frequency():
+    f = np.arange(1, 65537, dtype=np.uint64)
+    rng = np.random.Generator(np.random.PCG64(5))
+    xs = [np.full_like(f, 1 << 31), (f << np.uint64(47)) - np.uint64(1),
+          (f << np.uint64(47)) - f, (f << np.uint64(47)) - f - np.uint64(1),
+          (f << np.uint64(31)) + np.uint64(12345),
+          np.uint64(1 << 31) + (rng.random(f.size) * ((f << np.uint64(47)) - np.uint64(1 << 31))
+                                .astype(np.float64)).astype(np.uint64)]
+    for x in xs:
+        x = np.minimum(x, (f << np.uint64(47)) - np.uint64(1))
+        xt = torch.from_numpy(x.astype(np.int64)).cuda()
+        ft = torch.from_numpy(f.astype(np.int32)).cuda()
+        q = torch.empty_like(xt)
+        r = torch.empty_like(ft)
+        rb.check(rb.rans_debug_divide(xt, ft, q, r))
+        torch.cuda.synchronize()
+        assert np.array_equal(q.cpu().numpy().astype(np.uint64), x // f)
+        assert np.array_equal(r.cpu().numpy().astype(np.uint64), x % f)
+
+
+# --------------------------------------------------------------- tables --
+@pytest.mark.parametrize("which", ["tiny", "y64", "z", "sweep"])
+def test_tables_match_oracle(which):
+    w = {"tiny": WL.tiny(), "y64": WL.y_latent(), "z": WL.z_latent(),
+         "sweep": WL.sweep(log2_n=16)}[which]
+    c, l, o = oracle_tables(w)
+    gc, gl, go = gpu_rows(w)
+    torch.cuda.synchronize()
+    gc, gl, go = gc.cpu().numpy(), gl.cpu().numpy(), go.cpu().numpy()
+    assert gl.tolist() == l.tolist()
+    assert go.tolist() == o.tolist()
+    for r in range(len(l)):
+        assert gc[r, :l[r]].tolist() == c[r, :l[r]].tolist(), r
+
+
+def test_random_pmf_tables_match_oracle():
+    rng = np.random.Generator(np.random.PCG64(21))
+    K, S = 40, 700
+    pmfs = np.zeros((K, S), np.float32)
+    lens = rng.integers(1, S, size=K).astype(np.int32)
+    tails = np.zeros(K, np.float32)
+    for k in range(K):
+        n = lens[k]
+        kind = k % 4
+        if kind == 0:
+            p = rng.random(n) ** 10
+        elif kind == 1:
+            x = np.arange(n) - n / 2
+            p = np.exp(-0.5 * (x / rng.uniform(0.2, n / 3)) ** 2)
+        elif kind == 2:
+            p = rng.random(n)
+            p[rng.random(n) < 0.7] = 0
+            p[0] = 1
+        else:
+            p = 1.0 / (np.arange(n) + 1.0) ** 2.5
+        p = p / p.sum()
+        pmfs[k, :n] = (p * 0.999).astype(np.float32)
+        tails[k] = np.float32(0.001 if kind != 3 else 0.0)
+    w = dict(pmfs=pmfs, pmf_lengths=lens, tail=tails, offsets=np.zeros(K, np.int32))
+    c, l, _ = oracle_tables(w)
+    gc, gl, _ = gpu_rows(w)
+    gc, gl = gc.cpu().numpy(), gl.cpu().numpy()
+    assert gl.tolist() == l.tolist()
+    for r in range(K):
+        assert gc[r, :l[r]].tolist() == c[r, :l[r]].tolist(), r
+
+
+def test_bad_rows_are_reported():
+    pm = torch.tensor([[0.5, -0.1, 0.6], [0.0, 0.0, 0.0], [np.nan, 0.5, 0.5]],
+                      dtype=torch.float32, device="cuda")
+    cdfs, lens = rb.Tables.build_from_pmfs(pm, torch.tensor([3, 3, 3], dtype=torch.int32,
+                                                            device="cuda"),
+                                           torch.zeros(3, device="cuda"))
+    assert (lens.cpu() < 0).all()
+    sc = torch.tensor([1.0, -1.0], device="cuda")
+    lens = torch.empty(2, dtype=torch.int32, device="cuda")
+    offs = torch.empty(2, dtype=torch.int32, device="cuda")
+    rb.check(rb.rans_gaussian_lengths(sc, 1e-9, lens, offs))
+    assert lens[0].item() > 0 and lens[1].item() < 0
+    # a non-increasing row is rejected by prepare
+    c = torch.tensor([[0, 100, 100, 65536]], dtype=torch.int32, device="cuda")
+    with pytest.raises(rb.RansError) as e:
+        rb.Tables(c, torch.tensor([4], dtype=torch.int32, device="cuda"),
+                  torch.zeros(1, dtype=torch.int32, device="cuda"))
+    assert e.value.status == rb.ERR_TABLE
+
+
+# -------------------------------------------------------------- streams --
+@pytest.mark.parametrize("W", [1, 32])
+def test_tiny_with_range_edges(W):
+    _check_streams(_edge_tiny(W))
+
+
+def test_tiny_int16_symbols():
+    _check_streams(_edge_tiny(32, seed=3, dtype=np.int16))
+    _check_streams(_edge_tiny(1, seed=4, dtype=np.int16))
+
+
+@pytest.mark.parametrize("W", [1, 32])
+def test_z_latent(W):
+    w = WL.z_latent()
+    w["W"] = W
+    _check_streams(w)
+
+
+@pytest.mark.parametrize("W", [1, 32])
+def test_y_latent(W):
+    _check_streams(WL.y_latent(W=W))
+
+
+def test_batch_two_images_tiled():
+    _check_streams(WL.y_batch(n_images=2))
+
+
+@pytest.mark.parametrize("W", [1, 32])
+def test_batch_small_ragged_tiles(W):
+    """Tiles narrower than a warp and a channel group that does not divide C."""
+    w = WL.y_batch(n_images=1, cg=5, th=7, tw=11)
+    w["W"] = W
+    _check_streams(w)
+
+
+def test_tiled_with_index_blocks():
+    w = WL.y_batch(n_images=1, cg=4, th=16, tw=48)
+    n = np.asarray(w["symbols"]).size
+    rng = np.random.Generator(np.random.PCG64(8))
+    w["index_block"] = 64
+    w["indexes"] = rng.integers(0, 64, size=n // 64).astype(np.int32)
+    _check_streams(w)
+
+
+def test_sweep_uint8_blocks():
+    _check_streams(WL.sweep(log2_n=20, n_streams=32))
+
+
+def test_sweep_uint8_single_state():
+    w = WL.sweep(log2_n=16, n_streams=8)
+    w["W"] = 1
+    _check_streams(w)
+
+
+@pytest.mark.parametrize("W", [1, 32])
+def test_explicit_chunking_with_empty_streams(W):
+    w = WL.tiny(seed=6)
+    w["W"] = W
+    n = w["symbols"].size
+    starts = [0, 0, 5, 5, 37, 100, 100, 1500, n, n]
+    w["chunking"] = dict(kind="explicit", starts=starts)
+    _check_streams(w)
+
+
+@pytest.mark.parametrize("W", [1, 32])
+def test_more_streams_than_symbols(W):
+    w = WL.tiny(seed=7, n=45)
+    w["W"] = W
+    w["chunking"] = dict(kind="contig", n_streams=64)
+    _check_streams(w)
+
+
+def test_all_escape_row():
+    cdf = np.array([[0, 65536] + [0] * 3], dtype=np.int32)
+    rng = np.random.Generator(np.random.PCG64(12))
+    sym = rng.integers(-2**31, 2**31 - 1, size=3000, dtype=np.int64).astype(np.int32)
+    sym[:5] = [0, -1, 1, np.iinfo(np.int32).min, np.iinfo(np.int32).max]
+    for W in (1, 32):
+        w = dict(symbols=sym, indexes=np.zeros(3000, np.int32),
+                 chunking=dict(kind="contig", n_streams=3), W=W, index_block=1)
+        c, l, o = cdf, np.array([2], np.int32), np.array([0], np.int32)
+        tables = tables_from_numpy(c, l, o)
+        data, offs, dec, _, _ = gpu_encode_decode(w, tables)
+        want, woffs = oracle_encode(w, c, l, o)
+        assert offs.tolist() == woffs.tolist() and np.array_equal(data, want)
+        assert np.array_equal(dec, sym)
+
+
+def test_empty_input():
+    w = WL.tiny(n=0)
+    for W in (1, 32):
+        w["W"] = W
+        data, offs = _check_streams(w)
+        assert data.size == 8 * W
+
+
+def test_gpu_built_tables_code_like_oracle_tables():
+    w = WL.y_latent(W=32)
+    gpu_tables = rb.Tables(*gpu_rows(w))
+    data, offs, dec, _, _ = gpu_encode_decode(w, gpu_tables)
+    c, l, o = oracle_tables(w)
+    want, woffs = oracle_encode(w, c, l, o)
+    assert np.array_equal(data, want) and offs.tolist() == woffs.tolist()
+
+
+# --------------------------------------------------------------- errors --
+def _coded(w):
+    c, l, o = oracle_tables(w)
+    tables = tables_from_numpy(c, l, o)
+    data, offs, dec, _, _ = gpu_encode_decode(w, tables)
+    return tables, data, offs
+
+
+def _decode_status(w, tables, data, offs, indexes=None):
+    ch = chunking_of(w)
+    idx = torch.from_numpy(np.asarray(w["indexes"] if indexes is None else indexes,
+                                      np.int32)).cuda()
+    d = torch.from_numpy(data).cuda()
+    o = torch.from_numpy(offs.astype(np.int64)).cuda()
+    n = np.asarray(w["symbols"]).size
+    out = torch.empty(n, dtype=torch.int32, device="cuda")
+    ws = rb.aligned_empty(256)
+    rb.check(rb.rans_decode_with_indexes(d, o, idx, n, tables, ch, out, ws))
+    return rb.rans_get_status(ws)
+
+
+@pytest.mark.parametrize("W", [1, 32])
+def test_decoder_reports_corrupt_streams(W):
+    w = WL.y_latent(W=W)
+    tables, data, offs = _coded(w)
+    assert _decode_status(w, tables, data, offs) == rb.OK
+    # a word dropped from the end of stream 3
+    o2 = offs.copy()
+    o2[4:] -= 4
+    d2 = np.concatenate([data[:int(offs[4]) - 4], data[int(offs[4]):]])
+    assert _decode_status(w, tables, d2, o2) == rb.ERR_CORRUPT
+    # a flipped byte inside stream 5's words
+    d3 = data.copy()
+    d3[int(offs[5]) + 300] ^= 0x5A
+    assert _decode_status(w, tables, d3, offs) == rb.ERR_CORRUPT
+    # offsets running past the buffer
+    o4 = offs.copy()
+    o4[-1] += 64
+    assert _decode_status(w, tables, data, o4) == rb.ERR_CORRUPT
+    # an index out of range
+    bad = np.asarray(w["indexes"]).copy()
+    bad[777] = 1000
+    assert _decode_status(w, tables, data, offs, bad) == rb.ERR_INDEX
+
+
+def test_encoder_reports_bad_index_and_capacity():
+    w = WL.y_latent(W=32)
+    c, l, o = oracle_tables(w)
+    tables = tables_from_numpy(c, l, o)
+    sym = torch.from_numpy(np.asarray(w["symbols"]).reshape(-1)).cuda()
+    idx = torch.from_numpy(np.asarray(w["indexes"], np.int32)).cuda()
+    ch = chunking_of(w)
+    ws = rb.Workspaces(ch, sym.numel())
+    bad = idx.clone()
+    bad[12345] = -3
+    rb.check(rb.rans_encode_with_indexes(sym, bad, sym.numel(), tables, ch, ws.out, ws.offsets,
+                                         ws.enc))
+    assert rb.rans_get_status(ws.enc) == rb.ERR_INDEX
+    small = ws.out[:1000]
+    rb.check(rb.rans_encode_with_indexes(sym, idx, sym.numel(), tables, ch, small, ws.offsets,
+                                         ws.enc))
+    assert rb.rans_get_status(ws.enc) == rb.ERR_CAPACITY
+    # a workspace that is too small is refused on the host
+    st = rb.rans_encode_with_indexes(sym, idx, sym.numel(), tables, ch, ws.out, ws.offsets,
+                                     ws.enc[:1 << 20])
+    assert st == rb.ERR_CAPACITY
