@@ -46,6 +46,7 @@ def parse():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--group", type=int, default=4, help="channels per stream")
+    ap.add_argument("--images", type=int, default=N_IMAGES, help="images per GPU")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-clocks", action="store_true")
@@ -136,9 +137,8 @@ class ClockSampler:
                 "samples": len(rows)}
 
 
-def load_inputs(rank, group):
-    w = WL.y_batch(n_images=N_IMAGES, first_image=N_IMAGES * rank, cg=group)
-    return w
+def load_inputs(rank, group, images=N_IMAGES):
+    return WL.y_batch(n_images=images, first_image=images * rank, cg=group)
 
 
 # --------------------------------------------------------- CPU oracle leg --
@@ -203,7 +203,7 @@ def run_ours(args, world, rank, local):
     rb.lib()
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
-    w = load_inputs(rank, args.group)
+    w = load_inputs(rank, args.group, args.images)
     sym_np = np.ascontiguousarray(np.asarray(w["symbols"]).reshape(-1))
     idx_np = np.ascontiguousarray(w["indexes"], dtype=np.int32)
     n = sym_np.size

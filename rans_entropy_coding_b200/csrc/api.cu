@@ -60,6 +60,7 @@ int make_geom(const rans_chunking *ch, int64_t n, Geom &g) {
       g.S = ch->n_streams;
       g.per = cdiv(n, g.S);
       max_n = g.per;
+      if (g.per >= (int64_t(1) << 31) - 64) return RANS_ERR_ARG;
       break;
     case RANS_CHUNK_EXPLICIT:
       if (ch->n_streams < 0 || (ch->n_streams > 0 && ch->stream_starts == nullptr))
@@ -83,6 +84,43 @@ int make_geom(const rans_chunking *ch, int64_t n, Geom &g) {
       g.ntx = cdiv(W, g.tw);
       g.S = B * g.ng * g.nty * g.ntx;
       max_n = (g.cg < C ? g.cg : C) * (g.th < H ? g.th : H) * (g.tw < W ? g.tw : W);
+      if (C * H * W >= (int64_t(1) << 31) - 64) return RANS_ERR_ARG;
+      {
+        // tile classes (last group?, last tile row?, last tile column?), largest first
+        const int64_t full[3] = {C % g.cg ? g.ng - 1 : g.ng, H % g.th ? g.nty - 1 : g.nty,
+                                 W % g.tw ? g.ntx - 1 : g.ntx};
+        const int64_t part[3] = {C % g.cg ? 1 : 0, H % g.th ? 1 : 0, W % g.tw ? 1 : 0};
+        const int64_t fsz[3] = {g.cg, g.th, g.tw};
+        const int64_t psz[3] = {C % g.cg, H % g.th, W % g.tw};
+        int64_t size[8], count[8];
+        int bits[8], nc = 0;
+        for (int b = 0; b < 8; ++b) {
+          int64_t cnt = B, sz = 1;
+          for (int d = 0; d < 3; ++d) {
+            cnt *= (b >> d & 1) ? part[d] : full[d];
+            sz *= (b >> d & 1) ? psz[d] : fsz[d];
+          }
+          if (cnt == 0) continue;
+          int at = nc++;
+          while (at > 0 && size[at - 1] < sz) {  // stable insertion, larger first
+            size[at] = size[at - 1];
+            count[at] = count[at - 1];
+            bits[at] = bits[at - 1];
+            --at;
+          }
+          size[at] = sz;
+          count[at] = cnt;
+          bits[at] = b;
+        }
+        g.nclass = nc;
+        int64_t run = 0;
+        for (int i = 0; i < nc; ++i) {
+          g.cls_start[i] = run;
+          g.cls_bits[i] = bits[i];
+          run += count[i];
+        }
+        if (run != g.S) return RANS_ERR_ARG;
+      }
       break;
     }
     default:

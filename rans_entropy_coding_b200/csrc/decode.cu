@@ -4,9 +4,9 @@
 //    entry is <= cum = x mod 2^16 (the rule of CompressAI's linear scan,
 //    "Benchmark notes" section 4).  It is found through a per-row table of
 //    2^q slots keyed by the top q bits of cum ("torch_ans 0.3.0", Usage,
-//    inverse-CDF decoding): a slot either names the bucket, or holds one
-//    boundary to compare against, or bounds a short run of boundaries that
-//    the warp counts together (one ballot per 32 candidates);
+//    inverse-CDF decoding): a slot resolves up to two bucket boundaries with
+//    two compares; a slot with more is counted by the whole warp, one ballot
+//    per 32 candidates;
 //  * state update x = freq (x >> 16) + cum - start and a refill of one
 //    32-bit word when x < 2^31 (64-bit state / 32-bit words / 16-bit
 //    precision: "torch_ans 0.3.0", Usage, rans64 row);
@@ -20,6 +20,8 @@
 //    depends on what it reads ("torch_ans 0.3.0", Performance Tuning, GPU
 //    item 5: the bypass phase is sequential across the lanes and skipped by a
 //    group ballot).
+//  Latency: row indexes are loaded kRing groups ahead into registers; each
+//  stream's words are bulk prefetched into L2 when the warp starts it.
 //  Tables are staged into shared memory with bulk copies when they fit.
 #include "rans_common.cuh"
 #include "rans_internal.h"
@@ -29,6 +31,7 @@ namespace {
 
 constexpr int kDecMaxThreads32 = 768;
 constexpr int kDecThreads1 = 128;
+constexpr int kRing = 4;
 
 struct DecCtx {
   const uint8_t *in;
@@ -53,9 +56,99 @@ __device__ __forceinline__ bool stream_bounds(const DecCtx &c, int64_t s, int W,
   return true;
 }
 
-template <typename SymT>
-__device__ void decode_stream_w32(const DecCtx &c, const RowMeta *meta, const uint32_t *buckets,
-                                  const uint32_t *slots, int64_t s) {
+// Fast slot decode: bucket lo + (c > e1) + (c > e2); multi = three or more
+// boundaries inside the slot.
+__device__ __forceinline__ uint32_t slot_symbol(uint32_t se, uint32_t c, bool &multi) {
+  const uint32_t e1 = (se >> 16) & 0xffu, e2 = se >> 24;
+  multi = e1 > e2;
+  return (se & 0xffffu) + (c > e1 ? 1u : 0u) + (c > e2 ? 1u : 0u);
+}
+
+struct EscapeResult {
+  uint64_t x;
+  int64_t val;
+  uint64_t cur;
+  bool bad;
+};
+
+// The lane-serial part of a group holding an escape (after every lane's
+// symbol op): lanes take their words in ascending lane order; an escaping lane
+// reads its refill, count pieces and bypass pieces from the shared stream.
+__device__ __noinline__ EscapeResult escape_group(uint64_t x, bool active, bool esc,
+                                                  uint32_t maxv, uint64_t abs0,
+                                                  const uint32_t *words, uint64_t nw) {
+  const int lane = threadIdx.x & 31;
+  bool bad = false;
+  int64_t val = 0;
+  const bool need_sym = active && x < kL;
+  uint32_t cons = need_sym ? 1u : 0u;
+  uint32_t rem = __ballot_sync(kFull, esc);
+  while (rem) {
+    const int el = __ffs(rem) - 1;
+    rem &= rem - 1;
+    uint32_t inc = cons;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const uint32_t t = __shfl_up_sync(kFull, inc, o);
+      if (lane >= o) inc += t;
+    }
+    const uint32_t pre = __shfl_sync(kFull, inc - cons, el);
+    if (lane == el) {
+      uint64_t pp = abs0 + pre;
+      auto rd = [&]() -> uint32_t {
+        uint32_t v = 0;
+        if (pp < nw) v = __ldg(words + pp); else bad = true;
+        ++pp;
+        return v;
+      };
+      if (x < kL) x = (x << 32) | rd();
+      auto getbits = [&]() -> uint32_t {
+        const uint32_t v = (uint32_t)x & kBypassMax;
+        x >>= kBypassBits;
+        if (x < kL) x = (x << 32) | rd();
+        return v;
+      };
+      uint32_t v4 = getbits();
+      uint32_t nb = v4;
+      while (v4 == kBypassMax && nb <= 15) {
+        v4 = getbits();
+        nb += v4;
+      }
+      if (nb > 15) {
+        bad = true;
+        nb = 0;
+      }
+      uint64_t raw = 0;
+      for (uint32_t k = 0; k < nb; ++k) raw |= (uint64_t)getbits() << (kBypassBits * k);
+      const int64_t half = (int64_t)(raw >> 1);
+      val = (raw & 1) ? (-half - 1) : ((int64_t)maxv + half);
+      cons = (uint32_t)(pp - (abs0 + pre));
+    }
+  }
+  uint32_t inc = cons;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const uint32_t t = __shfl_up_sync(kFull, inc, o);
+    if (lane >= o) inc += t;
+  }
+  if (need_sym && !esc) {
+    const uint64_t pp = abs0 + (inc - cons);
+    uint32_t v = 0;
+    if (pp < nw) v = __ldg(words + pp); else bad = true;
+    x = (x << 32) | v;
+  }
+  EscapeResult r;
+  r.x = x;
+  r.val = val;
+  r.cur = abs0 + __shfl_sync(kFull, inc, 31);
+  r.bad = bad;
+  return r;
+}
+
+template <typename SymT, bool IB0>
+__device__ __forceinline__ void decode_stream_w32(const DecCtx &c, const RowMeta *meta,
+                                                  const uint32_t *buckets,
+                                                  const uint32_t *slots, int64_t s) {
   const int lane = threadIdx.x & 31;
   const StreamDesc d = stream_desc(c.g, s);
   const uint32_t *words = nullptr;
@@ -64,146 +157,108 @@ __device__ void decode_stream_w32(const DecCtx &c, const RowMeta *meta, const ui
     if (lane == 0) report(c.status, d.ok ? RANS_ERR_CORRUPT : RANS_ERR_ARG, s);
     return;
   }
+  if (lane == 0)
+    bulk_prefetch_l2(reinterpret_cast<const char *>(c.in),
+                     reinterpret_cast<const char *>(c.in) + c.in_bytes,
+                     reinterpret_cast<const char *>(words + 64), 4 * (nw - 64));
+  const int32_t n = (int32_t)d.n;
+  const int32_t G = (n + 31) >> 5;
+  const int64_t base = d.base;
   const int ib = c.g.ib_shift;
+  const int32_t *idx_s = c.idx + (IB0 ? base : 0);
+  SymT *out_s = reinterpret_cast<SymT *>(c.out) + base;
+  const uint32_t K = (uint32_t)c.K;
+  auto load_idx = [&](int32_t rel) -> int32_t {
+    return IB0 ? __ldg(idx_s + rel) : __ldg(c.idx + ((base + rel) >> ib));
+  };
+
   uint64_t x = (uint64_t)__ldg(words + 2 * lane) | ((uint64_t)__ldg(words + 2 * lane + 1) << 32);
   uint64_t cur = 64;  // absolute word index of the window start
   uint32_t off = 0;   // words of the window already consumed
   uint32_t w0 = cur + lane < nw ? __ldg(words + cur + lane) : 0u;
   uint32_t w1 = cur + 32 + lane < nw ? __ldg(words + cur + 32 + lane) : 0u;
-  bool bad = false;
+  bool bad = false, bad_idx = false;
 
-  const int64_t n = d.n;
-  const int64_t G = (n + 31) >> 5;
-  Walker wk;
-  wk.init(d, lane);
-  int32_t nr = 0;
-  int64_t np = 0;
-  if (lane < n) {
-    np = wk.pos();
-    nr = __ldg(c.idx + (np >> ib));
+  Stepper pl;
+  pl.init(d.t, lane);
+  int32_t rrel[kRing], ridx[kRing];
+#pragma unroll
+  for (int u = 0; u < kRing; ++u) {
+    rrel[u] = pl.rel;
+    ridx[u] = lane < n - u * 32 ? load_idx(pl.rel) : 0;
+    pl.fwd(32);
   }
-  for (int64_t g = 0; g < G; ++g) {
-    const bool active = g * 32 + lane < n;
-    const int32_t r = nr;
-    const int64_t p = np;
-    if (g + 1 < G) {
-      wk.fwd(32);
-      if ((g + 1) * 32 + lane < n) {
-        np = wk.pos();
-        nr = __ldg(c.idx + (np >> ib));
+
+  for (int32_t g0 = 0; g0 < G; g0 += kRing) {
+#pragma unroll
+    for (int u = 0; u < kRing; ++u) {
+      const int32_t g = g0 + u;
+      if (g >= G) break;
+      const bool active = lane < n - g * 32;
+      const int32_t rel = rrel[u];
+      uint32_t r = (uint32_t)ridx[u];
+      if (g + kRing < G) {
+        rrel[u] = pl.rel;
+        ridx[u] = lane < n - (g + kRing) * 32 ? load_idx(pl.rel) : 0;
+        pl.fwd(32);
       }
-    }
-    if (__any_sync(kFull, active && (uint32_t)r >= (uint32_t)c.K)) {
-      if (lane == 0) report(c.status, RANS_ERR_INDEX, s);
-      return;
-    }
-    const RowMeta m = meta[active ? r : 0];
-    const uint32_t cum = (uint32_t)x & (kTotal - 1);
-    const uint32_t sh = slot_shift(m.slot);
-    const uint32_t se = slots[slot_base(m.slot) + (cum >> sh)];
-    const uint32_t lo = se & 0xffffu;
-    const uint32_t code = se >> 16;
-    uint32_t sym = lo + ((cum & ((1u << sh) - 1u)) >= code ? 1u : 0u);
-    uint32_t mm = __ballot_sync(kFull, active && (code & 0x8000u));
-    while (mm) {
-      const int l = __ffs(mm) - 1;
-      mm &= mm - 1;
-      const uint32_t base_l = __shfl_sync(kFull, m.bucket_base + lo, l);
-      const uint32_t cnt_l = __shfl_sync(kFull, code & 0x7fffu, l);
-      const uint32_t cum_l = __shfl_sync(kFull, cum, l);
-      uint32_t cnt = 0;
-      for (uint32_t k0 = 0; k0 < cnt_l; k0 += 32) {
-        const uint32_t k = k0 + lane + 1;
-        const bool le = k <= cnt_l && bucket_start(buckets[base_l + k]) <= cum_l;
-        cnt += __popc(__ballot_sync(kFull, le));
+      bad_idx |= r >= K;
+      r = r < K ? r : 0u;
+      const RowMeta m = meta[r];
+      const uint32_t cum = (uint32_t)x & (kTotal - 1);
+      const uint32_t sh = slot_shift(m.slot);
+      const uint32_t se = slots[slot_base(m.slot) + (cum >> sh)];
+      bool multi;
+      uint32_t sym = slot_symbol(se, cum & ((1u << sh) - 1u), multi);
+      uint32_t mm = __ballot_sync(kFull, active && multi);
+      while (mm) {
+        const int l = __ffs(mm) - 1;
+        mm &= mm - 1;
+        const uint32_t base_l = __shfl_sync(kFull, m.bucket_base + (se & 0xffffu), l);
+        const uint32_t cnt_l = __shfl_sync(kFull, (se >> 24) + 3u, l);
+        const uint32_t cum_l = __shfl_sync(kFull, cum, l);
+        uint32_t cnt = 0;
+        for (uint32_t k0 = 0; k0 < cnt_l; k0 += 32) {
+          const uint32_t k = k0 + lane + 1;
+          const bool le = k <= cnt_l && bucket_start(buckets[base_l + k]) <= cum_l;
+          cnt += __popc(__ballot_sync(kFull, le));
+        }
+        if (lane == l) sym = (se & 0xffffu) + cnt;
       }
-      if (lane == l) sym = lo + cnt;
-    }
-    const uint32_t e = buckets[m.bucket_base + sym];
-    if (active) x = (uint64_t)bucket_freq(e) * (x >> kPrec) + cum - bucket_start(e);
-    const bool esc = active && sym == m.maxv;
-    int64_t val = (int64_t)sym;
-    if (!__any_sync(kFull, esc)) {
-      const bool need = active && x < kL;
-      const uint32_t nm = __ballot_sync(kFull, need);
-      const uint32_t j = off + __popc(nm & lanemask_lt());
-      const uint32_t a = __shfl_sync(kFull, w0, j & 31);
-      const uint32_t b = __shfl_sync(kFull, w1, j & 31);
-      if (need) x = (x << 32) | (j < 32 ? a : b);
-      off += __popc(nm);
-      if (off >= 32) {
-        w0 = w1;
-        cur += 32;
-        off -= 32;
+      const uint32_t e = buckets[m.bucket_base + sym];
+      if (active) x = (uint64_t)bucket_freq(e) * (x >> kPrec) + (cum - bucket_start(e));
+      const bool esc = active && sym == m.maxv;
+      int32_t val = (int32_t)sym + m.offset;
+      if (!__any_sync(kFull, esc)) {
+        const bool need = active && x < kL;
+        const uint32_t nm = __ballot_sync(kFull, need);
+        const uint32_t j = off + __popc(nm & lanemask_lt());
+        const uint32_t a = __shfl_sync(kFull, w0, j & 31);
+        const uint32_t b = __shfl_sync(kFull, w1, j & 31);
+        if (need) x = (x << 32) | (j < 32 ? a : b);
+        off += __popc(nm);
+        if (off >= 32) {
+          w0 = w1;
+          cur += 32;
+          off -= 32;
+          w1 = cur + 32 + lane < nw ? __ldg(words + cur + 32 + lane) : 0u;
+        }
+      } else {
+        const EscapeResult er = escape_group(x, active, esc, m.maxv, cur + off, words, nw);
+        x = er.x;
+        if (esc) val = (int32_t)(er.val + (int64_t)m.offset);
+        bad |= er.bad;
+        cur = er.cur;
+        off = 0;
+        w0 = cur + lane < nw ? __ldg(words + cur + lane) : 0u;
         w1 = cur + 32 + lane < nw ? __ldg(words + cur + 32 + lane) : 0u;
       }
-    } else {
-      // Lanes consume words in ascending lane order; an escaping lane's
-      // count is known only after it has read its pieces.
-      const uint64_t abs0 = cur + off;
-      const bool need_sym = active && x < kL;
-      uint32_t cons = need_sym ? 1u : 0u;
-      uint32_t rem = __ballot_sync(kFull, esc);
-      while (rem) {
-        const int el = __ffs(rem) - 1;
-        rem &= rem - 1;
-        uint32_t inc = cons;
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-          const uint32_t t = __shfl_up_sync(kFull, inc, o);
-          if (lane >= o) inc += t;
-        }
-        const uint32_t pre = __shfl_sync(kFull, inc - cons, el);
-        if (lane == el) {
-          uint64_t pp = abs0 + pre;
-          auto rd = [&]() -> uint32_t {
-            uint32_t v = 0;
-            if (pp < nw) v = __ldg(words + pp); else bad = true;
-            ++pp;
-            return v;
-          };
-          if (x < kL) x = (x << 32) | rd();
-          auto getbits = [&]() -> uint32_t {
-            const uint32_t v = (uint32_t)x & kBypassMax;
-            x >>= kBypassBits;
-            if (x < kL) x = (x << 32) | rd();
-            return v;
-          };
-          uint32_t v4 = getbits();
-          uint32_t nb = v4;
-          while (v4 == kBypassMax && nb <= 15) {
-            v4 = getbits();
-            nb += v4;
-          }
-          if (nb > 15) {
-            bad = true;
-            nb = 0;
-          }
-          uint64_t raw = 0;
-          for (uint32_t k = 0; k < nb; ++k) raw |= (uint64_t)getbits() << (kBypassBits * k);
-          const int64_t half = (int64_t)(raw >> 1);
-          val = (raw & 1) ? (-half - 1) : ((int64_t)m.maxv + half);
-          cons = (uint32_t)(pp - (abs0 + pre));
-        }
-      }
-      uint32_t inc = cons;
-#pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        const uint32_t t = __shfl_up_sync(kFull, inc, o);
-        if (lane >= o) inc += t;
-      }
-      if (need_sym && !esc) {
-        const uint64_t pp = abs0 + (inc - cons);
-        uint32_t v = 0;
-        if (pp < nw) v = __ldg(words + pp); else bad = true;
-        x = (x << 32) | v;
-      }
-      cur = abs0 + __shfl_sync(kFull, inc, 31);
-      off = 0;
-      w0 = cur + lane < nw ? __ldg(words + cur + lane) : 0u;
-      w1 = cur + 32 + lane < nw ? __ldg(words + cur + 32 + lane) : 0u;
+      if (active) out_s[rel] = (SymT)val;
     }
-    if (active) SymIO<SymT>::store(c.out, p, val + (int64_t)m.offset);
+  }
+  if (__any_sync(kFull, bad_idx)) {
+    if (lane == 0) report(c.status, RANS_ERR_INDEX, s);
+    return;
   }
   const bool ok = !bad && x == kL && cur + off == nw;
   if (!__all_sync(kFull, ok) && lane == 0) report(c.status, RANS_ERR_CORRUPT, s);
@@ -219,21 +274,36 @@ __device__ void decode_stream_w1(const DecCtx &c, const RowMeta *meta, const uin
     report(c.status, d.ok ? RANS_ERR_CORRUPT : RANS_ERR_ARG, s);
     return;
   }
+  bulk_prefetch_l2(reinterpret_cast<const char *>(c.in),
+                   reinterpret_cast<const char *>(c.in) + c.in_bytes,
+                   reinterpret_cast<const char *>(words), 4 * nw);
   const int ib = c.g.ib_shift;
+  const Tile t = d.t;
   uint64_t x = (uint64_t)__ldg(words) | ((uint64_t)__ldg(words + 1) << 32);
-  uint64_t pp = 2;
+  uint64_t pw = 2;
   bool bad = false;
   auto rd = [&]() -> uint32_t {
     uint32_t v = 0;
-    if (pp < nw) v = __ldg(words + pp); else bad = true;
-    ++pp;
+    if (pw < nw) v = __ldg(words + pw); else bad = true;
+    ++pw;
     return v;
   };
-  Walker wk;
-  wk.init(d, 0);
-  for (int64_t i = 0; i < d.n; ++i) {
-    const int64_t p = wk.pos();
-    wk.fwd(1);
+  RelPos pl, pp;
+  pl.init(t, 0);
+  pp = pl;
+  const int32_t n = (int32_t)d.n;
+  constexpr int32_t kAhead = 64;
+  for (int32_t u = 0; u < kAhead && u < n; ++u) {
+    prefetch_l2(c.idx + ((d.base + pp.rel(t)) >> ib));
+    pp.fwd(t, 1);
+  }
+  for (int32_t i = 0; i < n; ++i) {
+    const int64_t p = d.base + pl.rel(t);
+    pl.fwd(t, 1);
+    if (i + kAhead < n) {
+      prefetch_l2(c.idx + ((d.base + pp.rel(t)) >> ib));
+      pp.fwd(t, 1);
+    }
     const int32_t r = __ldg(c.idx + (p >> ib));
     if ((uint32_t)r >= (uint32_t)c.K) {
       report(c.status, RANS_ERR_INDEX, s);
@@ -243,18 +313,16 @@ __device__ void decode_stream_w1(const DecCtx &c, const RowMeta *meta, const uin
     const uint32_t cum = (uint32_t)x & (kTotal - 1);
     const uint32_t sh = slot_shift(m.slot);
     const uint32_t se = slots[slot_base(m.slot) + (cum >> sh)];
-    uint32_t sym = se & 0xffffu;
-    const uint32_t code = se >> 16;
-    if (code & 0x8000u) {
-      // last bucket in [sym, sym + count] whose start is <= cum
-      uint32_t lo = sym, hi = sym + (code & 0x7fffu);
+    bool multi;
+    uint32_t sym = slot_symbol(se, cum & ((1u << sh) - 1u), multi);
+    if (multi) {
+      // last bucket in [lo, lo + count] whose start is <= cum
+      uint32_t lo = se & 0xffffu, hi = lo + (se >> 24) + 3u;
       while (lo < hi) {
         const uint32_t mid = (lo + hi + 1) >> 1;
         if (bucket_start(buckets[m.bucket_base + mid]) <= cum) lo = mid; else hi = mid - 1;
       }
       sym = lo;
-    } else {
-      sym += (cum & ((1u << sh) - 1u)) >= code ? 1u : 0u;
     }
     const uint32_t e = buckets[m.bucket_base + sym];
     x = (uint64_t)bucket_freq(e) * (x >> kPrec) + cum - bucket_start(e);
@@ -284,10 +352,10 @@ __device__ void decode_stream_w1(const DecCtx &c, const RowMeta *meta, const uin
     }
     SymIO<SymT>::store(c.out, p, val + (int64_t)m.offset);
   }
-  if (bad || x != kL || pp != nw) report(c.status, RANS_ERR_CORRUPT, s);
+  if (bad || x != kL || pw != nw) report(c.status, RANS_ERR_CORRUPT, s);
 }
 
-template <int W, typename SymT, bool SMEM>
+template <int W, typename SymT, bool SMEM, bool IB0>
 __global__ void __launch_bounds__(W == 32 ? kDecMaxThreads32 : kDecThreads1)
     decode_kernel(DecCtx c) {
   extern __shared__ __align__(16) unsigned char smem[];
@@ -306,19 +374,19 @@ __global__ void __launch_bounds__(W == 32 ? kDecMaxThreads32 : kDecThreads1)
   const uint32_t *slots = reinterpret_cast<const uint32_t *>(tb + c.meta_bytes + c.bucket_bytes);
   if (W == 32) {
     const int warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
-    for (int64_t s = blockIdx.x + (int64_t)gridDim.x * warp; s < c.g.S;
-         s += (int64_t)gridDim.x * nw)
-      decode_stream_w32<SymT>(c, meta, buckets, slots, s);
+    for (int64_t k = blockIdx.x + (int64_t)gridDim.x * warp; k < c.g.S;
+         k += (int64_t)gridDim.x * nw)
+      decode_stream_w32<SymT, IB0>(c, meta, buckets, slots, stream_of(c.g, k));
   } else {
-    for (int64_t s = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; s < c.g.S;
-         s += (int64_t)gridDim.x * blockDim.x)
-      decode_stream_w1<SymT>(c, meta, buckets, slots, s);
+    for (int64_t k = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; k < c.g.S;
+         k += (int64_t)gridDim.x * blockDim.x)
+      decode_stream_w1<SymT>(c, meta, buckets, slots, stream_of(c.g, k));
   }
 }
 
-template <int W, typename SymT, bool SMEM>
+template <int W, typename SymT, bool SMEM, bool IB0>
 int launch_decode_t(const DecCtx &c, cudaStream_t st) {
-  auto kern = decode_kernel<W, SymT, SMEM>;
+  auto kern = decode_kernel<W, SymT, SMEM, IB0>;
   const uint32_t smem = SMEM ? c.meta_bytes + c.bucket_bytes + c.slot_bytes : 0;
   int dev = 0;
   cudaGetDevice(&dev);
@@ -365,7 +433,12 @@ int launch_decode_t(const DecCtx &c, cudaStream_t st) {
 
 template <int W, typename SymT>
 int launch_decode_w(const DecCtx &c, bool smem, cudaStream_t st) {
-  return smem ? launch_decode_t<W, SymT, true>(c, st) : launch_decode_t<W, SymT, false>(c, st);
+  const bool ib0 = c.g.ib_shift == 0;
+  if (smem)
+    return ib0 ? launch_decode_t<W, SymT, true, true>(c, st)
+               : launch_decode_t<W, SymT, true, false>(c, st);
+  return ib0 ? launch_decode_t<W, SymT, false, true>(c, st)
+             : launch_decode_t<W, SymT, false, false>(c, st);
 }
 
 template <typename SymT>

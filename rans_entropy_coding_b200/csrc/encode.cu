@@ -96,9 +96,35 @@ __device__ __forceinline__ uint32_t symbol_ops(uint64_t &x, uint32_t start, uint
   return k;
 }
 
-template <typename SymT>
-__device__ void encode_stream_w32(const EncCtx &c, const RowMeta *meta, const uint32_t *buckets,
-                                  int64_t s) {
+constexpr int kRing = 4;
+
+// A group holding an escape, off the fast path: every lane counts the words
+// its ops push, a suffix sum over lanes places each lane's block (lanes > l
+// push first in the serial order), then each lane writes its words.
+__device__ __noinline__ uint64_t escape_group_enc(uint64_t x, bool active, uint32_t start,
+                                                  uint32_t freq, double rcp, uint64_t raw,
+                                                  bool esc, uint32_t *end, uint32_t cursor,
+                                                  uint32_t *total) {
+  const int lane = threadIdx.x & 31;
+  uint32_t k = 0;
+  if (active) {
+    uint64_t y = x;
+    k = symbol_ops<false>(y, start, freq, rcp, raw, esc, end, 0);
+  }
+  uint32_t inc = k;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const uint32_t t = __shfl_down_sync(kFull, inc, o);
+    if (lane + o < 32) inc += t;
+  }
+  *total = __shfl_sync(kFull, inc, 0);
+  if (active) symbol_ops<true>(x, start, freq, rcp, raw, esc, end, cursor + inc - k);
+  return x;
+}
+
+template <typename SymT, bool IB0>
+__device__ __forceinline__ void encode_stream_w32(const EncCtx &c, const RowMeta *meta,
+                                                  const uint32_t *buckets, int64_t s) {
   const int lane = threadIdx.x & 31;
   const StreamDesc d = stream_desc(c.g, s);
   if (!d.ok) {
@@ -106,72 +132,83 @@ __device__ void encode_stream_w32(const EncCtx &c, const RowMeta *meta, const ui
     return;
   }
   uint32_t *end = reinterpret_cast<uint32_t *>(c.scratch + slot_end(c.g, d, s));
-  const int64_t n = d.n;
-  const int64_t G = (n + 31) >> 5;
+  const int32_t n = (int32_t)d.n;
+  const int32_t G = (n + 31) >> 5;
+  const int64_t base = d.base;
   const int ib = c.g.ib_shift;
+  const int32_t *idx_s = c.idx + (IB0 ? base : 0);
+  const SymT *sym_s = reinterpret_cast<const SymT *>(c.sym) + base;
+  const uint32_t K = (uint32_t)c.K;
+  auto load = [&](int32_t rel, int32_t &sv, int32_t &r) {
+    sv = SymIO<SymT>::load(sym_s, rel);
+    r = IB0 ? __ldg(idx_s + rel) : __ldg(c.idx + ((base + rel) >> ib));
+  };
   uint64_t x = kL;
   uint32_t cursor = 0;
+  bool bad_idx = false;
+  const uint32_t above = 0xfffffffeu << lane;   // lanes > this lane
 
-  Walker wk;
-  int32_t nsv = 0, nr = 0;
-  if (G > 0) {
-    wk.init(d, (G - 1) * 32 + lane);
-    if ((G - 1) * 32 + lane < n) {
-      const int64_t p = wk.pos();
-      nsv = SymIO<SymT>::load(c.sym, p);
-      nr = __ldg(c.idx + (p >> ib));
+  // groups are coded G-1 down to 0; ring slot u holds group G-1-(k+u)
+  Stepper pl;
+  pl.init(d.t, (G > 0 ? G - 1 : 0) * 32 + lane);
+  int32_t rsym[kRing], ridx[kRing];
+#pragma unroll
+  for (int u = 0; u < kRing; ++u) {
+    rsym[u] = 0;
+    ridx[u] = 0;
+    if (u < G && lane < n - (G - 1 - u) * 32) load(pl.rel, rsym[u], ridx[u]);
+    if (u + 1 < G) pl.back(32);
+  }
+
+  for (int32_t k0 = 0; k0 < G; k0 += kRing) {
+#pragma unroll
+    for (int u = 0; u < kRing; ++u) {
+      const int32_t k = k0 + u;
+      if (k >= G) break;
+      const int32_t g = G - 1 - k;
+      const bool active = lane < n - g * 32;
+      const int32_t sv = rsym[u];
+      uint32_t r = (uint32_t)ridx[u];
+      if (g - kRing >= 0) {     // every lane of an earlier group is active
+        load(pl.rel, rsym[u], ridx[u]);
+        if (g - kRing > 0) pl.back(32);
+      }
+      bad_idx |= r >= K;
+      r = r < K ? r : 0u;
+      const RowMeta m = meta[r];
+      // value mapping: in range iff 0 <= s - offset < maxv (64-bit, exact)
+      const int64_t v = (int64_t)sv - (int64_t)m.offset;
+      const bool in_range = (uint64_t)v < (uint64_t)m.maxv;
+      const uint32_t e = buckets[m.bucket_base + (in_range ? (uint32_t)v : m.maxv)];
+      const uint32_t start = bucket_start(e), freq = bucket_freq(e);
+      const bool esc = active && !in_range;
+      const double rcp = freq_reciprocal(freq);
+      if (!__any_sync(kFull, esc)) {
+        // x >= freq * 2^47  <=>  high word of x >= freq * 2^15
+        const bool need = active && (uint32_t)(x >> 32) >= (freq << 15);
+        const uint32_t bm = __ballot_sync(kFull, need);
+        if (need) {
+          end[-1 - (int64_t)(cursor + __popc(bm & above))] = (uint32_t)x;
+          x >>= 32;
+        }
+        cursor += __popc(bm);
+        if (active) x = enc_sym_step(x, start, freq, rcp);
+      } else {
+        uint64_t raw = 0;
+        if (esc) raw = v < 0 ? (uint64_t)(-2 * v - 1) : (uint64_t)(2 * (v - (int64_t)m.maxv));
+        if (__any_sync(kFull, esc && (raw >> 60) != 0)) {
+          if (lane == 0) report(c.status, RANS_ERR_RANGE, s);
+          return;
+        }
+        uint32_t total;
+        x = escape_group_enc(x, active, start, freq, rcp, raw, esc, end, cursor, &total);
+        cursor += total;
+      }
     }
   }
-  for (int64_t g = G - 1; g >= 0; --g) {
-    const bool active = g * 32 + lane < n;
-    const int32_t sv = nsv, r = nr;
-    if (g > 0) {
-      wk.back(32);
-      const int64_t p = wk.pos();
-      nsv = SymIO<SymT>::load(c.sym, p);
-      nr = __ldg(c.idx + (p >> ib));
-    }
-    if (__any_sync(kFull, active && (uint32_t)r >= (uint32_t)c.K)) {
-      if (lane == 0) report(c.status, RANS_ERR_INDEX, s);
-      return;
-    }
-    const RowMeta m = meta[active ? r : 0];
-    uint32_t start, freq;
-    uint64_t raw;
-    bool esc;
-    map_symbol(sv, m, buckets, start, freq, raw, esc);
-    esc = esc && active;
-    const double rcp = freq_reciprocal(freq);
-    if (!__any_sync(kFull, esc)) {
-      const bool need = active && x >= ((uint64_t)freq << 47);
-      const uint32_t bm = __ballot_sync(kFull, need);
-      if (need) {
-        const uint32_t k = cursor + __popc(bm & (0xfffffffeu << lane));
-        end[-1 - (int64_t)k] = (uint32_t)x;
-        x >>= 32;
-      }
-      cursor += __popc(bm);
-      if (active) x = enc_sym_step(x, start, freq, rcp);
-    } else {
-      if (__any_sync(kFull, esc && (raw >> 60) != 0)) {
-        if (lane == 0) report(c.status, RANS_ERR_RANGE, s);
-        return;
-      }
-      uint32_t k = 0;
-      if (active) {
-        uint64_t y = x;
-        k = symbol_ops<false>(y, start, freq, rcp, raw, esc, end, 0);
-      }
-      uint32_t inc = k;
-#pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        const uint32_t t = __shfl_down_sync(kFull, inc, o);
-        if (lane + o < 32) inc += t;
-      }
-      const uint32_t total = __shfl_sync(kFull, inc, 0);
-      if (active) symbol_ops<true>(x, start, freq, rcp, raw, esc, end, cursor + inc - k);
-      cursor += total;
-    }
+  if (__any_sync(kFull, bad_idx)) {
+    if (lane == 0) report(c.status, RANS_ERR_INDEX, s);
+    return;
   }
   // flush: lanes 31..0 push high then low, so lane 0's low word comes first
   const uint32_t kk = cursor + 2u * (31u - (uint32_t)lane);
@@ -191,13 +228,29 @@ __device__ void encode_stream_w1(const EncCtx &c, const RowMeta *meta, const uin
   }
   uint32_t *end = reinterpret_cast<uint32_t *>(c.scratch + slot_end(c.g, d, s));
   const int ib = c.g.ib_shift;
+  const Tile t = d.t;
+  const int32_t n = (int32_t)d.n;
   uint64_t x = kL;
   uint32_t cursor = 0;
-  Walker wk;
-  if (d.n > 0) wk.init(d, d.n - 1);
-  for (int64_t i = d.n - 1; i >= 0; --i) {
-    const int64_t p = wk.pos();
-    wk.back(1);
+  RelPos pl, pp;
+  pl.init(t, n > 0 ? n - 1 : 0);
+  pp = pl;
+  constexpr int32_t kAhead = 64;
+  for (int32_t u = 0; u < kAhead && u < n; ++u) {
+    const int64_t p = d.base + pp.rel(t);
+    prefetch_l2(reinterpret_cast<const SymT *>(c.sym) + p);
+    prefetch_l2(c.idx + (p >> ib));
+    pp.back(t, 1);
+  }
+  for (int32_t i = n - 1; i >= 0; --i) {
+    const int64_t p = d.base + pl.rel(t);
+    pl.back(t, 1);
+    if (i - kAhead >= 0) {
+      const int64_t q = d.base + pp.rel(t);
+      prefetch_l2(reinterpret_cast<const SymT *>(c.sym) + q);
+      prefetch_l2(c.idx + (q >> ib));
+      pp.back(t, 1);
+    }
     const int32_t sv = SymIO<SymT>::load(c.sym, p);
     const int32_t r = __ldg(c.idx + (p >> ib));
     if ((uint32_t)r >= (uint32_t)c.K) {
@@ -220,7 +273,7 @@ __device__ void encode_stream_w1(const EncCtx &c, const RowMeta *meta, const uin
   c.lens[s] = 4ull * cursor;
 }
 
-template <int W, typename SymT, bool SMEM>
+template <int W, typename SymT, bool SMEM, bool IB0>
 __global__ void __launch_bounds__(W == 32 ? kEncThreads32 : kEncThreads1)
     encode_kernel(EncCtx c) {
   extern __shared__ __align__(16) unsigned char smem[];
@@ -239,13 +292,13 @@ __global__ void __launch_bounds__(W == 32 ? kEncThreads32 : kEncThreads1)
   }
   if (W == 32) {
     const int warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
-    for (int64_t s = blockIdx.x + (int64_t)gridDim.x * warp; s < c.g.S;
-         s += (int64_t)gridDim.x * nw)
-      encode_stream_w32<SymT>(c, meta, buckets, s);
+    for (int64_t k = blockIdx.x + (int64_t)gridDim.x * warp; k < c.g.S;
+         k += (int64_t)gridDim.x * nw)
+      encode_stream_w32<SymT, IB0>(c, meta, buckets, stream_of(c.g, k));
   } else {
-    for (int64_t s = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; s < c.g.S;
-         s += (int64_t)gridDim.x * blockDim.x)
-      encode_stream_w1<SymT>(c, meta, buckets, s);
+    for (int64_t k = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; k < c.g.S;
+         k += (int64_t)gridDim.x * blockDim.x)
+      encode_stream_w1<SymT>(c, meta, buckets, stream_of(c.g, k));
   }
 }
 
@@ -327,10 +380,10 @@ __global__ void debug_divide_kernel(const uint64_t *x, const uint32_t *f, int64_
   }
 }
 
-template <int W, typename SymT, bool SMEM>
+template <int W, typename SymT, bool SMEM, bool IB0>
 int launch_encode_t(const EncCtx &c, cudaStream_t st) {
   const int dev_threads = W == 32 ? kEncThreads32 : kEncThreads1;
-  auto kern = encode_kernel<W, SymT, SMEM>;
+  auto kern = encode_kernel<W, SymT, SMEM, IB0>;
   const uint32_t smem = SMEM ? c.meta_bytes + c.bucket_bytes : 0;
   int dev = 0;
   cudaGetDevice(&dev);
@@ -353,7 +406,12 @@ int launch_encode_t(const EncCtx &c, cudaStream_t st) {
 
 template <int W, typename SymT>
 int launch_encode_w(const EncCtx &c, bool smem, cudaStream_t st) {
-  return smem ? launch_encode_t<W, SymT, true>(c, st) : launch_encode_t<W, SymT, false>(c, st);
+  const bool ib0 = c.g.ib_shift == 0;
+  if (smem)
+    return ib0 ? launch_encode_t<W, SymT, true, true>(c, st)
+               : launch_encode_t<W, SymT, true, false>(c, st);
+  return ib0 ? launch_encode_t<W, SymT, false, true>(c, st)
+             : launch_encode_t<W, SymT, false, false>(c, st);
 }
 
 template <typename SymT>

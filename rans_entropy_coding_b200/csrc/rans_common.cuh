@@ -23,12 +23,16 @@ constexpr unsigned kFull = 0xffffffffu;
 
 // ------------------------------------------------------------ table blob --
 // [header 256 B][RowMeta K][bucket words][slot words], sections 16-B padded.
-// A bucket word packs start | (width - 1) << 16.  A slot word packs
-// lo | code << 16 where lo is the row-local bucket holding the slot's first
-// cumulative value and code says what lies inside the slot:
-//   code < 0x8000: one bucket boundary at offset `code` from the slot start
-//                  (code == slot width: no boundary inside);
-//   code & 0x8000: (code & 0x7fff) boundaries inside (a few, searched).
+// A bucket word packs start | (width - 1) << 16.
+// Each row has 2^q slots (8 <= q <= 14) of width w = 2^(16-q) <= 256 over the
+// cumulative range; a slot word packs lo | e1 << 16 | e2 << 24 where lo is the
+// row-local bucket holding the slot's first cumulative value and e1, e2
+// describe the bucket boundaries strictly inside the slot, as offsets from the
+// slot start minus one (255 = none):
+//   e1 <= e2: at most two boundaries; for c = cum mod w the bucket is
+//             lo + (c > e1) + (c > e2);
+//   e1 > e2:  three or more: e1 = 255 and e2 + 3 boundaries, counted by the
+//             warp (rare).
 struct RowMeta {
   uint32_t bucket_base;  // index of the row's bucket 0 in the bucket words
   uint32_t maxv;         // escape bucket = cdf_length - 2
@@ -38,7 +42,7 @@ struct RowMeta {
 static_assert(sizeof(RowMeta) == 16, "RowMeta is one 16-byte load");
 
 constexpr uint32_t kHeaderBytes = 256;
-constexpr int kMinQ = 2;
+constexpr int kMinQ = 8;
 constexpr int kMaxQ = 14;
 
 __host__ __device__ inline uint32_t pad16(uint64_t b) {
@@ -78,31 +82,39 @@ struct Geom {
   int64_t cg, th, tw;    // TILED group / tile sizes
   int64_t ng, nty, ntx;  // TILED counts per image
   int32_t ib_shift;      // log2(index_block)
-  int32_t pad;
+  int32_t nclass;        // TILED: tile classes in scheduling order (<= 8)
   uint64_t slot_bytes;   // CONTIG / TILED: uniform scratch slot per stream
   uint64_t slot_extra;   // 16 W + 16: per-stream scratch beyond 8 B/symbol
+  // TILED: a class is the set of tiles sharing (last channel group?, last
+  // tile row?, last tile column?); classes are listed largest tile first.
+  int64_t cls_start[8];  // first work index of the class
+  int32_t cls_bits[8];   // bit 0: last group, bit 1: last tile row, 2: last column
 };
 
 // One stream's extent.  Element i of a stream (coding order) sits at flat
-// position base + i (contiguous) or base + c*plane + h*row + w with
-// i = (c * hh + h) * ww + w (tiled).
+// position base + rel(i), where rel(i) = c*plane + h*row + w for
+// i = (c * hh + h) * ww + w.  A contiguous stream is the case hh = 1,
+// ww = "infinite", plane = row = 0 (rel(i) = i).  rel() fits in 32 bits: the
+// host checks C*H*W (tiled) and every stream length (contiguous) against 2^31.
+struct Tile {
+  int32_t hh, ww, plane, row;
+};
+constexpr int32_t kNoWrap = 0x7fffffff;
+
 struct StreamDesc {
   int64_t n;
   int64_t base;
-  int64_t plane, row;
-  int32_t hh, ww;
-  bool tiled;
+  Tile t;
   bool ok;
 };
 
 __device__ __forceinline__ StreamDesc stream_desc(const Geom &g, int64_t s) {
   StreamDesc d;
-  d.tiled = false;
   d.ok = true;
-  d.plane = 0;
-  d.row = 0;
-  d.hh = 1;
-  d.ww = 1;
+  d.t.hh = 1;
+  d.t.ww = kNoWrap;
+  d.t.plane = 0;
+  d.t.row = 0;
   if (g.kind == RANS_CHUNK_CONTIG) {
     int64_t a = s * g.per;
     a = a < g.n ? a : g.n;
@@ -112,7 +124,7 @@ __device__ __forceinline__ StreamDesc stream_desc(const Geom &g, int64_t s) {
     d.n = b - a;
   } else if (g.kind == RANS_CHUNK_EXPLICIT) {
     int64_t a = g.starts[s], b = g.starts[s + 1];
-    d.ok = (a >= 0) && (a <= b) && (b <= g.n);
+    d.ok = (a >= 0) && (a <= b) && (b <= g.n) && (b - a < (int64_t(1) << 31) - 64);
     d.base = a;
     d.n = d.ok ? b - a : 0;
   } else {
@@ -127,15 +139,39 @@ __device__ __forceinline__ StreamDesc stream_desc(const Geom &g, int64_t s) {
     int64_t nc = g.C - c0 < g.cg ? g.C - c0 : g.cg;
     int64_t hh = g.H - h0 < g.th ? g.H - h0 : g.th;
     int64_t ww = g.Wd - w0 < g.tw ? g.Wd - w0 : g.tw;
-    d.tiled = true;
-    d.plane = g.H * g.Wd;
-    d.row = g.Wd;
-    d.hh = (int32_t)hh;
-    d.ww = (int32_t)ww;
+    d.t.plane = (int32_t)(g.H * g.Wd);
+    d.t.row = (int32_t)g.Wd;
+    d.t.hh = (int32_t)hh;
+    d.t.ww = (int32_t)ww;
     d.base = ((b * g.C + c0) * g.H + h0) * g.Wd + w0;
     d.n = nc * hh * ww;
   }
   return d;
+}
+
+// Work index k -> stream id, visiting streams in non-increasing length order
+// (tiled: tile classes largest first; contiguous and explicit: as numbered).
+// Warps take work indices in a stride that spreads consecutive indices over
+// CTAs, so the long streams are shared out evenly over SMs and sub-partitions.
+__device__ __forceinline__ int64_t stream_of(const Geom &g, int64_t k) {
+  if (g.kind != RANS_CHUNK_TILED || g.nclass <= 1) return k;
+  int ci = 0;
+  while (ci + 1 < g.nclass && k >= g.cls_start[ci + 1]) ++ci;
+  int64_t j = k - g.cls_start[ci];
+  const int bits = g.cls_bits[ci];
+  const int64_t ngs = (bits & 1) ? 1 : (g.C % g.cg ? g.ng - 1 : g.ng);
+  const int64_t nys = (bits & 2) ? 1 : (g.H % g.th ? g.nty - 1 : g.nty);
+  const int64_t nxs = (bits & 4) ? 1 : (g.Wd % g.tw ? g.ntx - 1 : g.ntx);
+  const int64_t tx0 = j % nxs;
+  j /= nxs;
+  const int64_t ty0 = j % nys;
+  j /= nys;
+  const int64_t g0 = j % ngs;
+  const int64_t b = j / ngs;
+  const int64_t gi = (bits & 1) ? g.ng - 1 : g0;
+  const int64_t ty = (bits & 2) ? g.nty - 1 : ty0;
+  const int64_t tx = (bits & 4) ? g.ntx - 1 : tx0;
+  return ((b * g.ng + gi) * g.nty + ty) * g.ntx + tx;
 }
 
 // Byte offset of stream s's scratch slot end (words are written downward).
@@ -147,52 +183,105 @@ __device__ __forceinline__ uint64_t slot_end(const Geom &g, const StreamDesc &d,
   return g.slot_bytes * (uint64_t)(s + 1);
 }
 
-// Position walker over a stream's elements, stepping by +-k.
-struct Walker {
-  int64_t base, plane, row;
-  int32_t c, h, w, hh, ww;
-  bool tiled;
-  __device__ __forceinline__ void init(const StreamDesc &d, int64_t i) {
-    base = d.base;
-    plane = d.plane;
-    row = d.row;
-    hh = d.hh;
-    ww = d.ww;
-    tiled = d.tiled;
-    if (tiled) {
-      int64_t per = (int64_t)hh * ww;
-      int64_t cc = i / per;
-      int64_t rem = i - cc * per;
-      c = (int32_t)cc;
-      h = (int32_t)(rem / ww);
-      w = (int32_t)(rem - (int64_t)h * ww);
-    } else {
+// A position inside a stream, stepped by +-k elements.
+struct RelPos {
+  int32_t c, h, w;
+  __device__ __forceinline__ void init(const Tile &t, int32_t i) {
+    if (t.ww == kNoWrap) {
       c = 0;
       h = 0;
-      w = 0;
-      base = d.base + i;
+      w = i;
+    } else {
+      const int32_t per = t.hh * t.ww;
+      c = i / per;
+      const int32_t rem = i - c * per;
+      h = rem / t.ww;
+      w = rem - h * t.ww;
     }
   }
-  __device__ __forceinline__ int64_t pos() const {
-    return tiled ? base + (int64_t)c * plane + (int64_t)h * row + w : base;
-  }
-  __device__ __forceinline__ void fwd(int k) {
-    if (!tiled) { base += k; return; }
+  __device__ __forceinline__ int32_t rel(const Tile &t) const { return c * t.plane + h * t.row + w; }
+  __device__ __forceinline__ void fwd(const Tile &t, int32_t k) {
     w += k;
-    while (w >= ww) {
-      w -= ww;
-      if (++h >= hh) { h = 0; ++c; }
+    while (w >= t.ww) {
+      w -= t.ww;
+      if (++h >= t.hh) { h = 0; ++c; }
     }
   }
-  __device__ __forceinline__ void back(int k) {
-    if (!tiled) { base -= k; return; }
+  __device__ __forceinline__ void back(const Tile &t, int32_t k) {
     w -= k;
     while (w < 0) {
-      w += ww;
-      if (--h < 0) { h = hh - 1; --c; }
+      w += t.ww;
+      if (--h < 0) { h = t.hh - 1; --c; }
     }
   }
 };
+
+// Incremental form of RelPos for the warp kernels: rel is kept up to date,
+// stepping by +-k with at most a few row / channel wraps (one when ww >= k).
+struct Stepper {
+  int32_t w, h, rel;
+  int32_t ww, hh, drow, dplane;  // drow = row - ww, dplane = plane - hh * row
+  __device__ __forceinline__ void init(const Tile &t, int32_t i) {
+    RelPos p;
+    p.init(t, i);
+    w = p.w;
+    h = p.h;
+    rel = p.rel(t);
+    ww = t.ww;
+    hh = t.hh;
+    drow = t.row - t.ww;
+    dplane = t.plane - t.hh * t.row;
+  }
+  __device__ __forceinline__ void fwd(int32_t k) {
+    w += k;
+    rel += k;
+    while (w >= ww) {
+      w -= ww;
+      rel += drow;
+      if (++h >= hh) {
+        h = 0;
+        rel += dplane;
+      }
+    }
+  }
+  __device__ __forceinline__ void back(int32_t k) {
+    w -= k;
+    rel -= k;
+    while (w < 0) {
+      w += ww;
+      rel -= drow;
+      if (--h < 0) {
+        h = hh - 1;
+        rel -= dplane;
+      }
+    }
+  }
+};
+
+// Hints that bring data towards L2 ahead of use (no effect on results);
+// callers issue them only for addresses inside their own buffers.
+__device__ __forceinline__ void prefetch_l2(const void *p) {
+  asm volatile("prefetch.global.L2 [%0];" ::"l"(p));
+}
+
+// Bulk L2 prefetch of [p, p + bytes) restricted to whole 16-byte units that
+// lie inside [lo, hi) (cp.async.bulk.prefetch wants 16-byte alignment).
+__device__ __forceinline__ void bulk_prefetch_l2(const char *lo, const char *hi, const char *p,
+                                                 uint64_t bytes) {
+  uintptr_t a = reinterpret_cast<uintptr_t>(p);
+  uintptr_t b = a + bytes;
+  const uintptr_t l = (reinterpret_cast<uintptr_t>(lo) + 15) & ~uintptr_t(15);
+  const uintptr_t h = reinterpret_cast<uintptr_t>(hi) & ~uintptr_t(15);
+  a = (a + 15) & ~uintptr_t(15);
+  b &= ~uintptr_t(15);
+  if (a < l) a = l;
+  if (b > h) b = h;
+  while (a < b) {
+    uint32_t sz = (b - a) > 65536 ? 65536u : (uint32_t)(b - a);
+    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(a), "r"(sz) : "memory");
+    a += sz;
+  }
+}
 
 // ------------------------------------------------------------- symbols --
 template <typename T> struct SymIO;

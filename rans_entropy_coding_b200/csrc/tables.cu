@@ -308,13 +308,15 @@ __global__ void fill_slots_kernel(const int32_t *cdfs, int Lmax, const RowMeta *
   const int w = 1 << shift;
   const int a = t * w, b = a + w - 1;
   const int lo = bucket_of(row, nb, a);
-  const int hi = bucket_of(row, nb, b);
-  const int inside = hi - lo;
-  uint32_t code;
-  if (inside == 0) code = (uint32_t)w;
-  else if (inside == 1) code = (uint32_t)(row[lo + 1] - a);
-  else code = 0x8000u | (uint32_t)(inside < 0x7fff ? inside : 0x7fff);
-  slots[slot_base(m.slot) + t] = (uint32_t)lo | (code << 16);
+  const int inside = bucket_of(row, nb, b) - lo;
+  uint32_t e1 = 255u, e2 = 255u;
+  if (inside >= 3) {
+    e2 = (uint32_t)(inside - 3);
+  } else {
+    if (inside >= 1) e1 = (uint32_t)(row[lo + 1] - a - 1);
+    if (inside == 2) e2 = (uint32_t)(row[lo + 2] - a - 1);
+  }
+  slots[slot_base(m.slot) + t] = (uint32_t)lo | (e1 << 16) | (e2 << 24);
 }
 
 int ceil_log2(int64_t v) {
@@ -350,7 +352,7 @@ int launch_pmf_rows(const float *pmfs, int K, int stride, const int32_t *pmf_len
 uint64_t tables_bytes_bound(int K, int Lmax) {
   if (K <= 0 || Lmax < 2) return 0;
   const int64_t nb = (int64_t)Lmax - 1;
-  int q = ceil_log2(nb) + 1;
+  int q = ceil_log2(nb);
   q = q < kMinQ ? kMinQ : (q > kMaxQ ? kMaxQ : q);
   return (uint64_t)kHeaderBytes + pad16(16ull * K) + pad16(4ull * K * nb) +
          pad16(4ull * K * (1ull << q));
@@ -383,7 +385,7 @@ int prepare_tables(const int32_t *cdfs, int K, int Lmax, const int32_t *lengths,
     meta[r].offset = off[r];
     nbuckets += (uint64_t)nb;
     if (nb > max_nb) max_nb = nb;
-    int qq = ceil_log2(nb) + 1;
+    const int qq = ceil_log2(nb);
     q[r] = qq < kMinQ ? kMinQ : (qq > kMaxQ ? kMaxQ : qq);
   }
   if (nbuckets > (1ull << 31)) return RANS_ERR_ARG;
@@ -402,7 +404,9 @@ int prepare_tables(const int32_t *cdfs, int K, int Lmax, const int32_t *lengths,
   bool dec_smem = false;
   if (enc_smem) {
     const int64_t room = budget - meta_bytes - bucket_bytes;
-    // Halve the largest row's lookup until the three sections fit.
+    // About one slot per bucket (fewer than ~2% of lookups then meet three or
+    // more boundaries on the scale table); halve the largest row's lookup
+    // until the three sections fit.
     while ((int64_t)pad16(4ull * slot_total()) > room) {
       int best = -1;
       for (int r = 0; r < K; ++r)

@@ -74,8 +74,9 @@ def tiny(seed=0, n=4096):
     k = np.floor(2.0 ** rng.uniform(0.0, 30.0, size=n))
     sym = np.where(force, sign * (65.0 + k), sym)
     sym = sym.astype(np.int64)
-    sym[1] = np.iinfo(np.int32).min
-    sym[2] = np.iinfo(np.int32).max
+    if n > 2:
+        sym[1] = np.iinfo(np.int32).min
+        sym[2] = np.iinfo(np.int32).max
     return dict(name="tiny", symbols=sym.astype(np.int32), indexes=idx, scales=scales,
                 tail_mass=1e-9, chunking=dict(kind="contig", n_streams=1), W=1,
                 index_block=1)
