@@ -2,8 +2,8 @@
 """Throughput of librans_b200 on the 16-image 1080p latent batch.
 
 One step = the whole coding path over one batch: the 64 Gaussian CDF rows
-built from the scale table, the coder's tables prepared, every stream encoded
-(with compaction) and decoded, on one GPU per rank.  Workload: 16 synthetic
+built from the scale table, the coder's tables rebuilt from them, every
+stream encoded (with compaction) and decoded, on one GPU per rank.  Workload: 16 synthetic
 y latents [16, 192, 68, 120] int32 (25,067,520 symbols), one stream per
 64 x 64 spatial tile per group of 4 channels (3,072 streams), 32 interleaved
 states per stream.  Ranks shard by image (weak scaling: every rank codes its
@@ -228,7 +228,7 @@ def run_ours(args, world, rank, local):
     def step(e=None):
         if e: e[0].record(stream)
         rb.check(rb.rans_build_cdfs_from_scales(scales, tail, cdfs, lengths, offsets), "cdfs")
-        rb.check(rb.rans_tables_prepare(cdfs, lengths, offsets, blob, tables.c), "prepare")
+        rb.check(rb.rans_tables_refresh(cdfs, lengths, offsets, tables), "refresh")
         if e: e[1].record(stream)
         rb.check(rb.rans_encode_with_indexes(sym, idx, n, tables, ch, ws.out, ws.offsets,
                                              ws.enc), "encode")
@@ -242,6 +242,7 @@ def run_ours(args, world, rank, local):
     torch.cuda.synchronize()
     rb.check(rb.rans_get_status(ws.enc), "encode status")
     rb.check(rb.rans_get_status(ws.dec), "decode status")
+    rb.check(rb.rans_get_status(blob), "tables status")
     assert torch.equal(dec, sym), "round trip failed"
     barrier(world)
 
@@ -307,7 +308,7 @@ def run_ours(args, world, rank, local):
             d_sym.copy_(h_sym, non_blocking=True)
             d_idx.copy_(h_idx, non_blocking=True)
             rb.check(rb.rans_build_cdfs_from_scales(scales, tail, cdfs, lengths, offsets))
-            rb.check(rb.rans_tables_prepare(cdfs, lengths, offsets, blob, tables.c))
+            rb.check(rb.rans_tables_refresh(cdfs, lengths, offsets, tables))
             rb.check(rb.rans_encode_with_indexes(d_sym, d_idx, n, tables, ch, ws.out,
                                                  ws.offsets, ws.enc))
             total = int(ws.offsets[-1].item())
@@ -344,7 +345,7 @@ def run_ours(args, world, rank, local):
                "sample": "oracle encode+decode of streams 0..767 (images 0-3, %d symbols), "
                          "one stream per call over %d threads" % (ns, workers)}
 
-    launches_per_step = 1 + 2 + 3 + 1   # rows, prepare (pack, slots), enc+scan+copy, dec
+    launches_per_step = 1 + 1 + 3 + 1   # rows, table refresh, enc+scan+copy, dec
     if rank == 0:
         line = {
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,

@@ -202,6 +202,21 @@ int rans_tables_prepare(const int32_t *cdfs, int32_t K, int32_t Lmax,
                         const int32_t *cdf_lengths, const int32_t *offsets,
                         void *blob, uint64_t blob_bytes, rans_tables *out, void *stream);
 
+/*
+ * Rebuilds a prepared table set in place from new CDF rows whose lengths equal
+ * the rows it was prepared from (for example a scale table rebuilt every
+ * call): offsets, packed buckets and lookup slots are rewritten on the device
+ * with the layout kept, with no host synchronisation.  A row whose length
+ * differs, or a malformed row, records RANS_ERR_TABLE in the blob's status
+ * word (read it with rans_get_status(tables->blob, stream)); the table set is
+ * then unusable until prepared again.  Asynchronous.
+ *   cdfs: device int32[K][Lmax]; cdf_lengths, offsets: device int32[K];
+ *   tables: filled by rans_tables_prepare for the same K.
+ */
+int rans_tables_refresh(const int32_t *cdfs, int32_t K, int32_t Lmax,
+                        const int32_t *cdf_lengths, const int32_t *offsets,
+                        const rans_tables *tables, void *stream);
+
 /* ------------------------------------------------- sizes and queries ---- */
 
 /* Number of streams the chunking makes of n symbols (< 0: invalid chunking). */

@@ -12,4 +12,4 @@ from ._lib import (  # noqa: F401
     rans_build_cdfs_from_scales, rans_chunking, rans_debug_divide, rans_decode_with_indexes,
     rans_decode_workspace_bytes, rans_encode_with_indexes, rans_encode_workspace_bytes,
     rans_gaussian_lengths, rans_get_status, rans_max_compressed_bytes, rans_num_streams,
-    rans_tables, rans_tables_bytes, rans_tables_prepare)
+    rans_tables, rans_tables_bytes, rans_tables_prepare, rans_tables_refresh)

@@ -65,6 +65,7 @@ SIGNATURES = [
     ("rans_build_cdfs_from_pmfs", ctypes.c_int, [_P, _I32, _I32, _P, _P, _P, _I32, _P, _P]),
     ("rans_tables_bytes", _U64, [_I32, _I32]),
     ("rans_tables_prepare", ctypes.c_int, [_P, _I32, _I32, _P, _P, _P, _U64, _TBP, _P]),
+    ("rans_tables_refresh", ctypes.c_int, [_P, _I32, _I32, _P, _P, _TBP, _P]),
     ("rans_num_streams", _I64, [_CHP, _I64]),
     ("rans_encode_workspace_bytes", _U64, [_CHP, _I64]),
     ("rans_decode_workspace_bytes", _U64, [_CHP, _I64]),
@@ -154,6 +155,12 @@ def rans_tables_prepare(cdfs, cdf_lengths, offsets, blob, out, stream=None):
     return lib().rans_tables_prepare(_ptr(cdfs), cdfs.shape[0], cdfs.shape[1], _ptr(cdf_lengths),
                                      _ptr(offsets), _ptr(blob), blob.numel(), ctypes.byref(out),
                                      _stream(stream))
+
+
+def rans_tables_refresh(cdfs, cdf_lengths, offsets, tables, stream=None):
+    _need_cuda(cdfs, cdf_lengths, offsets)
+    return lib().rans_tables_refresh(_ptr(cdfs), cdfs.shape[0], cdfs.shape[1], _ptr(cdf_lengths),
+                                     _ptr(offsets), ctypes.byref(tables.c), _stream(stream))
 
 
 def rans_num_streams(chunking, n):

@@ -209,6 +209,14 @@ RANS_API int rans_tables_prepare(const int32_t *cdfs, int32_t K, int32_t Lmax,
                             as_stream(stream));
 }
 
+RANS_API int rans_tables_refresh(const int32_t *cdfs, int32_t K, int32_t Lmax,
+                                 const int32_t *cdf_lengths, const int32_t *offsets,
+                                 const rans_tables *tables, void *stream) {
+  if (!tables_usable(tables) || K != tables->K || Lmax < 2 || !cdfs || !cdf_lengths || !offsets)
+    return RANS_ERR_ARG;
+  return rb::refresh_tables(cdfs, K, Lmax, cdf_lengths, offsets, *tables, as_stream(stream));
+}
+
 RANS_API int64_t rans_num_streams(const rans_chunking *chunking, int64_t n) {
   Geom g;
   int st = make_geom(chunking, n, g);

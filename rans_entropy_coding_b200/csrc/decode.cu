@@ -74,7 +74,7 @@ struct EscapeResult {
 // The lane-serial part of a group holding an escape (after every lane's
 // symbol op): lanes take their words in ascending lane order; an escaping lane
 // reads its refill, count pieces and bypass pieces from the shared stream.
-__device__ __noinline__ EscapeResult escape_group(uint64_t x, bool active, bool esc,
+__device__ __forceinline__ EscapeResult escape_group(uint64_t x, bool active, bool esc,
                                                   uint32_t maxv, uint64_t abs0,
                                                   const uint32_t *words, uint64_t nw) {
   const int lane = threadIdx.x & 31;
@@ -145,10 +145,163 @@ __device__ __noinline__ EscapeResult escape_group(uint64_t x, bool active, bool 
   return r;
 }
 
+// Per-warp decoder state for one stream.
+struct WarpDec {
+  uint64_t x;            // this lane's state
+  uint64_t cur;          // absolute word index of the register window
+  uint32_t off;          // words of the window already consumed (< 32)
+  uint32_t w0, w1, w2;   // window words cur + lane, + 32, + 64 (w2: lookahead)
+  uint32_t rmax;         // largest row index seen (checked once per stream)
+  bool bad;
+};
+
+__device__ __forceinline__ uint32_t word_at(const uint32_t *words, uint64_t nw, uint64_t i) {
+  return i < nw ? __ldg(words + i) : 0u;
+}
+
+__device__ __forceinline__ void load_window(WarpDec &st, const uint32_t *words, uint64_t nw) {
+  const int lane = threadIdx.x & 31;
+  st.w0 = word_at(words, nw, st.cur + lane);
+  st.w1 = word_at(words, nw, st.cur + 32 + lane);
+  st.w2 = word_at(words, nw, st.cur + 64 + lane);
+}
+
+// One group of 32 symbols: lookup, state update, refill, output.  m is the
+// group's row metadata, loaded one group ahead.
+template <typename SymT, bool FULL>
+__device__ __forceinline__ void dec_group(WarpDec &st, const RowMeta &m, const uint32_t *buckets,
+                                          const uint32_t *slots, bool active, SymT *dst,
+                                          const uint32_t *words, uint64_t nw) {
+  const int lane = threadIdx.x & 31;
+  if (FULL) active = true;
+  const uint32_t cum = (uint32_t)st.x & (kTotal - 1);
+  const uint32_t sh = slot_shift(m.slot);
+  const uint32_t se = slots[slot_base(m.slot) + (cum >> sh)];
+  const uint32_t e1 = (se >> 16) & 0xffu, e2 = se >> 24;
+  const uint32_t c = cum & ((1u << sh) - 1u);
+  uint32_t sym = (se & 0xffffu) + (c > e1 ? 1u : 0u) + (c > e2 ? 1u : 0u);
+  const bool multi = active && e1 > e2;
+  if (__any_sync(kFull, multi)) {
+    if (multi) {  // last bucket in [lo, lo + count] whose start is <= cum
+      uint32_t lo = se & 0xffffu, hi = lo + e2 + 3u;
+      while (lo < hi) {
+        const uint32_t mid = (lo + hi + 1) >> 1;
+        if (bucket_start(buckets[m.bucket_base + mid]) <= cum) lo = mid; else hi = mid - 1;
+      }
+      sym = lo;
+    }
+  }
+  const uint32_t e = buckets[m.bucket_base + sym];
+  uint64_t x = st.x;
+  if (active) x = (uint64_t)bucket_freq(e) * (x >> kPrec) + (cum - bucket_start(e));
+  const bool esc = active && sym == m.maxv;
+  int32_t val = (int32_t)sym + m.offset;
+  if (!__any_sync(kFull, esc)) {
+    const bool need = active && x < kL;
+    const uint32_t nm = __ballot_sync(kFull, need);
+    const uint32_t j = st.off + __popc(nm & lanemask_lt());
+    // the lane holding window word j (mod 32) sends it from w0 or w1
+    const uint32_t wv = __shfl_sync(kFull, (uint32_t)lane >= st.off ? st.w0 : st.w1, j & 31);
+    if (need) x = (x << 32) | wv;
+    st.off += __popc(nm);
+    if (st.off >= 32) {
+      st.w0 = st.w1;
+      st.w1 = st.w2;
+      st.cur += 32;
+      st.off -= 32;
+      st.w2 = word_at(words, nw, st.cur + 64 + lane);
+    }
+  } else {
+    const EscapeResult er = escape_group(x, active, esc, m.maxv, st.cur + st.off, words, nw);
+    x = er.x;
+    if (esc) val = (int32_t)(er.val + (int64_t)m.offset);
+    st.bad |= er.bad;
+    st.cur = er.cur;
+    st.off = 0;
+    load_window(st, words, nw);
+  }
+  st.x = x;
+  if (active) *dst = (SymT)val;
+}
+
+template <typename SymT, bool IB0, bool WIDE>
+__device__ __forceinline__ void decode_stream_w32(const DecCtx &c, const StreamDesc &d,
+                                                  const RowMeta *meta, const uint32_t *buckets,
+                                                  const uint32_t *slots, int64_t s,
+                                                  const uint32_t *words, uint64_t nw) {
+  const int lane = threadIdx.x & 31;
+  const int32_t n = (int32_t)d.n;
+  const int32_t G = (n + 31) >> 5;
+  const int64_t base = d.base;
+  const int ib = c.g.ib_shift;
+  const int32_t *idx_s = c.idx + (IB0 ? base : 0);
+  SymT *out_s = reinterpret_cast<SymT *>(c.out) + base;
+  const uint32_t kmax = (uint32_t)c.K - 1u;
+  auto load_idx = [&](int32_t rel) -> int32_t {
+    return IB0 ? __ldg(idx_s + rel) : __ldg(c.idx + ((base + rel) >> ib));
+  };
+
+  WarpDec st;
+  st.x = (uint64_t)__ldg(words + 2 * lane) | ((uint64_t)__ldg(words + 2 * lane + 1) << 32);
+  st.cur = 64;
+  st.off = 0;
+  load_window(st, words, nw);
+  st.rmax = 0;
+  st.bad = false;
+
+  Stepper<WIDE> pl;
+  pl.init(d.t, lane);
+  int32_t rrel[kRing], ridx[kRing];
+#pragma unroll
+  for (int u = 0; u < kRing; ++u) {
+    rrel[u] = pl.rel;
+    ridx[u] = lane < n - u * 32 ? load_idx(pl.rel) : 0;
+    pl.fwd(32);
+  }
+  auto meta_of = [&](int32_t r) -> RowMeta {
+    st.rmax = max(st.rmax, (uint32_t)r);
+    return row_meta(meta, min((uint32_t)r, kmax));
+  };
+  RowMeta m = meta_of(ridx[0]);
+  // Group g uses ring slot g mod kRing; its slot is refilled with group
+  // g + kRing, and the next group's metadata is loaded one group ahead.
+  auto step = [&](int u, int32_t g, bool full) {
+    const int32_t rel = rrel[u];
+    const RowMeta mn = meta_of(ridx[(u + 1) % kRing]);
+    if (g + kRing < G) {
+      rrel[u] = pl.rel;
+      ridx[u] = lane < n - (g + kRing) * 32 ? load_idx(pl.rel) : 0;
+      pl.fwd(32);
+    }
+    if (full)
+      dec_group<SymT, true>(st, m, buckets, slots, true, out_s + rel, words, nw);
+    else
+      dec_group<SymT, false>(st, m, buckets, slots, lane < n - g * 32, out_s + rel, words, nw);
+    m = mn;
+  };
+  // every group but the last is full
+  int32_t g0 = 0;
+  for (; g0 + kRing < G; g0 += kRing) {
+#pragma unroll
+    for (int u = 0; u < kRing; ++u) step(u, g0 + u, true);
+  }
+#pragma unroll
+  for (int u = 0; u < kRing; ++u) {
+    if (g0 + u >= G) break;
+    step(u, g0 + u, false);
+  }
+  if (__any_sync(kFull, st.rmax > kmax)) {
+    if (lane == 0) report(c.status, RANS_ERR_INDEX, s);
+    return;
+  }
+  const bool ok = !st.bad && st.x == kL && st.cur + st.off == nw;
+  if (!__all_sync(kFull, ok) && lane == 0) report(c.status, RANS_ERR_CORRUPT, s);
+}
+
 template <typename SymT, bool IB0>
-__device__ __forceinline__ void decode_stream_w32(const DecCtx &c, const RowMeta *meta,
-                                                  const uint32_t *buckets,
-                                                  const uint32_t *slots, int64_t s) {
+__device__ __forceinline__ void decode_stream_w32_entry(const DecCtx &c, const RowMeta *meta,
+                                                        const uint32_t *buckets,
+                                                        const uint32_t *slots, int64_t s) {
   const int lane = threadIdx.x & 31;
   const StreamDesc d = stream_desc(c.g, s);
   const uint32_t *words = nullptr;
@@ -161,107 +314,10 @@ __device__ __forceinline__ void decode_stream_w32(const DecCtx &c, const RowMeta
     bulk_prefetch_l2(reinterpret_cast<const char *>(c.in),
                      reinterpret_cast<const char *>(c.in) + c.in_bytes,
                      reinterpret_cast<const char *>(words + 64), 4 * (nw - 64));
-  const int32_t n = (int32_t)d.n;
-  const int32_t G = (n + 31) >> 5;
-  const int64_t base = d.base;
-  const int ib = c.g.ib_shift;
-  const int32_t *idx_s = c.idx + (IB0 ? base : 0);
-  SymT *out_s = reinterpret_cast<SymT *>(c.out) + base;
-  const uint32_t K = (uint32_t)c.K;
-  auto load_idx = [&](int32_t rel) -> int32_t {
-    return IB0 ? __ldg(idx_s + rel) : __ldg(c.idx + ((base + rel) >> ib));
-  };
-
-  uint64_t x = (uint64_t)__ldg(words + 2 * lane) | ((uint64_t)__ldg(words + 2 * lane + 1) << 32);
-  uint64_t cur = 64;  // absolute word index of the window start
-  uint32_t off = 0;   // words of the window already consumed
-  uint32_t w0 = cur + lane < nw ? __ldg(words + cur + lane) : 0u;
-  uint32_t w1 = cur + 32 + lane < nw ? __ldg(words + cur + 32 + lane) : 0u;
-  bool bad = false, bad_idx = false;
-
-  Stepper pl;
-  pl.init(d.t, lane);
-  int32_t rrel[kRing], ridx[kRing];
-#pragma unroll
-  for (int u = 0; u < kRing; ++u) {
-    rrel[u] = pl.rel;
-    ridx[u] = lane < n - u * 32 ? load_idx(pl.rel) : 0;
-    pl.fwd(32);
-  }
-
-  for (int32_t g0 = 0; g0 < G; g0 += kRing) {
-#pragma unroll
-    for (int u = 0; u < kRing; ++u) {
-      const int32_t g = g0 + u;
-      if (g >= G) break;
-      const bool active = lane < n - g * 32;
-      const int32_t rel = rrel[u];
-      uint32_t r = (uint32_t)ridx[u];
-      if (g + kRing < G) {
-        rrel[u] = pl.rel;
-        ridx[u] = lane < n - (g + kRing) * 32 ? load_idx(pl.rel) : 0;
-        pl.fwd(32);
-      }
-      bad_idx |= r >= K;
-      r = r < K ? r : 0u;
-      const RowMeta m = meta[r];
-      const uint32_t cum = (uint32_t)x & (kTotal - 1);
-      const uint32_t sh = slot_shift(m.slot);
-      const uint32_t se = slots[slot_base(m.slot) + (cum >> sh)];
-      bool multi;
-      uint32_t sym = slot_symbol(se, cum & ((1u << sh) - 1u), multi);
-      uint32_t mm = __ballot_sync(kFull, active && multi);
-      while (mm) {
-        const int l = __ffs(mm) - 1;
-        mm &= mm - 1;
-        const uint32_t base_l = __shfl_sync(kFull, m.bucket_base + (se & 0xffffu), l);
-        const uint32_t cnt_l = __shfl_sync(kFull, (se >> 24) + 3u, l);
-        const uint32_t cum_l = __shfl_sync(kFull, cum, l);
-        uint32_t cnt = 0;
-        for (uint32_t k0 = 0; k0 < cnt_l; k0 += 32) {
-          const uint32_t k = k0 + lane + 1;
-          const bool le = k <= cnt_l && bucket_start(buckets[base_l + k]) <= cum_l;
-          cnt += __popc(__ballot_sync(kFull, le));
-        }
-        if (lane == l) sym = (se & 0xffffu) + cnt;
-      }
-      const uint32_t e = buckets[m.bucket_base + sym];
-      if (active) x = (uint64_t)bucket_freq(e) * (x >> kPrec) + (cum - bucket_start(e));
-      const bool esc = active && sym == m.maxv;
-      int32_t val = (int32_t)sym + m.offset;
-      if (!__any_sync(kFull, esc)) {
-        const bool need = active && x < kL;
-        const uint32_t nm = __ballot_sync(kFull, need);
-        const uint32_t j = off + __popc(nm & lanemask_lt());
-        const uint32_t a = __shfl_sync(kFull, w0, j & 31);
-        const uint32_t b = __shfl_sync(kFull, w1, j & 31);
-        if (need) x = (x << 32) | (j < 32 ? a : b);
-        off += __popc(nm);
-        if (off >= 32) {
-          w0 = w1;
-          cur += 32;
-          off -= 32;
-          w1 = cur + 32 + lane < nw ? __ldg(words + cur + 32 + lane) : 0u;
-        }
-      } else {
-        const EscapeResult er = escape_group(x, active, esc, m.maxv, cur + off, words, nw);
-        x = er.x;
-        if (esc) val = (int32_t)(er.val + (int64_t)m.offset);
-        bad |= er.bad;
-        cur = er.cur;
-        off = 0;
-        w0 = cur + lane < nw ? __ldg(words + cur + lane) : 0u;
-        w1 = cur + 32 + lane < nw ? __ldg(words + cur + 32 + lane) : 0u;
-      }
-      if (active) out_s[rel] = (SymT)val;
-    }
-  }
-  if (__any_sync(kFull, bad_idx)) {
-    if (lane == 0) report(c.status, RANS_ERR_INDEX, s);
-    return;
-  }
-  const bool ok = !bad && x == kL && cur + off == nw;
-  if (!__all_sync(kFull, ok) && lane == 0) report(c.status, RANS_ERR_CORRUPT, s);
+  if (d.t.ww >= 32)
+    decode_stream_w32<SymT, IB0, true>(c, d, meta, buckets, slots, s, words, nw);
+  else
+    decode_stream_w32<SymT, IB0, false>(c, d, meta, buckets, slots, s, words, nw);
 }
 
 template <typename SymT>
@@ -309,7 +365,7 @@ __device__ void decode_stream_w1(const DecCtx &c, const RowMeta *meta, const uin
       report(c.status, RANS_ERR_INDEX, s);
       return;
     }
-    const RowMeta m = meta[r];
+    const RowMeta m = row_meta(meta, (uint32_t)r);
     const uint32_t cum = (uint32_t)x & (kTotal - 1);
     const uint32_t sh = slot_shift(m.slot);
     const uint32_t se = slots[slot_base(m.slot) + (cum >> sh)];
@@ -376,7 +432,7 @@ __global__ void __launch_bounds__(W == 32 ? kDecMaxThreads32 : kDecThreads1)
     const int warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
     for (int64_t k = blockIdx.x + (int64_t)gridDim.x * warp; k < c.g.S;
          k += (int64_t)gridDim.x * nw)
-      decode_stream_w32<SymT, IB0>(c, meta, buckets, slots, stream_of(c.g, k));
+      decode_stream_w32_entry<SymT, IB0>(c, meta, buckets, slots, stream_of(c.g, k));
   } else {
     for (int64_t k = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; k < c.g.S;
          k += (int64_t)gridDim.x * blockDim.x)

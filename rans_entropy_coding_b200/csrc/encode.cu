@@ -23,7 +23,7 @@
 namespace rb {
 namespace {
 
-constexpr int kEncThreads32 = 512;
+constexpr int kEncThreads32 = 1024;
 constexpr int kEncThreads1 = 128;
 
 struct EncCtx {
@@ -101,10 +101,10 @@ constexpr int kRing = 4;
 // A group holding an escape, off the fast path: every lane counts the words
 // its ops push, a suffix sum over lanes places each lane's block (lanes > l
 // push first in the serial order), then each lane writes its words.
-__device__ __noinline__ uint64_t escape_group_enc(uint64_t x, bool active, uint32_t start,
-                                                  uint32_t freq, double rcp, uint64_t raw,
-                                                  bool esc, uint32_t *end, uint32_t cursor,
-                                                  uint32_t *total) {
+__device__ __forceinline__ uint64_t escape_group_enc(uint64_t x, bool active, uint32_t start,
+                                                     uint32_t freq, double rcp, uint64_t raw,
+                                                     bool esc, uint32_t *end, uint32_t cursor,
+                                                     uint32_t &total) {
   const int lane = threadIdx.x & 31;
   uint32_t k = 0;
   if (active) {
@@ -117,20 +117,61 @@ __device__ __noinline__ uint64_t escape_group_enc(uint64_t x, bool active, uint3
     const uint32_t t = __shfl_down_sync(kFull, inc, o);
     if (lane + o < 32) inc += t;
   }
-  *total = __shfl_sync(kFull, inc, 0);
+  total = __shfl_sync(kFull, inc, 0);
   if (active) symbol_ops<true>(x, start, freq, rcp, raw, esc, end, cursor + inc - k);
   return x;
 }
 
-template <typename SymT, bool IB0>
-__device__ __forceinline__ void encode_stream_w32(const EncCtx &c, const RowMeta *meta,
-                                                  const uint32_t *buckets, int64_t s) {
-  const int lane = threadIdx.x & 31;
-  const StreamDesc d = stream_desc(c.g, s);
-  if (!d.ok) {
-    if (lane == 0) report(c.status, RANS_ERR_ARG, s);
-    return;
+// Per-warp encoder state for one stream.
+struct WarpEnc {
+  uint64_t x;        // this lane's state
+  uint32_t cursor;   // words pushed so far (written at end[-1 - k])
+  uint32_t rmax;     // largest row index seen (checked once per stream)
+  bool range_err;
+};
+
+// One group of 32 symbols, coded lane 31 first.  m is the group's row
+// metadata, loaded one group ahead.
+template <bool FULL>
+__device__ __forceinline__ void enc_group(WarpEnc &st, const RowMeta &m, const uint32_t *buckets,
+                                          int32_t sv, bool active, uint32_t above,
+                                          uint32_t *end) {
+  if (FULL) active = true;
+  // value mapping: in range iff 0 <= s - offset < maxv (64-bit, exact)
+  const int64_t v = (int64_t)sv - (int64_t)m.offset;
+  const bool in_range = (uint64_t)v < (uint64_t)m.maxv;
+  const uint32_t e = buckets[m.bucket_base + (in_range ? (uint32_t)v : m.maxv)];
+  const uint32_t start = bucket_start(e), freq = bucket_freq(e);
+  const bool esc = active && !in_range;
+  const double rcp = freq_reciprocal(freq);
+  uint64_t x = st.x;
+  if (!__any_sync(kFull, esc)) {
+    // x >= freq * 2^47  <=>  high word of x >= freq * 2^15
+    const bool need = active && (uint32_t)(x >> 32) >= (freq << 15);
+    const uint32_t bm = __ballot_sync(kFull, need);
+    if (need) {
+      end[-1 - (int64_t)(st.cursor + __popc(bm & above))] = (uint32_t)x;
+      x >>= 32;
+    }
+    st.cursor += __popc(bm);
+    if (active) x = enc_sym_step(x, start, freq, rcp);
+  } else {
+    uint64_t raw = 0;
+    if (esc) raw = v < 0 ? (uint64_t)(-2 * v - 1) : (uint64_t)(2 * (v - (int64_t)m.maxv));
+    st.range_err |= esc && (raw >> 60) != 0;
+    uint32_t total;
+    x = escape_group_enc(x, active, start, freq, rcp, raw & ((1ull << 60) - 1), esc, end,
+                         st.cursor, total);
+    st.cursor += total;
   }
+  st.x = x;
+}
+
+template <typename SymT, bool IB0, bool WIDE>
+__device__ __forceinline__ void encode_stream_w32(const EncCtx &c, const StreamDesc &d,
+                                                  const RowMeta *meta, const uint32_t *buckets,
+                                                  int64_t s) {
+  const int lane = threadIdx.x & 31;
   uint32_t *end = reinterpret_cast<uint32_t *>(c.scratch + slot_end(c.g, d, s));
   const int32_t n = (int32_t)d.n;
   const int32_t G = (n + 31) >> 5;
@@ -138,18 +179,21 @@ __device__ __forceinline__ void encode_stream_w32(const EncCtx &c, const RowMeta
   const int ib = c.g.ib_shift;
   const int32_t *idx_s = c.idx + (IB0 ? base : 0);
   const SymT *sym_s = reinterpret_cast<const SymT *>(c.sym) + base;
-  const uint32_t K = (uint32_t)c.K;
+  const uint32_t kmax = (uint32_t)c.K - 1u;
   auto load = [&](int32_t rel, int32_t &sv, int32_t &r) {
     sv = SymIO<SymT>::load(sym_s, rel);
     r = IB0 ? __ldg(idx_s + rel) : __ldg(c.idx + ((base + rel) >> ib));
   };
-  uint64_t x = kL;
-  uint32_t cursor = 0;
-  bool bad_idx = false;
   const uint32_t above = 0xfffffffeu << lane;   // lanes > this lane
+  WarpEnc st;
+  st.x = kL;
+  st.cursor = 0;
+  st.rmax = 0;
+  st.range_err = false;
 
-  // groups are coded G-1 down to 0; ring slot u holds group G-1-(k+u)
-  Stepper pl;
+  // Groups are coded G-1 down to 0; the k-th coded group (G-1-k) uses ring
+  // slot k mod kRing, which is then refilled with group G-1-(k+kRing).
+  Stepper<WIDE> pl;
   pl.init(d.t, (G > 0 ? G - 1 : 0) * 32 + lane);
   int32_t rsym[kRing], ridx[kRing];
 #pragma unroll
@@ -159,63 +203,64 @@ __device__ __forceinline__ void encode_stream_w32(const EncCtx &c, const RowMeta
     if (u < G && lane < n - (G - 1 - u) * 32) load(pl.rel, rsym[u], ridx[u]);
     if (u + 1 < G) pl.back(32);
   }
-
-  for (int32_t k0 = 0; k0 < G; k0 += kRing) {
-#pragma unroll
-    for (int u = 0; u < kRing; ++u) {
-      const int32_t k = k0 + u;
-      if (k >= G) break;
-      const int32_t g = G - 1 - k;
-      const bool active = lane < n - g * 32;
-      const int32_t sv = rsym[u];
-      uint32_t r = (uint32_t)ridx[u];
-      if (g - kRing >= 0) {     // every lane of an earlier group is active
-        load(pl.rel, rsym[u], ridx[u]);
-        if (g - kRing > 0) pl.back(32);
-      }
-      bad_idx |= r >= K;
-      r = r < K ? r : 0u;
-      const RowMeta m = meta[r];
-      // value mapping: in range iff 0 <= s - offset < maxv (64-bit, exact)
-      const int64_t v = (int64_t)sv - (int64_t)m.offset;
-      const bool in_range = (uint64_t)v < (uint64_t)m.maxv;
-      const uint32_t e = buckets[m.bucket_base + (in_range ? (uint32_t)v : m.maxv)];
-      const uint32_t start = bucket_start(e), freq = bucket_freq(e);
-      const bool esc = active && !in_range;
-      const double rcp = freq_reciprocal(freq);
-      if (!__any_sync(kFull, esc)) {
-        // x >= freq * 2^47  <=>  high word of x >= freq * 2^15
-        const bool need = active && (uint32_t)(x >> 32) >= (freq << 15);
-        const uint32_t bm = __ballot_sync(kFull, need);
-        if (need) {
-          end[-1 - (int64_t)(cursor + __popc(bm & above))] = (uint32_t)x;
-          x >>= 32;
-        }
-        cursor += __popc(bm);
-        if (active) x = enc_sym_step(x, start, freq, rcp);
-      } else {
-        uint64_t raw = 0;
-        if (esc) raw = v < 0 ? (uint64_t)(-2 * v - 1) : (uint64_t)(2 * (v - (int64_t)m.maxv));
-        if (__any_sync(kFull, esc && (raw >> 60) != 0)) {
-          if (lane == 0) report(c.status, RANS_ERR_RANGE, s);
-          return;
-        }
-        uint32_t total;
-        x = escape_group_enc(x, active, start, freq, rcp, raw, esc, end, cursor, &total);
-        cursor += total;
-      }
+  auto meta_of = [&](int32_t r) -> RowMeta {
+    st.rmax = max(st.rmax, (uint32_t)r);
+    return row_meta(meta, min((uint32_t)r, kmax));
+  };
+  RowMeta m = meta_of(ridx[0]);
+  auto step = [&](int u, int32_t k, bool full) {
+    const int32_t g = G - 1 - k;
+    const int32_t sv = rsym[u];
+    const RowMeta mn = meta_of(ridx[(u + 1) % kRing]);
+    if (g - kRing >= 0) {     // every lane of an earlier group is active
+      load(pl.rel, rsym[u], ridx[u]);
+      if (g - kRing > 0) pl.back(32);
     }
+    if (full)
+      enc_group<true>(st, m, buckets, sv, true, above, end);
+    else
+      enc_group<false>(st, m, buckets, sv, lane < n - g * 32, above, end);
+    m = mn;
+  };
+  // the last group (coded first) may be partial; every other group is full
+  if (G > 0) step(0, 0, false);
+  int32_t k0 = 1;
+  for (; k0 + kRing <= G; k0 += kRing) {
+#pragma unroll
+    for (int u = 0; u < kRing; ++u) step((u + 1) % kRing, k0 + u, true);
   }
-  if (__any_sync(kFull, bad_idx)) {
+#pragma unroll
+  for (int u = 0; u < kRing; ++u) {
+    if (k0 + u >= G) break;
+    step((u + 1) % kRing, k0 + u, true);
+  }
+  if (__any_sync(kFull, st.rmax > kmax)) {
     if (lane == 0) report(c.status, RANS_ERR_INDEX, s);
     return;
   }
+  if (__any_sync(kFull, st.range_err)) {
+    if (lane == 0) report(c.status, RANS_ERR_RANGE, s);
+    return;
+  }
   // flush: lanes 31..0 push high then low, so lane 0's low word comes first
-  const uint32_t kk = cursor + 2u * (31u - (uint32_t)lane);
-  end[-1 - (int64_t)kk] = (uint32_t)(x >> 32);
-  end[-2 - (int64_t)kk] = (uint32_t)x;
-  cursor += 64;
-  if (lane == 0) c.lens[s] = 4ull * cursor;
+  const uint32_t kk = st.cursor + 2u * (31u - (uint32_t)lane);
+  end[-1 - (int64_t)kk] = (uint32_t)(st.x >> 32);
+  end[-2 - (int64_t)kk] = (uint32_t)st.x;
+  if (lane == 0) c.lens[s] = 4ull * (st.cursor + 64);
+}
+
+template <typename SymT, bool IB0>
+__device__ __forceinline__ void encode_stream_w32_entry(const EncCtx &c, const RowMeta *meta,
+                                                        const uint32_t *buckets, int64_t s) {
+  const StreamDesc d = stream_desc(c.g, s);
+  if (!d.ok) {
+    if ((threadIdx.x & 31) == 0) report(c.status, RANS_ERR_ARG, s);
+    return;
+  }
+  if (d.t.ww >= 32)
+    encode_stream_w32<SymT, IB0, true>(c, d, meta, buckets, s);
+  else
+    encode_stream_w32<SymT, IB0, false>(c, d, meta, buckets, s);
 }
 
 template <typename SymT>
@@ -260,7 +305,7 @@ __device__ void encode_stream_w1(const EncCtx &c, const RowMeta *meta, const uin
     uint32_t start, freq;
     uint64_t raw;
     bool esc;
-    map_symbol(sv, meta[r], buckets, start, freq, raw, esc);
+    map_symbol(sv, row_meta(meta, (uint32_t)r), buckets, start, freq, raw, esc);
     if (esc && (raw >> 60) != 0) {
       report(c.status, RANS_ERR_RANGE, s);
       return;
@@ -294,7 +339,7 @@ __global__ void __launch_bounds__(W == 32 ? kEncThreads32 : kEncThreads1)
     const int warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
     for (int64_t k = blockIdx.x + (int64_t)gridDim.x * warp; k < c.g.S;
          k += (int64_t)gridDim.x * nw)
-      encode_stream_w32<SymT, IB0>(c, meta, buckets, stream_of(c.g, k));
+      encode_stream_w32_entry<SymT, IB0>(c, meta, buckets, stream_of(c.g, k));
   } else {
     for (int64_t k = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; k < c.g.S;
          k += (int64_t)gridDim.x * blockDim.x)

@@ -22,7 +22,10 @@ constexpr uint32_t kBypassMax = 15;
 constexpr unsigned kFull = 0xffffffffu;
 
 // ------------------------------------------------------------ table blob --
-// [header 256 B][RowMeta K][bucket words][slot words], sections 16-B padded.
+// [header 256 B][RowMeta K x 8][bucket words][slot words], sections 16-B
+// padded.  Each row's metadata is stored 8 times side by side (128 bytes per
+// row): lane l of a warp reads copy l mod 8, so the 8 lanes served by one
+// shared-memory wavefront of 16-byte loads always hit 8 different bank groups.
 // A bucket word packs start | (width - 1) << 16.
 // Each row has 2^q slots (8 <= q <= 14) of width w = 2^(16-q) <= 256 over the
 // cumulative range; a slot word packs lo | e1 << 16 | e2 << 24 where lo is the
@@ -40,6 +43,11 @@ struct RowMeta {
   uint32_t slot;         // slot base | (16 - q) << 27, q = log2(slots in row)
 };
 static_assert(sizeof(RowMeta) == 16, "RowMeta is one 16-byte load");
+constexpr int kMetaCopies = 8;
+
+__device__ __forceinline__ const RowMeta &row_meta(const RowMeta *meta, uint32_t r) {
+  return meta[r * kMetaCopies + (threadIdx.x & (kMetaCopies - 1))];
+}
 
 constexpr uint32_t kHeaderBytes = 256;
 constexpr int kMinQ = 8;
@@ -217,7 +225,9 @@ struct RelPos {
 };
 
 // Incremental form of RelPos for the warp kernels: rel is kept up to date,
-// stepping by +-k with at most a few row / channel wraps (one when ww >= k).
+// stepping by +-k.  WIDE (tile width >= k, or a contiguous stream) needs at
+// most one row wrap per step and runs branch-free; narrow tiles loop.
+template <bool WIDE>
 struct Stepper {
   int32_t w, h, rel;
   int32_t ww, hh, drow, dplane;  // drow = row - ww, dplane = plane - hh * row
@@ -235,24 +245,44 @@ struct Stepper {
   __device__ __forceinline__ void fwd(int32_t k) {
     w += k;
     rel += k;
-    while (w >= ww) {
-      w -= ww;
-      rel += drow;
-      if (++h >= hh) {
-        h = 0;
-        rel += dplane;
+    if (WIDE) {
+      const bool wr = w >= ww;
+      w -= wr ? ww : 0;
+      rel += wr ? drow : 0;
+      h += wr ? 1 : 0;
+      const bool cw = h >= hh;
+      h = cw ? 0 : h;
+      rel += cw ? dplane : 0;
+    } else {
+      while (w >= ww) {
+        w -= ww;
+        rel += drow;
+        if (++h >= hh) {
+          h = 0;
+          rel += dplane;
+        }
       }
     }
   }
   __device__ __forceinline__ void back(int32_t k) {
     w -= k;
     rel -= k;
-    while (w < 0) {
-      w += ww;
-      rel -= drow;
-      if (--h < 0) {
-        h = hh - 1;
-        rel -= dplane;
+    if (WIDE) {
+      const bool wr = w < 0;
+      w += wr ? ww : 0;
+      rel -= wr ? drow : 0;
+      h -= wr ? 1 : 0;
+      const bool cw = h < 0;
+      h = cw ? hh - 1 : h;
+      rel -= cw ? dplane : 0;
+    } else {
+      while (w < 0) {
+        w += ww;
+        rel -= drow;
+        if (--h < 0) {
+          h = hh - 1;
+          rel -= dplane;
+        }
       }
     }
   }

@@ -19,6 +19,8 @@ int launch_pmf_rows(const float *pmfs, int K, int stride, const int32_t *pmf_len
                     const float *tail, int32_t *cdfs, int Lmax, int32_t *lengths,
                     cudaStream_t st);
 uint64_t tables_bytes_bound(int K, int Lmax);
+int refresh_tables(const int32_t *cdfs, int K, int Lmax, const int32_t *lengths,
+                   const int32_t *offsets, const rans_tables &t, cudaStream_t st);
 int prepare_tables(const int32_t *cdfs, int K, int Lmax, const int32_t *lengths,
                    const int32_t *offsets, void *blob, uint64_t blob_bytes, rans_tables *out,
                    cudaStream_t st);

@@ -89,59 +89,93 @@ __device__ __forceinline__ long long scaled_freq(float p) {
 
 // Quantises n probabilities (pf(i), the last one the tail mass) into row[0..n]
 // of a CDF row.  Returns RANS_OK or RANS_ERR_TABLE (same value on every
-// thread).  row[] is used as scratch for the widths.
+// thread).  row[1..n] holds first the rounded probabilities, then the bucket
+// widths, then the CDF.
+constexpr int kHistMax = 64;  // widths 2..kHistMax are histogrammed for the steal step
+
 template <class PF>
-__device__ int quantise_row(const PF &pf, int n, int32_t *row, BlockScratch &sh) {
-  // pass 1: total of the rounded values
+__device__ int quantise_row(const PF &pf, int n, int32_t *row, BlockScratch &sh,
+                            unsigned int *hist) {
+  // pass 1: rounded values (each probability evaluated once) and their total
   unsigned long long local = 0;
   int bad = 0;
   for (int i = threadIdx.x; i < n; i += kRowThreads) {
     long long f = scaled_freq(pf(i));
-    if (f < 0) bad = 1; else local += (unsigned long long)f;
+    if (f < 0) {
+      bad = 1;
+      f = 0;
+    }
+    local += (unsigned long long)f;
+    row[i + 1] = (int32_t)(uint32_t)f;
   }
+  for (int i = threadIdx.x; i <= kHistMax; i += kRowThreads) hist[i] = 0;
   const unsigned long long T = block_sum(local, sh);
   bad = __syncthreads_or(bad);
   if (bad || T == 0) return RANS_ERR_TABLE;
 
-  // pass 2: widths of the rescaled running sum, floor(2^16 c / T)
-  unsigned long long carry = 0;
+  // pass 2: widths of the rescaled running sum floor(2^16 c / T); count the
+  // empty buckets and histogram the narrow ones
+  unsigned long long carry = 0, zl = 0;
   for (int base = 0; base < n; base += kRowThreads) {
     int i = base + threadIdx.x;
-    unsigned long long f = 0;
-    if (i < n) f = (unsigned long long)scaled_freq(pf(i));
+    unsigned long long f = i < n ? (unsigned long long)(uint32_t)row[i + 1] : 0ull;
     unsigned long long tot;
     unsigned long long ex = block_excl_scan(f, sh, &tot) + carry;
     if (i < n) {
       unsigned long long c0 = ((unsigned long long)kTotal * ex) / T;
       unsigned long long c1 = ((unsigned long long)kTotal * (ex + f)) / T;
-      row[i + 1] = (int32_t)(c1 - c0);
+      const uint32_t w = (uint32_t)(c1 - c0);
+      row[i + 1] = (int32_t)w;
+      zl += (w == 0);
+      if (w >= 2 && w <= kHistMax) atomicAdd(&hist[w], 1u);
     }
     carry += tot;
   }
-  __syncthreads();
-
-  // empty buckets
-  unsigned long long zl = 0;
-  for (int i = threadIdx.x; i < n; i += kRowThreads) zl += (row[i + 1] == 0);
   const unsigned long long Z = block_sum(zl, sh);
   if (Z > 0) {
-    // S(t) = sum over buckets with 1 < w <= t of (w - 1)
-    auto S = [&](long long t) -> unsigned long long {
-      unsigned long long s = 0;
-      for (int i = threadIdx.x; i < n; i += kRowThreads) {
-        long long w = row[i + 1];
-        if (w > 1 && w <= t) s += (unsigned long long)(w - 1);
+    // The Z units come from the buckets in (width, index) order, each drained
+    // to width 1: find the threshold width t, the smallest with
+    // S(t) = sum over 1 < w <= t of (w - 1) reaching Z.
+    long long t = 0;
+    unsigned long long below = 0;  // S(t - 1)
+    if (threadIdx.x == 0) {
+      unsigned long long run = 0;
+      for (int v = 2; v <= kHistMax; ++v) {
+        const unsigned long long add = (unsigned long long)hist[v] * (unsigned long long)(v - 1);
+        if (run + add >= Z) {
+          t = v;
+          below = run;
+          break;
+        }
+        run += add;
       }
-      return block_sum(s, sh);
-    };
-    if (S(kTotal) < Z) return RANS_ERR_TABLE;
-    long long lo = 2, hi = kTotal;
-    while (lo < hi) {
-      long long mid = (lo + hi) >> 1;
-      if (S(mid) >= Z) hi = mid; else lo = mid + 1;
+      sh.total = (unsigned long long)t;
+      sh.warp[0] = below;
     }
-    const long long t = lo;
-    const unsigned long long R = Z - S(t - 1);
+    __syncthreads();
+    t = (long long)sh.total;
+    below = sh.warp[0];
+    __syncthreads();
+    if (t == 0) {
+      // wider than the histogram: S(t) by block reductions, t by bisection
+      auto S = [&](long long tt) -> unsigned long long {
+        unsigned long long sacc = 0;
+        for (int i = threadIdx.x; i < n; i += kRowThreads) {
+          long long w = row[i + 1];
+          if (w > 1 && w <= tt) sacc += (unsigned long long)(w - 1);
+        }
+        return block_sum(sacc, sh);
+      };
+      if (S(kTotal) < Z) return RANS_ERR_TABLE;
+      long long lo = kHistMax + 1, hi = kTotal;
+      while (lo < hi) {
+        long long mid = (lo + hi) >> 1;
+        if (S(mid) >= Z) hi = mid; else lo = mid + 1;
+      }
+      t = lo;
+      below = S(t - 1);
+    }
+    const unsigned long long R = Z - below;
     const unsigned long long full = R / (unsigned long long)(t - 1);
     const unsigned long long part = R % (unsigned long long)(t - 1);
     unsigned long long rank_carry = 0;
@@ -171,7 +205,6 @@ __device__ int quantise_row(const PF &pf, int n, int32_t *row, BlockScratch &sh)
     unsigned long long w = i < n ? (unsigned long long)row[i + 1] : 0ull;
     unsigned long long tot;
     unsigned long long ex = block_excl_scan(w, sh, &tot) + run;
-    __syncthreads();
     if (i < n) row[i + 1] = (int32_t)(ex + w);
     run += tot;
   }
@@ -228,6 +261,7 @@ __global__ void __launch_bounds__(kRowThreads)
     gaussian_rows_kernel(const float *scales, double tail, int32_t *cdfs, int Lmax,
                          int32_t *lengths, int32_t *offsets) {
   __shared__ BlockScratch sh;
+  __shared__ unsigned int hist[kHistMax + 1];
   const int r = blockIdx.x;
   int32_t *row = cdfs + (size_t)r * (size_t)Lmax;
   int32_t c = 0;
@@ -236,7 +270,7 @@ __global__ void __launch_bounds__(kRowThreads)
   if (st == RANS_OK && len > Lmax) st = RANS_ERR_CAPACITY;
   if (st == RANS_OK) {
     GaussPmf pf{c, 2 * c + 1, (double)scales[r]};
-    st = quantise_row(pf, 2 * c + 2, row, sh);
+    st = quantise_row(pf, 2 * c + 2, row, sh, hist);
   }
   for (int j = (st == RANS_OK ? len : 0) + threadIdx.x; j < Lmax; j += kRowThreads) row[j] = 0;
   if (threadIdx.x == 0) {
@@ -249,6 +283,7 @@ __global__ void __launch_bounds__(kRowThreads)
     pmf_rows_kernel(const float *pmfs, int stride, const int32_t *pmf_lengths,
                     const float *tail, int32_t *cdfs, int Lmax, int32_t *lengths) {
   __shared__ BlockScratch sh;
+  __shared__ unsigned int hist[kHistMax + 1];
   const int r = blockIdx.x;
   int32_t *row = cdfs + (size_t)r * (size_t)Lmax;
   int n = pmf_lengths[r];
@@ -257,7 +292,7 @@ __global__ void __launch_bounds__(kRowThreads)
   else if (n + 2 > Lmax) st = RANS_ERR_CAPACITY;
   if (st == RANS_OK) {
     GivenPmf pf{pmfs + (size_t)r * (size_t)stride, n, tail[r]};
-    st = quantise_row(pf, n + 1, row, sh);
+    st = quantise_row(pf, n + 1, row, sh, hist);
   }
   for (int j = (st == RANS_OK ? n + 2 : 0) + threadIdx.x; j < Lmax; j += kRowThreads) row[j] = 0;
   if (threadIdx.x == 0) lengths[r] = st ? st : n + 2;
@@ -272,7 +307,7 @@ __global__ void pack_buckets_kernel(const int32_t *cdfs, int Lmax, const RowMeta
   const int r = blockIdx.x;
   const int32_t *row = cdfs + (size_t)r * (size_t)Lmax;
   const int len = lengths[r];
-  const uint32_t base = meta[r].bucket_base;
+  const uint32_t base = meta[r * kMetaCopies].bucket_base;
   if (threadIdx.x == 0 && (row[0] != 0 || row[len - 1] != (int32_t)kTotal))
     report(status, RANS_ERR_TABLE, r);
   for (int j = threadIdx.x; j < len - 1; j += blockDim.x) {
@@ -282,6 +317,56 @@ __global__ void pack_buckets_kernel(const int32_t *cdfs, int Lmax, const RowMeta
       continue;
     }
     buckets[base + j] = (uint32_t)(a & 0xffff) | ((uint32_t)(b - a - 1) << 16);
+  }
+}
+
+// Largest j in [0, nb) with row[j] <= v (row strictly increasing, row[0]=0).
+__device__ __forceinline__ int bucket_of(const int32_t *row, int nb, int v);
+
+// Rebuilds a prepared table set from new CDF rows with the same lengths:
+// block (x, r) fills slot chunk x of row r; block (0, r) also checks the
+// row's length against the layout, refreshes its offset and packs its
+// buckets.  Errors go to the blob's status word.
+__global__ void refresh_kernel(const int32_t *cdfs, int Lmax, const int32_t *lengths,
+                               const int32_t *offsets, RowMeta *meta, uint32_t *buckets,
+                               uint32_t *slots, int32_t *status) {
+  const int r = blockIdx.y;
+  const RowMeta m = meta[r * kMetaCopies];
+  const int len = lengths[r];
+  if (len != (int)m.maxv + 2) {
+    if (threadIdx.x == 0 && blockIdx.x == 0) report(status, RANS_ERR_TABLE, r);
+    return;
+  }
+  const int32_t *row = cdfs + (size_t)r * (size_t)Lmax;
+  const int nb = len - 1;
+  if (blockIdx.x == 0) {
+    if (threadIdx.x < kMetaCopies) meta[r * kMetaCopies + threadIdx.x].offset = offsets[r];
+    if (threadIdx.x == 0 && (row[0] != 0 || row[len - 1] != (int32_t)kTotal))
+      report(status, RANS_ERR_TABLE, r);
+    for (int j = threadIdx.x; j < nb; j += blockDim.x) {
+      const int32_t a = row[j], b = row[j + 1];
+      if (!(b > a) || a < 0 || b > (int32_t)kTotal) {
+        report(status, RANS_ERR_TABLE, r);
+        continue;
+      }
+      buckets[m.bucket_base + j] = (uint32_t)(a & 0xffff) | ((uint32_t)(b - a - 1) << 16);
+    }
+  }
+  const int shift = (int)slot_shift(m.slot);
+  const int nslots = 1 << (16 - shift);
+  const int w = 1 << shift;
+  for (int t = blockIdx.x * blockDim.x + threadIdx.x; t < nslots; t += gridDim.x * blockDim.x) {
+    const int a = t * w, b = a + w - 1;
+    const int lo = bucket_of(row, nb, a);
+    const int inside = bucket_of(row, nb, b) - lo;
+    uint32_t e1 = 255u, e2 = 255u;
+    if (inside >= 3) {
+      e2 = (uint32_t)(inside - 3);
+    } else {
+      if (inside >= 1) e1 = (uint32_t)(row[lo + 1] - a - 1);
+      if (inside == 2) e2 = (uint32_t)(row[lo + 2] - a - 1);
+    }
+    slots[slot_base(m.slot) + t] = (uint32_t)lo | (e1 << 16) | (e2 << 24);
   }
 }
 
@@ -298,7 +383,7 @@ __device__ __forceinline__ int bucket_of(const int32_t *row, int nb, int v) {
 __global__ void fill_slots_kernel(const int32_t *cdfs, int Lmax, const RowMeta *meta,
                                   const int32_t *lengths, uint32_t *slots) {
   const int r = blockIdx.y;
-  const RowMeta m = meta[r];
+  const RowMeta m = meta[r * kMetaCopies];
   const int shift = (int)slot_shift(m.slot);
   const int nslots = 1 << (16 - shift);
   const int t = blockIdx.x * blockDim.x + threadIdx.x;
@@ -349,12 +434,30 @@ int launch_pmf_rows(const float *pmfs, int K, int stride, const int32_t *pmf_len
   return cudaGetLastError() == cudaSuccess ? RANS_OK : RANS_ERR_CUDA;
 }
 
+int refresh_tables(const int32_t *cdfs, int K, int Lmax, const int32_t *lengths,
+                   const int32_t *offsets, const rans_tables &t, cudaStream_t st) {
+  if (K != t.K) return RANS_ERR_ARG;
+  char *b = reinterpret_cast<char *>(t.blob);
+  int32_t *status = reinterpret_cast<int32_t *>(b);
+  RowMeta *dmeta = reinterpret_cast<RowMeta *>(b + kHeaderBytes);
+  uint32_t *dbuckets = reinterpret_cast<uint32_t *>(b + kHeaderBytes + t.meta_bytes);
+  uint32_t *dslots =
+      reinterpret_cast<uint32_t *>(b + kHeaderBytes + t.meta_bytes + t.bucket_bytes);
+  // slot chunks of 256: the largest row has at most 2^14 slots
+  int64_t maxslots = 1;
+  while (maxslots * K < t.n_slots && maxslots < (1 << kMaxQ)) maxslots <<= 1;
+  dim3 grid((unsigned)((maxslots + 255) / 256), (unsigned)K);
+  refresh_kernel<<<grid, 256, 0, st>>>(cdfs, Lmax, lengths, offsets, dmeta, dbuckets, dslots,
+                                       status);
+  return cudaGetLastError() == cudaSuccess ? RANS_OK : RANS_ERR_CUDA;
+}
+
 uint64_t tables_bytes_bound(int K, int Lmax) {
   if (K <= 0 || Lmax < 2) return 0;
   const int64_t nb = (int64_t)Lmax - 1;
   int q = ceil_log2(nb);
   q = q < kMinQ ? kMinQ : (q > kMaxQ ? kMaxQ : q);
-  return (uint64_t)kHeaderBytes + pad16(16ull * K) + pad16(4ull * K * nb) +
+  return (uint64_t)kHeaderBytes + pad16(16ull * kMetaCopies * K) + pad16(4ull * K * nb) +
          pad16(4ull * K * (1ull << q));
 }
 
@@ -390,7 +493,7 @@ int prepare_tables(const int32_t *cdfs, int K, int Lmax, const int32_t *lengths,
   }
   if (nbuckets > (1ull << 31)) return RANS_ERR_ARG;
 
-  const uint32_t meta_bytes = pad16(16ull * K);
+  const uint32_t meta_bytes = pad16(16ull * kMetaCopies * K);
   const uint32_t bucket_bytes = pad16(4ull * nbuckets);
   int optin = 0;
   cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
@@ -433,8 +536,12 @@ int prepare_tables(const int32_t *cdfs, int K, int Lmax, const int32_t *lengths,
   uint32_t *dbuckets = reinterpret_cast<uint32_t *>(b + kHeaderBytes + meta_bytes);
   uint32_t *dslots = reinterpret_cast<uint32_t *>(b + kHeaderBytes + meta_bytes + bucket_bytes);
   if (cudaMemsetAsync(b, 0, kHeaderBytes, st) != cudaSuccess) return RANS_ERR_CUDA;
-  if (cudaMemcpyAsync(dmeta, meta.data(), sizeof(RowMeta) * K, cudaMemcpyHostToDevice, st) !=
-      cudaSuccess)
+  std::vector<RowMeta> meta8((size_t)K * kMetaCopies);
+  for (int r = 0; r < K; ++r)
+    for (int c = 0; c < kMetaCopies; ++c) meta8[(size_t)r * kMetaCopies + c] = meta[r];
+  if (cudaMemcpyAsync(dmeta, meta8.data(), sizeof(RowMeta) * meta8.size(),
+                      cudaMemcpyHostToDevice, st) != cudaSuccess ||
+      cudaStreamSynchronize(st) != cudaSuccess)
     return RANS_ERR_CUDA;
   pack_buckets_kernel<<<K, 256, 0, st>>>(cdfs, Lmax, dmeta, lengths, dbuckets, status);
   int maxslots = 0;

@@ -321,3 +321,38 @@ def test_encoder_reports_bad_index_and_capacity():
     st = rb.rans_encode_with_indexes(sym, idx, sym.numel(), tables, ch, ws.out, ws.offsets,
                                      ws.enc[:1 << 20])
     assert st == rb.ERR_CAPACITY
+
+
+def test_table_refresh_matches_fresh_prepare():
+    """A prepared table set refreshed from new rows of the same lengths codes
+    exactly like one prepared from those rows."""
+    w = WL.z_latent()
+    w["W"] = 32
+    c, l, o = oracle_tables(w)
+    tables = tables_from_numpy(c, l, o)
+    # the same pmf shapes flattened a little: same lengths, other quantised rows
+    w2 = dict(w)
+    pm = np.asarray(w["pmfs"], np.float64)
+    lens = np.asarray(w["pmf_lengths"])
+    flat = np.zeros_like(pm)
+    for r in range(pm.shape[0]):
+        flat[r, :lens[r]] = 1.0 / lens[r]
+    w2["pmfs"] = (0.97 * pm + 0.03 * flat).astype(np.float32)
+    w2["offsets"] = (np.asarray(w["offsets"]) - 1).astype(np.int32)
+    w2["symbols"] = (np.asarray(w["symbols"]) - 1).astype(np.int32)
+    c2, l2, o2 = oracle_tables(w2)
+    assert np.array_equal(l2, l) and not np.array_equal(c2, c)
+    dc2 = torch.from_numpy(np.ascontiguousarray(c2)).cuda()
+    dl2 = torch.from_numpy(l2).cuda()
+    do2 = torch.from_numpy(o2).cuda()
+    rb.check(rb.rans_tables_refresh(dc2, dl2, do2, tables))
+    assert rb.rans_get_status(tables.blob) == rb.OK
+    data, offs, dec, _, _ = gpu_encode_decode(w2, tables)
+    want, woffs = oracle_encode(w2, c2, l2, o2)
+    assert offs.tolist() == woffs.tolist() and np.array_equal(data, want)
+    assert np.array_equal(dec, np.asarray(w2["symbols"]).reshape(-1))
+    # a row of another length is refused on the device
+    bad_l = dl2.clone()
+    bad_l[3] += 2
+    rb.check(rb.rans_tables_refresh(dc2, bad_l, do2, tables))
+    assert rb.rans_get_status(tables.blob) == rb.ERR_TABLE
