@@ -108,7 +108,9 @@ typedef struct rans_chunking {
 /*
  * A prepared table set, filled by rans_tables_prepare.  `blob` is the
  * caller's device buffer; the other fields describe its layout and are read
- * by the encoder and decoder.  One table set serves both directions and every
+ * by the encoder and decoder.  The blob holds per-row metadata, every
+ * bucket's (start, width) in 32 bits for the encoder, the CDF entries as
+ * 16-bit starts for the decoder, and the decoder's lookup slots.  One table set serves both directions and every
  * chunking.  Treat the fields as opaque.
  */
 typedef struct rans_tables {
@@ -118,9 +120,9 @@ typedef struct rans_tables {
     int32_t max_buckets;    /* longest row's bucket count (cdf_length - 1) */
     int64_t n_buckets;      /* all rows' buckets */
     int64_t n_slots;        /* decode lookup slots */
-    uint32_t meta_bytes, bucket_bytes, slot_bytes;  /* section sizes (16-B padded) */
+    uint32_t meta_bytes, bucket_bytes, start_bytes, slot_bytes;  /* sections (16-B padded) */
     int32_t enc_in_smem;    /* 1: encode stages meta + buckets in shared memory */
-    int32_t dec_in_smem;    /* 1: decode stages all three sections */
+    int32_t dec_in_smem;    /* 1: decode stages meta + starts + slots */
     int32_t device;         /* CUDA device the blob lives on */
 } rans_tables;
 

@@ -48,7 +48,8 @@ class rans_tables(ctypes.Structure):
                 ("K", ctypes.c_int32), ("max_buckets", ctypes.c_int32),
                 ("n_buckets", ctypes.c_int64), ("n_slots", ctypes.c_int64),
                 ("meta_bytes", ctypes.c_uint32), ("bucket_bytes", ctypes.c_uint32),
-                ("slot_bytes", ctypes.c_uint32), ("enc_in_smem", ctypes.c_int32),
+                ("start_bytes", ctypes.c_uint32), ("slot_bytes", ctypes.c_uint32),
+                ("enc_in_smem", ctypes.c_int32),
                 ("dec_in_smem", ctypes.c_int32), ("device", ctypes.c_int32)]
 
 

@@ -20,8 +20,9 @@
 //    depends on what it reads ("torch_ans 0.3.0", Performance Tuning, GPU
 //    item 5: the bypass phase is sequential across the lanes and skipped by a
 //    group ballot).
-//  Latency: row indexes are loaded kRing groups ahead into registers; each
-//  stream's words are bulk prefetched into L2 when the warp starts it.
+//  Latency: row indexes stream through a per-warp shared-memory ring filled
+//  with cp.async kStage - 1 groups ahead; each stream's words are bulk
+//  prefetched into L2 when the warp starts it.
 //  Tables are staged into shared memory with bulk copies when they fit.
 #include "rans_common.cuh"
 #include "rans_internal.h"
@@ -29,9 +30,8 @@
 namespace rb {
 namespace {
 
-constexpr int kDecMaxThreads32 = 768;
+constexpr int kDecMaxThreads32 = kDecMaxWarps * 32;
 constexpr int kDecThreads1 = 128;
-constexpr int kRing = 4;
 
 struct DecCtx {
   const uint8_t *in;
@@ -39,7 +39,7 @@ struct DecCtx {
   const uint64_t *offs;
   const int32_t *idx;
   int32_t K;
-  uint32_t meta_bytes, bucket_bytes, slot_bytes;
+  uint32_t meta_bytes, bucket_bytes, start_bytes, slot_bytes;
   const char *blob;
   Geom g;
   void *out;
@@ -155,8 +155,11 @@ struct WarpDec {
   bool bad;
 };
 
+// Window word i, read from a clamped address (nw >= 64 always): reading past
+// the stream end returns its last word instead, so no select waits on the
+// load; a decoder that consumes past the end is caught by the final check.
 __device__ __forceinline__ uint32_t word_at(const uint32_t *words, uint64_t nw, uint64_t i) {
-  return i < nw ? __ldg(words + i) : 0u;
+  return __ldg(words + (i < nw ? i : nw - 1));
 }
 
 __device__ __forceinline__ void load_window(WarpDec &st, const uint32_t *words, uint64_t nw) {
@@ -169,7 +172,7 @@ __device__ __forceinline__ void load_window(WarpDec &st, const uint32_t *words, 
 // One group of 32 symbols: lookup, state update, refill, output.  m is the
 // group's row metadata, loaded one group ahead.
 template <typename SymT, bool FULL>
-__device__ __forceinline__ void dec_group(WarpDec &st, const RowMeta &m, const uint32_t *buckets,
+__device__ __forceinline__ void dec_group(WarpDec &st, const RowMeta &m, const uint16_t *starts,
                                           const uint32_t *slots, bool active, SymT *dst,
                                           const uint32_t *words, uint64_t nw) {
   const int lane = threadIdx.x & 31;
@@ -186,14 +189,15 @@ __device__ __forceinline__ void dec_group(WarpDec &st, const RowMeta &m, const u
       uint32_t lo = se & 0xffffu, hi = lo + e2 + 3u;
       while (lo < hi) {
         const uint32_t mid = (lo + hi + 1) >> 1;
-        if (bucket_start(buckets[m.bucket_base + mid]) <= cum) lo = mid; else hi = mid - 1;
+        if (starts[m.bucket_base + mid] <= cum) lo = mid; else hi = mid - 1;
       }
       sym = lo;
     }
   }
-  const uint32_t e = buckets[m.bucket_base + sym];
+  const uint32_t start = starts[m.bucket_base + sym];
+  const uint32_t freq = width_of(start, starts[m.bucket_base + sym + 1]);
   uint64_t x = st.x;
-  if (active) x = (uint64_t)bucket_freq(e) * (x >> kPrec) + (cum - bucket_start(e));
+  if (active) x = (uint64_t)freq * (x >> kPrec) + (cum - start);
   const bool esc = active && sym == m.maxv;
   int32_t val = (int32_t)sym + m.offset;
   if (!__any_sync(kFull, esc)) {
@@ -226,9 +230,9 @@ __device__ __forceinline__ void dec_group(WarpDec &st, const RowMeta &m, const u
 
 template <typename SymT, bool IB0, bool WIDE>
 __device__ __forceinline__ void decode_stream_w32(const DecCtx &c, const StreamDesc &d,
-                                                  const RowMeta *meta, const uint32_t *buckets,
-                                                  const uint32_t *slots, int64_t s,
-                                                  const uint32_t *words, uint64_t nw) {
+                                                  const RowMeta *meta, const uint16_t *buckets,
+                                                  const uint32_t *slots, uint32_t *stg,
+                                                  int64_t s, const uint32_t *words, uint64_t nw) {
   const int lane = threadIdx.x & 31;
   const int32_t n = (int32_t)d.n;
   const int32_t G = (n + 31) >> 5;
@@ -237,9 +241,6 @@ __device__ __forceinline__ void decode_stream_w32(const DecCtx &c, const StreamD
   const int32_t *idx_s = c.idx + (IB0 ? base : 0);
   SymT *out_s = reinterpret_cast<SymT *>(c.out) + base;
   const uint32_t kmax = (uint32_t)c.K - 1u;
-  auto load_idx = [&](int32_t rel) -> int32_t {
-    return IB0 ? __ldg(idx_s + rel) : __ldg(c.idx + ((base + rel) >> ib));
-  };
 
   WarpDec st;
   st.x = (uint64_t)__ldg(words + 2 * lane) | ((uint64_t)__ldg(words + 2 * lane + 1) << 32);
@@ -249,47 +250,42 @@ __device__ __forceinline__ void decode_stream_w32(const DecCtx &c, const StreamD
   st.rmax = 0;
   st.bad = false;
 
-  Stepper<WIDE> pl;
+  // Group g's row indexes land in stage slot g mod kStage, copied kStage - 1
+  // groups ahead; a lane past the stream end copies element 0 (ignored).
+  Stepper<WIDE> pl;  // next group to copy
   pl.init(d.t, lane);
-  int32_t rrel[kRing], ridx[kRing];
-#pragma unroll
-  for (int u = 0; u < kRing; ++u) {
-    rrel[u] = pl.rel;
-    ridx[u] = lane < n - u * 32 ? load_idx(pl.rel) : 0;
-    pl.fwd(32);
-  }
-  auto meta_of = [&](int32_t r) -> RowMeta {
-    st.rmax = max(st.rmax, (uint32_t)r);
-    return row_meta(meta, min((uint32_t)r, kmax));
-  };
-  RowMeta m = meta_of(ridx[0]);
-  // Group g uses ring slot g mod kRing; its slot is refilled with group
-  // g + kRing, and the next group's metadata is loaded one group ahead.
-  auto step = [&](int u, int32_t g, bool full) {
-    const int32_t rel = rrel[u];
-    const RowMeta mn = meta_of(ridx[(u + 1) % kRing]);
-    if (g + kRing < G) {
-      rrel[u] = pl.rel;
-      ridx[u] = lane < n - (g + kRing) * 32 ? load_idx(pl.rel) : 0;
+  Stepper<WIDE> pc = pl;  // group being decoded (output position)
+  auto issue = [&](int32_t gi) {
+    if (gi < G) {
+      const int32_t rel = lane < n - gi * 32 ? pl.rel : 0;
+      cp_async4(stg + (gi & (kStage - 1)) * 32 + lane,
+                IB0 ? idx_s + rel : c.idx + ((base + rel) >> ib));
       pl.fwd(32);
     }
-    if (full)
-      dec_group<SymT, true>(st, m, buckets, slots, true, out_s + rel, words, nw);
-    else
-      dec_group<SymT, false>(st, m, buckets, slots, lane < n - g * 32, out_s + rel, words, nw);
-    m = mn;
+    cp_async_commit();
   };
-  // every group but the last is full
-  int32_t g0 = 0;
-  for (; g0 + kRing < G; g0 += kRing) {
+  auto meta_of = [&](uint32_t r) -> RowMeta {
+    st.rmax = max(st.rmax, r);
+    return row_meta(meta, min(r, kmax));
+  };
 #pragma unroll
-    for (int u = 0; u < kRing; ++u) step(u, g0 + u, true);
+  for (int32_t u = 0; u < kStage - 1; ++u) issue(u);
+  cp_async_wait<kStage - 2>();
+  RowMeta m = meta_of(stg[lane]);
+  for (int32_t g = 0; g < G; ++g) {
+    issue(g + kStage - 1);
+    cp_async_wait<kStage - 2>();  // groups up to g + 1 have landed
+    // (after the last group the slot may hold another stream's data: unused)
+    const RowMeta mn = meta_of(g + 1 < G ? stg[((g + 1) & (kStage - 1)) * 32 + lane] : 0u);
+    if (g + 1 < G)
+      dec_group<SymT, true>(st, m, buckets, slots, true, out_s + pc.rel, words, nw);
+    else
+      dec_group<SymT, false>(st, m, buckets, slots, lane < n - g * 32, out_s + pc.rel, words,
+                             nw);
+    pc.fwd(32);
+    m = mn;
   }
-#pragma unroll
-  for (int u = 0; u < kRing; ++u) {
-    if (g0 + u >= G) break;
-    step(u, g0 + u, false);
-  }
+  cp_async_wait<0>();
   if (__any_sync(kFull, st.rmax > kmax)) {
     if (lane == 0) report(c.status, RANS_ERR_INDEX, s);
     return;
@@ -300,8 +296,9 @@ __device__ __forceinline__ void decode_stream_w32(const DecCtx &c, const StreamD
 
 template <typename SymT, bool IB0>
 __device__ __forceinline__ void decode_stream_w32_entry(const DecCtx &c, const RowMeta *meta,
-                                                        const uint32_t *buckets,
-                                                        const uint32_t *slots, int64_t s) {
+                                                        const uint16_t *buckets,
+                                                        const uint32_t *slots, uint32_t *stg,
+                                                        int64_t s) {
   const int lane = threadIdx.x & 31;
   const StreamDesc d = stream_desc(c.g, s);
   const uint32_t *words = nullptr;
@@ -314,14 +311,20 @@ __device__ __forceinline__ void decode_stream_w32_entry(const DecCtx &c, const R
     bulk_prefetch_l2(reinterpret_cast<const char *>(c.in),
                      reinterpret_cast<const char *>(c.in) + c.in_bytes,
                      reinterpret_cast<const char *>(words + 64), 4 * (nw - 64));
+  if (d.n == 0) {  // only the 32 initial states, each 2^31
+    const uint64_t x =
+        (uint64_t)__ldg(words + 2 * lane) | ((uint64_t)__ldg(words + 2 * lane + 1) << 32);
+    if (!__all_sync(kFull, x == kL && nw == 64) && lane == 0) report(c.status, RANS_ERR_CORRUPT, s);
+    return;
+  }
   if (d.t.ww >= 32)
-    decode_stream_w32<SymT, IB0, true>(c, d, meta, buckets, slots, s, words, nw);
+    decode_stream_w32<SymT, IB0, true>(c, d, meta, buckets, slots, stg, s, words, nw);
   else
-    decode_stream_w32<SymT, IB0, false>(c, d, meta, buckets, slots, s, words, nw);
+    decode_stream_w32<SymT, IB0, false>(c, d, meta, buckets, slots, stg, s, words, nw);
 }
 
 template <typename SymT>
-__device__ void decode_stream_w1(const DecCtx &c, const RowMeta *meta, const uint32_t *buckets,
+__device__ void decode_stream_w1(const DecCtx &c, const RowMeta *meta, const uint16_t *buckets,
                                  const uint32_t *slots, int64_t s) {
   const StreamDesc d = stream_desc(c.g, s);
   const uint32_t *words = nullptr;
@@ -376,12 +379,13 @@ __device__ void decode_stream_w1(const DecCtx &c, const RowMeta *meta, const uin
       uint32_t lo = se & 0xffffu, hi = lo + (se >> 24) + 3u;
       while (lo < hi) {
         const uint32_t mid = (lo + hi + 1) >> 1;
-        if (bucket_start(buckets[m.bucket_base + mid]) <= cum) lo = mid; else hi = mid - 1;
+        if (buckets[m.bucket_base + mid] <= cum) lo = mid; else hi = mid - 1;
       }
       sym = lo;
     }
-    const uint32_t e = buckets[m.bucket_base + sym];
-    x = (uint64_t)bucket_freq(e) * (x >> kPrec) + cum - bucket_start(e);
+    const uint32_t start = buckets[m.bucket_base + sym];
+    const uint32_t freq = width_of(start, buckets[m.bucket_base + sym + 1]);
+    x = (uint64_t)freq * (x >> kPrec) + cum - start;
     if (x < kL) x = (x << 32) | rd();
     int64_t val = (int64_t)sym;
     if (sym == m.maxv) {
@@ -416,23 +420,31 @@ __global__ void __launch_bounds__(W == 32 ? kDecMaxThreads32 : kDecThreads1)
     decode_kernel(DecCtx c) {
   extern __shared__ __align__(16) unsigned char smem[];
   __shared__ uint64_t bar;
-  const unsigned char *tb;
+  const RowMeta *meta;
+  const uint16_t *buckets;  // 16-bit starts
+  const uint32_t *slots;
+  const char *gb = c.blob + kHeaderBytes;
   if (SMEM) {
-    if (!stage_to_smem(smem, c.blob + kHeaderBytes, c.meta_bytes + c.bucket_bytes + c.slot_bytes,
-                       &bar, c.status))
+    // [meta][starts][slots] in shared memory, from two ranges of the blob
+    if (!stage_to_smem(smem, gb, c.meta_bytes, &bar, c.status, smem + c.meta_bytes,
+                       gb + c.meta_bytes + c.bucket_bytes, c.start_bytes + c.slot_bytes))
       return;
-    tb = smem;
+    meta = reinterpret_cast<const RowMeta *>(smem);
+    buckets = reinterpret_cast<const uint16_t *>(smem + c.meta_bytes);
+    slots = reinterpret_cast<const uint32_t *>(smem + c.meta_bytes + c.start_bytes);
   } else {
-    tb = reinterpret_cast<const unsigned char *>(c.blob + kHeaderBytes);
+    meta = reinterpret_cast<const RowMeta *>(gb);
+    buckets = reinterpret_cast<const uint16_t *>(gb + c.meta_bytes + c.bucket_bytes);
+    slots = reinterpret_cast<const uint32_t *>(gb + c.meta_bytes + c.bucket_bytes + c.start_bytes);
   }
-  const RowMeta *meta = reinterpret_cast<const RowMeta *>(tb);
-  const uint32_t *buckets = reinterpret_cast<const uint32_t *>(tb + c.meta_bytes);
-  const uint32_t *slots = reinterpret_cast<const uint32_t *>(tb + c.meta_bytes + c.bucket_bytes);
   if (W == 32) {
     const int warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+    uint32_t *stg = reinterpret_cast<uint32_t *>(
+                        smem + (SMEM ? c.meta_bytes + c.start_bytes + c.slot_bytes : 0)) +
+                    warp * kStage * 32;
     for (int64_t k = blockIdx.x + (int64_t)gridDim.x * warp; k < c.g.S;
          k += (int64_t)gridDim.x * nw)
-      decode_stream_w32_entry<SymT, IB0>(c, meta, buckets, slots, stream_of(c.g, k));
+      decode_stream_w32_entry<SymT, IB0>(c, meta, buckets, slots, stg, stream_of(c.g, k));
   } else {
     for (int64_t k = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; k < c.g.S;
          k += (int64_t)gridDim.x * blockDim.x)
@@ -443,28 +455,31 @@ __global__ void __launch_bounds__(W == 32 ? kDecMaxThreads32 : kDecThreads1)
 template <int W, typename SymT, bool SMEM, bool IB0>
 int launch_decode_t(const DecCtx &c, cudaStream_t st) {
   auto kern = decode_kernel<W, SymT, SMEM, IB0>;
-  const uint32_t smem = SMEM ? c.meta_bytes + c.bucket_bytes + c.slot_bytes : 0;
+  const uint32_t tab = SMEM ? c.meta_bytes + c.start_bytes + c.slot_bytes : 0;
+  const uint32_t per_warp = W == 32 ? kStage * 32 * 4 : 0;
   int dev = 0;
   cudaGetDevice(&dev);
-  if (SMEM && cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                   (int)smem) != cudaSuccess)
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           (int)(tab + kDecStageBytes)) != cudaSuccess)
     return RANS_ERR_CUDA;
   const int sms = num_sms(dev);
   int threads, blocks;
+  uint32_t smem = tab;
   if (W == 32) {
     // One or a few CTAs per SM (bounded by the staged tables); enough warps
     // for one stream each when possible.
     int per_sm = 0;
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, 32, smem) != cudaSuccess ||
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, 32, tab + per_warp) !=
+            cudaSuccess ||
         per_sm < 1)
       return RANS_ERR_CUDA;
     int64_t nblk = (int64_t)sms * per_sm;
     if (nblk > c.g.S) nblk = c.g.S < 1 ? 1 : c.g.S;
     int64_t warps = (c.g.S + nblk - 1) / nblk;
-    const int max_warps = kDecMaxThreads32 / 32;
-    if (warps > max_warps) warps = max_warps;
+    if (warps > kDecMaxWarps) warps = kDecMaxWarps;
     if (warps < 1) warps = 1;
     threads = (int)warps * 32;
+    smem = tab + (uint32_t)warps * per_warp;
     int fit = 0;
     if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&fit, kern, threads, smem) != cudaSuccess ||
         fit < 1)
@@ -516,6 +531,7 @@ int launch_decode(const uint8_t *in, uint64_t in_bytes, const uint64_t *offsets,
   c.K = t.K;
   c.meta_bytes = t.meta_bytes;
   c.bucket_bytes = t.bucket_bytes;
+  c.start_bytes = t.start_bytes;
   c.slot_bytes = t.slot_bytes;
   c.blob = reinterpret_cast<const char *>(t.blob);
   c.g = g;

@@ -23,7 +23,7 @@
 namespace rb {
 namespace {
 
-constexpr int kEncThreads32 = 1024;
+constexpr int kEncThreads32 = kEncMaxWarps * 32;
 constexpr int kEncThreads1 = 128;
 
 struct EncCtx {
@@ -96,7 +96,6 @@ __device__ __forceinline__ uint32_t symbol_ops(uint64_t &x, uint32_t start, uint
   return k;
 }
 
-constexpr int kRing = 4;
 
 // A group holding an escape, off the fast path: every lane counts the words
 // its ops push, a suffix sum over lanes places each lane's block (lanes > l
@@ -149,10 +148,9 @@ __device__ __forceinline__ void enc_group(WarpEnc &st, const RowMeta &m, const u
     // x >= freq * 2^47  <=>  high word of x >= freq * 2^15
     const bool need = active && (uint32_t)(x >> 32) >= (freq << 15);
     const uint32_t bm = __ballot_sync(kFull, need);
-    if (need) {
-      end[-1 - (int64_t)(st.cursor + __popc(bm & above))] = (uint32_t)x;
-      x >>= 32;
-    }
+    const uint32_t lo = (uint32_t)x;
+    if (need) end[-1 - (int64_t)(st.cursor + __popc(bm & above))] = lo;
+    x = need ? (x >> 32) : x;
     st.cursor += __popc(bm);
     if (active) x = enc_sym_step(x, start, freq, rcp);
   } else {
@@ -170,7 +168,8 @@ __device__ __forceinline__ void enc_group(WarpEnc &st, const RowMeta &m, const u
 template <typename SymT, bool IB0, bool WIDE>
 __device__ __forceinline__ void encode_stream_w32(const EncCtx &c, const StreamDesc &d,
                                                   const RowMeta *meta, const uint32_t *buckets,
-                                                  int64_t s) {
+                                                  uint32_t *stg, int64_t s) {
+  constexpr bool kStageSym = sizeof(SymT) == 4;
   const int lane = threadIdx.x & 31;
   uint32_t *end = reinterpret_cast<uint32_t *>(c.scratch + slot_end(c.g, d, s));
   const int32_t n = (int32_t)d.n;
@@ -180,60 +179,65 @@ __device__ __forceinline__ void encode_stream_w32(const EncCtx &c, const StreamD
   const int32_t *idx_s = c.idx + (IB0 ? base : 0);
   const SymT *sym_s = reinterpret_cast<const SymT *>(c.sym) + base;
   const uint32_t kmax = (uint32_t)c.K - 1u;
-  auto load = [&](int32_t rel, int32_t &sv, int32_t &r) {
-    sv = SymIO<SymT>::load(sym_s, rel);
-    r = IB0 ? __ldg(idx_s + rel) : __ldg(c.idx + ((base + rel) >> ib));
-  };
   const uint32_t above = 0xfffffffeu << lane;   // lanes > this lane
+  uint32_t *stg_idx = stg;
+  uint32_t *stg_sym = stg + kStage * 32;
   WarpEnc st;
   st.x = kL;
   st.cursor = 0;
   st.rmax = 0;
   st.range_err = false;
 
-  // Groups are coded G-1 down to 0; the k-th coded group (G-1-k) uses ring
-  // slot k mod kRing, which is then refilled with group G-1-(k+kRing).
+  // The k-th coded group (group G-1-k) lands in stage slot k mod kStage,
+  // copied kStage - 1 groups ahead; a lane without an element there copies
+  // element 0 (ignored).
   Stepper<WIDE> pl;
-  pl.init(d.t, (G > 0 ? G - 1 : 0) * 32 + lane);
-  int32_t rsym[kRing], ridx[kRing];
-#pragma unroll
-  for (int u = 0; u < kRing; ++u) {
-    rsym[u] = 0;
-    ridx[u] = 0;
-    if (u < G && lane < n - (G - 1 - u) * 32) load(pl.rel, rsym[u], ridx[u]);
-    if (u + 1 < G) pl.back(32);
-  }
-  auto meta_of = [&](int32_t r) -> RowMeta {
-    st.rmax = max(st.rmax, (uint32_t)r);
-    return row_meta(meta, min((uint32_t)r, kmax));
-  };
-  RowMeta m = meta_of(ridx[0]);
-  auto step = [&](int u, int32_t k, bool full) {
-    const int32_t g = G - 1 - k;
-    const int32_t sv = rsym[u];
-    const RowMeta mn = meta_of(ridx[(u + 1) % kRing]);
-    if (g - kRing >= 0) {     // every lane of an earlier group is active
-      load(pl.rel, rsym[u], ridx[u]);
-      if (g - kRing > 0) pl.back(32);
+  pl.init(d.t, (G - 1) * 32 + lane);
+  Stepper<WIDE> pn = pl;  // narrow symbols: next group's position
+  auto issue = [&](int32_t ki) {
+    if (ki < G) {
+      const int32_t g = G - 1 - ki;
+      const int32_t rel = lane < n - g * 32 ? pl.rel : 0;
+      const int slot = (ki & (kStage - 1)) * 32 + lane;
+      cp_async4(stg_idx + slot, IB0 ? idx_s + rel : c.idx + ((base + rel) >> ib));
+      if (kStageSym) cp_async4(stg_sym + slot, sym_s + rel);
+      if (g > 0) pl.back(32);
     }
-    if (full)
+    cp_async_commit();
+  };
+  auto meta_of = [&](uint32_t r) -> RowMeta {
+    st.rmax = max(st.rmax, r);
+    return row_meta(meta, min(r, kmax));
+  };
+#pragma unroll
+  for (int32_t u = 0; u < kStage - 1; ++u) issue(u);
+  cp_async_wait<kStage - 2>();
+  RowMeta m = meta_of(stg_idx[lane]);
+  int32_t sv_next = 0;
+  if (!kStageSym) sv_next = SymIO<SymT>::load(sym_s, lane < n - (G - 1) * 32 ? pn.rel : 0);
+  for (int32_t k = 0; k < G; ++k) {
+    issue(k + kStage - 1);
+    cp_async_wait<kStage - 2>();  // coded groups up to k + 1 have landed
+    const int slot = (k & (kStage - 1)) * 32 + lane;
+    int32_t sv;
+    if (kStageSym) {
+      sv = (int32_t)stg_sym[slot];
+    } else {
+      sv = sv_next;
+      if (k + 1 < G) {
+        pn.back(32);
+        sv_next = SymIO<SymT>::load(sym_s, pn.rel);
+      }
+    }
+    // (after the last group the slot may hold another stream's data: unused)
+    const RowMeta mn = meta_of(k + 1 < G ? stg_idx[((k + 1) & (kStage - 1)) * 32 + lane] : 0u);
+    if (k > 0)
       enc_group<true>(st, m, buckets, sv, true, above, end);
     else
-      enc_group<false>(st, m, buckets, sv, lane < n - g * 32, above, end);
+      enc_group<false>(st, m, buckets, sv, lane < n - (G - 1) * 32, above, end);
     m = mn;
-  };
-  // the last group (coded first) may be partial; every other group is full
-  if (G > 0) step(0, 0, false);
-  int32_t k0 = 1;
-  for (; k0 + kRing <= G; k0 += kRing) {
-#pragma unroll
-    for (int u = 0; u < kRing; ++u) step((u + 1) % kRing, k0 + u, true);
   }
-#pragma unroll
-  for (int u = 0; u < kRing; ++u) {
-    if (k0 + u >= G) break;
-    step((u + 1) % kRing, k0 + u, true);
-  }
+  cp_async_wait<0>();
   if (__any_sync(kFull, st.rmax > kmax)) {
     if (lane == 0) report(c.status, RANS_ERR_INDEX, s);
     return;
@@ -251,16 +255,25 @@ __device__ __forceinline__ void encode_stream_w32(const EncCtx &c, const StreamD
 
 template <typename SymT, bool IB0>
 __device__ __forceinline__ void encode_stream_w32_entry(const EncCtx &c, const RowMeta *meta,
-                                                        const uint32_t *buckets, int64_t s) {
+                                                        const uint32_t *buckets, uint32_t *stg,
+                                                        int64_t s) {
   const StreamDesc d = stream_desc(c.g, s);
   if (!d.ok) {
     if ((threadIdx.x & 31) == 0) report(c.status, RANS_ERR_ARG, s);
     return;
   }
+  if (d.n == 0) {  // flush the 32 initial states only
+    const int lane = threadIdx.x & 31;
+    uint32_t *end = reinterpret_cast<uint32_t *>(c.scratch + slot_end(c.g, d, s));
+    end[-1 - 2 * (31 - lane)] = (uint32_t)(kL >> 32);
+    end[-2 - 2 * (31 - lane)] = (uint32_t)kL;
+    if (lane == 0) c.lens[s] = 256;
+    return;
+  }
   if (d.t.ww >= 32)
-    encode_stream_w32<SymT, IB0, true>(c, d, meta, buckets, s);
+    encode_stream_w32<SymT, IB0, true>(c, d, meta, buckets, stg, s);
   else
-    encode_stream_w32<SymT, IB0, false>(c, d, meta, buckets, s);
+    encode_stream_w32<SymT, IB0, false>(c, d, meta, buckets, stg, s);
 }
 
 template <typename SymT>
@@ -337,9 +350,11 @@ __global__ void __launch_bounds__(W == 32 ? kEncThreads32 : kEncThreads1)
   }
   if (W == 32) {
     const int warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+    uint32_t *stg = reinterpret_cast<uint32_t *>(smem + (SMEM ? c.meta_bytes + c.bucket_bytes : 0)) +
+                    warp * kStage * 32 * 2;
     for (int64_t k = blockIdx.x + (int64_t)gridDim.x * warp; k < c.g.S;
          k += (int64_t)gridDim.x * nw)
-      encode_stream_w32_entry<SymT, IB0>(c, meta, buckets, stream_of(c.g, k));
+      encode_stream_w32_entry<SymT, IB0>(c, meta, buckets, stg, stream_of(c.g, k));
   } else {
     for (int64_t k = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; k < c.g.S;
          k += (int64_t)gridDim.x * blockDim.x)
@@ -427,25 +442,52 @@ __global__ void debug_divide_kernel(const uint64_t *x, const uint32_t *f, int64_
 
 template <int W, typename SymT, bool SMEM, bool IB0>
 int launch_encode_t(const EncCtx &c, cudaStream_t st) {
-  const int dev_threads = W == 32 ? kEncThreads32 : kEncThreads1;
   auto kern = encode_kernel<W, SymT, SMEM, IB0>;
-  const uint32_t smem = SMEM ? c.meta_bytes + c.bucket_bytes : 0;
+  const uint32_t tab = SMEM ? c.meta_bytes + c.bucket_bytes : 0;
+  const uint32_t per_warp = W == 32 ? kStage * 32 * 4 * 2 : 0;
+  uint32_t smem = tab;
   int dev = 0;
   cudaGetDevice(&dev);
-  if (SMEM && cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                   (int)smem) != cudaSuccess)
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           (int)(tab + kEncStageBytes)) != cudaSuccess)
     return RANS_ERR_CUDA;
-  int per_sm = 0;
-  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, dev_threads, smem) !=
-          cudaSuccess ||
-      per_sm < 1)
-    return RANS_ERR_CUDA;
-  const int64_t units_per_block = W == 32 ? dev_threads / 32 : dev_threads;
-  int64_t blocks = (c.g.S + units_per_block - 1) / units_per_block;
-  const int64_t cap = (int64_t)per_sm * num_sms(dev);
-  if (blocks > cap) blocks = cap;
+  const int sms = num_sms(dev);
+  int threads;
+  int64_t blocks;
+  if (W == 32) {
+    // Spread the streams over every SM: as many CTAs as fit per SM, each with
+    // enough warps for one stream per warp when possible.
+    int per_sm = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, 32, tab + per_warp) !=
+            cudaSuccess ||
+        per_sm < 1)
+      return RANS_ERR_CUDA;
+    int64_t nblk = (int64_t)sms * per_sm;
+    if (nblk > c.g.S) nblk = c.g.S < 1 ? 1 : c.g.S;
+    int64_t warps = (c.g.S + nblk - 1) / nblk;
+    if (warps > kEncMaxWarps) warps = kEncMaxWarps;
+    if (warps < 1) warps = 1;
+    threads = (int)warps * 32;
+    smem = tab + (uint32_t)warps * per_warp;
+    int fit = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&fit, kern, threads, smem) != cudaSuccess ||
+        fit < 1)
+      return RANS_ERR_CUDA;
+    const int64_t need = (c.g.S + warps - 1) / warps;
+    const int64_t cap = (int64_t)fit * sms;
+    blocks = need < cap ? need : cap;
+  } else {
+    threads = kEncThreads1;
+    int fit = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&fit, kern, threads, smem) != cudaSuccess ||
+        fit < 1)
+      return RANS_ERR_CUDA;
+    const int64_t need = (c.g.S + threads - 1) / threads;
+    const int64_t cap = (int64_t)fit * sms;
+    blocks = need < cap ? need : cap;
+  }
   if (blocks < 1) blocks = 1;
-  kern<<<(unsigned)blocks, dev_threads, smem, st>>>(c);
+  kern<<<(unsigned)blocks, threads, smem, st>>>(c);
   return cudaGetLastError() == cudaSuccess ? RANS_OK : RANS_ERR_CUDA;
 }
 

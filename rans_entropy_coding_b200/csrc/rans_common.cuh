@@ -22,8 +22,10 @@ constexpr uint32_t kBypassMax = 15;
 constexpr unsigned kFull = 0xffffffffu;
 
 // ------------------------------------------------------------ table blob --
-// [header 256 B][RowMeta K x 8][bucket words][slot words], sections 16-B
-// padded.  Each row's metadata is stored 8 times side by side (128 bytes per
+// [header 256 B][RowMeta K x 8][bucket words][16-bit starts][slot words],
+// sections 16-B padded.  The starts are the CDF entries mod 2^16 at the same
+// indexes as the bucket words, plus one trailing 0: bucket j of a row ends at
+// start[base + j + 1] (the next row's leading 0 stands for 65536).  Each row's metadata is stored 8 times side by side (128 bytes per
 // row): lane l of a warp reads copy l mod 8, so the 8 lanes served by one
 // shared-memory wavefront of 16-byte loads always hit 8 different bank groups.
 // A bucket word packs start | (width - 1) << 16.
@@ -53,11 +55,25 @@ constexpr uint32_t kHeaderBytes = 256;
 constexpr int kMinQ = 8;
 constexpr int kMaxQ = 14;
 
+// Streaming inputs (row indexes, and int32 symbols when encoding) reach the
+// warp coders through a per-warp shared-memory ring of kStage groups filled
+// with cp.async: one counting barrier tracks every copy in flight, so the
+// registers' dependency barriers stay free for the serial state chain.
+constexpr int kStage = 8;
+constexpr int kDecMaxWarps = 24;   // decoder CTA: up to 768 threads
+constexpr int kEncMaxWarps = 32;   // encoder CTA: up to 1024 threads
+constexpr uint32_t kDecStageBytes = kDecMaxWarps * kStage * 32 * 4;
+constexpr uint32_t kEncStageBytes = kEncMaxWarps * kStage * 32 * 4 * 2;
+
 __host__ __device__ inline uint32_t pad16(uint64_t b) {
   return (uint32_t)((b + 15) & ~uint64_t(15));
 }
 
 __device__ __forceinline__ uint32_t bucket_start(uint32_t e) { return e & 0xffffu; }
+// width of a bucket from its start and the next start (mod 2^16; never 0)
+__device__ __forceinline__ uint32_t width_of(uint32_t start, uint32_t next) {
+  return ((next - start - 1u) & 0xffffu) + 1u;
+}
 __device__ __forceinline__ uint32_t bucket_freq(uint32_t e) { return (e >> 16) + 1u; }
 __device__ __forceinline__ uint32_t slot_base(uint32_t s) { return s & 0x07ffffffu; }
 __device__ __forceinline__ uint32_t slot_shift(uint32_t s) { return s >> 27; }
@@ -340,31 +356,61 @@ template <> struct SymIO<uint8_t> {
   }
 };
 
+// ------------------------------------------------------------ cp.async --
+__device__ __forceinline__ void cp_async4(void *smem_dst, const void *gsrc) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(
+                   (uint32_t)__cvta_generic_to_shared(smem_dst)),
+               "l"(gsrc)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() {
+  asm volatile("cp.async.commit_group;" ::: "memory");
+}
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+
 // ------------------------------------------------------------- division --
-// x / f and x % f for x < 2^47 f and 1 <= f <= 2^16 (so the quotient is
-// below 2^47).  The quotient is estimated in double precision -- x rounded to
-// 53 bits times the correctly rounded reciprocal of f, relative error at most
-// about 3 * 2^-53, i.e. an absolute error below 0.05 -- so its truncation is
-// within one of the true quotient; an exact integer remainder check fixes it.
-// (The "float divide + rarely taken exact integer fix-up" of "torch_ans
-// 0.3.0", Performance Tuning, CPU item 3.)
+// x / f and x % f for x < 2^47 f and 1 <= f <= 2^16 (so the quotient is below
+// 2^47).  The quotient is estimated in double precision and corrected once in
+// 32-bit integers (the "float divide + rarely taken exact integer fix-up" of
+// "torch_ans 0.3.0", Performance Tuning, CPU item 3), branch-free:
+//  * an unsigned 32-bit integer u becomes a double exactly as
+//    (2^52 + u) - 2^52, with 2^52 + u assembled from its bit pattern (the
+//    classical "magic number" conversion);
+//  * x = xh 2^32 + xl is then formed with one fused multiply-add, rounded once
+//    (relative error <= 2^-53);
+//  * 1/f comes from the hardware reciprocal estimate refined by three
+//    Newton-Raphson steps r <- r + r (1 - f r) (relative error ~2^-52);
+//  * so q' = x * (1/f) is within 0.05 of the real quotient x/f; adding 2^52
+//    rounds it to the nearest integer, which is floor(x/f) or one more, read
+//    back from the low 52 bits of the sum;
+//  * the remainder x - q f is then in [-f, f): it fits in 32 bits, and a
+//    negative one means q was one too large.
+__device__ __forceinline__ double u32_to_double(uint32_t u) {
+  return __hiloint2double(0x43300000, (int)u) - 4503599627370496.0;  // 2^52
+}
+
 __device__ __forceinline__ double freq_reciprocal(uint32_t f) {
-  return __drcp_rn((double)f);
+  const double fd = u32_to_double(f);
+  double r;
+  asm("rcp.approx.ftz.f64 %0, %1;" : "=d"(r) : "d"(fd));
+#pragma unroll
+  for (int i = 0; i < 3; ++i) r = fma(r, fma(-fd, r, 1.0), r);
+  return r;
 }
 
 __device__ __forceinline__ void divmod_freq(uint64_t x, uint32_t f, double rcp, uint64_t &q,
                                             uint32_t &r) {
-  uint64_t qe = __double2ull_rz(__ull2double_rn(x) * rcp);
-  int64_t rem = (int64_t)(x - qe * (uint64_t)f);
-  if (rem < 0) {
-    qe -= 1;
-    rem += f;
-  } else if (rem >= (int64_t)f) {
-    qe += 1;
-    rem -= f;
-  }
-  q = qe;
-  r = (uint32_t)rem;
+  const double xd =
+      fma(u32_to_double((uint32_t)(x >> 32)), 4294967296.0, u32_to_double((uint32_t)x));
+  const double t = fma(xd, rcp, 4503599627370496.0);  // 2^52 + round(x / f)
+  uint64_t qe = (uint64_t)__double_as_longlong(t) & ((1ull << 52) - 1);
+  const int32_t rem = (int32_t)((uint32_t)x - (uint32_t)qe * f);
+  const bool over = rem < 0;
+  q = qe - (over ? 1u : 0u);
+  r = (uint32_t)(rem + (over ? (int32_t)f : 0));
 }
 
 // One symbol op of the encoder: x -> (x / f) 2^16 + x mod f + start.
@@ -373,7 +419,7 @@ __device__ __forceinline__ uint64_t enc_sym_step(uint64_t x, uint32_t start, uin
   uint64_t q;
   uint32_t r;
   divmod_freq(x, f, rcp, q, r);
-  return (q << kPrec) + r + start;
+  return (q << kPrec) + (r + start);
 }
 
 // ------------------------------------------------------- warp helpers --
@@ -405,7 +451,9 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
 }
 
 __device__ inline bool stage_to_smem(void *dst, const void *src, uint32_t bytes,
-                                     uint64_t *bar_storage, int32_t *status) {
+                                     uint64_t *bar_storage, int32_t *status,
+                                     void *dst2 = nullptr, const void *src2 = nullptr,
+                                     uint32_t bytes2 = 0) {
   const uint32_t bar = smem_addr(bar_storage);
   if (threadIdx.x == 0) {
     asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(bar) : "memory");
@@ -414,18 +462,22 @@ __device__ inline bool stage_to_smem(void *dst, const void *src, uint32_t bytes,
   }
   __syncthreads();
   if (threadIdx.x == 0) {
-    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes)
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar),
+                 "r"(bytes + bytes2)
                  : "memory");
     const uint32_t chunk = 32768;
-    const char *s = reinterpret_cast<const char *>(src);
-    uint32_t d = smem_addr(dst);
-    for (uint32_t off = 0; off < bytes; off += chunk) {
-      uint32_t sz = bytes - off < chunk ? bytes - off : chunk;
-      asm volatile(
-          "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, "
-          "[%3];" ::"r"(d + off),
-          "l"(s + off), "r"(sz), "r"(bar)
-          : "memory");
+    for (int part = 0; part < 2; ++part) {
+      const char *s = reinterpret_cast<const char *>(part ? src2 : src);
+      const uint32_t d = smem_addr(part ? dst2 : dst);
+      const uint32_t nb = part ? bytes2 : bytes;
+      for (uint32_t off = 0; off < nb; off += chunk) {
+        uint32_t sz = nb - off < chunk ? nb - off : chunk;
+        asm volatile(
+            "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, "
+            "[%3];" ::"r"(d + off),
+            "l"(s + off), "r"(sz), "r"(bar)
+            : "memory");
+      }
     }
   }
   bool done = false;

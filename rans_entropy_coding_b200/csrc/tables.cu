@@ -303,7 +303,7 @@ __global__ void __launch_bounds__(kRowThreads)
 // Validates row r and writes its packed buckets.  One block per row.
 __global__ void pack_buckets_kernel(const int32_t *cdfs, int Lmax, const RowMeta *meta,
                                     const int32_t *lengths, uint32_t *buckets,
-                                    int32_t *status) {
+                                    uint16_t *starts, int32_t *status) {
   const int r = blockIdx.x;
   const int32_t *row = cdfs + (size_t)r * (size_t)Lmax;
   const int len = lengths[r];
@@ -318,6 +318,9 @@ __global__ void pack_buckets_kernel(const int32_t *cdfs, int Lmax, const RowMeta
     }
     buckets[base + j] = (uint32_t)(a & 0xffff) | ((uint32_t)(b - a - 1) << 16);
   }
+  // 16-bit starts, row end included: it writes 0 over the next row's leading
+  // 0 (or the trailing sentinel), so overlapping rows agree
+  for (int j = threadIdx.x; j < len; j += blockDim.x) starts[base + j] = (uint16_t)row[j];
 }
 
 // Largest j in [0, nb) with row[j] <= v (row strictly increasing, row[0]=0).
@@ -329,7 +332,7 @@ __device__ __forceinline__ int bucket_of(const int32_t *row, int nb, int v);
 // buckets.  Errors go to the blob's status word.
 __global__ void refresh_kernel(const int32_t *cdfs, int Lmax, const int32_t *lengths,
                                const int32_t *offsets, RowMeta *meta, uint32_t *buckets,
-                               uint32_t *slots, int32_t *status) {
+                               uint16_t *starts, uint32_t *slots, int32_t *status) {
   const int r = blockIdx.y;
   const RowMeta m = meta[r * kMetaCopies];
   const int len = lengths[r];
@@ -351,6 +354,7 @@ __global__ void refresh_kernel(const int32_t *cdfs, int Lmax, const int32_t *len
       }
       buckets[m.bucket_base + j] = (uint32_t)(a & 0xffff) | ((uint32_t)(b - a - 1) << 16);
     }
+    for (int j = threadIdx.x; j < len; j += blockDim.x) starts[m.bucket_base + j] = (uint16_t)row[j];
   }
   const int shift = (int)slot_shift(m.slot);
   const int nslots = 1 << (16 - shift);
@@ -441,14 +445,16 @@ int refresh_tables(const int32_t *cdfs, int K, int Lmax, const int32_t *lengths,
   int32_t *status = reinterpret_cast<int32_t *>(b);
   RowMeta *dmeta = reinterpret_cast<RowMeta *>(b + kHeaderBytes);
   uint32_t *dbuckets = reinterpret_cast<uint32_t *>(b + kHeaderBytes + t.meta_bytes);
-  uint32_t *dslots =
-      reinterpret_cast<uint32_t *>(b + kHeaderBytes + t.meta_bytes + t.bucket_bytes);
+  uint16_t *dstarts =
+      reinterpret_cast<uint16_t *>(b + kHeaderBytes + t.meta_bytes + t.bucket_bytes);
+  uint32_t *dslots = reinterpret_cast<uint32_t *>(b + kHeaderBytes + t.meta_bytes +
+                                                  t.bucket_bytes + t.start_bytes);
   // slot chunks of 256: the largest row has at most 2^14 slots
   int64_t maxslots = 1;
   while (maxslots * K < t.n_slots && maxslots < (1 << kMaxQ)) maxslots <<= 1;
   dim3 grid((unsigned)((maxslots + 255) / 256), (unsigned)K);
-  refresh_kernel<<<grid, 256, 0, st>>>(cdfs, Lmax, lengths, offsets, dmeta, dbuckets, dslots,
-                                       status);
+  refresh_kernel<<<grid, 256, 0, st>>>(cdfs, Lmax, lengths, offsets, dmeta, dbuckets, dstarts,
+                                       dslots, status);
   return cudaGetLastError() == cudaSuccess ? RANS_OK : RANS_ERR_CUDA;
 }
 
@@ -458,6 +464,7 @@ uint64_t tables_bytes_bound(int K, int Lmax) {
   int q = ceil_log2(nb);
   q = q < kMinQ ? kMinQ : (q > kMaxQ ? kMaxQ : q);
   return (uint64_t)kHeaderBytes + pad16(16ull * kMetaCopies * K) + pad16(4ull * K * nb) +
+         pad16(2ull * K * nb + 2) +
          pad16(4ull * K * (1ull << q));
 }
 
@@ -495,6 +502,7 @@ int prepare_tables(const int32_t *cdfs, int K, int Lmax, const int32_t *lengths,
 
   const uint32_t meta_bytes = pad16(16ull * kMetaCopies * K);
   const uint32_t bucket_bytes = pad16(4ull * nbuckets);
+  const uint32_t start_bytes = pad16(2ull * nbuckets + 2);
   int optin = 0;
   cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
   const int64_t budget = (int64_t)optin - 1024;  // room for barriers and scratch
@@ -503,10 +511,10 @@ int prepare_tables(const int32_t *cdfs, int K, int Lmax, const int32_t *lengths,
     for (int r = 0; r < K; ++r) t += 1ull << q[r];
     return t;
   };
-  const bool enc_smem = (int64_t)meta_bytes + bucket_bytes <= budget;
+  const bool enc_smem = (int64_t)meta_bytes + bucket_bytes + kEncStageBytes <= budget;
   bool dec_smem = false;
-  if (enc_smem) {
-    const int64_t room = budget - meta_bytes - bucket_bytes;
+  if ((int64_t)meta_bytes + start_bytes + kDecStageBytes <= budget) {
+    const int64_t room = budget - meta_bytes - start_bytes - kDecStageBytes;
     // About one slot per bucket (fewer than ~2% of lookups then meet three or
     // more boundaries on the scale table); halve the largest row's lookup
     // until the three sections fit.
@@ -526,7 +534,7 @@ int prepare_tables(const int32_t *cdfs, int K, int Lmax, const int32_t *lengths,
   }
   if (sbase >= (1ull << 27)) return RANS_ERR_ARG;
   const uint32_t slot_bytes = pad16(4ull * sbase);
-  const uint64_t need = (uint64_t)kHeaderBytes + meta_bytes + bucket_bytes + slot_bytes;
+  const uint64_t need = (uint64_t)kHeaderBytes + meta_bytes + bucket_bytes + start_bytes + slot_bytes;
   if (blob == nullptr || blob_bytes < need) return RANS_ERR_CAPACITY;
   if ((reinterpret_cast<uintptr_t>(blob) & 255) != 0) return RANS_ERR_ARG;
 
@@ -534,7 +542,9 @@ int prepare_tables(const int32_t *cdfs, int K, int Lmax, const int32_t *lengths,
   int32_t *status = reinterpret_cast<int32_t *>(b);
   RowMeta *dmeta = reinterpret_cast<RowMeta *>(b + kHeaderBytes);
   uint32_t *dbuckets = reinterpret_cast<uint32_t *>(b + kHeaderBytes + meta_bytes);
-  uint32_t *dslots = reinterpret_cast<uint32_t *>(b + kHeaderBytes + meta_bytes + bucket_bytes);
+  uint16_t *dstarts = reinterpret_cast<uint16_t *>(b + kHeaderBytes + meta_bytes + bucket_bytes);
+  uint32_t *dslots =
+      reinterpret_cast<uint32_t *>(b + kHeaderBytes + meta_bytes + bucket_bytes + start_bytes);
   if (cudaMemsetAsync(b, 0, kHeaderBytes, st) != cudaSuccess) return RANS_ERR_CUDA;
   std::vector<RowMeta> meta8((size_t)K * kMetaCopies);
   for (int r = 0; r < K; ++r)
@@ -543,7 +553,8 @@ int prepare_tables(const int32_t *cdfs, int K, int Lmax, const int32_t *lengths,
                       cudaMemcpyHostToDevice, st) != cudaSuccess ||
       cudaStreamSynchronize(st) != cudaSuccess)
     return RANS_ERR_CUDA;
-  pack_buckets_kernel<<<K, 256, 0, st>>>(cdfs, Lmax, dmeta, lengths, dbuckets, status);
+  if (cudaMemsetAsync(dstarts, 0, start_bytes, st) != cudaSuccess) return RANS_ERR_CUDA;
+  pack_buckets_kernel<<<K, 256, 0, st>>>(cdfs, Lmax, dmeta, lengths, dbuckets, dstarts, status);
   int maxslots = 0;
   for (int r = 0; r < K; ++r) maxslots = maxslots > (1 << q[r]) ? maxslots : (1 << q[r]);
   dim3 grid((maxslots + 255) / 256, K);
@@ -563,6 +574,7 @@ int prepare_tables(const int32_t *cdfs, int K, int Lmax, const int32_t *lengths,
   out->n_slots = (int64_t)sbase;
   out->meta_bytes = meta_bytes;
   out->bucket_bytes = bucket_bytes;
+  out->start_bytes = start_bytes;
   out->slot_bytes = slot_bytes;
   out->enc_in_smem = enc_smem ? 1 : 0;
   out->dec_in_smem = dec_smem ? 1 : 0;
