@@ -65,9 +65,7 @@ constexpr int kEncMaxWarps = 32;   // encoder CTA: up to 1024 threads
 constexpr uint32_t kDecStageBytes = kDecMaxWarps * kStage * 32 * 4;
 constexpr uint32_t kEncStageBytes = kEncMaxWarps * kStage * 32 * 4 * 2;
 
-__host__ __device__ inline uint32_t pad16(uint64_t b) {
-  return (uint32_t)((b + 15) & ~uint64_t(15));
-}
+__host__ __device__ inline uint64_t pad16(uint64_t b) { return (b + 15) & ~uint64_t(15); }
 
 __device__ __forceinline__ uint32_t bucket_start(uint32_t e) { return e & 0xffffu; }
 // width of a bucket from its start and the next start (mod 2^16; never 0)

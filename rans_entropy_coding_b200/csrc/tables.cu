@@ -500,9 +500,9 @@ int prepare_tables(const int32_t *cdfs, int K, int Lmax, const int32_t *lengths,
   }
   if (nbuckets > (1ull << 31)) return RANS_ERR_ARG;
 
-  const uint32_t meta_bytes = pad16(16ull * kMetaCopies * K);
-  const uint32_t bucket_bytes = pad16(4ull * nbuckets);
-  const uint32_t start_bytes = pad16(2ull * nbuckets + 2);
+  const uint32_t meta_bytes = (uint32_t)pad16(16ull * kMetaCopies * K);
+  const uint32_t bucket_bytes = (uint32_t)pad16(4ull * nbuckets);
+  const uint32_t start_bytes = (uint32_t)pad16(2ull * nbuckets + 2);
   int optin = 0;
   cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
   const int64_t budget = (int64_t)optin - 1024;  // room for barriers and scratch
@@ -533,7 +533,7 @@ int prepare_tables(const int32_t *cdfs, int K, int Lmax, const int32_t *lengths,
     sbase += 1ull << q[r];
   }
   if (sbase >= (1ull << 27)) return RANS_ERR_ARG;
-  const uint32_t slot_bytes = pad16(4ull * sbase);
+  const uint32_t slot_bytes = (uint32_t)pad16(4ull * sbase);
   const uint64_t need = (uint64_t)kHeaderBytes + meta_bytes + bucket_bytes + start_bytes + slot_bytes;
   if (blob == nullptr || blob_bytes < need) return RANS_ERR_CAPACITY;
   if ((reinterpret_cast<uintptr_t>(blob) & 255) != 0) return RANS_ERR_ARG;

@@ -75,3 +75,11 @@ def test_cuda_calls_fail_cleanly_without_device(lib):
     st = lib.rans_encode_with_indexes(None, 0, None, 0, ctypes.byref(t), None, None, 0, None,
                                       None, 0, None)
     assert st == rb.ERR_ARG
+
+
+def test_workspace_sizes_do_not_truncate(lib):
+    """A single stream of 2^30 symbols needs more than 8 GiB of scratch; the
+    size must not wrap at 32 bits."""
+    big = rb.Chunking.contig(1, 32)
+    assert rb.rans_encode_workspace_bytes(big, 1 << 30) >= 8 << 30
+    assert rb.rans_max_compressed_bytes(big, 1 << 30) >= 8 << 30
