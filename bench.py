@@ -137,8 +137,15 @@ class ClockSampler:
                 "samples": len(rows)}
 
 
+def shard_images(rank, images=N_IMAGES):
+    """Image ids coded by `rank`: every rank codes its own `images` images
+    (weak scaling; streams never cross images, so no exchange is needed)."""
+    return list(range(images * rank, images * (rank + 1)))
+
+
 def load_inputs(rank, group, images=N_IMAGES):
-    return WL.y_batch(n_images=images, first_image=images * rank, cg=group)
+    ids = shard_images(rank, images)
+    return WL.y_batch(n_images=len(ids), first_image=ids[0], cg=group)
 
 
 # --------------------------------------------------------- CPU oracle leg --

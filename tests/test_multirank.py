@@ -1,0 +1,60 @@
+"""The multi-GPU path shards by image with no data exchange; its host logic
+(image shards, per-rank coding, max-over-ranks timing) runs here as two gloo
+ranks on the CPU, coding with the oracle."""
+import os
+import socket
+
+import numpy as np
+import torch.distributed as dist
+import torch.multiprocessing as mp
+
+import bench
+import oracle as O
+import workloads as WL
+
+
+def _free_port():
+    s = socket.socket()
+    s.bind(("127.0.0.1", 0))
+    port = s.getsockname()[1]
+    s.close()
+    return port
+
+
+def _rank(rank, world, port, out):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank),
+                      WORLD_SIZE=str(world))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        ids = bench.shard_images(rank, images=1)
+        w = WL.y_batch(n_images=1, first_image=ids[0], cg=4, th=64, tw=64)
+        c, l, o = O.build_cdfs_from_scales(w["scales"], w["tail_mass"])
+        sym = np.asarray(w["symbols"]).reshape(-1)
+        streams = list(range(8))            # a few streams of this rank's image
+        data, offs = O.encode_with_indexes(sym, w["indexes"], c, l, o, w["chunking"], W=32,
+                                           streams=streams)
+        t = float(rank + 1)                  # a per-rank "time"
+        tmax = bench.max_over_ranks(t, world)
+        gathered = [None] * world
+        dist.all_gather_object(gathered, (ids, int(sym.sum()), data.tobytes()[:64]))
+        out[rank] = (tmax, gathered)
+    finally:
+        dist.destroy_process_group()
+
+
+def test_two_ranks_shard_by_image():
+    world = 2
+    port = _free_port()
+    with mp.Manager() as m:
+        out = m.dict()
+        mp.spawn(_rank, args=(world, port, out), nprocs=world, join=True)
+        res = dict(out)
+    assert res[0][0] == res[1][0] == 2.0                     # max over ranks
+    shards = [g[0] for g in res[0][1]]
+    assert shards == [[0], [1]]                              # disjoint, covering
+    # each rank coded its own image: different data, different streams
+    assert res[0][1][0][1] != res[0][1][1][1]
+    assert res[0][1][0][2] != res[0][1][1][2]
+    # rank 1's shard equals image 1 of a two-image batch coded in one process
+    w = WL.y_batch(n_images=2)
+    assert int(np.asarray(w["symbols"])[1].sum()) == res[0][1][1][1]
