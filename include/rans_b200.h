@@ -278,6 +278,29 @@ int rans_decode_with_indexes(const uint8_t *in, uint64_t in_bytes,
                              int32_t sym_dtype, void *workspace, uint64_t workspace_bytes,
                              void *stream);
 
+/*
+ * rans_encode_with_indexes without a workspace argument, for callers that
+ * cannot allocate device memory themselves (for example code inside a host
+ * framework whose allocator owns all device memory, or a latency-critical path
+ * on which a cudaMalloc, which may synchronise the device, is not allowed).
+ * The pages have no counterpart: this is a packaging convenience of the
+ * library.
+ *   The workspace is a 32 MiB array inside the library that every GPU loading
+ *   it keeps until exit; inputs needing more (rans_encode_workspace_bytes)
+ *   return RANS_ERR_CAPACITY.  The first call on a device looks the array's
+ *   device address up (call it once before any stream capture).  All calls
+ *   share the array: calls that overlap on the GPU race, so serialise them.
+ *   Device errors cannot be read with rans_get_status here; instead
+ *   stream_offsets[S] is set to UINT64_MAX.  Other arguments, outputs and
+ *   results are those of rans_encode_with_indexes.  Allocates nothing.
+ */
+int rans_encode_with_indexes_noalloc(const void *symbols, int32_t sym_dtype,
+                                     const int32_t *indexes, int64_t n,
+                                     const rans_tables *tables,
+                                     const rans_chunking *chunking, uint8_t *out,
+                                     uint64_t out_capacity, uint64_t *stream_offsets,
+                                     void *stream);
+
 /* Synchronises `stream` and returns the first error recorded in `workspace`
  * (RANS_OK if none), then clears it. */
 int rans_get_status(void *workspace, void *stream);

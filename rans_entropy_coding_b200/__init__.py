@@ -10,6 +10,7 @@ from ._lib import (  # noqa: F401
     SYM_INT16, SYM_INT32, SYM_UINT8, Chunking, RansError, Tables, Workspaces, aligned_empty,
     check, decode_with_indexes, encode_with_indexes, lib, rans_build_cdfs_from_pmfs,
     rans_build_cdfs_from_scales, rans_chunking, rans_debug_divide, rans_decode_with_indexes,
-    rans_decode_workspace_bytes, rans_encode_with_indexes, rans_encode_workspace_bytes,
+    rans_decode_workspace_bytes, rans_encode_with_indexes, rans_encode_with_indexes_noalloc,
+    rans_encode_workspace_bytes,
     rans_gaussian_lengths, rans_get_status, rans_max_compressed_bytes, rans_num_streams,
     rans_tables, rans_tables_bytes, rans_tables_prepare, rans_tables_refresh)

@@ -75,6 +75,8 @@ SIGNATURES = [
      [_P, _I32, _P, _I64, _TBP, _CHP, _P, _U64, _P, _P, _U64, _P]),
     ("rans_decode_with_indexes", ctypes.c_int,
      [_P, _U64, _P, _P, _I64, _TBP, _CHP, _P, _I32, _P, _U64, _P]),
+    ("rans_encode_with_indexes_noalloc", ctypes.c_int,
+     [_P, _I32, _P, _I64, _TBP, _CHP, _P, _U64, _P, _P]),
     ("rans_get_status", ctypes.c_int, [_P, _P]),
     ("rans_debug_divide", ctypes.c_int, [_P, _P, _I64, _P, _P, _P]),
 ]
@@ -196,6 +198,14 @@ def rans_decode_with_indexes(data, stream_offsets, indexes, n, tables, chunking,
         _ptr(data), data.numel(), _ptr(stream_offsets), _ptr(indexes), n,
         ctypes.byref(tables.c), ctypes.byref(chunking.c), _ptr(symbols_out),
         _DTYPE_CODE[symbols_out.dtype], _ptr(workspace), workspace.numel(), _stream(stream))
+
+
+def rans_encode_with_indexes_noalloc(symbols, indexes, n, tables, chunking, out,
+                                     stream_offsets, stream=None):
+    _need_cuda(symbols, indexes, out, stream_offsets)
+    return lib().rans_encode_with_indexes_noalloc(
+        _ptr(symbols), _DTYPE_CODE[symbols.dtype], _ptr(indexes), n, ctypes.byref(tables.c),
+        ctypes.byref(chunking.c), _ptr(out), out.numel(), _ptr(stream_offsets), _stream(stream))
 
 
 def rans_get_status(workspace, stream=None):

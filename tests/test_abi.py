@@ -83,3 +83,7 @@ def test_workspace_sizes_do_not_truncate(lib):
     big = rb.Chunking.contig(1, 32)
     assert rb.rans_encode_workspace_bytes(big, 1 << 30) >= 8 << 30
     assert rb.rans_max_compressed_bytes(big, 1 << 30) >= 8 << 30
+    # the allocation-free encoder refuses it before touching the device
+    st = lib.rans_encode_with_indexes_noalloc(None, 0, None, 1 << 30, rb.rans_tables(), big.c,
+                                              None, 0, None, None)
+    assert st == rb.ERR_CAPACITY
