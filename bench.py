@@ -50,8 +50,38 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-clocks", action="store_true")
-    ap.add_argument("--traffic-json", default=os.path.join(ROOT, "profiles", "traffic.json"))
+    ap.add_argument("--traffic-file", default=os.path.join(ROOT, "profiles", "dram_traffic.txt"))
     return ap.parse_args()
+
+
+def kernel_sources_digest():
+    """sha256 over the CUDA sources, so a DRAM-traffic figure taken with ncu
+    is only reported while the kernels it measured are unchanged."""
+    import hashlib
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "rans_entropy_coding_b200", "csrc")
+    for name in sorted(os.listdir(csrc)):
+        if name.endswith((".cu", ".cuh", ".h")):
+            h.update(name.encode())
+            h.update(open(os.path.join(csrc, name), "rb").read())
+    return h.hexdigest()
+
+
+def measured_traffic(path, kernel, workload):
+    """Per-launch dram__bytes_read.sum + dram__bytes_write.sum for `kernel`
+    from the committed ncu summary, or None when the summary is missing, was
+    taken on another workload or on other kernel sources."""
+    if not os.path.exists(path):
+        return None
+    kv = {}
+    for line in open(path):
+        if ":" in line and not line.startswith("#"):
+            k, v = line.split(":", 1)
+            kv[k.strip()] = v.strip()
+    if kv.get("workload") != workload or kv.get("sources_sha256") != kernel_sources_digest():
+        return None
+    v = kv.get(kernel + "_bytes_per_launch")
+    return int(v) if v else None
 
 
 def dist_setup(args):
@@ -287,13 +317,8 @@ def run_ours(args, world, rank, local):
     enc_gbs = alg_enc / (enc_ms * 1e-3) / 1e9
     dec_gbs = alg_dec / (dec_ms * 1e-3) / 1e9
     dominant = "decode" if dec_ms >= enc_ms else "encode"
-    traffic = None
-    if os.path.exists(args.traffic_json):
-        try:
-            tj = json.load(open(args.traffic_json))
-            traffic = tj.get(dominant, {}).get("bytes_per_launch")
-        except (OSError, ValueError):
-            traffic = None
+    traffic = measured_traffic(args.traffic_file, dominant,
+                               "images=%d group=%d" % (args.images, args.group))
     ach = dec_gbs if dominant == "decode" else enc_gbs
     total_syms = n * world
     ms_per_step = elapsed_ms / args.steps
