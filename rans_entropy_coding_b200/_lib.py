@@ -275,13 +275,15 @@ class Chunking:
 class Tables:
     """CDF rows (cdfs, cdf_lengths, offsets) plus the prepared table blob."""
 
-    def __init__(self, cdfs, cdf_lengths, offsets, stream=None):
+    def __init__(self, cdfs, cdf_lengths, offsets, stream=None, blob_bytes=None):
+        """blob_bytes: the blob's size (default rans_tables_bytes(K, Lmax)); a
+        smaller blob leaves the decoder fewer bitmap words."""
         self.cdfs, self.cdf_lengths, self.offsets = cdfs, cdf_lengths, offsets
         K, Lmax = cdfs.shape
-        self.blob = torch.empty(rans_tables_bytes(K, Lmax) + 256, dtype=torch.uint8,
-                                device=cdfs.device)
+        nbytes = rans_tables_bytes(K, Lmax) if blob_bytes is None else int(blob_bytes)
+        self.blob = torch.empty(nbytes + 256, dtype=torch.uint8, device=cdfs.device)
         off = (-self.blob.data_ptr()) % 256
-        self.blob = self.blob[off:off + rans_tables_bytes(K, Lmax)]
+        self.blob = self.blob[off:off + nbytes]
         self.c = rans_tables()
         check(rans_tables_prepare(cdfs, cdf_lengths, offsets, self.blob, self.c, stream),
               "tables_prepare")

@@ -5,8 +5,9 @@
 //    "Benchmark notes" section 4).  It is found through a per-row table of
 //    2^q slots keyed by the top q bits of cum ("torch_ans 0.3.0", Usage,
 //    inverse-CDF decoding): a slot resolves up to two bucket boundaries with
-//    two compares; a slot with more is counted by the whole warp, one ballot
-//    per 32 candidates;
+//    two compares, and a slot with more points to boundary bitmaps that a
+//    population count resolves; only a table that ran out of bitmap room
+//    searches;
 //  * state update x = freq (x >> 16) + cum - start and a refill of one
 //    32-bit word when x < 2^31 (64-bit state / 32-bit words / 16-bit
 //    precision: "torch_ans 0.3.0", Usage, rans64 row);
@@ -19,11 +20,15 @@
 //    order, reading their bypass pieces, since how many words a lane takes
 //    depends on what it reads ("torch_ans 0.3.0", Performance Tuning, GPU
 //    item 5: the bypass phase is sequential across the lanes and skipped by a
-//    group ballot).
+//    group ballot).  The group is first decoded as if nothing escaped; the
+//    ballot, taken beside the refill, sends it down the slow path.
 //  Latency: row indexes stream through a per-warp shared-memory ring filled
-//  with cp.async kStage - 1 groups ahead; each stream's words are bulk
+//  with cp.async kDecStage - 1 groups ahead, the next group's row metadata
+//  is read while this group decodes, and each stream's words are bulk
 //  prefetched into L2 when the warp starts it.
 //  Tables are staged into shared memory with bulk copies when they fit.
+#include <type_traits>
+
 #include "rans_common.cuh"
 #include "rans_internal.h"
 
@@ -56,12 +61,42 @@ __device__ __forceinline__ bool stream_bounds(const DecCtx &c, int64_t s, int W,
   return true;
 }
 
-// Fast slot decode: bucket lo + (c > e1) + (c > e2); multi = three or more
-// boundaries inside the slot.
-__device__ __forceinline__ uint32_t slot_symbol(uint32_t se, uint32_t c, bool &multi) {
+// The bucket holding cum in row m: the slot's own two boundaries, or its
+// boundary bitmap (the bitmap word is read for every lane, from the slot
+// itself when the slot needs none, so the lookup takes no branch).  With
+// SEARCH (a table with slots that ran out of bitmap room) those slots take a
+// binary search over the starts; WARP: the search is entered once per warp.
+template <bool SEARCH, bool WARP>
+__device__ __forceinline__ uint32_t lookup(uint32_t cum, const RowMeta &m, const uint16_t *starts,
+                                           const uint32_t *slots, bool active) {
+  const uint32_t sh = slot_shift(m.slot);
+  const uint32_t i1 = slot_base(m.slot) + (cum >> sh);
+  const uint32_t se = slots[i1];
   const uint32_t e1 = (se >> 16) & 0xffu, e2 = se >> 24;
-  multi = e1 > e2;
-  return (se & 0xffffu) + (c > e1 ? 1u : 0u) + (c > e2 ? 1u : 0u);
+  const uint32_t c = cum & ((1u << sh) - 1u);
+  const uint32_t lo = se & 0xffffu;
+  uint32_t sym = lo + (c > e1 ? 1u : 0u) + (c > e2 ? 1u : 0u);
+  const bool bitmap = e1 == 0xffu && e2 != 0xffu;
+  const uint32_t i2 = bitmap ? (lo | ((se >> 8) & 0xff0000u)) + (c >> 4) : i1;
+  const uint32_t ce = slots[i2];
+  const uint32_t sym2 = (ce >> 16) + __popc(ce & ((2u << (c & 15u)) - 1u));
+  sym = bitmap ? sym2 : sym;
+  if (SEARCH) {
+    const bool srch = active && e1 > e2 && e1 != 0xffu;
+    if (WARP ? __any_sync(kFull, srch) : srch) {
+      if (srch) {  // last bucket in [lo, lo + e2 + 3] whose start is <= cum
+        uint32_t l = lo, h = lo + e2 + 3u;
+        while (l < h) {
+          const uint32_t mid = (l + h + 1) >> 1;
+          if (starts[m.bucket_base + mid] <= cum) l = mid; else h = mid - 1;
+        }
+        sym = l;
+      }
+    }
+  }
+  // never past the row's last bucket, whatever the slots hold (a refresh that
+  // rejected a row leaves that row's slots stale)
+  return min(sym, m.maxv);
 }
 
 struct EscapeResult {
@@ -170,43 +205,31 @@ __device__ __forceinline__ void load_window(WarpDec &st, const uint32_t *words, 
 }
 
 // One group of 32 symbols: lookup, state update, refill, output.  m is the
-// group's row metadata, loaded one group ahead.
-template <typename SymT, bool FULL>
+// group's row metadata, read one group ahead.  The refill is taken as if no
+// lane escaped; the escape ballot, issued beside it, sends the group down
+// the lane-serial path from the state after the symbol op.
+template <typename SymT, bool FULL, bool SEARCH>
 __device__ __forceinline__ void dec_group(WarpDec &st, const RowMeta &m, const uint16_t *starts,
                                           const uint32_t *slots, bool active, SymT *dst,
                                           const uint32_t *words, uint64_t nw) {
   const int lane = threadIdx.x & 31;
   if (FULL) active = true;
   const uint32_t cum = (uint32_t)st.x & (kTotal - 1);
-  const uint32_t sh = slot_shift(m.slot);
-  const uint32_t se = slots[slot_base(m.slot) + (cum >> sh)];
-  const uint32_t e1 = (se >> 16) & 0xffu, e2 = se >> 24;
-  const uint32_t c = cum & ((1u << sh) - 1u);
-  uint32_t sym = (se & 0xffffu) + (c > e1 ? 1u : 0u) + (c > e2 ? 1u : 0u);
-  const bool multi = active && e1 > e2;
-  if (__any_sync(kFull, multi)) {
-    if (multi) {  // last bucket in [lo, lo + count] whose start is <= cum
-      uint32_t lo = se & 0xffffu, hi = lo + e2 + 3u;
-      while (lo < hi) {
-        const uint32_t mid = (lo + hi + 1) >> 1;
-        if (starts[m.bucket_base + mid] <= cum) lo = mid; else hi = mid - 1;
-      }
-      sym = lo;
-    }
-  }
+  const uint32_t sym = lookup<SEARCH, true>(cum, m, starts, slots, active);
   const uint32_t start = starts[m.bucket_base + sym];
   const uint32_t freq = width_of(start, starts[m.bucket_base + sym + 1]);
-  uint64_t x = st.x;
-  if (active) x = (uint64_t)freq * (x >> kPrec) + (cum - start);
+  uint64_t x = (uint64_t)freq * (st.x >> kPrec) + (cum - start);
+  if (!FULL) x = active ? x : st.x;
   const bool esc = active && sym == m.maxv;
+  const bool need = active && x < kL;
+  const uint32_t nm = __ballot_sync(kFull, need);
+  const bool any_esc = __any_sync(kFull, esc);
+  const uint32_t j = st.off + __popc(nm & lanemask_lt());
+  // the lane holding window word j (mod 32) sends it from w0 or w1
+  const uint32_t wv = __shfl_sync(kFull, (uint32_t)lane >= st.off ? st.w0 : st.w1, j & 31);
   int32_t val = (int32_t)sym + m.offset;
-  if (!__any_sync(kFull, esc)) {
-    const bool need = active && x < kL;
-    const uint32_t nm = __ballot_sync(kFull, need);
-    const uint32_t j = st.off + __popc(nm & lanemask_lt());
-    // the lane holding window word j (mod 32) sends it from w0 or w1
-    const uint32_t wv = __shfl_sync(kFull, (uint32_t)lane >= st.off ? st.w0 : st.w1, j & 31);
-    if (need) x = (x << 32) | wv;
+  if (!any_esc) {
+    st.x = need ? ((x << 32) | wv) : x;
     st.off += __popc(nm);
     if (st.off >= 32) {
       st.w0 = st.w1;
@@ -217,22 +240,25 @@ __device__ __forceinline__ void dec_group(WarpDec &st, const RowMeta &m, const u
     }
   } else {
     const EscapeResult er = escape_group(x, active, esc, m.maxv, st.cur + st.off, words, nw);
-    x = er.x;
+    st.x = er.x;
     if (esc) val = (int32_t)(er.val + (int64_t)m.offset);
     st.bad |= er.bad;
     st.cur = er.cur;
     st.off = 0;
     load_window(st, words, nw);
   }
-  st.x = x;
-  if (active) *dst = (SymT)val;
+  if (active) st_global(dst, (SymT)val);
 }
 
-template <typename SymT, bool IB0, bool WIDE>
+// One warp decodes one stream, a group of 32 symbols per step: the copies
+// for group g + kDecStage - 1, group g+1's row metadata from the ring, then
+// group g's decode.
+template <typename SymT, bool IB0, bool WIDE, bool SEARCH>
 __device__ __forceinline__ void decode_stream_w32(const DecCtx &c, const StreamDesc &d,
-                                                  const RowMeta *meta, const uint16_t *buckets,
+                                                  const RowMeta *meta, const uint16_t *starts,
                                                   const uint32_t *slots, uint32_t *stg,
                                                   int64_t s, const uint32_t *words, uint64_t nw) {
+  constexpr int kS = kDecStage;
   const int lane = threadIdx.x & 31;
   const int32_t n = (int32_t)d.n;
   const int32_t G = (n + 31) >> 5;
@@ -250,41 +276,38 @@ __device__ __forceinline__ void decode_stream_w32(const DecCtx &c, const StreamD
   st.rmax = 0;
   st.bad = false;
 
-  // Group g's row indexes land in stage slot g mod kStage, copied kStage - 1
-  // groups ahead; a lane past the stream end copies element 0 (ignored).
+  // Group g's row indexes land in stage slot g mod kS, copied kS - 1 groups
+  // ahead.  Copies for groups past the end (and lanes past the stream end)
+  // read the stream's element 0 and are never used.
   Stepper<WIDE> pl;  // next group to copy
   pl.init(d.t, lane);
   Stepper<WIDE> pc = pl;  // group being decoded (output position)
   auto issue = [&](int32_t gi) {
-    if (gi < G) {
-      const int32_t rel = lane < n - gi * 32 ? pl.rel : 0;
-      cp_async4(stg + (gi & (kStage - 1)) * 32 + lane,
-                IB0 ? idx_s + rel : c.idx + ((base + rel) >> ib));
-      pl.fwd(32);
-    }
+    const int32_t rel = gi < G && lane < n - gi * 32 ? pl.rel : 0;
+    cp_async4(stg + (gi & (kS - 1)) * 32 + lane,
+              IB0 ? idx_s + rel : c.idx + ((base + rel) >> ib));
     cp_async_commit();
+    pl.fwd(32);
   };
   auto meta_of = [&](uint32_t r) -> RowMeta {
     st.rmax = max(st.rmax, r);
     return row_meta(meta, min(r, kmax));
   };
-#pragma unroll
-  for (int32_t u = 0; u < kStage - 1; ++u) issue(u);
-  cp_async_wait<kStage - 2>();
+#pragma unroll 1
+  for (int32_t u = 0; u < kS - 1; ++u) issue(u);
+  cp_async_wait<kS - 2>();
   RowMeta m = meta_of(stg[lane]);
-  for (int32_t g = 0; g < G; ++g) {
-    issue(g + kStage - 1);
-    cp_async_wait<kStage - 2>();  // groups up to g + 1 have landed
-    // (after the last group the slot may hold another stream's data: unused)
-    const RowMeta mn = meta_of(g + 1 < G ? stg[((g + 1) & (kStage - 1)) * 32 + lane] : 0u);
-    if (g + 1 < G)
-      dec_group<SymT, true>(st, m, buckets, slots, true, out_s + pc.rel, words, nw);
-    else
-      dec_group<SymT, false>(st, m, buckets, slots, lane < n - g * 32, out_s + pc.rel, words,
-                             nw);
+#pragma unroll 1
+  for (int32_t g = 0; g + 1 < G; ++g) {
+    issue(g + kS - 1);
+    cp_async_wait<kS - 2>();  // groups up to g + 1 have landed
+    const RowMeta mn = meta_of(stg[((g + 1) & (kS - 1)) * 32 + lane]);
+    dec_group<SymT, true, SEARCH>(st, m, starts, slots, true, out_s + pc.rel, words, nw);
     pc.fwd(32);
     m = mn;
   }
+  dec_group<SymT, false, SEARCH>(st, m, starts, slots, lane < n - (G - 1) * 32, out_s + pc.rel,
+                                 words, nw);
   cp_async_wait<0>();
   if (__any_sync(kFull, st.rmax > kmax)) {
     if (lane == 0) report(c.status, RANS_ERR_INDEX, s);
@@ -294,7 +317,7 @@ __device__ __forceinline__ void decode_stream_w32(const DecCtx &c, const StreamD
   if (!__all_sync(kFull, ok) && lane == 0) report(c.status, RANS_ERR_CORRUPT, s);
 }
 
-template <typename SymT, bool IB0>
+template <typename SymT, bool IB0, bool SEARCH>
 __device__ __forceinline__ void decode_stream_w32_entry(const DecCtx &c, const RowMeta *meta,
                                                         const uint16_t *buckets,
                                                         const uint32_t *slots, uint32_t *stg,
@@ -318,9 +341,9 @@ __device__ __forceinline__ void decode_stream_w32_entry(const DecCtx &c, const R
     return;
   }
   if (d.t.ww >= 32)
-    decode_stream_w32<SymT, IB0, true>(c, d, meta, buckets, slots, stg, s, words, nw);
+    decode_stream_w32<SymT, IB0, true, SEARCH>(c, d, meta, buckets, slots, stg, s, words, nw);
   else
-    decode_stream_w32<SymT, IB0, false>(c, d, meta, buckets, slots, stg, s, words, nw);
+    decode_stream_w32<SymT, IB0, false, SEARCH>(c, d, meta, buckets, slots, stg, s, words, nw);
 }
 
 template <typename SymT>
@@ -370,19 +393,7 @@ __device__ void decode_stream_w1(const DecCtx &c, const RowMeta *meta, const uin
     }
     const RowMeta m = row_meta(meta, (uint32_t)r);
     const uint32_t cum = (uint32_t)x & (kTotal - 1);
-    const uint32_t sh = slot_shift(m.slot);
-    const uint32_t se = slots[slot_base(m.slot) + (cum >> sh)];
-    bool multi;
-    uint32_t sym = slot_symbol(se, cum & ((1u << sh) - 1u), multi);
-    if (multi) {
-      // last bucket in [lo, lo + count] whose start is <= cum
-      uint32_t lo = se & 0xffffu, hi = lo + (se >> 24) + 3u;
-      while (lo < hi) {
-        const uint32_t mid = (lo + hi + 1) >> 1;
-        if (buckets[m.bucket_base + mid] <= cum) lo = mid; else hi = mid - 1;
-      }
-      sym = lo;
-    }
+    const uint32_t sym = lookup<true, false>(cum, m, buckets, slots, true);
     const uint32_t start = buckets[m.bucket_base + sym];
     const uint32_t freq = width_of(start, buckets[m.bucket_base + sym + 1]);
     x = (uint64_t)freq * (x >> kPrec) + cum - start;
@@ -441,10 +452,16 @@ __global__ void __launch_bounds__(W == 32 ? kDecMaxThreads32 : kDecThreads1)
     const int warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
     uint32_t *stg = reinterpret_cast<uint32_t *>(
                         smem + (SMEM ? c.meta_bytes + c.start_bytes + c.slot_bytes : 0)) +
-                    warp * kStage * 32;
+                    warp * kDecStage * 32;
+    // slots that ran out of bitmap room (flagged in the blob header) search
+    const bool search = reinterpret_cast<const uint32_t *>(c.blob)[kSearchFlagWord] != 0;
     for (int64_t k = blockIdx.x + (int64_t)gridDim.x * warp; k < c.g.S;
-         k += (int64_t)gridDim.x * nw)
-      decode_stream_w32_entry<SymT, IB0>(c, meta, buckets, slots, stg, stream_of(c.g, k));
+         k += (int64_t)gridDim.x * nw) {
+      if (search)
+        decode_stream_w32_entry<SymT, IB0, true>(c, meta, buckets, slots, stg, stream_of(c.g, k));
+      else
+        decode_stream_w32_entry<SymT, IB0, false>(c, meta, buckets, slots, stg, stream_of(c.g, k));
+    }
   } else {
     for (int64_t k = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; k < c.g.S;
          k += (int64_t)gridDim.x * blockDim.x)
@@ -456,7 +473,7 @@ template <int W, typename SymT, bool SMEM, bool IB0>
 int launch_decode_t(const DecCtx &c, cudaStream_t st) {
   auto kern = decode_kernel<W, SymT, SMEM, IB0>;
   const uint32_t tab = SMEM ? c.meta_bytes + c.start_bytes + c.slot_bytes : 0;
-  const uint32_t per_warp = W == 32 ? kStage * 32 * 4 : 0;
+  const uint32_t per_warp = W == 32 ? kDecStage * 32 * 4 : 0;
   int dev = 0;
   cudaGetDevice(&dev);
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,

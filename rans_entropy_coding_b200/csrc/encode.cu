@@ -17,6 +17,8 @@
 //    lanes > l: a ballot + popc places them.  A group holding an escape is
 //    coded off the fast path: each lane counts its words, a suffix sum over
 //    lanes places them, and the lane writes them.
+#include <type_traits>
+
 #include "rans_common.cuh"
 #include "rans_internal.h"
 
@@ -64,7 +66,7 @@ template <bool WRITE>
 __device__ __forceinline__ void bits_op(uint64_t &x, uint32_t val, uint32_t *end, uint32_t &k,
                                         uint32_t pos0) {
   if (x >= (1ull << 59)) {
-    if (WRITE) end[-1 - (int64_t)(pos0 + k)] = (uint32_t)x;
+    if (WRITE) st_global(end - 1 - (pos0 + k), (uint32_t)x);
     ++k;
     x >>= 32;
   }
@@ -88,7 +90,7 @@ __device__ __forceinline__ uint32_t symbol_ops(uint64_t &x, uint32_t start, uint
     for (uint32_t t = 0; t < nb / kBypassMax; ++t) bits_op<WRITE>(x, kBypassMax, end, k, pos0);
   }
   if (x >= ((uint64_t)freq << 47)) {
-    if (WRITE) end[-1 - (int64_t)(pos0 + k)] = (uint32_t)x;
+    if (WRITE) st_global(end - 1 - (pos0 + k), (uint32_t)x);
     ++k;
     x >>= 32;
   }
@@ -129,47 +131,92 @@ struct WarpEnc {
   bool range_err;
 };
 
-// One group of 32 symbols, coded lane 31 first.  m is the group's row
-// metadata, loaded one group ahead.
-template <bool FULL>
-__device__ __forceinline__ void enc_group(WarpEnc &st, const RowMeta &m, const uint32_t *buckets,
-                                          int32_t sv, bool active, uint32_t above,
-                                          uint32_t *end) {
-  if (FULL) active = true;
-  // value mapping: in range iff 0 <= s - offset < maxv (64-bit, exact)
-  const int64_t v = (int64_t)sv - (int64_t)m.offset;
-  const bool in_range = (uint64_t)v < (uint64_t)m.maxv;
-  const uint32_t e = buckets[m.bucket_base + (in_range ? (uint32_t)v : m.maxv)];
-  const uint32_t start = bucket_start(e), freq = bucket_freq(e);
-  const bool esc = active && !in_range;
-  const double rcp = freq_reciprocal(freq);
-  uint64_t x = st.x;
-  if (!__any_sync(kFull, esc)) {
-    // x >= freq * 2^47  <=>  high word of x >= freq * 2^15
-    const bool need = active && (uint32_t)(x >> 32) >= (freq << 15);
-    const uint32_t bm = __ballot_sync(kFull, need);
-    const uint32_t lo = (uint32_t)x;
-    if (need) end[-1 - (int64_t)(st.cursor + __popc(bm & above))] = lo;
-    x = need ? (x >> 32) : x;
-    st.cursor += __popc(bm);
-    if (active) x = enc_sym_step(x, start, freq, rcp);
-  } else {
-    uint64_t raw = 0;
-    if (esc) raw = v < 0 ? (uint64_t)(-2 * v - 1) : (uint64_t)(2 * (v - (int64_t)m.maxv));
-    st.range_err |= esc && (raw >> 60) != 0;
-    uint32_t total;
-    x = escape_group_enc(x, active, start, freq, rcp, raw & ((1ull << 60) - 1), esc, end,
-                         st.cursor, total);
-    st.cursor += total;
-  }
-  st.x = x;
+// A group's table lookups, done one group ahead of its state update: they
+// do not depend on the state, so they run while the previous group's
+// division does.  The shared-memory read comes first (enc_bucket), the
+// arithmetic on it later (enc_look), with the other group's state update in
+// between.
+struct EncLook {
+  uint32_t start, freq;
+  double rcp;
+  int64_t v;         // s - offset (escape path)
+  uint32_t maxv;
+  bool esc;          // this lane escapes
+  bool any_esc;      // some lane of the group escapes
+};
+
+struct EncBucket {
+  uint32_t e;        // bucket word
+  int64_t v;
+  uint32_t maxv;
+  bool in_range;
+};
+
+// value mapping: in range iff 0 <= s - offset < maxv (64-bit, exact)
+__device__ __forceinline__ EncBucket enc_bucket(int32_t sv, const RowMeta &m,
+                                                const uint32_t *buckets) {
+  EncBucket b;
+  b.v = (int64_t)sv - (int64_t)m.offset;
+  b.maxv = m.maxv;
+  b.in_range = (uint64_t)b.v < (uint64_t)m.maxv;
+  b.e = buckets[m.bucket_base + (b.in_range ? (uint32_t)b.v : m.maxv)];
+  return b;
 }
 
+__device__ __forceinline__ EncLook enc_look(const EncBucket &b, bool active) {
+  EncLook L;
+  L.v = b.v;
+  L.maxv = b.maxv;
+  L.start = bucket_start(b.e);
+  L.freq = bucket_freq(b.e);
+  L.rcp = freq_reciprocal(L.freq);
+  L.esc = active && !b.in_range;
+  L.any_esc = __any_sync(kFull, L.esc);
+  return L;
+}
+
+// One group of 32 symbols with no escape, coded lane 31 first: lanes whose
+// state reaches freq * 2^47 push its low word (ballot + popc place the
+// words), then every lane takes its symbol op.
+template <bool FULL>
+__device__ __forceinline__ void enc_group_fast(WarpEnc &st, const EncLook &L, bool active,
+                                               uint32_t above, uint32_t *end) {
+  if (FULL) active = true;
+  uint64_t x = st.x;
+  // x >= freq * 2^47  <=>  high word of x >= freq * 2^15
+  const bool need = active && (uint32_t)(x >> 32) >= (L.freq << 15);
+  const uint32_t bm = __ballot_sync(kFull, need);
+  if (need) st_global(end - 1 - (st.cursor + __popc(bm & above)), (uint32_t)x);
+  x = need ? (x >> 32) : x;
+  st.cursor += __popc(bm);
+  const uint64_t y = enc_sym_step(x, L.start, L.freq, L.rcp);
+  st.x = active ? y : x;
+}
+
+// The same group holding an escape, from the state and cursor before it.
+__device__ __forceinline__ void enc_group_escape(WarpEnc &st, uint64_t x0, uint32_t cursor0,
+                                                 const EncLook &L, bool active, uint32_t *end) {
+  uint64_t raw = 0;
+  if (L.esc) raw = L.v < 0 ? (uint64_t)(-2 * L.v - 1) : (uint64_t)(2 * (L.v - (int64_t)L.maxv));
+  st.range_err |= L.esc && (raw >> 60) != 0;
+  uint32_t total;
+  st.x = escape_group_enc(x0, active, L.start, L.freq, L.rcp, raw & ((1ull << 60) - 1), L.esc,
+                          end, cursor0, total);
+  st.cursor = cursor0 + total;
+}
+
+// One warp codes one stream.  Per coded group k the loop runs, in this
+// order: group k+1's bucket read, group k's state update, group k+1's
+// reciprocal, then the copies for group k + kEncStage - 1 and the ring reads
+// of groups k+2 (symbols, row metadata) and k+3 (row index); group k's rare
+// escape path comes last.  Nothing in group k's state chain waits on a
+// memory access issued in the same iteration.
 template <typename SymT, bool IB0, bool WIDE>
 __device__ __forceinline__ void encode_stream_w32(const EncCtx &c, const StreamDesc &d,
                                                   const RowMeta *meta, const uint32_t *buckets,
                                                   uint32_t *stg, int64_t s) {
   constexpr bool kStageSym = sizeof(SymT) == 4;
+  constexpr int kS = kEncStage;
   const int lane = threadIdx.x & 31;
   uint32_t *end = reinterpret_cast<uint32_t *>(c.scratch + slot_end(c.g, d, s));
   const int32_t n = (int32_t)d.n;
@@ -181,62 +228,84 @@ __device__ __forceinline__ void encode_stream_w32(const EncCtx &c, const StreamD
   const uint32_t kmax = (uint32_t)c.K - 1u;
   const uint32_t above = 0xfffffffeu << lane;   // lanes > this lane
   uint32_t *stg_idx = stg;
-  uint32_t *stg_sym = stg + kStage * 32;
+  uint32_t *stg_sym = stg + kS * 32;
   WarpEnc st;
   st.x = kL;
   st.cursor = 0;
   st.rmax = 0;
   st.range_err = false;
 
-  // The k-th coded group (group G-1-k) lands in stage slot k mod kStage,
-  // copied kStage - 1 groups ahead; a lane without an element there copies
-  // element 0 (ignored).
+  // The k-th coded group (group G-1-k) lands in stage slot k mod kS, copied
+  // kS - 1 groups ahead.  Copies for groups past the end (and lanes without
+  // an element) read the stream's element 0, never used.  Narrow symbols are
+  // read with plain loads one group ahead of use, after an L2 prefetch issued
+  // with the copies.
   Stepper<WIDE> pl;
   pl.init(d.t, (G - 1) * 32 + lane);
-  Stepper<WIDE> pn = pl;  // narrow symbols: next group's position
+  Stepper<WIDE> pn = pl;  // narrow symbols: position of the next load
   auto issue = [&](int32_t ki) {
-    if (ki < G) {
-      const int32_t g = G - 1 - ki;
-      const int32_t rel = lane < n - g * 32 ? pl.rel : 0;
-      const int slot = (ki & (kStage - 1)) * 32 + lane;
-      cp_async4(stg_idx + slot, IB0 ? idx_s + rel : c.idx + ((base + rel) >> ib));
-      if (kStageSym) cp_async4(stg_sym + slot, sym_s + rel);
-      if (g > 0) pl.back(32);
-    }
+    const int32_t g = G - 1 - ki;
+    const int32_t rel = ki < G && lane < n - g * 32 ? pl.rel : 0;
+    const int slot = (ki & (kS - 1)) * 32 + lane;
+    cp_async4(stg_idx + slot, IB0 ? idx_s + rel : c.idx + ((base + rel) >> ib));
+    if (kStageSym) cp_async4(stg_sym + slot, sym_s + rel);
+    else prefetch_l2(sym_s + rel);
     cp_async_commit();
+    pl.back(32);
   };
+  auto ring = [&](int32_t ki) { return (ki & (kS - 1)) * 32 + lane; };
   auto meta_of = [&](uint32_t r) -> RowMeta {
     st.rmax = max(st.rmax, r);
     return row_meta(meta, min(r, kmax));
   };
-#pragma unroll
-  for (int32_t u = 0; u < kStage - 1; ++u) issue(u);
-  cp_async_wait<kStage - 2>();
-  RowMeta m = meta_of(stg_idx[lane]);
-  int32_t sv_next = 0;
-  if (!kStageSym) sv_next = SymIO<SymT>::load(sym_s, lane < n - (G - 1) * 32 ? pn.rel : 0);
-  for (int32_t k = 0; k < G; ++k) {
-    issue(k + kStage - 1);
-    cp_async_wait<kStage - 2>();  // coded groups up to k + 1 have landed
-    const int slot = (k & (kStage - 1)) * 32 + lane;
-    int32_t sv;
-    if (kStageSym) {
-      sv = (int32_t)stg_sym[slot];
-    } else {
-      sv = sv_next;
-      if (k + 1 < G) {
-        pn.back(32);
-        sv_next = SymIO<SymT>::load(sym_s, pn.rel);
-      }
-    }
-    // (after the last group the slot may hold another stream's data: unused)
-    const RowMeta mn = meta_of(k + 1 < G ? stg_idx[((k + 1) & (kStage - 1)) * 32 + lane] : 0u);
-    if (k > 0)
-      enc_group<true>(st, m, buckets, sv, true, above, end);
-    else
-      enc_group<false>(st, m, buckets, sv, lane < n - (G - 1) * 32, above, end);
-    m = mn;
+  // symbols of coded group ki (ki < G), from the ring or a plain load
+  auto sym_of = [&](int32_t ki) -> int32_t {
+    if (kStageSym) return (int32_t)stg_sym[ring(ki)];
+    const int32_t v = SymIO<SymT>::load(sym_s, ki < G ? pn.rel : 0);
+    pn.back(32);
+    return v;
+  };
+#pragma unroll 1
+  for (int32_t u = 0; u < kS - 1; ++u) issue(u);
+  cp_async_wait<kS - 4>();  // coded groups 0..2 have landed
+  // group G - 1 (coded first) may be partial
+  const bool active0 = lane < n - (G - 1) * 32;
+  int32_t s0;
+  if (kStageSym) {
+    s0 = sym_of(0);
+  } else {
+    s0 = SymIO<SymT>::load(sym_s, active0 ? pn.rel : 0);
+    pn.back(32);
   }
+  EncLook L = enc_look(enc_bucket(s0, meta_of(stg_idx[ring(0)]), buckets), active0);
+  int32_t s1 = G > 1 ? sym_of(1) : 0;
+  RowMeta m1 = meta_of(G > 1 ? stg_idx[ring(1)] : 0u);
+  uint32_t r2 = G > 2 ? stg_idx[ring(2)] : 0u;
+
+  auto step = [&](int32_t k, bool active, auto full) {
+    // group k+1's bucket (after the last group: row 0, unused)
+    const EncBucket b1 = enc_bucket(s1, m1, buckets);
+    // group k's state update
+    const uint64_t x0 = st.x;
+    const uint32_t c0 = st.cursor;
+    enc_group_fast<decltype(full)::value>(st, L, active, above, end);
+    // group k+1's reciprocal and escape ballot
+    const EncLook L1 = enc_look(b1, true);
+    // copies, then the ring reads two and three groups ahead
+    issue(k + kS - 1);
+    cp_async_wait<kS - 4>();  // coded groups up to k + 3 have landed
+    const int32_t s2 = k + 2 < G ? sym_of(k + 2) : 0;
+    const RowMeta m2 = meta_of(r2);
+    const uint32_t r3 = k + 3 < G ? stg_idx[ring(k + 3)] : 0u;
+    if (L.any_esc) enc_group_escape(st, x0, c0, L, active, end);
+    L = L1;
+    s1 = s2;
+    m1 = m2;
+    r2 = r3;
+  };
+  step(0, active0, std::false_type());
+#pragma unroll 2
+  for (int32_t k = 1; k < G; ++k) step(k, true, std::true_type());
   cp_async_wait<0>();
   if (__any_sync(kFull, st.rmax > kmax)) {
     if (lane == 0) report(c.status, RANS_ERR_INDEX, s);
@@ -248,8 +317,8 @@ __device__ __forceinline__ void encode_stream_w32(const EncCtx &c, const StreamD
   }
   // flush: lanes 31..0 push high then low, so lane 0's low word comes first
   const uint32_t kk = st.cursor + 2u * (31u - (uint32_t)lane);
-  end[-1 - (int64_t)kk] = (uint32_t)(st.x >> 32);
-  end[-2 - (int64_t)kk] = (uint32_t)st.x;
+  st_global(end - 1 - kk, (uint32_t)(st.x >> 32));
+  st_global(end - 2 - kk, (uint32_t)st.x);
   if (lane == 0) c.lens[s] = 4ull * (st.cursor + 64);
 }
 
@@ -351,7 +420,7 @@ __global__ void __launch_bounds__(W == 32 ? kEncThreads32 : kEncThreads1)
   if (W == 32) {
     const int warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
     uint32_t *stg = reinterpret_cast<uint32_t *>(smem + (SMEM ? c.meta_bytes + c.bucket_bytes : 0)) +
-                    warp * kStage * 32 * 2;
+                    warp * kEncStage * 32 * 2;
     for (int64_t k = blockIdx.x + (int64_t)gridDim.x * warp; k < c.g.S;
          k += (int64_t)gridDim.x * nw)
       encode_stream_w32_entry<SymT, IB0>(c, meta, buckets, stg, stream_of(c.g, k));
@@ -444,7 +513,7 @@ template <int W, typename SymT, bool SMEM, bool IB0>
 int launch_encode_t(const EncCtx &c, cudaStream_t st) {
   auto kern = encode_kernel<W, SymT, SMEM, IB0>;
   const uint32_t tab = SMEM ? c.meta_bytes + c.bucket_bytes : 0;
-  const uint32_t per_warp = W == 32 ? kStage * 32 * 4 * 2 : 0;
+  const uint32_t per_warp = W == 32 ? kEncStage * 32 * 4 * 2 : 0;
   uint32_t smem = tab;
   int dev = 0;
   cudaGetDevice(&dev);

@@ -34,10 +34,19 @@ constexpr unsigned kFull = 0xffffffffu;
 // row-local bucket holding the slot's first cumulative value and e1, e2
 // describe the bucket boundaries strictly inside the slot, as offsets from the
 // slot start minus one (255 = none):
-//   e1 <= e2: at most two boundaries; for c = cum mod w the bucket is
-//             lo + (c > e1) + (c > e2);
-//   e1 > e2:  three or more: e1 = 255 and e2 + 3 boundaries, counted by the
-//             warp (rare).
+//   e1 <= e2:         at most two boundaries; for c = cum mod w the bucket is
+//                     lo + (c > e1) + (c > e2);
+//   e1 = 255 > e2:    three or more, resolved by boundary bitmaps: the 24-bit
+//                     index p = lo | e2 << 16 (into the slot words) starts
+//                     max(1, w / 16) bitmap words, word k covering cumulative
+//                     values [16 k, 16 k + 16) of the slot as
+//                     bits | j << 16, where j is the bucket holding the first
+//                     value and bit i (1..15) marks a bucket starting i values
+//                     later; the bucket is j + popc(bits & (2^(i+1) - 1));
+//   255 > e1 > e2:    three or more with no bitmap room left (e2 + 3
+//                     boundaries): a short binary search over the starts.
+// Bitmap words follow the slots of all rows; the blob header counts the words
+// handed out and flags whether any slot fell back to searching.
 struct RowMeta {
   uint32_t bucket_base;  // index of the row's bucket 0 in the bucket words
   uint32_t maxv;         // escape bucket = cdf_length - 2
@@ -52,18 +61,22 @@ __device__ __forceinline__ const RowMeta &row_meta(const RowMeta *meta, uint32_t
 }
 
 constexpr uint32_t kHeaderBytes = 256;
+constexpr uint32_t kChunkUsedWord = 16;    // header word: bitmap words handed out
+constexpr uint32_t kSearchFlagWord = 17;   // header word: 1 if a slot searches
+constexpr uint32_t kMaxChunkIndex = 0xff0000u;  // bitmap indexes fit lo | e2 << 16
 constexpr int kMinQ = 8;
 constexpr int kMaxQ = 14;
 
 // Streaming inputs (row indexes, and int32 symbols when encoding) reach the
-// warp coders through a per-warp shared-memory ring of kStage groups filled
-// with cp.async: one counting barrier tracks every copy in flight, so the
+// warp coders through a per-warp shared-memory ring of groups filled with
+// cp.async: one counting barrier tracks every copy in flight, so the
 // registers' dependency barriers stay free for the serial state chain.
-constexpr int kStage = 8;
+constexpr int kDecStage = 8;       // decoder ring: 8 groups of row indexes
+constexpr int kEncStage = 16;      // encoder ring: 16 groups of indexes + symbols
 constexpr int kDecMaxWarps = 24;   // decoder CTA: up to 768 threads
-constexpr int kEncMaxWarps = 32;   // encoder CTA: up to 1024 threads
-constexpr uint32_t kDecStageBytes = kDecMaxWarps * kStage * 32 * 4;
-constexpr uint32_t kEncStageBytes = kEncMaxWarps * kStage * 32 * 4 * 2;
+constexpr int kEncMaxWarps = 24;   // encoder CTA: up to 768 threads
+constexpr uint32_t kDecStageBytes = kDecMaxWarps * kDecStage * 32 * 4;
+constexpr uint32_t kEncStageBytes = kEncMaxWarps * kEncStage * 32 * 4 * 2;
 
 __host__ __device__ inline uint64_t pad16(uint64_t b) { return (b + 15) & ~uint64_t(15); }
 
@@ -327,6 +340,14 @@ __device__ __forceinline__ void bulk_prefetch_l2(const char *lo, const char *hi,
   }
 }
 
+// Stores through the global state space (st.global), so that the compiler
+// knows they cannot touch shared memory and may move shared-memory loads
+// across them.
+__device__ __forceinline__ void st_global(uint32_t *p, uint32_t v) { __stcg(p, v); }
+__device__ __forceinline__ void st_global(int32_t *p, int32_t v) { __stcs(p, v); }
+__device__ __forceinline__ void st_global(int16_t *p, int16_t v) { __stcs(p, v); }
+__device__ __forceinline__ void st_global(uint8_t *p, uint8_t v) { __stcs(p, v); }
+
 // ------------------------------------------------------------- symbols --
 template <typename T> struct SymIO;
 template <> struct SymIO<int32_t> {
@@ -379,8 +400,10 @@ __device__ __forceinline__ void cp_async_wait() {
 //    classical "magic number" conversion);
 //  * x = xh 2^32 + xl is then formed with one fused multiply-add, rounded once
 //    (relative error <= 2^-53);
-//  * 1/f comes from the hardware reciprocal estimate refined by three
-//    Newton-Raphson steps r <- r + r (1 - f r) (relative error ~2^-52);
+//  * 1/f comes from the hardware reciprocal estimate refined by two
+//    Newton-Raphson steps r <- r + r (1 - f r), each of which squares the
+//    relative error (about 2^-52 after the second; a test divides exactly
+//    for every f at the largest x);
 //  * so q' = x * (1/f) is within 0.05 of the real quotient x/f; adding 2^52
 //    rounds it to the nearest integer, which is floor(x/f) or one more, read
 //    back from the low 52 bits of the sum;
@@ -395,7 +418,7 @@ __device__ __forceinline__ double freq_reciprocal(uint32_t f) {
   double r;
   asm("rcp.approx.ftz.f64 %0, %1;" : "=d"(r) : "d"(fd));
 #pragma unroll
-  for (int i = 0; i < 3; ++i) r = fma(r, fma(-fd, r, 1.0), r);
+  for (int i = 0; i < 2; ++i) r = fma(r, fma(-fd, r, 1.0), r);
   return r;
 }
 

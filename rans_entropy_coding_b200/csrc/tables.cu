@@ -6,9 +6,9 @@
 //  * pmf -> quantised CDF ("torch_ans 0.3.0", High-level API, init_params;
 //    FAQ: increasing positive integers up to 2^precision).
 //  * The decoder lookup table: the top q bits of the state's low 16 bits pick
-//    a slot that names the bucket directly or bounds a short search
-//    ("torch_ans 0.3.0", Usage: inverse-CDF decoding with a 2^q table and a
-//    bounded walk).
+//    a slot that resolves up to two bucket boundaries itself and points to
+//    boundary bitmaps when it holds more ("torch_ans 0.3.0", Usage:
+//    inverse-CDF decoding with a 2^q table instead of a search).
 //
 // One CUDA block quantises one row.  The steal step (every empty bucket takes
 // one unit from the narrowest bucket wider than 1, first on ties, in ascending
@@ -27,47 +27,31 @@ namespace rb {
 
 namespace {
 
-constexpr int kRowThreads = 256;
+constexpr int kRowThreads = 1024;
 
-// Block-wide sum / exclusive scan of a 64-bit value (kRowThreads threads).
+// Block-wide exclusive scan of a 64-bit value over kRowThreads threads (warp
+// shuffles, then one thread over the warp totals); *total gets the block sum.
 struct BlockScratch {
   unsigned long long warp[kRowThreads / 32];
   unsigned long long total;
+  unsigned long long aux;
 };
 
-__device__ unsigned long long block_sum(unsigned long long v, BlockScratch &sh) {
-  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(kFull, v, o);
-  __syncthreads();
-  if (lane == 0) sh.warp[wid] = v;
-  __syncthreads();
-  if (threadIdx.x == 0) {
-    unsigned long long t = 0;
-    for (int i = 0; i < kRowThreads / 32; ++i) t += sh.warp[i];
-    sh.total = t;
-  }
-  __syncthreads();
-  return sh.total;
-}
-
-// Returns the exclusive prefix of v over threads; *total gets the block sum.
 __device__ unsigned long long block_excl_scan(unsigned long long v, BlockScratch &sh,
                                               unsigned long long *total) {
   const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
   unsigned long long inc = v;
 #pragma unroll
   for (int o = 1; o < 32; o <<= 1) {
-    unsigned long long t = __shfl_up_sync(kFull, inc, o);
+    const unsigned long long t = __shfl_up_sync(kFull, inc, o);
     if (lane >= o) inc += t;
   }
-  __syncthreads();
   if (lane == 31) sh.warp[wid] = inc;
   __syncthreads();
   if (threadIdx.x == 0) {
     unsigned long long run = 0;
     for (int i = 0; i < kRowThreads / 32; ++i) {
-      unsigned long long w = sh.warp[i];
+      const unsigned long long w = sh.warp[i];
       sh.warp[i] = run;
       run += w;
     }
@@ -75,7 +59,15 @@ __device__ unsigned long long block_excl_scan(unsigned long long v, BlockScratch
   }
   __syncthreads();
   *total = sh.total;
-  return sh.warp[wid] + inc - v;
+  const unsigned long long ex = sh.warp[wid] + inc - v;
+  __syncthreads();  // every thread has read the scratch before anyone reuses it
+  return ex;
+}
+
+__device__ unsigned long long block_sum(unsigned long long v, BlockScratch &sh) {
+  unsigned long long t;
+  block_excl_scan(v, sh, &t);
+  return t;
 }
 
 // Scaled and rounded probability: round(p * 2^16) half away from zero, or
@@ -87,59 +79,51 @@ __device__ __forceinline__ long long scaled_freq(float p) {
   return (long long)r;
 }
 
-// Quantises n probabilities (pf(i), the last one the tail mass) into row[0..n]
-// of a CDF row.  Returns RANS_OK or RANS_ERR_TABLE (same value on every
-// thread).  row[1..n] holds first the rounded probabilities, then the bucket
-// widths, then the CDF.
+// Quantises n probabilities (the last one the tail mass) into row[0..n] of a
+// CDF row.  Returns RANS_OK or RANS_ERR_TABLE (same value on every thread).
+// Thread t owns the contiguous entries [t * per, (t + 1) * per): each pass
+// walks its own entries in order and block scans join the threads, three
+// scans in all.  row[1..n] holds first the rounded probabilities (written by
+// pf.eval), then the bucket widths, then the CDF.
 constexpr int kHistMax = 64;  // widths 2..kHistMax are histogrammed for the steal step
 
 template <class PF>
 __device__ int quantise_row(const PF &pf, int n, int32_t *row, BlockScratch &sh,
                             unsigned int *hist) {
-  // pass 1: rounded values (each probability evaluated once) and their total
-  unsigned long long local = 0;
+  const int per = (n + kRowThreads - 1) / kRowThreads;
+  const int i0 = min(n, (int)threadIdx.x * per), i1 = min(n, i0 + per);
+  // pass 1: rounded values, each probability evaluated once
   int bad = 0;
-  for (int i = threadIdx.x; i < n; i += kRowThreads) {
-    long long f = scaled_freq(pf(i));
-    if (f < 0) {
-      bad = 1;
-      f = 0;
-    }
-    local += (unsigned long long)f;
-    row[i + 1] = (int32_t)(uint32_t)f;
-  }
+  const unsigned long long local = pf.eval(i0, i1, row + 1, bad);
   for (int i = threadIdx.x; i <= kHistMax; i += kRowThreads) hist[i] = 0;
-  const unsigned long long T = block_sum(local, sh);
+  unsigned long long T;
+  const unsigned long long before = block_excl_scan(local, sh, &T);
   bad = __syncthreads_or(bad);
   if (bad || T == 0) return RANS_ERR_TABLE;
 
   // pass 2: widths of the rescaled running sum floor(2^16 c / T); count the
   // empty buckets and histogram the narrow ones
-  unsigned long long carry = 0, zl = 0;
-  for (int base = 0; base < n; base += kRowThreads) {
-    int i = base + threadIdx.x;
-    unsigned long long f = i < n ? (unsigned long long)(uint32_t)row[i + 1] : 0ull;
-    unsigned long long tot;
-    unsigned long long ex = block_excl_scan(f, sh, &tot) + carry;
-    if (i < n) {
-      unsigned long long c0 = ((unsigned long long)kTotal * ex) / T;
-      unsigned long long c1 = ((unsigned long long)kTotal * (ex + f)) / T;
-      const uint32_t w = (uint32_t)(c1 - c0);
+  unsigned long long zl = 0;
+  {
+    unsigned long long c = before;
+    unsigned long long b0 = ((unsigned long long)kTotal * c) / T;
+    for (int i = i0; i < i1; ++i) {
+      c += (uint32_t)row[i + 1];
+      const unsigned long long b1 = ((unsigned long long)kTotal * c) / T;
+      const uint32_t w = (uint32_t)(b1 - b0);
+      b0 = b1;
       row[i + 1] = (int32_t)w;
       zl += (w == 0);
       if (w >= 2 && w <= kHistMax) atomicAdd(&hist[w], 1u);
     }
-    carry += tot;
   }
   const unsigned long long Z = block_sum(zl, sh);
   if (Z > 0) {
     // The Z units come from the buckets in (width, index) order, each drained
     // to width 1: find the threshold width t, the smallest with
     // S(t) = sum over 1 < w <= t of (w - 1) reaching Z.
-    long long t = 0;
-    unsigned long long below = 0;  // S(t - 1)
     if (threadIdx.x == 0) {
-      unsigned long long run = 0;
+      unsigned long long run = 0, t = 0, below = 0;
       for (int v = 2; v <= kHistMax; ++v) {
         const unsigned long long add = (unsigned long long)hist[v] * (unsigned long long)(v - 1);
         if (run + add >= Z) {
@@ -149,19 +133,19 @@ __device__ int quantise_row(const PF &pf, int n, int32_t *row, BlockScratch &sh,
         }
         run += add;
       }
-      sh.total = (unsigned long long)t;
-      sh.warp[0] = below;
+      sh.total = t;
+      sh.aux = below;
     }
     __syncthreads();
-    t = (long long)sh.total;
-    below = sh.warp[0];
+    long long t = (long long)sh.total;
+    unsigned long long below = sh.aux;
     __syncthreads();
     if (t == 0) {
-      // wider than the histogram: S(t) by block reductions, t by bisection
+      // wider than the histogram: S(t) by block sums, t by bisection
       auto S = [&](long long tt) -> unsigned long long {
         unsigned long long sacc = 0;
-        for (int i = threadIdx.x; i < n; i += kRowThreads) {
-          long long w = row[i + 1];
+        for (int i = i0; i < i1; ++i) {
+          const long long w = row[i + 1];
           if (w > 1 && w <= tt) sacc += (unsigned long long)(w - 1);
         }
         return block_sum(sacc, sh);
@@ -169,7 +153,7 @@ __device__ int quantise_row(const PF &pf, int n, int32_t *row, BlockScratch &sh,
       if (S(kTotal) < Z) return RANS_ERR_TABLE;
       long long lo = kHistMax + 1, hi = kTotal;
       while (lo < hi) {
-        long long mid = (lo + hi) >> 1;
+        const long long mid = (lo + hi) >> 1;
         if (S(mid) >= Z) hi = mid; else lo = mid + 1;
       }
       t = lo;
@@ -178,35 +162,33 @@ __device__ int quantise_row(const PF &pf, int n, int32_t *row, BlockScratch &sh,
     const unsigned long long R = Z - below;
     const unsigned long long full = R / (unsigned long long)(t - 1);
     const unsigned long long part = R % (unsigned long long)(t - 1);
-    unsigned long long rank_carry = 0;
-    for (int base = 0; base < n; base += kRowThreads) {
-      int i = base + threadIdx.x;
-      long long w = i < n ? row[i + 1] : 0;
-      unsigned long long tot;
-      unsigned long long rk = block_excl_scan(w == t ? 1ull : 0ull, sh, &tot) + rank_carry;
-      if (i < n) {
-        if (w > 1 && w < t) w = 1;
-        else if (w == t) {
-          if (rk < full) w = 1;
-          else if (rk == full) w -= (long long)part;
-        }
-        if (w == 0) w = 1;
-        row[i + 1] = (int32_t)w;
+    // rank of each width-t bucket among the width-t buckets, in index order
+    unsigned long long nt = 0;
+    for (int i = i0; i < i1; ++i) nt += row[i + 1] == t;
+    unsigned long long tot;
+    unsigned long long rk = block_excl_scan(nt, sh, &tot);
+    for (int i = i0; i < i1; ++i) {
+      long long w = row[i + 1];
+      if (w > 1 && w < t) {
+        w = 1;
+      } else if (w == t) {
+        if (rk < full) w = 1;
+        else if (rk == full) w -= (long long)part;
+        ++rk;
       }
-      rank_carry += tot;
+      if (w == 0) w = 1;
+      row[i + 1] = (int32_t)w;
     }
-    __syncthreads();
   }
 
   // widths -> CDF in place
-  unsigned long long run = 0;
-  for (int base = 0; base < n; base += kRowThreads) {
-    int i = base + threadIdx.x;
-    unsigned long long w = i < n ? (unsigned long long)row[i + 1] : 0ull;
-    unsigned long long tot;
-    unsigned long long ex = block_excl_scan(w, sh, &tot) + run;
-    if (i < n) row[i + 1] = (int32_t)(ex + w);
-    run += tot;
+  unsigned long long wl = 0;
+  for (int i = i0; i < i1; ++i) wl += (uint32_t)row[i + 1];
+  unsigned long long tot;
+  unsigned long long run = block_excl_scan(wl, sh, &tot);
+  for (int i = i0; i < i1; ++i) {
+    run += (uint32_t)row[i + 1];
+    row[i + 1] = (int32_t)run;
   }
   if (threadIdx.x == 0) row[0] = 0;
   __syncthreads();
@@ -238,15 +220,47 @@ __global__ void gaussian_lengths_kernel(const float *scales, int K, double tail,
   offsets[r] = st ? 0 : -c;
 }
 
+// Entry i < npmf of a Gaussian row is Phi((0.5 - d)/s) - Phi((-0.5 - d)/s)
+// with d = |i - center|, and entry npmf the tail mass 2 Phi((-0.5 - center)/s).
+// With u(d) = Phi((0.5 - d)/s) the entry is u(d) - u(d + 1) (the arguments
+// (-0.5 - d) and (0.5 - (d + 1)) are the same double), so a walk over
+// consecutive entries evaluates one new u per entry.
 struct GaussPmf {
   int center, npmf;
   double s;
-  __device__ float operator()(int i) const {
-    if (i == npmf) return (float)(2.0 * std_normal_cdf((-0.5 - (double)center) / s));
-    double d = fabs((double)(i - center));
-    double upper = std_normal_cdf((0.5 - d) / s);
-    double lower = std_normal_cdf((-0.5 - d) / s);
-    return (float)(upper - lower);
+  __device__ unsigned long long eval(int i0, int i1, int32_t *f, int &bad) const {
+    unsigned long long sum = 0;
+    int da = -1, db = -1;  // the two most recent u values
+    double ua = 0.0, ub = 0.0;
+    auto u = [&](int d) -> double {
+      if (d == da) return ua;
+      if (d == db) return ub;
+      const double v = std_normal_cdf((0.5 - (double)d) / s);
+      db = da;
+      ub = ua;
+      da = d;
+      ua = v;
+      return v;
+    };
+    for (int i = i0; i < i1; ++i) {
+      float p;
+      if (i == npmf) {
+        p = (float)(2.0 * std_normal_cdf((-0.5 - (double)center) / s));
+      } else {
+        const int d = abs(i - center);
+        const double hi = u(d);
+        const double lo = u(d + 1);
+        p = (float)(hi - lo);
+      }
+      long long q = scaled_freq(p);
+      if (q < 0) {
+        bad = 1;
+        q = 0;
+      }
+      f[i] = (int32_t)(uint32_t)q;
+      sum += (unsigned long long)q;
+    }
+    return sum;
   }
 };
 
@@ -254,7 +268,19 @@ struct GivenPmf {
   const float *p;
   int n;
   float tail;
-  __device__ float operator()(int i) const { return i == n ? tail : p[i]; }
+  __device__ unsigned long long eval(int i0, int i1, int32_t *f, int &bad) const {
+    unsigned long long sum = 0;
+    for (int i = i0; i < i1; ++i) {
+      long long q = scaled_freq(i == n ? tail : p[i]);
+      if (q < 0) {
+        bad = 1;
+        q = 0;
+      }
+      f[i] = (int32_t)(uint32_t)q;
+      sum += (unsigned long long)q;
+    }
+    return sum;
+  }
 };
 
 __global__ void __launch_bounds__(kRowThreads)
@@ -324,7 +350,62 @@ __global__ void pack_buckets_kernel(const int32_t *cdfs, int Lmax, const RowMeta
 }
 
 // Largest j in [0, nb) with row[j] <= v (row strictly increasing, row[0]=0).
-__device__ __forceinline__ int bucket_of(const int32_t *row, int nb, int v);
+__device__ __forceinline__ int bucket_of(const int32_t *row, int nb, int v) {
+  int lo = 0, hi = nb - 1;
+  while (lo < hi) {
+    int mid = (lo + hi + 1) >> 1;
+    if (row[mid] <= v) lo = mid; else hi = mid - 1;
+  }
+  return lo;
+}
+
+// Where a table set's bitmap words go: they follow the slots of all rows.
+struct ChunkArea {
+  uint32_t base;      // slot-word index of the first bitmap word
+  uint32_t cap;       // bitmap words available
+  uint32_t *used;     // header counter of words handed out
+  uint32_t *search;   // header flag: some slot fell back to searching
+};
+
+// Slot t of a row with nb buckets (row[0..nb], row[nb] = 65536) and slot
+// width 2^shift: writes its slot word and, for three or more boundaries, its
+// bitmap words (taken from the chunk area; a slot that finds it full keeps
+// the search form).
+__device__ void fill_slot(const int32_t *row, int nb, int t, int shift, uint32_t *slots,
+                          uint32_t index, const ChunkArea &ca) {
+  const int w = 1 << shift;
+  const int a = t * w, b = a + w - 1;
+  const int lo = bucket_of(row, nb, a);
+  const int inside = bucket_of(row, nb, b) - lo;
+  uint32_t word;
+  if (inside <= 2) {
+    uint32_t e1 = 255u, e2 = 255u;
+    if (inside >= 1) e1 = (uint32_t)(row[lo + 1] - a - 1);
+    if (inside == 2) e2 = (uint32_t)(row[lo + 2] - a - 1);
+    word = (uint32_t)lo | (e1 << 16) | (e2 << 24);
+  } else {
+    const uint32_t nch = w > 16 ? (uint32_t)(w >> 4) : 1u;
+    const uint32_t at = atomicAdd(ca.used, nch);
+    if (at <= ca.cap && nch <= ca.cap - at && ca.base + at + nch <= kMaxChunkIndex) {
+      const uint32_t p = ca.base + at;
+      int j = lo;
+      for (uint32_t k = 0; k < nch; ++k) {
+        const int c0 = a + 16 * (int)k;
+        const int c1 = c0 + 16 < a + w ? c0 + 16 : a + w;
+        while (row[j + 1] <= c0) ++j;  // bucket holding c0 (row[nb] > c0)
+        uint32_t bits = 0;
+        for (int i = j + 1; i < nb && row[i] < c1; ++i) bits |= 1u << (row[i] - c0);
+        slots[p + k] = bits | ((uint32_t)j << 16);
+      }
+      word = (p & 0xffffu) | (255u << 16) | ((p >> 16) << 24);
+    } else {
+      *ca.search = 1u;
+      const uint32_t e2 = (uint32_t)(inside - 3);
+      word = (uint32_t)lo | ((e2 + 1u) << 16) | (e2 << 24);
+    }
+  }
+  slots[index] = word;
+}
 
 // Rebuilds a prepared table set from new CDF rows with the same lengths:
 // block (x, r) fills slot chunk x of row r; block (0, r) also checks the
@@ -332,7 +413,8 @@ __device__ __forceinline__ int bucket_of(const int32_t *row, int nb, int v);
 // buckets.  Errors go to the blob's status word.
 __global__ void refresh_kernel(const int32_t *cdfs, int Lmax, const int32_t *lengths,
                                const int32_t *offsets, RowMeta *meta, uint32_t *buckets,
-                               uint16_t *starts, uint32_t *slots, int32_t *status) {
+                               uint16_t *starts, uint32_t *slots, ChunkArea ca,
+                               int32_t *status) {
   const int r = blockIdx.y;
   const RowMeta m = meta[r * kMetaCopies];
   const int len = lengths[r];
@@ -342,10 +424,12 @@ __global__ void refresh_kernel(const int32_t *cdfs, int Lmax, const int32_t *len
   }
   const int32_t *row = cdfs + (size_t)r * (size_t)Lmax;
   const int nb = len - 1;
+  if (row[0] != 0 || row[len - 1] != (int32_t)kTotal) {
+    if (threadIdx.x == 0 && blockIdx.x == 0) report(status, RANS_ERR_TABLE, r);
+    return;
+  }
   if (blockIdx.x == 0) {
     if (threadIdx.x < kMetaCopies) meta[r * kMetaCopies + threadIdx.x].offset = offsets[r];
-    if (threadIdx.x == 0 && (row[0] != 0 || row[len - 1] != (int32_t)kTotal))
-      report(status, RANS_ERR_TABLE, r);
     for (int j = threadIdx.x; j < nb; j += blockDim.x) {
       const int32_t a = row[j], b = row[j + 1];
       if (!(b > a) || a < 0 || b > (int32_t)kTotal) {
@@ -358,34 +442,14 @@ __global__ void refresh_kernel(const int32_t *cdfs, int Lmax, const int32_t *len
   }
   const int shift = (int)slot_shift(m.slot);
   const int nslots = 1 << (16 - shift);
-  const int w = 1 << shift;
-  for (int t = blockIdx.x * blockDim.x + threadIdx.x; t < nslots; t += gridDim.x * blockDim.x) {
-    const int a = t * w, b = a + w - 1;
-    const int lo = bucket_of(row, nb, a);
-    const int inside = bucket_of(row, nb, b) - lo;
-    uint32_t e1 = 255u, e2 = 255u;
-    if (inside >= 3) {
-      e2 = (uint32_t)(inside - 3);
-    } else {
-      if (inside >= 1) e1 = (uint32_t)(row[lo + 1] - a - 1);
-      if (inside == 2) e2 = (uint32_t)(row[lo + 2] - a - 1);
-    }
-    slots[slot_base(m.slot) + t] = (uint32_t)lo | (e1 << 16) | (e2 << 24);
-  }
+  for (int t = blockIdx.x * blockDim.x + threadIdx.x; t < nslots; t += gridDim.x * blockDim.x)
+    fill_slot(row, nb, t, shift, slots, slot_base(m.slot) + t, ca);
 }
 
-// Largest j in [0, nb) with row[j] <= v (row strictly increasing, row[0]=0).
-__device__ __forceinline__ int bucket_of(const int32_t *row, int nb, int v) {
-  int lo = 0, hi = nb - 1;
-  while (lo < hi) {
-    int mid = (lo + hi + 1) >> 1;
-    if (row[mid] <= v) lo = mid; else hi = mid - 1;
-  }
-  return lo;
-}
-
+// The slot fill of rans_tables_prepare (rows already validated by
+// pack_buckets_kernel; a malformed row only leaves its own slots undefined).
 __global__ void fill_slots_kernel(const int32_t *cdfs, int Lmax, const RowMeta *meta,
-                                  const int32_t *lengths, uint32_t *slots) {
+                                  const int32_t *lengths, uint32_t *slots, ChunkArea ca) {
   const int r = blockIdx.y;
   const RowMeta m = meta[r * kMetaCopies];
   const int shift = (int)slot_shift(m.slot);
@@ -393,19 +457,9 @@ __global__ void fill_slots_kernel(const int32_t *cdfs, int Lmax, const RowMeta *
   const int t = blockIdx.x * blockDim.x + threadIdx.x;
   if (t >= nslots) return;
   const int32_t *row = cdfs + (size_t)r * (size_t)Lmax;
-  const int nb = lengths[r] - 1;
-  const int w = 1 << shift;
-  const int a = t * w, b = a + w - 1;
-  const int lo = bucket_of(row, nb, a);
-  const int inside = bucket_of(row, nb, b) - lo;
-  uint32_t e1 = 255u, e2 = 255u;
-  if (inside >= 3) {
-    e2 = (uint32_t)(inside - 3);
-  } else {
-    if (inside >= 1) e1 = (uint32_t)(row[lo + 1] - a - 1);
-    if (inside == 2) e2 = (uint32_t)(row[lo + 2] - a - 1);
-  }
-  slots[slot_base(m.slot) + t] = (uint32_t)lo | (e1 << 16) | (e2 << 24);
+  const int len = lengths[r];
+  if (row[0] != 0 || row[len - 1] != (int32_t)kTotal) return;
+  fill_slot(row, len - 1, t, shift, slots, slot_base(m.slot) + t, ca);
 }
 
 int ceil_log2(int64_t v) {
@@ -449,23 +503,32 @@ int refresh_tables(const int32_t *cdfs, int K, int Lmax, const int32_t *lengths,
       reinterpret_cast<uint16_t *>(b + kHeaderBytes + t.meta_bytes + t.bucket_bytes);
   uint32_t *dslots = reinterpret_cast<uint32_t *>(b + kHeaderBytes + t.meta_bytes +
                                                   t.bucket_bytes + t.start_bytes);
+  ChunkArea ca;
+  ca.base = (uint32_t)t.n_slots;
+  ca.cap = t.slot_bytes / 4 - (uint32_t)t.n_slots;
+  ca.used = reinterpret_cast<uint32_t *>(b) + kChunkUsedWord;
+  ca.search = reinterpret_cast<uint32_t *>(b) + kSearchFlagWord;
+  if (cudaMemsetAsync(ca.used, 0, 8, st) != cudaSuccess) return RANS_ERR_CUDA;
   // slot chunks of 256: the largest row has at most 2^14 slots
   int64_t maxslots = 1;
   while (maxslots * K < t.n_slots && maxslots < (1 << kMaxQ)) maxslots <<= 1;
   dim3 grid((unsigned)((maxslots + 255) / 256), (unsigned)K);
   refresh_kernel<<<grid, 256, 0, st>>>(cdfs, Lmax, lengths, offsets, dmeta, dbuckets, dstarts,
-                                       dslots, status);
+                                       dslots, ca, status);
   return cudaGetLastError() == cudaSuccess ? RANS_OK : RANS_ERR_CUDA;
 }
 
+// Room for the slots and bitmap words: the slots of every row at the largest
+// q, as many bitmap words again, and 256 KB (shared-memory tables plan up to
+// a quarter of their slot room as bitmap words; tables read from global
+// memory as many words as slots).
 uint64_t tables_bytes_bound(int K, int Lmax) {
   if (K <= 0 || Lmax < 2) return 0;
   const int64_t nb = (int64_t)Lmax - 1;
   int q = ceil_log2(nb);
   q = q < kMinQ ? kMinQ : (q > kMaxQ ? kMaxQ : q);
   return (uint64_t)kHeaderBytes + pad16(16ull * kMetaCopies * K) + pad16(4ull * K * nb) +
-         pad16(2ull * K * nb + 2) +
-         pad16(4ull * K * (1ull << q));
+         pad16(2ull * K * nb + 2) + pad16(8ull * K * (1ull << q)) + 262144ull;
 }
 
 int prepare_tables(const int32_t *cdfs, int K, int Lmax, const int32_t *lengths,
@@ -513,19 +576,22 @@ int prepare_tables(const int32_t *cdfs, int K, int Lmax, const int32_t *lengths,
   };
   const bool enc_smem = (int64_t)meta_bytes + bucket_bytes + kEncStageBytes <= budget;
   bool dec_smem = false;
+  uint64_t chunk_words = 0;
   if ((int64_t)meta_bytes + start_bytes + kDecStageBytes <= budget) {
     const int64_t room = budget - meta_bytes - start_bytes - kDecStageBytes;
-    // About one slot per bucket (fewer than ~2% of lookups then meet three or
-    // more boundaries on the scale table); halve the largest row's lookup
-    // until the three sections fit.
-    while ((int64_t)pad16(4ull * slot_total()) > room) {
+    // About one slot per bucket; halve the largest row's lookup until the
+    // slots take at most three quarters of the room, the rest going to
+    // bitmap words.
+    while ((int64_t)pad16(4ull * slot_total()) > room - room / 4) {
       int best = -1;
       for (int r = 0; r < K; ++r)
         if (q[r] > kMinQ && (best < 0 || q[r] >= q[best])) best = r;
       if (best < 0) break;
       --q[best];
     }
-    dec_smem = (int64_t)pad16(4ull * slot_total()) <= room;
+    const int64_t left = room - (int64_t)pad16(4ull * slot_total());
+    dec_smem = left >= 0;
+    if (dec_smem) chunk_words = (uint64_t)(left / 16) * 4;
   }
   uint64_t sbase = 0;
   for (int r = 0; r < K; ++r) {
@@ -533,9 +599,15 @@ int prepare_tables(const int32_t *cdfs, int K, int Lmax, const int32_t *lengths,
     sbase += 1ull << q[r];
   }
   if (sbase >= (1ull << 27)) return RANS_ERR_ARG;
-  const uint32_t slot_bytes = (uint32_t)pad16(4ull * sbase);
+  if (!dec_smem) chunk_words = sbase;
+  const uint64_t base_need = (uint64_t)kHeaderBytes + meta_bytes + bucket_bytes + start_bytes +
+                             pad16(4ull * sbase);
+  if (blob == nullptr || blob_bytes < base_need) return RANS_ERR_CAPACITY;
+  // a smaller blob gets fewer bitmap words (slots then search instead)
+  if (base_need + 4ull * chunk_words > blob_bytes)
+    chunk_words = ((blob_bytes - base_need) / 16) * 4;
+  const uint32_t slot_bytes = (uint32_t)pad16(4ull * (sbase + chunk_words));
   const uint64_t need = (uint64_t)kHeaderBytes + meta_bytes + bucket_bytes + start_bytes + slot_bytes;
-  if (blob == nullptr || blob_bytes < need) return RANS_ERR_CAPACITY;
   if ((reinterpret_cast<uintptr_t>(blob) & 255) != 0) return RANS_ERR_ARG;
 
   char *b = reinterpret_cast<char *>(blob);
@@ -558,7 +630,12 @@ int prepare_tables(const int32_t *cdfs, int K, int Lmax, const int32_t *lengths,
   int maxslots = 0;
   for (int r = 0; r < K; ++r) maxslots = maxslots > (1 << q[r]) ? maxslots : (1 << q[r]);
   dim3 grid((maxslots + 255) / 256, K);
-  fill_slots_kernel<<<grid, 256, 0, st>>>(cdfs, Lmax, dmeta, lengths, dslots);
+  ChunkArea ca;
+  ca.base = (uint32_t)sbase;
+  ca.cap = (uint32_t)(slot_bytes / 4 - sbase);
+  ca.used = reinterpret_cast<uint32_t *>(b) + kChunkUsedWord;
+  ca.search = reinterpret_cast<uint32_t *>(b) + kSearchFlagWord;
+  fill_slots_kernel<<<grid, 256, 0, st>>>(cdfs, Lmax, dmeta, lengths, dslots, ca);
   if (cudaGetLastError() != cudaSuccess) return RANS_ERR_CUDA;
   StatusWord sw;
   if (cudaMemcpyAsync(&sw, status, sizeof(sw), cudaMemcpyDeviceToHost, st) != cudaSuccess ||

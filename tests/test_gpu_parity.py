@@ -323,6 +323,50 @@ def test_encoder_reports_bad_index_and_capacity():
     assert st == rb.ERR_CAPACITY
 
 
+def _header(tables):
+    """The blob header's words (an internal layout: word 16 counts the bitmap
+    words handed out, word 17 flags slots that search)."""
+    return tables.blob[:256].view(torch.int32).cpu().numpy()
+
+
+@pytest.mark.parametrize("W", [1, 32])
+def test_slots_without_bitmap_room_search(W):
+    """Prepared in a blob with no room for boundary bitmaps, the slots that
+    hold three or more boundaries fall back to a search: same symbols."""
+    w = WL.y_latent()
+    w["W"] = W
+    c, l, o = oracle_tables(w)
+    full = tables_from_numpy(c, l, o)
+    h = _header(full)
+    assert h[16] > 0 and h[17] == 0 and full.c.dec_in_smem == 1
+    spare = full.c.slot_bytes - 4 * full.c.n_slots
+    assert spare >= 4 * h[16]
+    dev = lambda a: torch.from_numpy(np.ascontiguousarray(a)).cuda()
+    tight = rb.Tables(dev(c), dev(l), dev(o), blob_bytes=full.c.blob_bytes - spare)
+    assert tight.c.slot_bytes == 4 * tight.c.n_slots
+    assert _header(tight)[17] == 1
+    data, offs, dec, _, _ = gpu_encode_decode(w, tight)
+    want, woffs = oracle_encode(w, c, l, o)
+    assert offs.tolist() == woffs.tolist() and np.array_equal(data, want)
+    assert np.array_equal(dec, np.asarray(w["symbols"]).reshape(-1))
+    # a refresh from the same rows keeps the fallback and the results
+    rb.check(rb.rans_tables_refresh(dev(c), dev(l), dev(o), tight))
+    assert rb.rans_get_status(tight.blob) == rb.OK and _header(tight)[17] == 1
+    _, _, dec2, _, _ = gpu_encode_decode(w, tight)
+    assert np.array_equal(dec2, np.asarray(w["symbols"]).reshape(-1))
+
+
+@pytest.mark.parametrize("W", [1, 32])
+def test_tables_too_large_for_shared_memory(W):
+    """256 Gaussian rows (0.4 MB of bucket words): both coders read the tables
+    from global memory."""
+    w = WL.many_rows(W=W)
+    c, l, o = oracle_tables(w)
+    tables = tables_from_numpy(c, l, o)
+    assert tables.c.enc_in_smem == 0 and tables.c.dec_in_smem == 0
+    _check_streams(w)
+
+
 def test_table_refresh_matches_fresh_prepare():
     """A prepared table set refreshed from new rows of the same lengths codes
     exactly like one prepared from those rows."""

@@ -120,6 +120,20 @@ def _y_image(seed):
     return sym, idx
 
 
+def many_rows(seed=5000, n=1 << 18, n_rows=256, n_streams=64, W=32):
+    """The y recipe over a finer scale table (n_rows rows from 0.11 to 256):
+    about 0.4 MB of bucket words, more than one CUDA block's shared memory holds."""
+    rng = _rng(seed)
+    lo, hi = math.log(SCALE_MIN), math.log(SCALE_MAX_Y)
+    u = rng.uniform(lo, hi, size=n)
+    step = (hi - lo) / (n_rows - 1)
+    idx = np.clip(np.rint((u - lo) / step), 0, n_rows - 1).astype(np.int32)
+    sym = np.rint(rng.standard_normal(n) * np.exp(u)).astype(np.int32)
+    return dict(name="many_rows", symbols=sym, indexes=idx,
+                scales=log_spaced_scales(SCALE_MIN, SCALE_MAX_Y, n_rows), tail_mass=1e-9,
+                chunking=dict(kind="contig", n_streams=n_streams), W=W, index_block=1)
+
+
 def y_latent(seed=2000, W=1):
     sym, idx = _y_image(seed)
     return dict(name="y", symbols=sym.reshape((1,) + Y_SHAPE), indexes=idx,
