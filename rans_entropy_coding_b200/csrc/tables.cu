@@ -82,27 +82,45 @@ __device__ __forceinline__ long long scaled_freq(float p) {
 // Quantises n probabilities (the last one the tail mass) into row[0..n] of a
 // CDF row.  Returns RANS_OK or RANS_ERR_TABLE (same value on every thread).
 // Thread t owns the contiguous entries [t * per, (t + 1) * per): each pass
-// walks its own entries in order and block scans join the threads, three
-// scans in all.  row[1..n] holds first the rounded probabilities (written by
-// pf.eval), then the bucket widths, then the CDF.
-constexpr int kHistMax = 64;  // widths 2..kHistMax are histogrammed for the steal step
+// walks its own entries in order and block scans join the threads.  row[1..n]
+// holds first the rounded probabilities (written by pf.eval), then the bucket
+// widths, then the CDF.
+//
+// The steal step in closed form: the Z units that the empty buckets take
+// come from the buckets in (width, index) order, each drained to width 1
+// before the next is touched.  So with S(t) = sum over buckets of width
+// 1 < w <= t of (w - 1), the threshold t is the smallest width with
+// S(t) >= Z: buckets narrower than t end at width 1, and of the width-t
+// buckets (in index order) the first floor(R / (t - 1)) end at 1 and the
+// next gives up R mod (t - 1) units, R = Z - S(t - 1).  Widths below kBins
+// are counted in a histogram (one bin per thread, so one scan finds t); the
+// wider ones, at most 2^16 / kBins of them, are kept in a list.
+constexpr int kBins = kRowThreads;
+constexpr int kBigMax = 65536 / kBins;
+
+struct QuantScratch {
+  unsigned int hist[kBins];
+  unsigned int big[kBigMax];
+  unsigned int nbig;
+};
 
 template <class PF>
 __device__ int quantise_row(const PF &pf, int n, int32_t *row, BlockScratch &sh,
-                            unsigned int *hist) {
+                            QuantScratch &q) {
   const int per = (n + kRowThreads - 1) / kRowThreads;
   const int i0 = min(n, (int)threadIdx.x * per), i1 = min(n, i0 + per);
   // pass 1: rounded values, each probability evaluated once
   int bad = 0;
   const unsigned long long local = pf.eval(i0, i1, row + 1, bad);
-  for (int i = threadIdx.x; i <= kHistMax; i += kRowThreads) hist[i] = 0;
+  q.hist[threadIdx.x] = 0;
+  if (threadIdx.x == 0) q.nbig = 0;
   unsigned long long T;
   const unsigned long long before = block_excl_scan(local, sh, &T);
   bad = __syncthreads_or(bad);
   if (bad || T == 0) return RANS_ERR_TABLE;
 
   // pass 2: widths of the rescaled running sum floor(2^16 c / T); count the
-  // empty buckets and histogram the narrow ones
+  // empty buckets and the widths of the others
   unsigned long long zl = 0;
   {
     unsigned long long c = before;
@@ -114,51 +132,43 @@ __device__ int quantise_row(const PF &pf, int n, int32_t *row, BlockScratch &sh,
       b0 = b1;
       row[i + 1] = (int32_t)w;
       zl += (w == 0);
-      if (w >= 2 && w <= kHistMax) atomicAdd(&hist[w], 1u);
+      if (w >= 2 && w < (uint32_t)kBins) atomicAdd(&q.hist[w], 1u);
+      else if (w >= (uint32_t)kBins) q.big[atomicAdd(&q.nbig, 1u)] = w;
     }
   }
-  const unsigned long long Z = block_sum(zl, sh);
+  const unsigned long long Z = block_sum(zl, sh);  // (its barriers also publish q)
   if (Z > 0) {
-    // The Z units come from the buckets in (width, index) order, each drained
-    // to width 1: find the threshold width t, the smallest with
-    // S(t) = sum over 1 < w <= t of (w - 1) reaching Z.
-    if (threadIdx.x == 0) {
-      unsigned long long run = 0, t = 0, below = 0;
-      for (int v = 2; v <= kHistMax; ++v) {
-        const unsigned long long add = (unsigned long long)hist[v] * (unsigned long long)(v - 1);
-        if (run + add >= Z) {
-          t = v;
-          below = run;
-          break;
-        }
-        run += add;
+    // t below kBins: the bin whose running S(t) first reaches Z
+    const unsigned int b = threadIdx.x;
+    const unsigned long long vb = b >= 2 ? (unsigned long long)(b - 1) * q.hist[b] : 0ull;
+    unsigned long long s_all;
+    const unsigned long long sb = block_excl_scan(vb, sh, &s_all);  // S(b - 1)
+    if (threadIdx.x == 0) sh.total = 0;
+    __syncthreads();
+    if (vb > 0 && sb < Z && sb + vb >= Z) {
+      sh.total = b;
+      sh.aux = sb;
+    }
+    // t among the wide buckets: the smallest listed width whose S reaches Z
+    const unsigned int nbig = q.nbig;
+    if (s_all < Z && b < nbig) {
+      const unsigned int wb = q.big[b];
+      unsigned long long s_le = s_all, s_lt = s_all;  // S(wb), S(wb - 1)
+      for (unsigned int k = 0; k < nbig; ++k) {
+        const unsigned int wk = q.big[k];
+        if (wk <= wb) s_le += wk - 1;
+        if (wk < wb) s_lt += wk - 1;
       }
-      sh.total = t;
-      sh.aux = below;
+      if (s_le >= Z && s_lt < Z) {  // every bucket of the smallest such width agrees
+        sh.total = wb;
+        sh.aux = s_lt;
+      }
     }
     __syncthreads();
-    long long t = (long long)sh.total;
-    unsigned long long below = sh.aux;
+    const long long t = (long long)sh.total;
+    const unsigned long long below = sh.aux;
     __syncthreads();
-    if (t == 0) {
-      // wider than the histogram: S(t) by block sums, t by bisection
-      auto S = [&](long long tt) -> unsigned long long {
-        unsigned long long sacc = 0;
-        for (int i = i0; i < i1; ++i) {
-          const long long w = row[i + 1];
-          if (w > 1 && w <= tt) sacc += (unsigned long long)(w - 1);
-        }
-        return block_sum(sacc, sh);
-      };
-      if (S(kTotal) < Z) return RANS_ERR_TABLE;
-      long long lo = kHistMax + 1, hi = kTotal;
-      while (lo < hi) {
-        const long long mid = (lo + hi) >> 1;
-        if (S(mid) >= Z) hi = mid; else lo = mid + 1;
-      }
-      t = lo;
-      below = S(t - 1);
-    }
+    if (t == 0) return RANS_ERR_TABLE;  // nothing left to steal from
     const unsigned long long R = Z - below;
     const unsigned long long full = R / (unsigned long long)(t - 1);
     const unsigned long long part = R % (unsigned long long)(t - 1);
@@ -287,7 +297,7 @@ __global__ void __launch_bounds__(kRowThreads)
     gaussian_rows_kernel(const float *scales, double tail, int32_t *cdfs, int Lmax,
                          int32_t *lengths, int32_t *offsets) {
   __shared__ BlockScratch sh;
-  __shared__ unsigned int hist[kHistMax + 1];
+  __shared__ QuantScratch qs;
   const int r = blockIdx.x;
   int32_t *row = cdfs + (size_t)r * (size_t)Lmax;
   int32_t c = 0;
@@ -296,7 +306,7 @@ __global__ void __launch_bounds__(kRowThreads)
   if (st == RANS_OK && len > Lmax) st = RANS_ERR_CAPACITY;
   if (st == RANS_OK) {
     GaussPmf pf{c, 2 * c + 1, (double)scales[r]};
-    st = quantise_row(pf, 2 * c + 2, row, sh, hist);
+    st = quantise_row(pf, 2 * c + 2, row, sh, qs);
   }
   for (int j = (st == RANS_OK ? len : 0) + threadIdx.x; j < Lmax; j += kRowThreads) row[j] = 0;
   if (threadIdx.x == 0) {
@@ -309,7 +319,7 @@ __global__ void __launch_bounds__(kRowThreads)
     pmf_rows_kernel(const float *pmfs, int stride, const int32_t *pmf_lengths,
                     const float *tail, int32_t *cdfs, int Lmax, int32_t *lengths) {
   __shared__ BlockScratch sh;
-  __shared__ unsigned int hist[kHistMax + 1];
+  __shared__ QuantScratch qs;
   const int r = blockIdx.x;
   int32_t *row = cdfs + (size_t)r * (size_t)Lmax;
   int n = pmf_lengths[r];
@@ -318,7 +328,7 @@ __global__ void __launch_bounds__(kRowThreads)
   else if (n + 2 > Lmax) st = RANS_ERR_CAPACITY;
   if (st == RANS_OK) {
     GivenPmf pf{pmfs + (size_t)r * (size_t)stride, n, tail[r]};
-    st = quantise_row(pf, n + 1, row, sh, hist);
+    st = quantise_row(pf, n + 1, row, sh, qs);
   }
   for (int j = (st == RANS_OK ? n + 2 : 0) + threadIdx.x; j < Lmax; j += kRowThreads) row[j] = 0;
   if (threadIdx.x == 0) lengths[r] = st ? st : n + 2;
@@ -367,54 +377,129 @@ struct ChunkArea {
   uint32_t *search;   // header flag: some slot fell back to searching
 };
 
-// Slot t of a row with nb buckets (row[0..nb], row[nb] = 65536) and slot
-// width 2^shift: writes its slot word and, for three or more boundaries, its
-// bitmap words (taken from the chunk area; a slot that finds it full keeps
-// the search form).
-__device__ void fill_slot(const int32_t *row, int nb, int t, int shift, uint32_t *slots,
-                          uint32_t index, const ChunkArea &ca) {
-  const int w = 1 << shift;
-  const int a = t * w, b = a + w - 1;
-  const int lo = bucket_of(row, nb, a);
-  const int inside = bucket_of(row, nb, b) - lo;
-  uint32_t word;
-  if (inside <= 2) {
-    uint32_t e1 = 255u, e2 = 255u;
-    if (inside >= 1) e1 = (uint32_t)(row[lo + 1] - a - 1);
-    if (inside == 2) e2 = (uint32_t)(row[lo + 2] - a - 1);
-    word = (uint32_t)lo | (e1 << 16) | (e2 << 24);
-  } else {
-    const uint32_t nch = w > 16 ? (uint32_t)(w >> 4) : 1u;
-    const uint32_t at = atomicAdd(ca.used, nch);
-    if (at <= ca.cap && nch <= ca.cap - at && ca.base + at + nch <= kMaxChunkIndex) {
-      const uint32_t p = ca.base + at;
-      int j = lo;
-      for (uint32_t k = 0; k < nch; ++k) {
-        const int c0 = a + 16 * (int)k;
-        const int c1 = c0 + 16 < a + w ? c0 + 16 : a + w;
-        while (row[j + 1] <= c0) ++j;  // bucket holding c0 (row[nb] > c0)
-        uint32_t bits = 0;
-        for (int i = j + 1; i < nb && row[i] < c1; ++i) bits |= 1u << (row[i] - c0);
-        slots[p + k] = bits | ((uint32_t)j << 16);
-      }
-      word = (p & 0xffffu) | (255u << 16) | ((p >> 16) << 24);
-    } else {
-      *ca.search = 1u;
-      const uint32_t e2 = (uint32_t)(inside - 3);
-      word = (uint32_t)lo | ((e2 + 1u) << 16) | (e2 << 24);
+// Slots are filled kSlotsPerThread consecutive ones per thread, each from
+// two binary searches (the buckets holding its first and last cumulative
+// values), so no thread's work depends on how the buckets fall.  A block
+// covers kSlotsPerBlock slots of one row and stages the row in shared
+// memory when it has at most kRowSmem entries.
+constexpr int kSlotThreads = 256;
+constexpr int kSlotsPerThread = 4;
+constexpr int kSlotsPerBlock = kSlotThreads * kSlotsPerThread;
+constexpr int kRowSmem = 8192;
+constexpr uint32_t kSlotSmemBytes = 4u * kRowSmem;
+
+// The bitmap word of the 16 cumulative values [c0, c0 + 16) cut to [c0, c1),
+// given jj, the bucket holding c0: bit i marks a bucket starting at c0 + i.
+// The row is strictly increasing, so the buckets starting inside are
+// jj + 1 .. jj + 15 at most and their loads do not wait on one another.
+__device__ __forceinline__ uint32_t boundary_bits(const int32_t *row, int nb, int jj, int c0,
+                                                  int c1) {
+  uint32_t bits = 0;
+#pragma unroll
+  for (int u = 1; u <= 15; ++u) {
+    const int i = jj + u;
+    const int v = i < nb ? row[i] : (int)kTotal;
+    if (v < c1) bits |= 1u << ((v - c0) & 31);
+  }
+  return bits;
+}
+
+// The slots [tb, tb + kSlotsPerBlock) of a row (row in shared or global
+// memory).
+__device__ void fill_slot_block(const int32_t *row, int nb, uint32_t slot0, int w, int nslots,
+                                int tb, uint32_t *slots, const ChunkArea &ca) {
+  const int lane = threadIdx.x & 31;
+  const int t0 = tb + (int)threadIdx.x * kSlotsPerThread;
+  const uint32_t nch = w > 16 ? (uint32_t)(w >> 4) : 1u;  // bitmap words of a slot
+  int lo[kSlotsPerThread], hi[kSlotsPerThread];
+  uint32_t need = 0;
+#pragma unroll
+  for (int u = 0; u < kSlotsPerThread; ++u) {
+    const int t = t0 + u;
+    lo[u] = hi[u] = 0;
+    if (t < nslots) {
+      lo[u] = bucket_of(row, nb, t * w);
+      hi[u] = bucket_of(row, nb, t * w + w - 1);
+      if (hi[u] - lo[u] >= 3) need += nch;
     }
   }
-  slots[index] = word;
+  // bitmap words: one allocation per warp
+  uint32_t incl = need;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const uint32_t v = __shfl_up_sync(kFull, incl, o);
+    if (lane >= o) incl += v;
+  }
+  const uint32_t wtot = __shfl_sync(kFull, incl, 31);
+  uint32_t wbase = 0;
+  if (lane == 31 && wtot > 0) wbase = atomicAdd(ca.used, wtot);
+  uint32_t at = __shfl_sync(kFull, wbase, 31) + incl - need;
+#pragma unroll
+  for (int u = 0; u < kSlotsPerThread; ++u) {
+    const int t = t0 + u;
+    if (t >= nslots) continue;
+    const int a = t * w;
+    const int inside = hi[u] - lo[u];
+    uint32_t word;
+    if (inside <= 2) {
+      uint32_t e1 = 255u, e2 = 255u;
+      if (inside >= 1) e1 = (uint32_t)(row[lo[u] + 1] - a - 1);
+      if (inside == 2) e2 = (uint32_t)(row[lo[u] + 2] - a - 1);
+      word = (uint32_t)lo[u] | (e1 << 16) | (e2 << 24);
+    } else {
+      if (at <= ca.cap && nch <= ca.cap - at && ca.base + at + nch <= kMaxChunkIndex) {
+        const uint32_t p = ca.base + at;
+        int jj = lo[u];  // bucket holding the word's first value
+        for (uint32_t k = 0; k < nch; ++k) {
+          const int c0 = a + 16 * (int)k;
+          const int c1 = c0 + 16 < a + w ? c0 + 16 : a + w;
+          const uint32_t bits = boundary_bits(row, nb, jj, c0, c1);
+          slots[p + k] = bits | ((uint32_t)jj << 16);
+          // the bucket holding c0 + 16: past the boundaries inside, and one
+          // more if a bucket starts exactly there
+          jj += __popc(bits);
+          if (jj + 1 < nb && row[jj + 1] == c0 + 16) ++jj;
+        }
+        word = (p & 0xffffu) | (255u << 16) | ((p >> 16) << 24);
+      } else {
+        *ca.search = 1u;
+        const uint32_t e2 = (uint32_t)(inside - 3);
+        word = (uint32_t)lo[u] | ((e2 + 1u) << 16) | (e2 << 24);
+      }
+      at += nch;
+    }
+    slots[slot0 + t] = word;
+  }
+}
+
+// Slot words (and bitmap words) of a row with nb buckets, blocks x, x +
+// gridDim.x, ... of kSlotsPerBlock slots; grow[0..nb] is the row (grow[0] =
+// 0, grow[nb] = 65536), shift the row's slot width log2.  Every thread of
+// the block must call it.
+__device__ void fill_row_slots(const int32_t *grow, int nb, uint32_t slot0, int shift,
+                               uint32_t *slots, const ChunkArea &ca, int32_t *srow) {
+  const int nslots = 1 << (16 - shift);
+  const int w = 1 << shift;
+  if ((int)blockIdx.x * kSlotsPerBlock >= nslots) return;  // (the whole block)
+  const int32_t *row = grow;
+  if (nb + 1 <= kRowSmem) {
+    for (int i = threadIdx.x; i <= nb; i += blockDim.x) srow[i] = grow[i];
+    __syncthreads();
+    row = srow;
+  }
+  for (int tb = blockIdx.x * kSlotsPerBlock; tb < nslots; tb += gridDim.x * kSlotsPerBlock)
+    fill_slot_block(row, nb, slot0, w, nslots, tb, slots, ca);
 }
 
 // Rebuilds a prepared table set from new CDF rows with the same lengths:
-// block (x, r) fills slot chunk x of row r; block (0, r) also checks the
+// block (x, r) fills slot block x of row r; block (0, r) also checks the
 // row's length against the layout, refreshes its offset and packs its
 // buckets.  Errors go to the blob's status word.
-__global__ void refresh_kernel(const int32_t *cdfs, int Lmax, const int32_t *lengths,
-                               const int32_t *offsets, RowMeta *meta, uint32_t *buckets,
-                               uint16_t *starts, uint32_t *slots, ChunkArea ca,
-                               int32_t *status) {
+__global__ void __launch_bounds__(kSlotThreads)
+    refresh_kernel(const int32_t *cdfs, int Lmax, const int32_t *lengths,
+                   const int32_t *offsets, RowMeta *meta, uint32_t *buckets, uint16_t *starts,
+                   uint32_t *slots, ChunkArea ca, int32_t *status) {
+  extern __shared__ int32_t srow[];
   const int r = blockIdx.y;
   const RowMeta m = meta[r * kMetaCopies];
   const int len = lengths[r];
@@ -440,26 +525,21 @@ __global__ void refresh_kernel(const int32_t *cdfs, int Lmax, const int32_t *len
     }
     for (int j = threadIdx.x; j < len; j += blockDim.x) starts[m.bucket_base + j] = (uint16_t)row[j];
   }
-  const int shift = (int)slot_shift(m.slot);
-  const int nslots = 1 << (16 - shift);
-  for (int t = blockIdx.x * blockDim.x + threadIdx.x; t < nslots; t += gridDim.x * blockDim.x)
-    fill_slot(row, nb, t, shift, slots, slot_base(m.slot) + t, ca);
+  fill_row_slots(row, nb, slot_base(m.slot), (int)slot_shift(m.slot), slots, ca, srow);
 }
 
 // The slot fill of rans_tables_prepare (rows already validated by
 // pack_buckets_kernel; a malformed row only leaves its own slots undefined).
-__global__ void fill_slots_kernel(const int32_t *cdfs, int Lmax, const RowMeta *meta,
-                                  const int32_t *lengths, uint32_t *slots, ChunkArea ca) {
+__global__ void __launch_bounds__(kSlotThreads)
+    fill_slots_kernel(const int32_t *cdfs, int Lmax, const RowMeta *meta,
+                      const int32_t *lengths, uint32_t *slots, ChunkArea ca) {
+  extern __shared__ int32_t srow[];
   const int r = blockIdx.y;
   const RowMeta m = meta[r * kMetaCopies];
-  const int shift = (int)slot_shift(m.slot);
-  const int nslots = 1 << (16 - shift);
-  const int t = blockIdx.x * blockDim.x + threadIdx.x;
-  if (t >= nslots) return;
   const int32_t *row = cdfs + (size_t)r * (size_t)Lmax;
   const int len = lengths[r];
-  if (row[0] != 0 || row[len - 1] != (int32_t)kTotal) return;
-  fill_slot(row, len - 1, t, shift, slots, slot_base(m.slot) + t, ca);
+  if (len < 2 || row[0] != 0 || row[len - 1] != (int32_t)kTotal) return;
+  fill_row_slots(row, len - 1, slot_base(m.slot), (int)slot_shift(m.slot), slots, ca, srow);
 }
 
 int ceil_log2(int64_t v) {
@@ -509,12 +589,11 @@ int refresh_tables(const int32_t *cdfs, int K, int Lmax, const int32_t *lengths,
   ca.used = reinterpret_cast<uint32_t *>(b) + kChunkUsedWord;
   ca.search = reinterpret_cast<uint32_t *>(b) + kSearchFlagWord;
   if (cudaMemsetAsync(ca.used, 0, 8, st) != cudaSuccess) return RANS_ERR_CUDA;
-  // slot chunks of 256: the largest row has at most 2^14 slots
-  int64_t maxslots = 1;
-  while (maxslots * K < t.n_slots && maxslots < (1 << kMaxQ)) maxslots <<= 1;
-  dim3 grid((unsigned)((maxslots + 255) / 256), (unsigned)K);
-  refresh_kernel<<<grid, 256, 0, st>>>(cdfs, Lmax, lengths, offsets, dmeta, dbuckets, dstarts,
-                                       dslots, ca, status);
+  // blocks of kSlotsPerBlock slots, enough for the largest possible row
+  // (2^kMaxQ slots); blocks past a smaller row's slots return at once
+  dim3 grid((unsigned)((1 << kMaxQ) / kSlotsPerBlock), (unsigned)K);
+  refresh_kernel<<<grid, kSlotThreads, kSlotSmemBytes, st>>>(
+      cdfs, Lmax, lengths, offsets, dmeta, dbuckets, dstarts, dslots, ca, status);
   return cudaGetLastError() == cudaSuccess ? RANS_OK : RANS_ERR_CUDA;
 }
 
@@ -629,13 +708,14 @@ int prepare_tables(const int32_t *cdfs, int K, int Lmax, const int32_t *lengths,
   pack_buckets_kernel<<<K, 256, 0, st>>>(cdfs, Lmax, dmeta, lengths, dbuckets, dstarts, status);
   int maxslots = 0;
   for (int r = 0; r < K; ++r) maxslots = maxslots > (1 << q[r]) ? maxslots : (1 << q[r]);
-  dim3 grid((maxslots + 255) / 256, K);
+  dim3 grid((maxslots + kSlotsPerBlock - 1) / kSlotsPerBlock, K);
   ChunkArea ca;
   ca.base = (uint32_t)sbase;
   ca.cap = (uint32_t)(slot_bytes / 4 - sbase);
   ca.used = reinterpret_cast<uint32_t *>(b) + kChunkUsedWord;
   ca.search = reinterpret_cast<uint32_t *>(b) + kSearchFlagWord;
-  fill_slots_kernel<<<grid, 256, 0, st>>>(cdfs, Lmax, dmeta, lengths, dslots, ca);
+  fill_slots_kernel<<<grid, kSlotThreads, kSlotSmemBytes, st>>>(cdfs, Lmax, dmeta, lengths,
+                                                                 dslots, ca);
   if (cudaGetLastError() != cudaSuccess) return RANS_ERR_CUDA;
   StatusWord sw;
   if (cudaMemcpyAsync(&sw, status, sizeof(sw), cudaMemcpyDeviceToHost, st) != cudaSuccess ||
