@@ -11,6 +11,13 @@ own 16 images; no collective on the data path).
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 
+--workload picks one of the other synthetic configurations instead (one
+GPU, for the per-configuration table): tiny (4,096 int32, 8 rows, W=1),
+z (128x17x30 int32, 128 pmf rows, 32 contiguous streams, W=1),
+y (192x68x120 int32, 24 contiguous streams, --interleave 1 or 32) and
+sweep (2^28 uint8, 16 Zipf rows, one index per 4,096 symbols, 8,192
+streams, W=32).
+
 Prints one JSON line (rank 0).  Inputs (200 MB of symbols and indexes) are
 larger than the 126 MB L2, so no flush is needed between steps.
 """
@@ -51,6 +58,8 @@ def parse():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-clocks", action="store_true")
     ap.add_argument("--traffic-file", default=os.path.join(ROOT, "profiles", "dram_traffic.txt"))
+    ap.add_argument("--workload", choices=["batch", "tiny", "z", "y", "sweep"], default="batch")
+    ap.add_argument("--interleave", type=int, default=None, help="W for --workload y")
     return ap.parse_args()
 
 
@@ -173,27 +182,57 @@ def shard_images(rank, images=N_IMAGES):
     return list(range(images * rank, images * (rank + 1)))
 
 
-def load_inputs(rank, group, images=N_IMAGES):
-    ids = shard_images(rank, images)
-    return WL.y_batch(n_images=len(ids), first_image=ids[0], cg=group)
+def load_inputs(rank, group, images=N_IMAGES, workload="batch", interleave=None):
+    if workload == "tiny":
+        w = WL.tiny()
+    elif workload == "z":
+        w = WL.z_latent()
+    elif workload == "y":
+        w = WL.y_latent(W=interleave or 32)
+    elif workload == "sweep":
+        w = WL.sweep(log2_n=28)
+    else:
+        ids = shard_images(rank, images)
+        w = WL.y_batch(n_images=len(ids), first_image=ids[0], cg=group)
+        w["W"] = 32
+    if interleave is not None and workload not in ("batch", "sweep"):
+        w["W"] = interleave
+    return w
+
+
+def workload_name(w, args):
+    if args.workload == "batch":
+        return WORKLOAD
+    n = int(np.asarray(w["symbols"]).size)
+    rows = len(w["scales"]) if "scales" in w else len(w["pmf_lengths"])
+    return "%s: %d %s symbols, %d %s rows, %s %d streams, W=%d, index block %d" % (
+        args.workload, n, np.asarray(w["symbols"]).dtype, rows,
+        "Gaussian" if "scales" in w else "pmf", w["chunking"]["kind"],
+        w["chunking"].get("n_streams", 0), w["W"], w["index_block"])
 
 
 # --------------------------------------------------------- CPU oracle leg --
 def oracle_sample(w, max_streams, workers):
-    """Oracle encode + decode of the first max_streams streams of the batch,
-    one stream per call, spread over `workers` threads (the C oracle runs
-    without the GIL).  Returns (symbols coded, seconds)."""
+    """Oracle encode + decode of the first max_streams streams of the
+    workload, one stream per call, spread over `workers` threads (the C
+    oracle runs without the GIL).  Returns (symbols coded, seconds)."""
     import oracle as O
-    c, l, o = O.build_cdfs_from_scales(w["scales"], w["tail_mass"])
+    if "scales" in w:
+        c, l, o = O.build_cdfs_from_scales(w["scales"], w["tail_mass"])
+    else:
+        c, l = O.build_cdfs_from_pmfs(w["pmfs"], w["pmf_lengths"], w["tail"])
+        o = np.asarray(w["offsets"], dtype=np.int32)
     flat = np.asarray(w["symbols"]).reshape(-1)
     pos = O.stream_positions(flat.size, w["chunking"])[:max_streams]
     idx = np.asarray(w["indexes"], dtype=np.int32)
+    blk = int(w.get("index_block", 1))
+    W = int(w.get("W", 32))
 
     def one(p):
         s = flat[p].astype(np.int64)
-        r = idx[p]
-        b = O.encode_stream(s, r, c, l, o, W=32)
-        back = O.decode_stream(b, r, c, l, o, W=32)
+        r = idx[p // blk]
+        b = O.encode_stream(s, r, c, l, o, W=W)
+        back = O.decode_stream(b, r, c, l, o, W=W)
         assert np.array_equal(back, s)
         return p.size
 
@@ -207,9 +246,9 @@ def run_reference(args, world, rank):
     """--impl reference: the oracle as it stands on the host cores."""
     if rank != 0:
         return
-    w = load_inputs(0, args.group)
+    w = load_inputs(0, args.group, workload=args.workload, interleave=args.interleave)
     workers = os.cpu_count() or 1
-    max_streams = 768     # 4 of the 16 images per step: a bounded sample
+    max_streams = 768     # batch: 4 of the 16 images per step, a bounded sample
     for _ in range(args.warmup):
         oracle_sample(w, 48, workers)
     tot_n, tot_t = 0, 0.0
@@ -224,7 +263,8 @@ def run_reference(args, world, rank):
         "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": 1,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * tot_t / args.steps,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "u64",
-        "data": "synthetic", "config": {"workload": WORKLOAD, "streams_per_step": max_streams},
+        "data": "synthetic", "config": {"workload": workload_name(w, args),
+                                        "streams_per_step": max_streams},
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": workers, "kind": "oracle",
                          "sample": sample},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
@@ -240,31 +280,53 @@ def run_ours(args, world, rank, local):
     rb.lib()
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
-    w = load_inputs(rank, args.group, args.images)
+    w = load_inputs(rank, args.group, args.images, args.workload, args.interleave)
     sym_np = np.ascontiguousarray(np.asarray(w["symbols"]).reshape(-1))
     idx_np = np.ascontiguousarray(w["indexes"], dtype=np.int32)
     n = sym_np.size
     sym = torch.from_numpy(sym_np).to(dev)
     idx = torch.from_numpy(idx_np).to(dev)
-    scales = torch.from_numpy(w["scales"]).to(dev)
-    tail = w["tail_mass"]
-    ch = rb.Chunking.from_spec(w["chunking"], 32)
+    ch = rb.Chunking.from_spec(w["chunking"], w["W"], w["index_block"], device=dev)
     S = rb.rans_num_streams(ch, n)
 
-    # tables: sized once; rebuilt inside every step
-    cdfs, lengths, offsets = rb.Tables.build_from_scales(scales, tail)
+    # tables: sized once; rebuilt inside every step (from the scale table, or
+    # from the pmfs)
+    if "scales" in w:
+        scales = torch.from_numpy(w["scales"]).to(dev)
+        tail = w["tail_mass"]
+        cdfs, lengths, offsets = rb.Tables.build_from_scales(scales, tail)
+
+        def build_rows():
+            rb.check(rb.rans_build_cdfs_from_scales(scales, tail, cdfs, lengths, offsets),
+                     "cdfs")
+    else:
+        pmfs = torch.from_numpy(np.ascontiguousarray(w["pmfs"])).to(dev)
+        plen = torch.from_numpy(np.asarray(w["pmf_lengths"], np.int32)).to(dev)
+        ptail = torch.from_numpy(np.asarray(w["tail"], np.float32)).to(dev)
+        cdfs, lengths = rb.Tables.build_from_pmfs(pmfs, plen, ptail)
+        offsets = torch.from_numpy(np.asarray(w["offsets"], np.int32)).to(dev)
+
+        def build_rows():
+            rb.check(rb.rans_build_cdfs_from_pmfs(pmfs, plen, ptail, cdfs, lengths), "cdfs")
     K, Lmax = cdfs.shape
     tables = rb.Tables(cdfs, lengths, offsets)
     blob = tables.blob
     ws = rb.Workspaces(ch, n, dev)
     dec = torch.empty_like(sym)
     stream = torch.cuda.current_stream()
+    # inputs smaller than L2: flush it (a 256 MB write) before every step,
+    # outside the phase events
+    in_bytes = n * (sym.element_size() + 4)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev) if in_bytes < (126 << 20) \
+        else None
 
     ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
 
     def step(e=None):
+        if flush is not None:
+            flush.fill_(1)
         if e: e[0].record(stream)
-        rb.check(rb.rans_build_cdfs_from_scales(scales, tail, cdfs, lengths, offsets), "cdfs")
+        build_rows()
         rb.check(rb.rans_tables_refresh(cdfs, lengths, offsets, tables), "refresh")
         if e: e[1].record(stream)
         rb.check(rb.rans_encode_with_indexes(sym, idx, n, tables, ch, ws.out, ws.offsets,
@@ -317,11 +379,14 @@ def run_ours(args, world, rank, local):
     enc_gbs = alg_enc / (enc_ms * 1e-3) / 1e9
     dec_gbs = alg_dec / (dec_ms * 1e-3) / 1e9
     dominant = "decode" if dec_ms >= enc_ms else "encode"
-    traffic = measured_traffic(args.traffic_file, dominant,
-                               "images=%d group=%d" % (args.images, args.group))
+    traffic = (measured_traffic(args.traffic_file, dominant,
+                                "images=%d group=%d" % (args.images, args.group))
+               if args.workload == "batch" else None)
     ach = dec_gbs if dominant == "decode" else enc_gbs
     total_syms = n * world
     ms_per_step = elapsed_ms / args.steps
+    if flush is not None:  # the steps' coding time, without the L2 flushes
+        ms_per_step = tab_ms + enc_ms + dec_ms
     value = total_syms / (ms_per_step * 1e-3) / 1e9
 
     # end to end through the public API with host buffers
@@ -330,7 +395,7 @@ def run_ours(args, world, rank, local):
         h_sym = torch.from_numpy(sym_np).pin_memory()
         h_idx = torch.from_numpy(idx_np).pin_memory()
         h_out = torch.empty(ws.out.numel(), dtype=torch.uint8).pin_memory()
-        h_dec = torch.empty(n, dtype=torch.int32).pin_memory()
+        h_dec = torch.empty(n, dtype=sym.dtype).pin_memory()
         d_sym = torch.empty_like(sym)
         d_idx = torch.empty_like(idx)
         h2d = d2h = 0
@@ -339,7 +404,7 @@ def run_ours(args, world, rank, local):
             nonlocal h2d, d2h
             d_sym.copy_(h_sym, non_blocking=True)
             d_idx.copy_(h_idx, non_blocking=True)
-            rb.check(rb.rans_build_cdfs_from_scales(scales, tail, cdfs, lengths, offsets))
+            build_rows()
             rb.check(rb.rans_tables_refresh(cdfs, lengths, offsets, tables))
             rb.check(rb.rans_encode_with_indexes(d_sym, d_idx, n, tables, ch, ws.out,
                                                  ws.offsets, ws.enc))
@@ -372,10 +437,11 @@ def run_ours(args, world, rank, local):
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         workers = os.cpu_count() or 1
-        ns, ts = oracle_sample(w, 768, workers)
+        ms = 768 if args.workload == "batch" else (64 if args.workload == "sweep" else S)
+        ns, ts = oracle_sample(w, ms, workers)
         cpu = {"value": ns / ts / 1e9, "unit": UNIT, "cores": workers, "kind": "oracle",
-               "sample": "oracle encode+decode of streams 0..767 (images 0-3, %d symbols), "
-                         "one stream per call over %d threads" % (ns, workers)}
+               "sample": "oracle encode+decode of the first %d streams (%d symbols), "
+                         "one stream per call over %d threads" % (ms, ns, workers)}
 
     launches_per_step = 1 + 1 + 3 + 1   # rows, table refresh, enc+scan+copy, dec
     if rank == 0:
@@ -384,11 +450,13 @@ def run_ours(args, world, rank, local):
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "u64",
             "data": "synthetic",
-            "config": {"workload": WORKLOAD, "symbols_per_gpu": n, "streams_per_gpu": S,
-                       "channel_group": args.group, "interleave": 32, "rows": K,
+            "config": {"workload": workload_name(w, args), "symbols_per_gpu": n,
+                       "streams_per_gpu": S, "channel_group": args.group,
+                       "interleave": w["W"], "rows": K,
                        "lmax": Lmax, "parallelism": "shard-by-image x%d" % world,
-                       "l2": "inputs larger than L2 (%d MB read per encode)" %
-                             (n * (sym_b + 4) // 2**20)},
+                       "l2": ("inputs larger than L2 (%d MB read per encode)" %
+                              (n * (sym_b + 4) // 2**20)) if flush is None else
+                             "L2 flushed before every step (256 MB write, not timed)"},
             "encode": {"ms": enc_ms, "gsym_s": n / enc_ms / 1e6, "GBps": enc_gbs,
                        "frac_hbm": enc_gbs / peak, "alg_bytes": alg_enc},
             "decode": {"ms": dec_ms, "gsym_s": n / dec_ms / 1e6, "GBps": dec_gbs,

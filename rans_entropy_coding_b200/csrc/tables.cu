@@ -472,6 +472,15 @@ __device__ void fill_slot_block(const int32_t *row, int nb, uint32_t slot0, int 
   }
 }
 
+// Copies n row entries into shared memory with cp.async (every copy in
+// flight at once, one wait), then a block barrier.
+__device__ __forceinline__ void stage_row(int32_t *srow, const int32_t *grow, int n) {
+  for (int i = threadIdx.x; i < n; i += blockDim.x) cp_async4(srow + i, grow + i);
+  cp_async_commit();
+  cp_async_wait<0>();
+  __syncthreads();
+}
+
 // Slot words (and bitmap words) of a row with nb buckets, blocks x, x +
 // gridDim.x, ... of kSlotsPerBlock slots; grow[0..nb] is the row (grow[0] =
 // 0, grow[nb] = 65536), shift the row's slot width log2.  Every thread of
@@ -483,8 +492,7 @@ __device__ void fill_row_slots(const int32_t *grow, int nb, uint32_t slot0, int 
   if ((int)blockIdx.x * kSlotsPerBlock >= nslots) return;  // (the whole block)
   const int32_t *row = grow;
   if (nb + 1 <= kRowSmem) {
-    for (int i = threadIdx.x; i <= nb; i += blockDim.x) srow[i] = grow[i];
-    __syncthreads();
+    stage_row(srow, grow, nb + 1);
     row = srow;
   }
   for (int tb = blockIdx.x * kSlotsPerBlock; tb < nslots; tb += gridDim.x * kSlotsPerBlock)
@@ -514,16 +522,22 @@ __global__ void __launch_bounds__(kSlotThreads)
     return;
   }
   if (blockIdx.x == 0) {
+    const int32_t *prow = row;
+    if (len <= kRowSmem) {
+      stage_row(srow, row, len);
+      prow = srow;
+    }
     if (threadIdx.x < kMetaCopies) meta[r * kMetaCopies + threadIdx.x].offset = offsets[r];
     for (int j = threadIdx.x; j < nb; j += blockDim.x) {
-      const int32_t a = row[j], b = row[j + 1];
+      const int32_t a = prow[j], b = prow[j + 1];
       if (!(b > a) || a < 0 || b > (int32_t)kTotal) {
         report(status, RANS_ERR_TABLE, r);
         continue;
       }
       buckets[m.bucket_base + j] = (uint32_t)(a & 0xffff) | ((uint32_t)(b - a - 1) << 16);
     }
-    for (int j = threadIdx.x; j < len; j += blockDim.x) starts[m.bucket_base + j] = (uint16_t)row[j];
+    for (int j = threadIdx.x; j < len; j += blockDim.x) starts[m.bucket_base + j] = (uint16_t)prow[j];
+    __syncthreads();  // the staged row is staged again below
   }
   fill_row_slots(row, nb, slot_base(m.slot), (int)slot_shift(m.slot), slots, ca, srow);
 }
