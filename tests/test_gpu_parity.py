@@ -185,6 +185,19 @@ def test_batch_small_ragged_tiles(W):
     _check_streams(w)
 
 
+@pytest.mark.parametrize("per", [4, 8, 36, 64, 68, 100, 132, 160, 292, 644])
+def test_contiguous_streams_of_every_block_phase(per):
+    """Streams of per symbols (a multiple of 4, so the encoder copies its
+    inputs in 16-byte blocks of 4 groups): stream lengths of 1 to 21 groups
+    put the partial last block in every phase; the last stream is shorter."""
+    S = 5
+    n = S * per - (4 if per > 4 else 0)
+    w = WL.tiny(seed=per, n=n)
+    w["W"] = 32
+    w["chunking"] = dict(kind="contig", n_streams=S)
+    _check_streams(w)
+
+
 def test_tiled_with_index_blocks():
     w = WL.y_batch(n_images=1, cg=4, th=16, tw=48)
     n = np.asarray(w["symbols"]).size
