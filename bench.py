@@ -16,7 +16,9 @@ GPU, for the per-configuration table): tiny (4,096 int32, 8 rows, W=1),
 z (128x17x30 int32, 128 pmf rows, 32 contiguous streams, W=1),
 y (192x68x120 int32, 24 contiguous streams, --interleave 1 or 32) and
 sweep (2^28 uint8, 16 Zipf rows, one index per 4,096 symbols, 8,192
-streams, W=32).
+streams, W=32) and float (the batch as float latents: y, means and scales
+per element in, rows and symbols computed inside the coders, float values
+out).
 
 Prints one JSON line (rank 0).  Inputs (200 MB of symbols and indexes) are
 larger than the 126 MB L2, so no flush is needed between steps.
@@ -58,7 +60,8 @@ def parse():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-clocks", action="store_true")
     ap.add_argument("--traffic-file", default=os.path.join(ROOT, "profiles", "dram_traffic.txt"))
-    ap.add_argument("--workload", choices=["batch", "tiny", "z", "y", "sweep"], default="batch")
+    ap.add_argument("--workload", choices=["batch", "tiny", "z", "y", "sweep", "float"],
+                    default="batch")
     ap.add_argument("--interleave", type=int, default=None, help="W for --workload y")
     return ap.parse_args()
 
@@ -191,6 +194,9 @@ def load_inputs(rank, group, images=N_IMAGES, workload="batch", interleave=None)
         w = WL.y_latent(W=interleave or 32)
     elif workload == "sweep":
         w = WL.sweep(log2_n=28)
+    elif workload == "float":
+        ids = shard_images(rank, images)
+        w = WL.y_float(seed=6000 + ids[0], n_images=len(ids), cg=group)
     else:
         ids = shard_images(rank, images)
         w = WL.y_batch(n_images=len(ids), first_image=ids[0], cg=group)
@@ -203,6 +209,10 @@ def load_inputs(rank, group, images=N_IMAGES, workload="batch", interleave=None)
 def workload_name(w, args):
     if args.workload == "batch":
         return WORKLOAD
+    if args.workload == "float":
+        return ("float_batch%d: %dx192x68x120 float32 y, means and scales per element, "
+                "64-entry scale table, tiles 64x64 x %d channels, W=32" %
+                (args.images, args.images, args.group))
     n = int(np.asarray(w["symbols"]).size)
     rows = len(w["scales"]) if "scales" in w else len(w["pmf_lengths"])
     return "%s: %d %s symbols, %d %s rows, %s %d streams, W=%d, index block %d" % (
@@ -247,6 +257,11 @@ def run_reference(args, world, rank):
     if rank != 0:
         return
     w = load_inputs(0, args.group, workload=args.workload, interleave=args.interleave)
+    if args.workload == "float":  # the oracle codes rows and symbols computed first
+        import oracle as O
+        w = dict(w, symbols=O.quantize(w["y"], w["means"]), W=32,
+                 indexes=O.build_indexes(w["fscales"], w["scales"],
+                                         w["scale_bound"]).reshape(-1))
     workers = os.cpu_count() or 1
     max_streams = 768     # batch: 4 of the 16 images per step, a bounded sample
     for _ in range(args.warmup):
@@ -474,12 +489,120 @@ def run_ours(args, world, rank, local):
         print(json.dumps(line), flush=True)
 
 
+def run_float(args, world, rank, local):
+    """--workload float: the batch as float latents through
+    rans_encode_from_scales / rans_decode_to_values."""
+    import torch
+
+    import rans_entropy_coding_b200 as rb
+
+    rb.lib()
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    w = load_inputs(rank, args.group, args.images, "float")
+    flat = lambda a: torch.from_numpy(np.ascontiguousarray(a).reshape(-1)).to(dev)
+    y, sc, mu = flat(w["y"]), flat(w["fscales"]), flat(w["means"])
+    n = y.numel()
+    table = torch.from_numpy(np.asarray(w["scales"], np.float32)).to(dev)
+    bound, tail = w["scale_bound"], w["tail_mass"]
+    ch = rb.Chunking.from_spec(w["chunking"], 32, 1, device=dev)
+    S = rb.rans_num_streams(ch, n)
+    cdfs, lengths, offsets = rb.Tables.build_from_scales(table, tail)
+    K, Lmax = cdfs.shape
+    tables = rb.Tables(cdfs, lengths, offsets)
+    ws = rb.Workspaces(ch, n, dev)
+    vals = torch.empty_like(y)
+    want = torch.round(y - mu).to(torch.int32).to(torch.float32) + mu
+    stream = torch.cuda.current_stream()
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+
+    def step(e=None):
+        if e: e[0].record(stream)
+        rb.check(rb.rans_build_cdfs_from_scales(table, tail, cdfs, lengths, offsets), "cdfs")
+        rb.check(rb.rans_tables_refresh(cdfs, lengths, offsets, tables), "refresh")
+        if e: e[1].record(stream)
+        rb.check(rb.rans_encode_from_scales(y, mu, sc, n, table, bound, tables, ch, ws.out,
+                                            ws.offsets, ws.enc), "encode")
+        if e: e[2].record(stream)
+        rb.check(rb.rans_decode_to_values(ws.out, ws.offsets, sc, mu, n, table, bound, tables,
+                                          ch, vals, ws.dec), "decode")
+        if e: e[3].record(stream)
+
+    for _ in range(max(args.warmup, 0)):
+        step()
+    torch.cuda.synchronize()
+    for what, b in (("encode", ws.enc), ("decode", ws.dec), ("tables", tables.blob)):
+        rb.check(rb.rans_get_status(b), what + " status")
+    assert torch.equal(vals, want), "round trip failed"
+    barrier(world)
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local, enabled=not args.no_clocks) as clk:
+        torch.cuda.synchronize()
+        barrier(world)
+        t0.record(stream)
+        for i in range(args.steps):
+            step(ev[i])
+        t1.record(stream)
+        torch.cuda.synchronize()
+        barrier(world)
+    elapsed_ms = max_over_ranks(t0.elapsed_time(t1), world, dev)
+    assert torch.equal(vals, want), "round trip failed"
+    tab_ms = float(np.mean([e[0].elapsed_time(e[1]) for e in ev]))
+    enc_ms = float(np.mean([e[1].elapsed_time(e[2]) for e in ev]))
+    dec_ms = float(np.mean([e[2].elapsed_time(e[3]) for e in ev]))
+    comp = int(ws.offsets[-1].item())
+    alg_enc = n * 12 + comp      # y, scale, mean read; bytes written
+    alg_dec = n * 12 + comp      # bytes, scale, mean read; values written
+    peak = (json.load(open(os.path.join(ROOT, "MEASURED_PEAKS.json"))).get("hbm_gbs")
+            if os.path.exists(os.path.join(ROOT, "MEASURED_PEAKS.json")) else None) or 6650.0
+    enc_gbs = alg_enc / (enc_ms * 1e-3) / 1e9
+    dec_gbs = alg_dec / (dec_ms * 1e-3) / 1e9
+    ms_per_step = elapsed_ms / args.steps
+    value = n * world / (ms_per_step * 1e-3) / 1e9
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        import oracle as O
+        wi = dict(w, symbols=O.quantize(w["y"], w["means"]),
+                  indexes=O.build_indexes(w["fscales"], w["scales"], bound).reshape(-1), W=32)
+        workers = os.cpu_count() or 1
+        ns, ts = oracle_sample(wi, 768, workers)
+        cpu = {"value": ns / ts / 1e9, "unit": UNIT, "cores": workers, "kind": "oracle",
+               "sample": "oracle encode+decode of the first 768 streams (%d symbols), rows "
+                         "and symbols computed beforehand" % ns}
+    if rank == 0:
+        dominant = "decode" if dec_ms >= enc_ms else "encode"
+        ach = dec_gbs if dominant == "decode" else enc_gbs
+        print(json.dumps({
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "u64",
+            "data": "synthetic",
+            "config": {"workload": workload_name(w, args), "symbols_per_gpu": n,
+                       "streams_per_gpu": S, "channel_group": args.group, "interleave": 32,
+                       "rows": K, "lmax": Lmax, "parallelism": "shard-by-image x%d" % world,
+                       "l2": "inputs larger than L2 (%d MB read per encode)" % (n * 12 >> 20)},
+            "encode": {"ms": enc_ms, "gsym_s": n / enc_ms / 1e6, "GBps": enc_gbs,
+                       "frac_hbm": enc_gbs / peak, "alg_bytes": alg_enc},
+            "decode": {"ms": dec_ms, "gsym_s": n / dec_ms / 1e6, "GBps": dec_gbs,
+                       "frac_hbm": dec_gbs / peak, "alg_bytes": alg_dec},
+            "tables": {"ms": tab_ms}, "compressed_bytes": comp,
+            "bits_per_symbol": 8.0 * comp / n,
+            "roofline": {"bound": "hbm", "achieved": ach, "peak": peak, "unit": "GB/s",
+                         "frac": ach / peak, "traffic": None, "kernel": dominant},
+            "cpu_baseline": cpu, "e2e": None, "clocks": clk.summary(),
+            "gpu_launches": 6 * args.steps,
+        }), flush=True)
+
+
 def main():
     args = parse()
     world, rank, local = dist_setup(args)
     try:
         if args.impl == "reference":
             run_reference(args, world, rank)
+        elif args.workload == "float":
+            run_float(args, world, rank, local)
         else:
             run_ours(args, world, rank, local)
     finally:

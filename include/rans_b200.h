@@ -301,6 +301,59 @@ int rans_encode_with_indexes_noalloc(const void *symbols, int32_t sym_dtype,
                                      uint64_t out_capacity, uint64_t *stream_offsets,
                                      void *stream);
 
+/* --------------------------------------------------- float latents ---- */
+
+/*
+ * The coder fed straight from a mean-scale model's float tensors (the y latent
+ * of "Benchmark notes" section 3, whose per-stage breakdown shows the scales
+ * mapped to table rows by CompressAI's build_indexes before the coder runs).
+ * The pages name these steps without spelling them out; the library's reading:
+ *   row:    for a scale s, the first of the K scale-table entries (increasing)
+ *           that is >= max(s, scale_bound), a NaN scale counting as the bound;
+ *           the last row when none of the first K - 1 entries is;
+ *   symbol: y - mean in float32, rounded to the nearest integer, ties to even
+ *           (mean 0 when `means` is NULL); a value that is not finite or not
+ *           an int32 is RANS_ERR_RANGE;
+ *   value:  the decoder returns float32(symbol) + mean, in float32.
+ * The row of element i is what rans_encode_with_indexes takes as indexes[i]
+ * and the symbol its symbols[i], so the streams are byte-identical to
+ * encoding those.
+ */
+
+/* Rows of n scales (device float[n] in, device int32[n] out) for a K-entry
+ * device scale table.  Asynchronous. */
+int rans_build_indexes(const float *scales, int64_t n, const float *scale_table, int32_t K,
+                       float scale_bound, int32_t *indexes, void *stream);
+
+/*
+ * encode_with_indexes from float latents, rows and symbols computed inside the
+ * coder (no index or symbol array is written).
+ *   y, scales:   device float[n]; means: device float[n] or NULL.
+ *   scale_table: device float[table_len], table_len == tables->K: the scales
+ *                the table rows were built from.
+ *   chunking:    index_block must be 1 (one scale per element).
+ * Other arguments, outputs and errors as rans_encode_with_indexes.
+ */
+int rans_encode_from_scales(const float *y, const float *means, const float *scales,
+                            int64_t n, const float *scale_table, int32_t table_len,
+                            float scale_bound, const rans_tables *tables,
+                            const rans_chunking *chunking, uint8_t *out,
+                            uint64_t out_capacity, uint64_t *stream_offsets, void *workspace,
+                            uint64_t workspace_bytes, void *stream);
+
+/*
+ * decode_with_indexes back to float values: values[i] = float32(symbol) +
+ * means[i] (or the symbol alone when means is NULL), rows from the scales as
+ * above.  values: device float[n].  Other arguments and errors as
+ * rans_decode_with_indexes.
+ */
+int rans_decode_to_values(const uint8_t *in, uint64_t in_bytes, const uint64_t *stream_offsets,
+                          const float *scales, const float *means, int64_t n,
+                          const float *scale_table, int32_t table_len, float scale_bound,
+                          const rans_tables *tables, const rans_chunking *chunking,
+                          float *values, void *workspace, uint64_t workspace_bytes,
+                          void *stream);
+
 /* Synchronises `stream` and returns the first error recorded in `workspace`
  * (RANS_OK if none), then clears it. */
 int rans_get_status(void *workspace, void *stream);

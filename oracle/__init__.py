@@ -251,3 +251,47 @@ def decode_with_indexes(data, stream_offsets, indexes, cdfs, lengths, offsets, c
         out[p] = decode_stream(d[a:b], _rows_for(p, indexes, index_block), cdfs, lengths,
                                offsets, W)
     return out.astype(dtype)
+
+
+# --------------------------------------------------- float latents -------
+# Readings (the pages name CompressAI's build_indexes and the quantisation of
+# a mean-scale model -- symbol = round(y - mean) -- but print neither):
+#   * a scale below ``scale_bound`` counts as the bound (a NaN scale too);
+#   * the row of a scale s is the first of the K table entries that is >= s,
+#     the last row when none of the first K - 1 is: CompressAI starts every
+#     index at K - 1 and takes one off for each of the first K - 1 entries
+#     that is >= s;
+#   * the symbol is y - mean computed in float32, rounded to the nearest
+#     integer with ties to even (torch.round); a value that is not finite or
+#     falls outside int32 is a range error;
+#   * decoding gives back float32(symbol) + mean, in float32.
+def build_indexes(scales, scale_table, scale_bound):
+    """Row index of every scale (int32 array of the scales' shape)."""
+    s = np.asarray(scales, dtype=np.float32)
+    s = np.where(np.isnan(s) | (s < np.float32(scale_bound)), np.float32(scale_bound), s)
+    t = np.asarray(scale_table, dtype=np.float32)
+    K = t.size
+    idx = np.full(s.shape, K - 1, dtype=np.int32)
+    for i in range(K - 1):
+        idx -= (s <= t[i]).astype(np.int32)
+    return idx
+
+
+def quantize(y, means=None):
+    """Symbols round(y - mean) (float32, ties to even); raises OracleError
+    (ERR_RANGE) for a value that is not finite or not in int32."""
+    d = np.asarray(y, dtype=np.float32)
+    if means is not None:
+        d = d - np.asarray(means, dtype=np.float32)
+    r = np.rint(d)
+    if not np.all(np.isfinite(r)) or np.any(r < -2147483648.0) or np.any(r >= 2147483648.0):
+        raise OracleError(ERR_RANGE, "quantize")
+    return r.astype(np.int32)
+
+
+def dequantize(symbols, means=None):
+    """float32(symbol) + mean, in float32."""
+    v = np.asarray(symbols).astype(np.float32)
+    if means is not None:
+        v = v + np.asarray(means, dtype=np.float32)
+    return v

@@ -8,7 +8,9 @@ from ._lib import (  # noqa: F401
     CHUNK_CONTIG, CHUNK_EXPLICIT, CHUNK_TILED, ERR_ARG, ERR_CAPACITY, ERR_CORRUPT, ERR_CUDA,
     ERR_INDEX, ERR_RANGE, ERR_TABLE, ERR_TIMEOUT, ERR_ZERO_FREQ, LIB_PATH, OK, SIGNATURES,
     SYM_INT16, SYM_INT32, SYM_UINT8, Chunking, RansError, Tables, Workspaces, aligned_empty,
-    check, decode_with_indexes, encode_with_indexes, lib, rans_build_cdfs_from_pmfs,
+    check, decode_to_values, decode_with_indexes, encode_from_scales, encode_with_indexes, lib,
+    rans_build_cdfs_from_pmfs, rans_build_indexes, rans_decode_to_values,
+    rans_encode_from_scales,
     rans_build_cdfs_from_scales, rans_chunking, rans_debug_divide, rans_decode_with_indexes,
     rans_decode_workspace_bytes, rans_encode_with_indexes, rans_encode_with_indexes_noalloc,
     rans_encode_workspace_bytes,

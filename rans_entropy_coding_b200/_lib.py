@@ -54,8 +54,8 @@ class rans_tables(ctypes.Structure):
 
 
 # (name, restype, argtypes) for every exported symbol of include/rans_b200.h
-_P, _I32, _I64, _U64, _F64 = (ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64,
-                              ctypes.c_uint64, ctypes.c_double)
+_P, _I32, _I64, _U64, _F64, _F32 = (ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64,
+                                   ctypes.c_uint64, ctypes.c_double, ctypes.c_float)
 _CHP = ctypes.POINTER(rans_chunking)
 _TBP = ctypes.POINTER(rans_tables)
 SIGNATURES = [
@@ -77,6 +77,11 @@ SIGNATURES = [
      [_P, _U64, _P, _P, _I64, _TBP, _CHP, _P, _I32, _P, _U64, _P]),
     ("rans_encode_with_indexes_noalloc", ctypes.c_int,
      [_P, _I32, _P, _I64, _TBP, _CHP, _P, _U64, _P, _P]),
+    ("rans_build_indexes", ctypes.c_int, [_P, _I64, _P, _I32, _F32, _P, _P]),
+    ("rans_encode_from_scales", ctypes.c_int,
+     [_P, _P, _P, _I64, _P, _I32, _F32, _TBP, _CHP, _P, _U64, _P, _P, _U64, _P]),
+    ("rans_decode_to_values", ctypes.c_int,
+     [_P, _U64, _P, _P, _P, _I64, _P, _I32, _F32, _TBP, _CHP, _P, _P, _U64, _P]),
     ("rans_get_status", ctypes.c_int, [_P, _P]),
     ("rans_debug_divide", ctypes.c_int, [_P, _P, _I64, _P, _P, _P]),
 ]
@@ -206,6 +211,32 @@ def rans_encode_with_indexes_noalloc(symbols, indexes, n, tables, chunking, out,
     return lib().rans_encode_with_indexes_noalloc(
         _ptr(symbols), _DTYPE_CODE[symbols.dtype], _ptr(indexes), n, ctypes.byref(tables.c),
         ctypes.byref(chunking.c), _ptr(out), out.numel(), _ptr(stream_offsets), _stream(stream))
+
+
+def rans_build_indexes(scales, scale_table, scale_bound, indexes, stream=None):
+    _need_cuda(scales, scale_table, indexes)
+    return lib().rans_build_indexes(_ptr(scales), scales.numel(), _ptr(scale_table),
+                                    scale_table.numel(), float(scale_bound), _ptr(indexes),
+                                    _stream(stream))
+
+
+def rans_encode_from_scales(y, means, scales, n, scale_table, scale_bound, tables, chunking,
+                            out, stream_offsets, workspace, stream=None):
+    _need_cuda(y, means, scales, scale_table, out, stream_offsets, workspace)
+    return lib().rans_encode_from_scales(
+        _ptr(y), _ptr(means), _ptr(scales), n, _ptr(scale_table), scale_table.numel(),
+        float(scale_bound), ctypes.byref(tables.c), ctypes.byref(chunking.c), _ptr(out),
+        out.numel(), _ptr(stream_offsets), _ptr(workspace), workspace.numel(), _stream(stream))
+
+
+def rans_decode_to_values(data, stream_offsets, scales, means, n, scale_table, scale_bound,
+                          tables, chunking, values, workspace, stream=None):
+    _need_cuda(data, stream_offsets, scales, means, scale_table, values, workspace)
+    return lib().rans_decode_to_values(
+        _ptr(data), data.numel(), _ptr(stream_offsets), _ptr(scales), _ptr(means), n,
+        _ptr(scale_table), scale_table.numel(), float(scale_bound), ctypes.byref(tables.c),
+        ctypes.byref(chunking.c), _ptr(values), _ptr(workspace), workspace.numel(),
+        _stream(stream))
 
 
 def rans_get_status(workspace, stream=None):
@@ -356,6 +387,30 @@ def encode_with_indexes(symbols, indexes, tables, chunking, ws=None, stream=None
     check(rans_encode_with_indexes(symbols, indexes, n, tables, chunking, ws.out, ws.offsets,
                                    ws.enc, stream), "encode")
     return ws.out, ws.offsets, ws
+
+
+def encode_from_scales(y, scales, scale_table, scale_bound, tables, chunking, means=None,
+                       ws=None, stream=None):
+    """Float latents in: like encode_with_indexes, rows from the scales and
+    symbols rint(y - mean) computed inside the coder."""
+    n = y.numel()
+    if ws is None:
+        ws = Workspaces(chunking, n, y.device)
+    check(rans_encode_from_scales(y, means, scales, n, scale_table, scale_bound, tables,
+                                  chunking, ws.out, ws.offsets, ws.enc, stream), "encode")
+    return ws.out, ws.offsets, ws
+
+
+def decode_to_values(data, stream_offsets, scales, scale_table, scale_bound, tables, chunking,
+                     means=None, out=None, ws=None, stream=None):
+    """Float values out: float32(symbol) + mean."""
+    n = scales.numel()
+    if out is None:
+        out = torch.empty(n, dtype=torch.float32, device=data.device)
+    wsd = ws.dec if ws is not None else aligned_empty(256, data.device)
+    check(rans_decode_to_values(data, stream_offsets, scales, means, n, scale_table,
+                                scale_bound, tables, chunking, out, wsd, stream), "decode")
+    return out, wsd
 
 
 def decode_with_indexes(data, stream_offsets, indexes, tables, chunking, n, dtype=torch.int32,

@@ -296,6 +296,79 @@ RANS_API int rans_decode_with_indexes(const uint8_t *in, uint64_t in_bytes,
                            sym_dtype, status, s);
 }
 
+// ---- float latents ------------------------------------------------------
+
+RANS_API int rans_build_indexes(const float *scales, int64_t n, const float *scale_table,
+                                int32_t K, float scale_bound, int32_t *indexes, void *stream) {
+  if (n < 0 || K < 1 || (n > 0 && (!scales || !scale_table || !indexes))) return RANS_ERR_ARG;
+  return rb::launch_build_indexes(scales, n, scale_table, K, scale_bound, indexes,
+                                  as_stream(stream));
+}
+
+// The float entry points take one scale per element (index_block 1) and a
+// scale table with one entry per table row.
+static int float_args(const rans_tables *tables, const rans_chunking *chunking,
+                      int32_t table_len) {
+  if (!tables_usable(tables) || !chunking) return RANS_ERR_ARG;
+  if (table_len != tables->K || chunking->index_block != 1) return RANS_ERR_ARG;
+  return RANS_OK;
+}
+
+RANS_API int rans_encode_from_scales(const float *y, const float *means, const float *scales,
+                                     int64_t n, const float *scale_table, int32_t table_len,
+                                     float scale_bound, const rans_tables *tables,
+                                     const rans_chunking *chunking, uint8_t *out,
+                                     uint64_t out_capacity, uint64_t *stream_offsets,
+                                     void *workspace, uint64_t workspace_bytes, void *stream) {
+  int st = float_args(tables, chunking, table_len);
+  if (st) return st;
+  if (n > 0 && (!y || !scales || !scale_table)) return RANS_ERR_ARG;
+  if (!stream_offsets || !workspace || (out_capacity > 0 && !out)) return RANS_ERR_ARG;
+  if ((reinterpret_cast<uintptr_t>(workspace) & 255) != 0) return RANS_ERR_ARG;
+  Geom g;
+  st = make_geom(chunking, n, g);
+  if (st) return st;
+  if (workspace_bytes < enc_ws_bytes(g)) return RANS_ERR_CAPACITY;
+  cudaStream_t s = as_stream(stream);
+  char *ws = reinterpret_cast<char *>(workspace);
+  int32_t *status = reinterpret_cast<int32_t *>(ws);
+  uint64_t *lens = reinterpret_cast<uint64_t *>(ws + kWsHeader);
+  char *scratch = ws + kWsHeader + lens_bytes(g);
+  if (cudaMemsetAsync(ws, 0, kWsHeader + 8ull * (uint64_t)g.S, s) != cudaSuccess)
+    return RANS_ERR_CUDA;
+  if (g.S > 0) {
+    st = rb::launch_encode_float(y, means, scales, scale_table, scale_bound, *tables, g,
+                                 scratch, lens, status, s);
+    if (st) return st;
+  }
+  return rb::launch_compact(g, scratch, lens, out, out_capacity, stream_offsets, status, s);
+}
+
+RANS_API int rans_decode_to_values(const uint8_t *in, uint64_t in_bytes,
+                                   const uint64_t *stream_offsets, const float *scales,
+                                   const float *means, int64_t n, const float *scale_table,
+                                   int32_t table_len, float scale_bound,
+                                   const rans_tables *tables, const rans_chunking *chunking,
+                                   float *values, void *workspace, uint64_t workspace_bytes,
+                                   void *stream) {
+  int st = float_args(tables, chunking, table_len);
+  if (st) return st;
+  if (n > 0 && (!values || !scales || !scale_table)) return RANS_ERR_ARG;
+  if (!stream_offsets || !workspace || (in_bytes > 0 && !in)) return RANS_ERR_ARG;
+  if ((reinterpret_cast<uintptr_t>(workspace) & 255) != 0) return RANS_ERR_ARG;
+  if ((reinterpret_cast<uintptr_t>(in) & 3) != 0) return RANS_ERR_ARG;
+  Geom g;
+  st = make_geom(chunking, n, g);
+  if (st) return st;
+  if (workspace_bytes < kWsHeader) return RANS_ERR_CAPACITY;
+  cudaStream_t s = as_stream(stream);
+  int32_t *status = reinterpret_cast<int32_t *>(workspace);
+  if (cudaMemsetAsync(workspace, 0, kWsHeader, s) != cudaSuccess) return RANS_ERR_CUDA;
+  if (g.S == 0) return RANS_OK;
+  return rb::launch_decode_float(in, in_bytes, stream_offsets, scales, means, scale_table,
+                                 scale_bound, *tables, g, values, status, s);
+}
+
 RANS_API int rans_get_status(void *workspace, void *stream) {
   if (!workspace) return RANS_ERR_ARG;
   cudaStream_t s = as_stream(stream);

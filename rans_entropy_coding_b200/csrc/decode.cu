@@ -49,6 +49,11 @@ struct DecCtx {
   Geom g;
   void *out;
   int32_t *status;
+  // float latents: rows from scales (one per element) and values
+  // float(symbol) + mean written to `out` as float
+  const float *fscale, *fmean, *stab;
+  float bound;
+  int32_t stab_top;
 };
 
 __device__ __forceinline__ bool stream_bounds(const DecCtx &c, int64_t s, int W,
@@ -211,7 +216,7 @@ __device__ __forceinline__ void load_window(WarpDec &st, const uint32_t *words, 
 template <typename SymT, bool FULL, bool SEARCH>
 __device__ __forceinline__ void dec_group(WarpDec &st, const RowMeta &m, const uint16_t *starts,
                                           const uint32_t *slots, bool active, SymT *dst,
-                                          const uint32_t *words, uint64_t nw) {
+                                          const uint32_t *words, uint64_t nw, float mean = 0.0f) {
   const int lane = threadIdx.x & 31;
   if (FULL) active = true;
   const uint32_t cum = (uint32_t)st.x & (kTotal - 1);
@@ -247,12 +252,18 @@ __device__ __forceinline__ void dec_group(WarpDec &st, const RowMeta &m, const u
     st.off = 0;
     load_window(st, words, nw);
   }
-  if (active) st_global(dst, (SymT)val);
+  if (active) {
+    if (std::is_same<SymT, float>::value) st_global(dst, (SymT)((float)val + mean));
+    else st_global(dst, (SymT)val);
+  }
 }
 
 // One warp decodes one stream, a group of 32 symbols per step: the copies
 // for group g + kDecStage - 1, group g+1's row metadata from the ring, then
 // group g's decode.
+// SymT = float: the ring holds scales, each group's row is its scale's table
+// row, and the output is float(symbol) + mean, the means read one group
+// ahead with plain loads.
 template <typename SymT, bool IB0, bool WIDE, bool SEARCH>
 __device__ __forceinline__ void decode_stream_w32(const DecCtx &c, const StreamDesc &d,
                                                   const RowMeta *meta, const uint16_t *starts,
@@ -282,32 +293,50 @@ __device__ __forceinline__ void decode_stream_w32(const DecCtx &c, const StreamD
   Stepper<WIDE> pl;  // next group to copy
   pl.init(d.t, lane);
   Stepper<WIDE> pc = pl;  // group being decoded (output position)
+  constexpr bool kFlt = std::is_same<SymT, float>::value;
+  const float *fs_s = kFlt ? c.fscale + base : nullptr;
+  const float *fm_s = kFlt && c.fmean ? c.fmean + base : nullptr;
   auto issue = [&](int32_t gi) {
     const int32_t rel = gi < G && lane < n - gi * 32 ? pl.rel : 0;
-    cp_async4(stg + (gi & (kS - 1)) * 32 + lane,
-              IB0 ? idx_s + rel : c.idx + ((base + rel) >> ib));
+    if (kFlt) {
+      cp_async4(stg + (gi & (kS - 1)) * 32 + lane, fs_s + rel);
+      if (fm_s) prefetch_l2(fm_s + rel);
+    } else {
+      cp_async4(stg + (gi & (kS - 1)) * 32 + lane,
+                IB0 ? idx_s + rel : c.idx + ((base + rel) >> ib));
+    }
     cp_async_commit();
     pl.fwd(32);
   };
-  auto meta_of = [&](uint32_t r) -> RowMeta {
+  auto meta_of = [&](uint32_t v) -> RowMeta {
+    const uint32_t r =
+        kFlt ? scale_row(bound_scale(__uint_as_float(v), c.bound), c.stab, c.K, c.stab_top) : v;
     st.rmax = max(st.rmax, r);
     return row_meta(meta, min(r, kmax));
+  };
+  // the mean of group g's element for this lane (0 past the stream end)
+  auto mean_at = [&](int32_t g, int32_t rel) -> float {
+    return fm_s && g < G && lane < n - g * 32 ? __ldg(fm_s + rel) : 0.0f;
   };
 #pragma unroll 1
   for (int32_t u = 0; u < kS - 1; ++u) issue(u);
   cp_async_wait<kS - 2>();
   RowMeta m = meta_of(stg[lane]);
+  float mean = kFlt ? mean_at(0, pc.rel) : 0.0f;
 #pragma unroll 1
   for (int32_t g = 0; g + 1 < G; ++g) {
     issue(g + kS - 1);
     cp_async_wait<kS - 2>();  // groups up to g + 1 have landed
     const RowMeta mn = meta_of(stg[((g + 1) & (kS - 1)) * 32 + lane]);
-    dec_group<SymT, true, SEARCH>(st, m, starts, slots, true, out_s + pc.rel, words, nw);
+    const int32_t rel = pc.rel;
     pc.fwd(32);
+    const float mean_n = kFlt ? mean_at(g + 1, pc.rel) : 0.0f;
+    dec_group<SymT, true, SEARCH>(st, m, starts, slots, true, out_s + rel, words, nw, mean);
     m = mn;
+    mean = mean_n;
   }
   dec_group<SymT, false, SEARCH>(st, m, starts, slots, lane < n - (G - 1) * 32, out_s + pc.rel,
-                                 words, nw);
+                                 words, nw, mean);
   cp_async_wait<0>();
   if (__any_sync(kFull, st.rmax > kmax)) {
     if (lane == 0) report(c.status, RANS_ERR_INDEX, s);
@@ -375,18 +404,26 @@ __device__ void decode_stream_w1(const DecCtx &c, const RowMeta *meta, const uin
   pp = pl;
   const int32_t n = (int32_t)d.n;
   constexpr int32_t kAhead = 64;
+  constexpr bool kFlt = std::is_same<SymT, float>::value;
+  auto prefetch = [&](int64_t q) {
+    if (kFlt) prefetch_l2(c.fscale + q);
+    else prefetch_l2(c.idx + (q >> ib));
+  };
   for (int32_t u = 0; u < kAhead && u < n; ++u) {
-    prefetch_l2(c.idx + ((d.base + pp.rel(t)) >> ib));
+    prefetch(d.base + pp.rel(t));
     pp.fwd(t, 1);
   }
   for (int32_t i = 0; i < n; ++i) {
     const int64_t p = d.base + pl.rel(t);
     pl.fwd(t, 1);
     if (i + kAhead < n) {
-      prefetch_l2(c.idx + ((d.base + pp.rel(t)) >> ib));
+      prefetch(d.base + pp.rel(t));
       pp.fwd(t, 1);
     }
-    const int32_t r = __ldg(c.idx + (p >> ib));
+    const int32_t r =
+        kFlt ? (int32_t)scale_row(bound_scale(__ldg(c.fscale + p), c.bound), c.stab, c.K,
+                                  c.stab_top)
+             : __ldg(c.idx + (p >> ib));
     if ((uint32_t)r >= (uint32_t)c.K) {
       report(c.status, RANS_ERR_INDEX, s);
       return;
@@ -421,7 +458,12 @@ __device__ void decode_stream_w1(const DecCtx &c, const RowMeta *meta, const uin
       const int64_t half = (int64_t)(raw >> 1);
       val = (raw & 1) ? (-half - 1) : ((int64_t)m.maxv + half);
     }
-    SymIO<SymT>::store(c.out, p, val + (int64_t)m.offset);
+    if constexpr (kFlt)
+      st_global(reinterpret_cast<float *>(c.out) + p,
+                (float)(int32_t)(val + (int64_t)m.offset) +
+                    (c.fmean ? __ldg(c.fmean + p) : 0.0f));
+    else
+      SymIO<SymT>::store(c.out, p, val + (int64_t)m.offset);
   }
   if (bad || x != kL || pw != nw) report(c.status, RANS_ERR_CORRUPT, s);
 }
@@ -537,6 +579,35 @@ int launch_decode_s(const DecCtx &c, bool smem, cudaStream_t st) {
 
 }  // namespace
 
+int launch_decode_float(const uint8_t *in, uint64_t in_bytes, const uint64_t *offsets,
+                        const float *scales, const float *means, const float *scale_table,
+                        float scale_bound, const rans_tables &t, const Geom &g, float *values,
+                        int32_t *status, cudaStream_t st) {
+  DecCtx c;
+  c.in = in;
+  c.in_bytes = in_bytes;
+  c.offs = offsets;
+  c.idx = nullptr;
+  c.K = t.K;
+  c.meta_bytes = t.meta_bytes;
+  c.bucket_bytes = t.bucket_bytes;
+  c.start_bytes = t.start_bytes;
+  c.slot_bytes = t.slot_bytes;
+  c.blob = reinterpret_cast<const char *>(t.blob);
+  c.g = g;
+  c.out = values;
+  c.status = status;
+  c.fscale = scales;
+  c.fmean = means;
+  c.stab = scale_table;
+  c.bound = scale_bound;
+  c.stab_top = 0;
+  while (2 * c.stab_top <= t.K - 1 && t.K > 1) c.stab_top = c.stab_top ? 2 * c.stab_top : 1;
+  const bool smem = t.dec_in_smem != 0;
+  return g.W == 32 ? launch_decode_w<32, float>(c, smem, st)
+                   : launch_decode_w<1, float>(c, smem, st);
+}
+
 int launch_decode(const uint8_t *in, uint64_t in_bytes, const uint64_t *offsets,
                   const int32_t *indexes, const rans_tables &t, const Geom &g, void *symbols,
                   int sym_dtype, int32_t *status, cudaStream_t st) {
@@ -554,6 +625,9 @@ int launch_decode(const uint8_t *in, uint64_t in_bytes, const uint64_t *offsets,
   c.g = g;
   c.out = symbols;
   c.status = status;
+  c.fscale = c.fmean = c.stab = nullptr;
+  c.bound = 0.0f;
+  c.stab_top = 0;
   const bool smem = t.dec_in_smem != 0;
   switch (sym_dtype) {
     case RANS_SYM_INT32: return launch_decode_s<int32_t>(c, smem, st);

@@ -31,6 +31,11 @@ constexpr int kEncThreads1 = 128;
 struct EncCtx {
   const void *sym;
   const int32_t *idx;
+  // float latents instead of sym / idx (one scale per element): y, means
+  // (or null), scales, the K-entry scale table, its lower bound
+  const float *fy, *fmean, *fscale, *stab;
+  float bound;
+  int32_t stab_top;  // largest power of two <= K - 1
   int32_t K;
   uint32_t meta_bytes, bucket_bytes;
   const char *blob;
@@ -211,11 +216,14 @@ __device__ __forceinline__ void enc_group_escape(WarpEnc &st, uint64_t x0, uint3
 // of groups k+2 (symbols, row metadata) and k+3 (row index); group k's rare
 // escape path comes last.  Nothing in group k's state chain waits on a
 // memory access issued in the same iteration.
-template <typename SymT, bool IB0, bool WIDE>
+// FLT: the stream's inputs are float latents: the ring holds scales (as the
+// row source) and y; each group's row is its scale's table row and its
+// symbol rint(y - mean), the means read one group ahead with plain loads.
+template <typename SymT, bool IB0, bool WIDE, bool FLT>
 __device__ __forceinline__ void encode_stream_w32(const EncCtx &c, const StreamDesc &d,
                                                   const RowMeta *meta, const uint32_t *buckets,
                                                   uint32_t *stg, int64_t s) {
-  constexpr bool kStageSym = sizeof(SymT) == 4;
+  constexpr bool kStageSym = FLT || sizeof(SymT) == 4;
   constexpr int kS = kEncStage;
   const int lane = threadIdx.x & 31;
   uint32_t *end = reinterpret_cast<uint32_t *>(c.scratch + slot_end(c.g, d, s));
@@ -243,15 +251,42 @@ __device__ __forceinline__ void encode_stream_w32(const EncCtx &c, const StreamD
   Stepper<WIDE> pl;
   pl.init(d.t, (G - 1) * 32 + lane);
   Stepper<WIDE> pn = pl;  // narrow symbols: position of the next load
+  const float *fy_s = FLT ? c.fy + base : nullptr;
+  const float *fs_s = FLT ? c.fscale + base : nullptr;
+  const float *fm_s = FLT && c.fmean ? c.fmean + base : nullptr;
   auto issue = [&](int32_t ki) {
     const int32_t g = G - 1 - ki;
     const int32_t rel = ki < G && lane < n - g * 32 ? pl.rel : 0;
     const int slot = (ki & (kS - 1)) * 32 + lane;
-    cp_async4(stg_idx + slot, IB0 ? idx_s + rel : c.idx + ((base + rel) >> ib));
-    if (kStageSym) cp_async4(stg_sym + slot, sym_s + rel);
-    else prefetch_l2(sym_s + rel);
+    if (FLT) {
+      cp_async4(stg_idx + slot, fs_s + rel);
+      cp_async4(stg_sym + slot, fy_s + rel);
+      if (fm_s) prefetch_l2(fm_s + rel);
+    } else {
+      cp_async4(stg_idx + slot, IB0 ? idx_s + rel : c.idx + ((base + rel) >> ib));
+      if (kStageSym) cp_async4(stg_sym + slot, sym_s + rel);
+      else prefetch_l2(sym_s + rel);
+    }
     cp_async_commit();
     pl.back(32);
+  };
+  // FLT: the row of a staged scale, and the symbol of a staged y with its
+  // mean (an out-of-range value is recorded and coded as 0)
+  auto row_of = [&](uint32_t v) -> uint32_t {
+    if (!FLT) return v;
+    return scale_row(bound_scale(__uint_as_float(v), c.bound), c.stab, c.K, c.stab_top);
+  };
+  auto quant = [&](int32_t ybits, float mean) -> int32_t {
+    bool ok;
+    const int32_t q = quantize(__int_as_float(ybits), mean, ok);
+    st.range_err |= !ok;
+    return q;
+  };
+  Stepper<WIDE> pm = pl;  // FLT: position of the next mean load
+  auto mean_of = [&](int32_t ki, bool valid) -> float {
+    const float v = fm_s && valid ? __ldg(fm_s + pm.rel) : 0.0f;
+    pm.back(32);
+    return v;
   };
   auto ring = [&](int32_t ki) { return (ki & (kS - 1)) * 32 + lane; };
   auto meta_of = [&](uint32_t r) -> RowMeta {
@@ -271,19 +306,25 @@ __device__ __forceinline__ void encode_stream_w32(const EncCtx &c, const StreamD
   // group G - 1 (coded first) may be partial
   const bool active0 = lane < n - (G - 1) * 32;
   int32_t s0;
-  if (kStageSym) {
+  if (FLT) {
+    const float mean0 = mean_of(0, active0);
+    s0 = active0 ? quant(sym_of(0), mean0) : 0;
+  } else if (kStageSym) {
     s0 = sym_of(0);
   } else {
     s0 = SymIO<SymT>::load(sym_s, active0 ? pn.rel : 0);
     pn.back(32);
   }
-  EncLook L = enc_look(enc_bucket(s0, meta_of(stg_idx[ring(0)]), buckets), active0);
+  EncLook L = enc_look(enc_bucket(s0, meta_of(row_of(stg_idx[ring(0)])), buckets), active0);
+  // group 1's symbol (FLT: its y and mean, quantised when used)
   int32_t s1 = G > 1 ? sym_of(1) : 0;
-  RowMeta m1 = meta_of(G > 1 ? stg_idx[ring(1)] : 0u);
-  uint32_t r2 = G > 2 ? stg_idx[ring(2)] : 0u;
+  float mean1 = FLT && G > 1 ? mean_of(1, true) : 0.0f;
+  RowMeta m1 = meta_of(G > 1 ? row_of(stg_idx[ring(1)]) : 0u);
+  uint32_t r2 = G > 2 ? row_of(stg_idx[ring(2)]) : 0u;
 
   auto step = [&](int32_t k, bool active, auto full) {
     // group k+1's bucket (after the last group: row 0, unused)
+    if (FLT) s1 = k + 1 < G ? quant(s1, mean1) : 0;
     const EncBucket b1 = enc_bucket(s1, m1, buckets);
     // group k's state update
     const uint64_t x0 = st.x;
@@ -295,11 +336,13 @@ __device__ __forceinline__ void encode_stream_w32(const EncCtx &c, const StreamD
     issue(k + kS - 1);
     cp_async_wait<kS - 4>();  // coded groups up to k + 3 have landed
     const int32_t s2 = k + 2 < G ? sym_of(k + 2) : 0;
+    const float mean2 = FLT && k + 2 < G ? mean_of(k + 2, true) : 0.0f;
     const RowMeta m2 = meta_of(r2);
-    const uint32_t r3 = k + 3 < G ? stg_idx[ring(k + 3)] : 0u;
+    const uint32_t r3 = k + 3 < G ? row_of(stg_idx[ring(k + 3)]) : 0u;
     if (L.any_esc) enc_group_escape(st, x0, c0, L, active, end);
     L = L1;
     s1 = s2;
+    mean1 = mean2;
     m1 = m2;
     r2 = r3;
   };
@@ -322,7 +365,7 @@ __device__ __forceinline__ void encode_stream_w32(const EncCtx &c, const StreamD
   if (lane == 0) c.lens[s] = 4ull * (st.cursor + 64);
 }
 
-template <typename SymT, bool IB0>
+template <typename SymT, bool IB0, bool FLT>
 __device__ __forceinline__ void encode_stream_w32_entry(const EncCtx &c, const RowMeta *meta,
                                                         const uint32_t *buckets, uint32_t *stg,
                                                         int64_t s) {
@@ -340,12 +383,12 @@ __device__ __forceinline__ void encode_stream_w32_entry(const EncCtx &c, const R
     return;
   }
   if (d.t.ww >= 32)
-    encode_stream_w32<SymT, IB0, true>(c, d, meta, buckets, stg, s);
+    encode_stream_w32<SymT, IB0, true, FLT>(c, d, meta, buckets, stg, s);
   else
-    encode_stream_w32<SymT, IB0, false>(c, d, meta, buckets, stg, s);
+    encode_stream_w32<SymT, IB0, false, FLT>(c, d, meta, buckets, stg, s);
 }
 
-template <typename SymT>
+template <typename SymT, bool FLT>
 __device__ void encode_stream_w1(const EncCtx &c, const RowMeta *meta, const uint32_t *buckets,
                                  int64_t s) {
   const StreamDesc d = stream_desc(c.g, s);
@@ -365,8 +408,13 @@ __device__ void encode_stream_w1(const EncCtx &c, const RowMeta *meta, const uin
   constexpr int32_t kAhead = 64;
   for (int32_t u = 0; u < kAhead && u < n; ++u) {
     const int64_t p = d.base + pp.rel(t);
-    prefetch_l2(reinterpret_cast<const SymT *>(c.sym) + p);
-    prefetch_l2(c.idx + (p >> ib));
+    if (FLT) {
+      prefetch_l2(c.fy + p);
+      prefetch_l2(c.fscale + p);
+    } else {
+      prefetch_l2(reinterpret_cast<const SymT *>(c.sym) + p);
+      prefetch_l2(c.idx + (p >> ib));
+    }
     pp.back(t, 1);
   }
   for (int32_t i = n - 1; i >= 0; --i) {
@@ -374,12 +422,28 @@ __device__ void encode_stream_w1(const EncCtx &c, const RowMeta *meta, const uin
     pl.back(t, 1);
     if (i - kAhead >= 0) {
       const int64_t q = d.base + pp.rel(t);
-      prefetch_l2(reinterpret_cast<const SymT *>(c.sym) + q);
-      prefetch_l2(c.idx + (q >> ib));
+      if (FLT) {
+        prefetch_l2(c.fy + q);
+        prefetch_l2(c.fscale + q);
+      } else {
+        prefetch_l2(reinterpret_cast<const SymT *>(c.sym) + q);
+        prefetch_l2(c.idx + (q >> ib));
+      }
       pp.back(t, 1);
     }
-    const int32_t sv = SymIO<SymT>::load(c.sym, p);
-    const int32_t r = __ldg(c.idx + (p >> ib));
+    int32_t sv, r;
+    if (FLT) {
+      bool ok;
+      sv = quantize(__ldg(c.fy + p), c.fmean ? __ldg(c.fmean + p) : 0.0f, ok);
+      if (!ok) {
+        report(c.status, RANS_ERR_RANGE, s);
+        return;
+      }
+      r = (int32_t)scale_row(bound_scale(__ldg(c.fscale + p), c.bound), c.stab, c.K, c.stab_top);
+    } else {
+      sv = SymIO<SymT>::load(c.sym, p);
+      r = __ldg(c.idx + (p >> ib));
+    }
     if ((uint32_t)r >= (uint32_t)c.K) {
       report(c.status, RANS_ERR_INDEX, s);
       return;
@@ -400,7 +464,7 @@ __device__ void encode_stream_w1(const EncCtx &c, const RowMeta *meta, const uin
   c.lens[s] = 4ull * cursor;
 }
 
-template <int W, typename SymT, bool SMEM, bool IB0>
+template <int W, typename SymT, bool SMEM, bool IB0, bool FLT>
 __global__ void __launch_bounds__(W == 32 ? kEncThreads32 : kEncThreads1)
     encode_kernel(EncCtx c) {
   extern __shared__ __align__(16) unsigned char smem[];
@@ -423,11 +487,11 @@ __global__ void __launch_bounds__(W == 32 ? kEncThreads32 : kEncThreads1)
                     warp * kEncStage * 32 * 2;
     for (int64_t k = blockIdx.x + (int64_t)gridDim.x * warp; k < c.g.S;
          k += (int64_t)gridDim.x * nw)
-      encode_stream_w32_entry<SymT, IB0>(c, meta, buckets, stg, stream_of(c.g, k));
+      encode_stream_w32_entry<SymT, IB0, FLT>(c, meta, buckets, stg, stream_of(c.g, k));
   } else {
     for (int64_t k = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; k < c.g.S;
          k += (int64_t)gridDim.x * blockDim.x)
-      encode_stream_w1<SymT>(c, meta, buckets, stream_of(c.g, k));
+      encode_stream_w1<SymT, FLT>(c, meta, buckets, stream_of(c.g, k));
   }
 }
 
@@ -509,9 +573,9 @@ __global__ void debug_divide_kernel(const uint64_t *x, const uint32_t *f, int64_
   }
 }
 
-template <int W, typename SymT, bool SMEM, bool IB0>
+template <int W, typename SymT, bool SMEM, bool IB0, bool FLT>
 int launch_encode_t(const EncCtx &c, cudaStream_t st) {
-  auto kern = encode_kernel<W, SymT, SMEM, IB0>;
+  auto kern = encode_kernel<W, SymT, SMEM, IB0, FLT>;
   const uint32_t tab = SMEM ? c.meta_bytes + c.bucket_bytes : 0;
   const uint32_t per_warp = W == 32 ? kEncStage * 32 * 4 * 2 : 0;
   uint32_t smem = tab;
@@ -564,10 +628,10 @@ template <int W, typename SymT>
 int launch_encode_w(const EncCtx &c, bool smem, cudaStream_t st) {
   const bool ib0 = c.g.ib_shift == 0;
   if (smem)
-    return ib0 ? launch_encode_t<W, SymT, true, true>(c, st)
-               : launch_encode_t<W, SymT, true, false>(c, st);
-  return ib0 ? launch_encode_t<W, SymT, false, true>(c, st)
-             : launch_encode_t<W, SymT, false, false>(c, st);
+    return ib0 ? launch_encode_t<W, SymT, true, true, false>(c, st)
+               : launch_encode_t<W, SymT, true, false, false>(c, st);
+  return ib0 ? launch_encode_t<W, SymT, false, true, false>(c, st)
+             : launch_encode_t<W, SymT, false, false, false>(c, st);
 }
 
 template <typename SymT>
@@ -592,6 +656,9 @@ int launch_encode(const void *symbols, int sym_dtype, const int32_t *indexes,
   c.scratch = scratch;
   c.lens = lens;
   c.status = status;
+  c.fy = c.fmean = c.fscale = c.stab = nullptr;
+  c.bound = 0.0f;
+  c.stab_top = 0;
   const bool smem = t.enc_in_smem != 0;
   switch (sym_dtype) {
     case RANS_SYM_INT32: return launch_encode_s<int32_t>(c, smem, st);
@@ -599,6 +666,36 @@ int launch_encode(const void *symbols, int sym_dtype, const int32_t *indexes,
     case RANS_SYM_INT16: return launch_encode_s<int16_t>(c, smem, st);
     default: return RANS_ERR_ARG;
   }
+}
+
+int launch_encode_float(const float *y, const float *means, const float *scales,
+                        const float *scale_table, float scale_bound, const rans_tables &t,
+                        const Geom &g, char *scratch, uint64_t *lens, int32_t *status,
+                        cudaStream_t st) {
+  EncCtx c;
+  c.sym = nullptr;
+  c.idx = nullptr;
+  c.fy = y;
+  c.fmean = means;
+  c.fscale = scales;
+  c.stab = scale_table;
+  c.bound = scale_bound;
+  c.stab_top = 0;
+  while (2 * c.stab_top <= t.K - 1 && t.K > 1) c.stab_top = c.stab_top ? 2 * c.stab_top : 1;
+  c.K = t.K;
+  c.meta_bytes = t.meta_bytes;
+  c.bucket_bytes = t.bucket_bytes;
+  c.blob = reinterpret_cast<const char *>(t.blob);
+  c.g = g;
+  c.scratch = scratch;
+  c.lens = lens;
+  c.status = status;
+  const bool smem = t.enc_in_smem != 0;
+  if (g.W == 32)
+    return smem ? launch_encode_t<32, int32_t, true, true, true>(c, st)
+                : launch_encode_t<32, int32_t, false, true, true>(c, st);
+  return smem ? launch_encode_t<1, int32_t, true, true, true>(c, st)
+              : launch_encode_t<1, int32_t, false, true, true>(c, st);
 }
 
 int launch_compact(const Geom &g, const char *scratch, const uint64_t *lens, uint8_t *out,

@@ -347,6 +347,37 @@ __device__ __forceinline__ void st_global(uint32_t *p, uint32_t v) { __stcg(p, v
 __device__ __forceinline__ void st_global(int32_t *p, int32_t v) { __stcs(p, v); }
 __device__ __forceinline__ void st_global(int16_t *p, int16_t v) { __stcs(p, v); }
 __device__ __forceinline__ void st_global(uint8_t *p, uint8_t v) { __stcs(p, v); }
+__device__ __forceinline__ void st_global(float *p, float v) { __stcs(p, v); }
+
+// ------------------------------------------------------ float latents --
+// For coders that start from float latents (a mean-scale model's y, means
+// and scales) instead of int32 symbols and row indexes: the pages name
+// CompressAI's build_indexes and symbol = round(y - mean) without spelling
+// them out, so the library takes their plain reading.
+//
+// Row of a scale s: the first of the K table entries (increasing) that is
+// >= max(s, bound), a NaN scale counting as the bound; the last row when none
+// of the first K - 1 is.  A binary search with the same steps on every lane:
+// pos counts the entries below s among the first K - 1.
+__device__ __forceinline__ uint32_t scale_row(float s, const float *table, int K, int top) {
+  // top: the largest power of two <= K - 1 (0 when K == 1)
+  int pos = 0;
+  for (int step = top; step > 0; step >>= 1)
+    if (pos + step <= K - 1 && __ldg(table + pos + step - 1) < s) pos += step;
+  return (uint32_t)pos;
+}
+__device__ __forceinline__ float bound_scale(float s, float bound) {
+  return s >= bound ? s : bound;  // NaN fails the compare: the bound
+}
+
+// Symbol of y given its mean: y - mean in float32, rounded to the nearest
+// integer, ties to even.  ok is false (symbol 0) when it is not finite or not
+// an int32.
+__device__ __forceinline__ int32_t quantize(float y, float mean, bool &ok) {
+  const float r = rintf(y - mean);
+  ok = r >= -2147483648.0f && r < 2147483648.0f;
+  return ok ? (int32_t)r : 0;
+}
 
 // ------------------------------------------------------------- symbols --
 template <typename T> struct SymIO;

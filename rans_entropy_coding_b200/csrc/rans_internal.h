@@ -30,10 +30,24 @@ int prepare_tables(const int32_t *cdfs, int K, int Lmax, const int32_t *lengths,
 int launch_encode(const void *symbols, int sym_dtype, const int32_t *indexes,
                   const rans_tables &t, const Geom &g, char *scratch, uint64_t *lens,
                   int32_t *status, cudaStream_t st);
+// Float latents in (one scale per element): rows from the scale table, symbols
+// rint(y - mean); same outputs as launch_encode.
+int launch_encode_float(const float *y, const float *means, const float *scales,
+                        const float *scale_table, float scale_bound, const rans_tables &t,
+                        const Geom &g, char *scratch, uint64_t *lens, int32_t *status,
+                        cudaStream_t st);
 // Compaction: exclusive scan of lens into offsets[S+1], then a copy of every
 // stream from the end of its scratch slot to out + offsets[k].
 int launch_compact(const Geom &g, const char *scratch, const uint64_t *lens, uint8_t *out,
                    uint64_t out_capacity, uint64_t *offsets, int32_t *status, cudaStream_t st);
+// Float values out: float(symbol) + mean, rows from the scales.
+int launch_decode_float(const uint8_t *in, uint64_t in_bytes, const uint64_t *offsets,
+                        const float *scales, const float *means, const float *scale_table,
+                        float scale_bound, const rans_tables &t, const Geom &g, float *values,
+                        int32_t *status, cudaStream_t st);
+// Row index of every scale (the float latents' rows), one thread per element.
+int launch_build_indexes(const float *scales, int64_t n, const float *scale_table, int32_t K,
+                         float scale_bound, int32_t *indexes, cudaStream_t st);
 int launch_decode(const uint8_t *in, uint64_t in_bytes, const uint64_t *offsets,
                   const int32_t *indexes, const rans_tables &t, const Geom &g, void *symbols,
                   int sym_dtype, int32_t *status, cudaStream_t st);

@@ -556,6 +556,14 @@ __global__ void __launch_bounds__(kSlotThreads)
   fill_row_slots(row, len - 1, slot_base(m.slot), (int)slot_shift(m.slot), slots, ca, srow);
 }
 
+// Row index of every scale (scale_row in rans_common.cuh).
+__global__ void build_indexes_kernel(const float *scales, int64_t n, const float *table, int K,
+                                     int top, float bound, int32_t *indexes) {
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n;
+       i += (int64_t)gridDim.x * blockDim.x)
+    indexes[i] = (int32_t)scale_row(bound_scale(__ldg(scales + i), bound), table, K, top);
+}
+
 int ceil_log2(int64_t v) {
   int q = 0;
   while ((int64_t(1) << q) < v) ++q;
@@ -583,6 +591,21 @@ int launch_pmf_rows(const float *pmfs, int K, int stride, const int32_t *pmf_len
                     cudaStream_t st) {
   pmf_rows_kernel<<<K, kRowThreads, 0, st>>>(pmfs, stride, pmf_lengths, tail, cdfs, Lmax,
                                               lengths);
+  return cudaGetLastError() == cudaSuccess ? RANS_OK : RANS_ERR_CUDA;
+}
+
+int launch_build_indexes(const float *scales, int64_t n, const float *scale_table, int32_t K,
+                         float scale_bound, int32_t *indexes, cudaStream_t st) {
+  if (n <= 0) return RANS_OK;
+  int top = 0;
+  while (K > 1 && 2 * top <= K - 1) top = top ? 2 * top : 1;
+  int dev = 0;
+  cudaGetDevice(&dev);
+  int64_t blocks = (n + 255) / 256;
+  const int64_t cap = 16LL * num_sms(dev);
+  if (blocks > cap) blocks = cap;
+  build_indexes_kernel<<<(unsigned)blocks, 256, 0, st>>>(scales, n, scale_table, K, top,
+                                                         scale_bound, indexes);
   return cudaGetLastError() == cudaSuccess ? RANS_OK : RANS_ERR_CUDA;
 }
 

@@ -413,3 +413,63 @@ def test_table_refresh_matches_fresh_prepare():
     bad_l[3] += 2
     rb.check(rb.rans_tables_refresh(dc2, bad_l, do2, tables))
     assert rb.rans_get_status(tables.blob) == rb.ERR_TABLE
+
+
+# -------------------------------------------------------- float latents --
+def _float_case(W=32, with_means=True, n_images=1, **kw):
+    w = WL.y_float(n_images=n_images, W=W, with_means=with_means, **kw)
+    c, l, o = O.build_cdfs_from_scales(w["scales"], w["tail_mass"])
+    rows = O.build_indexes(w["fscales"], w["scales"], w["scale_bound"]).reshape(-1)
+    sym = O.quantize(w["y"], w["means"]).reshape(-1)
+    wi = dict(w, symbols=sym, indexes=rows)
+    return w, wi, (c, l, o)
+
+
+def test_build_indexes_matches_oracle():
+    t = WL.log_spaced_scales(WL.SCALE_MIN, WL.SCALE_MAX_Y, WL.N_ROWS_Y).astype(np.float32)
+    rng = np.random.Generator(np.random.PCG64(31))
+    s = np.concatenate([np.exp(rng.uniform(np.log(1e-3), np.log(1e4), 100000)), t,
+                        np.nextafter(t, np.float32(0)), np.nextafter(t, np.float32(np.inf)),
+                        [0.0, -1.0, np.inf, np.nan]]).astype(np.float32)
+    got = torch.empty(s.size, dtype=torch.int32, device="cuda")
+    rb.check(rb.rans_build_indexes(torch.from_numpy(s).cuda(), torch.from_numpy(t).cuda(),
+                                   WL.SCALE_MIN, got))
+    assert np.array_equal(got.cpu().numpy(), O.build_indexes(s, t, WL.SCALE_MIN))
+
+
+@pytest.mark.parametrize("W,with_means", [(32, True), (32, False), (1, True)])
+def test_encode_from_scales_matches_oracle(W, with_means):
+    """Float latents in: the streams equal the oracle's encode of
+    build_indexes(scales) and rint(y - mean); decoding gives back
+    float32(symbol) + mean exactly."""
+    kw = {} if W == 32 else dict(th=17, tw=30)
+    w, wi, (c, l, o) = _float_case(W=W, with_means=with_means, **kw)
+    want, woffs = oracle_encode(wi, c, l, o)
+    dev = lambda a: None if a is None else torch.from_numpy(np.ascontiguousarray(a).reshape(-1)).cuda()
+    tables = tables_from_numpy(c, l, o)
+    ch = chunking_of(w)
+    table = dev(np.asarray(w["scales"], np.float32))
+    out, offs, ws = rb.encode_from_scales(dev(w["y"]), dev(w["fscales"]), table,
+                                          w["scale_bound"], tables, ch, means=dev(w["means"]))
+    assert rb.rans_get_status(ws.enc) == rb.OK
+    total = int(offs[-1].item())
+    assert offs.cpu().numpy().astype(np.uint64).tolist() == woffs.tolist()
+    assert np.array_equal(out[:total].cpu().numpy(), want)
+    vals, wsd = rb.decode_to_values(out[:total], offs, dev(w["fscales"]), table,
+                                    w["scale_bound"], tables, ch, means=dev(w["means"]))
+    assert rb.rans_get_status(wsd) == rb.OK
+    ref = O.dequantize(wi["symbols"], None if w["means"] is None else w["means"].reshape(-1))
+    assert np.array_equal(vals.cpu().numpy(), ref)
+
+
+def test_encode_from_scales_reports_values_out_of_range():
+    w, wi, (c, l, o) = _float_case(W=32)
+    y = np.array(w["y"], copy=True).reshape(-1)
+    y[12345] = np.inf
+    tables = tables_from_numpy(c, l, o)
+    ch = chunking_of(w)
+    dev = lambda a: torch.from_numpy(np.ascontiguousarray(a).reshape(-1)).cuda()
+    out, offs, ws = rb.encode_from_scales(dev(y), dev(w["fscales"]),
+                                          dev(np.asarray(w["scales"], np.float32)),
+                                          w["scale_bound"], tables, ch, means=dev(w["means"]))
+    assert rb.rans_get_status(ws.enc) == rb.ERR_RANGE

@@ -134,6 +134,27 @@ def many_rows(seed=5000, n=1 << 18, n_rows=256, n_streams=64, W=32):
                 chunking=dict(kind="contig", n_streams=n_streams), W=W, index_block=1)
 
 
+def y_float(seed=6000, n_images=2, cg=4, th=64, tw=64, W=32, with_means=True):
+    """Float latents of a mean-scale model, [n_images, 192, 68, 120]: per
+    element a scale exp(U(ln 0.11, ln 256)), a mean U(-8, 8) (or none) and
+    y = mean + N(0, scale), all float32; the 64-entry scale table and its
+    lower bound 0.11.  Rows and symbols come from the scales and y - mean."""
+    rng = _rng(seed)
+    shape = (n_images,) + Y_SHAPE
+    n = int(np.prod(shape))
+    scales = np.exp(rng.uniform(math.log(SCALE_MIN), math.log(SCALE_MAX_Y), n)).astype(np.float32)
+    means = rng.uniform(-8.0, 8.0, n).astype(np.float32) if with_means else None
+    y = (rng.standard_normal(n) * scales.astype(np.float64)).astype(np.float32)
+    if means is not None:
+        y = (y + means).astype(np.float32)
+    return dict(name="y_float", y=y.reshape(shape), means=None if means is None else
+                means.reshape(shape), fscales=scales.reshape(shape),
+                scales=log_spaced_scales(SCALE_MIN, SCALE_MAX_Y, N_ROWS_Y), tail_mass=1e-9,
+                scale_bound=SCALE_MIN,
+                chunking=dict(kind="tiled", shape=shape, cg=cg, th=th, tw=tw), W=W,
+                index_block=1)
+
+
 def y_latent(seed=2000, W=1):
     sym, idx = _y_image(seed)
     return dict(name="y", symbols=sym.reshape((1,) + Y_SHAPE), indexes=idx,
