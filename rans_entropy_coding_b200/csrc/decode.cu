@@ -53,7 +53,7 @@ struct DecCtx {
   // float(symbol) + mean written to `out` as float
   const float *fscale, *fmean, *stab;
   float bound;
-  int32_t stab_top;
+  int32_t stab_smem;  // 1: the kernel copies the scale table into shared memory
 };
 
 __device__ __forceinline__ bool stream_bounds(const DecCtx &c, int64_t s, int W,
@@ -268,7 +268,8 @@ template <typename SymT, bool IB0, bool WIDE, bool SEARCH>
 __device__ __forceinline__ void decode_stream_w32(const DecCtx &c, const StreamDesc &d,
                                                   const RowMeta *meta, const uint16_t *starts,
                                                   const uint32_t *slots, uint32_t *stg,
-                                                  int64_t s, const uint32_t *words, uint64_t nw) {
+                                                  int64_t s, const uint32_t *words, uint64_t nw,
+                                                  const float *stab) {
   constexpr int kS = kDecStage;
   const int lane = threadIdx.x & 31;
   const int32_t n = (int32_t)d.n;
@@ -310,7 +311,7 @@ __device__ __forceinline__ void decode_stream_w32(const DecCtx &c, const StreamD
   };
   auto meta_of = [&](uint32_t v) -> RowMeta {
     const uint32_t r =
-        kFlt ? scale_row(bound_scale(__uint_as_float(v), c.bound), c.stab, c.K, c.stab_top) : v;
+        kFlt ? scale_row(bound_scale(__uint_as_float(v), c.bound), stab, c.K) : v;
     st.rmax = max(st.rmax, r);
     return row_meta(meta, min(r, kmax));
   };
@@ -322,18 +323,24 @@ __device__ __forceinline__ void decode_stream_w32(const DecCtx &c, const StreamD
   for (int32_t u = 0; u < kS - 1; ++u) issue(u);
   cp_async_wait<kS - 2>();
   RowMeta m = meta_of(stg[lane]);
-  float mean = kFlt ? mean_at(0, pc.rel) : 0.0f;
+  // float values: means read two groups ahead (pm: position of the next)
+  Stepper<WIDE> pm = pc;
+  float mean = kFlt ? mean_at(0, pm.rel) : 0.0f;
+  if (kFlt) pm.fwd(32);
+  float mean_n = kFlt ? mean_at(1, pm.rel) : 0.0f;
+  if (kFlt) pm.fwd(32);
 #pragma unroll 1
   for (int32_t g = 0; g + 1 < G; ++g) {
     issue(g + kS - 1);
     cp_async_wait<kS - 2>();  // groups up to g + 1 have landed
     const RowMeta mn = meta_of(stg[((g + 1) & (kS - 1)) * 32 + lane]);
-    const int32_t rel = pc.rel;
+    const float mean_nn = kFlt ? mean_at(g + 2, pm.rel) : 0.0f;
+    if (kFlt) pm.fwd(32);
+    dec_group<SymT, true, SEARCH>(st, m, starts, slots, true, out_s + pc.rel, words, nw, mean);
     pc.fwd(32);
-    const float mean_n = kFlt ? mean_at(g + 1, pc.rel) : 0.0f;
-    dec_group<SymT, true, SEARCH>(st, m, starts, slots, true, out_s + rel, words, nw, mean);
     m = mn;
     mean = mean_n;
+    mean_n = mean_nn;
   }
   dec_group<SymT, false, SEARCH>(st, m, starts, slots, lane < n - (G - 1) * 32, out_s + pc.rel,
                                  words, nw, mean);
@@ -350,7 +357,7 @@ template <typename SymT, bool IB0, bool SEARCH>
 __device__ __forceinline__ void decode_stream_w32_entry(const DecCtx &c, const RowMeta *meta,
                                                         const uint16_t *buckets,
                                                         const uint32_t *slots, uint32_t *stg,
-                                                        int64_t s) {
+                                                        int64_t s, const float *stab) {
   const int lane = threadIdx.x & 31;
   const StreamDesc d = stream_desc(c.g, s);
   const uint32_t *words = nullptr;
@@ -370,14 +377,16 @@ __device__ __forceinline__ void decode_stream_w32_entry(const DecCtx &c, const R
     return;
   }
   if (d.t.ww >= 32)
-    decode_stream_w32<SymT, IB0, true, SEARCH>(c, d, meta, buckets, slots, stg, s, words, nw);
+    decode_stream_w32<SymT, IB0, true, SEARCH>(c, d, meta, buckets, slots, stg, s, words, nw,
+                                               stab);
   else
-    decode_stream_w32<SymT, IB0, false, SEARCH>(c, d, meta, buckets, slots, stg, s, words, nw);
+    decode_stream_w32<SymT, IB0, false, SEARCH>(c, d, meta, buckets, slots, stg, s, words, nw,
+                                                stab);
 }
 
 template <typename SymT>
 __device__ void decode_stream_w1(const DecCtx &c, const RowMeta *meta, const uint16_t *buckets,
-                                 const uint32_t *slots, int64_t s) {
+                                 const uint32_t *slots, int64_t s, const float *stab) {
   const StreamDesc d = stream_desc(c.g, s);
   const uint32_t *words = nullptr;
   uint64_t nw = 0;
@@ -421,8 +430,7 @@ __device__ void decode_stream_w1(const DecCtx &c, const RowMeta *meta, const uin
       pp.fwd(t, 1);
     }
     const int32_t r =
-        kFlt ? (int32_t)scale_row(bound_scale(__ldg(c.fscale + p), c.bound), c.stab, c.K,
-                                  c.stab_top)
+        kFlt ? (int32_t)scale_row(bound_scale(__ldg(c.fscale + p), c.bound), stab, c.K)
              : __ldg(c.idx + (p >> ib));
     if ((uint32_t)r >= (uint32_t)c.K) {
       report(c.status, RANS_ERR_INDEX, s);
@@ -490,6 +498,16 @@ __global__ void __launch_bounds__(W == 32 ? kDecMaxThreads32 : kDecThreads1)
     buckets = reinterpret_cast<const uint16_t *>(gb + c.meta_bytes + c.bucket_bytes);
     slots = reinterpret_cast<const uint32_t *>(gb + c.meta_bytes + c.bucket_bytes + c.start_bytes);
   }
+  // float values: the scale table, copied after the stage rings when it fits
+  const float *stab = c.stab;
+  if (std::is_same<SymT, float>::value && c.stab_smem) {
+    float *t = reinterpret_cast<float *>(
+        smem + (SMEM ? c.meta_bytes + c.start_bytes + c.slot_bytes : 0) +
+        (W == 32 ? (blockDim.x >> 5) * (uint32_t)(kDecStage * 32 * 4) : 0));
+    for (int i = threadIdx.x; i < c.K; i += blockDim.x) t[i] = c.stab[i];
+    __syncthreads();
+    stab = t;
+  }
   if (W == 32) {
     const int warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
     uint32_t *stg = reinterpret_cast<uint32_t *>(
@@ -500,14 +518,16 @@ __global__ void __launch_bounds__(W == 32 ? kDecMaxThreads32 : kDecThreads1)
     for (int64_t k = blockIdx.x + (int64_t)gridDim.x * warp; k < c.g.S;
          k += (int64_t)gridDim.x * nw) {
       if (search)
-        decode_stream_w32_entry<SymT, IB0, true>(c, meta, buckets, slots, stg, stream_of(c.g, k));
+        decode_stream_w32_entry<SymT, IB0, true>(c, meta, buckets, slots, stg, stream_of(c.g, k),
+                                                 stab);
       else
-        decode_stream_w32_entry<SymT, IB0, false>(c, meta, buckets, slots, stg, stream_of(c.g, k));
+        decode_stream_w32_entry<SymT, IB0, false>(c, meta, buckets, slots, stg,
+                                                  stream_of(c.g, k), stab);
     }
   } else {
     for (int64_t k = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; k < c.g.S;
          k += (int64_t)gridDim.x * blockDim.x)
-      decode_stream_w1<SymT>(c, meta, buckets, slots, stream_of(c.g, k));
+      decode_stream_w1<SymT>(c, meta, buckets, slots, stream_of(c.g, k), stab);
   }
 }
 
@@ -518,8 +538,13 @@ int launch_decode_t(const DecCtx &c, cudaStream_t st) {
   const uint32_t per_warp = W == 32 ? kDecStage * 32 * 4 : 0;
   int dev = 0;
   cudaGetDevice(&dev);
-  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           (int)(tab + kDecStageBytes)) != cudaSuccess)
+  // float latents: the scale table goes after the stage rings when it fits
+  const uint32_t tbl = std::is_same<SymT, float>::value ? (uint32_t)pad16(4ull * (uint64_t)c.K) : 0u;
+  const int optin = smem_optin(dev);
+  const uint32_t lim = (uint32_t)optin - 64u;  // room for the kernel's static shared memory
+  const uint32_t max_dyn = tab + kDecStageBytes + tbl <= lim ? tab + kDecStageBytes + tbl : lim;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)max_dyn) !=
+      cudaSuccess)
     return RANS_ERR_CUDA;
   const int sms = num_sms(dev);
   int threads, blocks;
@@ -557,7 +582,10 @@ int launch_decode_t(const DecCtx &c, cudaStream_t st) {
     blocks = (int)(need < cap ? need : cap);
   }
   if (blocks < 1) blocks = 1;
-  kern<<<blocks, threads, smem, st>>>(c);
+  DecCtx cc = c;
+  cc.stab_smem = tbl > 0 && smem + tbl <= max_dyn ? 1 : 0;
+  if (cc.stab_smem) smem += tbl;
+  kern<<<blocks, threads, smem, st>>>(cc);
   return cudaGetLastError() == cudaSuccess ? RANS_OK : RANS_ERR_CUDA;
 }
 
@@ -601,8 +629,6 @@ int launch_decode_float(const uint8_t *in, uint64_t in_bytes, const uint64_t *of
   c.fmean = means;
   c.stab = scale_table;
   c.bound = scale_bound;
-  c.stab_top = 0;
-  while (2 * c.stab_top <= t.K - 1 && t.K > 1) c.stab_top = c.stab_top ? 2 * c.stab_top : 1;
   const bool smem = t.dec_in_smem != 0;
   return g.W == 32 ? launch_decode_w<32, float>(c, smem, st)
                    : launch_decode_w<1, float>(c, smem, st);
@@ -627,7 +653,7 @@ int launch_decode(const uint8_t *in, uint64_t in_bytes, const uint64_t *offsets,
   c.status = status;
   c.fscale = c.fmean = c.stab = nullptr;
   c.bound = 0.0f;
-  c.stab_top = 0;
+  c.stab_smem = 0;
   const bool smem = t.dec_in_smem != 0;
   switch (sym_dtype) {
     case RANS_SYM_INT32: return launch_decode_s<int32_t>(c, smem, st);

@@ -26,6 +26,15 @@ namespace rb {
 namespace {
 
 constexpr int kEncThreads32 = kEncMaxWarps * 32;
+
+// Per-warp ring: 16 groups of row indexes and symbols, or for float latents
+// 8 groups of scales, y and means (the same shared memory budget).
+__host__ __device__ constexpr int enc_ring_groups(bool flt) { return flt ? 8 : kEncStage; }
+__host__ __device__ constexpr uint32_t enc_stage_bytes_per_warp(bool flt) {
+  return (uint32_t)enc_ring_groups(flt) * 32u * 4u * (flt ? 3u : 2u);
+}
+static_assert(enc_stage_bytes_per_warp(true) <= enc_stage_bytes_per_warp(false),
+              "the float ring fits the shared memory the tables leave for rings");
 constexpr int kEncThreads1 = 128;
 
 struct EncCtx {
@@ -35,7 +44,7 @@ struct EncCtx {
   // (or null), scales, the K-entry scale table, its lower bound
   const float *fy, *fmean, *fscale, *stab;
   float bound;
-  int32_t stab_top;  // largest power of two <= K - 1
+  int32_t stab_smem; // 1: the kernel copies the scale table into shared memory
   int32_t K;
   uint32_t meta_bytes, bucket_bytes;
   const char *blob;
@@ -216,15 +225,15 @@ __device__ __forceinline__ void enc_group_escape(WarpEnc &st, uint64_t x0, uint3
 // of groups k+2 (symbols, row metadata) and k+3 (row index); group k's rare
 // escape path comes last.  Nothing in group k's state chain waits on a
 // memory access issued in the same iteration.
-// FLT: the stream's inputs are float latents: the ring holds scales (as the
-// row source) and y; each group's row is its scale's table row and its
-// symbol rint(y - mean), the means read one group ahead with plain loads.
+// FLT: the stream's inputs are float latents: an 8-group ring holds scales
+// (as the row source), y and the means; each group's row is its scale's
+// table row and its symbol rint(y - mean).
 template <typename SymT, bool IB0, bool WIDE, bool FLT>
 __device__ __forceinline__ void encode_stream_w32(const EncCtx &c, const StreamDesc &d,
                                                   const RowMeta *meta, const uint32_t *buckets,
-                                                  uint32_t *stg, int64_t s) {
+                                                  uint32_t *stg, int64_t s, const float *stab) {
   constexpr bool kStageSym = FLT || sizeof(SymT) == 4;
-  constexpr int kS = kEncStage;
+  constexpr int kS = enc_ring_groups(FLT);
   const int lane = threadIdx.x & 31;
   uint32_t *end = reinterpret_cast<uint32_t *>(c.scratch + slot_end(c.g, d, s));
   const int32_t n = (int32_t)d.n;
@@ -237,6 +246,7 @@ __device__ __forceinline__ void encode_stream_w32(const EncCtx &c, const StreamD
   const uint32_t above = 0xfffffffeu << lane;   // lanes > this lane
   uint32_t *stg_idx = stg;
   uint32_t *stg_sym = stg + kS * 32;
+  uint32_t *stg_mean = stg + 2 * kS * 32;  // FLT
   WarpEnc st;
   st.x = kL;
   st.cursor = 0;
@@ -261,7 +271,7 @@ __device__ __forceinline__ void encode_stream_w32(const EncCtx &c, const StreamD
     if (FLT) {
       cp_async4(stg_idx + slot, fs_s + rel);
       cp_async4(stg_sym + slot, fy_s + rel);
-      if (fm_s) prefetch_l2(fm_s + rel);
+      if (fm_s) cp_async4(stg_mean + slot, fm_s + rel);
     } else {
       cp_async4(stg_idx + slot, IB0 ? idx_s + rel : c.idx + ((base + rel) >> ib));
       if (kStageSym) cp_async4(stg_sym + slot, sym_s + rel);
@@ -274,7 +284,7 @@ __device__ __forceinline__ void encode_stream_w32(const EncCtx &c, const StreamD
   // mean (an out-of-range value is recorded and coded as 0)
   auto row_of = [&](uint32_t v) -> uint32_t {
     if (!FLT) return v;
-    return scale_row(bound_scale(__uint_as_float(v), c.bound), c.stab, c.K, c.stab_top);
+    return scale_row(bound_scale(__uint_as_float(v), c.bound), stab, c.K);
   };
   auto quant = [&](int32_t ybits, float mean) -> int32_t {
     bool ok;
@@ -282,11 +292,9 @@ __device__ __forceinline__ void encode_stream_w32(const EncCtx &c, const StreamD
     st.range_err |= !ok;
     return q;
   };
-  Stepper<WIDE> pm = pl;  // FLT: position of the next mean load
-  auto mean_of = [&](int32_t ki, bool valid) -> float {
-    const float v = fm_s && valid ? __ldg(fm_s + pm.rel) : 0.0f;
-    pm.back(32);
-    return v;
+  // FLT: the mean of coded group ki's element (from the ring, like y)
+  auto mean_of = [&](int32_t ki) -> float {
+    return fm_s ? __uint_as_float(stg_mean[(ki & (kS - 1)) * 32 + lane]) : 0.0f;
   };
   auto ring = [&](int32_t ki) { return (ki & (kS - 1)) * 32 + lane; };
   auto meta_of = [&](uint32_t r) -> RowMeta {
@@ -307,8 +315,7 @@ __device__ __forceinline__ void encode_stream_w32(const EncCtx &c, const StreamD
   const bool active0 = lane < n - (G - 1) * 32;
   int32_t s0;
   if (FLT) {
-    const float mean0 = mean_of(0, active0);
-    s0 = active0 ? quant(sym_of(0), mean0) : 0;
+    s0 = active0 ? quant(sym_of(0), mean_of(0)) : 0;
   } else if (kStageSym) {
     s0 = sym_of(0);
   } else {
@@ -318,7 +325,7 @@ __device__ __forceinline__ void encode_stream_w32(const EncCtx &c, const StreamD
   EncLook L = enc_look(enc_bucket(s0, meta_of(row_of(stg_idx[ring(0)])), buckets), active0);
   // group 1's symbol (FLT: its y and mean, quantised when used)
   int32_t s1 = G > 1 ? sym_of(1) : 0;
-  float mean1 = FLT && G > 1 ? mean_of(1, true) : 0.0f;
+  float mean1 = FLT && G > 1 ? mean_of(1) : 0.0f;
   RowMeta m1 = meta_of(G > 1 ? row_of(stg_idx[ring(1)]) : 0u);
   uint32_t r2 = G > 2 ? row_of(stg_idx[ring(2)]) : 0u;
 
@@ -336,7 +343,7 @@ __device__ __forceinline__ void encode_stream_w32(const EncCtx &c, const StreamD
     issue(k + kS - 1);
     cp_async_wait<kS - 4>();  // coded groups up to k + 3 have landed
     const int32_t s2 = k + 2 < G ? sym_of(k + 2) : 0;
-    const float mean2 = FLT && k + 2 < G ? mean_of(k + 2, true) : 0.0f;
+    const float mean2 = FLT && k + 2 < G ? mean_of(k + 2) : 0.0f;
     const RowMeta m2 = meta_of(r2);
     const uint32_t r3 = k + 3 < G ? row_of(stg_idx[ring(k + 3)]) : 0u;
     if (L.any_esc) enc_group_escape(st, x0, c0, L, active, end);
@@ -368,7 +375,7 @@ __device__ __forceinline__ void encode_stream_w32(const EncCtx &c, const StreamD
 template <typename SymT, bool IB0, bool FLT>
 __device__ __forceinline__ void encode_stream_w32_entry(const EncCtx &c, const RowMeta *meta,
                                                         const uint32_t *buckets, uint32_t *stg,
-                                                        int64_t s) {
+                                                        int64_t s, const float *stab) {
   const StreamDesc d = stream_desc(c.g, s);
   if (!d.ok) {
     if ((threadIdx.x & 31) == 0) report(c.status, RANS_ERR_ARG, s);
@@ -383,14 +390,14 @@ __device__ __forceinline__ void encode_stream_w32_entry(const EncCtx &c, const R
     return;
   }
   if (d.t.ww >= 32)
-    encode_stream_w32<SymT, IB0, true, FLT>(c, d, meta, buckets, stg, s);
+    encode_stream_w32<SymT, IB0, true, FLT>(c, d, meta, buckets, stg, s, stab);
   else
-    encode_stream_w32<SymT, IB0, false, FLT>(c, d, meta, buckets, stg, s);
+    encode_stream_w32<SymT, IB0, false, FLT>(c, d, meta, buckets, stg, s, stab);
 }
 
 template <typename SymT, bool FLT>
 __device__ void encode_stream_w1(const EncCtx &c, const RowMeta *meta, const uint32_t *buckets,
-                                 int64_t s) {
+                                 int64_t s, const float *stab) {
   const StreamDesc d = stream_desc(c.g, s);
   if (!d.ok) {
     report(c.status, RANS_ERR_ARG, s);
@@ -439,7 +446,7 @@ __device__ void encode_stream_w1(const EncCtx &c, const RowMeta *meta, const uin
         report(c.status, RANS_ERR_RANGE, s);
         return;
       }
-      r = (int32_t)scale_row(bound_scale(__ldg(c.fscale + p), c.bound), c.stab, c.K, c.stab_top);
+      r = (int32_t)scale_row(bound_scale(__ldg(c.fscale + p), c.bound), stab, c.K);
     } else {
       sv = SymIO<SymT>::load(c.sym, p);
       r = __ldg(c.idx + (p >> ib));
@@ -481,17 +488,27 @@ __global__ void __launch_bounds__(W == 32 ? kEncThreads32 : kEncThreads1)
     meta = reinterpret_cast<const RowMeta *>(c.blob + kHeaderBytes);
     buckets = reinterpret_cast<const uint32_t *>(c.blob + kHeaderBytes + c.meta_bytes);
   }
+  // FLT: the scale table, copied after the stage rings when it fits
+  const float *stab = c.stab;
+  if (FLT && c.stab_smem) {
+    float *t = reinterpret_cast<float *>(
+        smem + (SMEM ? c.meta_bytes + c.bucket_bytes : 0) +
+        (W == 32 ? (blockDim.x >> 5) * enc_stage_bytes_per_warp(FLT) : 0));
+    for (int i = threadIdx.x; i < c.K; i += blockDim.x) t[i] = c.stab[i];
+    __syncthreads();
+    stab = t;
+  }
   if (W == 32) {
     const int warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
     uint32_t *stg = reinterpret_cast<uint32_t *>(smem + (SMEM ? c.meta_bytes + c.bucket_bytes : 0)) +
-                    warp * kEncStage * 32 * 2;
+                    warp * (enc_stage_bytes_per_warp(FLT) / 4);
     for (int64_t k = blockIdx.x + (int64_t)gridDim.x * warp; k < c.g.S;
          k += (int64_t)gridDim.x * nw)
-      encode_stream_w32_entry<SymT, IB0, FLT>(c, meta, buckets, stg, stream_of(c.g, k));
+      encode_stream_w32_entry<SymT, IB0, FLT>(c, meta, buckets, stg, stream_of(c.g, k), stab);
   } else {
     for (int64_t k = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; k < c.g.S;
          k += (int64_t)gridDim.x * blockDim.x)
-      encode_stream_w1<SymT, FLT>(c, meta, buckets, stream_of(c.g, k));
+      encode_stream_w1<SymT, FLT>(c, meta, buckets, stream_of(c.g, k), stab);
   }
 }
 
@@ -577,12 +594,17 @@ template <int W, typename SymT, bool SMEM, bool IB0, bool FLT>
 int launch_encode_t(const EncCtx &c, cudaStream_t st) {
   auto kern = encode_kernel<W, SymT, SMEM, IB0, FLT>;
   const uint32_t tab = SMEM ? c.meta_bytes + c.bucket_bytes : 0;
-  const uint32_t per_warp = W == 32 ? kEncStage * 32 * 4 * 2 : 0;
+  const uint32_t per_warp = W == 32 ? enc_stage_bytes_per_warp(FLT) : 0;
   uint32_t smem = tab;
   int dev = 0;
   cudaGetDevice(&dev);
-  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           (int)(tab + kEncStageBytes)) != cudaSuccess)
+  // float latents: the scale table goes after the stage rings when it fits
+  const uint32_t tbl = FLT ? (uint32_t)pad16(4ull * (uint64_t)c.K) : 0u;
+  const int optin = smem_optin(dev);
+  const uint32_t lim = (uint32_t)optin - 64u;  // room for the kernel's static shared memory
+  const uint32_t max_dyn = tab + kEncStageBytes + tbl <= lim ? tab + kEncStageBytes + tbl : lim;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)max_dyn) !=
+      cudaSuccess)
     return RANS_ERR_CUDA;
   const int sms = num_sms(dev);
   int threads;
@@ -620,7 +642,10 @@ int launch_encode_t(const EncCtx &c, cudaStream_t st) {
     blocks = need < cap ? need : cap;
   }
   if (blocks < 1) blocks = 1;
-  kern<<<(unsigned)blocks, threads, smem, st>>>(c);
+  EncCtx cc = c;
+  cc.stab_smem = tbl > 0 && smem + tbl <= max_dyn ? 1 : 0;
+  if (cc.stab_smem) smem += tbl;
+  kern<<<(unsigned)blocks, threads, smem, st>>>(cc);
   return cudaGetLastError() == cudaSuccess ? RANS_OK : RANS_ERR_CUDA;
 }
 
@@ -658,7 +683,7 @@ int launch_encode(const void *symbols, int sym_dtype, const int32_t *indexes,
   c.status = status;
   c.fy = c.fmean = c.fscale = c.stab = nullptr;
   c.bound = 0.0f;
-  c.stab_top = 0;
+  c.stab_smem = 0;
   const bool smem = t.enc_in_smem != 0;
   switch (sym_dtype) {
     case RANS_SYM_INT32: return launch_encode_s<int32_t>(c, smem, st);
@@ -680,8 +705,6 @@ int launch_encode_float(const float *y, const float *means, const float *scales,
   c.fscale = scales;
   c.stab = scale_table;
   c.bound = scale_bound;
-  c.stab_top = 0;
-  while (2 * c.stab_top <= t.K - 1 && t.K > 1) c.stab_top = c.stab_top ? 2 * c.stab_top : 1;
   c.K = t.K;
   c.meta_bytes = t.meta_bytes;
   c.bucket_bytes = t.bucket_bytes;

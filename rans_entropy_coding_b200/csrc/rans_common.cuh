@@ -357,14 +357,24 @@ __device__ __forceinline__ void st_global(float *p, float v) { __stcs(p, v); }
 //
 // Row of a scale s: the first of the K table entries (increasing) that is
 // >= max(s, bound), a NaN scale counting as the bound; the last row when none
-// of the first K - 1 is.  A binary search with the same steps on every lane:
-// pos counts the entries below s among the first K - 1.
-__device__ __forceinline__ uint32_t scale_row(float s, const float *table, int K, int top) {
-  // top: the largest power of two <= K - 1 (0 when K == 1)
+// of the first K - 1 is.  An unrolled binary search with the same STEPS steps
+// on every lane (2^STEPS > K - 1): pos counts the entries below s among the
+// first K - 1.  The table is read with plain loads: the coders keep a copy in
+// shared memory when it fits.
+template <int STEPS>
+__device__ __forceinline__ uint32_t scale_row(float s, const float *table, int K) {
   int pos = 0;
-  for (int step = top; step > 0; step >>= 1)
-    if (pos + step <= K - 1 && __ldg(table + pos + step - 1) < s) pos += step;
+#pragma unroll
+  for (int i = STEPS - 1; i >= 0; --i) {
+    const int step = 1 << i;
+    if (pos + step <= K - 1 && table[pos + step - 1] < s) pos += step;
+  }
   return (uint32_t)pos;
+}
+// The search for any K <= 65536: 6 steps up to 65 entries (a uniform branch
+// on K), else 16.
+__device__ __forceinline__ uint32_t scale_row(float s, const float *table, int K) {
+  return K - 1 < 64 ? scale_row<6>(s, table, K) : scale_row<16>(s, table, K);
 }
 __device__ __forceinline__ float bound_scale(float s, float bound) {
   return s >= bound ? s : bound;  // NaN fails the compare: the bound

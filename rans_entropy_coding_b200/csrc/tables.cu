@@ -558,10 +558,10 @@ __global__ void __launch_bounds__(kSlotThreads)
 
 // Row index of every scale (scale_row in rans_common.cuh).
 __global__ void build_indexes_kernel(const float *scales, int64_t n, const float *table, int K,
-                                     int top, float bound, int32_t *indexes) {
+                                     float bound, int32_t *indexes) {
   for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n;
        i += (int64_t)gridDim.x * blockDim.x)
-    indexes[i] = (int32_t)scale_row(bound_scale(__ldg(scales + i), bound), table, K, top);
+    indexes[i] = (int32_t)scale_row(bound_scale(__ldg(scales + i), bound), table, K);
 }
 
 int ceil_log2(int64_t v) {
@@ -597,14 +597,12 @@ int launch_pmf_rows(const float *pmfs, int K, int stride, const int32_t *pmf_len
 int launch_build_indexes(const float *scales, int64_t n, const float *scale_table, int32_t K,
                          float scale_bound, int32_t *indexes, cudaStream_t st) {
   if (n <= 0) return RANS_OK;
-  int top = 0;
-  while (K > 1 && 2 * top <= K - 1) top = top ? 2 * top : 1;
   int dev = 0;
   cudaGetDevice(&dev);
   int64_t blocks = (n + 255) / 256;
   const int64_t cap = 16LL * num_sms(dev);
   if (blocks > cap) blocks = cap;
-  build_indexes_kernel<<<(unsigned)blocks, 256, 0, st>>>(scales, n, scale_table, K, top,
+  build_indexes_kernel<<<(unsigned)blocks, 256, 0, st>>>(scales, n, scale_table, K,
                                                          scale_bound, indexes);
   return cudaGetLastError() == cudaSuccess ? RANS_OK : RANS_ERR_CUDA;
 }
