@@ -55,6 +55,20 @@ def lib():
         i32, i64, f64 = ctypes.c_int32, ctypes.c_int64, ctypes.c_double
         L.orc_pmf_to_cdf.argtypes = [P, ctypes.c_int, P]
         L.orc_pmf_to_cdf.restype = ctypes.c_int
+        L.orc_pmf_to_cdf_prec.argtypes = [P, ctypes.c_int, ctypes.c_int, P]
+        L.orc_pmf_to_cdf_prec.restype = ctypes.c_int
+        L.orc_build_cdfs_from_scales_prec.argtypes = [P, ctypes.c_int, f64, ctypes.c_int, P,
+                                                      ctypes.c_int, P, P]
+        L.orc_build_cdfs_from_scales_prec.restype = ctypes.c_int
+        L.orc_build_cdfs_from_pmfs_prec.argtypes = [P, ctypes.c_int, ctypes.c_int, P, P,
+                                                    ctypes.c_int, P, ctypes.c_int, P]
+        L.orc_build_cdfs_from_pmfs_prec.restype = ctypes.c_int
+        L.orc_encode_stream16.argtypes = [P, P, i64, P, ctypes.c_int, ctypes.c_int, P, P,
+                                          ctypes.c_int, ctypes.c_int, P, i64]
+        L.orc_encode_stream16.restype = i64
+        L.orc_decode_stream16.argtypes = [P, i64, P, i64, P, ctypes.c_int, ctypes.c_int, P, P,
+                                          ctypes.c_int, ctypes.c_int, P]
+        L.orc_decode_stream16.restype = ctypes.c_int
         L.orc_gaussian_multiplier.argtypes = [f64]
         L.orc_gaussian_multiplier.restype = f64
         L.orc_gaussian_center.argtypes = [ctypes.c_float, f64, P]
@@ -86,11 +100,15 @@ def _ptr(a):
 
 
 # ------------------------------------------------------------------ tables --
-def pmf_to_cdf(pmf):
-    """pmf (tail mass last) -> quantised cdf row of len(pmf) + 1 entries."""
+def pmf_to_cdf(pmf, precision=16):
+    """pmf (tail mass last) -> quantised cdf row of len(pmf) + 1 entries,
+    summing to 2^precision."""
     p = np.ascontiguousarray(pmf, dtype=np.float32)
     out = np.zeros(p.size + 1, dtype=np.int32)
-    st = lib().orc_pmf_to_cdf(_ptr(p), p.size, _ptr(out))
+    if precision == 16:
+        st = lib().orc_pmf_to_cdf(_ptr(p), p.size, _ptr(out))
+    else:
+        st = lib().orc_pmf_to_cdf_prec(_ptr(p), p.size, precision, _ptr(out))
     if st:
         raise OracleError(st, "pmf_to_cdf")
     return out
@@ -108,8 +126,9 @@ def gaussian_center(scale, tail_mass=1e-9):
     return int(c[0])
 
 
-def build_cdfs_from_scales(scales, tail_mass=1e-9, Lmax=None):
-    """Gaussian rows -> (cdfs[K, Lmax] int32, lengths[K], offsets[K])."""
+def build_cdfs_from_scales(scales, tail_mass=1e-9, Lmax=None, precision=16):
+    """Gaussian rows -> (cdfs[K, Lmax] int32, lengths[K], offsets[K]); rows sum
+    to 2^precision."""
     s = np.ascontiguousarray(scales, dtype=np.float32)
     K = s.size
     if Lmax is None:
@@ -117,15 +136,15 @@ def build_cdfs_from_scales(scales, tail_mass=1e-9, Lmax=None):
     cdfs = np.zeros((K, Lmax), dtype=np.int32)
     lengths = np.zeros(K, dtype=np.int32)
     offsets = np.zeros(K, dtype=np.int32)
-    st = lib().orc_build_cdfs_from_scales(_ptr(s), K, tail_mass, _ptr(cdfs), Lmax,
-                                          _ptr(lengths), _ptr(offsets))
+    st = lib().orc_build_cdfs_from_scales_prec(_ptr(s), K, tail_mass, precision, _ptr(cdfs),
+                                               Lmax, _ptr(lengths), _ptr(offsets))
     if st:
         raise OracleError(st, "build_cdfs_from_scales")
     return cdfs, lengths, offsets
 
 
-def build_cdfs_from_pmfs(pmfs, pmf_lengths, tail_mass, Lmax=None):
-    """pmf rows -> (cdfs[K, Lmax] int32, lengths[K])."""
+def build_cdfs_from_pmfs(pmfs, pmf_lengths, tail_mass, Lmax=None, precision=16):
+    """pmf rows -> (cdfs[K, Lmax] int32, lengths[K]); rows sum to 2^precision."""
     p = np.ascontiguousarray(pmfs, dtype=np.float32)
     K, S = p.shape
     pl = np.ascontiguousarray(pmf_lengths, dtype=np.int32)
@@ -134,15 +153,21 @@ def build_cdfs_from_pmfs(pmfs, pmf_lengths, tail_mass, Lmax=None):
         Lmax = int(pl.max()) + 2
     cdfs = np.zeros((K, Lmax), dtype=np.int32)
     lengths = np.zeros(K, dtype=np.int32)
-    st = lib().orc_build_cdfs_from_pmfs(_ptr(p), K, S, _ptr(pl), _ptr(tm), _ptr(cdfs),
-                                        Lmax, _ptr(lengths))
+    st = lib().orc_build_cdfs_from_pmfs_prec(_ptr(p), K, S, _ptr(pl), _ptr(tm), precision,
+                                             _ptr(cdfs), Lmax, _ptr(lengths))
     if st:
         raise OracleError(st, "build_cdfs_from_pmfs")
     return cdfs, lengths
 
 
 # ----------------------------------------------------------------- streams --
-def encode_stream(symbols, rows, cdfs, lengths, offsets, W=1):
+# Coder formats ("torch_ans 0.3.0", Usage, variants table): "rans64" has a
+# 64-bit state, 32-bit words and rows summing to 2^16; "rans32_16" a 32-bit
+# state, 16-bit words and rows summing to 2^precision, precision <= 15.
+FORMATS = ("rans64", "rans32_16")
+
+
+def encode_stream(symbols, rows, cdfs, lengths, offsets, W=1, fmt="rans64", precision=None):
     """Codes one stream; returns its bytes as a uint8 array."""
     s = np.ascontiguousarray(symbols, dtype=np.int64)
     r = np.ascontiguousarray(rows, dtype=np.int32)
@@ -152,14 +177,21 @@ def encode_stream(symbols, rows, cdfs, lengths, offsets, W=1):
     K, Lmax = c.shape
     cap = 8 * W + 16 + 8 * s.size + 64
     out = np.zeros(cap, dtype=np.uint8)
-    n = lib().orc_encode_stream(_ptr(s), _ptr(r), s.size, _ptr(c), K, Lmax, _ptr(ln),
-                                _ptr(of), W, _ptr(out), cap)
+    if fmt == "rans64":
+        n = lib().orc_encode_stream(_ptr(s), _ptr(r), s.size, _ptr(c), K, Lmax, _ptr(ln),
+                                    _ptr(of), W, _ptr(out), cap)
+    elif fmt == "rans32_16":
+        n = lib().orc_encode_stream16(_ptr(s), _ptr(r), s.size, _ptr(c), K, Lmax, _ptr(ln),
+                                      _ptr(of), 15 if precision is None else precision, W,
+                                      _ptr(out), cap)
+    else:
+        raise ValueError("unknown format %r" % fmt)
     if n < 0:
         raise OracleError(int(n), "encode_stream")
     return out[:n].copy()
 
 
-def decode_stream(data, rows, cdfs, lengths, offsets, W=1):
+def decode_stream(data, rows, cdfs, lengths, offsets, W=1, fmt="rans64", precision=None):
     """Decodes len(rows) symbols of one stream; returns int64 symbols."""
     d = np.ascontiguousarray(data, dtype=np.uint8)
     r = np.ascontiguousarray(rows, dtype=np.int32)
@@ -168,8 +200,15 @@ def decode_stream(data, rows, cdfs, lengths, offsets, W=1):
     of = np.ascontiguousarray(offsets, dtype=np.int32)
     K, Lmax = c.shape
     out = np.zeros(r.size, dtype=np.int64)
-    st = lib().orc_decode_stream(_ptr(d), d.size, _ptr(r), r.size, _ptr(c), K, Lmax,
-                                 _ptr(ln), _ptr(of), W, _ptr(out))
+    if fmt == "rans64":
+        st = lib().orc_decode_stream(_ptr(d), d.size, _ptr(r), r.size, _ptr(c), K, Lmax,
+                                     _ptr(ln), _ptr(of), W, _ptr(out))
+    elif fmt == "rans32_16":
+        st = lib().orc_decode_stream16(_ptr(d), d.size, _ptr(r), r.size, _ptr(c), K, Lmax,
+                                       _ptr(ln), _ptr(of), 15 if precision is None else precision,
+                                       W, _ptr(out))
+    else:
+        raise ValueError("unknown format %r" % fmt)
     if st:
         raise OracleError(st, "decode_stream")
     return out
@@ -220,7 +259,7 @@ def _rows_for(positions, indexes, index_block):
 
 
 def encode_with_indexes(symbols, indexes, cdfs, lengths, offsets, chunking, W=1,
-                        index_block=1, streams=None):
+                        index_block=1, streams=None, fmt="rans64", precision=None):
     """Container encode: returns (bytes uint8[total], offsets uint64[S+1]).
 
     ``streams`` optionally restricts the work to a subset of stream ids; the
@@ -232,7 +271,7 @@ def encode_with_indexes(symbols, indexes, cdfs, lengths, offsets, chunking, W=1,
     for k in ids:
         p = pos[k]
         b = encode_stream(flat[p].astype(np.int64), _rows_for(p, indexes, index_block),
-                          cdfs, lengths, offsets, W)
+                          cdfs, lengths, offsets, W, fmt, precision)
         parts.append(b)
         offs.append(offs[-1] + b.size)
     data = np.concatenate(parts) if parts else np.zeros(0, dtype=np.uint8)
@@ -240,7 +279,7 @@ def encode_with_indexes(symbols, indexes, cdfs, lengths, offsets, chunking, W=1,
 
 
 def decode_with_indexes(data, stream_offsets, indexes, cdfs, lengths, offsets, chunking,
-                        n, W=1, index_block=1, dtype=np.int32):
+                        n, W=1, index_block=1, dtype=np.int32, fmt="rans64", precision=None):
     """Container decode of n elements; returns a flat array of ``dtype``."""
     pos = stream_positions(n, chunking)
     out = np.zeros(n, dtype=np.int64)
@@ -249,7 +288,7 @@ def decode_with_indexes(data, stream_offsets, indexes, cdfs, lengths, offsets, c
     for k, p in enumerate(pos):
         a, b = int(so[k]), int(so[k + 1])
         out[p] = decode_stream(d[a:b], _rows_for(p, indexes, index_block), cdfs, lengths,
-                               offsets, W)
+                               offsets, W, fmt, precision)
     return out.astype(dtype)
 
 

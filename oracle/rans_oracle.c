@@ -68,14 +68,24 @@
  */
 int orc_pmf_to_cdf(const float *pmf, int n, int32_t *cdf)
 {
-    if (n < 1) return ORC_ERR_ARG;
+    return orc_pmf_to_cdf_prec(pmf, n, (int)PREC, cdf);
+}
+
+/* The same at precision p (rows summing to 2^p): [TA] Usage, the variants
+ * table gives rans32_16 frequencies of at most 15 bits, and the FAQ bounds
+ * the cdf values by 2^freq_precision.  Reading: steps 1-4 above with 2^16
+ * replaced by 2^p. */
+int orc_pmf_to_cdf_prec(const float *pmf, int n, int prec, int32_t *cdf)
+{
+    if (n < 1 || prec < 1 || prec > 16) return ORC_ERR_ARG;
+    const uint32_t total = 1u << prec;
     uint64_t *c = (uint64_t *)calloc((size_t)n + 1, sizeof(uint64_t));
     if (!c) return ORC_ERR_ARG;
 
     /* steps 1 and 2 */
     c[0] = 0;
     for (int i = 0; i < n; ++i) {
-        float scaled = pmf[i] * (float)TOTAL;   /* exact: times a power of 2 */
+        float scaled = pmf[i] * (float)total;   /* exact: times a power of 2 */
         double r = round((double)scaled);       /* half away from zero */
         if (!(r >= 0.0) || r > 4294967295.0) { free(c); return ORC_ERR_ARG; }
         c[i + 1] = c[i] + (uint64_t)r;
@@ -85,7 +95,7 @@ int orc_pmf_to_cdf(const float *pmf, int n, int32_t *cdf)
 
     /* step 3 */
     for (int i = 0; i <= n; ++i)
-        c[i] = ((uint64_t)TOTAL * c[i]) / T;
+        c[i] = ((uint64_t)total * c[i]) / T;
 
     /* step 4 */
     for (int i = 0; i < n; ++i) {
@@ -155,6 +165,14 @@ int orc_build_cdfs_from_scales(const float *scales, int K, double tail_mass,
                                int32_t *cdfs, int Lmax, int32_t *lengths,
                                int32_t *offsets)
 {
+    return orc_build_cdfs_from_scales_prec(scales, K, tail_mass, (int)PREC, cdfs, Lmax,
+                                           lengths, offsets);
+}
+
+int orc_build_cdfs_from_scales_prec(const float *scales, int K, double tail_mass, int prec,
+                                    int32_t *cdfs, int Lmax, int32_t *lengths,
+                                    int32_t *offsets)
+{
     if (K <= 0 || Lmax < 3) return ORC_ERR_ARG;
     for (int r = 0; r < K; ++r) {
         int32_t center;
@@ -175,7 +193,7 @@ int orc_build_cdfs_from_scales(const float *scales, int K, double tail_mass,
         p[npmf] = (float)(2.0 * std_normal_cdf((-0.5 - (double)center) / s));
         int32_t *row = cdfs + (size_t)r * (size_t)Lmax;
         for (int j = 0; j < Lmax; ++j) row[j] = 0;
-        st = orc_pmf_to_cdf(p, npmf + 1, row);
+        st = orc_pmf_to_cdf_prec(p, npmf + 1, prec, row);
         free(p);
         if (st) return st;
         lengths[r] = len;
@@ -191,6 +209,14 @@ int orc_build_cdfs_from_pmfs(const float *pmfs, int K, int stride,
                              const int32_t *pmf_lengths, const float *tail_mass,
                              int32_t *cdfs, int Lmax, int32_t *lengths)
 {
+    return orc_build_cdfs_from_pmfs_prec(pmfs, K, stride, pmf_lengths, tail_mass, (int)PREC,
+                                         cdfs, Lmax, lengths);
+}
+
+int orc_build_cdfs_from_pmfs_prec(const float *pmfs, int K, int stride,
+                                  const int32_t *pmf_lengths, const float *tail_mass,
+                                  int prec, int32_t *cdfs, int Lmax, int32_t *lengths)
+{
     if (K <= 0 || stride <= 0) return ORC_ERR_ARG;
     for (int r = 0; r < K; ++r) {
         int n = pmf_lengths[r];
@@ -202,7 +228,7 @@ int orc_build_cdfs_from_pmfs(const float *pmfs, int K, int stride,
         p[n] = tail_mass[r];
         int32_t *row = cdfs + (size_t)r * (size_t)Lmax;
         for (int j = 0; j < Lmax; ++j) row[j] = 0;
-        int st = orc_pmf_to_cdf(p, n + 1, row);
+        int st = orc_pmf_to_cdf_prec(p, n + 1, prec, row);
         free(p);
         if (st) return st;
         lengths[r] = n + 2;
@@ -476,5 +502,186 @@ int orc_decode_stream(const uint8_t *in, int64_t len, const int32_t *row, int64_
     if (R.pos != R.len) return ORC_ERR_CORRUPT;
     for (int l = 0; l < W; ++l)
         if (x[l] != RANS_L) return ORC_ERR_CORRUPT;
+    return ORC_OK;
+}
+
+/* ------------------------------------------------------------ rans32_16 ----
+ * The 32-bit-state variant.  [TA] Usage, variants table: rans32_16 keeps a
+ * 32-bit state, emits 16-bit stream words and takes frequencies of at most 15
+ * bits (state bits > stream bits + frequency bits); its interleaved forms use
+ * 1, 2, 4, 8 or 32 states per stream, one shared stream of words ([TA] FAQ).
+ * Reading, by the same argument as O1: the lower bound is L16 = 2^16, the
+ * only value for which one 16-bit word brings a state below it back into
+ * [L16, 2^16 L16).  So, with rows summing to 2^p (1 <= p <= 15):
+ *   SYM(start, freq): if x >= 2^(32-p) freq, push the low 16 bits and shift x
+ *     right by 16; then x = (x / freq) 2^p + x mod freq + start;
+ *   BITS(v): if x >= 2^28, push a word likewise; then x = 16 x + v;
+ *   flush: lanes W-1 .. 0 push their state as two 16-bit words, high first;
+ *   the stream is the words in reverse push order, each little-endian, so it
+ *   starts with lane 0's low and high halves.  The symbol -> op mapping (O4)
+ *   and the lane of a symbol (index mod W) are those of the 64-bit coder.
+ * Decoding mirrors it: cum = x mod 2^p, the linear scan of [KB] section 4,
+ * x = freq (x >> p) + cum - start, and a state below 2^16 takes the next word
+ * as its low 16 bits.
+ */
+#define R16_L (1u << 16)
+
+typedef struct {
+    uint16_t *w;
+    size_t n, cap;
+} words16_t;
+
+static int push_word16(words16_t *W, uint16_t v)
+{
+    if (W->n == W->cap) {
+        size_t nc = W->cap ? 2 * W->cap : 1024;
+        uint16_t *p = (uint16_t *)realloc(W->w, nc * sizeof(uint16_t));
+        if (!p) return ORC_ERR_ARG;
+        W->w = p;
+        W->cap = nc;
+    }
+    W->w[W->n++] = v;
+    return ORC_OK;
+}
+
+static int valid_interleave16(int W)
+{
+    return W == 1 || W == 2 || W == 4 || W == 8 || W == 32;
+}
+
+int64_t orc_encode_stream16(const int64_t *sym, const int32_t *row, int64_t n,
+                            const int32_t *cdfs, int K, int Lmax,
+                            const int32_t *lengths, const int32_t *offsets,
+                            int prec, int W, uint8_t *out, int64_t cap)
+{
+    if (!valid_interleave16(W) || n < 0 || prec < 1 || prec > 15) return ORC_ERR_ARG;
+    oplist_t ops = {NULL, 0, 0};
+    words16_t words = {NULL, 0, 0};
+    int64_t result = ORC_OK;
+
+    for (int64_t i = 0; i < n; ++i) {
+        int st = symbol_ops(sym[i], row[i], K, cdfs, Lmax, lengths, offsets,
+                            (int)(i % W), &ops);
+        if (st) { result = st; goto done; }
+    }
+
+    uint32_t x[32];
+    for (int l = 0; l < W; ++l) x[l] = R16_L;
+
+    for (size_t k = ops.n; k-- > 0;) {
+        const op_t *o = &ops.ops[k];
+        uint32_t *s = &x[o->lane];
+        uint64_t xmax = o->freq ? ((uint64_t)o->freq << (32 - prec)) : ((uint64_t)1 << 28);
+        if ((uint64_t)*s >= xmax) {
+            if (push_word16(&words, (uint16_t)*s)) { result = ORC_ERR_ARG; goto done; }
+            *s >>= 16;
+        }
+        if (o->freq)
+            *s = ((*s / o->freq) << prec) + (*s % o->freq) + o->start;
+        else
+            *s = (*s << BYPASS_BITS) | o->val;
+    }
+    for (int l = W - 1; l >= 0; --l) {
+        if (push_word16(&words, (uint16_t)(x[l] >> 16)) ||
+            push_word16(&words, (uint16_t)x[l])) { result = ORC_ERR_ARG; goto done; }
+    }
+
+    int64_t nbytes = (int64_t)words.n * 2;
+    if (nbytes > cap) { result = ORC_ERR_CAPACITY; goto done; }
+    for (size_t k = 0; k < words.n; ++k) {
+        uint16_t v = words.w[words.n - 1 - k];
+        out[2 * k + 0] = (uint8_t)(v);
+        out[2 * k + 1] = (uint8_t)(v >> 8);
+    }
+    result = nbytes;
+done:
+    free(ops.ops);
+    free(words.w);
+    return result;
+}
+
+static int read_word16(reader_t *R, uint32_t *v)
+{
+    if (R->pos + 2 > R->len) return ORC_ERR_CORRUPT;
+    const uint8_t *b = R->p + R->pos;
+    *v = (uint32_t)b[0] | ((uint32_t)b[1] << 8);
+    R->pos += 2;
+    return ORC_OK;
+}
+
+static int refill16(uint32_t *x, reader_t *R)
+{
+    if (*x < R16_L) {
+        uint32_t w;
+        int st = read_word16(R, &w);
+        if (st) return st;
+        *x = (*x << 16) | w;
+    }
+    return ORC_OK;
+}
+
+static int get_bits16(uint32_t *x, reader_t *R, uint32_t *val)
+{
+    *val = *x & BYPASS_MAX;
+    *x >>= BYPASS_BITS;
+    return refill16(x, R);
+}
+
+int orc_decode_stream16(const uint8_t *in, int64_t len, const int32_t *row, int64_t n,
+                        const int32_t *cdfs, int K, int Lmax,
+                        const int32_t *lengths, const int32_t *offsets,
+                        int prec, int W, int64_t *sym_out)
+{
+    if (!valid_interleave16(W) || prec < 1 || prec > 15) return ORC_ERR_ARG;
+    reader_t R = {in, len, 0};
+    uint32_t x[32];
+    for (int l = 0; l < W; ++l) {
+        uint32_t lo, hi;
+        if (read_word16(&R, &lo) || read_word16(&R, &hi)) return ORC_ERR_CORRUPT;
+        x[l] = (hi << 16) | lo;
+    }
+    const uint32_t mask = (1u << prec) - 1u;
+    for (int64_t i = 0; i < n; ++i) {
+        int32_t r = row[i];
+        if (r < 0 || r >= K) return ORC_ERR_INDEX;
+        const int32_t *cdf = cdfs + (size_t)r * (size_t)Lmax;
+        int32_t Lr = lengths[r];
+        int32_t maxv = Lr - 2;
+        uint32_t *s = &x[i % W];
+
+        uint32_t cum = *s & mask;
+        int j = 1;
+        while (j < Lr && (uint32_t)cdf[j] <= cum) ++j;
+        if (j >= Lr) return ORC_ERR_CORRUPT;    /* a malformed row */
+        int32_t v = j - 1;
+        uint32_t start = (uint32_t)cdf[v];
+        uint32_t freq = (uint32_t)(cdf[v + 1] - cdf[v]);
+        *s = freq * (*s >> prec) + cum - start;
+        int st = refill16(s, &R);
+        if (st) return st;
+
+        int64_t value = v;
+        if (v == maxv) {
+            uint32_t val;
+            if ((st = get_bits16(s, &R, &val))) return st;
+            uint32_t nb = val;
+            while (val == BYPASS_MAX) {
+                if ((st = get_bits16(s, &R, &val))) return st;
+                nb += val;
+            }
+            if (nb > 15) return ORC_ERR_CORRUPT;   /* raw would exceed 60 bits */
+            uint64_t raw = 0;
+            for (uint32_t k = 0; k < nb; ++k) {
+                if ((st = get_bits16(s, &R, &val))) return st;
+                raw |= (uint64_t)val << (BYPASS_BITS * k);
+            }
+            int64_t half = (int64_t)(raw >> 1);
+            value = (raw & 1) ? (-half - 1) : ((int64_t)maxv + half);
+        }
+        sym_out[i] = value + (int64_t)offsets[r];
+    }
+    if (R.pos != R.len) return ORC_ERR_CORRUPT;
+    for (int l = 0; l < W; ++l)
+        if (x[l] != R16_L) return ORC_ERR_CORRUPT;
     return ORC_OK;
 }

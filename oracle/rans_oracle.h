@@ -26,6 +26,9 @@ extern "C" {
 /* pmf (n entries, the last one the tail mass) -> cdf row of n + 1 entries. */
 int orc_pmf_to_cdf(const float *pmf, int n, int32_t *cdf);
 
+/* The same at precision prec (1..16): the row sums to 2^prec. */
+int orc_pmf_to_cdf_prec(const float *pmf, int n, int prec, int32_t *cdf);
+
 /* -Phi^-1(tail_mass / 2) by bisection on erfc. */
 double orc_gaussian_multiplier(double tail_mass);
 int orc_gaussian_center(float scale, double tail_mass, int32_t *center);
@@ -35,11 +38,19 @@ int orc_build_cdfs_from_scales(const float *scales, int K, double tail_mass,
                                int32_t *cdfs, int Lmax, int32_t *lengths,
                                int32_t *offsets);
 
+int orc_build_cdfs_from_scales_prec(const float *scales, int K, double tail_mass, int prec,
+                                    int32_t *cdfs, int Lmax, int32_t *lengths,
+                                    int32_t *offsets);
+
 /* K rows from pmfs: row r is pmfs[r*stride .. r*stride + pmf_lengths[r]) plus
  * tail_mass[r]; cdf length pmf_lengths[r] + 2. */
 int orc_build_cdfs_from_pmfs(const float *pmfs, int K, int stride,
                              const int32_t *pmf_lengths, const float *tail_mass,
                              int32_t *cdfs, int Lmax, int32_t *lengths);
+
+int orc_build_cdfs_from_pmfs_prec(const float *pmfs, int K, int stride,
+                                  const int32_t *pmf_lengths, const float *tail_mass,
+                                  int prec, int32_t *cdfs, int Lmax, int32_t *lengths);
 
 /* One stream of n symbols (in stream order) with their row indexes; W = 1 or
  * 32 interleaved states.  Returns the byte length, or a negative status. */
@@ -53,6 +64,17 @@ int orc_decode_stream(const uint8_t *in, int64_t len, const int32_t *row, int64_
                       const int32_t *cdfs, int K, int Lmax,
                       const int32_t *lengths, const int32_t *offsets,
                       int W, int64_t *sym_out);
+
+/* The rans32_16 variant: 32-bit state, 16-bit words, rows summing to 2^prec
+ * (1 <= prec <= 15), W = 1, 2, 4, 8 or 32.  Byte lengths are even. */
+int64_t orc_encode_stream16(const int64_t *sym, const int32_t *row, int64_t n,
+                            const int32_t *cdfs, int K, int Lmax,
+                            const int32_t *lengths, const int32_t *offsets,
+                            int prec, int W, uint8_t *out, int64_t cap);
+int orc_decode_stream16(const uint8_t *in, int64_t len, const int32_t *row, int64_t n,
+                        const int32_t *cdfs, int K, int Lmax,
+                        const int32_t *lengths, const int32_t *offsets,
+                        int prec, int W, int64_t *sym_out);
 
 #ifdef __cplusplus
 }
