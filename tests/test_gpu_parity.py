@@ -425,8 +425,13 @@ def _float_case(W=32, with_means=True, n_images=1, **kw):
     return w, wi, (c, l, o)
 
 
-def test_build_indexes_matches_oracle():
-    t = WL.log_spaced_scales(WL.SCALE_MIN, WL.SCALE_MAX_Y, WL.N_ROWS_Y).astype(np.float32)
+@pytest.mark.parametrize("K", [1, 2, 64, 65, 66, 300])
+def test_build_indexes_matches_oracle(K):
+    """Tables of 1 to 300 entries (the 6-step search up to 65 entries, the
+    16-step one above), exact table values, values beside them, out of
+    range, NaN."""
+    t = WL.log_spaced_scales(WL.SCALE_MIN, WL.SCALE_MAX_Y, K).astype(np.float32) if K > 1 \
+        else np.float32([WL.SCALE_MIN])
     rng = np.random.Generator(np.random.PCG64(31))
     s = np.concatenate([np.exp(rng.uniform(np.log(1e-3), np.log(1e4), 100000)), t,
                         np.nextafter(t, np.float32(0)), np.nextafter(t, np.float32(np.inf)),
@@ -437,13 +442,15 @@ def test_build_indexes_matches_oracle():
     assert np.array_equal(got.cpu().numpy(), O.build_indexes(s, t, WL.SCALE_MIN))
 
 
-@pytest.mark.parametrize("W,with_means", [(32, True), (32, False), (1, True)])
-def test_encode_from_scales_matches_oracle(W, with_means):
+@pytest.mark.parametrize("W,with_means,n_rows", [(32, True, 64), (32, False, 64), (1, True, 64),
+                                                (32, True, 256)])
+def test_encode_from_scales_matches_oracle(W, with_means, n_rows):
     """Float latents in: the streams equal the oracle's encode of
     build_indexes(scales) and rint(y - mean); decoding gives back
     float32(symbol) + mean exactly."""
     kw = {} if W == 32 else dict(th=17, tw=30)
-    w, wi, (c, l, o) = _float_case(W=W, with_means=with_means, **kw)
+    # 256 rows: a 16-step table search, and tables read from global memory
+    w, wi, (c, l, o) = _float_case(W=W, with_means=with_means, n_rows=n_rows, **kw)
     want, woffs = oracle_encode(wi, c, l, o)
     dev = lambda a: None if a is None else torch.from_numpy(np.ascontiguousarray(a).reshape(-1)).cuda()
     tables = tables_from_numpy(c, l, o)

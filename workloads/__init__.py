@@ -134,11 +134,13 @@ def many_rows(seed=5000, n=1 << 18, n_rows=256, n_streams=64, W=32):
                 chunking=dict(kind="contig", n_streams=n_streams), W=W, index_block=1)
 
 
-def y_float(seed=6000, n_images=2, cg=4, th=64, tw=64, W=32, with_means=True):
+def y_float(seed=6000, n_images=2, cg=4, th=64, tw=64, W=32, with_means=True,
+            n_rows=N_ROWS_Y):
     """Float latents of a mean-scale model, [n_images, 192, 68, 120]: per
     element a scale exp(U(ln 0.11, ln 256)), a mean U(-8, 8) (or none) and
-    y = mean + N(0, scale), all float32; the 64-entry scale table and its
-    lower bound 0.11.  Rows and symbols come from the scales and y - mean."""
+    y = mean + N(0, scale), all float32; the n_rows-entry scale table (64 by
+    default) and its lower bound 0.11.  Rows and symbols come from the scales
+    and y - mean."""
     rng = _rng(seed)
     shape = (n_images,) + Y_SHAPE
     n = int(np.prod(shape))
@@ -149,7 +151,7 @@ def y_float(seed=6000, n_images=2, cg=4, th=64, tw=64, W=32, with_means=True):
         y = (y + means).astype(np.float32)
     return dict(name="y_float", y=y.reshape(shape), means=None if means is None else
                 means.reshape(shape), fscales=scales.reshape(shape),
-                scales=log_spaced_scales(SCALE_MIN, SCALE_MAX_Y, N_ROWS_Y), tail_mass=1e-9,
+                scales=log_spaced_scales(SCALE_MIN, SCALE_MAX_Y, n_rows), tail_mass=1e-9,
                 scale_bound=SCALE_MIN,
                 chunking=dict(kind="tiled", shape=shape, cg=cg, th=th, tw=tw), W=W,
                 index_block=1)
