@@ -60,9 +60,11 @@ def parse():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-clocks", action="store_true")
     ap.add_argument("--traffic-file", default=os.path.join(ROOT, "profiles", "dram_traffic.txt"))
-    ap.add_argument("--workload", choices=["batch", "tiny", "z", "y", "sweep", "float"],
+    ap.add_argument("--workload", choices=["batch", "tiny", "z", "y", "sweep", "float", "r16"],
                     default="batch")
     ap.add_argument("--interleave", type=int, default=None, help="W for --workload y")
+    ap.add_argument("--format", choices=["rans64", "rans32_16"], default=None,
+                    help="coder format (default: rans32_16 for --workload r16, else rans64)")
     return ap.parse_args()
 
 
@@ -194,6 +196,8 @@ def load_inputs(rank, group, images=N_IMAGES, workload="batch", interleave=None)
         w = WL.y_latent(W=interleave or 32)
     elif workload == "sweep":
         w = WL.sweep(log2_n=28)
+    elif workload == "r16":
+        w = WL.r16_rows()
     elif workload == "float":
         ids = shard_images(rank, images)
         w = WL.y_float(seed=6000 + ids[0], n_images=len(ids), cg=group)
@@ -206,7 +210,18 @@ def load_inputs(rank, group, images=N_IMAGES, workload="batch", interleave=None)
     return w
 
 
+def apply_format(w, fmt):
+    """Sets the coder format (and its row precision) on a workload dict."""
+    fmt = fmt or w.get("fmt", "rans64")
+    w["fmt"] = fmt
+    w["precision"] = 15 if fmt == "rans32_16" else 16
+    return w
+
+
 def workload_name(w, args):
+    if w.get("fmt", "rans64") != "rans64":
+        return "%s [%s, precision %d]" % (workload_name(dict(w, fmt="rans64"), args), w["fmt"],
+                                          w["precision"])
     if args.workload == "batch":
         return WORKLOAD
     if args.workload == "float":
@@ -227,10 +242,11 @@ def oracle_sample(w, max_streams, workers):
     workload, one stream per call, spread over `workers` threads (the C
     oracle runs without the GIL).  Returns (symbols coded, seconds)."""
     import oracle as O
+    fmt, prec = w.get("fmt", "rans64"), w.get("precision", 16)
     if "scales" in w:
-        c, l, o = O.build_cdfs_from_scales(w["scales"], w["tail_mass"])
+        c, l, o = O.build_cdfs_from_scales(w["scales"], w["tail_mass"], precision=prec)
     else:
-        c, l = O.build_cdfs_from_pmfs(w["pmfs"], w["pmf_lengths"], w["tail"])
+        c, l = O.build_cdfs_from_pmfs(w["pmfs"], w["pmf_lengths"], w["tail"], precision=prec)
         o = np.asarray(w["offsets"], dtype=np.int32)
     flat = np.asarray(w["symbols"]).reshape(-1)
     pos = O.stream_positions(flat.size, w["chunking"])[:max_streams]
@@ -241,8 +257,8 @@ def oracle_sample(w, max_streams, workers):
     def one(p):
         s = flat[p].astype(np.int64)
         r = idx[p // blk]
-        b = O.encode_stream(s, r, c, l, o, W=W)
-        back = O.decode_stream(b, r, c, l, o, W=W)
+        b = O.encode_stream(s, r, c, l, o, W=W, fmt=fmt, precision=prec)
+        back = O.decode_stream(b, r, c, l, o, W=W, fmt=fmt, precision=prec)
         assert np.array_equal(back, s)
         return p.size
 
@@ -256,7 +272,8 @@ def run_reference(args, world, rank):
     """--impl reference: the oracle as it stands on the host cores."""
     if rank != 0:
         return
-    w = load_inputs(0, args.group, workload=args.workload, interleave=args.interleave)
+    w = apply_format(load_inputs(0, args.group, workload=args.workload,
+                                 interleave=args.interleave), args.format)
     if args.workload == "float":  # the oracle codes rows and symbols computed first
         import oracle as O
         w = dict(w, symbols=O.quantize(w["y"], w["means"]), W=32,
@@ -277,7 +294,8 @@ def run_reference(args, world, rank):
     print(json.dumps({
         "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": 1,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * tot_t / args.steps,
-        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "u64",
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "u64" if w["fmt"] == "rans64" else "u32",
         "data": "synthetic", "config": {"workload": workload_name(w, args),
                                         "streams_per_step": max_streams},
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": workers, "kind": "oracle",
@@ -295,13 +313,15 @@ def run_ours(args, world, rank, local):
     rb.lib()
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
-    w = load_inputs(rank, args.group, args.images, args.workload, args.interleave)
+    w = apply_format(load_inputs(rank, args.group, args.images, args.workload, args.interleave),
+                     args.format)
+    fmt, prec = w["fmt"], w["precision"]
     sym_np = np.ascontiguousarray(np.asarray(w["symbols"]).reshape(-1))
     idx_np = np.ascontiguousarray(w["indexes"], dtype=np.int32)
     n = sym_np.size
     sym = torch.from_numpy(sym_np).to(dev)
     idx = torch.from_numpy(idx_np).to(dev)
-    ch = rb.Chunking.from_spec(w["chunking"], w["W"], w["index_block"], device=dev)
+    ch = rb.Chunking.from_spec(w["chunking"], w["W"], w["index_block"], device=dev, fmt=fmt)
     S = rb.rans_num_streams(ch, n)
 
     # tables: sized once; rebuilt inside every step (from the scale table, or
@@ -309,22 +329,23 @@ def run_ours(args, world, rank, local):
     if "scales" in w:
         scales = torch.from_numpy(w["scales"]).to(dev)
         tail = w["tail_mass"]
-        cdfs, lengths, offsets = rb.Tables.build_from_scales(scales, tail)
+        cdfs, lengths, offsets = rb.Tables.build_from_scales(scales, tail, precision=prec)
 
         def build_rows():
-            rb.check(rb.rans_build_cdfs_from_scales(scales, tail, cdfs, lengths, offsets),
-                     "cdfs")
+            rb.check(rb.rans_build_cdfs_from_scales(scales, tail, cdfs, lengths, offsets,
+                                                    precision=prec), "cdfs")
     else:
         pmfs = torch.from_numpy(np.ascontiguousarray(w["pmfs"])).to(dev)
         plen = torch.from_numpy(np.asarray(w["pmf_lengths"], np.int32)).to(dev)
         ptail = torch.from_numpy(np.asarray(w["tail"], np.float32)).to(dev)
-        cdfs, lengths = rb.Tables.build_from_pmfs(pmfs, plen, ptail)
+        cdfs, lengths = rb.Tables.build_from_pmfs(pmfs, plen, ptail, precision=prec)
         offsets = torch.from_numpy(np.asarray(w["offsets"], np.int32)).to(dev)
 
         def build_rows():
-            rb.check(rb.rans_build_cdfs_from_pmfs(pmfs, plen, ptail, cdfs, lengths), "cdfs")
+            rb.check(rb.rans_build_cdfs_from_pmfs(pmfs, plen, ptail, cdfs, lengths,
+                                                  precision=prec), "cdfs")
     K, Lmax = cdfs.shape
-    tables = rb.Tables(cdfs, lengths, offsets)
+    tables = rb.Tables(cdfs, lengths, offsets, precision=prec)
     blob = tables.blob
     ws = rb.Workspaces(ch, n, dev)
     dec = torch.empty_like(sym)
@@ -499,7 +520,7 @@ def run_ours(args, world, rank, local):
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         workers = os.cpu_count() or 1
-        ms = 768 if args.workload == "batch" else (64 if args.workload == "sweep" else S)
+        ms = {"batch": 768, "sweep": 64, "r16": 256}.get(args.workload, S)
         ns, ts = oracle_sample(w, ms, workers)
         cpu = {"value": ns / ts / 1e9, "unit": UNIT, "cores": workers, "kind": "oracle",
                "sample": "oracle encode+decode of the first %d streams (%d symbols), "
@@ -510,7 +531,8 @@ def run_ours(args, world, rank, local):
         line = {
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
-            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "u64",
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "u64" if fmt == "rans64" else "u32",
             "data": "synthetic",
             "config": {"workload": workload_name(w, args), "symbols_per_gpu": n,
                        "streams_per_gpu": S, "channel_group": args.group,

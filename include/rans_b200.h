@@ -78,6 +78,23 @@ enum { RANS_SYM_INT32 = 0, RANS_SYM_UINT8 = 1, RANS_SYM_INT16 = 2 };
 enum { RANS_CHUNK_CONTIG = 0, RANS_CHUNK_EXPLICIT = 1, RANS_CHUNK_TILED = 2 };
 
 /*
+ * Coder formats ("torch_ans 0.3.0", Usage, variants table):
+ *   RANS_FMT_RANS64:    64-bit state, 32-bit little-endian stream words, CDF
+ *                       rows summing to 2^16 (precision 16); lower state
+ *                       bound 2^31; each state flushed as 2 words.
+ *   RANS_FMT_RANS32_16: 32-bit state, 16-bit little-endian stream words, CDF
+ *                       rows summing to 2^p with 1 <= p <= 15; lower state
+ *                       bound 2^16 (the value for which one 16-bit word
+ *                       restores a state below it); each state flushed as 2
+ *                       words, so stream lengths are even.
+ * Both code the same symbol -> op mapping (escape bucket, zig-zag raw value,
+ * 4-bit bypass pieces); a bypass op renormalises at 2^59 / 2^28.  A table
+ * set's precision picks the formats it serves: 16 -> RANS64, <= 15 ->
+ * RANS32_16.
+ */
+enum { RANS_FMT_RANS64 = 0, RANS_FMT_RANS32_16 = 1 };
+
+/*
  * How the n symbols are cut into streams, and how indexes map to symbols.
  *   CONTIG:   n_streams streams; stream k covers elements
  *             [k*ceil(n/S), min((k+1)*ceil(n/S), n)) (trailing streams may be
@@ -94,6 +111,7 @@ enum { RANS_CHUNK_CONTIG = 0, RANS_CHUNK_EXPLICIT = 1, RANS_CHUNK_TILED = 2 };
  *   index_block: element p (flat position in the symbol array) uses row
  *             indexes[p / index_block]; 1 = one index per symbol; must be a
  *             power of two.
+ *   format:   RANS_FMT_* (0, the zero-initialised default, is RANS64).
  */
 typedef struct rans_chunking {
     int32_t kind;
@@ -103,6 +121,8 @@ typedef struct rans_chunking {
     int64_t shape[4];
     int64_t group, tile_h, tile_w;
     int64_t index_block;
+    int32_t format;
+    int32_t reserved;
 } rans_chunking;
 
 /*
@@ -124,6 +144,7 @@ typedef struct rans_tables {
     int32_t enc_in_smem;    /* 1: encode stages meta + buckets in shared memory */
     int32_t dec_in_smem;    /* 1: decode stages meta + starts + slots */
     int32_t device;         /* CUDA device the blob lives on */
+    int32_t precision;      /* the rows sum to 2^precision */
 } rans_tables;
 
 /* ------------------------------------------------------------ status ---- */
@@ -153,24 +174,26 @@ int rans_gaussian_lengths(const float *scales, int32_t K, double tail_mass,
 /*
  * K Gaussian CDF rows.  Row r's pmf is Phi((0.5-|k|)/s) - Phi((-0.5-|k|)/s)
  * for k = -c..c (Phi in double, cast to float), followed by the tail mass
- * 2 Phi((-0.5-c)/s); the pmf is quantised as in rans_build_cdfs_from_pmfs.
+ * 2 Phi((-0.5-c)/s); the pmf is quantised as in rans_build_cdfs_from_pmfs,
+ * to rows summing to 2^precision (1 <= precision <= 16).
  *   cdfs: device int32[K][Lmax] out; entries past a row's length are 0.
  *   cdf_lengths, offsets: device int32[K] out (as rans_gaussian_lengths);
  *   a row longer than Lmax, or one that cannot be quantised, gets a negative
  *   status as its length.  Asynchronous.
  */
 int rans_build_cdfs_from_scales(const float *scales, int32_t K, double tail_mass,
-                                int32_t *cdfs, int32_t Lmax, int32_t *cdf_lengths,
-                                int32_t *offsets, void *stream);
+                                int32_t precision, int32_t *cdfs, int32_t Lmax,
+                                int32_t *cdf_lengths, int32_t *offsets, void *stream);
 
 /*
  * K CDF rows from pmfs ("torch_ans 0.3.0", High-level API, init_params; FAQ:
  * rows are increasing positive integers up to 2^precision).  Row r takes
  * pmf_lengths[r] probabilities pmfs[r*pmf_stride ...] and then tail_mass[r];
- * each is scaled by 2^16 and rounded half away from zero, the running sum is
- * rescaled to floor(2^16 c / total), and every empty bucket then takes one
- * unit from the narrowest bucket wider than 1 (the first such on ties) --
- * scanning empty buckets in ascending order.
+ * with M = 2^precision (1 <= precision <= 16) each is scaled by M and
+ * rounded half away from zero, the running sum is rescaled to
+ * floor(M c / total), and every empty bucket then takes one unit from the
+ * narrowest bucket wider than 1 (the first such on ties) -- scanning empty
+ * buckets in ascending order.
  *   pmfs:        device float[K][pmf_stride].
  *   pmf_lengths: device int32[K], each in [0, pmf_stride].
  *   tail_mass:   device float[K].
@@ -182,8 +205,8 @@ int rans_build_cdfs_from_scales(const float *scales, int32_t K, double tail_mass
  */
 int rans_build_cdfs_from_pmfs(const float *pmfs, int32_t K, int32_t pmf_stride,
                               const int32_t *pmf_lengths, const float *tail_mass,
-                              int32_t *cdfs, int32_t Lmax, int32_t *cdf_lengths,
-                              void *stream);
+                              int32_t precision, int32_t *cdfs, int32_t Lmax,
+                              int32_t *cdf_lengths, void *stream);
 
 /* Upper bound on the blob size rans_tables_prepare needs for K rows of at
  * most Lmax entries. */
@@ -194,19 +217,21 @@ uint64_t rans_tables_bytes(int32_t K, int32_t Lmax);
  * blob_bytes >= rans_tables_bytes(K, Lmax)): per-row metadata, every bucket's
  * (start, width) packed in 32 bits, and a per-row lookup table mapping the
  * top bits of a decoder state's low 16 bits to its bucket.  Each row must
- * have 2 <= cdf_lengths[r] <= Lmax, cdf[0] = 0, cdf[len-1] = 65536 and
- * strictly increasing entries; otherwise RANS_ERR_TABLE (or the negative
- * length left by a builder).  Synchronous (reads back the K lengths and the
- * validation status); fills *out.
- *   cdfs: device int32[K][Lmax]; cdf_lengths, offsets: device int32[K].
+ * have 2 <= cdf_lengths[r] <= Lmax, cdf[0] = 0, cdf[len-1] = 2^precision
+ * and strictly increasing entries; otherwise RANS_ERR_TABLE (or the negative
+ * length left by a builder).  Rows of precision p < 16 are stored scaled to
+ * 16 bits (entries times 2^(16-p)).  Synchronous (reads back the K lengths
+ * and the validation status); fills *out.
+ *   cdfs: device int32[K][Lmax]; cdf_lengths, offsets: device int32[K];
+ *   precision: 16 (RANS64) or 1..15 (RANS32_16).
  */
 int rans_tables_prepare(const int32_t *cdfs, int32_t K, int32_t Lmax,
-                        const int32_t *cdf_lengths, const int32_t *offsets,
+                        const int32_t *cdf_lengths, const int32_t *offsets, int32_t precision,
                         void *blob, uint64_t blob_bytes, rans_tables *out, void *stream);
 
 /*
- * Rebuilds a prepared table set in place from new CDF rows whose lengths equal
- * the rows it was prepared from (for example a scale table rebuilt every
+ * Rebuilds a prepared table set in place from new CDF rows whose lengths (and
+ * precision) equal the rows it was prepared from (for example a scale table rebuilt every
  * call): offsets, packed buckets and lookup slots are rewritten on the device
  * with the layout kept, with no host synchronisation.  A row whose length
  * differs, or a malformed row, records RANS_ERR_TABLE in the blob's status
@@ -250,6 +275,8 @@ uint64_t rans_max_compressed_bytes(const rans_chunking *chunking, int64_t n);
  *   out:       device uint8[out_capacity].
  *   stream_offsets: device uint64[S + 1].
  *   workspace: device, >= rans_encode_workspace_bytes; 256-byte aligned.
+ *   chunking->format picks the coder (RANS_FMT_*); the tables' precision
+ *   must be 16 for RANS64 and at most 15 for RANS32_16 (else RANS_ERR_ARG).
  * Asynchronous; device errors via rans_get_status(workspace).
  */
 int rans_encode_with_indexes(const void *symbols, int32_t sym_dtype, const int32_t *indexes,
@@ -260,16 +287,20 @@ int rans_encode_with_indexes(const void *symbols, int32_t sym_dtype, const int32
 
 /*
  * decode_with_indexes ("torch_ans 0.3.0", Low-level API rans_pop; the decoded
- * symbol is the row's last bucket whose CDF entry is <= the state's low 16
- * bits, the rule of the linear scan in "Benchmark notes" section 4).
- *   in:             device uint8[in_bytes]: the packed streams.
+ * symbol is the row's last bucket whose CDF entry is <= the state's low
+ * `precision` bits, the rule of the linear scan in "Benchmark notes" section
+ * 4).
+ *   in:             device uint8[in_bytes]: the packed streams, aligned to
+ *                   the format's word (4 bytes, or 2 for RANS32_16).
  *   stream_offsets: device uint64[S + 1] from the encoder.
  *   indexes:        as for encode; must equal the encoder's.
  *   symbols_out:    device array of n elements of sym_dtype.
  *   workspace:      device, >= rans_decode_workspace_bytes; 256-byte aligned.
  * Every read is bounded by its stream's [offsets[k], offsets[k+1]); a stream
  * that does not end exactly where its words end with every lane back at the
- * initial state 2^31 is reported as RANS_ERR_CORRUPT.  Asynchronous.
+ * initial state (2^31, or 2^16 for RANS32_16) is reported as
+ * RANS_ERR_CORRUPT.  chunking->format and the tables' precision as for
+ * encode.  Asynchronous.
  */
 int rans_decode_with_indexes(const uint8_t *in, uint64_t in_bytes,
                              const uint64_t *stream_offsets, const int32_t *indexes,
@@ -331,7 +362,8 @@ int rans_build_indexes(const float *scales, int64_t n, const float *scale_table,
  *   y, scales:   device float[n]; means: device float[n] or NULL.
  *   scale_table: device float[table_len], table_len == tables->K: the scales
  *                the table rows were built from.
- *   chunking:    index_block must be 1 (one scale per element).
+ *   chunking:    index_block must be 1 (one scale per element); format
+ *                RANS64 (the float path codes the 64-bit format only).
  * Other arguments, outputs and errors as rans_encode_with_indexes.
  */
 int rans_encode_from_scales(const float *y, const float *means, const float *scales,

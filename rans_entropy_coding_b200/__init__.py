@@ -6,6 +6,7 @@ See include/rans_b200.h for the boundary.  Build the library with
 """
 from ._lib import (  # noqa: F401
     CHUNK_CONTIG, CHUNK_EXPLICIT, CHUNK_TILED, ERR_ARG, ERR_CAPACITY, ERR_CORRUPT, ERR_CUDA,
+    FMT_RANS32_16, FMT_RANS64,
     ERR_INDEX, ERR_RANGE, ERR_TABLE, ERR_TIMEOUT, ERR_ZERO_FREQ, LIB_PATH, OK, SIGNATURES,
     SYM_INT16, SYM_INT32, SYM_UINT8, Chunking, RansError, Tables, Workspaces, aligned_empty,
     check, decode_to_values, decode_with_indexes, encode_from_scales, encode_with_indexes, lib,

@@ -31,6 +31,10 @@ ERR_TIMEOUT = -9
 
 SYM_INT32, SYM_UINT8, SYM_INT16 = 0, 1, 2
 CHUNK_CONTIG, CHUNK_EXPLICIT, CHUNK_TILED = 0, 1, 2
+# coder formats: 64-bit state / 32-bit words / precision 16, and 32-bit
+# state / 16-bit words / precision <= 15
+FMT_RANS64, FMT_RANS32_16 = 0, 1
+_FMT_CODE = {"rans64": FMT_RANS64, "rans32_16": FMT_RANS32_16}
 
 _DTYPE_CODE = {torch.int32: SYM_INT32, torch.uint8: SYM_UINT8, torch.int16: SYM_INT16}
 
@@ -40,7 +44,8 @@ class rans_chunking(ctypes.Structure):
                 ("n_streams", ctypes.c_int64), ("stream_starts", ctypes.c_void_p),
                 ("shape", ctypes.c_int64 * 4), ("group", ctypes.c_int64),
                 ("tile_h", ctypes.c_int64), ("tile_w", ctypes.c_int64),
-                ("index_block", ctypes.c_int64)]
+                ("index_block", ctypes.c_int64), ("format", ctypes.c_int32),
+                ("reserved", ctypes.c_int32)]
 
 
 class rans_tables(ctypes.Structure):
@@ -50,7 +55,8 @@ class rans_tables(ctypes.Structure):
                 ("meta_bytes", ctypes.c_uint32), ("bucket_bytes", ctypes.c_uint32),
                 ("start_bytes", ctypes.c_uint32), ("slot_bytes", ctypes.c_uint32),
                 ("enc_in_smem", ctypes.c_int32),
-                ("dec_in_smem", ctypes.c_int32), ("device", ctypes.c_int32)]
+                ("dec_in_smem", ctypes.c_int32), ("device", ctypes.c_int32),
+                ("precision", ctypes.c_int32)]
 
 
 # (name, restype, argtypes) for every exported symbol of include/rans_b200.h
@@ -62,10 +68,11 @@ SIGNATURES = [
     ("rans_status_string", ctypes.c_char_p, [ctypes.c_int]),
     ("rans_version", ctypes.c_int, []),
     ("rans_gaussian_lengths", ctypes.c_int, [_P, _I32, _F64, _P, _P, _P]),
-    ("rans_build_cdfs_from_scales", ctypes.c_int, [_P, _I32, _F64, _P, _I32, _P, _P, _P]),
-    ("rans_build_cdfs_from_pmfs", ctypes.c_int, [_P, _I32, _I32, _P, _P, _P, _I32, _P, _P]),
+    ("rans_build_cdfs_from_scales", ctypes.c_int, [_P, _I32, _F64, _I32, _P, _I32, _P, _P, _P]),
+    ("rans_build_cdfs_from_pmfs", ctypes.c_int,
+     [_P, _I32, _I32, _P, _P, _I32, _P, _I32, _P, _P]),
     ("rans_tables_bytes", _U64, [_I32, _I32]),
-    ("rans_tables_prepare", ctypes.c_int, [_P, _I32, _I32, _P, _P, _P, _U64, _TBP, _P]),
+    ("rans_tables_prepare", ctypes.c_int, [_P, _I32, _I32, _P, _P, _I32, _P, _U64, _TBP, _P]),
     ("rans_tables_refresh", ctypes.c_int, [_P, _I32, _I32, _P, _P, _TBP, _P]),
     ("rans_num_streams", _I64, [_CHP, _I64]),
     ("rans_encode_workspace_bytes", _U64, [_CHP, _I64]),
@@ -140,29 +147,32 @@ def rans_gaussian_lengths(scales, tail_mass, cdf_lengths, offsets, stream=None):
                                        _ptr(cdf_lengths), _ptr(offsets), _stream(stream))
 
 
-def rans_build_cdfs_from_scales(scales, tail_mass, cdfs, cdf_lengths, offsets, stream=None):
+def rans_build_cdfs_from_scales(scales, tail_mass, cdfs, cdf_lengths, offsets, stream=None,
+                                precision=16):
     _need_cuda(scales, cdfs, cdf_lengths, offsets)
-    return lib().rans_build_cdfs_from_scales(_ptr(scales), scales.numel(), tail_mass, _ptr(cdfs),
-                                             cdfs.shape[1], _ptr(cdf_lengths), _ptr(offsets),
-                                             _stream(stream))
+    return lib().rans_build_cdfs_from_scales(_ptr(scales), scales.numel(), tail_mass, precision,
+                                             _ptr(cdfs), cdfs.shape[1], _ptr(cdf_lengths),
+                                             _ptr(offsets), _stream(stream))
 
 
-def rans_build_cdfs_from_pmfs(pmfs, pmf_lengths, tail_mass, cdfs, cdf_lengths, stream=None):
+def rans_build_cdfs_from_pmfs(pmfs, pmf_lengths, tail_mass, cdfs, cdf_lengths, stream=None,
+                              precision=16):
     _need_cuda(pmfs, pmf_lengths, tail_mass, cdfs, cdf_lengths)
     return lib().rans_build_cdfs_from_pmfs(_ptr(pmfs), pmfs.shape[0], pmfs.shape[1],
-                                           _ptr(pmf_lengths), _ptr(tail_mass), _ptr(cdfs),
-                                           cdfs.shape[1], _ptr(cdf_lengths), _stream(stream))
+                                           _ptr(pmf_lengths), _ptr(tail_mass), precision,
+                                           _ptr(cdfs), cdfs.shape[1], _ptr(cdf_lengths),
+                                           _stream(stream))
 
 
 def rans_tables_bytes(K, Lmax):
     return lib().rans_tables_bytes(K, Lmax)
 
 
-def rans_tables_prepare(cdfs, cdf_lengths, offsets, blob, out, stream=None):
+def rans_tables_prepare(cdfs, cdf_lengths, offsets, blob, out, stream=None, precision=16):
     _need_cuda(cdfs, cdf_lengths, offsets, blob)
     return lib().rans_tables_prepare(_ptr(cdfs), cdfs.shape[0], cdfs.shape[1], _ptr(cdf_lengths),
-                                     _ptr(offsets), _ptr(blob), blob.numel(), ctypes.byref(out),
-                                     _stream(stream))
+                                     _ptr(offsets), precision, _ptr(blob), blob.numel(),
+                                     ctypes.byref(out), _stream(stream))
 
 
 def rans_tables_refresh(cdfs, cdf_lengths, offsets, tables, stream=None):
@@ -262,14 +272,15 @@ class Chunking:
         return self.c.interleave
 
     @staticmethod
-    def contig(n_streams, interleave=1, index_block=1):
+    def contig(n_streams, interleave=1, index_block=1, fmt="rans64"):
         c = rans_chunking()
         c.kind, c.interleave, c.n_streams, c.index_block = (CHUNK_CONTIG, interleave, n_streams,
                                                             index_block)
+        c.format = _FMT_CODE[fmt]
         return Chunking(c)
 
     @staticmethod
-    def explicit(starts, interleave=1, index_block=1):
+    def explicit(starts, interleave=1, index_block=1, fmt="rans64"):
         """starts: CUDA int64 tensor of S + 1 element offsets."""
         _need_cuda(starts)
         assert starts.dtype == torch.int64
@@ -277,50 +288,55 @@ class Chunking:
         c.kind, c.interleave, c.n_streams, c.index_block = (CHUNK_EXPLICIT, interleave,
                                                             starts.numel() - 1, index_block)
         c.stream_starts = starts.data_ptr()
+        c.format = _FMT_CODE[fmt]
         return Chunking(c, keep=starts)
 
     @staticmethod
-    def tiled(shape, group, tile_h, tile_w, interleave=32, index_block=1):
+    def tiled(shape, group, tile_h, tile_w, interleave=32, index_block=1, fmt="rans64"):
         c = rans_chunking()
         c.kind, c.interleave, c.index_block = CHUNK_TILED, interleave, index_block
         for i, v in enumerate(shape):
             c.shape[i] = int(v)
         c.group, c.tile_h, c.tile_w = group, tile_h, tile_w
+        c.format = _FMT_CODE[fmt]
         return Chunking(c)
 
     @staticmethod
-    def from_spec(spec, interleave, index_block=1, device="cuda"):
+    def from_spec(spec, interleave, index_block=1, device="cuda", fmt="rans64"):
         """From the dict form used by the workloads module."""
         k = spec["kind"]
         if k == "contig":
-            return Chunking.contig(spec["n_streams"], interleave, index_block)
+            return Chunking.contig(spec["n_streams"], interleave, index_block, fmt)
         if k == "tiled":
             return Chunking.tiled(spec["shape"], spec["cg"], spec["th"], spec["tw"], interleave,
-                                  index_block)
+                                  index_block, fmt)
         if k == "explicit":
             st = torch.as_tensor(spec["starts"], dtype=torch.int64, device=device)
-            return Chunking.explicit(st, interleave, index_block)
+            return Chunking.explicit(st, interleave, index_block, fmt)
         raise ValueError(k)
 
 
 class Tables:
     """CDF rows (cdfs, cdf_lengths, offsets) plus the prepared table blob."""
 
-    def __init__(self, cdfs, cdf_lengths, offsets, stream=None, blob_bytes=None):
+    def __init__(self, cdfs, cdf_lengths, offsets, stream=None, blob_bytes=None, precision=16):
         """blob_bytes: the blob's size (default rans_tables_bytes(K, Lmax)); a
-        smaller blob leaves the decoder fewer bitmap words."""
+        smaller blob leaves the decoder fewer bitmap words.  precision: the
+        rows sum to 2^precision (16 for the rans64 format, <= 15 for
+        rans32_16)."""
         self.cdfs, self.cdf_lengths, self.offsets = cdfs, cdf_lengths, offsets
+        self.precision = precision
         K, Lmax = cdfs.shape
         nbytes = rans_tables_bytes(K, Lmax) if blob_bytes is None else int(blob_bytes)
         self.blob = torch.empty(nbytes + 256, dtype=torch.uint8, device=cdfs.device)
         off = (-self.blob.data_ptr()) % 256
         self.blob = self.blob[off:off + nbytes]
         self.c = rans_tables()
-        check(rans_tables_prepare(cdfs, cdf_lengths, offsets, self.blob, self.c, stream),
-              "tables_prepare")
+        check(rans_tables_prepare(cdfs, cdf_lengths, offsets, self.blob, self.c, stream,
+                                  precision), "tables_prepare")
 
     @staticmethod
-    def build_from_scales(scales, tail_mass=1e-9, stream=None):
+    def build_from_scales(scales, tail_mass=1e-9, stream=None, precision=16):
         """Gaussian rows for a float32 CUDA scale table; returns
         (cdfs, cdf_lengths, offsets)."""
         K = scales.numel()
@@ -333,28 +349,29 @@ class Tables:
             raise RansError(lmin, "gaussian_lengths")
         Lmax = int(lengths.max().item())
         cdfs = torch.empty((K, Lmax), dtype=torch.int32, device=dev)
-        check(rans_build_cdfs_from_scales(scales, tail_mass, cdfs, lengths, offsets, stream),
-              "build_cdfs_from_scales")
+        check(rans_build_cdfs_from_scales(scales, tail_mass, cdfs, lengths, offsets, stream,
+                                          precision), "build_cdfs_from_scales")
         return cdfs, lengths, offsets
 
     @staticmethod
-    def build_from_pmfs(pmfs, pmf_lengths, tail_mass, stream=None):
+    def build_from_pmfs(pmfs, pmf_lengths, tail_mass, stream=None, precision=16):
         K = pmfs.shape[0]
         Lmax = int(pmf_lengths.max().item()) + 2
         cdfs = torch.empty((K, Lmax), dtype=torch.int32, device=pmfs.device)
         lengths = torch.empty(K, dtype=torch.int32, device=pmfs.device)
-        check(rans_build_cdfs_from_pmfs(pmfs, pmf_lengths, tail_mass, cdfs, lengths, stream),
-              "build_cdfs_from_pmfs")
+        check(rans_build_cdfs_from_pmfs(pmfs, pmf_lengths, tail_mass, cdfs, lengths, stream,
+                                        precision), "build_cdfs_from_pmfs")
         return cdfs, lengths
 
     @staticmethod
-    def from_scales(scales, tail_mass=1e-9, stream=None):
-        return Tables(*Tables.build_from_scales(scales, tail_mass, stream), stream=stream)
+    def from_scales(scales, tail_mass=1e-9, stream=None, precision=16):
+        return Tables(*Tables.build_from_scales(scales, tail_mass, stream, precision),
+                      stream=stream, precision=precision)
 
     @staticmethod
-    def from_pmfs(pmfs, pmf_lengths, tail_mass, offsets, stream=None):
-        cdfs, lengths = Tables.build_from_pmfs(pmfs, pmf_lengths, tail_mass, stream)
-        return Tables(cdfs, lengths, offsets, stream=stream)
+    def from_pmfs(pmfs, pmf_lengths, tail_mass, offsets, stream=None, precision=16):
+        cdfs, lengths = Tables.build_from_pmfs(pmfs, pmf_lengths, tail_mass, stream, precision)
+        return Tables(cdfs, lengths, offsets, stream=stream, precision=precision)
 
 
 def aligned_empty(nbytes, device="cuda"):

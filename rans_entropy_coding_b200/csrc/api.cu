@@ -45,8 +45,10 @@ int make_geom(const rans_chunking *ch, int64_t n, Geom &g) {
   if (ch == nullptr || n < 0) return RANS_ERR_ARG;
   if (ch->interleave != 1 && ch->interleave != 32) return RANS_ERR_ARG;
   if (!is_pow2(ch->index_block)) return RANS_ERR_ARG;
+  if (ch->format != RANS_FMT_RANS64 && ch->format != RANS_FMT_RANS32_16) return RANS_ERR_ARG;
   std::memset(&g, 0, sizeof(g));
   g.kind = ch->kind;
+  g.fmt = ch->format;
   g.W = ch->interleave;
   g.n = n;
   int ib = 0;
@@ -141,10 +143,19 @@ uint64_t enc_ws_bytes(const Geom &g) { return kWsHeader + lens_bytes(g) + scratc
 
 bool tables_usable(const rans_tables *t) {
   if (t == nullptr || t->blob == nullptr || t->K < 1) return false;
+  if (t->precision < 1 || t->precision > 16) return false;
   int dev = -1;
   if (cudaGetDevice(&dev) != cudaSuccess || dev != t->device) return false;
   return true;
 }
+
+// RANS64 codes rows of precision 16, RANS32_16 rows of precision <= 15.
+bool format_fits(const Geom &g, const rans_tables *t) {
+  return g.fmt == RANS_FMT_RANS64 ? t->precision == 16 : t->precision <= 15;
+}
+
+// Bytes of the format's stream word.
+uint64_t word_bytes(const Geom &g) { return g.fmt == RANS_FMT_RANS32_16 ? 2 : 4; }
 
 cudaStream_t as_stream(void *s) { return static_cast<cudaStream_t>(s); }
 
@@ -177,23 +188,25 @@ RANS_API int rans_gaussian_lengths(const float *scales, int32_t K, double tail_m
 }
 
 RANS_API int rans_build_cdfs_from_scales(const float *scales, int32_t K, double tail_mass,
-                                         int32_t *cdfs, int32_t Lmax, int32_t *cdf_lengths,
-                                         int32_t *offsets, void *stream) {
+                                         int32_t precision, int32_t *cdfs, int32_t Lmax,
+                                         int32_t *cdf_lengths, int32_t *offsets, void *stream) {
   if (K < 1 || Lmax < 3 || !scales || !cdfs || !cdf_lengths || !offsets) return RANS_ERR_ARG;
   if (!(tail_mass > 0.0) || !(tail_mass < 1.0)) return RANS_ERR_ARG;
-  return rb::launch_gaussian_rows(scales, K, tail_mass, cdfs, Lmax, cdf_lengths, offsets,
-                                  as_stream(stream));
+  if (precision < 1 || precision > 16) return RANS_ERR_ARG;
+  return rb::launch_gaussian_rows(scales, K, tail_mass, precision, cdfs, Lmax, cdf_lengths,
+                                  offsets, as_stream(stream));
 }
 
 RANS_API int rans_build_cdfs_from_pmfs(const float *pmfs, int32_t K, int32_t pmf_stride,
                                        const int32_t *pmf_lengths, const float *tail_mass,
-                                       int32_t *cdfs, int32_t Lmax, int32_t *cdf_lengths,
-                                       void *stream) {
+                                       int32_t precision, int32_t *cdfs, int32_t Lmax,
+                                       int32_t *cdf_lengths, void *stream) {
   if (K < 1 || pmf_stride < 1 || Lmax < 2 || !pmfs || !pmf_lengths || !tail_mass || !cdfs ||
       !cdf_lengths)
     return RANS_ERR_ARG;
-  return rb::launch_pmf_rows(pmfs, K, pmf_stride, pmf_lengths, tail_mass, cdfs, Lmax,
-                             cdf_lengths, as_stream(stream));
+  if (precision < 1 || precision > 16) return RANS_ERR_ARG;
+  return rb::launch_pmf_rows(pmfs, K, pmf_stride, pmf_lengths, tail_mass, precision, cdfs,
+                             Lmax, cdf_lengths, as_stream(stream));
 }
 
 RANS_API uint64_t rans_tables_bytes(int32_t K, int32_t Lmax) {
@@ -201,12 +214,14 @@ RANS_API uint64_t rans_tables_bytes(int32_t K, int32_t Lmax) {
 }
 
 RANS_API int rans_tables_prepare(const int32_t *cdfs, int32_t K, int32_t Lmax,
-                                 const int32_t *cdf_lengths, const int32_t *offsets, void *blob,
-                                 uint64_t blob_bytes, rans_tables *out, void *stream) {
+                                 const int32_t *cdf_lengths, const int32_t *offsets,
+                                 int32_t precision, void *blob, uint64_t blob_bytes,
+                                 rans_tables *out, void *stream) {
   if (K < 1 || Lmax < 2 || Lmax > 65537 || !cdfs || !cdf_lengths || !offsets || !blob || !out)
     return RANS_ERR_ARG;
-  return rb::prepare_tables(cdfs, K, Lmax, cdf_lengths, offsets, blob, blob_bytes, out,
-                            as_stream(stream));
+  if (precision < 1 || precision > 16) return RANS_ERR_ARG;
+  return rb::prepare_tables(cdfs, K, Lmax, cdf_lengths, offsets, precision, blob, blob_bytes,
+                            out, as_stream(stream));
 }
 
 RANS_API int rans_tables_refresh(const int32_t *cdfs, int32_t K, int32_t Lmax,
@@ -256,6 +271,7 @@ RANS_API int rans_encode_with_indexes(const void *symbols, int32_t sym_dtype,
   Geom g;
   int st = make_geom(chunking, n, g);
   if (st) return st;
+  if (!format_fits(g, tables)) return RANS_ERR_ARG;
   if (workspace_bytes < enc_ws_bytes(g)) return RANS_ERR_CAPACITY;
   cudaStream_t s = as_stream(stream);
   char *ws = reinterpret_cast<char *>(workspace);
@@ -283,10 +299,11 @@ RANS_API int rans_decode_with_indexes(const uint8_t *in, uint64_t in_bytes,
   if (sym_dtype != RANS_SYM_INT32 && sym_dtype != RANS_SYM_UINT8 && sym_dtype != RANS_SYM_INT16)
     return RANS_ERR_ARG;
   if ((reinterpret_cast<uintptr_t>(workspace) & 255) != 0) return RANS_ERR_ARG;
-  if ((reinterpret_cast<uintptr_t>(in) & 3) != 0) return RANS_ERR_ARG;
   Geom g;
   int st = make_geom(chunking, n, g);
   if (st) return st;
+  if (!format_fits(g, tables)) return RANS_ERR_ARG;
+  if ((reinterpret_cast<uintptr_t>(in) & (word_bytes(g) - 1)) != 0) return RANS_ERR_ARG;
   if (workspace_bytes < kWsHeader) return RANS_ERR_CAPACITY;
   cudaStream_t s = as_stream(stream);
   int32_t *status = reinterpret_cast<int32_t *>(workspace);
@@ -311,6 +328,7 @@ static int float_args(const rans_tables *tables, const rans_chunking *chunking,
                       int32_t table_len) {
   if (!tables_usable(tables) || !chunking) return RANS_ERR_ARG;
   if (table_len != tables->K || chunking->index_block != 1) return RANS_ERR_ARG;
+  if (chunking->format != RANS_FMT_RANS64 || tables->precision != 16) return RANS_ERR_ARG;
   return RANS_OK;
 }
 

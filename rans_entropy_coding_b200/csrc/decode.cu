@@ -10,7 +10,11 @@
 //    searches;
 //  * state update x = freq (x >> 16) + cum - start and a refill of one
 //    32-bit word when x < 2^31 (64-bit state / 32-bit words / 16-bit
-//    precision: "torch_ans 0.3.0", Usage, rans64 row);
+//    precision: "torch_ans 0.3.0", Usage, rans64 row); for the rans32_16
+//    format (same table, rans32_16 row) cum = x mod 2^p,
+//    x = freq (x >> p) + cum - start and a refill of one 16-bit word when
+//    x < 2^16 (the F template parameter: Rans64 / Rans32 in rans_common.cuh;
+//    the tables hold 16-bit-scaled entries, so the lookup takes cum << sh);
 //  * W = 32: one warp per stream, lane = symbol index mod 32; refills take
 //    the next words of the shared stream in lane order (ballot + popc),
 //    served from a two-window register buffer of 64 prefetched words
@@ -44,6 +48,7 @@ struct DecCtx {
   const uint64_t *offs;
   const int32_t *idx;
   int32_t K;
+  uint32_t sh;  // 16 - precision of the rows (Rans32; 0 for Rans64)
   uint32_t meta_bytes, bucket_bytes, start_bytes, slot_bytes;
   const char *blob;
   Geom g;
@@ -56,13 +61,17 @@ struct DecCtx {
   int32_t stab_smem;  // 1: the kernel copies the scale table into shared memory
 };
 
+// A stream's words: its byte range must be word-aligned and hold at least
+// the W flushed states (two words each).
+template <class F>
 __device__ __forceinline__ bool stream_bounds(const DecCtx &c, int64_t s, int W,
-                                              const uint32_t *&words, uint64_t &nw) {
+                                              const typename F::Word *&words, uint64_t &nw) {
+  constexpr uint64_t kWB = sizeof(typename F::Word);
   const uint64_t b0 = c.offs[s], b1 = c.offs[s + 1];
-  if (b1 < b0 || b1 > c.in_bytes || ((b0 | b1) & 3ull) != 0 || (b1 - b0) < 8ull * W)
+  if (b1 < b0 || b1 > c.in_bytes || ((b0 | b1) & (kWB - 1)) != 0 || (b1 - b0) < 2 * kWB * W)
     return false;
-  words = reinterpret_cast<const uint32_t *>(c.in + b0);
-  nw = (b1 - b0) >> 2;
+  words = reinterpret_cast<const typename F::Word *>(c.in + b0);
+  nw = (b1 - b0) / kWB;
   return true;
 }
 
@@ -104,8 +113,9 @@ __device__ __forceinline__ uint32_t lookup(uint32_t cum, const RowMeta &m, const
   return min(sym, m.maxv);
 }
 
+template <class F>
 struct EscapeResult {
-  uint64_t x;
+  typename F::State x;
   int64_t val;
   uint64_t cur;
   bool bad;
@@ -114,13 +124,15 @@ struct EscapeResult {
 // The lane-serial part of a group holding an escape (after every lane's
 // symbol op): lanes take their words in ascending lane order; an escaping lane
 // reads its refill, count pieces and bypass pieces from the shared stream.
-__device__ __forceinline__ EscapeResult escape_group(uint64_t x, bool active, bool esc,
-                                                  uint32_t maxv, uint64_t abs0,
-                                                  const uint32_t *words, uint64_t nw) {
+template <class F>
+__device__ __forceinline__ EscapeResult<F> escape_group(typename F::State x, bool active,
+                                                     bool esc, uint32_t maxv, uint64_t abs0,
+                                                     const typename F::Word *words,
+                                                     uint64_t nw) {
   const int lane = threadIdx.x & 31;
   bool bad = false;
   int64_t val = 0;
-  const bool need_sym = active && x < kL;
+  const bool need_sym = active && x < F::kLow;
   uint32_t cons = need_sym ? 1u : 0u;
   uint32_t rem = __ballot_sync(kFull, esc);
   while (rem) {
@@ -141,11 +153,11 @@ __device__ __forceinline__ EscapeResult escape_group(uint64_t x, bool active, bo
         ++pp;
         return v;
       };
-      if (x < kL) x = (x << 32) | rd();
+      if (x < F::kLow) x = (x << F::kWordBits) | rd();
       auto getbits = [&]() -> uint32_t {
         const uint32_t v = (uint32_t)x & kBypassMax;
         x >>= kBypassBits;
-        if (x < kL) x = (x << 32) | rd();
+        if (x < F::kLow) x = (x << F::kWordBits) | rd();
         return v;
       };
       uint32_t v4 = getbits();
@@ -175,9 +187,9 @@ __device__ __forceinline__ EscapeResult escape_group(uint64_t x, bool active, bo
     const uint64_t pp = abs0 + (inc - cons);
     uint32_t v = 0;
     if (pp < nw) v = __ldg(words + pp); else bad = true;
-    x = (x << 32) | v;
+    x = (x << F::kWordBits) | v;
   }
-  EscapeResult r;
+  EscapeResult<F> r;
   r.x = x;
   r.val = val;
   r.cur = abs0 + __shfl_sync(kFull, inc, 31);
@@ -186,8 +198,9 @@ __device__ __forceinline__ EscapeResult escape_group(uint64_t x, bool active, bo
 }
 
 // Per-warp decoder state for one stream.
+template <class F>
 struct WarpDec {
-  uint64_t x;            // this lane's state
+  typename F::State x;   // this lane's state
   uint64_t cur;          // absolute word index of the register window
   uint32_t off;          // words of the window already consumed (< 32)
   uint32_t w0, w1, w2;   // window words cur + lane, + 32, + 64 (w2: lookahead)
@@ -198,11 +211,14 @@ struct WarpDec {
 // Window word i, read from a clamped address (nw >= 64 always): reading past
 // the stream end returns its last word instead, so no select waits on the
 // load; a decoder that consumes past the end is caught by the final check.
-__device__ __forceinline__ uint32_t word_at(const uint32_t *words, uint64_t nw, uint64_t i) {
+template <typename Word>
+__device__ __forceinline__ uint32_t word_at(const Word *words, uint64_t nw, uint64_t i) {
   return __ldg(words + (i < nw ? i : nw - 1));
 }
 
-__device__ __forceinline__ void load_window(WarpDec &st, const uint32_t *words, uint64_t nw) {
+template <class F>
+__device__ __forceinline__ void load_window(WarpDec<F> &st, const typename F::Word *words,
+                                            uint64_t nw) {
   const int lane = threadIdx.x & 31;
   st.w0 = word_at(words, nw, st.cur + lane);
   st.w1 = word_at(words, nw, st.cur + 32 + lane);
@@ -213,20 +229,21 @@ __device__ __forceinline__ void load_window(WarpDec &st, const uint32_t *words, 
 // group's row metadata, read one group ahead.  The refill is taken as if no
 // lane escaped; the escape ballot, issued beside it, sends the group down
 // the lane-serial path from the state after the symbol op.
-template <typename SymT, bool FULL, bool SEARCH>
-__device__ __forceinline__ void dec_group(WarpDec &st, const RowMeta &m, const uint16_t *starts,
-                                          const uint32_t *slots, bool active, SymT *dst,
-                                          const uint32_t *words, uint64_t nw, float mean = 0.0f) {
+template <class F, typename SymT, bool FULL, bool SEARCH>
+__device__ __forceinline__ void dec_group(WarpDec<F> &st, const RowMeta &m,
+                                          const uint16_t *starts, const uint32_t *slots,
+                                          bool active, SymT *dst, const typename F::Word *words,
+                                          uint64_t nw, uint32_t sh, float mean = 0.0f) {
   const int lane = threadIdx.x & 31;
   if (FULL) active = true;
-  const uint32_t cum = (uint32_t)st.x & (kTotal - 1);
+  const uint32_t cum = F::cum16(st.x, sh);
   const uint32_t sym = lookup<SEARCH, true>(cum, m, starts, slots, active);
   const uint32_t start = starts[m.bucket_base + sym];
   const uint32_t freq = width_of(start, starts[m.bucket_base + sym + 1]);
-  uint64_t x = (uint64_t)freq * (st.x >> kPrec) + (cum - start);
+  typename F::State x = F::dec_step(st.x, cum, start, freq, sh);
   if (!FULL) x = active ? x : st.x;
   const bool esc = active && sym == m.maxv;
-  const bool need = active && x < kL;
+  const bool need = active && x < F::kLow;
   const uint32_t nm = __ballot_sync(kFull, need);
   const bool any_esc = __any_sync(kFull, esc);
   const uint32_t j = st.off + __popc(nm & lanemask_lt());
@@ -234,7 +251,7 @@ __device__ __forceinline__ void dec_group(WarpDec &st, const RowMeta &m, const u
   const uint32_t wv = __shfl_sync(kFull, (uint32_t)lane >= st.off ? st.w0 : st.w1, j & 31);
   int32_t val = (int32_t)sym + m.offset;
   if (!any_esc) {
-    st.x = need ? ((x << 32) | wv) : x;
+    st.x = need ? ((x << F::kWordBits) | wv) : x;
     st.off += __popc(nm);
     if (st.off >= 32) {
       st.w0 = st.w1;
@@ -244,7 +261,8 @@ __device__ __forceinline__ void dec_group(WarpDec &st, const RowMeta &m, const u
       st.w2 = word_at(words, nw, st.cur + 64 + lane);
     }
   } else {
-    const EscapeResult er = escape_group(x, active, esc, m.maxv, st.cur + st.off, words, nw);
+    const EscapeResult<F> er =
+        escape_group<F>(x, active, esc, m.maxv, st.cur + st.off, words, nw);
     st.x = er.x;
     if (esc) val = (int32_t)(er.val + (int64_t)m.offset);
     st.bad |= er.bad;
@@ -264,12 +282,13 @@ __device__ __forceinline__ void dec_group(WarpDec &st, const RowMeta &m, const u
 // SymT = float: the ring holds scales, each group's row is its scale's table
 // row, and the output is float(symbol) + mean, the means read one group
 // ahead with plain loads.
-template <typename SymT, bool IB0, bool WIDE, bool SEARCH>
+template <class F, typename SymT, bool IB0, bool WIDE, bool SEARCH>
 __device__ __forceinline__ void decode_stream_w32(const DecCtx &c, const StreamDesc &d,
                                                   const RowMeta *meta, const uint16_t *starts,
                                                   const uint32_t *slots, uint32_t *stg,
-                                                  int64_t s, const uint32_t *words, uint64_t nw,
-                                                  const float *stab) {
+                                                  int64_t s, const typename F::Word *words,
+                                                  uint64_t nw, const float *stab) {
+  using State = typename F::State;
   constexpr int kS = kDecStage;
   const int lane = threadIdx.x & 31;
   const int32_t n = (int32_t)d.n;
@@ -279,9 +298,10 @@ __device__ __forceinline__ void decode_stream_w32(const DecCtx &c, const StreamD
   const int32_t *idx_s = c.idx + (IB0 ? base : 0);
   SymT *out_s = reinterpret_cast<SymT *>(c.out) + base;
   const uint32_t kmax = (uint32_t)c.K - 1u;
+  const uint32_t sh = F::shift(c.sh);
 
-  WarpDec st;
-  st.x = (uint64_t)__ldg(words + 2 * lane) | ((uint64_t)__ldg(words + 2 * lane + 1) << 32);
+  WarpDec<F> st;
+  st.x = (State)__ldg(words + 2 * lane) | ((State)__ldg(words + 2 * lane + 1) << F::kWordBits);
   st.cur = 64;
   st.off = 0;
   load_window(st, words, nw);
@@ -336,70 +356,77 @@ __device__ __forceinline__ void decode_stream_w32(const DecCtx &c, const StreamD
     const RowMeta mn = meta_of(stg[((g + 1) & (kS - 1)) * 32 + lane]);
     const float mean_nn = kFlt ? mean_at(g + 2, pm.rel) : 0.0f;
     if (kFlt) pm.fwd(32);
-    dec_group<SymT, true, SEARCH>(st, m, starts, slots, true, out_s + pc.rel, words, nw, mean);
+    dec_group<F, SymT, true, SEARCH>(st, m, starts, slots, true, out_s + pc.rel, words, nw, sh,
+                                     mean);
     pc.fwd(32);
     m = mn;
     mean = mean_n;
     mean_n = mean_nn;
   }
-  dec_group<SymT, false, SEARCH>(st, m, starts, slots, lane < n - (G - 1) * 32, out_s + pc.rel,
-                                 words, nw, mean);
+  dec_group<F, SymT, false, SEARCH>(st, m, starts, slots, lane < n - (G - 1) * 32,
+                                    out_s + pc.rel, words, nw, sh, mean);
   cp_async_wait<0>();
   if (__any_sync(kFull, st.rmax > kmax)) {
     if (lane == 0) report(c.status, RANS_ERR_INDEX, s);
     return;
   }
-  const bool ok = !st.bad && st.x == kL && st.cur + st.off == nw;
+  const bool ok = !st.bad && st.x == F::kLow && st.cur + st.off == nw;
   if (!__all_sync(kFull, ok) && lane == 0) report(c.status, RANS_ERR_CORRUPT, s);
 }
 
-template <typename SymT, bool IB0, bool SEARCH>
+template <class F, typename SymT, bool IB0, bool SEARCH>
 __device__ __forceinline__ void decode_stream_w32_entry(const DecCtx &c, const RowMeta *meta,
                                                         const uint16_t *buckets,
                                                         const uint32_t *slots, uint32_t *stg,
                                                         int64_t s, const float *stab) {
+  using State = typename F::State;
+  using Word = typename F::Word;
   const int lane = threadIdx.x & 31;
   const StreamDesc d = stream_desc(c.g, s);
-  const uint32_t *words = nullptr;
+  const Word *words = nullptr;
   uint64_t nw = 0;
-  if (!d.ok || !stream_bounds(c, s, 32, words, nw)) {
+  if (!d.ok || !stream_bounds<F>(c, s, 32, words, nw)) {
     if (lane == 0) report(c.status, d.ok ? RANS_ERR_CORRUPT : RANS_ERR_ARG, s);
     return;
   }
   if (lane == 0)
     bulk_prefetch_l2(reinterpret_cast<const char *>(c.in),
                      reinterpret_cast<const char *>(c.in) + c.in_bytes,
-                     reinterpret_cast<const char *>(words + 64), 4 * (nw - 64));
-  if (d.n == 0) {  // only the 32 initial states, each 2^31
-    const uint64_t x =
-        (uint64_t)__ldg(words + 2 * lane) | ((uint64_t)__ldg(words + 2 * lane + 1) << 32);
-    if (!__all_sync(kFull, x == kL && nw == 64) && lane == 0) report(c.status, RANS_ERR_CORRUPT, s);
+                     reinterpret_cast<const char *>(words + 64), sizeof(Word) * (nw - 64));
+  if (d.n == 0) {  // only the 32 initial states
+    const State x =
+        (State)__ldg(words + 2 * lane) | ((State)__ldg(words + 2 * lane + 1) << F::kWordBits);
+    if (!__all_sync(kFull, x == F::kLow && nw == 64) && lane == 0)
+      report(c.status, RANS_ERR_CORRUPT, s);
     return;
   }
   if (d.t.ww >= 32)
-    decode_stream_w32<SymT, IB0, true, SEARCH>(c, d, meta, buckets, slots, stg, s, words, nw,
-                                               stab);
+    decode_stream_w32<F, SymT, IB0, true, SEARCH>(c, d, meta, buckets, slots, stg, s, words, nw,
+                                                  stab);
   else
-    decode_stream_w32<SymT, IB0, false, SEARCH>(c, d, meta, buckets, slots, stg, s, words, nw,
-                                                stab);
+    decode_stream_w32<F, SymT, IB0, false, SEARCH>(c, d, meta, buckets, slots, stg, s, words,
+                                                   nw, stab);
 }
 
-template <typename SymT>
+template <class F, typename SymT>
 __device__ void decode_stream_w1(const DecCtx &c, const RowMeta *meta, const uint16_t *buckets,
                                  const uint32_t *slots, int64_t s, const float *stab) {
+  using State = typename F::State;
+  using Word = typename F::Word;
   const StreamDesc d = stream_desc(c.g, s);
-  const uint32_t *words = nullptr;
+  const Word *words = nullptr;
   uint64_t nw = 0;
-  if (!d.ok || !stream_bounds(c, s, 1, words, nw)) {
+  if (!d.ok || !stream_bounds<F>(c, s, 1, words, nw)) {
     report(c.status, d.ok ? RANS_ERR_CORRUPT : RANS_ERR_ARG, s);
     return;
   }
   bulk_prefetch_l2(reinterpret_cast<const char *>(c.in),
                    reinterpret_cast<const char *>(c.in) + c.in_bytes,
-                   reinterpret_cast<const char *>(words), 4 * nw);
+                   reinterpret_cast<const char *>(words), sizeof(Word) * nw);
+  const uint32_t sh = F::shift(c.sh);
   const int ib = c.g.ib_shift;
   const Tile t = d.t;
-  uint64_t x = (uint64_t)__ldg(words) | ((uint64_t)__ldg(words + 1) << 32);
+  State x = (State)__ldg(words) | ((State)__ldg(words + 1) << F::kWordBits);
   uint64_t pw = 2;
   bool bad = false;
   auto rd = [&]() -> uint32_t {
@@ -437,18 +464,18 @@ __device__ void decode_stream_w1(const DecCtx &c, const RowMeta *meta, const uin
       return;
     }
     const RowMeta m = row_meta(meta, (uint32_t)r);
-    const uint32_t cum = (uint32_t)x & (kTotal - 1);
+    const uint32_t cum = F::cum16(x, sh);
     const uint32_t sym = lookup<true, false>(cum, m, buckets, slots, true);
     const uint32_t start = buckets[m.bucket_base + sym];
     const uint32_t freq = width_of(start, buckets[m.bucket_base + sym + 1]);
-    x = (uint64_t)freq * (x >> kPrec) + cum - start;
-    if (x < kL) x = (x << 32) | rd();
+    x = F::dec_step(x, cum, start, freq, sh);
+    if (x < F::kLow) x = (x << F::kWordBits) | rd();
     int64_t val = (int64_t)sym;
     if (sym == m.maxv) {
       auto getbits = [&]() -> uint32_t {
         const uint32_t v = (uint32_t)x & kBypassMax;
         x >>= kBypassBits;
-        if (x < kL) x = (x << 32) | rd();
+        if (x < F::kLow) x = (x << F::kWordBits) | rd();
         return v;
       };
       uint32_t v4 = getbits();
@@ -473,10 +500,10 @@ __device__ void decode_stream_w1(const DecCtx &c, const RowMeta *meta, const uin
     else
       SymIO<SymT>::store(c.out, p, val + (int64_t)m.offset);
   }
-  if (bad || x != kL || pw != nw) report(c.status, RANS_ERR_CORRUPT, s);
+  if (bad || x != F::kLow || pw != nw) report(c.status, RANS_ERR_CORRUPT, s);
 }
 
-template <int W, typename SymT, bool SMEM, bool IB0>
+template <class F, int W, typename SymT, bool SMEM, bool IB0>
 __global__ void __launch_bounds__(W == 32 ? kDecMaxThreads32 : kDecThreads1)
     decode_kernel(DecCtx c) {
   extern __shared__ __align__(16) unsigned char smem[];
@@ -518,22 +545,22 @@ __global__ void __launch_bounds__(W == 32 ? kDecMaxThreads32 : kDecThreads1)
     for (int64_t k = blockIdx.x + (int64_t)gridDim.x * warp; k < c.g.S;
          k += (int64_t)gridDim.x * nw) {
       if (search)
-        decode_stream_w32_entry<SymT, IB0, true>(c, meta, buckets, slots, stg, stream_of(c.g, k),
-                                                 stab);
+        decode_stream_w32_entry<F, SymT, IB0, true>(c, meta, buckets, slots, stg,
+                                                    stream_of(c.g, k), stab);
       else
-        decode_stream_w32_entry<SymT, IB0, false>(c, meta, buckets, slots, stg,
-                                                  stream_of(c.g, k), stab);
+        decode_stream_w32_entry<F, SymT, IB0, false>(c, meta, buckets, slots, stg,
+                                                     stream_of(c.g, k), stab);
     }
   } else {
     for (int64_t k = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; k < c.g.S;
          k += (int64_t)gridDim.x * blockDim.x)
-      decode_stream_w1<SymT>(c, meta, buckets, slots, stream_of(c.g, k), stab);
+      decode_stream_w1<F, SymT>(c, meta, buckets, slots, stream_of(c.g, k), stab);
   }
 }
 
-template <int W, typename SymT, bool SMEM, bool IB0>
+template <class F, int W, typename SymT, bool SMEM, bool IB0>
 int launch_decode_t(const DecCtx &c, cudaStream_t st) {
-  auto kern = decode_kernel<W, SymT, SMEM, IB0>;
+  auto kern = decode_kernel<F, W, SymT, SMEM, IB0>;
   const uint32_t tab = SMEM ? c.meta_bytes + c.start_bytes + c.slot_bytes : 0;
   const uint32_t per_warp = W == 32 ? kDecStage * 32 * 4 : 0;
   int dev = 0;
@@ -589,20 +616,26 @@ int launch_decode_t(const DecCtx &c, cudaStream_t st) {
   return cudaGetLastError() == cudaSuccess ? RANS_OK : RANS_ERR_CUDA;
 }
 
-template <int W, typename SymT>
+template <class F, int W, typename SymT>
 int launch_decode_w(const DecCtx &c, bool smem, cudaStream_t st) {
   const bool ib0 = c.g.ib_shift == 0;
   if (smem)
-    return ib0 ? launch_decode_t<W, SymT, true, true>(c, st)
-               : launch_decode_t<W, SymT, true, false>(c, st);
-  return ib0 ? launch_decode_t<W, SymT, false, true>(c, st)
-             : launch_decode_t<W, SymT, false, false>(c, st);
+    return ib0 ? launch_decode_t<F, W, SymT, true, true>(c, st)
+               : launch_decode_t<F, W, SymT, true, false>(c, st);
+  return ib0 ? launch_decode_t<F, W, SymT, false, true>(c, st)
+             : launch_decode_t<F, W, SymT, false, false>(c, st);
+}
+
+template <class F, typename SymT>
+int launch_decode_f(const DecCtx &c, bool smem, cudaStream_t st) {
+  return c.g.W == 32 ? launch_decode_w<F, 32, SymT>(c, smem, st)
+                     : launch_decode_w<F, 1, SymT>(c, smem, st);
 }
 
 template <typename SymT>
 int launch_decode_s(const DecCtx &c, bool smem, cudaStream_t st) {
-  return c.g.W == 32 ? launch_decode_w<32, SymT>(c, smem, st)
-                     : launch_decode_w<1, SymT>(c, smem, st);
+  return c.g.fmt == RANS_FMT_RANS32_16 ? launch_decode_f<Rans32, SymT>(c, smem, st)
+                                       : launch_decode_f<Rans64, SymT>(c, smem, st);
 }
 
 }  // namespace
@@ -617,6 +650,7 @@ int launch_decode_float(const uint8_t *in, uint64_t in_bytes, const uint64_t *of
   c.offs = offsets;
   c.idx = nullptr;
   c.K = t.K;
+  c.sh = 0;
   c.meta_bytes = t.meta_bytes;
   c.bucket_bytes = t.bucket_bytes;
   c.start_bytes = t.start_bytes;
@@ -630,8 +664,9 @@ int launch_decode_float(const uint8_t *in, uint64_t in_bytes, const uint64_t *of
   c.stab = scale_table;
   c.bound = scale_bound;
   const bool smem = t.dec_in_smem != 0;
-  return g.W == 32 ? launch_decode_w<32, float>(c, smem, st)
-                   : launch_decode_w<1, float>(c, smem, st);
+  // float values decode the 64-bit format only (the caller checks)
+  return g.W == 32 ? launch_decode_w<Rans64, 32, float>(c, smem, st)
+                   : launch_decode_w<Rans64, 1, float>(c, smem, st);
 }
 
 int launch_decode(const uint8_t *in, uint64_t in_bytes, const uint64_t *offsets,
@@ -643,6 +678,7 @@ int launch_decode(const uint8_t *in, uint64_t in_bytes, const uint64_t *offsets,
   c.offs = offsets;
   c.idx = indexes;
   c.K = t.K;
+  c.sh = (uint32_t)(kPrec - t.precision);
   c.meta_bytes = t.meta_bytes;
   c.bucket_bytes = t.bucket_bytes;
   c.start_bytes = t.start_bytes;

@@ -8,7 +8,11 @@
 //    pieces; "kompressor" README, Correctness: the bypass path);
 //  * symbol op: renormalise when x >= 2^47 freq, then
 //    x = (x / freq) 2^16 + x mod freq + start (64-bit state, 32-bit words,
-//    16-bit precision: "torch_ans 0.3.0", Usage, rans64 row);
+//    16-bit precision: "torch_ans 0.3.0", Usage, rans64 row); or, for the
+//    rans32_16 format (same table, rans32_16 row), renormalise when
+//    x >= 2^(32-p) freq and x = (x / freq) 2^p + x mod freq + start with
+//    16-bit words and a 32-bit state (the F template parameter; see
+//    Rans64 / Rans32 in rans_common.cuh);
 //  * W = 32: one warp per stream, lane = symbol index mod 32, one shared word
 //    stream ("torch_ans 0.3.0", Usage legend: __ballot_sync-based warp
 //    renormalisation with one shared cursor; FAQ: interleaved states share
@@ -46,6 +50,7 @@ struct EncCtx {
   float bound;
   int32_t stab_smem; // 1: the kernel copies the scale table into shared memory
   int32_t K;
+  uint32_t sh;       // 16 - precision of the rows (Rans32; 0 for Rans64)
   uint32_t meta_bytes, bucket_bytes;
   const char *blob;
   Geom g;
@@ -75,14 +80,14 @@ __device__ __forceinline__ void map_symbol(int32_t s, const RowMeta &m, const ui
   freq = bucket_freq(e);
 }
 
-// Bypass op: renormalise when x >= 2^59, then append 4 bits.
-template <bool WRITE>
-__device__ __forceinline__ void bits_op(uint64_t &x, uint32_t val, uint32_t *end, uint32_t &k,
-                                        uint32_t pos0) {
-  if (x >= (1ull << 59)) {
-    if (WRITE) st_global(end - 1 - (pos0 + k), (uint32_t)x);
+// Bypass op: renormalise when x >= 2^59 (Rans32: 2^28), then append 4 bits.
+template <class F, bool WRITE>
+__device__ __forceinline__ void bits_op(typename F::State &x, uint32_t val,
+                                        typename F::Word *end, uint32_t &k, uint32_t pos0) {
+  if (x >= F::kBitsBound) {
+    if (WRITE) st_global(end - 1 - (pos0 + k), (typename F::Word)x);
     ++k;
-    x >>= 32;
+    x >>= F::kWordBits;
   }
   x = (x << kBypassBits) | val;
 }
@@ -90,25 +95,27 @@ __device__ __forceinline__ void bits_op(uint64_t &x, uint32_t val, uint32_t *end
 // All ops of one symbol, in reverse op order (bypass pieces last to first,
 // then the count pieces last to first, then the symbol op).  Returns the
 // number of words pushed; with WRITE they go to end[-1 - (pos0 + j)].
-template <bool WRITE>
-__device__ __forceinline__ uint32_t symbol_ops(uint64_t &x, uint32_t start, uint32_t freq,
-                                               double rcp, uint64_t raw, bool esc,
-                                               uint32_t *end, uint32_t pos0) {
+template <class F, bool WRITE>
+__device__ __forceinline__ uint32_t symbol_ops(typename F::State &x, uint32_t start,
+                                               uint32_t freq, double rcp, uint64_t raw, bool esc,
+                                               typename F::Word *end, uint32_t pos0,
+                                               uint32_t sh) {
   uint32_t k = 0;
   if (esc) {
     uint32_t nb = 0;
     while (nb < 16 && (raw >> (kBypassBits * nb)) != 0) ++nb;
     for (int j = (int)nb - 1; j >= 0; --j)
-      bits_op<WRITE>(x, (uint32_t)(raw >> (kBypassBits * j)) & kBypassMax, end, k, pos0);
-    bits_op<WRITE>(x, nb % kBypassMax, end, k, pos0);
-    for (uint32_t t = 0; t < nb / kBypassMax; ++t) bits_op<WRITE>(x, kBypassMax, end, k, pos0);
+      bits_op<F, WRITE>(x, (uint32_t)(raw >> (kBypassBits * j)) & kBypassMax, end, k, pos0);
+    bits_op<F, WRITE>(x, nb % kBypassMax, end, k, pos0);
+    for (uint32_t t = 0; t < nb / kBypassMax; ++t)
+      bits_op<F, WRITE>(x, kBypassMax, end, k, pos0);
   }
-  if (x >= ((uint64_t)freq << 47)) {
-    if (WRITE) st_global(end - 1 - (pos0 + k), (uint32_t)x);
+  if (F::need_word(x, freq)) {
+    if (WRITE) st_global(end - 1 - (pos0 + k), (typename F::Word)x);
     ++k;
-    x >>= 32;
+    x >>= F::kWordBits;
   }
-  x = enc_sym_step(x, start, freq, rcp);
+  x = F::sym_step(x, start, freq, rcp, sh);
   return k;
 }
 
@@ -116,15 +123,15 @@ __device__ __forceinline__ uint32_t symbol_ops(uint64_t &x, uint32_t start, uint
 // A group holding an escape, off the fast path: every lane counts the words
 // its ops push, a suffix sum over lanes places each lane's block (lanes > l
 // push first in the serial order), then each lane writes its words.
-__device__ __forceinline__ uint64_t escape_group_enc(uint64_t x, bool active, uint32_t start,
-                                                     uint32_t freq, double rcp, uint64_t raw,
-                                                     bool esc, uint32_t *end, uint32_t cursor,
-                                                     uint32_t &total) {
+template <class F>
+__device__ __forceinline__ typename F::State escape_group_enc(
+    typename F::State x, bool active, uint32_t start, uint32_t freq, double rcp, uint64_t raw,
+    bool esc, typename F::Word *end, uint32_t cursor, uint32_t &total, uint32_t sh) {
   const int lane = threadIdx.x & 31;
   uint32_t k = 0;
   if (active) {
-    uint64_t y = x;
-    k = symbol_ops<false>(y, start, freq, rcp, raw, esc, end, 0);
+    typename F::State y = x;
+    k = symbol_ops<F, false>(y, start, freq, rcp, raw, esc, end, 0, sh);
   }
   uint32_t inc = k;
 #pragma unroll
@@ -133,13 +140,14 @@ __device__ __forceinline__ uint64_t escape_group_enc(uint64_t x, bool active, ui
     if (lane + o < 32) inc += t;
   }
   total = __shfl_sync(kFull, inc, 0);
-  if (active) symbol_ops<true>(x, start, freq, rcp, raw, esc, end, cursor + inc - k);
+  if (active) symbol_ops<F, true>(x, start, freq, rcp, raw, esc, end, cursor + inc - k, sh);
   return x;
 }
 
 // Per-warp encoder state for one stream.
+template <class F>
 struct WarpEnc {
-  uint64_t x;        // this lane's state
+  typename F::State x;  // this lane's state
   uint32_t cursor;   // words pushed so far (written at end[-1 - k])
   uint32_t rmax;     // largest row index seen (checked once per stream)
   bool range_err;
@@ -177,45 +185,48 @@ __device__ __forceinline__ EncBucket enc_bucket(int32_t sv, const RowMeta &m,
   return b;
 }
 
-__device__ __forceinline__ EncLook enc_look(const EncBucket &b, bool active) {
+template <class F>
+__device__ __forceinline__ EncLook enc_look(const EncBucket &b, bool active, uint32_t sh) {
   EncLook L;
   L.v = b.v;
   L.maxv = b.maxv;
   L.start = bucket_start(b.e);
   L.freq = bucket_freq(b.e);
-  L.rcp = freq_reciprocal(L.freq);
+  L.rcp = F::rcp(L.freq, sh);
   L.esc = active && !b.in_range;
   L.any_esc = __any_sync(kFull, L.esc);
   return L;
 }
 
 // One group of 32 symbols with no escape, coded lane 31 first: lanes whose
-// state reaches freq * 2^47 push its low word (ballot + popc place the
-// words), then every lane takes its symbol op.
-template <bool FULL>
-__device__ __forceinline__ void enc_group_fast(WarpEnc &st, const EncLook &L, bool active,
-                                               uint32_t above, uint32_t *end) {
+// state reaches the renormalisation bound push its low word (ballot + popc
+// place the words), then every lane takes its symbol op.
+template <class F, bool FULL>
+__device__ __forceinline__ void enc_group_fast(WarpEnc<F> &st, const EncLook &L, bool active,
+                                               uint32_t above, typename F::Word *end,
+                                               uint32_t sh) {
   if (FULL) active = true;
-  uint64_t x = st.x;
-  // x >= freq * 2^47  <=>  high word of x >= freq * 2^15
-  const bool need = active && (uint32_t)(x >> 32) >= (L.freq << 15);
+  typename F::State x = st.x;
+  const bool need = active && F::need_word(x, L.freq);
   const uint32_t bm = __ballot_sync(kFull, need);
-  if (need) st_global(end - 1 - (st.cursor + __popc(bm & above)), (uint32_t)x);
-  x = need ? (x >> 32) : x;
+  if (need) st_global(end - 1 - (st.cursor + __popc(bm & above)), (typename F::Word)x);
+  x = need ? (x >> F::kWordBits) : x;
   st.cursor += __popc(bm);
-  const uint64_t y = enc_sym_step(x, L.start, L.freq, L.rcp);
+  const typename F::State y = F::sym_step(x, L.start, L.freq, L.rcp, sh);
   st.x = active ? y : x;
 }
 
 // The same group holding an escape, from the state and cursor before it.
-__device__ __forceinline__ void enc_group_escape(WarpEnc &st, uint64_t x0, uint32_t cursor0,
-                                                 const EncLook &L, bool active, uint32_t *end) {
+template <class F>
+__device__ __forceinline__ void enc_group_escape(WarpEnc<F> &st, typename F::State x0,
+                                                 uint32_t cursor0, const EncLook &L, bool active,
+                                                 typename F::Word *end, uint32_t sh) {
   uint64_t raw = 0;
   if (L.esc) raw = L.v < 0 ? (uint64_t)(-2 * L.v - 1) : (uint64_t)(2 * (L.v - (int64_t)L.maxv));
   st.range_err |= L.esc && (raw >> 60) != 0;
   uint32_t total;
-  st.x = escape_group_enc(x0, active, L.start, L.freq, L.rcp, raw & ((1ull << 60) - 1), L.esc,
-                          end, cursor0, total);
+  st.x = escape_group_enc<F>(x0, active, L.start, L.freq, L.rcp, raw & ((1ull << 60) - 1),
+                             L.esc, end, cursor0, total, sh);
   st.cursor = cursor0 + total;
 }
 
@@ -228,14 +239,16 @@ __device__ __forceinline__ void enc_group_escape(WarpEnc &st, uint64_t x0, uint3
 // FLT: the stream's inputs are float latents: an 8-group ring holds scales
 // (as the row source), y and the means; each group's row is its scale's
 // table row and its symbol rint(y - mean).
-template <typename SymT, bool IB0, bool WIDE, bool FLT>
+template <class F, typename SymT, bool IB0, bool WIDE, bool FLT>
 __device__ __forceinline__ void encode_stream_w32(const EncCtx &c, const StreamDesc &d,
                                                   const RowMeta *meta, const uint32_t *buckets,
                                                   uint32_t *stg, int64_t s, const float *stab) {
   constexpr bool kStageSym = FLT || sizeof(SymT) == 4;
   constexpr int kS = enc_ring_groups(FLT);
+  using Word = typename F::Word;
   const int lane = threadIdx.x & 31;
-  uint32_t *end = reinterpret_cast<uint32_t *>(c.scratch + slot_end(c.g, d, s));
+  Word *end = reinterpret_cast<Word *>(c.scratch + slot_end(c.g, d, s));
+  const uint32_t sh = F::shift(c.sh);
   const int32_t n = (int32_t)d.n;
   const int32_t G = (n + 31) >> 5;
   const int64_t base = d.base;
@@ -247,8 +260,8 @@ __device__ __forceinline__ void encode_stream_w32(const EncCtx &c, const StreamD
   uint32_t *stg_idx = stg;
   uint32_t *stg_sym = stg + kS * 32;
   uint32_t *stg_mean = stg + 2 * kS * 32;  // FLT
-  WarpEnc st;
-  st.x = kL;
+  WarpEnc<F> st;
+  st.x = F::kLow;
   st.cursor = 0;
   st.rmax = 0;
   st.range_err = false;
@@ -322,7 +335,8 @@ __device__ __forceinline__ void encode_stream_w32(const EncCtx &c, const StreamD
     s0 = SymIO<SymT>::load(sym_s, active0 ? pn.rel : 0);
     pn.back(32);
   }
-  EncLook L = enc_look(enc_bucket(s0, meta_of(row_of(stg_idx[ring(0)])), buckets), active0);
+  EncLook L =
+      enc_look<F>(enc_bucket(s0, meta_of(row_of(stg_idx[ring(0)])), buckets), active0, sh);
   // group 1's symbol (FLT: its y and mean, quantised when used)
   int32_t s1 = G > 1 ? sym_of(1) : 0;
   float mean1 = FLT && G > 1 ? mean_of(1) : 0.0f;
@@ -334,11 +348,11 @@ __device__ __forceinline__ void encode_stream_w32(const EncCtx &c, const StreamD
     if (FLT) s1 = k + 1 < G ? quant(s1, mean1) : 0;
     const EncBucket b1 = enc_bucket(s1, m1, buckets);
     // group k's state update
-    const uint64_t x0 = st.x;
+    const typename F::State x0 = st.x;
     const uint32_t c0 = st.cursor;
-    enc_group_fast<decltype(full)::value>(st, L, active, above, end);
+    enc_group_fast<F, decltype(full)::value>(st, L, active, above, end, sh);
     // group k+1's reciprocal and escape ballot
-    const EncLook L1 = enc_look(b1, true);
+    const EncLook L1 = enc_look<F>(b1, true, sh);
     // copies, then the ring reads two and three groups ahead
     issue(k + kS - 1);
     cp_async_wait<kS - 4>();  // coded groups up to k + 3 have landed
@@ -346,7 +360,7 @@ __device__ __forceinline__ void encode_stream_w32(const EncCtx &c, const StreamD
     const float mean2 = FLT && k + 2 < G ? mean_of(k + 2) : 0.0f;
     const RowMeta m2 = meta_of(r2);
     const uint32_t r3 = k + 3 < G ? row_of(stg_idx[ring(k + 3)]) : 0u;
-    if (L.any_esc) enc_group_escape(st, x0, c0, L, active, end);
+    if (L.any_esc) enc_group_escape<F>(st, x0, c0, L, active, end, sh);
     L = L1;
     s1 = s2;
     mean1 = mean2;
@@ -367,12 +381,12 @@ __device__ __forceinline__ void encode_stream_w32(const EncCtx &c, const StreamD
   }
   // flush: lanes 31..0 push high then low, so lane 0's low word comes first
   const uint32_t kk = st.cursor + 2u * (31u - (uint32_t)lane);
-  st_global(end - 1 - kk, (uint32_t)(st.x >> 32));
-  st_global(end - 2 - kk, (uint32_t)st.x);
-  if (lane == 0) c.lens[s] = 4ull * (st.cursor + 64);
+  st_global(end - 1 - kk, (Word)(st.x >> F::kWordBits));
+  st_global(end - 2 - kk, (Word)st.x);
+  if (lane == 0) c.lens[s] = sizeof(Word) * (uint64_t)(st.cursor + 64);
 }
 
-template <typename SymT, bool IB0, bool FLT>
+template <class F, typename SymT, bool IB0, bool FLT>
 __device__ __forceinline__ void encode_stream_w32_entry(const EncCtx &c, const RowMeta *meta,
                                                         const uint32_t *buckets, uint32_t *stg,
                                                         int64_t s, const float *stab) {
@@ -382,32 +396,35 @@ __device__ __forceinline__ void encode_stream_w32_entry(const EncCtx &c, const R
     return;
   }
   if (d.n == 0) {  // flush the 32 initial states only
+    using Word = typename F::Word;
     const int lane = threadIdx.x & 31;
-    uint32_t *end = reinterpret_cast<uint32_t *>(c.scratch + slot_end(c.g, d, s));
-    end[-1 - 2 * (31 - lane)] = (uint32_t)(kL >> 32);
-    end[-2 - 2 * (31 - lane)] = (uint32_t)kL;
-    if (lane == 0) c.lens[s] = 256;
+    Word *end = reinterpret_cast<Word *>(c.scratch + slot_end(c.g, d, s));
+    end[-1 - 2 * (31 - lane)] = (Word)(F::kLow >> F::kWordBits);
+    end[-2 - 2 * (31 - lane)] = (Word)F::kLow;
+    if (lane == 0) c.lens[s] = 64 * sizeof(Word);
     return;
   }
   if (d.t.ww >= 32)
-    encode_stream_w32<SymT, IB0, true, FLT>(c, d, meta, buckets, stg, s, stab);
+    encode_stream_w32<F, SymT, IB0, true, FLT>(c, d, meta, buckets, stg, s, stab);
   else
-    encode_stream_w32<SymT, IB0, false, FLT>(c, d, meta, buckets, stg, s, stab);
+    encode_stream_w32<F, SymT, IB0, false, FLT>(c, d, meta, buckets, stg, s, stab);
 }
 
-template <typename SymT, bool FLT>
+template <class F, typename SymT, bool FLT>
 __device__ void encode_stream_w1(const EncCtx &c, const RowMeta *meta, const uint32_t *buckets,
                                  int64_t s, const float *stab) {
+  using Word = typename F::Word;
   const StreamDesc d = stream_desc(c.g, s);
   if (!d.ok) {
     report(c.status, RANS_ERR_ARG, s);
     return;
   }
-  uint32_t *end = reinterpret_cast<uint32_t *>(c.scratch + slot_end(c.g, d, s));
+  Word *end = reinterpret_cast<Word *>(c.scratch + slot_end(c.g, d, s));
+  const uint32_t sh = F::shift(c.sh);
   const int ib = c.g.ib_shift;
   const Tile t = d.t;
   const int32_t n = (int32_t)d.n;
-  uint64_t x = kL;
+  typename F::State x = F::kLow;
   uint32_t cursor = 0;
   RelPos pl, pp;
   pl.init(t, n > 0 ? n - 1 : 0);
@@ -463,15 +480,15 @@ __device__ void encode_stream_w1(const EncCtx &c, const RowMeta *meta, const uin
       report(c.status, RANS_ERR_RANGE, s);
       return;
     }
-    cursor += symbol_ops<true>(x, start, freq, freq_reciprocal(freq), raw, esc, end, cursor);
+    cursor += symbol_ops<F, true>(x, start, freq, F::rcp(freq, sh), raw, esc, end, cursor, sh);
   }
-  end[-1 - (int64_t)cursor] = (uint32_t)(x >> 32);
-  end[-2 - (int64_t)cursor] = (uint32_t)x;
+  end[-1 - (int64_t)cursor] = (Word)(x >> F::kWordBits);
+  end[-2 - (int64_t)cursor] = (Word)x;
   cursor += 2;
-  c.lens[s] = 4ull * cursor;
+  c.lens[s] = sizeof(Word) * (uint64_t)cursor;
 }
 
-template <int W, typename SymT, bool SMEM, bool IB0, bool FLT>
+template <class F, int W, typename SymT, bool SMEM, bool IB0, bool FLT>
 __global__ void __launch_bounds__(W == 32 ? kEncThreads32 : kEncThreads1)
     encode_kernel(EncCtx c) {
   extern __shared__ __align__(16) unsigned char smem[];
@@ -504,11 +521,12 @@ __global__ void __launch_bounds__(W == 32 ? kEncThreads32 : kEncThreads1)
                     warp * (enc_stage_bytes_per_warp(FLT) / 4);
     for (int64_t k = blockIdx.x + (int64_t)gridDim.x * warp; k < c.g.S;
          k += (int64_t)gridDim.x * nw)
-      encode_stream_w32_entry<SymT, IB0, FLT>(c, meta, buckets, stg, stream_of(c.g, k), stab);
+      encode_stream_w32_entry<F, SymT, IB0, FLT>(c, meta, buckets, stg, stream_of(c.g, k),
+                                                 stab);
   } else {
     for (int64_t k = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; k < c.g.S;
          k += (int64_t)gridDim.x * blockDim.x)
-      encode_stream_w1<SymT, FLT>(c, meta, buckets, stream_of(c.g, k), stab);
+      encode_stream_w1<F, SymT, FLT>(c, meta, buckets, stream_of(c.g, k), stab);
   }
 }
 
@@ -559,6 +577,9 @@ __global__ void __launch_bounds__(kScanThreads)
   if (threadIdx.x == 0 && carry_sh > capacity) report(status, RANS_ERR_CAPACITY, -1);
 }
 
+// Word: the format's stream word (stream lengths and offsets are multiples
+// of its size).
+template <typename Word>
 __global__ void copy_streams_kernel(Geom g, const char *scratch, const uint64_t *lens,
                                     const uint64_t *offsets, uint8_t *out, uint64_t capacity) {
   const int lane = threadIdx.x & 31;
@@ -570,10 +591,9 @@ __global__ void copy_streams_kernel(Geom g, const char *scratch, const uint64_t 
     const uint64_t len = lens[s];
     const uint64_t off = offsets[s];
     if (off + len > capacity) continue;
-    const uint32_t *src =
-        reinterpret_cast<const uint32_t *>(scratch + slot_end(g, d, s) - len);
-    uint32_t *dst = reinterpret_cast<uint32_t *>(out + off);
-    const uint64_t words = len >> 2;
+    const Word *src = reinterpret_cast<const Word *>(scratch + slot_end(g, d, s) - len);
+    Word *dst = reinterpret_cast<Word *>(out + off);
+    const uint64_t words = len / sizeof(Word);
     for (uint64_t k = lane; k < words; k += 32) dst[k] = __ldg(src + k);
   }
 }
@@ -590,9 +610,9 @@ __global__ void debug_divide_kernel(const uint64_t *x, const uint32_t *f, int64_
   }
 }
 
-template <int W, typename SymT, bool SMEM, bool IB0, bool FLT>
+template <class F, int W, typename SymT, bool SMEM, bool IB0, bool FLT>
 int launch_encode_t(const EncCtx &c, cudaStream_t st) {
-  auto kern = encode_kernel<W, SymT, SMEM, IB0, FLT>;
+  auto kern = encode_kernel<F, W, SymT, SMEM, IB0, FLT>;
   const uint32_t tab = SMEM ? c.meta_bytes + c.bucket_bytes : 0;
   const uint32_t per_warp = W == 32 ? enc_stage_bytes_per_warp(FLT) : 0;
   uint32_t smem = tab;
@@ -649,20 +669,26 @@ int launch_encode_t(const EncCtx &c, cudaStream_t st) {
   return cudaGetLastError() == cudaSuccess ? RANS_OK : RANS_ERR_CUDA;
 }
 
-template <int W, typename SymT>
+template <class F, int W, typename SymT>
 int launch_encode_w(const EncCtx &c, bool smem, cudaStream_t st) {
   const bool ib0 = c.g.ib_shift == 0;
   if (smem)
-    return ib0 ? launch_encode_t<W, SymT, true, true, false>(c, st)
-               : launch_encode_t<W, SymT, true, false, false>(c, st);
-  return ib0 ? launch_encode_t<W, SymT, false, true, false>(c, st)
-             : launch_encode_t<W, SymT, false, false, false>(c, st);
+    return ib0 ? launch_encode_t<F, W, SymT, true, true, false>(c, st)
+               : launch_encode_t<F, W, SymT, true, false, false>(c, st);
+  return ib0 ? launch_encode_t<F, W, SymT, false, true, false>(c, st)
+             : launch_encode_t<F, W, SymT, false, false, false>(c, st);
+}
+
+template <class F, typename SymT>
+int launch_encode_f(const EncCtx &c, bool smem, cudaStream_t st) {
+  return c.g.W == 32 ? launch_encode_w<F, 32, SymT>(c, smem, st)
+                     : launch_encode_w<F, 1, SymT>(c, smem, st);
 }
 
 template <typename SymT>
 int launch_encode_s(const EncCtx &c, bool smem, cudaStream_t st) {
-  return c.g.W == 32 ? launch_encode_w<32, SymT>(c, smem, st)
-                     : launch_encode_w<1, SymT>(c, smem, st);
+  return c.g.fmt == RANS_FMT_RANS32_16 ? launch_encode_f<Rans32, SymT>(c, smem, st)
+                                       : launch_encode_f<Rans64, SymT>(c, smem, st);
 }
 
 }  // namespace
@@ -674,6 +700,7 @@ int launch_encode(const void *symbols, int sym_dtype, const int32_t *indexes,
   c.sym = symbols;
   c.idx = indexes;
   c.K = t.K;
+  c.sh = (uint32_t)(kPrec - t.precision);
   c.meta_bytes = t.meta_bytes;
   c.bucket_bytes = t.bucket_bytes;
   c.blob = reinterpret_cast<const char *>(t.blob);
@@ -706,6 +733,7 @@ int launch_encode_float(const float *y, const float *means, const float *scales,
   c.stab = scale_table;
   c.bound = scale_bound;
   c.K = t.K;
+  c.sh = 0;
   c.meta_bytes = t.meta_bytes;
   c.bucket_bytes = t.bucket_bytes;
   c.blob = reinterpret_cast<const char *>(t.blob);
@@ -714,11 +742,12 @@ int launch_encode_float(const float *y, const float *means, const float *scales,
   c.lens = lens;
   c.status = status;
   const bool smem = t.enc_in_smem != 0;
+  // float latents code the 64-bit format only (the caller checks)
   if (g.W == 32)
-    return smem ? launch_encode_t<32, int32_t, true, true, true>(c, st)
-                : launch_encode_t<32, int32_t, false, true, true>(c, st);
-  return smem ? launch_encode_t<1, int32_t, true, true, true>(c, st)
-              : launch_encode_t<1, int32_t, false, true, true>(c, st);
+    return smem ? launch_encode_t<Rans64, 32, int32_t, true, true, true>(c, st)
+                : launch_encode_t<Rans64, 32, int32_t, false, true, true>(c, st);
+  return smem ? launch_encode_t<Rans64, 1, int32_t, true, true, true>(c, st)
+              : launch_encode_t<Rans64, 1, int32_t, false, true, true>(c, st);
 }
 
 int launch_compact(const Geom &g, const char *scratch, const uint64_t *lens, uint8_t *out,
@@ -731,8 +760,12 @@ int launch_compact(const Geom &g, const char *scratch, const uint64_t *lens, uin
     int64_t blocks = (g.S + 7) / 8;
     const int64_t cap = 8LL * num_sms(dev);
     if (blocks > cap) blocks = cap;
-    copy_streams_kernel<<<(unsigned)blocks, 256, 0, st>>>(g, scratch, lens, offsets, out,
-                                                          out_capacity);
+    if (g.fmt == RANS_FMT_RANS32_16)
+      copy_streams_kernel<uint16_t><<<(unsigned)blocks, 256, 0, st>>>(g, scratch, lens, offsets,
+                                                                      out, out_capacity);
+    else
+      copy_streams_kernel<uint32_t><<<(unsigned)blocks, 256, 0, st>>>(g, scratch, lens, offsets,
+                                                                      out, out_capacity);
   }
   return cudaGetLastError() == cudaSuccess ? RANS_OK : RANS_ERR_CUDA;
 }

@@ -118,6 +118,8 @@ struct Geom {
   int64_t ng, nty, ntx;  // TILED counts per image
   int32_t ib_shift;      // log2(index_block)
   int32_t nclass;        // TILED: tile classes in scheduling order (<= 8)
+  int32_t fmt;           // RANS_FMT_*
+  int32_t pad_;
   uint64_t slot_bytes;   // CONTIG / TILED: uniform scratch slot per stream
   uint64_t slot_extra;   // 16 W + 16: per-stream scratch beyond 8 B/symbol
   // TILED: a class is the set of tiles sharing (last channel group?, last
@@ -344,6 +346,7 @@ __device__ __forceinline__ void bulk_prefetch_l2(const char *lo, const char *hi,
 // knows they cannot touch shared memory and may move shared-memory loads
 // across them.
 __device__ __forceinline__ void st_global(uint32_t *p, uint32_t v) { __stcg(p, v); }
+__device__ __forceinline__ void st_global(uint16_t *p, uint16_t v) { __stcg(p, v); }
 __device__ __forceinline__ void st_global(int32_t *p, int32_t v) { __stcs(p, v); }
 __device__ __forceinline__ void st_global(int16_t *p, int16_t v) { __stcs(p, v); }
 __device__ __forceinline__ void st_global(uint8_t *p, uint8_t v) { __stcs(p, v); }
@@ -483,6 +486,87 @@ __device__ __forceinline__ uint64_t enc_sym_step(uint64_t x, uint32_t start, uin
   divmod_freq(x, f, rcp, q, r);
   return (q << kPrec) + (r + start);
 }
+
+// The same division for a 32-bit state (x < 2^32 is exact in a double, so the
+// argument above holds with room to spare).
+__device__ __forceinline__ void divmod_freq32(uint32_t x, uint32_t f, double rcp, uint32_t &q,
+                                              uint32_t &r) {
+  const double t = fma(u32_to_double(x), rcp, 4503599627370496.0);  // 2^52 + round(x / f)
+  const uint32_t qe = (uint32_t)__double_as_longlong(t);
+  const int32_t rem = (int32_t)(x - qe * f);
+  const bool over = rem < 0;
+  q = qe - (over ? 1u : 0u);
+  r = (uint32_t)(rem + (over ? (int32_t)f : 0));
+}
+
+// ------------------------------------------------------- coder formats --
+// Two formats ("torch_ans 0.3.0", Usage, variants table):
+//   Rans64: 64-bit state, 32-bit words, 16-bit precision, lower bound 2^31;
+//   Rans32: 32-bit state, 16-bit words, precision p <= 15, lower bound 2^16
+//           (the bound for which one 16-bit word restores the state).
+// The prepared tables hold every CDF entry scaled to 16 bits (entry << sh,
+// sh = 16 - p), so the lookup works on cum << sh and the coder shifts starts
+// and widths back down.  In 16-bit units the renormalisation bound of either
+// format is width16 * 2^(log2 L + word bits - 16): 2^47 and 2^16.
+// A bypass op renormalises when x >= 2^(state bits - 5): 2^59 and 2^28.
+struct Rans64 {
+  using State = uint64_t;
+  using Word = uint32_t;
+  static constexpr uint32_t kWordBits = 32;
+  static constexpr uint64_t kLow = 1ull << 31;
+  static constexpr uint64_t kBitsBound = 1ull << 59;
+  static constexpr int kFmt = RANS_FMT_RANS64;
+  __device__ __forceinline__ static uint32_t shift(uint32_t) { return 0; }
+  // x >= width16 * 2^47  <=>  high word of x >= width16 * 2^15
+  __device__ __forceinline__ static bool need_word(uint64_t x, uint32_t f16) {
+    return (uint32_t)(x >> 32) >= (f16 << 15);
+  }
+  __device__ __forceinline__ static double rcp(uint32_t f16, uint32_t) {
+    return freq_reciprocal(f16);
+  }
+  __device__ __forceinline__ static uint64_t sym_step(uint64_t x, uint32_t start16, uint32_t f16,
+                                                      double rcp, uint32_t) {
+    return enc_sym_step(x, start16, f16, rcp);
+  }
+  // decoder: x -> width (x >> 16) + cum - start
+  __device__ __forceinline__ static uint32_t cum16(uint64_t x, uint32_t) {
+    return (uint32_t)x & (kTotal - 1);
+  }
+  __device__ __forceinline__ static uint64_t dec_step(uint64_t x, uint32_t cum16, uint32_t start16,
+                                                      uint32_t f16, uint32_t) {
+    return (uint64_t)f16 * (x >> kPrec) + (cum16 - start16);
+  }
+};
+
+struct Rans32 {
+  using State = uint32_t;
+  using Word = uint16_t;
+  static constexpr uint32_t kWordBits = 16;
+  static constexpr uint32_t kLow = 1u << 16;
+  static constexpr uint32_t kBitsBound = 1u << 28;
+  static constexpr int kFmt = RANS_FMT_RANS32_16;
+  __device__ __forceinline__ static uint32_t shift(uint32_t sh) { return sh; }
+  __device__ __forceinline__ static bool need_word(uint32_t x, uint32_t f16) {
+    return (x >> 16) >= f16;
+  }
+  __device__ __forceinline__ static double rcp(uint32_t f16, uint32_t sh) {
+    return freq_reciprocal(f16 >> sh);
+  }
+  // x -> (x / f) 2^p + x mod f + start with f, start at precision p
+  __device__ __forceinline__ static uint32_t sym_step(uint32_t x, uint32_t start16, uint32_t f16,
+                                                      double rcp, uint32_t sh) {
+    uint32_t q, r;
+    divmod_freq32(x, f16 >> sh, rcp, q, r);
+    return (q << (kPrec - sh)) + r + (start16 >> sh);
+  }
+  __device__ __forceinline__ static uint32_t cum16(uint32_t x, uint32_t sh) {
+    return (x << sh) & (kTotal - 1);
+  }
+  __device__ __forceinline__ static uint32_t dec_step(uint32_t x, uint32_t cum16, uint32_t start16,
+                                                      uint32_t f16, uint32_t sh) {
+    return (f16 >> sh) * (x >> (kPrec - sh)) + ((cum16 - start16) >> sh);
+  }
+};
 
 // ------------------------------------------------------- warp helpers --
 __device__ __forceinline__ uint32_t lanemask_lt() {

@@ -13,20 +13,22 @@ struct Geom;
 
 int launch_gaussian_lengths(const float *scales, int K, double tail, int32_t *lengths,
                             int32_t *offsets, cudaStream_t st);
-int launch_gaussian_rows(const float *scales, int K, double tail, int32_t *cdfs, int Lmax,
-                         int32_t *lengths, int32_t *offsets, cudaStream_t st);
+// Rows summing to 2^prec (1 <= prec <= 16).
+int launch_gaussian_rows(const float *scales, int K, double tail, int prec, int32_t *cdfs,
+                         int Lmax, int32_t *lengths, int32_t *offsets, cudaStream_t st);
 int launch_pmf_rows(const float *pmfs, int K, int stride, const int32_t *pmf_lengths,
-                    const float *tail, int32_t *cdfs, int Lmax, int32_t *lengths,
+                    const float *tail, int prec, int32_t *cdfs, int Lmax, int32_t *lengths,
                     cudaStream_t st);
 uint64_t tables_bytes_bound(int K, int Lmax);
 int refresh_tables(const int32_t *cdfs, int K, int Lmax, const int32_t *lengths,
                    const int32_t *offsets, const rans_tables &t, cudaStream_t st);
+// Rows summing to 2^prec, stored scaled to 16 bits.
 int prepare_tables(const int32_t *cdfs, int K, int Lmax, const int32_t *lengths,
-                   const int32_t *offsets, void *blob, uint64_t blob_bytes, rans_tables *out,
-                   cudaStream_t st);
+                   const int32_t *offsets, int prec, void *blob, uint64_t blob_bytes,
+                   rans_tables *out, cudaStream_t st);
 
 // Encoder: codes every stream into its scratch slot and records its byte
-// length in lens[S].
+// length in lens[S] (coder format g.fmt, rows of precision t.precision).
 int launch_encode(const void *symbols, int sym_dtype, const int32_t *indexes,
                   const rans_tables &t, const Geom &g, char *scratch, uint64_t *lens,
                   int32_t *status, cudaStream_t st);

@@ -70,10 +70,10 @@ __device__ unsigned long long block_sum(unsigned long long v, BlockScratch &sh) 
   return t;
 }
 
-// Scaled and rounded probability: round(p * 2^16) half away from zero, or
-// -1 when p is negative, not finite or too large.
-__device__ __forceinline__ long long scaled_freq(float p) {
-  float v = p * (float)kTotal;            // exact: times a power of two
+// Scaled and rounded probability: round(p * total) half away from zero
+// (total = 2^precision), or -1 when p is negative, not finite or too large.
+__device__ __forceinline__ long long scaled_freq(float p, uint32_t total) {
+  float v = p * (float)total;             // exact: times a power of two
   float r = roundf(v);                    // half away from zero
   if (!(r >= 0.0f) || (double)r > 4294967295.0) return -1;
   return (long long)r;
@@ -106,7 +106,7 @@ struct QuantScratch {
 
 template <class PF>
 __device__ int quantise_row(const PF &pf, int n, int32_t *row, BlockScratch &sh,
-                            QuantScratch &q) {
+                            QuantScratch &q, uint32_t total) {
   const int per = (n + kRowThreads - 1) / kRowThreads;
   const int i0 = min(n, (int)threadIdx.x * per), i1 = min(n, i0 + per);
   // pass 1: rounded values, each probability evaluated once
@@ -119,15 +119,15 @@ __device__ int quantise_row(const PF &pf, int n, int32_t *row, BlockScratch &sh,
   bad = __syncthreads_or(bad);
   if (bad || T == 0) return RANS_ERR_TABLE;
 
-  // pass 2: widths of the rescaled running sum floor(2^16 c / T); count the
+  // pass 2: widths of the rescaled running sum floor(total c / T); count the
   // empty buckets and the widths of the others
   unsigned long long zl = 0;
   {
     unsigned long long c = before;
-    unsigned long long b0 = ((unsigned long long)kTotal * c) / T;
+    unsigned long long b0 = ((unsigned long long)total * c) / T;
     for (int i = i0; i < i1; ++i) {
       c += (uint32_t)row[i + 1];
-      const unsigned long long b1 = ((unsigned long long)kTotal * c) / T;
+      const unsigned long long b1 = ((unsigned long long)total * c) / T;
       const uint32_t w = (uint32_t)(b1 - b0);
       b0 = b1;
       row[i + 1] = (int32_t)w;
@@ -238,6 +238,7 @@ __global__ void gaussian_lengths_kernel(const float *scales, int K, double tail,
 struct GaussPmf {
   int center, npmf;
   double s;
+  uint32_t total;  // 2^precision
   __device__ unsigned long long eval(int i0, int i1, int32_t *f, int &bad) const {
     unsigned long long sum = 0;
     int da = -1, db = -1;  // the two most recent u values
@@ -262,7 +263,7 @@ struct GaussPmf {
         const double lo = u(d + 1);
         p = (float)(hi - lo);
       }
-      long long q = scaled_freq(p);
+      long long q = scaled_freq(p, total);
       if (q < 0) {
         bad = 1;
         q = 0;
@@ -278,10 +279,11 @@ struct GivenPmf {
   const float *p;
   int n;
   float tail;
+  uint32_t total;  // 2^precision
   __device__ unsigned long long eval(int i0, int i1, int32_t *f, int &bad) const {
     unsigned long long sum = 0;
     for (int i = i0; i < i1; ++i) {
-      long long q = scaled_freq(i == n ? tail : p[i]);
+      long long q = scaled_freq(i == n ? tail : p[i], total);
       if (q < 0) {
         bad = 1;
         q = 0;
@@ -294,7 +296,7 @@ struct GivenPmf {
 };
 
 __global__ void __launch_bounds__(kRowThreads)
-    gaussian_rows_kernel(const float *scales, double tail, int32_t *cdfs, int Lmax,
+    gaussian_rows_kernel(const float *scales, double tail, int prec, int32_t *cdfs, int Lmax,
                          int32_t *lengths, int32_t *offsets) {
   __shared__ BlockScratch sh;
   __shared__ QuantScratch qs;
@@ -305,8 +307,8 @@ __global__ void __launch_bounds__(kRowThreads)
   int len = 2 * c + 3;
   if (st == RANS_OK && len > Lmax) st = RANS_ERR_CAPACITY;
   if (st == RANS_OK) {
-    GaussPmf pf{c, 2 * c + 1, (double)scales[r]};
-    st = quantise_row(pf, 2 * c + 2, row, sh, qs);
+    GaussPmf pf{c, 2 * c + 1, (double)scales[r], 1u << prec};
+    st = quantise_row(pf, 2 * c + 2, row, sh, qs, 1u << prec);
   }
   for (int j = (st == RANS_OK ? len : 0) + threadIdx.x; j < Lmax; j += kRowThreads) row[j] = 0;
   if (threadIdx.x == 0) {
@@ -317,7 +319,7 @@ __global__ void __launch_bounds__(kRowThreads)
 
 __global__ void __launch_bounds__(kRowThreads)
     pmf_rows_kernel(const float *pmfs, int stride, const int32_t *pmf_lengths,
-                    const float *tail, int32_t *cdfs, int Lmax, int32_t *lengths) {
+                    const float *tail, int prec, int32_t *cdfs, int Lmax, int32_t *lengths) {
   __shared__ BlockScratch sh;
   __shared__ QuantScratch qs;
   const int r = blockIdx.x;
@@ -327,8 +329,8 @@ __global__ void __launch_bounds__(kRowThreads)
   if (n < 0 || n > stride) st = RANS_ERR_ARG;
   else if (n + 2 > Lmax) st = RANS_ERR_CAPACITY;
   if (st == RANS_OK) {
-    GivenPmf pf{pmfs + (size_t)r * (size_t)stride, n, tail[r]};
-    st = quantise_row(pf, n + 1, row, sh, qs);
+    GivenPmf pf{pmfs + (size_t)r * (size_t)stride, n, tail[r], 1u << prec};
+    st = quantise_row(pf, n + 1, row, sh, qs, 1u << prec);
   }
   for (int j = (st == RANS_OK ? n + 2 : 0) + threadIdx.x; j < Lmax; j += kRowThreads) row[j] = 0;
   if (threadIdx.x == 0) lengths[r] = st ? st : n + 2;
@@ -336,35 +338,44 @@ __global__ void __launch_bounds__(kRowThreads)
 
 // ---- prepared tables ----------------------------------------------------
 
+// Rows of precision p are stored scaled to 16 bits: entry << sh, sh = 16 - p.
+// The bucket word of entries a < b: start | (width - 1) << 16, scaled.
+__device__ __forceinline__ uint32_t bucket_word(int32_t a, int32_t b, uint32_t sh) {
+  return (uint32_t)((a << sh) & 0xffff) | ((uint32_t)(((b - a) << sh) - 1) << 16);
+}
+
 // Validates row r and writes its packed buckets.  One block per row.
 __global__ void pack_buckets_kernel(const int32_t *cdfs, int Lmax, const RowMeta *meta,
-                                    const int32_t *lengths, uint32_t *buckets,
+                                    const int32_t *lengths, uint32_t sh, uint32_t *buckets,
                                     uint16_t *starts, int32_t *status) {
   const int r = blockIdx.x;
   const int32_t *row = cdfs + (size_t)r * (size_t)Lmax;
   const int len = lengths[r];
+  const int32_t top = (int32_t)(kTotal >> sh);
   const uint32_t base = meta[r * kMetaCopies].bucket_base;
-  if (threadIdx.x == 0 && (row[0] != 0 || row[len - 1] != (int32_t)kTotal))
+  if (threadIdx.x == 0 && (row[0] != 0 || row[len - 1] != top))
     report(status, RANS_ERR_TABLE, r);
   for (int j = threadIdx.x; j < len - 1; j += blockDim.x) {
     int32_t a = row[j], b = row[j + 1];
-    if (!(b > a) || a < 0 || b > (int32_t)kTotal) {
+    if (!(b > a) || a < 0 || b > top) {
       report(status, RANS_ERR_TABLE, r);
       continue;
     }
-    buckets[base + j] = (uint32_t)(a & 0xffff) | ((uint32_t)(b - a - 1) << 16);
+    buckets[base + j] = bucket_word(a, b, sh);
   }
   // 16-bit starts, row end included: it writes 0 over the next row's leading
   // 0 (or the trailing sentinel), so overlapping rows agree
-  for (int j = threadIdx.x; j < len; j += blockDim.x) starts[base + j] = (uint16_t)row[j];
+  for (int j = threadIdx.x; j < len; j += blockDim.x)
+    starts[base + j] = (uint16_t)(row[j] << sh);
 }
 
-// Largest j in [0, nb) with row[j] <= v (row strictly increasing, row[0]=0).
-__device__ __forceinline__ int bucket_of(const int32_t *row, int nb, int v) {
+// Largest j in [0, nb) with row[j] << sh <= v (row strictly increasing,
+// row[0] = 0).
+__device__ __forceinline__ int bucket_of(const int32_t *row, int nb, int v, uint32_t sh) {
   int lo = 0, hi = nb - 1;
   while (lo < hi) {
     int mid = (lo + hi + 1) >> 1;
-    if (row[mid] <= v) lo = mid; else hi = mid - 1;
+    if ((row[mid] << sh) <= v) lo = mid; else hi = mid - 1;
   }
   return lo;
 }
@@ -393,21 +404,21 @@ constexpr uint32_t kSlotSmemBytes = 4u * kRowSmem;
 // The row is strictly increasing, so the buckets starting inside are
 // jj + 1 .. jj + 15 at most and their loads do not wait on one another.
 __device__ __forceinline__ uint32_t boundary_bits(const int32_t *row, int nb, int jj, int c0,
-                                                  int c1) {
+                                                  int c1, uint32_t sh) {
   uint32_t bits = 0;
 #pragma unroll
   for (int u = 1; u <= 15; ++u) {
     const int i = jj + u;
-    const int v = i < nb ? row[i] : (int)kTotal;
+    const int v = i < nb ? row[i] << sh : (int)kTotal;
     if (v < c1) bits |= 1u << ((v - c0) & 31);
   }
   return bits;
 }
 
 // The slots [tb, tb + kSlotsPerBlock) of a row (row in shared or global
-// memory).
+// memory, entries scaled by << sh).
 __device__ void fill_slot_block(const int32_t *row, int nb, uint32_t slot0, int w, int nslots,
-                                int tb, uint32_t *slots, const ChunkArea &ca) {
+                                int tb, uint32_t *slots, const ChunkArea &ca, uint32_t sh) {
   const int lane = threadIdx.x & 31;
   const int t0 = tb + (int)threadIdx.x * kSlotsPerThread;
   const uint32_t nch = w > 16 ? (uint32_t)(w >> 4) : 1u;  // bitmap words of a slot
@@ -418,8 +429,8 @@ __device__ void fill_slot_block(const int32_t *row, int nb, uint32_t slot0, int 
     const int t = t0 + u;
     lo[u] = hi[u] = 0;
     if (t < nslots) {
-      lo[u] = bucket_of(row, nb, t * w);
-      hi[u] = bucket_of(row, nb, t * w + w - 1);
+      lo[u] = bucket_of(row, nb, t * w, sh);
+      hi[u] = bucket_of(row, nb, t * w + w - 1, sh);
       if (hi[u] - lo[u] >= 3) need += nch;
     }
   }
@@ -443,8 +454,8 @@ __device__ void fill_slot_block(const int32_t *row, int nb, uint32_t slot0, int 
     uint32_t word;
     if (inside <= 2) {
       uint32_t e1 = 255u, e2 = 255u;
-      if (inside >= 1) e1 = (uint32_t)(row[lo[u] + 1] - a - 1);
-      if (inside == 2) e2 = (uint32_t)(row[lo[u] + 2] - a - 1);
+      if (inside >= 1) e1 = (uint32_t)((row[lo[u] + 1] << sh) - a - 1);
+      if (inside == 2) e2 = (uint32_t)((row[lo[u] + 2] << sh) - a - 1);
       word = (uint32_t)lo[u] | (e1 << 16) | (e2 << 24);
     } else {
       if (at <= ca.cap && nch <= ca.cap - at && ca.base + at + nch <= kMaxChunkIndex) {
@@ -453,12 +464,12 @@ __device__ void fill_slot_block(const int32_t *row, int nb, uint32_t slot0, int 
         for (uint32_t k = 0; k < nch; ++k) {
           const int c0 = a + 16 * (int)k;
           const int c1 = c0 + 16 < a + w ? c0 + 16 : a + w;
-          const uint32_t bits = boundary_bits(row, nb, jj, c0, c1);
+          const uint32_t bits = boundary_bits(row, nb, jj, c0, c1, sh);
           slots[p + k] = bits | ((uint32_t)jj << 16);
           // the bucket holding c0 + 16: past the boundaries inside, and one
           // more if a bucket starts exactly there
           jj += __popc(bits);
-          if (jj + 1 < nb && row[jj + 1] == c0 + 16) ++jj;
+          if (jj + 1 < nb && (row[jj + 1] << sh) == c0 + 16) ++jj;
         }
         word = (p & 0xffffu) | (255u << 16) | ((p >> 16) << 24);
       } else {
@@ -483,10 +494,11 @@ __device__ __forceinline__ void stage_row(int32_t *srow, const int32_t *grow, in
 
 // Slot words (and bitmap words) of a row with nb buckets, blocks x, x +
 // gridDim.x, ... of kSlotsPerBlock slots; grow[0..nb] is the row (grow[0] =
-// 0, grow[nb] = 65536), shift the row's slot width log2.  Every thread of
-// the block must call it.
+// 0, grow[nb] << sh = 65536), shift the row's slot width log2.  Every thread
+// of the block must call it.
 __device__ void fill_row_slots(const int32_t *grow, int nb, uint32_t slot0, int shift,
-                               uint32_t *slots, const ChunkArea &ca, int32_t *srow) {
+                               uint32_t *slots, const ChunkArea &ca, int32_t *srow,
+                               uint32_t sh) {
   const int nslots = 1 << (16 - shift);
   const int w = 1 << shift;
   if ((int)blockIdx.x * kSlotsPerBlock >= nslots) return;  // (the whole block)
@@ -496,7 +508,7 @@ __device__ void fill_row_slots(const int32_t *grow, int nb, uint32_t slot0, int 
     row = srow;
   }
   for (int tb = blockIdx.x * kSlotsPerBlock; tb < nslots; tb += gridDim.x * kSlotsPerBlock)
-    fill_slot_block(row, nb, slot0, w, nslots, tb, slots, ca);
+    fill_slot_block(row, nb, slot0, w, nslots, tb, slots, ca, sh);
 }
 
 // Rebuilds a prepared table set from new CDF rows with the same lengths:
@@ -505,8 +517,8 @@ __device__ void fill_row_slots(const int32_t *grow, int nb, uint32_t slot0, int 
 // buckets.  Errors go to the blob's status word.
 __global__ void __launch_bounds__(kSlotThreads)
     refresh_kernel(const int32_t *cdfs, int Lmax, const int32_t *lengths,
-                   const int32_t *offsets, RowMeta *meta, uint32_t *buckets, uint16_t *starts,
-                   uint32_t *slots, ChunkArea ca, int32_t *status) {
+                   const int32_t *offsets, uint32_t sh, RowMeta *meta, uint32_t *buckets,
+                   uint16_t *starts, uint32_t *slots, ChunkArea ca, int32_t *status) {
   extern __shared__ int32_t srow[];
   const int r = blockIdx.y;
   const RowMeta m = meta[r * kMetaCopies];
@@ -517,7 +529,8 @@ __global__ void __launch_bounds__(kSlotThreads)
   }
   const int32_t *row = cdfs + (size_t)r * (size_t)Lmax;
   const int nb = len - 1;
-  if (row[0] != 0 || row[len - 1] != (int32_t)kTotal) {
+  const int32_t top = (int32_t)(kTotal >> sh);
+  if (row[0] != 0 || row[len - 1] != top) {
     if (threadIdx.x == 0 && blockIdx.x == 0) report(status, RANS_ERR_TABLE, r);
     return;
   }
@@ -530,30 +543,31 @@ __global__ void __launch_bounds__(kSlotThreads)
     if (threadIdx.x < kMetaCopies) meta[r * kMetaCopies + threadIdx.x].offset = offsets[r];
     for (int j = threadIdx.x; j < nb; j += blockDim.x) {
       const int32_t a = prow[j], b = prow[j + 1];
-      if (!(b > a) || a < 0 || b > (int32_t)kTotal) {
+      if (!(b > a) || a < 0 || b > top) {
         report(status, RANS_ERR_TABLE, r);
         continue;
       }
-      buckets[m.bucket_base + j] = (uint32_t)(a & 0xffff) | ((uint32_t)(b - a - 1) << 16);
+      buckets[m.bucket_base + j] = bucket_word(a, b, sh);
     }
-    for (int j = threadIdx.x; j < len; j += blockDim.x) starts[m.bucket_base + j] = (uint16_t)prow[j];
+    for (int j = threadIdx.x; j < len; j += blockDim.x)
+      starts[m.bucket_base + j] = (uint16_t)(prow[j] << sh);
     __syncthreads();  // the staged row is staged again below
   }
-  fill_row_slots(row, nb, slot_base(m.slot), (int)slot_shift(m.slot), slots, ca, srow);
+  fill_row_slots(row, nb, slot_base(m.slot), (int)slot_shift(m.slot), slots, ca, srow, sh);
 }
 
 // The slot fill of rans_tables_prepare (rows already validated by
 // pack_buckets_kernel; a malformed row only leaves its own slots undefined).
 __global__ void __launch_bounds__(kSlotThreads)
     fill_slots_kernel(const int32_t *cdfs, int Lmax, const RowMeta *meta,
-                      const int32_t *lengths, uint32_t *slots, ChunkArea ca) {
+                      const int32_t *lengths, uint32_t sh, uint32_t *slots, ChunkArea ca) {
   extern __shared__ int32_t srow[];
   const int r = blockIdx.y;
   const RowMeta m = meta[r * kMetaCopies];
   const int32_t *row = cdfs + (size_t)r * (size_t)Lmax;
   const int len = lengths[r];
-  if (len < 2 || row[0] != 0 || row[len - 1] != (int32_t)kTotal) return;
-  fill_row_slots(row, len - 1, slot_base(m.slot), (int)slot_shift(m.slot), slots, ca, srow);
+  if (len < 2 || row[0] != 0 || row[len - 1] != (int32_t)(kTotal >> sh)) return;
+  fill_row_slots(row, len - 1, slot_base(m.slot), (int)slot_shift(m.slot), slots, ca, srow, sh);
 }
 
 // Row index of every scale (scale_row in rans_common.cuh).
@@ -580,16 +594,17 @@ int launch_gaussian_lengths(const float *scales, int K, double tail, int32_t *le
   return cudaGetLastError() == cudaSuccess ? RANS_OK : RANS_ERR_CUDA;
 }
 
-int launch_gaussian_rows(const float *scales, int K, double tail, int32_t *cdfs, int Lmax,
-                         int32_t *lengths, int32_t *offsets, cudaStream_t st) {
-  gaussian_rows_kernel<<<K, kRowThreads, 0, st>>>(scales, tail, cdfs, Lmax, lengths, offsets);
+int launch_gaussian_rows(const float *scales, int K, double tail, int prec, int32_t *cdfs,
+                         int Lmax, int32_t *lengths, int32_t *offsets, cudaStream_t st) {
+  gaussian_rows_kernel<<<K, kRowThreads, 0, st>>>(scales, tail, prec, cdfs, Lmax, lengths,
+                                                  offsets);
   return cudaGetLastError() == cudaSuccess ? RANS_OK : RANS_ERR_CUDA;
 }
 
 int launch_pmf_rows(const float *pmfs, int K, int stride, const int32_t *pmf_lengths,
-                    const float *tail, int32_t *cdfs, int Lmax, int32_t *lengths,
+                    const float *tail, int prec, int32_t *cdfs, int Lmax, int32_t *lengths,
                     cudaStream_t st) {
-  pmf_rows_kernel<<<K, kRowThreads, 0, st>>>(pmfs, stride, pmf_lengths, tail, cdfs, Lmax,
+  pmf_rows_kernel<<<K, kRowThreads, 0, st>>>(pmfs, stride, pmf_lengths, tail, prec, cdfs, Lmax,
                                               lengths);
   return cudaGetLastError() == cudaSuccess ? RANS_OK : RANS_ERR_CUDA;
 }
@@ -628,7 +643,8 @@ int refresh_tables(const int32_t *cdfs, int K, int Lmax, const int32_t *lengths,
   // (2^kMaxQ slots); blocks past a smaller row's slots return at once
   dim3 grid((unsigned)((1 << kMaxQ) / kSlotsPerBlock), (unsigned)K);
   refresh_kernel<<<grid, kSlotThreads, kSlotSmemBytes, st>>>(
-      cdfs, Lmax, lengths, offsets, dmeta, dbuckets, dstarts, dslots, ca, status);
+      cdfs, Lmax, lengths, offsets, (uint32_t)(kPrec - t.precision), dmeta, dbuckets, dstarts,
+      dslots, ca, status);
   return cudaGetLastError() == cudaSuccess ? RANS_OK : RANS_ERR_CUDA;
 }
 
@@ -646,8 +662,9 @@ uint64_t tables_bytes_bound(int K, int Lmax) {
 }
 
 int prepare_tables(const int32_t *cdfs, int K, int Lmax, const int32_t *lengths,
-                   const int32_t *offsets, void *blob, uint64_t blob_bytes, rans_tables *out,
-                   cudaStream_t st) {
+                   const int32_t *offsets, int prec, void *blob, uint64_t blob_bytes,
+                   rans_tables *out, cudaStream_t st) {
+  const uint32_t sh = (uint32_t)(kPrec - prec);
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return RANS_ERR_CUDA;
   if (K > 65535) return RANS_ERR_ARG;  // one grid row per table row below
@@ -740,7 +757,8 @@ int prepare_tables(const int32_t *cdfs, int K, int Lmax, const int32_t *lengths,
       cudaStreamSynchronize(st) != cudaSuccess)
     return RANS_ERR_CUDA;
   if (cudaMemsetAsync(dstarts, 0, start_bytes, st) != cudaSuccess) return RANS_ERR_CUDA;
-  pack_buckets_kernel<<<K, 256, 0, st>>>(cdfs, Lmax, dmeta, lengths, dbuckets, dstarts, status);
+  pack_buckets_kernel<<<K, 256, 0, st>>>(cdfs, Lmax, dmeta, lengths, sh, dbuckets, dstarts,
+                                         status);
   int maxslots = 0;
   for (int r = 0; r < K; ++r) maxslots = maxslots > (1 << q[r]) ? maxslots : (1 << q[r]);
   dim3 grid((maxslots + kSlotsPerBlock - 1) / kSlotsPerBlock, K);
@@ -749,7 +767,7 @@ int prepare_tables(const int32_t *cdfs, int K, int Lmax, const int32_t *lengths,
   ca.cap = (uint32_t)(slot_bytes / 4 - sbase);
   ca.used = reinterpret_cast<uint32_t *>(b) + kChunkUsedWord;
   ca.search = reinterpret_cast<uint32_t *>(b) + kSearchFlagWord;
-  fill_slots_kernel<<<grid, kSlotThreads, kSlotSmemBytes, st>>>(cdfs, Lmax, dmeta, lengths,
+  fill_slots_kernel<<<grid, kSlotThreads, kSlotSmemBytes, st>>>(cdfs, Lmax, dmeta, lengths, sh,
                                                                  dslots, ca);
   if (cudaGetLastError() != cudaSuccess) return RANS_ERR_CUDA;
   StatusWord sw;
@@ -771,6 +789,7 @@ int prepare_tables(const int32_t *cdfs, int K, int Lmax, const int32_t *lengths,
   out->enc_in_smem = enc_smem ? 1 : 0;
   out->dec_in_smem = dec_smem ? 1 : 0;
   out->device = dev;
+  out->precision = prec;
   return RANS_OK;
 }
 

@@ -1,6 +1,7 @@
 """Runs one workload through the oracle and through librans_b200 (C ABI) so
 tests can compare them.  Both sides code the same seeded arrays; the GPU
-side never feeds the oracle."""
+side never feeds the oracle.  A workload dict may name a coder format
+("fmt": "rans64" | "rans32_16") and the rows' "precision"."""
 import numpy as np
 import torch
 
@@ -8,35 +9,46 @@ import oracle as O
 import rans_entropy_coding_b200 as rb
 
 
+def fmt_of(w):
+    return w.get("fmt", "rans64")
+
+
+def precision_of(w):
+    return w.get("precision", 16 if fmt_of(w) == "rans64" else 15)
+
+
 def oracle_tables(w):
+    p = precision_of(w)
     if "scales" in w:
-        c, l, o = O.build_cdfs_from_scales(w["scales"], w["tail_mass"])
+        c, l, o = O.build_cdfs_from_scales(w["scales"], w["tail_mass"], precision=p)
     else:
-        c, l = O.build_cdfs_from_pmfs(w["pmfs"], w["pmf_lengths"], w["tail"])
+        c, l = O.build_cdfs_from_pmfs(w["pmfs"], w["pmf_lengths"], w["tail"], precision=p)
         o = np.asarray(w["offsets"], dtype=np.int32)
     return c, l, o
 
 
 def gpu_rows(w, dev="cuda"):
     """CDF rows built on the GPU: (cdfs, lengths, offsets) CUDA tensors."""
+    p = precision_of(w)
     if "scales" in w:
         return rb.Tables.build_from_scales(torch.from_numpy(np.asarray(w["scales"])).to(dev),
-                                           w["tail_mass"])
+                                           w["tail_mass"], precision=p)
     cdfs, lengths = rb.Tables.build_from_pmfs(
         torch.from_numpy(np.ascontiguousarray(w["pmfs"])).to(dev),
         torch.from_numpy(np.asarray(w["pmf_lengths"], np.int32)).to(dev),
-        torch.from_numpy(np.asarray(w["tail"], np.float32)).to(dev))
+        torch.from_numpy(np.asarray(w["tail"], np.float32)).to(dev), precision=p)
     return cdfs, lengths, torch.from_numpy(np.asarray(w["offsets"], np.int32)).to(dev)
 
 
-def tables_from_numpy(c, l, o, dev="cuda"):
+def tables_from_numpy(c, l, o, dev="cuda", precision=16):
     return rb.Tables(torch.from_numpy(np.ascontiguousarray(c)).to(dev),
                      torch.from_numpy(np.ascontiguousarray(l)).to(dev),
-                     torch.from_numpy(np.ascontiguousarray(o)).to(dev))
+                     torch.from_numpy(np.ascontiguousarray(o)).to(dev), precision=precision)
 
 
 def chunking_of(w, dev="cuda"):
-    return rb.Chunking.from_spec(w["chunking"], w["W"], w["index_block"], device=dev)
+    return rb.Chunking.from_spec(w["chunking"], w["W"], w["index_block"], device=dev,
+                                 fmt=fmt_of(w))
 
 
 def gpu_encode_decode(w, tables, dev="cuda", expect_ok=True):
@@ -61,4 +73,5 @@ def gpu_encode_decode(w, tables, dev="cuda", expect_ok=True):
 def oracle_encode(w, c, l, o, streams=None):
     sym = np.asarray(w["symbols"]).reshape(-1)
     return O.encode_with_indexes(sym, w["indexes"], c, l, o, w["chunking"], W=w["W"],
-                                 index_block=w["index_block"], streams=streams)
+                                 index_block=w["index_block"], streams=streams, fmt=fmt_of(w),
+                                 precision=precision_of(w))

@@ -206,3 +206,27 @@ def sweep(log2_n=28, seed=4000, n_streams=None, block=4096, n_rows=16):
                 tail=np.zeros(n_rows, dtype=np.float32),
                 offsets=np.zeros(n_rows, dtype=np.int32),
                 chunking=dict(kind="contig", n_streams=n_streams), W=32, index_block=block)
+
+
+def r16_rows(seed=7000, n_streams=1024, per_stream=4096, n_dists=256, alphabet=255):
+    """The rans32_16 benchmark shape of "torch_ans 0.3.0" (Performance
+    Tuning, GPU table): n_streams streams of per_stream int32 symbols coded
+    32-way, alphabet 255 with bypass coding (cdf rows of 257 entries),
+    n_dists distributions.  The page gives no distributions; here each row's
+    pmf is a Dirichlet(1) draw over the alphabet (about 7.4 bits of entropy),
+    every symbol takes a row uniformly at random and is drawn from it, and the
+    tail mass is 0 (the escape bucket gets its unit by stealing)."""
+    rng = _rng(seed)
+    pmfs = rng.gamma(1.0, size=(n_dists, alphabet))
+    pmfs = (pmfs / pmfs.sum(axis=1, keepdims=True)).astype(np.float32)
+    n = n_streams * per_stream
+    idx = rng.integers(0, n_dists, size=n).astype(np.int32)
+    cum = [np.cumsum(pmfs[r].astype(np.float64)) for r in range(n_dists)]
+    sym = _sample_from_pmfs(rng, cum, idx).astype(np.int32)
+    return dict(name="r16", symbols=sym, indexes=idx, pmfs=pmfs,
+                pmf_lengths=np.full(n_dists, alphabet, dtype=np.int32),
+                tail=np.zeros(n_dists, dtype=np.float32),
+                offsets=np.zeros(n_dists, dtype=np.int32),
+                chunking=dict(kind="contig", n_streams=n_streams), W=32, index_block=1,
+                fmt="rans32_16", precision=15)
+
