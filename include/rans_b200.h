@@ -141,8 +141,11 @@ typedef struct rans_tables {
     int64_t n_buckets;      /* all rows' buckets */
     int64_t n_slots;        /* decode lookup slots */
     uint32_t meta_bytes, bucket_bytes, start_bytes, slot_bytes;  /* sections (16-B padded) */
-    int32_t enc_in_smem;    /* 1: encode stages meta + buckets in shared memory */
-    int32_t dec_in_smem;    /* 1: decode stages meta + starts + slots */
+    int32_t enc_in_smem;    /* encode table mode: 1 stages meta + buckets in shared
+                               memory, 2 meta + 16-bit starts, 0 reads global */
+    int32_t dec_in_smem;    /* decode table mode: 1 stages meta + starts + slots,
+                               2 meta + starts (a binary search per lookup), 0 reads
+                               global */
     int32_t device;         /* CUDA device the blob lives on */
     int32_t precision;      /* the rows sum to 2^precision */
 } rans_tables;

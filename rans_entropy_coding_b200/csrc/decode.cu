@@ -113,6 +113,23 @@ __device__ __forceinline__ uint32_t lookup(uint32_t cum, const RowMeta &m, const
   return min(sym, m.maxv);
 }
 
+// The bucket holding cum when the row's slots are not on chip: the last of
+// the row's maxv + 1 buckets whose start is <= cum, by a binary search over
+// its 16-bit starts in power-of-two steps (every probe is in the row; the
+// row end is never read).
+__device__ __forceinline__ uint32_t search_row(uint32_t cum, const RowMeta &m,
+                                               const uint16_t *starts) {
+  const uint32_t last = m.maxv;  // buckets 0 .. maxv
+  const uint16_t *row = starts + m.bucket_base;
+  uint32_t j = 0;
+  for (uint32_t step = last ? 1u << (31 - __clz(last)) : 0u; step != 0; step >>= 1) {
+    const uint32_t t = j + step;
+    const uint32_t v = row[t <= last ? t : last];
+    j = (t <= last && v <= cum) ? t : j;
+  }
+  return j;
+}
+
 template <class F>
 struct EscapeResult {
   typename F::State x;
@@ -229,7 +246,7 @@ __device__ __forceinline__ void load_window(WarpDec<F> &st, const typename F::Wo
 // group's row metadata, read one group ahead.  The refill is taken as if no
 // lane escaped; the escape ballot, issued beside it, sends the group down
 // the lane-serial path from the state after the symbol op.
-template <class F, typename SymT, bool FULL, bool SEARCH>
+template <class F, typename SymT, bool FULL, bool SEARCH, bool ROWS>
 __device__ __forceinline__ void dec_group(WarpDec<F> &st, const RowMeta &m,
                                           const uint16_t *starts, const uint32_t *slots,
                                           bool active, SymT *dst, const typename F::Word *words,
@@ -237,7 +254,8 @@ __device__ __forceinline__ void dec_group(WarpDec<F> &st, const RowMeta &m,
   const int lane = threadIdx.x & 31;
   if (FULL) active = true;
   const uint32_t cum = F::cum16(st.x, sh);
-  const uint32_t sym = lookup<SEARCH, true>(cum, m, starts, slots, active);
+  const uint32_t sym =
+      ROWS ? search_row(cum, m, starts) : lookup<SEARCH, true>(cum, m, starts, slots, active);
   const uint32_t start = starts[m.bucket_base + sym];
   const uint32_t freq = width_of(start, starts[m.bucket_base + sym + 1]);
   typename F::State x = F::dec_step(st.x, cum, start, freq, sh);
@@ -282,7 +300,7 @@ __device__ __forceinline__ void dec_group(WarpDec<F> &st, const RowMeta &m,
 // SymT = float: the ring holds scales, each group's row is its scale's table
 // row, and the output is float(symbol) + mean, the means read one group
 // ahead with plain loads.
-template <class F, typename SymT, bool IB0, bool WIDE, bool SEARCH>
+template <class F, typename SymT, bool IB0, bool WIDE, bool SEARCH, bool ROWS>
 __device__ __forceinline__ void decode_stream_w32(const DecCtx &c, const StreamDesc &d,
                                                   const RowMeta *meta, const uint16_t *starts,
                                                   const uint32_t *slots, uint32_t *stg,
@@ -356,15 +374,15 @@ __device__ __forceinline__ void decode_stream_w32(const DecCtx &c, const StreamD
     const RowMeta mn = meta_of(stg[((g + 1) & (kS - 1)) * 32 + lane]);
     const float mean_nn = kFlt ? mean_at(g + 2, pm.rel) : 0.0f;
     if (kFlt) pm.fwd(32);
-    dec_group<F, SymT, true, SEARCH>(st, m, starts, slots, true, out_s + pc.rel, words, nw, sh,
-                                     mean);
+    dec_group<F, SymT, true, SEARCH, ROWS>(st, m, starts, slots, true, out_s + pc.rel, words,
+                                           nw, sh, mean);
     pc.fwd(32);
     m = mn;
     mean = mean_n;
     mean_n = mean_nn;
   }
-  dec_group<F, SymT, false, SEARCH>(st, m, starts, slots, lane < n - (G - 1) * 32,
-                                    out_s + pc.rel, words, nw, sh, mean);
+  dec_group<F, SymT, false, SEARCH, ROWS>(st, m, starts, slots, lane < n - (G - 1) * 32,
+                                          out_s + pc.rel, words, nw, sh, mean);
   cp_async_wait<0>();
   if (__any_sync(kFull, st.rmax > kmax)) {
     if (lane == 0) report(c.status, RANS_ERR_INDEX, s);
@@ -374,7 +392,7 @@ __device__ __forceinline__ void decode_stream_w32(const DecCtx &c, const StreamD
   if (!__all_sync(kFull, ok) && lane == 0) report(c.status, RANS_ERR_CORRUPT, s);
 }
 
-template <class F, typename SymT, bool IB0, bool SEARCH>
+template <class F, typename SymT, bool IB0, bool SEARCH, bool ROWS>
 __device__ __forceinline__ void decode_stream_w32_entry(const DecCtx &c, const RowMeta *meta,
                                                         const uint16_t *buckets,
                                                         const uint32_t *slots, uint32_t *stg,
@@ -401,14 +419,14 @@ __device__ __forceinline__ void decode_stream_w32_entry(const DecCtx &c, const R
     return;
   }
   if (d.t.ww >= 32)
-    decode_stream_w32<F, SymT, IB0, true, SEARCH>(c, d, meta, buckets, slots, stg, s, words, nw,
-                                                  stab);
+    decode_stream_w32<F, SymT, IB0, true, SEARCH, ROWS>(c, d, meta, buckets, slots, stg, s,
+                                                        words, nw, stab);
   else
-    decode_stream_w32<F, SymT, IB0, false, SEARCH>(c, d, meta, buckets, slots, stg, s, words,
-                                                   nw, stab);
+    decode_stream_w32<F, SymT, IB0, false, SEARCH, ROWS>(c, d, meta, buckets, slots, stg, s,
+                                                         words, nw, stab);
 }
 
-template <class F, typename SymT>
+template <class F, typename SymT, bool ROWS>
 __device__ void decode_stream_w1(const DecCtx &c, const RowMeta *meta, const uint16_t *buckets,
                                  const uint32_t *slots, int64_t s, const float *stab) {
   using State = typename F::State;
@@ -465,7 +483,8 @@ __device__ void decode_stream_w1(const DecCtx &c, const RowMeta *meta, const uin
     }
     const RowMeta m = row_meta(meta, (uint32_t)r);
     const uint32_t cum = F::cum16(x, sh);
-    const uint32_t sym = lookup<true, false>(cum, m, buckets, slots, true);
+    const uint32_t sym =
+        ROWS ? search_row(cum, m, buckets) : lookup<true, false>(cum, m, buckets, slots, true);
     const uint32_t start = buckets[m.bucket_base + sym];
     const uint32_t freq = width_of(start, buckets[m.bucket_base + sym + 1]);
     x = F::dec_step(x, cum, start, freq, sh);
@@ -503,19 +522,30 @@ __device__ void decode_stream_w1(const DecCtx &c, const RowMeta *meta, const uin
   if (bad || x != F::kLow || pw != nw) report(c.status, RANS_ERR_CORRUPT, s);
 }
 
-template <class F, int W, typename SymT, bool SMEM, bool IB0>
+// Shared-memory bytes of a table mode: 0 reads the tables from global
+// memory, 1 stages the row metadata, starts and lookup slots, 2 (tables whose
+// slots do not fit) the row metadata and starts, the lookup then searching
+// each row's starts.
+__host__ __device__ inline uint32_t dec_table_bytes(int mode, const DecCtx &c) {
+  return mode == 1 ? c.meta_bytes + c.start_bytes + c.slot_bytes
+                   : (mode == 2 ? c.meta_bytes + c.start_bytes : 0u);
+}
+
+template <class F, int W, typename SymT, int MODE, bool IB0>
 __global__ void __launch_bounds__(W == 32 ? kDecMaxThreads32 : kDecThreads1)
     decode_kernel(DecCtx c) {
+  constexpr bool ROWS = MODE == 2;
   extern __shared__ __align__(16) unsigned char smem[];
   __shared__ uint64_t bar;
   const RowMeta *meta;
   const uint16_t *buckets;  // 16-bit starts
   const uint32_t *slots;
   const char *gb = c.blob + kHeaderBytes;
-  if (SMEM) {
-    // [meta][starts][slots] in shared memory, from two ranges of the blob
+  if (MODE != 0) {
+    // [meta][starts]([slots]) in shared memory, from two ranges of the blob
     if (!stage_to_smem(smem, gb, c.meta_bytes, &bar, c.status, smem + c.meta_bytes,
-                       gb + c.meta_bytes + c.bucket_bytes, c.start_bytes + c.slot_bytes))
+                       gb + c.meta_bytes + c.bucket_bytes,
+                       c.start_bytes + (MODE == 1 ? c.slot_bytes : 0u)))
       return;
     meta = reinterpret_cast<const RowMeta *>(smem);
     buckets = reinterpret_cast<const uint16_t *>(smem + c.meta_bytes);
@@ -525,43 +555,42 @@ __global__ void __launch_bounds__(W == 32 ? kDecMaxThreads32 : kDecThreads1)
     buckets = reinterpret_cast<const uint16_t *>(gb + c.meta_bytes + c.bucket_bytes);
     slots = reinterpret_cast<const uint32_t *>(gb + c.meta_bytes + c.bucket_bytes + c.start_bytes);
   }
+  const uint32_t tab = dec_table_bytes(MODE, c);
   // float values: the scale table, copied after the stage rings when it fits
   const float *stab = c.stab;
   if (std::is_same<SymT, float>::value && c.stab_smem) {
     float *t = reinterpret_cast<float *>(
-        smem + (SMEM ? c.meta_bytes + c.start_bytes + c.slot_bytes : 0) +
-        (W == 32 ? (blockDim.x >> 5) * (uint32_t)(kDecStage * 32 * 4) : 0));
+        smem + tab + (W == 32 ? (blockDim.x >> 5) * (uint32_t)(kDecStage * 32 * 4) : 0));
     for (int i = threadIdx.x; i < c.K; i += blockDim.x) t[i] = c.stab[i];
     __syncthreads();
     stab = t;
   }
   if (W == 32) {
     const int warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
-    uint32_t *stg = reinterpret_cast<uint32_t *>(
-                        smem + (SMEM ? c.meta_bytes + c.start_bytes + c.slot_bytes : 0)) +
-                    warp * kDecStage * 32;
+    uint32_t *stg = reinterpret_cast<uint32_t *>(smem + tab) + warp * kDecStage * 32;
     // slots that ran out of bitmap room (flagged in the blob header) search
-    const bool search = reinterpret_cast<const uint32_t *>(c.blob)[kSearchFlagWord] != 0;
+    const bool search =
+        !ROWS && reinterpret_cast<const uint32_t *>(c.blob)[kSearchFlagWord] != 0;
     for (int64_t k = blockIdx.x + (int64_t)gridDim.x * warp; k < c.g.S;
          k += (int64_t)gridDim.x * nw) {
       if (search)
-        decode_stream_w32_entry<F, SymT, IB0, true>(c, meta, buckets, slots, stg,
-                                                    stream_of(c.g, k), stab);
+        decode_stream_w32_entry<F, SymT, IB0, true, ROWS>(c, meta, buckets, slots, stg,
+                                                          stream_of(c.g, k), stab);
       else
-        decode_stream_w32_entry<F, SymT, IB0, false>(c, meta, buckets, slots, stg,
-                                                     stream_of(c.g, k), stab);
+        decode_stream_w32_entry<F, SymT, IB0, false, ROWS>(c, meta, buckets, slots, stg,
+                                                           stream_of(c.g, k), stab);
     }
   } else {
     for (int64_t k = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; k < c.g.S;
          k += (int64_t)gridDim.x * blockDim.x)
-      decode_stream_w1<F, SymT>(c, meta, buckets, slots, stream_of(c.g, k), stab);
+      decode_stream_w1<F, SymT, ROWS>(c, meta, buckets, slots, stream_of(c.g, k), stab);
   }
 }
 
-template <class F, int W, typename SymT, bool SMEM, bool IB0>
+template <class F, int W, typename SymT, int MODE, bool IB0>
 int launch_decode_t(const DecCtx &c, cudaStream_t st) {
-  auto kern = decode_kernel<F, W, SymT, SMEM, IB0>;
-  const uint32_t tab = SMEM ? c.meta_bytes + c.start_bytes + c.slot_bytes : 0;
+  auto kern = decode_kernel<F, W, SymT, MODE, IB0>;
+  const uint32_t tab = dec_table_bytes(MODE, c);
   const uint32_t per_warp = W == 32 ? kDecStage * 32 * 4 : 0;
   int dev = 0;
   cudaGetDevice(&dev);
@@ -616,26 +645,29 @@ int launch_decode_t(const DecCtx &c, cudaStream_t st) {
   return cudaGetLastError() == cudaSuccess ? RANS_OK : RANS_ERR_CUDA;
 }
 
+template <class F, int W, typename SymT, int MODE>
+int launch_decode_m(const DecCtx &c, cudaStream_t st) {
+  return c.g.ib_shift == 0 ? launch_decode_t<F, W, SymT, MODE, true>(c, st)
+                           : launch_decode_t<F, W, SymT, MODE, false>(c, st);
+}
+
 template <class F, int W, typename SymT>
-int launch_decode_w(const DecCtx &c, bool smem, cudaStream_t st) {
-  const bool ib0 = c.g.ib_shift == 0;
-  if (smem)
-    return ib0 ? launch_decode_t<F, W, SymT, true, true>(c, st)
-               : launch_decode_t<F, W, SymT, true, false>(c, st);
-  return ib0 ? launch_decode_t<F, W, SymT, false, true>(c, st)
-             : launch_decode_t<F, W, SymT, false, false>(c, st);
+int launch_decode_w(const DecCtx &c, int mode, cudaStream_t st) {
+  if (mode == 1) return launch_decode_m<F, W, SymT, 1>(c, st);
+  if (mode == 2) return launch_decode_m<F, W, SymT, 2>(c, st);
+  return launch_decode_m<F, W, SymT, 0>(c, st);
 }
 
 template <class F, typename SymT>
-int launch_decode_f(const DecCtx &c, bool smem, cudaStream_t st) {
-  return c.g.W == 32 ? launch_decode_w<F, 32, SymT>(c, smem, st)
-                     : launch_decode_w<F, 1, SymT>(c, smem, st);
+int launch_decode_f(const DecCtx &c, int mode, cudaStream_t st) {
+  return c.g.W == 32 ? launch_decode_w<F, 32, SymT>(c, mode, st)
+                     : launch_decode_w<F, 1, SymT>(c, mode, st);
 }
 
 template <typename SymT>
-int launch_decode_s(const DecCtx &c, bool smem, cudaStream_t st) {
-  return c.g.fmt == RANS_FMT_RANS32_16 ? launch_decode_f<Rans32, SymT>(c, smem, st)
-                                       : launch_decode_f<Rans64, SymT>(c, smem, st);
+int launch_decode_s(const DecCtx &c, int mode, cudaStream_t st) {
+  return c.g.fmt == RANS_FMT_RANS32_16 ? launch_decode_f<Rans32, SymT>(c, mode, st)
+                                       : launch_decode_f<Rans64, SymT>(c, mode, st);
 }
 
 }  // namespace
@@ -663,10 +695,9 @@ int launch_decode_float(const uint8_t *in, uint64_t in_bytes, const uint64_t *of
   c.fmean = means;
   c.stab = scale_table;
   c.bound = scale_bound;
-  const bool smem = t.dec_in_smem != 0;
   // float values decode the 64-bit format only (the caller checks)
-  return g.W == 32 ? launch_decode_w<Rans64, 32, float>(c, smem, st)
-                   : launch_decode_w<Rans64, 1, float>(c, smem, st);
+  return g.W == 32 ? launch_decode_w<Rans64, 32, float>(c, t.dec_in_smem, st)
+                   : launch_decode_w<Rans64, 1, float>(c, t.dec_in_smem, st);
 }
 
 int launch_decode(const uint8_t *in, uint64_t in_bytes, const uint64_t *offsets,
@@ -690,11 +721,11 @@ int launch_decode(const uint8_t *in, uint64_t in_bytes, const uint64_t *offsets,
   c.fscale = c.fmean = c.stab = nullptr;
   c.bound = 0.0f;
   c.stab_smem = 0;
-  const bool smem = t.dec_in_smem != 0;
+  const int mode = t.dec_in_smem;
   switch (sym_dtype) {
-    case RANS_SYM_INT32: return launch_decode_s<int32_t>(c, smem, st);
-    case RANS_SYM_UINT8: return launch_decode_s<uint8_t>(c, smem, st);
-    case RANS_SYM_INT16: return launch_decode_s<int16_t>(c, smem, st);
+    case RANS_SYM_INT32: return launch_decode_s<int32_t>(c, mode, st);
+    case RANS_SYM_UINT8: return launch_decode_s<uint8_t>(c, mode, st);
+    case RANS_SYM_INT16: return launch_decode_s<int16_t>(c, mode, st);
     default: return RANS_ERR_ARG;
   }
 }

@@ -51,7 +51,7 @@ struct EncCtx {
   int32_t stab_smem; // 1: the kernel copies the scale table into shared memory
   int32_t K;
   uint32_t sh;       // 16 - precision of the rows (Rans32; 0 for Rans64)
-  uint32_t meta_bytes, bucket_bytes;
+  uint32_t meta_bytes, bucket_bytes, start_bytes;
   const char *blob;
   Geom g;
   char *scratch;
@@ -59,8 +59,21 @@ struct EncCtx {
   int32_t *status;
 };
 
+// Table modes of the encoder: 32-bit bucket words (start | (width - 1) <<
+// 16), or, for tables too large to stage those, the 16-bit starts (a bucket's
+// width is the distance to the next start).  bucket_word<ST> reads bucket i
+// of the table `tab` in either form.
+template <bool ST>
+__device__ __forceinline__ uint32_t bucket_word(const uint32_t *tab, uint32_t i) {
+  if (!ST) return tab[i];
+  const uint16_t *starts = reinterpret_cast<const uint16_t *>(tab);
+  const uint32_t a = starts[i], b = starts[i + 1];
+  return a | (((b - a - 1u) & 0xffffu) << 16);
+}
+
 // Maps symbol s through row m: bucket start / width, and the escape's raw
 // value (zig-zag: below the range 2|v| - 1, above it 2 (v - maxv)).
+template <bool ST>
 __device__ __forceinline__ void map_symbol(int32_t s, const RowMeta &m, const uint32_t *buckets,
                                            uint32_t &start, uint32_t &freq, uint64_t &raw,
                                            bool &esc) {
@@ -75,7 +88,7 @@ __device__ __forceinline__ void map_symbol(int32_t s, const RowMeta &m, const ui
     v = maxv;
   }
   esc = (v == maxv);
-  const uint32_t e = buckets[m.bucket_base + (uint32_t)v];
+  const uint32_t e = bucket_word<ST>(buckets, m.bucket_base + (uint32_t)v);
   start = bucket_start(e);
   freq = bucket_freq(e);
 }
@@ -175,13 +188,14 @@ struct EncBucket {
 };
 
 // value mapping: in range iff 0 <= s - offset < maxv (64-bit, exact)
+template <bool ST>
 __device__ __forceinline__ EncBucket enc_bucket(int32_t sv, const RowMeta &m,
                                                 const uint32_t *buckets) {
   EncBucket b;
   b.v = (int64_t)sv - (int64_t)m.offset;
   b.maxv = m.maxv;
   b.in_range = (uint64_t)b.v < (uint64_t)m.maxv;
-  b.e = buckets[m.bucket_base + (b.in_range ? (uint32_t)b.v : m.maxv)];
+  b.e = bucket_word<ST>(buckets, m.bucket_base + (b.in_range ? (uint32_t)b.v : m.maxv));
   return b;
 }
 
@@ -239,7 +253,7 @@ __device__ __forceinline__ void enc_group_escape(WarpEnc<F> &st, typename F::Sta
 // FLT: the stream's inputs are float latents: an 8-group ring holds scales
 // (as the row source), y and the means; each group's row is its scale's
 // table row and its symbol rint(y - mean).
-template <class F, typename SymT, bool IB0, bool WIDE, bool FLT>
+template <class F, typename SymT, bool IB0, bool WIDE, bool FLT, bool ST>
 __device__ __forceinline__ void encode_stream_w32(const EncCtx &c, const StreamDesc &d,
                                                   const RowMeta *meta, const uint32_t *buckets,
                                                   uint32_t *stg, int64_t s, const float *stab) {
@@ -336,7 +350,7 @@ __device__ __forceinline__ void encode_stream_w32(const EncCtx &c, const StreamD
     pn.back(32);
   }
   EncLook L =
-      enc_look<F>(enc_bucket(s0, meta_of(row_of(stg_idx[ring(0)])), buckets), active0, sh);
+      enc_look<F>(enc_bucket<ST>(s0, meta_of(row_of(stg_idx[ring(0)])), buckets), active0, sh);
   // group 1's symbol (FLT: its y and mean, quantised when used)
   int32_t s1 = G > 1 ? sym_of(1) : 0;
   float mean1 = FLT && G > 1 ? mean_of(1) : 0.0f;
@@ -346,7 +360,7 @@ __device__ __forceinline__ void encode_stream_w32(const EncCtx &c, const StreamD
   auto step = [&](int32_t k, bool active, auto full) {
     // group k+1's bucket (after the last group: row 0, unused)
     if (FLT) s1 = k + 1 < G ? quant(s1, mean1) : 0;
-    const EncBucket b1 = enc_bucket(s1, m1, buckets);
+    const EncBucket b1 = enc_bucket<ST>(s1, m1, buckets);
     // group k's state update
     const typename F::State x0 = st.x;
     const uint32_t c0 = st.cursor;
@@ -386,7 +400,7 @@ __device__ __forceinline__ void encode_stream_w32(const EncCtx &c, const StreamD
   if (lane == 0) c.lens[s] = sizeof(Word) * (uint64_t)(st.cursor + 64);
 }
 
-template <class F, typename SymT, bool IB0, bool FLT>
+template <class F, typename SymT, bool IB0, bool FLT, bool ST>
 __device__ __forceinline__ void encode_stream_w32_entry(const EncCtx &c, const RowMeta *meta,
                                                         const uint32_t *buckets, uint32_t *stg,
                                                         int64_t s, const float *stab) {
@@ -405,12 +419,12 @@ __device__ __forceinline__ void encode_stream_w32_entry(const EncCtx &c, const R
     return;
   }
   if (d.t.ww >= 32)
-    encode_stream_w32<F, SymT, IB0, true, FLT>(c, d, meta, buckets, stg, s, stab);
+    encode_stream_w32<F, SymT, IB0, true, FLT, ST>(c, d, meta, buckets, stg, s, stab);
   else
-    encode_stream_w32<F, SymT, IB0, false, FLT>(c, d, meta, buckets, stg, s, stab);
+    encode_stream_w32<F, SymT, IB0, false, FLT, ST>(c, d, meta, buckets, stg, s, stab);
 }
 
-template <class F, typename SymT, bool FLT>
+template <class F, typename SymT, bool FLT, bool ST>
 __device__ void encode_stream_w1(const EncCtx &c, const RowMeta *meta, const uint32_t *buckets,
                                  int64_t s, const float *stab) {
   using Word = typename F::Word;
@@ -475,7 +489,7 @@ __device__ void encode_stream_w1(const EncCtx &c, const RowMeta *meta, const uin
     uint32_t start, freq;
     uint64_t raw;
     bool esc;
-    map_symbol(sv, row_meta(meta, (uint32_t)r), buckets, start, freq, raw, esc);
+    map_symbol<ST>(sv, row_meta(meta, (uint32_t)r), buckets, start, freq, raw, esc);
     if (esc && (raw >> 60) != 0) {
       report(c.status, RANS_ERR_RANGE, s);
       return;
@@ -488,45 +502,59 @@ __device__ void encode_stream_w1(const EncCtx &c, const RowMeta *meta, const uin
   c.lens[s] = sizeof(Word) * (uint64_t)cursor;
 }
 
-template <class F, int W, typename SymT, bool SMEM, bool IB0, bool FLT>
+// Shared-memory bytes of a table mode: 0 reads the tables from global
+// memory, 1 stages the row metadata and bucket words, 2 the row metadata
+// and the 16-bit starts.
+__host__ __device__ inline uint32_t enc_table_bytes(int mode, const EncCtx &c) {
+  return mode == 1 ? c.meta_bytes + c.bucket_bytes
+                   : (mode == 2 ? c.meta_bytes + c.start_bytes : 0u);
+}
+
+template <class F, int W, typename SymT, int MODE, bool IB0, bool FLT>
 __global__ void __launch_bounds__(W == 32 ? kEncThreads32 : kEncThreads1)
     encode_kernel(EncCtx c) {
+  constexpr bool ST = MODE == 2;
   extern __shared__ __align__(16) unsigned char smem[];
   __shared__ uint64_t bar;
   const RowMeta *meta;
-  const uint32_t *buckets;
-  if (SMEM) {
-    if (!stage_to_smem(smem, c.blob + kHeaderBytes, c.meta_bytes + c.bucket_bytes, &bar,
-                       c.status))
+  const uint32_t *buckets;  // bucket words, or (ST) the 16-bit starts
+  const char *gb = c.blob + kHeaderBytes;
+  if (MODE == 1) {
+    if (!stage_to_smem(smem, gb, c.meta_bytes + c.bucket_bytes, &bar, c.status)) return;
+    meta = reinterpret_cast<const RowMeta *>(smem);
+    buckets = reinterpret_cast<const uint32_t *>(smem + c.meta_bytes);
+  } else if (MODE == 2) {
+    if (!stage_to_smem(smem, gb, c.meta_bytes, &bar, c.status, smem + c.meta_bytes,
+                       gb + c.meta_bytes + c.bucket_bytes, c.start_bytes))
       return;
     meta = reinterpret_cast<const RowMeta *>(smem);
     buckets = reinterpret_cast<const uint32_t *>(smem + c.meta_bytes);
   } else {
-    meta = reinterpret_cast<const RowMeta *>(c.blob + kHeaderBytes);
-    buckets = reinterpret_cast<const uint32_t *>(c.blob + kHeaderBytes + c.meta_bytes);
+    meta = reinterpret_cast<const RowMeta *>(gb);
+    buckets = reinterpret_cast<const uint32_t *>(gb + c.meta_bytes);
   }
+  const uint32_t tab = enc_table_bytes(MODE, c);
   // FLT: the scale table, copied after the stage rings when it fits
   const float *stab = c.stab;
   if (FLT && c.stab_smem) {
     float *t = reinterpret_cast<float *>(
-        smem + (SMEM ? c.meta_bytes + c.bucket_bytes : 0) +
-        (W == 32 ? (blockDim.x >> 5) * enc_stage_bytes_per_warp(FLT) : 0));
+        smem + tab + (W == 32 ? (blockDim.x >> 5) * enc_stage_bytes_per_warp(FLT) : 0));
     for (int i = threadIdx.x; i < c.K; i += blockDim.x) t[i] = c.stab[i];
     __syncthreads();
     stab = t;
   }
   if (W == 32) {
     const int warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
-    uint32_t *stg = reinterpret_cast<uint32_t *>(smem + (SMEM ? c.meta_bytes + c.bucket_bytes : 0)) +
+    uint32_t *stg = reinterpret_cast<uint32_t *>(smem + tab) +
                     warp * (enc_stage_bytes_per_warp(FLT) / 4);
     for (int64_t k = blockIdx.x + (int64_t)gridDim.x * warp; k < c.g.S;
          k += (int64_t)gridDim.x * nw)
-      encode_stream_w32_entry<F, SymT, IB0, FLT>(c, meta, buckets, stg, stream_of(c.g, k),
-                                                 stab);
+      encode_stream_w32_entry<F, SymT, IB0, FLT, ST>(c, meta, buckets, stg, stream_of(c.g, k),
+                                                     stab);
   } else {
     for (int64_t k = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; k < c.g.S;
          k += (int64_t)gridDim.x * blockDim.x)
-      encode_stream_w1<F, SymT, FLT>(c, meta, buckets, stream_of(c.g, k), stab);
+      encode_stream_w1<F, SymT, FLT, ST>(c, meta, buckets, stream_of(c.g, k), stab);
   }
 }
 
@@ -610,10 +638,10 @@ __global__ void debug_divide_kernel(const uint64_t *x, const uint32_t *f, int64_
   }
 }
 
-template <class F, int W, typename SymT, bool SMEM, bool IB0, bool FLT>
+template <class F, int W, typename SymT, int MODE, bool IB0, bool FLT>
 int launch_encode_t(const EncCtx &c, cudaStream_t st) {
-  auto kern = encode_kernel<F, W, SymT, SMEM, IB0, FLT>;
-  const uint32_t tab = SMEM ? c.meta_bytes + c.bucket_bytes : 0;
+  auto kern = encode_kernel<F, W, SymT, MODE, IB0, FLT>;
+  const uint32_t tab = enc_table_bytes(MODE, c);
   const uint32_t per_warp = W == 32 ? enc_stage_bytes_per_warp(FLT) : 0;
   uint32_t smem = tab;
   int dev = 0;
@@ -641,7 +669,10 @@ int launch_encode_t(const EncCtx &c, cudaStream_t st) {
     if (nblk > c.g.S) nblk = c.g.S < 1 ? 1 : c.g.S;
     int64_t warps = (c.g.S + nblk - 1) / nblk;
     if (warps > kEncMaxWarps) warps = kEncMaxWarps;
-    if (warps < 1) warps = 1;
+    // large staged tables leave room for fewer rings
+    const int64_t room = ((int64_t)lim - (int64_t)tab) / (int64_t)(per_warp ? per_warp : 1u);
+    if (warps > room) warps = room;
+    if (warps < 1) return RANS_ERR_CAPACITY;
     threads = (int)warps * 32;
     smem = tab + (uint32_t)warps * per_warp;
     int fit = 0;
@@ -669,26 +700,29 @@ int launch_encode_t(const EncCtx &c, cudaStream_t st) {
   return cudaGetLastError() == cudaSuccess ? RANS_OK : RANS_ERR_CUDA;
 }
 
+template <class F, int W, typename SymT, int MODE>
+int launch_encode_m(const EncCtx &c, cudaStream_t st) {
+  return c.g.ib_shift == 0 ? launch_encode_t<F, W, SymT, MODE, true, false>(c, st)
+                           : launch_encode_t<F, W, SymT, MODE, false, false>(c, st);
+}
+
 template <class F, int W, typename SymT>
-int launch_encode_w(const EncCtx &c, bool smem, cudaStream_t st) {
-  const bool ib0 = c.g.ib_shift == 0;
-  if (smem)
-    return ib0 ? launch_encode_t<F, W, SymT, true, true, false>(c, st)
-               : launch_encode_t<F, W, SymT, true, false, false>(c, st);
-  return ib0 ? launch_encode_t<F, W, SymT, false, true, false>(c, st)
-             : launch_encode_t<F, W, SymT, false, false, false>(c, st);
+int launch_encode_w(const EncCtx &c, int mode, cudaStream_t st) {
+  if (mode == 1) return launch_encode_m<F, W, SymT, 1>(c, st);
+  if (mode == 2) return launch_encode_m<F, W, SymT, 2>(c, st);
+  return launch_encode_m<F, W, SymT, 0>(c, st);
 }
 
 template <class F, typename SymT>
-int launch_encode_f(const EncCtx &c, bool smem, cudaStream_t st) {
-  return c.g.W == 32 ? launch_encode_w<F, 32, SymT>(c, smem, st)
-                     : launch_encode_w<F, 1, SymT>(c, smem, st);
+int launch_encode_f(const EncCtx &c, int mode, cudaStream_t st) {
+  return c.g.W == 32 ? launch_encode_w<F, 32, SymT>(c, mode, st)
+                     : launch_encode_w<F, 1, SymT>(c, mode, st);
 }
 
 template <typename SymT>
-int launch_encode_s(const EncCtx &c, bool smem, cudaStream_t st) {
-  return c.g.fmt == RANS_FMT_RANS32_16 ? launch_encode_f<Rans32, SymT>(c, smem, st)
-                                       : launch_encode_f<Rans64, SymT>(c, smem, st);
+int launch_encode_s(const EncCtx &c, int mode, cudaStream_t st) {
+  return c.g.fmt == RANS_FMT_RANS32_16 ? launch_encode_f<Rans32, SymT>(c, mode, st)
+                                       : launch_encode_f<Rans64, SymT>(c, mode, st);
 }
 
 }  // namespace
@@ -703,6 +737,7 @@ int launch_encode(const void *symbols, int sym_dtype, const int32_t *indexes,
   c.sh = (uint32_t)(kPrec - t.precision);
   c.meta_bytes = t.meta_bytes;
   c.bucket_bytes = t.bucket_bytes;
+  c.start_bytes = t.start_bytes;
   c.blob = reinterpret_cast<const char *>(t.blob);
   c.g = g;
   c.scratch = scratch;
@@ -711,11 +746,11 @@ int launch_encode(const void *symbols, int sym_dtype, const int32_t *indexes,
   c.fy = c.fmean = c.fscale = c.stab = nullptr;
   c.bound = 0.0f;
   c.stab_smem = 0;
-  const bool smem = t.enc_in_smem != 0;
+  const int mode = t.enc_in_smem;
   switch (sym_dtype) {
-    case RANS_SYM_INT32: return launch_encode_s<int32_t>(c, smem, st);
-    case RANS_SYM_UINT8: return launch_encode_s<uint8_t>(c, smem, st);
-    case RANS_SYM_INT16: return launch_encode_s<int16_t>(c, smem, st);
+    case RANS_SYM_INT32: return launch_encode_s<int32_t>(c, mode, st);
+    case RANS_SYM_UINT8: return launch_encode_s<uint8_t>(c, mode, st);
+    case RANS_SYM_INT16: return launch_encode_s<int16_t>(c, mode, st);
     default: return RANS_ERR_ARG;
   }
 }
@@ -736,18 +771,21 @@ int launch_encode_float(const float *y, const float *means, const float *scales,
   c.sh = 0;
   c.meta_bytes = t.meta_bytes;
   c.bucket_bytes = t.bucket_bytes;
+  c.start_bytes = t.start_bytes;
   c.blob = reinterpret_cast<const char *>(t.blob);
   c.g = g;
   c.scratch = scratch;
   c.lens = lens;
   c.status = status;
-  const bool smem = t.enc_in_smem != 0;
-  // float latents code the 64-bit format only (the caller checks)
+  // float latents code the 64-bit format only (the caller checks); tables
+  // too large for the bucket words in shared memory are read from global
+  // memory here
+  const bool smem = t.enc_in_smem == 1;
   if (g.W == 32)
-    return smem ? launch_encode_t<Rans64, 32, int32_t, true, true, true>(c, st)
-                : launch_encode_t<Rans64, 32, int32_t, false, true, true>(c, st);
-  return smem ? launch_encode_t<Rans64, 1, int32_t, true, true, true>(c, st)
-              : launch_encode_t<Rans64, 1, int32_t, false, true, true>(c, st);
+    return smem ? launch_encode_t<Rans64, 32, int32_t, 1, true, true>(c, st)
+                : launch_encode_t<Rans64, 32, int32_t, 0, true, true>(c, st);
+  return smem ? launch_encode_t<Rans64, 1, int32_t, 1, true, true>(c, st)
+              : launch_encode_t<Rans64, 1, int32_t, 0, true, true>(c, st);
 }
 
 int launch_compact(const Geom &g, const char *scratch, const uint64_t *lens, uint8_t *out,

@@ -705,7 +705,12 @@ int prepare_tables(const int32_t *cdfs, int K, int Lmax, const int32_t *lengths,
     for (int r = 0; r < K; ++r) t += 1ull << q[r];
     return t;
   };
-  const bool enc_smem = (int64_t)meta_bytes + bucket_bytes + kEncStageBytes <= budget;
+  // encoder: bucket words in shared memory when they fit beside the rings,
+  // else the 16-bit starts (with room for at least 4 warps' rings), else
+  // global memory
+  const int enc_mode = (int64_t)meta_bytes + bucket_bytes + kEncStageBytes <= budget ? 1
+                       : ((int64_t)meta_bytes + start_bytes + kEncStageBytes / 6 <= budget ? 2
+                                                                                          : 0);
   bool dec_smem = false;
   uint64_t chunk_words = 0;
   if ((int64_t)meta_bytes + start_bytes + kDecStageBytes <= budget) {
@@ -786,8 +791,11 @@ int prepare_tables(const int32_t *cdfs, int K, int Lmax, const int32_t *lengths,
   out->bucket_bytes = bucket_bytes;
   out->start_bytes = start_bytes;
   out->slot_bytes = slot_bytes;
-  out->enc_in_smem = enc_smem ? 1 : 0;
-  out->dec_in_smem = dec_smem ? 1 : 0;
+  // decoder: metadata, starts and slots in shared memory when they fit, else
+  // metadata and starts (each lookup searching its row), else global memory
+  out->enc_in_smem = enc_mode;
+  out->dec_in_smem =
+      dec_smem ? 1 : ((int64_t)meta_bytes + start_bytes + kDecStageBytes <= budget ? 2 : 0);
   out->device = dev;
   out->precision = prec;
   return RANS_OK;

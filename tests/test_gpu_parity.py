@@ -380,6 +380,20 @@ def test_tables_too_large_for_shared_memory(W):
     _check_streams(w)
 
 
+@pytest.mark.parametrize("W", [1, 32])
+def test_large_tables_staged_as_starts(W):
+    """256 pmf rows of 257 entries (the rans32_16 benchmark shape at the
+    64-bit format): too large for bucket words or lookup slots in shared
+    memory, so both coders stage the row metadata and 16-bit starts and the
+    decoder searches each row."""
+    w = WL.r16_rows(n_streams=96, per_stream=1000)
+    w = dict(w, fmt="rans64", precision=16, W=W)
+    c, l, o = oracle_tables(w)
+    tables = tables_from_numpy(c, l, o)
+    assert tables.c.enc_in_smem == 2 and tables.c.dec_in_smem == 2
+    _check_streams(w)
+
+
 def test_table_refresh_matches_fresh_prepare():
     """A prepared table set refreshed from new rows of the same lengths codes
     exactly like one prepared from those rows."""
@@ -443,7 +457,7 @@ def test_build_indexes_matches_oracle(K):
 
 
 @pytest.mark.parametrize("W,with_means,n_rows", [(32, True, 64), (32, False, 64), (1, True, 64),
-                                                (32, True, 256)])
+                                                (32, True, 256), (32, True, 128)])
 def test_encode_from_scales_matches_oracle(W, with_means, n_rows):
     """Float latents in: the streams equal the oracle's encode of
     build_indexes(scales) and rint(y - mean); decoding gives back

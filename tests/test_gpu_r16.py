@@ -97,6 +97,17 @@ def test_uint8_sweep_with_index_blocks():
     _check_streams(w)
 
 
+@pytest.mark.parametrize("W", [1, 32])
+def test_large_tables_staged_as_starts(W):
+    """The benchmark shape's 256 rows of 257 entries at precision 15: row
+    metadata and starts in shared memory, a row search per lookup."""
+    w = _r16(WL.r16_rows(n_streams=96, per_stream=1000), W=W)
+    c, l, o = oracle_tables(w)
+    tables = tables_from_numpy(c, l, o, precision=15)
+    assert tables.c.enc_in_smem == 2 and tables.c.dec_in_smem == 2
+    _check_streams(w)
+
+
 def test_streams_of_every_length_phase():
     """Contiguous streams of 1 to 70 symbols (partial first groups of every
     size) and empty streams."""
