@@ -648,8 +648,9 @@ int refresh_tables(const int32_t *cdfs, int K, int Lmax, const int32_t *lengths,
   return cudaGetLastError() == cudaSuccess ? RANS_OK : RANS_ERR_CUDA;
 }
 
-// Room for the slots and bitmap words: the slots of every row at the largest
-// q, as many bitmap words again, and 256 KB (shared-memory tables plan up to
+// Room for the bucket words and starts (each row with up to 63 entries of
+// bank skew), the slots of every row at the largest q, as many bitmap words
+// again, and 256 KB (shared-memory tables plan up to
 // a quarter of their slot room as bitmap words; tables read from global
 // memory as many words as slots).
 uint64_t tables_bytes_bound(int K, int Lmax) {
@@ -657,8 +658,9 @@ uint64_t tables_bytes_bound(int K, int Lmax) {
   const int64_t nb = (int64_t)Lmax - 1;
   int q = ceil_log2(nb);
   q = q < kMinQ ? kMinQ : (q > kMaxQ ? kMaxQ : q);
-  return (uint64_t)kHeaderBytes + pad16(16ull * kMetaCopies * K) + pad16(4ull * K * nb) +
-         pad16(2ull * K * nb + 2) + pad16(8ull * K * (1ull << q)) + 262144ull;
+  const uint64_t nbp = (uint64_t)nb + 63;  // with the bank skew pad
+  return (uint64_t)kHeaderBytes + pad16(16ull * kMetaCopies * K) + pad16(4ull * K * nbp) +
+         pad16(2ull * K * nbp + 2) + pad16(8ull * K * (1ull << q)) + 262144ull;
 }
 
 int prepare_tables(const int32_t *cdfs, int K, int Lmax, const int32_t *lengths,
@@ -680,10 +682,26 @@ int prepare_tables(const int32_t *cdfs, int K, int Lmax, const int32_t *lengths,
   std::vector<int> q(K);
   uint64_t nbuckets = 0;
   int max_nb = 0;
+  // Row bases are skewed across shared-memory banks: rows of equal length
+  // would otherwise start in the same bank, and the lanes of a warp, each
+  // reading the same position of its own row (the first probe of a row
+  // search), would all hit it.  Each row takes the smallest pad (< 64
+  // entries) that starts its 16-bit starts in the least-used bank so far.
+  uint32_t bank_use[32] = {0};
   for (int r = 0; r < K; ++r) {
     if (len[r] < 0) return len[r];
     if (len[r] < 2 || len[r] > Lmax) return RANS_ERR_TABLE;
     const int nb = len[r] - 1;
+    uint32_t pad = 0, best = UINT32_MAX;
+    for (uint32_t p = 0; p < 64; ++p) {
+      const uint32_t use = bank_use[((nbuckets + p) >> 1) & 31];
+      if (use < best) {
+        best = use;
+        pad = p;
+      }
+    }
+    nbuckets += pad;
+    ++bank_use[(nbuckets >> 1) & 31];
     meta[r].bucket_base = (uint32_t)nbuckets;
     meta[r].maxv = (uint32_t)(len[r] - 2);
     meta[r].offset = off[r];
