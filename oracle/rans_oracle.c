@@ -324,8 +324,16 @@ static int symbol_ops(int64_t s, int32_t r, int K, const int32_t *cdfs, int Lmax
  * + start.  BITS(v): if x >= 2^59, push a word likewise; then x = 16 x + v.
  * Flush: lanes W-1 .. 0 push their state as two words, high first.  The
  * stream is the pushed words in reverse push order, each little-endian.
- * Reading: lane = symbol index mod W and lane 0 first in the flush.
+ * Reading: lane = symbol index mod W and lane 0 first in the flush.  W is 1,
+ * 2, 4, 8 ([TA] Usage, variants table: rans64 interleaves 1, 2, 4 or 8
+ * states) or 32 (the warp-wide interleave of the same table's rans32_16
+ * row, applied to this format).
  */
+static int valid_interleave(int W)
+{
+    return W == 1 || W == 2 || W == 4 || W == 8 || W == 32;
+}
+
 typedef struct {
     uint32_t *w;
     size_t n, cap;
@@ -349,7 +357,7 @@ int64_t orc_encode_stream(const int64_t *sym, const int32_t *row, int64_t n,
                           const int32_t *lengths, const int32_t *offsets,
                           int W, uint8_t *out, int64_t cap)
 {
-    if (W != 1 && W != 32) return ORC_ERR_ARG;
+    if (!valid_interleave(W)) return ORC_ERR_ARG;
     if (n < 0) return ORC_ERR_ARG;
     oplist_t ops = {NULL, 0, 0};
     words_t words = {NULL, 0, 0};
@@ -452,7 +460,7 @@ int orc_decode_stream(const uint8_t *in, int64_t len, const int32_t *row, int64_
                       const int32_t *lengths, const int32_t *offsets,
                       int W, int64_t *sym_out)
 {
-    if (W != 1 && W != 32) return ORC_ERR_ARG;
+    if (!valid_interleave(W)) return ORC_ERR_ARG;
     reader_t R = {in, len, 0};
     uint64_t x[32];
     for (int l = 0; l < W; ++l) {
@@ -544,17 +552,13 @@ static int push_word16(words16_t *W, uint16_t v)
     return ORC_OK;
 }
 
-static int valid_interleave16(int W)
-{
-    return W == 1 || W == 2 || W == 4 || W == 8 || W == 32;
-}
 
 int64_t orc_encode_stream16(const int64_t *sym, const int32_t *row, int64_t n,
                             const int32_t *cdfs, int K, int Lmax,
                             const int32_t *lengths, const int32_t *offsets,
                             int prec, int W, uint8_t *out, int64_t cap)
 {
-    if (!valid_interleave16(W) || n < 0 || prec < 1 || prec > 15) return ORC_ERR_ARG;
+    if (!valid_interleave(W) || n < 0 || prec < 1 || prec > 15) return ORC_ERR_ARG;
     oplist_t ops = {NULL, 0, 0};
     words16_t words = {NULL, 0, 0};
     int64_t result = ORC_OK;
@@ -632,7 +636,7 @@ int orc_decode_stream16(const uint8_t *in, int64_t len, const int32_t *row, int6
                         const int32_t *lengths, const int32_t *offsets,
                         int prec, int W, int64_t *sym_out)
 {
-    if (!valid_interleave16(W) || prec < 1 || prec > 15) return ORC_ERR_ARG;
+    if (!valid_interleave(W) || prec < 1 || prec > 15) return ORC_ERR_ARG;
     reader_t R = {in, len, 0};
     uint32_t x[32];
     for (int l = 0; l < W; ++l) {

@@ -52,8 +52,8 @@ int orc_build_cdfs_from_pmfs_prec(const float *pmfs, int K, int stride,
                                   const int32_t *pmf_lengths, const float *tail_mass,
                                   int prec, int32_t *cdfs, int Lmax, int32_t *lengths);
 
-/* One stream of n symbols (in stream order) with their row indexes; W = 1 or
- * 32 interleaved states.  Returns the byte length, or a negative status. */
+/* One stream of n symbols (in stream order) with their row indexes; W = 1, 2,
+ * 4, 8 or 32 interleaved states.  Returns the byte length, or a negative status. */
 int64_t orc_encode_stream(const int64_t *sym, const int32_t *row, int64_t n,
                           const int32_t *cdfs, int K, int Lmax,
                           const int32_t *lengths, const int32_t *offsets,

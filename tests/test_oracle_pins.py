@@ -56,6 +56,39 @@ def test_interleaved_single_symbol_reduces_to_single_state(golden):
         assert b32[256:] == b1[8:]
 
 
+@pytest.mark.parametrize("W", [2, 4, 8])
+def test_few_state_interleave_reduces_to_single_state(golden, W):
+    """The same reduction for 2, 4 and 8 interleaved states ("torch_ans
+    0.3.0", Usage, variants table: rans64 interleaves 1, 2, 4 or 8 states)."""
+    cdf, lengths, offsets = _row_from(golden("e1_two_symbols.txt"))
+    idle = bytes([0, 0, 0, 0x80, 0, 0, 0, 0])
+    for s in [-7, -1, 0, 2, 11, 1 << 20]:
+        rows = np.zeros(1, dtype=np.int32)
+        b1 = O.encode_stream([s], rows, cdf, lengths, offsets, W=1).tobytes()
+        bw = O.encode_stream([s], rows, cdf, lengths, offsets, W=W).tobytes()
+        assert bw[:8] == b1[:8]
+        assert bw[8:8 * W] == idle * (W - 1)
+        assert bw[8 * W:] == b1[8:]
+
+
+def test_interleaved_lanes_are_independent_single_state_streams(golden):
+    """With symbols that never renormalise, W interleaved states hold W
+    single-state codings of the every-W-th subsequences: lane l's state is
+    the single-state stream of symbols l, l + W, ... (E1's row, symbols in
+    its coded range, few enough per lane that no word leaves)."""
+    cdf, lengths, offsets = _row_from(golden("e1_two_symbols.txt"))
+    rng = np.random.Generator(np.random.PCG64(17))
+    for W in (2, 4, 8, 32):
+        n = 2 * W
+        sym = rng.integers(-1, 2, size=n)
+        rows = np.zeros(n, dtype=np.int32)
+        bw = O.encode_stream(sym, rows, cdf, lengths, offsets, W=W).tobytes()
+        assert len(bw) == 8 * W                 # no word left any lane
+        for l in range(W):
+            b1 = O.encode_stream(sym[l::W], rows[l::W], cdf, lengths, offsets, W=1).tobytes()
+            assert len(b1) == 8 and bw[8 * l:8 * l + 8] == b1
+
+
 def test_empty_stream_is_initial_state():
     cdf = np.array([[0, 32768, 65536]], dtype=np.int32)
     one = np.array([3], dtype=np.int32)

@@ -56,7 +56,7 @@ def test_uniform_row_matches_packing():
         assert back.tolist() == u
 
 
-@pytest.mark.parametrize("W", [1, 32])
+@pytest.mark.parametrize("W", [1, 4, 32])
 def test_brute_force_round_trip_and_injectivity(W):
     cdf, lengths, offsets = E_ROW
     for n in range(0, 5):
@@ -98,7 +98,7 @@ def _information_bits(sym, rows, cdfs, lengths, offsets):
     return bits, nops
 
 
-@pytest.mark.parametrize("W", [1, 32])
+@pytest.mark.parametrize("W", [1, 8, 32])
 def test_size_within_bound_of_information_content(W):
     t = WL.tiny(seed=5)
     cdfs, lengths, offsets = O.build_cdfs_from_scales(t["scales"], t["tail_mass"])
@@ -111,7 +111,7 @@ def test_size_within_bound_of_information_content(W):
         I, nops = _information_bits(sym, rows, cdfs, lengths, offsets)
         eps = 2e-4 * nops / 8
         b = O.encode_stream(sym, rows, cdfs, lengths, offsets, W=W)
-        lo, hi = (4, 8) if W == 1 else (128, 256)
+        lo, hi = 4 * W, 8 * W
         assert I / 8 + lo - eps < b.size <= I / 8 + hi + eps, (n, b.size, I / 8)
 
 
