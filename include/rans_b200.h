@@ -107,7 +107,11 @@ enum { RANS_FMT_RANS64 = 0, RANS_FMT_RANS32_16 = 1 };
  *             tile_h x tile_w), ordered (b, g, tile row, tile column); inside a
  *             stream the elements go (channel, row, column); edge tiles are
  *             partial.  n must equal B*C*H*W.
- *   interleave: 1 or 32 states per stream.
+ *   interleave: 1, 2, 4, 8 or 32 states per stream ("torch_ans 0.3.0",
+ *             Usage, variants table: 1/2/4/8 for rans64, also 32 for
+ *             rans32_16); symbol i of a stream codes on state i mod W.  32
+ *             maps a stream onto a warp, the others onto one thread.  The
+ *             float-latent entry points take 1 or 32.
  *   index_block: element p (flat position in the symbol array) uses row
  *             indexes[p / index_block]; 1 = one index per symbol; must be a
  *             power of two.

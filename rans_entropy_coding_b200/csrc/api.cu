@@ -43,7 +43,9 @@ bool is_pow2(int64_t v) { return v > 0 && (v & (v - 1)) == 0; }
 
 int make_geom(const rans_chunking *ch, int64_t n, Geom &g) {
   if (ch == nullptr || n < 0) return RANS_ERR_ARG;
-  if (ch->interleave != 1 && ch->interleave != 32) return RANS_ERR_ARG;
+  if (ch->interleave != 1 && ch->interleave != 2 && ch->interleave != 4 && ch->interleave != 8 &&
+      ch->interleave != 32)
+    return RANS_ERR_ARG;
   if (!is_pow2(ch->index_block)) return RANS_ERR_ARG;
   if (ch->format != RANS_FMT_RANS64 && ch->format != RANS_FMT_RANS32_16) return RANS_ERR_ARG;
   std::memset(&g, 0, sizeof(g));
@@ -329,6 +331,7 @@ static int float_args(const rans_tables *tables, const rans_chunking *chunking,
   if (!tables_usable(tables) || !chunking) return RANS_ERR_ARG;
   if (table_len != tables->K || chunking->index_block != 1) return RANS_ERR_ARG;
   if (chunking->format != RANS_FMT_RANS64 || tables->precision != 16) return RANS_ERR_ARG;
+  if (chunking->interleave != 1 && chunking->interleave != 32) return RANS_ERR_ARG;
   return RANS_OK;
 }
 

@@ -522,6 +522,177 @@ __device__ void decode_stream_w1(const DecCtx &c, const RowMeta *meta, const uin
   if (bad || x != F::kLow || pw != nw) report(c.status, RANS_ERR_CORRUPT, s);
 }
 
+// W = 2, 4 or 8 interleaved states on W consecutive lanes of a warp, 32 / W
+// streams per warp ("torch_ans 0.3.0", Usage legend: num_interleaves 2, 4
+// and 8 map to that many consecutive lanes, sub-warp groups).  Lane l of a
+// segment holds state l and decodes symbols l, l + W, ...; refills take the
+// segment's next words in lane order (ballot + popc within the segment's
+// lanes); a group holding an escape goes lane by lane in ascending order,
+// every segment's scans restarting at its first lane.  All lanes run the
+// same number of groups (the warp's longest stream), idle lanes masked.
+template <class F>
+__device__ __forceinline__ EscapeResult<F> escape_group_seg(
+    typename F::State x, bool active, bool esc, uint32_t maxv, uint64_t abs0,
+    const typename F::Word *words, uint64_t nw, int l, int W, int seg_last) {
+  const int lane = threadIdx.x & 31;
+  bool bad = false;
+  int64_t val = 0;
+  const bool need_sym = active && x < F::kLow;
+  uint32_t cons = need_sym ? 1u : 0u;
+  auto seg_scan = [&](uint32_t v) {  // inclusive scan over the segment's lanes
+    uint32_t inc = v;
+    for (int o = 1; o < W; o <<= 1) {
+      const uint32_t t = __shfl_up_sync(kFull, inc, o);
+      if (l >= o) inc += t;
+    }
+    return inc;
+  };
+  uint32_t rem = __ballot_sync(kFull, esc);
+  while (rem) {
+    const int el = __ffs(rem) - 1;
+    rem &= rem - 1;
+    const uint32_t inc = seg_scan(cons);
+    const uint32_t pre = __shfl_sync(kFull, inc - cons, el);
+    if (lane == el) {
+      uint64_t pp = abs0 + pre;
+      auto rd = [&]() -> uint32_t {
+        uint32_t v = 0;
+        if (pp < nw) v = __ldg(words + pp); else bad = true;
+        ++pp;
+        return v;
+      };
+      if (x < F::kLow) x = (x << F::kWordBits) | rd();
+      auto getbits = [&]() -> uint32_t {
+        const uint32_t v = (uint32_t)x & kBypassMax;
+        x >>= kBypassBits;
+        if (x < F::kLow) x = (x << F::kWordBits) | rd();
+        return v;
+      };
+      uint32_t v4 = getbits();
+      uint32_t nb = v4;
+      while (v4 == kBypassMax && nb <= 15) {
+        v4 = getbits();
+        nb += v4;
+      }
+      if (nb > 15) {
+        bad = true;
+        nb = 0;
+      }
+      uint64_t raw = 0;
+      for (uint32_t k = 0; k < nb; ++k) raw |= (uint64_t)getbits() << (kBypassBits * k);
+      const int64_t half = (int64_t)(raw >> 1);
+      val = (raw & 1) ? (-half - 1) : ((int64_t)maxv + half);
+      cons = (uint32_t)(pp - (abs0 + pre));
+    }
+  }
+  const uint32_t inc = seg_scan(cons);
+  if (need_sym && !esc) {
+    const uint64_t pp = abs0 + (inc - cons);
+    uint32_t v = 0;
+    if (pp < nw) v = __ldg(words + pp); else bad = true;
+    x = (x << F::kWordBits) | v;
+  }
+  EscapeResult<F> r;
+  r.x = x;
+  r.val = val;
+  r.cur = abs0 + __shfl_sync(kFull, inc, seg_last);
+  r.bad = bad;
+  return r;
+}
+
+// One segment's stream (s < 0: an idle segment, still taking part in the
+// warp's votes and shuffles).
+template <class F, typename SymT, bool ROWS>
+__device__ void decode_segment(const DecCtx &c, const RowMeta *meta, const uint16_t *starts,
+                               const uint32_t *slots, int64_t s, int W) {
+  using State = typename F::State;
+  using Word = typename F::Word;
+  const int lane = threadIdx.x & 31;
+  const int l = lane & (W - 1);
+  const int seg0 = lane - l;
+  const uint32_t segmask = (W == 32 ? kFull : ((1u << W) - 1u)) << seg0;
+  const uint32_t sh = F::shift(c.sh);
+  StreamDesc d;
+  d.ok = false;
+  d.n = 0;
+  d.base = 0;
+  d.t = Tile{1, kNoWrap, 0, 0};
+  const Word *words = nullptr;
+  uint64_t nw = 0;
+  bool live = false;
+  if (s >= 0) {
+    d = stream_desc(c.g, s);
+    live = d.ok && stream_bounds<F>(c, s, W, words, nw);
+    if (!live && l == 0) report(c.status, d.ok ? RANS_ERR_CORRUPT : RANS_ERR_ARG, s);
+    if (live && l == 0)
+      bulk_prefetch_l2(reinterpret_cast<const char *>(c.in),
+                       reinterpret_cast<const char *>(c.in) + c.in_bytes,
+                       reinterpret_cast<const char *>(words), sizeof(Word) * nw);
+  }
+  State x = F::kLow;
+  if (live) x = (State)__ldg(words + 2 * l) | ((State)__ldg(words + 2 * l + 1) << F::kWordBits);
+  uint64_t cur = 2 * (uint64_t)W;
+  const int32_t n = live ? (int32_t)d.n : 0;
+  const int32_t G = (n + W - 1) / W;
+  const int32_t Gmax = (int32_t)__reduce_max_sync(kFull, (uint32_t)G);
+  const int ib = c.g.ib_shift;
+  const uint32_t kmax = (uint32_t)c.K - 1u;
+  bool bad = false, bad_index = false;
+  // the row index of this lane's element in group k, read one group ahead
+  auto pos_of = [&](int32_t k) -> int64_t {
+    RelPos rp;
+    rp.init(d.t, k * W + l);
+    return d.base + rp.rel(d.t);
+  };
+  int32_t rn = 0;
+  if (0 < G && l < n) rn = __ldg(c.idx + (pos_of(0) >> ib));
+  for (int32_t k = 0; k < Gmax; ++k) {
+    const int32_t i = k * W + l;
+    const bool active = i < n;
+    const uint32_t r = (uint32_t)rn;
+    rn = 0;
+    if (i + W < n) rn = __ldg(c.idx + (pos_of(k + 1) >> ib));
+    bad_index |= active && r > kmax;
+    const RowMeta m = row_meta(meta, active && r <= kmax ? r : 0u);
+    const uint32_t cum = F::cum16(x, sh);
+    const uint32_t sym =
+        ROWS ? search_row(cum, m, starts) : lookup<true, true>(cum, m, starts, slots, active);
+    const uint32_t start = starts[m.bucket_base + sym];
+    const uint32_t freq = width_of(start, starts[m.bucket_base + sym + 1]);
+    State y = F::dec_step(x, cum, start, freq, sh);
+    if (!active) y = x;
+    const bool esc = active && sym == m.maxv;
+    const bool need = active && y < F::kLow;
+    const uint32_t nm = __ballot_sync(kFull, need);
+    int64_t val = (int64_t)sym;
+    if (!__any_sync(kFull, esc)) {
+      if (need) {
+        const uint64_t pp = cur + __popc(nm & segmask & lanemask_lt());
+        uint32_t v = 0;
+        if (pp < nw) v = __ldg(words + pp); else bad = true;
+        y = (y << F::kWordBits) | v;
+      }
+      cur += __popc(nm & segmask);
+    } else {
+      const EscapeResult<F> er =
+          escape_group_seg<F>(y, active, esc, m.maxv, cur, words, nw, l, W, seg0 + W - 1);
+      y = er.x;
+      if (esc) val = er.val;
+      bad |= er.bad;
+      cur = er.cur;
+    }
+    x = y;
+    if (active) SymIO<SymT>::store(c.out, pos_of(k), val + (int64_t)m.offset);
+  }
+  // every lane votes (idle segments too), then each live segment's first
+  // lane reports
+  const bool ok = !live || (!bad && x == F::kLow && cur == nw);
+  const uint32_t fails = __ballot_sync(kFull, !ok) & segmask;
+  const uint32_t idx_fails = __ballot_sync(kFull, bad_index) & segmask;
+  if (live && l == 0 && idx_fails) report(c.status, RANS_ERR_INDEX, s);
+  else if (live && l == 0 && fails) report(c.status, RANS_ERR_CORRUPT, s);
+}
+
 // Shared-memory bytes of a table mode: 0 reads the tables from global
 // memory, 1 stages the row metadata, starts and lookup slots, 2 (tables whose
 // slots do not fit) the row metadata and starts, the lookup then searching
@@ -585,6 +756,66 @@ __global__ void __launch_bounds__(W == 32 ? kDecMaxThreads32 : kDecThreads1)
          k += (int64_t)gridDim.x * blockDim.x)
       decode_stream_w1<F, SymT, ROWS>(c, meta, buckets, slots, stream_of(c.g, k), stab);
   }
+}
+
+// W = 2, 4 or 8: 32 / W streams per warp (decode_segment); the table mode is
+// a run-time argument.
+constexpr int kSegThreads = 256;
+
+template <class F, typename SymT>
+__global__ void __launch_bounds__(kSegThreads) decode_kernel_wn(DecCtx c, int mode) {
+  extern __shared__ __align__(16) unsigned char smem[];
+  __shared__ uint64_t bar;
+  const char *gb = c.blob + kHeaderBytes;
+  const RowMeta *meta = reinterpret_cast<const RowMeta *>(gb);
+  const uint16_t *buckets = reinterpret_cast<const uint16_t *>(gb + c.meta_bytes + c.bucket_bytes);
+  const uint32_t *slots =
+      reinterpret_cast<const uint32_t *>(gb + c.meta_bytes + c.bucket_bytes + c.start_bytes);
+  if (mode != 0) {
+    if (!stage_to_smem(smem, gb, c.meta_bytes, &bar, c.status, smem + c.meta_bytes,
+                       gb + c.meta_bytes + c.bucket_bytes,
+                       c.start_bytes + (mode == 1 ? c.slot_bytes : 0u)))
+      return;
+    meta = reinterpret_cast<const RowMeta *>(smem);
+    buckets = reinterpret_cast<const uint16_t *>(smem + c.meta_bytes);
+    slots = reinterpret_cast<const uint32_t *>(smem + c.meta_bytes + c.start_bytes);
+  }
+  const int W = c.g.W;
+  const int per_warp = 32 / W;
+  const int seg = (threadIdx.x & 31) / W;
+  const int64_t warp = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  const int64_t nwarps = (int64_t)gridDim.x * (blockDim.x >> 5);
+  for (int64_t k0 = warp * per_warp; k0 < c.g.S; k0 += nwarps * per_warp) {
+    const int64_t k = k0 + seg;
+    const int64_t s = k < c.g.S ? stream_of(c.g, k) : -1;
+    if (mode == 2)
+      decode_segment<F, SymT, true>(c, meta, buckets, slots, s, W);
+    else
+      decode_segment<F, SymT, false>(c, meta, buckets, slots, s, W);
+  }
+}
+
+template <class F, typename SymT>
+int launch_decode_wn(const DecCtx &c, int mode, cudaStream_t st) {
+  auto kern = decode_kernel_wn<F, SymT>;
+  const uint32_t tab = dec_table_bytes(mode, c);
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)tab) !=
+      cudaSuccess)
+    return RANS_ERR_CUDA;
+  int fit = 0;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&fit, kern, kSegThreads, tab) !=
+          cudaSuccess ||
+      fit < 1)
+    return RANS_ERR_CUDA;
+  const int64_t warps = (c.g.S + 32 / c.g.W - 1) / (32 / c.g.W);
+  const int64_t need = (warps + kSegThreads / 32 - 1) / (kSegThreads / 32);
+  const int64_t cap = (int64_t)fit * num_sms(dev);
+  int64_t blocks = need < cap ? need : cap;
+  if (blocks < 1) blocks = 1;
+  kern<<<(unsigned)blocks, kSegThreads, tab, st>>>(c, mode);
+  return cudaGetLastError() == cudaSuccess ? RANS_OK : RANS_ERR_CUDA;
 }
 
 template <class F, int W, typename SymT, int MODE, bool IB0>
@@ -660,8 +891,9 @@ int launch_decode_w(const DecCtx &c, int mode, cudaStream_t st) {
 
 template <class F, typename SymT>
 int launch_decode_f(const DecCtx &c, int mode, cudaStream_t st) {
-  return c.g.W == 32 ? launch_decode_w<F, 32, SymT>(c, mode, st)
-                     : launch_decode_w<F, 1, SymT>(c, mode, st);
+  if (c.g.W == 32) return launch_decode_w<F, 32, SymT>(c, mode, st);
+  if (c.g.W == 1) return launch_decode_w<F, 1, SymT>(c, mode, st);
+  return launch_decode_wn<F, SymT>(c, mode, st);
 }
 
 template <typename SymT>

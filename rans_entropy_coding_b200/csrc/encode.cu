@@ -502,6 +502,115 @@ __device__ void encode_stream_w1(const EncCtx &c, const RowMeta *meta, const uin
   c.lens[s] = sizeof(Word) * (uint64_t)cursor;
 }
 
+// W = 2, 4 or 8 interleaved states on W consecutive lanes of a warp, 32 / W
+// streams per warp (the sub-warp groups of "torch_ans 0.3.0", Usage legend).
+// Lane l of a segment holds state l and codes symbols l, l + W, ... in
+// reverse group order; within a group lane W-1 codes first, so lane l's
+// words land below those of the segment's lanes > l (ballot + popc within
+// the segment); a group holding an escape counts each lane's words and
+// places them by a suffix sum over the segment.  The flush pushes lanes
+// W-1 .. 0, high word first.  All lanes run the warp's longest stream's
+// group count, idle lanes masked.
+template <class F, typename SymT, bool ST>
+__device__ void encode_segment(const EncCtx &c, const RowMeta *meta, const uint32_t *buckets,
+                               int64_t s, int W) {
+  using Word = typename F::Word;
+  using State = typename F::State;
+  const int lane = threadIdx.x & 31;
+  const int l = lane & (W - 1);
+  const int seg0 = lane - l;
+  const uint32_t segmask = ((1u << W) - 1u) << seg0;
+  const uint32_t above = segmask & (0xfffffffeu << lane);  // the segment's lanes > l
+  const uint32_t sh = F::shift(c.sh);
+  StreamDesc d;
+  d.ok = false;
+  d.n = 0;
+  d.base = 0;
+  d.t = Tile{1, kNoWrap, 0, 0};
+  bool live = false;
+  if (s >= 0) {
+    d = stream_desc(c.g, s);
+    live = d.ok;
+    if (!live && l == 0) report(c.status, RANS_ERR_ARG, s);
+  }
+  Word *end = live ? reinterpret_cast<Word *>(c.scratch + slot_end(c.g, d, s)) : nullptr;
+  const int32_t n = live ? (int32_t)d.n : 0;
+  const int32_t G = (n + W - 1) / W;
+  const int32_t Gmax = (int32_t)__reduce_max_sync(kFull, (uint32_t)G);
+  const int ib = c.g.ib_shift;
+  const uint32_t kmax = (uint32_t)c.K - 1u;
+  State x = F::kLow;
+  uint32_t cursor = 0;
+  bool bad_index = false, bad_range = false;
+  auto pos_of = [&](int32_t k) -> int64_t {
+    RelPos rp;
+    rp.init(d.t, k * W + l);
+    return d.base + rp.rel(d.t);
+  };
+  // this lane's symbol and row index of group k, read one group ahead
+  int32_t sn = 0, rn = 0;
+  auto load = [&](int32_t k) {
+    sn = 0;
+    rn = 0;
+    if (k >= 0 && k * W + l < n) {
+      const int64_t p = pos_of(k);
+      sn = SymIO<SymT>::load(c.sym, p);
+      rn = __ldg(c.idx + (p >> ib));
+    }
+  };
+  load(Gmax - 1);
+  for (int32_t k = Gmax - 1; k >= 0; --k) {
+    const bool active = k * W + l < n;
+    const int32_t sv = sn;
+    const uint32_t r = (uint32_t)rn;
+    load(k - 1);
+    bad_index |= active && r > kmax;
+    uint32_t start, freq;
+    uint64_t raw;
+    bool esc;
+    map_symbol<ST>(sv, row_meta(meta, active && r <= kmax ? r : 0u), buckets, start, freq, raw,
+                   esc);
+    esc = esc && active;
+    bad_range |= esc && (raw >> 60) != 0;
+    raw &= (1ull << 60) - 1;
+    const double rcp = F::rcp(freq, sh);
+    if (!__any_sync(kFull, esc)) {
+      const bool need = active && F::need_word(x, freq);
+      const uint32_t bm = __ballot_sync(kFull, need);
+      if (need) st_global(end - 1 - (cursor + __popc(bm & above)), (Word)x);
+      if (need) x >>= F::kWordBits;
+      cursor += __popc(bm & segmask);
+      if (active) x = F::sym_step(x, start, freq, rcp, sh);
+    } else {
+      // every lane counts its words, a suffix sum over the segment places them
+      uint32_t kw = 0;
+      if (active) {
+        State y = x;
+        kw = symbol_ops<F, false>(y, start, freq, rcp, raw, esc, end, 0, sh);
+      }
+      uint32_t inc = kw;
+      for (int o = 1; o < W; o <<= 1) {
+        const uint32_t t = __shfl_down_sync(kFull, inc, o);
+        if (l + o < W) inc += t;
+      }
+      const uint32_t total = __shfl_sync(kFull, inc, seg0);
+      if (active) symbol_ops<F, true>(x, start, freq, rcp, raw, esc, end, cursor + inc - kw, sh);
+      cursor += total;
+    }
+  }
+  const uint32_t idx_fails = __ballot_sync(kFull, bad_index) & segmask;
+  const uint32_t rng_fails = __ballot_sync(kFull, bad_range) & segmask;
+  if (!live) return;
+  if (idx_fails || rng_fails) {
+    if (l == 0) report(c.status, idx_fails ? RANS_ERR_INDEX : RANS_ERR_RANGE, s);
+    return;
+  }
+  const uint32_t kk = cursor + 2u * (uint32_t)(W - 1 - l);
+  st_global(end - 1 - kk, (Word)(x >> F::kWordBits));
+  st_global(end - 2 - kk, (Word)x);
+  if (l == 0) c.lens[s] = sizeof(Word) * (uint64_t)(cursor + 2 * W);
+}
+
 // Shared-memory bytes of a table mode: 0 reads the tables from global
 // memory, 1 stages the row metadata and bucket words, 2 the row metadata
 // and the 16-bit starts.
@@ -555,6 +664,43 @@ __global__ void __launch_bounds__(W == 32 ? kEncThreads32 : kEncThreads1)
     for (int64_t k = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; k < c.g.S;
          k += (int64_t)gridDim.x * blockDim.x)
       encode_stream_w1<F, SymT, FLT, ST>(c, meta, buckets, stream_of(c.g, k), stab);
+  }
+}
+
+// W = 2, 4 or 8: 32 / W streams per warp (encode_segment); the table mode
+// (0, 1 or 2 as for encode_kernel) is a run-time argument.
+constexpr int kSegThreads = 256;
+
+template <class F, typename SymT>
+__global__ void __launch_bounds__(kSegThreads) encode_kernel_wn(EncCtx c, int mode) {
+  extern __shared__ __align__(16) unsigned char smem[];
+  __shared__ uint64_t bar;
+  const RowMeta *meta = reinterpret_cast<const RowMeta *>(c.blob + kHeaderBytes);
+  const char *gb = c.blob + kHeaderBytes;
+  const uint32_t *buckets = reinterpret_cast<const uint32_t *>(gb + c.meta_bytes);
+  if (mode == 1) {
+    if (!stage_to_smem(smem, gb, c.meta_bytes + c.bucket_bytes, &bar, c.status)) return;
+  } else if (mode == 2) {
+    if (!stage_to_smem(smem, gb, c.meta_bytes, &bar, c.status, smem + c.meta_bytes,
+                       gb + c.meta_bytes + c.bucket_bytes, c.start_bytes))
+      return;
+  }
+  if (mode != 0) {
+    meta = reinterpret_cast<const RowMeta *>(smem);
+    buckets = reinterpret_cast<const uint32_t *>(smem + c.meta_bytes);
+  }
+  const int W = c.g.W;
+  const int per_warp = 32 / W;
+  const int seg = (threadIdx.x & 31) / W;
+  const int64_t warp = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  const int64_t nwarps = (int64_t)gridDim.x * (blockDim.x >> 5);
+  for (int64_t k0 = warp * per_warp; k0 < c.g.S; k0 += nwarps * per_warp) {
+    const int64_t k = k0 + seg;
+    const int64_t s = k < c.g.S ? stream_of(c.g, k) : -1;
+    if (mode == 2)
+      encode_segment<F, SymT, true>(c, meta, buckets, s, W);
+    else
+      encode_segment<F, SymT, false>(c, meta, buckets, s, W);
   }
 }
 
@@ -700,6 +846,29 @@ int launch_encode_t(const EncCtx &c, cudaStream_t st) {
   return cudaGetLastError() == cudaSuccess ? RANS_OK : RANS_ERR_CUDA;
 }
 
+template <class F, typename SymT>
+int launch_encode_wn(const EncCtx &c, int mode, cudaStream_t st) {
+  auto kern = encode_kernel_wn<F, SymT>;
+  const uint32_t tab = enc_table_bytes(mode, c);
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)tab) !=
+      cudaSuccess)
+    return RANS_ERR_CUDA;
+  int fit = 0;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&fit, kern, kSegThreads, tab) !=
+          cudaSuccess ||
+      fit < 1)
+    return RANS_ERR_CUDA;
+  const int64_t warps = (c.g.S + 32 / c.g.W - 1) / (32 / c.g.W);
+  const int64_t need = (warps + kSegThreads / 32 - 1) / (kSegThreads / 32);
+  const int64_t cap = (int64_t)fit * num_sms(dev);
+  int64_t blocks = need < cap ? need : cap;
+  if (blocks < 1) blocks = 1;
+  kern<<<(unsigned)blocks, kSegThreads, tab, st>>>(c, mode);
+  return cudaGetLastError() == cudaSuccess ? RANS_OK : RANS_ERR_CUDA;
+}
+
 template <class F, int W, typename SymT, int MODE>
 int launch_encode_m(const EncCtx &c, cudaStream_t st) {
   return c.g.ib_shift == 0 ? launch_encode_t<F, W, SymT, MODE, true, false>(c, st)
@@ -715,8 +884,9 @@ int launch_encode_w(const EncCtx &c, int mode, cudaStream_t st) {
 
 template <class F, typename SymT>
 int launch_encode_f(const EncCtx &c, int mode, cudaStream_t st) {
-  return c.g.W == 32 ? launch_encode_w<F, 32, SymT>(c, mode, st)
-                     : launch_encode_w<F, 1, SymT>(c, mode, st);
+  if (c.g.W == 32) return launch_encode_w<F, 32, SymT>(c, mode, st);
+  if (c.g.W == 1) return launch_encode_w<F, 1, SymT>(c, mode, st);
+  return launch_encode_wn<F, SymT>(c, mode, st);
 }
 
 template <typename SymT>

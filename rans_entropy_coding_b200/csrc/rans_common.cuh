@@ -108,7 +108,7 @@ __device__ __forceinline__ void report(int32_t *status, int code, int64_t detail
 // Host-computed description of a chunking, passed by value to kernels.
 struct Geom {
   int32_t kind;          // RANS_CHUNK_*
-  int32_t W;             // 1 or 32
+  int32_t W;             // 1, 2, 4, 8 or 32
   int64_t n;             // symbols
   int64_t S;             // streams
   int64_t per;           // CONTIG: ceil(n / S)

@@ -57,7 +57,11 @@ def test_stream_counts_and_workspace_sizes(lib):
     c = rb.Chunking.contig(24, interleave=1)
     assert rb.rans_num_streams(c, 1566720) == 24
     assert rb.rans_max_compressed_bytes(c, 1566720) == 8 * 1566720 + 24 * 32
-    bad = rb.Chunking.contig(24, interleave=8)
+    for W in (2, 4, 8):
+        assert rb.rans_num_streams(rb.Chunking.contig(24, interleave=W), 10) == 24
+    bad = rb.Chunking.contig(24, interleave=3)
+    assert rb.rans_num_streams(bad, 10) == rb.ERR_ARG
+    bad = rb.Chunking.contig(24, interleave=16)
     assert rb.rans_num_streams(bad, 10) == rb.ERR_ARG
     nb = rb.Chunking.contig(4, interleave=32, index_block=3000)
     assert rb.rans_num_streams(nb, 10) == rb.ERR_ARG             # not a power of two

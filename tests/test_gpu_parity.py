@@ -151,7 +151,7 @@ def test_bad_rows_are_reported():
 
 
 # -------------------------------------------------------------- streams --
-@pytest.mark.parametrize("W", [1, 32])
+@pytest.mark.parametrize("W", [1, 2, 4, 8, 32])
 def test_tiny_with_range_edges(W):
     _check_streams(_edge_tiny(W))
 
@@ -161,7 +161,7 @@ def test_tiny_int16_symbols():
     _check_streams(_edge_tiny(1, seed=4, dtype=np.int16))
 
 
-@pytest.mark.parametrize("W", [1, 32])
+@pytest.mark.parametrize("W", [1, 2, 4, 8, 32])
 def test_z_latent(W):
     w = WL.z_latent()
     w["W"] = W
@@ -177,7 +177,7 @@ def test_batch_two_images_tiled():
     _check_streams(WL.y_batch(n_images=2))
 
 
-@pytest.mark.parametrize("W", [1, 32])
+@pytest.mark.parametrize("W", [1, 2, 4, 8, 32])
 def test_batch_small_ragged_tiles(W):
     """Tiles narrower than a warp and a channel group that does not divide C."""
     w = WL.y_batch(n_images=1, cg=5, th=7, tw=11)
@@ -211,13 +211,28 @@ def test_sweep_uint8_blocks():
     _check_streams(WL.sweep(log2_n=20, n_streams=32))
 
 
+@pytest.mark.parametrize("W", [2, 4, 8])
+def test_few_state_interleaves(W):
+    """2, 4 and 8 interleaved states per stream, one thread per stream:
+    int16 symbols, uint8 symbols with index blocks, tables read from global
+    memory (256 rows) and tables staged as starts (256 rows of 257)."""
+    _check_streams(_edge_tiny(W, seed=9, dtype=np.int16))
+    sw = WL.sweep(log2_n=16, n_streams=8)
+    sw["W"] = W
+    _check_streams(sw)
+    mr = WL.many_rows(n=1 << 15, W=W)
+    _check_streams(mr)
+    big = dict(WL.r16_rows(n_streams=24, per_stream=777), fmt="rans64", precision=16, W=W)
+    _check_streams(big)
+
+
 def test_sweep_uint8_single_state():
     w = WL.sweep(log2_n=16, n_streams=8)
     w["W"] = 1
     _check_streams(w)
 
 
-@pytest.mark.parametrize("W", [1, 32])
+@pytest.mark.parametrize("W", [1, 2, 4, 8, 32])
 def test_explicit_chunking_with_empty_streams(W):
     w = WL.tiny(seed=6)
     w["W"] = W
@@ -227,7 +242,7 @@ def test_explicit_chunking_with_empty_streams(W):
     _check_streams(w)
 
 
-@pytest.mark.parametrize("W", [1, 32])
+@pytest.mark.parametrize("W", [1, 2, 4, 8, 32])
 def test_more_streams_than_symbols(W):
     w = WL.tiny(seed=7, n=45)
     w["W"] = W

@@ -69,7 +69,7 @@ def test_tables_at_precision_match_oracle(which, precision):
         assert c[r, l[r] - 1] == 1 << precision
 
 
-@pytest.mark.parametrize("W", [1, 32])
+@pytest.mark.parametrize("W", [1, 2, 4, 8, 32])
 def test_tiny_with_escapes(W):
     """4,096 symbols over 8 rows, 1% far outside the rows (bypass pieces of
     up to 8 nibbles) and the int32 extremes."""
@@ -82,8 +82,9 @@ def test_contiguous_streams_at_several_precisions(precision):
     _check_streams(w)
 
 
-def test_z_latent_single_state():
-    _check_streams(_r16(WL.z_latent()))
+@pytest.mark.parametrize("W", [1, 2, 8])
+def test_z_latent(W):
+    _check_streams(_r16(WL.z_latent(), W=W))
 
 
 def test_y_tiles_two_images():
@@ -97,7 +98,7 @@ def test_uint8_sweep_with_index_blocks():
     _check_streams(w)
 
 
-@pytest.mark.parametrize("W", [1, 32])
+@pytest.mark.parametrize("W", [1, 4, 32])
 def test_large_tables_staged_as_starts(W):
     """The benchmark shape's 256 rows of 257 entries at precision 15: row
     metadata and starts in shared memory, a row search per lookup."""
