@@ -397,6 +397,14 @@ def run_ours(args, world, rank, local):
     rb.check(rb.rans_get_status(ws.enc), "encode status")
     rb.check(rb.rans_get_status(ws.dec), "decode status")
     assert torch.equal(dec, sym), "round trip failed"
+    # N > 1: the ranks' streams form one sharded container; its index is one
+    # all-gather of every rank's stream offsets (after the timed region)
+    container = None
+    if world > 1:
+        from rans_entropy_coding_b200 import shard
+        gidx, base, counts = shard.global_index(ws.offsets)
+        container = {"streams": int(sum(counts)), "bytes": int(gidx[-1].item()),
+                     "rank0_base": base if rank == 0 else None}
 
     tab_ms = float(np.mean([e[0].elapsed_time(e[1]) for e in ev]))
     enc_ms = float(np.mean([e[1].elapsed_time(e[2]) for e in ev]))
@@ -555,6 +563,8 @@ def run_ours(args, world, rank, local):
             "clocks": clocks,
             "gpu_launches": launches_per_step * args.steps,
         }
+        if container is not None:
+            line["config"]["container"] = container
         print(json.dumps(line), flush=True)
 
 

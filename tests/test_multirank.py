@@ -1,16 +1,19 @@
 """The multi-GPU path shards by image with no data exchange; its host logic
-(image shards, per-rank coding, max-over-ranks timing) runs here as two gloo
-ranks on the CPU, coding with the oracle."""
+(image shards, per-rank coding, max-over-ranks timing, the sharded
+container's index) runs here as two gloo ranks on the CPU, coding with the
+oracle."""
 import os
 import socket
 
 import numpy as np
+import torch
 import torch.distributed as dist
 import torch.multiprocessing as mp
 
 import bench
 import oracle as O
 import workloads as WL
+from rans_entropy_coding_b200 import shard
 
 
 def _free_port():
@@ -37,7 +40,12 @@ def _rank(rank, world, port, out):
         tmax = bench.max_over_ranks(t, world)
         gathered = [None] * world
         dist.all_gather_object(gathered, (ids, int(sym.sum()), data.tobytes()[:64]))
-        out[rank] = (tmax, gathered)
+        # the sharded container: rank r codes 8 + r streams of its image
+        offs = O.encode_with_indexes(sym, w["indexes"], c, l, o, w["chunking"], W=32,
+                                     streams=list(range(8 + rank)))[1]
+        gidx, base, counts = shard.global_index(torch.from_numpy(offs.astype(np.int64)))
+        out[rank] = (tmax, gathered, gidx.numpy().tolist(), base, counts,
+                     offs.astype(np.int64).tolist())
     finally:
         dist.destroy_process_group()
 
@@ -58,3 +66,21 @@ def test_two_ranks_shard_by_image():
     # rank 1's shard equals image 1 of a two-image batch coded in one process
     w = WL.y_batch(n_images=2)
     assert int(np.asarray(w["symbols"])[1].sum()) == res[0][1][1][1]
+
+
+def test_sharded_container_index():
+    """Each rank keeps its own streams' bytes; the all-gathered index places
+    rank 1's streams after rank 0's, as one container of both."""
+    world = 2
+    port = _free_port()
+    with mp.Manager() as m:
+        out = m.dict()
+        mp.spawn(_rank, args=(world, port, out), nprocs=world, join=True)
+        res = dict(out)
+    g0, g1 = res[0][2], res[1][2]
+    assert g0 == g1                                          # every rank has the index
+    o0, o1 = res[0][5], res[1][5]
+    assert res[0][4] == [8, 9] and len(g0) == 8 + 9 + 1
+    assert res[0][3] == 0 and res[1][3] == o0[-1]            # rank bases
+    assert g0 == o0 + [v + o0[-1] for v in o1[1:]]
+
