@@ -69,6 +69,14 @@ def lib():
         L.orc_decode_stream16.argtypes = [P, i64, P, i64, P, ctypes.c_int, ctypes.c_int, P, P,
                                           ctypes.c_int, ctypes.c_int, P]
         L.orc_decode_stream16.restype = ctypes.c_int
+        L.orc_alias_build.argtypes = [P, ctypes.c_int, ctypes.c_int, P, P, P, P]
+        L.orc_alias_build.restype = ctypes.c_int
+        L.orc_encode_stream_alias.argtypes = [P, P, i64, P, ctypes.c_int, ctypes.c_int, P, P,
+                                              ctypes.c_int, ctypes.c_int, P, i64]
+        L.orc_encode_stream_alias.restype = i64
+        L.orc_decode_stream_alias.argtypes = [P, i64, P, i64, P, ctypes.c_int, ctypes.c_int, P,
+                                              P, ctypes.c_int, ctypes.c_int, P]
+        L.orc_decode_stream_alias.restype = ctypes.c_int
         L.orc_gaussian_multiplier.argtypes = [f64]
         L.orc_gaussian_multiplier.restype = f64
         L.orc_gaussian_center.argtypes = [ctypes.c_float, f64, P]
@@ -167,8 +175,28 @@ def build_cdfs_from_pmfs(pmfs, pmf_lengths, tail_mass, Lmax=None, precision=16):
 FORMATS = ("rans64", "rans32_16")
 
 
-def encode_stream(symbols, rows, cdfs, lengths, offsets, W=1, fmt="rans64", precision=None):
-    """Codes one stream; returns its bytes as a uint8 array."""
+def _precision(fmt, precision):
+    return precision if precision is not None else (16 if fmt == "rans64" else 15)
+
+
+def alias_build(cdf_row, precision):
+    """Alias table of one row (its cdf entries, bucket count a power of two):
+    (d, a, base, remap) as int32 arrays."""
+    c = np.ascontiguousarray(cdf_row, dtype=np.int32)
+    n = c.size - 1
+    d, a, b = (np.zeros(max(n, 1), np.int32) for _ in range(3))
+    remap = np.zeros(1 << precision, np.int32)
+    st = lib().orc_alias_build(_ptr(c), c.size, precision, _ptr(d), _ptr(a), _ptr(b),
+                               _ptr(remap))
+    if st:
+        raise OracleError(st, "alias_build")
+    return d[:n], a[:n], b[:n], remap
+
+
+def encode_stream(symbols, rows, cdfs, lengths, offsets, W=1, fmt="rans64", precision=None,
+                  alias=False):
+    """Codes one stream; returns its bytes as a uint8 array.  alias: the
+    alias-coded variant (bucket counts powers of two; W = 1, 2, 4 or 8)."""
     s = np.ascontiguousarray(symbols, dtype=np.int64)
     r = np.ascontiguousarray(rows, dtype=np.int32)
     c = np.ascontiguousarray(cdfs, dtype=np.int32)
@@ -177,7 +205,13 @@ def encode_stream(symbols, rows, cdfs, lengths, offsets, W=1, fmt="rans64", prec
     K, Lmax = c.shape
     cap = 8 * W + 16 + 8 * s.size + 64
     out = np.zeros(cap, dtype=np.uint8)
-    if fmt == "rans64":
+    if alias:
+        if fmt not in FORMATS:
+            raise ValueError("unknown format %r" % fmt)
+        n = lib().orc_encode_stream_alias(_ptr(s), _ptr(r), s.size, _ptr(c), K, Lmax, _ptr(ln),
+                                          _ptr(of), _precision(fmt, precision), W, _ptr(out),
+                                          cap)
+    elif fmt == "rans64":
         n = lib().orc_encode_stream(_ptr(s), _ptr(r), s.size, _ptr(c), K, Lmax, _ptr(ln),
                                     _ptr(of), W, _ptr(out), cap)
     elif fmt == "rans32_16":
@@ -191,7 +225,8 @@ def encode_stream(symbols, rows, cdfs, lengths, offsets, W=1, fmt="rans64", prec
     return out[:n].copy()
 
 
-def decode_stream(data, rows, cdfs, lengths, offsets, W=1, fmt="rans64", precision=None):
+def decode_stream(data, rows, cdfs, lengths, offsets, W=1, fmt="rans64", precision=None,
+                  alias=False):
     """Decodes len(rows) symbols of one stream; returns int64 symbols."""
     d = np.ascontiguousarray(data, dtype=np.uint8)
     r = np.ascontiguousarray(rows, dtype=np.int32)
@@ -200,7 +235,13 @@ def decode_stream(data, rows, cdfs, lengths, offsets, W=1, fmt="rans64", precisi
     of = np.ascontiguousarray(offsets, dtype=np.int32)
     K, Lmax = c.shape
     out = np.zeros(r.size, dtype=np.int64)
-    if fmt == "rans64":
+    if alias:
+        if fmt not in FORMATS:
+            raise ValueError("unknown format %r" % fmt)
+        st = lib().orc_decode_stream_alias(_ptr(d), d.size, _ptr(r), r.size, _ptr(c), K, Lmax,
+                                           _ptr(ln), _ptr(of), _precision(fmt, precision), W,
+                                           _ptr(out))
+    elif fmt == "rans64":
         st = lib().orc_decode_stream(_ptr(d), d.size, _ptr(r), r.size, _ptr(c), K, Lmax,
                                      _ptr(ln), _ptr(of), W, _ptr(out))
     elif fmt == "rans32_16":
@@ -259,7 +300,7 @@ def _rows_for(positions, indexes, index_block):
 
 
 def encode_with_indexes(symbols, indexes, cdfs, lengths, offsets, chunking, W=1,
-                        index_block=1, streams=None, fmt="rans64", precision=None):
+                        index_block=1, streams=None, fmt="rans64", precision=None, alias=False):
     """Container encode: returns (bytes uint8[total], offsets uint64[S+1]).
 
     ``streams`` optionally restricts the work to a subset of stream ids; the
@@ -271,7 +312,7 @@ def encode_with_indexes(symbols, indexes, cdfs, lengths, offsets, chunking, W=1,
     for k in ids:
         p = pos[k]
         b = encode_stream(flat[p].astype(np.int64), _rows_for(p, indexes, index_block),
-                          cdfs, lengths, offsets, W, fmt, precision)
+                          cdfs, lengths, offsets, W, fmt, precision, alias)
         parts.append(b)
         offs.append(offs[-1] + b.size)
     data = np.concatenate(parts) if parts else np.zeros(0, dtype=np.uint8)
@@ -279,7 +320,8 @@ def encode_with_indexes(symbols, indexes, cdfs, lengths, offsets, chunking, W=1,
 
 
 def decode_with_indexes(data, stream_offsets, indexes, cdfs, lengths, offsets, chunking,
-                        n, W=1, index_block=1, dtype=np.int32, fmt="rans64", precision=None):
+                        n, W=1, index_block=1, dtype=np.int32, fmt="rans64", precision=None,
+                        alias=False):
     """Container decode of n elements; returns a flat array of ``dtype``."""
     pos = stream_positions(n, chunking)
     out = np.zeros(n, dtype=np.int64)
@@ -288,7 +330,7 @@ def decode_with_indexes(data, stream_offsets, indexes, cdfs, lengths, offsets, c
     for k, p in enumerate(pos):
         a, b = int(so[k]), int(so[k + 1])
         out[p] = decode_stream(d[a:b], _rows_for(p, indexes, index_block), cdfs, lengths,
-                               offsets, W, fmt, precision)
+                               offsets, W, fmt, precision, alias)
     return out.astype(dtype)
 
 

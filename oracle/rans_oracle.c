@@ -253,6 +253,7 @@ typedef struct {
     uint32_t freq;    /* SYM: cdf[v+1] - cdf[v]; 0 marks a BITS op */
     uint32_t val;     /* BITS: the 4-bit value */
     int32_t lane;     /* which interleaved state codes it */
+    int32_t row;      /* SYM: the row (for the alias mapping) */
 } op_t;
 
 typedef struct {
@@ -292,7 +293,7 @@ static int symbol_ops(int64_t s, int32_t r, int K, const int32_t *cdfs, int Lmax
     }
     int64_t freq = (int64_t)cdf[v + 1] - (int64_t)cdf[v];
     if (freq <= 0) return ORC_ERR_ZERO_FREQ;
-    op_t o = {(uint32_t)cdf[v], (uint32_t)freq, 0u, lane};
+    op_t o = {(uint32_t)cdf[v], (uint32_t)freq, 0u, lane, r};
     int st = push_op(L, o);
     if (st) return st;
     if (v == maxv) {
@@ -301,18 +302,169 @@ static int symbol_ops(int64_t s, int32_t r, int K, const int32_t *cdfs, int Lmax
         while ((raw >> (BYPASS_BITS * nb)) != 0) ++nb;
         uint32_t cnt = nb;
         while (cnt >= BYPASS_MAX) {
-            op_t b = {0u, 0u, BYPASS_MAX, lane};
+            op_t b = {0u, 0u, BYPASS_MAX, lane, r};
             if ((st = push_op(L, b))) return st;
             cnt -= BYPASS_MAX;
         }
-        op_t b = {0u, 0u, cnt, lane};
+        op_t b = {0u, 0u, cnt, lane, r};
         if ((st = push_op(L, b))) return st;
         for (uint32_t j = 0; j < nb; ++j) {
-            op_t piece = {0u, 0u, (uint32_t)((raw >> (BYPASS_BITS * j)) & BYPASS_MAX), lane};
+            op_t piece = {0u, 0u, (uint32_t)((raw >> (BYPASS_BITS * j)) & BYPASS_MAX), lane, r};
             if ((st = push_op(L, piece))) return st;
         }
     }
     return ORC_OK;
+}
+
+/* ------------------------------------------------------------- alias ----
+ * Alias coding ([TA] Usage, Alias Coding: it changes both push and pop, pop
+ * finding the symbol in constant time; Performance Tuning, GPU items 2-4:
+ * the bucket count of a row (cdf size - 1) must be a power of two, and push
+ * reads a remap table that spans the whole 2^precision range).  Reading
+ * (the pages give no construction): the 2^p cumulative positions are cut
+ * into n = cdf size - 1 slots of B = 2^p / n positions; slot j holds
+ * positions [jB, jB + d_j) of symbol j and the rest of the slot for symbol
+ * a_j.  The d_j and a_j come from Vose's alias method on the frequencies f_s:
+ * symbols with f < B form the small list and those with f > B the large one,
+ * both in ascending order and worked first-in first-out; the head of small
+ * keeps d = its remaining frequency and takes the head of large as its alias,
+ * which gives up B - d and moves to the back of small once below B (and is
+ * done, d = B, at exactly B).  Within symbol s the positions are ranked:
+ * first its own slot's [0, d_s), then its alias parts in slot order.
+ * Encoding codes symbol s on the position of rank x mod f_s (instead of
+ * cdf[s] + x mod f_s); decoding finds the slot of x mod 2^p, its symbol and
+ * rank.  A row whose every frequency is B reduces to the plain coder.
+ */
+typedef struct {
+    int logB;        /* log2 of the slot width B */
+    int32_t *d;      /* per slot: positions of the slot's own symbol */
+    int32_t *a;      /* per slot: the alias symbol of the rest */
+    int32_t *base;   /* per slot: rank (within a_j) of the rest's first position */
+    int32_t *remap;  /* 2^p entries: remap[cdf[s] + r] = position of rank r of s */
+} alias_t;
+
+int orc_alias_build(const int32_t *cdf, int len, int prec, int32_t *d, int32_t *a,
+                    int32_t *base, int32_t *remap)
+{
+    const int n = len - 1;
+    if (n < 1 || (n & (n - 1)) != 0 || prec < 1 || prec > 16) return ORC_ERR_ARG;
+    const int32_t M = (int32_t)1 << prec;
+    if (n > M || cdf[0] != 0 || cdf[n] != M) return ORC_ERR_ARG;
+    const int32_t B = M / n;
+    int32_t *rem = (int32_t *)malloc(sizeof(int32_t) * (size_t)n);
+    int32_t *small = (int32_t *)malloc(sizeof(int32_t) * (size_t)n);
+    int32_t *large = (int32_t *)malloc(sizeof(int32_t) * (size_t)n);
+    int32_t *cnt = (int32_t *)malloc(sizeof(int32_t) * (size_t)n);
+    int st = ORC_OK;
+    if (!rem || !small || !large || !cnt) { st = ORC_ERR_ARG; goto done; }
+    int ns = 0, nl = 0, hs = 0, hl = 0;
+    for (int j = 0; j < n; ++j) {
+        const int32_t f = cdf[j + 1] - cdf[j];
+        if (f <= 0) { st = ORC_ERR_ZERO_FREQ; goto done; }
+        rem[j] = f;
+        d[j] = B;
+        a[j] = j;
+        base[j] = 0;
+        if (f < B) small[ns++] = j;
+        else if (f > B) large[nl++] = j;
+    }
+    while (hs < ns && hl < nl) {
+        const int32_t l = small[hs++];
+        const int32_t g = large[hl];
+        d[l] = rem[l];
+        a[l] = g;
+        rem[g] -= B - rem[l];
+        if (rem[g] <= B) {
+            ++hl;
+            if (rem[g] < B) small[ns++] = g;   /* at exactly B it keeps d = B */
+        }
+    }
+    if (hs < ns || hl < nl) { st = ORC_ERR_ARG; goto done; }   /* cannot happen */
+    /* ranks: own part first, then alias parts in slot order */
+    for (int j = 0; j < n; ++j) cnt[j] = d[j];
+    for (int j = 0; j < n; ++j) {
+        if (d[j] == B) continue;
+        base[j] = cnt[a[j]];
+        cnt[a[j]] += B - d[j];
+    }
+    for (int j = 0; j < n; ++j)
+        if (cnt[j] != cdf[j + 1] - cdf[j]) { st = ORC_ERR_ARG; goto done; }
+    if (remap) {
+        for (int j = 0; j < n; ++j) {
+            for (int32_t o = 0; o < B; ++o) {
+                const int32_t pos = j * B + o;
+                if (o < d[j]) remap[cdf[j] + o] = pos;
+                else remap[cdf[a[j]] + base[j] + (o - d[j])] = pos;
+            }
+        }
+    }
+done:
+    free(rem);
+    free(small);
+    free(large);
+    free(cnt);
+    return st;
+}
+
+/* Alias tables of all K rows (NULL on error: a row whose bucket count is not
+ * a power of two, or a malformed row). */
+static alias_t *alias_tables(const int32_t *cdfs, int K, int Lmax, const int32_t *lengths,
+                             int prec)
+{
+    alias_t *al = (alias_t *)calloc((size_t)K, sizeof(alias_t));
+    if (!al) return NULL;
+    for (int r = 0; r < K; ++r) {
+        const int n = lengths[r] - 1;
+        const int32_t M = (int32_t)1 << prec;
+        al[r].d = (int32_t *)malloc(sizeof(int32_t) * (size_t)(n > 0 ? n : 1));
+        al[r].a = (int32_t *)malloc(sizeof(int32_t) * (size_t)(n > 0 ? n : 1));
+        al[r].base = (int32_t *)malloc(sizeof(int32_t) * (size_t)(n > 0 ? n : 1));
+        al[r].remap = (int32_t *)malloc(sizeof(int32_t) * (size_t)M);
+        int lb = 0;
+        while (n > 0 && (M / n) > (1 << lb)) ++lb;
+        al[r].logB = lb;
+        if (!al[r].d || !al[r].a || !al[r].base || !al[r].remap ||
+            orc_alias_build(cdfs + (size_t)r * (size_t)Lmax, lengths[r], prec, al[r].d, al[r].a,
+                            al[r].base, al[r].remap) != ORC_OK) {
+            for (int q = 0; q <= r; ++q) {
+                free(al[q].d); free(al[q].a); free(al[q].base); free(al[q].remap);
+            }
+            free(al);
+            return NULL;
+        }
+    }
+    return al;
+}
+
+static void alias_free(alias_t *al, int K)
+{
+    if (!al) return;
+    for (int r = 0; r < K; ++r) {
+        free(al[r].d); free(al[r].a); free(al[r].base); free(al[r].remap);
+    }
+    free(al);
+}
+
+/* The position a SYM op codes on: cdf[s] + rank, or the alias position of
+ * that rank. */
+static uint32_t code_position(const alias_t *al, const op_t *o, uint64_t rank)
+{
+    return al ? (uint32_t)al[o->row].remap[o->start + rank] : o->start + (uint32_t)rank;
+}
+
+/* The alias decoder's symbol and rank of position c in row r. */
+static void alias_lookup(const alias_t *al, int r, uint32_t c, int32_t *v, uint32_t *rank)
+{
+    const alias_t *t = &al[r];
+    const uint32_t j = c >> t->logB;
+    const uint32_t o = c & ((1u << t->logB) - 1u);
+    if (o < (uint32_t)t->d[j]) {
+        *v = (int32_t)j;
+        *rank = o;
+    } else {
+        *v = t->a[j];
+        *rank = (uint32_t)t->base[j] + (o - (uint32_t)t->d[j]);
+    }
 }
 
 /* ------------------------------------------------------------ O5 / O7 ----
@@ -352,10 +504,10 @@ static int push_word(words_t *W, uint32_t v)
     return ORC_OK;
 }
 
-int64_t orc_encode_stream(const int64_t *sym, const int32_t *row, int64_t n,
-                          const int32_t *cdfs, int K, int Lmax,
-                          const int32_t *lengths, const int32_t *offsets,
-                          int W, uint8_t *out, int64_t cap)
+static int64_t encode64(const int64_t *sym, const int32_t *row, int64_t n,
+                        const int32_t *cdfs, int K, int Lmax,
+                        const int32_t *lengths, const int32_t *offsets,
+                        int W, uint8_t *out, int64_t cap, const alias_t *al)
 {
     if (!valid_interleave(W)) return ORC_ERR_ARG;
     if (n < 0) return ORC_ERR_ARG;
@@ -381,7 +533,7 @@ int64_t orc_encode_stream(const int64_t *sym, const int32_t *row, int64_t n,
                 if (push_word(&words, (uint32_t)*s)) { result = ORC_ERR_ARG; goto done; }
                 *s >>= 32;
             }
-            *s = ((*s / o->freq) << PREC) + (*s % o->freq) + o->start;
+            *s = ((*s / o->freq) << PREC) + code_position(al, o, *s % o->freq);
         } else {
             uint64_t xmax = (uint64_t)1 << 59;
             if (*s >= xmax) {
@@ -455,10 +607,10 @@ static int get_bits(uint64_t *x, reader_t *R, uint32_t *val)
     return refill(x, R);
 }
 
-int orc_decode_stream(const uint8_t *in, int64_t len, const int32_t *row, int64_t n,
-                      const int32_t *cdfs, int K, int Lmax,
-                      const int32_t *lengths, const int32_t *offsets,
-                      int W, int64_t *sym_out)
+static int decode64(const uint8_t *in, int64_t len, const int32_t *row, int64_t n,
+                    const int32_t *cdfs, int K, int Lmax,
+                    const int32_t *lengths, const int32_t *offsets,
+                    int W, int64_t *sym_out, const alias_t *al)
 {
     if (!valid_interleave(W)) return ORC_ERR_ARG;
     reader_t R = {in, len, 0};
@@ -477,13 +629,19 @@ int orc_decode_stream(const uint8_t *in, int64_t len, const int32_t *row, int64_
         uint64_t *s = &x[i % W];
 
         uint32_t cum = (uint32_t)(*s & (TOTAL - 1));
-        int j = 1;
-        while (j < Lr && (uint32_t)cdf[j] <= cum) ++j;
-        if (j >= Lr) return ORC_ERR_CORRUPT;    /* a malformed row */
-        int32_t v = j - 1;
-        uint32_t start = (uint32_t)cdf[v];
+        int32_t v;
+        uint32_t rank;
+        if (al) {
+            alias_lookup(al, r, cum, &v, &rank);
+        } else {
+            int j = 1;
+            while (j < Lr && (uint32_t)cdf[j] <= cum) ++j;
+            if (j >= Lr) return ORC_ERR_CORRUPT;    /* a malformed row */
+            v = j - 1;
+            rank = cum - (uint32_t)cdf[v];
+        }
         uint32_t freq = (uint32_t)(cdf[v + 1] - cdf[v]);
-        *s = (uint64_t)freq * (*s >> PREC) + cum - start;
+        *s = (uint64_t)freq * (*s >> PREC) + rank;
         int st = refill(s, &R);
         if (st) return st;
 
@@ -511,6 +669,22 @@ int orc_decode_stream(const uint8_t *in, int64_t len, const int32_t *row, int64_
     for (int l = 0; l < W; ++l)
         if (x[l] != RANS_L) return ORC_ERR_CORRUPT;
     return ORC_OK;
+}
+
+int64_t orc_encode_stream(const int64_t *sym, const int32_t *row, int64_t n,
+                          const int32_t *cdfs, int K, int Lmax,
+                          const int32_t *lengths, const int32_t *offsets,
+                          int W, uint8_t *out, int64_t cap)
+{
+    return encode64(sym, row, n, cdfs, K, Lmax, lengths, offsets, W, out, cap, NULL);
+}
+
+int orc_decode_stream(const uint8_t *in, int64_t len, const int32_t *row, int64_t n,
+                      const int32_t *cdfs, int K, int Lmax,
+                      const int32_t *lengths, const int32_t *offsets,
+                      int W, int64_t *sym_out)
+{
+    return decode64(in, len, row, n, cdfs, K, Lmax, lengths, offsets, W, sym_out, NULL);
 }
 
 /* ------------------------------------------------------------ rans32_16 ----
@@ -553,10 +727,10 @@ static int push_word16(words16_t *W, uint16_t v)
 }
 
 
-int64_t orc_encode_stream16(const int64_t *sym, const int32_t *row, int64_t n,
-                            const int32_t *cdfs, int K, int Lmax,
-                            const int32_t *lengths, const int32_t *offsets,
-                            int prec, int W, uint8_t *out, int64_t cap)
+static int64_t encode16(const int64_t *sym, const int32_t *row, int64_t n,
+                        const int32_t *cdfs, int K, int Lmax,
+                        const int32_t *lengths, const int32_t *offsets,
+                        int prec, int W, uint8_t *out, int64_t cap, const alias_t *al)
 {
     if (!valid_interleave(W) || n < 0 || prec < 1 || prec > 15) return ORC_ERR_ARG;
     oplist_t ops = {NULL, 0, 0};
@@ -581,7 +755,7 @@ int64_t orc_encode_stream16(const int64_t *sym, const int32_t *row, int64_t n,
             *s >>= 16;
         }
         if (o->freq)
-            *s = ((*s / o->freq) << prec) + (*s % o->freq) + o->start;
+            *s = ((*s / o->freq) << prec) + code_position(al, o, *s % o->freq);
         else
             *s = (*s << BYPASS_BITS) | o->val;
     }
@@ -631,10 +805,10 @@ static int get_bits16(uint32_t *x, reader_t *R, uint32_t *val)
     return refill16(x, R);
 }
 
-int orc_decode_stream16(const uint8_t *in, int64_t len, const int32_t *row, int64_t n,
-                        const int32_t *cdfs, int K, int Lmax,
-                        const int32_t *lengths, const int32_t *offsets,
-                        int prec, int W, int64_t *sym_out)
+static int decode16(const uint8_t *in, int64_t len, const int32_t *row, int64_t n,
+                    const int32_t *cdfs, int K, int Lmax,
+                    const int32_t *lengths, const int32_t *offsets,
+                    int prec, int W, int64_t *sym_out, const alias_t *al)
 {
     if (!valid_interleave(W) || prec < 1 || prec > 15) return ORC_ERR_ARG;
     reader_t R = {in, len, 0};
@@ -654,13 +828,19 @@ int orc_decode_stream16(const uint8_t *in, int64_t len, const int32_t *row, int6
         uint32_t *s = &x[i % W];
 
         uint32_t cum = *s & mask;
-        int j = 1;
-        while (j < Lr && (uint32_t)cdf[j] <= cum) ++j;
-        if (j >= Lr) return ORC_ERR_CORRUPT;    /* a malformed row */
-        int32_t v = j - 1;
-        uint32_t start = (uint32_t)cdf[v];
+        int32_t v;
+        uint32_t rank;
+        if (al) {
+            alias_lookup(al, r, cum, &v, &rank);
+        } else {
+            int j = 1;
+            while (j < Lr && (uint32_t)cdf[j] <= cum) ++j;
+            if (j >= Lr) return ORC_ERR_CORRUPT;    /* a malformed row */
+            v = j - 1;
+            rank = cum - (uint32_t)cdf[v];
+        }
         uint32_t freq = (uint32_t)(cdf[v + 1] - cdf[v]);
-        *s = freq * (*s >> prec) + cum - start;
+        *s = freq * (*s >> prec) + rank;
         int st = refill16(s, &R);
         if (st) return st;
 
@@ -688,4 +868,54 @@ int orc_decode_stream16(const uint8_t *in, int64_t len, const int32_t *row, int6
     for (int l = 0; l < W; ++l)
         if (x[l] != R16_L) return ORC_ERR_CORRUPT;
     return ORC_OK;
+}
+
+int64_t orc_encode_stream16(const int64_t *sym, const int32_t *row, int64_t n,
+                            const int32_t *cdfs, int K, int Lmax,
+                            const int32_t *lengths, const int32_t *offsets,
+                            int prec, int W, uint8_t *out, int64_t cap)
+{
+    return encode16(sym, row, n, cdfs, K, Lmax, lengths, offsets, prec, W, out, cap, NULL);
+}
+
+int orc_decode_stream16(const uint8_t *in, int64_t len, const int32_t *row, int64_t n,
+                        const int32_t *cdfs, int K, int Lmax,
+                        const int32_t *lengths, const int32_t *offsets,
+                        int prec, int W, int64_t *sym_out)
+{
+    return decode16(in, len, row, n, cdfs, K, Lmax, lengths, offsets, prec, W, sym_out, NULL);
+}
+
+/* Alias-coded streams (see "alias" above) in either format: prec 16 codes
+ * the 64-bit format, prec <= 15 the rans32_16 one.  Every row's bucket count
+ * must be a power of two (else ORC_ERR_ARG).  The pages list the alias coder
+ * for 1, 2, 4 and 8 interleaved states. */
+int64_t orc_encode_stream_alias(const int64_t *sym, const int32_t *row, int64_t n,
+                                const int32_t *cdfs, int K, int Lmax,
+                                const int32_t *lengths, const int32_t *offsets,
+                                int prec, int W, uint8_t *out, int64_t cap)
+{
+    if (W != 1 && W != 2 && W != 4 && W != 8) return ORC_ERR_ARG;
+    alias_t *al = alias_tables(cdfs, K, Lmax, lengths, prec);
+    if (!al) return ORC_ERR_ARG;
+    int64_t st = prec == 16
+        ? encode64(sym, row, n, cdfs, K, Lmax, lengths, offsets, W, out, cap, al)
+        : encode16(sym, row, n, cdfs, K, Lmax, lengths, offsets, prec, W, out, cap, al);
+    alias_free(al, K);
+    return st;
+}
+
+int orc_decode_stream_alias(const uint8_t *in, int64_t len, const int32_t *row, int64_t n,
+                            const int32_t *cdfs, int K, int Lmax,
+                            const int32_t *lengths, const int32_t *offsets,
+                            int prec, int W, int64_t *sym_out)
+{
+    if (W != 1 && W != 2 && W != 4 && W != 8) return ORC_ERR_ARG;
+    alias_t *al = alias_tables(cdfs, K, Lmax, lengths, prec);
+    if (!al) return ORC_ERR_ARG;
+    int st = prec == 16
+        ? decode64(in, len, row, n, cdfs, K, Lmax, lengths, offsets, W, sym_out, al)
+        : decode16(in, len, row, n, cdfs, K, Lmax, lengths, offsets, prec, W, sym_out, al);
+    alias_free(al, K);
+    return st;
 }

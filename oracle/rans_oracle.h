@@ -76,6 +76,23 @@ int orc_decode_stream16(const uint8_t *in, int64_t len, const int32_t *row, int6
                         const int32_t *lengths, const int32_t *offsets,
                         int prec, int W, int64_t *sym_out);
 
+/* Alias table of one row of len entries at precision prec (len - 1 a power
+ * of two): per slot d, a, base (len - 1 entries each) and, unless NULL, the
+ * 2^prec-entry remap. */
+int orc_alias_build(const int32_t *cdf, int len, int prec, int32_t *d, int32_t *a,
+                    int32_t *base, int32_t *remap);
+
+/* Alias-coded streams: prec 16 = the 64-bit format, <= 15 = rans32_16;
+ * W = 1, 2, 4 or 8. */
+int64_t orc_encode_stream_alias(const int64_t *sym, const int32_t *row, int64_t n,
+                                const int32_t *cdfs, int K, int Lmax,
+                                const int32_t *lengths, const int32_t *offsets,
+                                int prec, int W, uint8_t *out, int64_t cap);
+int orc_decode_stream_alias(const uint8_t *in, int64_t len, const int32_t *row, int64_t n,
+                            const int32_t *cdfs, int K, int Lmax,
+                            const int32_t *lengths, const int32_t *offsets,
+                            int prec, int W, int64_t *sym_out);
+
 #ifdef __cplusplus
 }
 #endif
