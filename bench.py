@@ -65,6 +65,8 @@ def parse():
     ap.add_argument("--interleave", type=int, default=None, help="W for --workload y")
     ap.add_argument("--format", choices=["rans64", "rans32_16"], default=None,
                     help="coder format (default: rans32_16 for --workload r16, else rans64)")
+    ap.add_argument("--alias", action="store_true",
+                    help="alias-coded streams (rows of power-of-two bucket counts, W <= 8)")
     return ap.parse_args()
 
 
@@ -210,18 +212,20 @@ def load_inputs(rank, group, images=N_IMAGES, workload="batch", interleave=None)
     return w
 
 
-def apply_format(w, fmt):
+def apply_format(w, fmt, alias=False):
     """Sets the coder format (and its row precision) on a workload dict."""
     fmt = fmt or w.get("fmt", "rans64")
     w["fmt"] = fmt
     w["precision"] = 15 if fmt == "rans32_16" else 16
+    w["alias"] = bool(alias)
     return w
 
 
 def workload_name(w, args):
-    if w.get("fmt", "rans64") != "rans64":
-        return "%s [%s, precision %d]" % (workload_name(dict(w, fmt="rans64"), args), w["fmt"],
-                                          w["precision"])
+    if w.get("fmt", "rans64") != "rans64" or w.get("alias"):
+        return "%s [%s%s, precision %d]" % (
+            workload_name(dict(w, fmt="rans64", alias=False), args), w["fmt"],
+            " alias" if w.get("alias") else "", w["precision"])
     if args.workload == "batch":
         return WORKLOAD
     if args.workload == "float":
@@ -242,7 +246,7 @@ def oracle_sample(w, max_streams, workers):
     workload, one stream per call, spread over `workers` threads (the C
     oracle runs without the GIL).  Returns (symbols coded, seconds)."""
     import oracle as O
-    fmt, prec = w.get("fmt", "rans64"), w.get("precision", 16)
+    fmt, prec, alias = w.get("fmt", "rans64"), w.get("precision", 16), w.get("alias", False)
     if "scales" in w:
         c, l, o = O.build_cdfs_from_scales(w["scales"], w["tail_mass"], precision=prec)
     else:
@@ -257,8 +261,8 @@ def oracle_sample(w, max_streams, workers):
     def one(p):
         s = flat[p].astype(np.int64)
         r = idx[p // blk]
-        b = O.encode_stream(s, r, c, l, o, W=W, fmt=fmt, precision=prec)
-        back = O.decode_stream(b, r, c, l, o, W=W, fmt=fmt, precision=prec)
+        b = O.encode_stream(s, r, c, l, o, W=W, fmt=fmt, precision=prec, alias=alias)
+        back = O.decode_stream(b, r, c, l, o, W=W, fmt=fmt, precision=prec, alias=alias)
         assert np.array_equal(back, s)
         return p.size
 
@@ -273,7 +277,7 @@ def run_reference(args, world, rank):
     if rank != 0:
         return
     w = apply_format(load_inputs(0, args.group, workload=args.workload,
-                                 interleave=args.interleave), args.format)
+                                 interleave=args.interleave), args.format, args.alias)
     if args.workload == "float":  # the oracle codes rows and symbols computed first
         import oracle as O
         w = dict(w, symbols=O.quantize(w["y"], w["means"]), W=32,
@@ -314,14 +318,15 @@ def run_ours(args, world, rank, local):
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
     w = apply_format(load_inputs(rank, args.group, args.images, args.workload, args.interleave),
-                     args.format)
+                     args.format, args.alias)
     fmt, prec = w["fmt"], w["precision"]
     sym_np = np.ascontiguousarray(np.asarray(w["symbols"]).reshape(-1))
     idx_np = np.ascontiguousarray(w["indexes"], dtype=np.int32)
     n = sym_np.size
     sym = torch.from_numpy(sym_np).to(dev)
     idx = torch.from_numpy(idx_np).to(dev)
-    ch = rb.Chunking.from_spec(w["chunking"], w["W"], w["index_block"], device=dev, fmt=fmt)
+    ch = rb.Chunking.from_spec(w["chunking"], w["W"], w["index_block"], device=dev, fmt=fmt,
+                               alias=w["alias"])
     S = rb.rans_num_streams(ch, n)
 
     # tables: sized once; rebuilt inside every step (from the scale table, or
@@ -346,6 +351,8 @@ def run_ours(args, world, rank, local):
                                                   precision=prec), "cdfs")
     K, Lmax = cdfs.shape
     tables = rb.Tables(cdfs, lengths, offsets, precision=prec)
+    if w["alias"]:  # built once, before timing: the rows do not change between steps
+        tables.prepare_alias()
     blob = tables.blob
     ws = rb.Workspaces(ch, n, dev)
     dec = torch.empty_like(sym)

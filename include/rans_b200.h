@@ -95,6 +95,23 @@ enum { RANS_CHUNK_CONTIG = 0, RANS_CHUNK_EXPLICIT = 1, RANS_CHUNK_TILED = 2 };
 enum { RANS_FMT_RANS64 = 0, RANS_FMT_RANS32_16 = 1 };
 
 /*
+ * RANS_FMT_ALIAS, or'ed into the format: alias-coded streams ("torch_ans
+ * 0.3.0", Usage, Alias Coding: push and pop both change, pop finds the symbol
+ * in constant time; Performance Tuning: a row's bucket count, cdf_length - 1,
+ * must be a power of two; 1, 2, 4 or 8 interleaved states, no 32-way form).
+ * The library's reading of the method (the pages give no construction):
+ * the 2^p positions are cut into n = cdf_length - 1 slots of 2^p / n; Vose's
+ * alias method (first-in first-out worklists of the symbols below and above
+ * the slot width, each in ascending order) leaves slot j with d_j positions
+ * of symbol j and the rest for an alias symbol; a symbol ranks its own slot's
+ * positions first, then its alias parts in slot order.  The encoder codes
+ * symbol s on the position of rank x mod f_s (x -> (x / f) 2^p + position),
+ * the decoder reads symbol and rank from the slot of x mod 2^p
+ * (x -> f (x >> p) + rank).  Needs alias tables (rans_alias_prepare).
+ */
+enum { RANS_FMT_ALIAS = 0x100 };
+
+/*
  * How the n symbols are cut into streams, and how indexes map to symbols.
  *   CONTIG:   n_streams streams; stream k covers elements
  *             [k*ceil(n/S), min((k+1)*ceil(n/S), n)) (trailing streams may be
@@ -152,6 +169,10 @@ typedef struct rans_tables {
                                global */
     int32_t device;         /* CUDA device the blob lives on */
     int32_t precision;      /* the rows sum to 2^precision */
+    int32_t reserved;
+    void *alias;            /* alias tables (rans_alias_prepare), or NULL */
+    uint64_t alias_bytes;
+    uint64_t alias_remap_offset;  /* byte offset of the remap entries in `alias` */
 } rans_tables;
 
 /* ------------------------------------------------------------ status ---- */
@@ -250,6 +271,22 @@ int rans_tables_prepare(const int32_t *cdfs, int32_t K, int32_t Lmax,
 int rans_tables_refresh(const int32_t *cdfs, int32_t K, int32_t Lmax,
                         const int32_t *cdf_lengths, const int32_t *offsets,
                         const rans_tables *tables, void *stream);
+
+/* Bytes of the alias tables of a prepared table set: 8 bytes per bucket
+ * (slot words) and 2^precision 16-bit remap entries per row. */
+uint64_t rans_alias_bytes(const rans_tables *tables);
+
+/*
+ * Builds the alias tables (see RANS_FMT_ALIAS) of a prepared table set from
+ * the rows it was prepared from, into the caller's device buffer `alias`
+ * (256-byte aligned, >= rans_alias_bytes), and records it in *tables.  Every
+ * row's bucket count (cdf_length - 1) must be a power of two of at most 8192
+ * (else RANS_ERR_ARG).  Synchronous: reads back the lengths and the status.
+ *   cdfs, cdf_lengths: as for rans_tables_prepare (same rows).
+ */
+int rans_alias_prepare(const int32_t *cdfs, int32_t K, int32_t Lmax,
+                       const int32_t *cdf_lengths, rans_tables *tables, void *alias,
+                       uint64_t alias_bytes, void *stream);
 
 /* ------------------------------------------------- sizes and queries ---- */
 

@@ -6,11 +6,11 @@ See include/rans_b200.h for the boundary.  Build the library with
 """
 from ._lib import (  # noqa: F401
     CHUNK_CONTIG, CHUNK_EXPLICIT, CHUNK_TILED, ERR_ARG, ERR_CAPACITY, ERR_CORRUPT, ERR_CUDA,
-    FMT_RANS32_16, FMT_RANS64,
+    FMT_ALIAS, FMT_RANS32_16, FMT_RANS64,
     ERR_INDEX, ERR_RANGE, ERR_TABLE, ERR_TIMEOUT, ERR_ZERO_FREQ, LIB_PATH, OK, SIGNATURES,
     SYM_INT16, SYM_INT32, SYM_UINT8, Chunking, RansError, Tables, Workspaces, aligned_empty,
     check, decode_to_values, decode_with_indexes, encode_from_scales, encode_with_indexes, lib,
-    rans_build_cdfs_from_pmfs, rans_build_indexes, rans_decode_to_values,
+    rans_alias_bytes, rans_alias_prepare, rans_build_cdfs_from_pmfs, rans_build_indexes, rans_decode_to_values,
     rans_encode_from_scales,
     rans_build_cdfs_from_scales, rans_chunking, rans_debug_divide, rans_decode_with_indexes,
     rans_decode_workspace_bytes, rans_encode_with_indexes, rans_encode_with_indexes_noalloc,

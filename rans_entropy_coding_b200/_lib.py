@@ -34,6 +34,7 @@ CHUNK_CONTIG, CHUNK_EXPLICIT, CHUNK_TILED = 0, 1, 2
 # coder formats: 64-bit state / 32-bit words / precision 16, and 32-bit
 # state / 16-bit words / precision <= 15
 FMT_RANS64, FMT_RANS32_16 = 0, 1
+FMT_ALIAS = 0x100  # or'ed into a format: alias-coded streams
 _FMT_CODE = {"rans64": FMT_RANS64, "rans32_16": FMT_RANS32_16}
 
 _DTYPE_CODE = {torch.int32: SYM_INT32, torch.uint8: SYM_UINT8, torch.int16: SYM_INT16}
@@ -56,7 +57,9 @@ class rans_tables(ctypes.Structure):
                 ("start_bytes", ctypes.c_uint32), ("slot_bytes", ctypes.c_uint32),
                 ("enc_in_smem", ctypes.c_int32),
                 ("dec_in_smem", ctypes.c_int32), ("device", ctypes.c_int32),
-                ("precision", ctypes.c_int32)]
+                ("precision", ctypes.c_int32), ("reserved", ctypes.c_int32),
+                ("alias", ctypes.c_void_p), ("alias_bytes", ctypes.c_uint64),
+                ("alias_remap_offset", ctypes.c_uint64)]
 
 
 # (name, restype, argtypes) for every exported symbol of include/rans_b200.h
@@ -74,6 +77,8 @@ SIGNATURES = [
     ("rans_tables_bytes", _U64, [_I32, _I32]),
     ("rans_tables_prepare", ctypes.c_int, [_P, _I32, _I32, _P, _P, _I32, _P, _U64, _TBP, _P]),
     ("rans_tables_refresh", ctypes.c_int, [_P, _I32, _I32, _P, _P, _TBP, _P]),
+    ("rans_alias_bytes", _U64, [_TBP]),
+    ("rans_alias_prepare", ctypes.c_int, [_P, _I32, _I32, _P, _TBP, _P, _U64, _P]),
     ("rans_num_streams", _I64, [_CHP, _I64]),
     ("rans_encode_workspace_bytes", _U64, [_CHP, _I64]),
     ("rans_decode_workspace_bytes", _U64, [_CHP, _I64]),
@@ -181,6 +186,17 @@ def rans_tables_refresh(cdfs, cdf_lengths, offsets, tables, stream=None):
                                      _ptr(offsets), ctypes.byref(tables.c), _stream(stream))
 
 
+def rans_alias_bytes(tables):
+    return lib().rans_alias_bytes(ctypes.byref(tables.c))
+
+
+def rans_alias_prepare(cdfs, cdf_lengths, tables, alias, stream=None):
+    _need_cuda(cdfs, cdf_lengths, alias)
+    return lib().rans_alias_prepare(_ptr(cdfs), cdfs.shape[0], cdfs.shape[1], _ptr(cdf_lengths),
+                                    ctypes.byref(tables.c), _ptr(alias), alias.numel(),
+                                    _stream(stream))
+
+
 def rans_num_streams(chunking, n):
     return lib().rans_num_streams(ctypes.byref(chunking.c), n)
 
@@ -272,15 +288,19 @@ class Chunking:
         return self.c.interleave
 
     @staticmethod
-    def contig(n_streams, interleave=1, index_block=1, fmt="rans64"):
+    def _format(fmt, alias):
+        return _FMT_CODE[fmt] | (FMT_ALIAS if alias else 0)
+
+    @staticmethod
+    def contig(n_streams, interleave=1, index_block=1, fmt="rans64", alias=False):
         c = rans_chunking()
         c.kind, c.interleave, c.n_streams, c.index_block = (CHUNK_CONTIG, interleave, n_streams,
                                                             index_block)
-        c.format = _FMT_CODE[fmt]
+        c.format = Chunking._format(fmt, alias)
         return Chunking(c)
 
     @staticmethod
-    def explicit(starts, interleave=1, index_block=1, fmt="rans64"):
+    def explicit(starts, interleave=1, index_block=1, fmt="rans64", alias=False):
         """starts: CUDA int64 tensor of S + 1 element offsets."""
         _need_cuda(starts)
         assert starts.dtype == torch.int64
@@ -288,31 +308,32 @@ class Chunking:
         c.kind, c.interleave, c.n_streams, c.index_block = (CHUNK_EXPLICIT, interleave,
                                                             starts.numel() - 1, index_block)
         c.stream_starts = starts.data_ptr()
-        c.format = _FMT_CODE[fmt]
+        c.format = Chunking._format(fmt, alias)
         return Chunking(c, keep=starts)
 
     @staticmethod
-    def tiled(shape, group, tile_h, tile_w, interleave=32, index_block=1, fmt="rans64"):
+    def tiled(shape, group, tile_h, tile_w, interleave=32, index_block=1, fmt="rans64",
+              alias=False):
         c = rans_chunking()
         c.kind, c.interleave, c.index_block = CHUNK_TILED, interleave, index_block
         for i, v in enumerate(shape):
             c.shape[i] = int(v)
         c.group, c.tile_h, c.tile_w = group, tile_h, tile_w
-        c.format = _FMT_CODE[fmt]
+        c.format = Chunking._format(fmt, alias)
         return Chunking(c)
 
     @staticmethod
-    def from_spec(spec, interleave, index_block=1, device="cuda", fmt="rans64"):
+    def from_spec(spec, interleave, index_block=1, device="cuda", fmt="rans64", alias=False):
         """From the dict form used by the workloads module."""
         k = spec["kind"]
         if k == "contig":
-            return Chunking.contig(spec["n_streams"], interleave, index_block, fmt)
+            return Chunking.contig(spec["n_streams"], interleave, index_block, fmt, alias)
         if k == "tiled":
             return Chunking.tiled(spec["shape"], spec["cg"], spec["th"], spec["tw"], interleave,
-                                  index_block, fmt)
+                                  index_block, fmt, alias)
         if k == "explicit":
             st = torch.as_tensor(spec["starts"], dtype=torch.int64, device=device)
-            return Chunking.explicit(st, interleave, index_block, fmt)
+            return Chunking.explicit(st, interleave, index_block, fmt, alias)
         raise ValueError(k)
 
 
@@ -334,6 +355,15 @@ class Tables:
         self.c = rans_tables()
         check(rans_tables_prepare(cdfs, cdf_lengths, offsets, self.blob, self.c, stream,
                                   precision), "tables_prepare")
+
+    def prepare_alias(self, stream=None):
+        """Builds the alias tables (every row's bucket count a power of two)
+        for alias-coded streams (Chunking(..., alias=True))."""
+        nbytes = rans_alias_bytes(self)
+        self.alias = aligned_empty(nbytes, self.cdfs.device)
+        check(rans_alias_prepare(self.cdfs, self.cdf_lengths, self, self.alias, stream),
+              "alias_prepare")
+        return self
 
     @staticmethod
     def build_from_scales(scales, tail_mass=1e-9, stream=None, precision=16):

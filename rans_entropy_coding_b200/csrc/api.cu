@@ -47,10 +47,14 @@ int make_geom(const rans_chunking *ch, int64_t n, Geom &g) {
       ch->interleave != 32)
     return RANS_ERR_ARG;
   if (!is_pow2(ch->index_block)) return RANS_ERR_ARG;
-  if (ch->format != RANS_FMT_RANS64 && ch->format != RANS_FMT_RANS32_16) return RANS_ERR_ARG;
+  const int base_fmt = ch->format & ~RANS_FMT_ALIAS;
+  const bool alias = (ch->format & RANS_FMT_ALIAS) != 0;
+  if (base_fmt != RANS_FMT_RANS64 && base_fmt != RANS_FMT_RANS32_16) return RANS_ERR_ARG;
+  if (alias && ch->interleave == 32) return RANS_ERR_ARG;  // no 32-way alias coder
   std::memset(&g, 0, sizeof(g));
   g.kind = ch->kind;
-  g.fmt = ch->format;
+  g.fmt = base_fmt;
+  g.alias = alias ? 1 : 0;
   g.W = ch->interleave;
   g.n = n;
   int ib = 0;
@@ -151,8 +155,10 @@ bool tables_usable(const rans_tables *t) {
   return true;
 }
 
-// RANS64 codes rows of precision 16, RANS32_16 rows of precision <= 15.
+// RANS64 codes rows of precision 16, RANS32_16 rows of precision <= 15;
+// alias coding needs the alias tables.
 bool format_fits(const Geom &g, const rans_tables *t) {
+  if (g.alias && t->alias == nullptr) return false;
   return g.fmt == RANS_FMT_RANS64 ? t->precision == 16 : t->precision <= 15;
 }
 
@@ -232,6 +238,21 @@ RANS_API int rans_tables_refresh(const int32_t *cdfs, int32_t K, int32_t Lmax,
   if (!tables_usable(tables) || K != tables->K || Lmax < 2 || !cdfs || !cdf_lengths || !offsets)
     return RANS_ERR_ARG;
   return rb::refresh_tables(cdfs, K, Lmax, cdf_lengths, offsets, *tables, as_stream(stream));
+}
+
+RANS_API uint64_t rans_alias_bytes(const rans_tables *tables) {
+  if (!tables || tables->K < 1 || tables->precision < 1 || tables->precision > 16) return 0;
+  return ((8ull * (uint64_t)tables->n_buckets + 255) & ~255ull) +
+         2ull * (uint64_t)tables->K * (1ull << tables->precision);
+}
+
+RANS_API int rans_alias_prepare(const int32_t *cdfs, int32_t K, int32_t Lmax,
+                                const int32_t *cdf_lengths, rans_tables *tables, void *alias,
+                                uint64_t alias_bytes, void *stream) {
+  if (!tables_usable(tables) || K != tables->K || Lmax < 2 || !cdfs || !cdf_lengths || !alias)
+    return RANS_ERR_ARG;
+  return rb::prepare_alias(cdfs, K, Lmax, cdf_lengths, *tables, alias, alias_bytes,
+                           as_stream(stream));
 }
 
 RANS_API int64_t rans_num_streams(const rans_chunking *chunking, int64_t n) {

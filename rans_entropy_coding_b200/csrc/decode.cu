@@ -49,6 +49,7 @@ struct DecCtx {
   const int32_t *idx;
   int32_t K;
   uint32_t sh;  // 16 - precision of the rows (Rans32; 0 for Rans64)
+  const uint2 *aslots;  // alias coding: the slot words (at the bucket indexes)
   uint32_t meta_bytes, bucket_bytes, start_bytes, slot_bytes;
   const char *blob;
   Geom g;
@@ -601,8 +602,9 @@ __device__ __forceinline__ EscapeResult<F> escape_group_seg(
 }
 
 // One segment's stream (s < 0: an idle segment, still taking part in the
-// warp's votes and shuffles).
-template <class F, typename SymT, bool ROWS>
+// warp's votes and shuffles).  ALIAS: alias-coded streams (the slot of the
+// position gives symbol and rank).
+template <class F, typename SymT, bool ROWS, bool ALIAS>
 __device__ void decode_segment(const DecCtx &c, const RowMeta *meta, const uint16_t *starts,
                                const uint32_t *slots, int64_t s, int W) {
   using State = typename F::State;
@@ -655,11 +657,12 @@ __device__ void decode_segment(const DecCtx &c, const RowMeta *meta, const uint1
     bad_index |= active && r > kmax;
     const RowMeta m = row_meta(meta, active && r <= kmax ? r : 0u);
     const uint32_t cum = F::cum16(x, sh);
-    const uint32_t sym =
-        ROWS ? search_row(cum, m, starts) : lookup<true, true>(cum, m, starts, slots, active);
+    uint32_t sym, rank = 0;
+    if constexpr (ALIAS) sym = alias_lookup(cum >> sh, m, c.aslots, kPrec - sh, rank);
+    else sym = ROWS ? search_row(cum, m, starts) : lookup<true, true>(cum, m, starts, slots, active);
     const uint32_t start = starts[m.bucket_base + sym];
     const uint32_t freq = width_of(start, starts[m.bucket_base + sym + 1]);
-    State y = F::dec_step(x, cum, start, freq, sh);
+    State y = ALIAS ? F::dec_rank_step(x, freq, rank, sh) : F::dec_step(x, cum, start, freq, sh);
     if (!active) y = x;
     const bool esc = active && sym == m.maxv;
     const bool need = active && y < F::kLow;
@@ -762,7 +765,7 @@ __global__ void __launch_bounds__(W == 32 ? kDecMaxThreads32 : kDecThreads1)
 // a run-time argument.
 constexpr int kSegThreads = 256;
 
-template <class F, typename SymT>
+template <class F, typename SymT, bool ALIAS>
 __global__ void __launch_bounds__(kSegThreads) decode_kernel_wn(DecCtx c, int mode) {
   extern __shared__ __align__(16) unsigned char smem[];
   __shared__ uint64_t bar;
@@ -789,15 +792,15 @@ __global__ void __launch_bounds__(kSegThreads) decode_kernel_wn(DecCtx c, int mo
     const int64_t k = k0 + seg;
     const int64_t s = k < c.g.S ? stream_of(c.g, k) : -1;
     if (mode == 2)
-      decode_segment<F, SymT, true>(c, meta, buckets, slots, s, W);
+      decode_segment<F, SymT, true, ALIAS>(c, meta, buckets, slots, s, W);
     else
-      decode_segment<F, SymT, false>(c, meta, buckets, slots, s, W);
+      decode_segment<F, SymT, false, ALIAS>(c, meta, buckets, slots, s, W);
   }
 }
 
-template <class F, typename SymT>
+template <class F, typename SymT, bool ALIAS>
 int launch_decode_wn(const DecCtx &c, int mode, cudaStream_t st) {
-  auto kern = decode_kernel_wn<F, SymT>;
+  auto kern = decode_kernel_wn<F, SymT, ALIAS>;
   const uint32_t tab = dec_table_bytes(mode, c);
   int dev = 0;
   cudaGetDevice(&dev);
@@ -891,9 +894,10 @@ int launch_decode_w(const DecCtx &c, int mode, cudaStream_t st) {
 
 template <class F, typename SymT>
 int launch_decode_f(const DecCtx &c, int mode, cudaStream_t st) {
+  if (c.g.alias) return launch_decode_wn<F, SymT, true>(c, mode, st);  // W = 1, 2, 4, 8
   if (c.g.W == 32) return launch_decode_w<F, 32, SymT>(c, mode, st);
   if (c.g.W == 1) return launch_decode_w<F, 1, SymT>(c, mode, st);
-  return launch_decode_wn<F, SymT>(c, mode, st);
+  return launch_decode_wn<F, SymT, false>(c, mode, st);
 }
 
 template <typename SymT>
@@ -915,6 +919,7 @@ int launch_decode_float(const uint8_t *in, uint64_t in_bytes, const uint64_t *of
   c.idx = nullptr;
   c.K = t.K;
   c.sh = 0;
+  c.aslots = nullptr;
   c.meta_bytes = t.meta_bytes;
   c.bucket_bytes = t.bucket_bytes;
   c.start_bytes = t.start_bytes;
@@ -942,6 +947,7 @@ int launch_decode(const uint8_t *in, uint64_t in_bytes, const uint64_t *offsets,
   c.idx = indexes;
   c.K = t.K;
   c.sh = (uint32_t)(kPrec - t.precision);
+  c.aslots = g.alias ? reinterpret_cast<const uint2 *>(t.alias) : nullptr;
   c.meta_bytes = t.meta_bytes;
   c.bucket_bytes = t.bucket_bytes;
   c.start_bytes = t.start_bytes;

@@ -51,6 +51,7 @@ struct EncCtx {
   int32_t stab_smem; // 1: the kernel copies the scale table into shared memory
   int32_t K;
   uint32_t sh;       // 16 - precision of the rows (Rans32; 0 for Rans64)
+  const uint16_t *remap;  // alias coding: 2^p remap entries per row
   uint32_t meta_bytes, bucket_bytes, start_bytes;
   const char *blob;
   Geom g;
@@ -108,11 +109,11 @@ __device__ __forceinline__ void bits_op(typename F::State &x, uint32_t val,
 // All ops of one symbol, in reverse op order (bypass pieces last to first,
 // then the count pieces last to first, then the symbol op).  Returns the
 // number of words pushed; with WRITE they go to end[-1 - (pos0 + j)].
-template <class F, bool WRITE>
+template <class F, bool WRITE, bool ALIAS = false>
 __device__ __forceinline__ uint32_t symbol_ops(typename F::State &x, uint32_t start,
                                                uint32_t freq, double rcp, uint64_t raw, bool esc,
                                                typename F::Word *end, uint32_t pos0,
-                                               uint32_t sh) {
+                                               uint32_t sh, const uint16_t *remap_row = nullptr) {
   uint32_t k = 0;
   if (esc) {
     uint32_t nb = 0;
@@ -128,7 +129,8 @@ __device__ __forceinline__ uint32_t symbol_ops(typename F::State &x, uint32_t st
     ++k;
     x >>= F::kWordBits;
   }
-  x = F::sym_step(x, start, freq, rcp, sh);
+  if constexpr (ALIAS) x = F::alias_step(x, start, freq, rcp, sh, remap_row);
+  else x = F::sym_step(x, start, freq, rcp, sh);
   return k;
 }
 
@@ -511,7 +513,8 @@ __device__ void encode_stream_w1(const EncCtx &c, const RowMeta *meta, const uin
 // places them by a suffix sum over the segment.  The flush pushes lanes
 // W-1 .. 0, high word first.  All lanes run the warp's longest stream's
 // group count, idle lanes masked.
-template <class F, typename SymT, bool ST>
+// ALIAS: alias-coded streams (the symbol op codes on the remapped position).
+template <class F, typename SymT, bool ST, bool ALIAS>
 __device__ void encode_segment(const EncCtx &c, const RowMeta *meta, const uint32_t *buckets,
                                int64_t s, int W) {
   using Word = typename F::Word;
@@ -574,19 +577,24 @@ __device__ void encode_segment(const EncCtx &c, const RowMeta *meta, const uint3
     bad_range |= esc && (raw >> 60) != 0;
     raw &= (1ull << 60) - 1;
     const double rcp = F::rcp(freq, sh);
+    const uint16_t *remap_row =
+        ALIAS ? c.remap + ((size_t)(active && r <= kmax ? r : 0u) << (kPrec - sh)) : nullptr;
     if (!__any_sync(kFull, esc)) {
       const bool need = active && F::need_word(x, freq);
       const uint32_t bm = __ballot_sync(kFull, need);
       if (need) st_global(end - 1 - (cursor + __popc(bm & above)), (Word)x);
       if (need) x >>= F::kWordBits;
       cursor += __popc(bm & segmask);
-      if (active) x = F::sym_step(x, start, freq, rcp, sh);
+      if (active) {
+        if constexpr (ALIAS) x = F::alias_step(x, start, freq, rcp, sh, remap_row);
+        else x = F::sym_step(x, start, freq, rcp, sh);
+      }
     } else {
       // every lane counts its words, a suffix sum over the segment places them
       uint32_t kw = 0;
       if (active) {
         State y = x;
-        kw = symbol_ops<F, false>(y, start, freq, rcp, raw, esc, end, 0, sh);
+        kw = symbol_ops<F, false, ALIAS>(y, start, freq, rcp, raw, esc, end, 0, sh, remap_row);
       }
       uint32_t inc = kw;
       for (int o = 1; o < W; o <<= 1) {
@@ -594,7 +602,9 @@ __device__ void encode_segment(const EncCtx &c, const RowMeta *meta, const uint3
         if (l + o < W) inc += t;
       }
       const uint32_t total = __shfl_sync(kFull, inc, seg0);
-      if (active) symbol_ops<F, true>(x, start, freq, rcp, raw, esc, end, cursor + inc - kw, sh);
+      if (active)
+        symbol_ops<F, true, ALIAS>(x, start, freq, rcp, raw, esc, end, cursor + inc - kw, sh,
+                                   remap_row);
       cursor += total;
     }
   }
@@ -671,7 +681,7 @@ __global__ void __launch_bounds__(W == 32 ? kEncThreads32 : kEncThreads1)
 // (0, 1 or 2 as for encode_kernel) is a run-time argument.
 constexpr int kSegThreads = 256;
 
-template <class F, typename SymT>
+template <class F, typename SymT, bool ALIAS>
 __global__ void __launch_bounds__(kSegThreads) encode_kernel_wn(EncCtx c, int mode) {
   extern __shared__ __align__(16) unsigned char smem[];
   __shared__ uint64_t bar;
@@ -698,9 +708,9 @@ __global__ void __launch_bounds__(kSegThreads) encode_kernel_wn(EncCtx c, int mo
     const int64_t k = k0 + seg;
     const int64_t s = k < c.g.S ? stream_of(c.g, k) : -1;
     if (mode == 2)
-      encode_segment<F, SymT, true>(c, meta, buckets, s, W);
+      encode_segment<F, SymT, true, ALIAS>(c, meta, buckets, s, W);
     else
-      encode_segment<F, SymT, false>(c, meta, buckets, s, W);
+      encode_segment<F, SymT, false, ALIAS>(c, meta, buckets, s, W);
   }
 }
 
@@ -846,9 +856,9 @@ int launch_encode_t(const EncCtx &c, cudaStream_t st) {
   return cudaGetLastError() == cudaSuccess ? RANS_OK : RANS_ERR_CUDA;
 }
 
-template <class F, typename SymT>
+template <class F, typename SymT, bool ALIAS>
 int launch_encode_wn(const EncCtx &c, int mode, cudaStream_t st) {
-  auto kern = encode_kernel_wn<F, SymT>;
+  auto kern = encode_kernel_wn<F, SymT, ALIAS>;
   const uint32_t tab = enc_table_bytes(mode, c);
   int dev = 0;
   cudaGetDevice(&dev);
@@ -884,9 +894,10 @@ int launch_encode_w(const EncCtx &c, int mode, cudaStream_t st) {
 
 template <class F, typename SymT>
 int launch_encode_f(const EncCtx &c, int mode, cudaStream_t st) {
+  if (c.g.alias) return launch_encode_wn<F, SymT, true>(c, mode, st);  // W = 1, 2, 4, 8
   if (c.g.W == 32) return launch_encode_w<F, 32, SymT>(c, mode, st);
   if (c.g.W == 1) return launch_encode_w<F, 1, SymT>(c, mode, st);
-  return launch_encode_wn<F, SymT>(c, mode, st);
+  return launch_encode_wn<F, SymT, false>(c, mode, st);
 }
 
 template <typename SymT>
@@ -905,6 +916,9 @@ int launch_encode(const void *symbols, int sym_dtype, const int32_t *indexes,
   c.idx = indexes;
   c.K = t.K;
   c.sh = (uint32_t)(kPrec - t.precision);
+  c.remap = g.alias ? reinterpret_cast<const uint16_t *>(
+                          reinterpret_cast<const char *>(t.alias) + t.alias_remap_offset)
+                    : nullptr;
   c.meta_bytes = t.meta_bytes;
   c.bucket_bytes = t.bucket_bytes;
   c.start_bytes = t.start_bytes;
@@ -939,6 +953,7 @@ int launch_encode_float(const float *y, const float *means, const float *scales,
   c.bound = scale_bound;
   c.K = t.K;
   c.sh = 0;
+  c.remap = nullptr;
   c.meta_bytes = t.meta_bytes;
   c.bucket_bytes = t.bucket_bytes;
   c.start_bytes = t.start_bytes;

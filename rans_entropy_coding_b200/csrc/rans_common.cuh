@@ -118,8 +118,8 @@ struct Geom {
   int64_t ng, nty, ntx;  // TILED counts per image
   int32_t ib_shift;      // log2(index_block)
   int32_t nclass;        // TILED: tile classes in scheduling order (<= 8)
-  int32_t fmt;           // RANS_FMT_*
-  int32_t pad_;
+  int32_t fmt;           // RANS_FMT_RANS64 or RANS_FMT_RANS32_16
+  int32_t alias;         // 1: alias-coded streams (RANS_FMT_ALIAS)
   uint64_t slot_bytes;   // CONTIG / TILED: uniform scratch slot per stream
   uint64_t slot_extra;   // 16 W + 16: per-stream scratch beyond 8 B/symbol
   // TILED: a class is the set of tiles sharing (last channel group?, last
@@ -536,6 +536,20 @@ struct Rans64 {
                                                       uint32_t f16, uint32_t) {
     return (uint64_t)f16 * (x >> kPrec) + (cum16 - start16);
   }
+  // alias coding: the symbol's rank-th position from the row's remap
+  // (encode), and x -> width (x >> 16) + rank (decode)
+  __device__ __forceinline__ static uint64_t alias_step(uint64_t x, uint32_t start16, uint32_t f16,
+                                                        double rcp, uint32_t,
+                                                        const uint16_t *remap_row) {
+    uint64_t q;
+    uint32_t r;
+    divmod_freq(x, f16, rcp, q, r);
+    return (q << kPrec) + __ldg(remap_row + start16 + r);
+  }
+  __device__ __forceinline__ static uint64_t dec_rank_step(uint64_t x, uint32_t f16,
+                                                           uint32_t rank, uint32_t) {
+    return (uint64_t)f16 * (x >> kPrec) + rank;
+  }
 };
 
 struct Rans32 {
@@ -566,7 +580,39 @@ struct Rans32 {
                                                       uint32_t f16, uint32_t sh) {
     return (f16 >> sh) * (x >> (kPrec - sh)) + ((cum16 - start16) >> sh);
   }
+  __device__ __forceinline__ static uint32_t alias_step(uint32_t x, uint32_t start16, uint32_t f16,
+                                                        double rcp, uint32_t sh,
+                                                        const uint16_t *remap_row) {
+    uint32_t q, r;
+    divmod_freq32(x, f16 >> sh, rcp, q, r);
+    return (q << (kPrec - sh)) + __ldg(remap_row + (start16 >> sh) + r);
+  }
+  __device__ __forceinline__ static uint32_t dec_rank_step(uint32_t x, uint32_t f16,
+                                                           uint32_t rank, uint32_t sh) {
+    return (f16 >> sh) * (x >> (kPrec - sh)) + rank;
+  }
 };
+
+// ------------------------------------------------------------- alias ----
+// Alias tables (a second blob, built by rans_alias_prepare): per row, slot
+// words at the row's bucket indexes (bucket_base + j, slot j of the row's n
+// = maxv + 1 slots of 2^p / n positions) packing d | (a | base << 16) << 32:
+// positions [0, d) of the slot are the slot's own symbol j at ranks [0, d),
+// the rest the alias symbol a at ranks base + (o - d); then 2^p 16-bit
+// remap entries per row: remap[start + rank] = the position of that rank.
+// The symbol and rank of position c (precision p) in row m.
+__device__ __forceinline__ uint32_t alias_lookup(uint32_t c, const RowMeta &m,
+                                                 const uint2 *slots, uint32_t prec,
+                                                 uint32_t &rank) {
+  const uint32_t log_n = 31 - __clz(m.maxv + 1);
+  const uint32_t log_b = prec - log_n;
+  const uint32_t j = c >> log_b;
+  const uint32_t o = c & ((1u << log_b) - 1u);
+  const uint2 e = __ldg(slots + m.bucket_base + j);
+  const bool own = o < e.x;
+  rank = own ? o : (e.y >> 16) + (o - e.x);
+  return own ? j : (e.y & 0xffffu);
+}
 
 // ------------------------------------------------------- warp helpers --
 __device__ __forceinline__ uint32_t lanemask_lt() {

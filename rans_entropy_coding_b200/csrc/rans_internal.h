@@ -20,6 +20,9 @@ int launch_pmf_rows(const float *pmfs, int K, int stride, const int32_t *pmf_len
                     const float *tail, int prec, int32_t *cdfs, int Lmax, int32_t *lengths,
                     cudaStream_t st);
 uint64_t tables_bytes_bound(int K, int Lmax);
+// Alias tables of a prepared table set into `alias` (synchronous).
+int prepare_alias(const int32_t *cdfs, int K, int Lmax, const int32_t *lengths,
+                  rans_tables &t, void *alias, uint64_t alias_bytes, cudaStream_t st);
 int refresh_tables(const int32_t *cdfs, int K, int Lmax, const int32_t *lengths,
                    const int32_t *offsets, const rans_tables &t, cudaStream_t st);
 // Rows summing to 2^prec, stored scaled to 16 bits.

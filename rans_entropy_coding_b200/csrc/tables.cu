@@ -570,6 +570,86 @@ __global__ void __launch_bounds__(kSlotThreads)
   fill_row_slots(row, len - 1, slot_base(m.slot), (int)slot_shift(m.slot), slots, ca, srow, sh);
 }
 
+// Alias tables, one row per block (the reading of the alias method given
+// with RANS_FMT_ALIAS: Vose with first-in first-out worklists in ascending
+// order, a symbol's own slot part ranked first and its alias parts after in
+// slot order).  Thread 0 builds the slots (a short sequential pass over the
+// row's n <= 8192 buckets, in shared memory); then every thread writes slot
+// words and remap entries.
+constexpr int kAliasMaxBuckets = 8192;
+
+__global__ void __launch_bounds__(256)
+    alias_build_kernel(const int32_t *cdfs, int Lmax, const int32_t *lengths,
+                       const RowMeta *meta, int prec, int nmax, uint2 *aslots,
+                       uint16_t *remap, int32_t *status) {
+  extern __shared__ int32_t asm_[];
+  __shared__ int ok_sh;
+  const int r = blockIdx.x;
+  const int n = lengths[r] - 1;
+  const int32_t *row = cdfs + (size_t)r * (size_t)Lmax;
+  const int32_t M = 1 << prec;
+  int32_t *rem = asm_, *small = asm_ + nmax, *large = asm_ + 2 * nmax;
+  int32_t *d = asm_ + 3 * nmax, *a = asm_ + 4 * nmax, *base = asm_ + 5 * nmax;
+  if (threadIdx.x == 0) {
+    int ok = n >= 1 && n <= nmax && (n & (n - 1)) == 0 && n <= M && row[0] == 0 && row[n] == M;
+    const int32_t B = ok ? M / n : 1;
+    int ns = 0, nl = 0, hs = 0, hl = 0;
+    for (int j = 0; ok && j < n; ++j) {
+      const int32_t f = row[j + 1] - row[j];
+      if (f <= 0) {
+        ok = 0;
+        break;
+      }
+      rem[j] = f;
+      d[j] = B;
+      a[j] = j;
+      base[j] = 0;
+      if (f < B) small[ns++] = j;
+      else if (f > B) large[nl++] = j;
+    }
+    while (ok && hs < ns && hl < nl) {
+      const int32_t l = small[hs++];
+      const int32_t g = large[hl];
+      d[l] = rem[l];
+      a[l] = g;
+      rem[g] -= B - rem[l];
+      if (rem[g] <= B) {
+        ++hl;
+        if (rem[g] < B) small[ns++] = g;
+      }
+    }
+    if (ok && (hs < ns || hl < nl)) ok = 0;
+    if (ok) {
+      int32_t *cnt = rem;  // each symbol's next rank: own part first
+      for (int j = 0; j < n; ++j) cnt[j] = d[j];
+      for (int j = 0; j < n; ++j) {
+        if (d[j] == B) continue;
+        base[j] = cnt[a[j]];
+        cnt[a[j]] += B - d[j];
+      }
+      // every symbol ends with exactly its frequency's positions, so the
+      // remap writes below stay inside the row
+      for (int j = 0; j < n; ++j)
+        if (cnt[j] != row[j + 1] - row[j]) ok = 0;
+    }
+    if (!ok) report(status, RANS_ERR_TABLE, r);
+    ok_sh = ok;
+  }
+  __syncthreads();
+  if (!ok_sh) return;
+  const uint32_t bb = meta[r * kMetaCopies].bucket_base;
+  int log_b = 0;
+  while ((n << log_b) < M) ++log_b;
+  for (int j = threadIdx.x; j < n; j += blockDim.x)
+    aslots[bb + j] = make_uint2((uint32_t)d[j], (uint32_t)a[j] | ((uint32_t)base[j] << 16));
+  uint16_t *rm = remap + ((size_t)r << prec);
+  for (int32_t c = threadIdx.x; c < M; c += blockDim.x) {
+    const int32_t j = c >> log_b, o = c & ((1 << log_b) - 1);
+    if (o < d[j]) rm[row[j] + o] = (uint16_t)c;
+    else rm[row[a[j]] + base[j] + (o - d[j])] = (uint16_t)c;
+  }
+}
+
 // Row index of every scale (scale_row in rans_common.cuh).
 __global__ void build_indexes_kernel(const float *scales, int64_t n, const float *table, int K,
                                      float bound, int32_t *indexes) {
@@ -816,6 +896,48 @@ int prepare_tables(const int32_t *cdfs, int K, int Lmax, const int32_t *lengths,
       dec_smem ? 1 : ((int64_t)meta_bytes + start_bytes + kDecStageBytes <= budget ? 2 : 0);
   out->device = dev;
   out->precision = prec;
+  return RANS_OK;
+}
+
+int prepare_alias(const int32_t *cdfs, int K, int Lmax, const int32_t *lengths,
+                  rans_tables &t, void *alias, uint64_t alias_bytes, cudaStream_t st) {
+  if (K != t.K || alias == nullptr || (reinterpret_cast<uintptr_t>(alias) & 255) != 0)
+    return RANS_ERR_ARG;
+  const uint64_t slot_bytes = (8ull * (uint64_t)t.n_buckets + 255) & ~255ull;
+  const uint64_t need = slot_bytes + 2ull * (uint64_t)K * (1ull << t.precision);
+  if (alias_bytes < need) return RANS_ERR_CAPACITY;
+  std::vector<int32_t> len(K);
+  if (cudaMemcpyAsync(len.data(), lengths, sizeof(int32_t) * K, cudaMemcpyDeviceToHost, st) !=
+          cudaSuccess ||
+      cudaStreamSynchronize(st) != cudaSuccess)
+    return RANS_ERR_CUDA;
+  int nmax = 1;
+  for (int r = 0; r < K; ++r) {
+    const int n = len[r] - 1;
+    if (n < 1 || (n & (n - 1)) != 0 || n > kAliasMaxBuckets) return RANS_ERR_ARG;
+    nmax = n > nmax ? n : nmax;
+  }
+  char *b = reinterpret_cast<char *>(t.blob);
+  int32_t *status = reinterpret_cast<int32_t *>(b);
+  const RowMeta *dmeta = reinterpret_cast<const RowMeta *>(b + kHeaderBytes);
+  uint2 *aslots = reinterpret_cast<uint2 *>(alias);
+  uint16_t *remap = reinterpret_cast<uint16_t *>(reinterpret_cast<char *>(alias) + slot_bytes);
+  const uint32_t smem = 6u * 4u * (uint32_t)nmax;
+  if (cudaFuncSetAttribute(alias_build_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           (int)smem) != cudaSuccess)
+    return RANS_ERR_CUDA;
+  if (cudaMemsetAsync(alias, 0, slot_bytes, st) != cudaSuccess) return RANS_ERR_CUDA;
+  alias_build_kernel<<<K, 256, smem, st>>>(cdfs, Lmax, lengths, dmeta, t.precision, nmax, aslots,
+                                           remap, status);
+  if (cudaGetLastError() != cudaSuccess) return RANS_ERR_CUDA;
+  StatusWord sw;
+  if (cudaMemcpyAsync(&sw, status, sizeof(sw), cudaMemcpyDeviceToHost, st) != cudaSuccess ||
+      cudaStreamSynchronize(st) != cudaSuccess)
+    return RANS_ERR_CUDA;
+  if (sw.code != 0) return sw.code;
+  t.alias = alias;
+  t.alias_bytes = need;
+  t.alias_remap_offset = slot_bytes;
   return RANS_OK;
 }
 

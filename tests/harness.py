@@ -13,6 +13,10 @@ def fmt_of(w):
     return w.get("fmt", "rans64")
 
 
+def alias_of(w):
+    return bool(w.get("alias", False))
+
+
 def precision_of(w):
     return w.get("precision", 16 if fmt_of(w) == "rans64" else 15)
 
@@ -48,7 +52,7 @@ def tables_from_numpy(c, l, o, dev="cuda", precision=16):
 
 def chunking_of(w, dev="cuda"):
     return rb.Chunking.from_spec(w["chunking"], w["W"], w["index_block"], device=dev,
-                                 fmt=fmt_of(w))
+                                 fmt=fmt_of(w), alias=alias_of(w))
 
 
 def gpu_encode_decode(w, tables, dev="cuda", expect_ok=True):
@@ -74,4 +78,4 @@ def oracle_encode(w, c, l, o, streams=None):
     sym = np.asarray(w["symbols"]).reshape(-1)
     return O.encode_with_indexes(sym, w["indexes"], c, l, o, w["chunking"], W=w["W"],
                                  index_block=w["index_block"], streams=streams, fmt=fmt_of(w),
-                                 precision=precision_of(w))
+                                 precision=precision_of(w), alias=alias_of(w))
