@@ -468,16 +468,41 @@ __device__ void decode_stream_w1(const DecCtx &c, const RowMeta *meta, const uin
     prefetch(d.base + pp.rel(t));
     pp.fwd(t, 1);
   }
+  // The rows (and, for float values, the means) of the next kRing symbols
+  // wait in registers, each read kRing symbols before it is decoded, so
+  // that the state chain does not wait on their loads.
+  constexpr int kRing = 4;
+  RelPos pf = pl;  // next symbol to fetch into the ring
+  int32_t rrow[kRing];
+  float rmean[kRing];
+  auto fetch = [&](int32_t &r, float &mean) {
+    const int64_t q = d.base + pf.rel(t);
+    pf.fwd(t, 1);
+    r = kFlt ? (int32_t)scale_row(bound_scale(__ldg(c.fscale + q), c.bound), stab, c.K)
+             : __ldg(c.idx + (q >> ib));
+    mean = kFlt && c.fmean ? __ldg(c.fmean + q) : 0.0f;
+  };
+#pragma unroll
+  for (int u = 0; u < kRing; ++u) {
+    rrow[u] = 0;
+    rmean[u] = 0.0f;
+    if (u < n) fetch(rrow[u], rmean[u]);
+  }
   for (int32_t i = 0; i < n; ++i) {
     const int64_t p = d.base + pl.rel(t);
     pl.fwd(t, 1);
+    const int32_t r = rrow[0];
+    const float mean_i = rmean[0];
+#pragma unroll
+    for (int u = 0; u + 1 < kRing; ++u) {
+      rrow[u] = rrow[u + 1];
+      rmean[u] = rmean[u + 1];
+    }
+    if (i + kRing < n) fetch(rrow[kRing - 1], rmean[kRing - 1]);
     if (i + kAhead < n) {
       prefetch(d.base + pp.rel(t));
       pp.fwd(t, 1);
     }
-    const int32_t r =
-        kFlt ? (int32_t)scale_row(bound_scale(__ldg(c.fscale + p), c.bound), stab, c.K)
-             : __ldg(c.idx + (p >> ib));
     if ((uint32_t)r >= (uint32_t)c.K) {
       report(c.status, RANS_ERR_INDEX, s);
       return;
@@ -515,8 +540,7 @@ __device__ void decode_stream_w1(const DecCtx &c, const RowMeta *meta, const uin
     }
     if constexpr (kFlt)
       st_global(reinterpret_cast<float *>(c.out) + p,
-                (float)(int32_t)(val + (int64_t)m.offset) +
-                    (c.fmean ? __ldg(c.fmean + p) : 0.0f));
+                (float)(int32_t)(val + (int64_t)m.offset) + mean_i);
     else
       SymIO<SymT>::store(c.out, p, val + (int64_t)m.offset);
   }

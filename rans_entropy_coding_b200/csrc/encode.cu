@@ -442,9 +442,9 @@ __device__ void encode_stream_w1(const EncCtx &c, const RowMeta *meta, const uin
   const int32_t n = (int32_t)d.n;
   typename F::State x = F::kLow;
   uint32_t cursor = 0;
-  RelPos pl, pp;
-  pl.init(t, n > 0 ? n - 1 : 0);
-  pp = pl;
+  RelPos pf, pp;  // next symbol to fetch into the ring; next L2 prefetch
+  pf.init(t, n > 0 ? n - 1 : 0);
+  pp = pf;
   constexpr int32_t kAhead = 64;
   for (int32_t u = 0; u < kAhead && u < n; ++u) {
     const int64_t p = d.base + pp.rel(t);
@@ -457,9 +457,41 @@ __device__ void encode_stream_w1(const EncCtx &c, const RowMeta *meta, const uin
     }
     pp.back(t, 1);
   }
+  // The symbols and rows of the next kRing symbols (in coding order) wait in
+  // registers, each read kRing symbols before it is coded, so that the state
+  // chain does not wait on their loads.  FLT: the row and the quantised
+  // symbol are computed when read (ok: the value was in range).
+  constexpr int kRing = 4;
+  int32_t rsym[kRing], rrow[kRing];
+  bool rok[kRing];
+  auto fetch = [&](int32_t &sv, int32_t &r, bool &ok) {
+    const int64_t p = d.base + pf.rel(t);
+    pf.back(t, 1);
+    ok = true;
+    if (FLT) {
+      sv = quantize(__ldg(c.fy + p), c.fmean ? __ldg(c.fmean + p) : 0.0f, ok);
+      r = (int32_t)scale_row(bound_scale(__ldg(c.fscale + p), c.bound), stab, c.K);
+    } else {
+      sv = SymIO<SymT>::load(c.sym, p);
+      r = __ldg(c.idx + (p >> ib));
+    }
+  };
+#pragma unroll
+  for (int u = 0; u < kRing; ++u) {
+    rsym[u] = rrow[u] = 0;
+    rok[u] = true;
+    if (u < n) fetch(rsym[u], rrow[u], rok[u]);
+  }
   for (int32_t i = n - 1; i >= 0; --i) {
-    const int64_t p = d.base + pl.rel(t);
-    pl.back(t, 1);
+    const int32_t sv = rsym[0], r = rrow[0];
+    const bool ok = rok[0];
+#pragma unroll
+    for (int u = 0; u + 1 < kRing; ++u) {
+      rsym[u] = rsym[u + 1];
+      rrow[u] = rrow[u + 1];
+      rok[u] = rok[u + 1];
+    }
+    if (i - kRing >= 0) fetch(rsym[kRing - 1], rrow[kRing - 1], rok[kRing - 1]);
     if (i - kAhead >= 0) {
       const int64_t q = d.base + pp.rel(t);
       if (FLT) {
@@ -471,18 +503,9 @@ __device__ void encode_stream_w1(const EncCtx &c, const RowMeta *meta, const uin
       }
       pp.back(t, 1);
     }
-    int32_t sv, r;
-    if (FLT) {
-      bool ok;
-      sv = quantize(__ldg(c.fy + p), c.fmean ? __ldg(c.fmean + p) : 0.0f, ok);
-      if (!ok) {
-        report(c.status, RANS_ERR_RANGE, s);
-        return;
-      }
-      r = (int32_t)scale_row(bound_scale(__ldg(c.fscale + p), c.bound), stab, c.K);
-    } else {
-      sv = SymIO<SymT>::load(c.sym, p);
-      r = __ldg(c.idx + (p >> ib));
+    if (!ok) {
+      report(c.status, RANS_ERR_RANGE, s);
+      return;
     }
     if ((uint32_t)r >= (uint32_t)c.K) {
       report(c.status, RANS_ERR_INDEX, s);
