@@ -14,15 +14,19 @@
  *     in 4-bit bypass pieces (same section, "Range limit"; "kompressor"
  *     README, Correctness: the bypass path).
  *   - Many independent streams: contiguous chunks or spatial tiles ("kompressor"
- *     README, Why: zero cross-chunk dependency), each coded with W = 1 state
- *     or W = 32 interleaved states sharing one word stream, lane i mod 32
- *     ("torch_ans 0.3.0", Usage legend and FAQ: interleaved states share one
- *     bitstream; the 32-way form maps the states onto the lanes of a warp).
+ *     README, Why: zero cross-chunk dependency), each coded with W = 1, 2, 4,
+ *     8 or 32 interleaved states sharing one word stream, symbol i on state
+ *     i mod W ("torch_ans 0.3.0", Usage legend and FAQ: interleaved states
+ *     share one bitstream; the 32-way form maps the states onto the lanes of
+ *     a warp, the 2/4/8-way forms onto sub-warp lane groups).
+ *   - Two coder formats: the 64/32/16 one described below (RANS_FMT_RANS64)
+ *     and torch_ans's rans32_16 (RANS_FMT_RANS32_16: 32-bit state, 16-bit
+ *     words, precision <= 15), each also alias-coded (RANS_FMT_ALIAS).
  *   - pmf -> quantised CDF rows ("torch_ans 0.3.0", High-level API,
  *     init_params) and Gaussian rows from a scale table ("kompressor" README,
  *     Getting Started: 64 CDF rows for the y latent).
  *
- * Fixed format: state bound L = 2^31 (initial encoder state, final decoder
+ * The RANS64 format: state bound L = 2^31 (initial encoder state, final decoder
  * state), symbol op renormalises when x >= 2^47 * freq, bypass op when
  * x >= 2^59; the stream of one chunk is its W lane states (low word, high
  * word; lane 0 first) followed by the renormalisation words in the order the
@@ -36,8 +40,8 @@
  *   - The caller allocates every buffer; the library never allocates device
  *     memory (sizes come from the *_bytes queries).
  *   - `stream` is a cudaStream_t (NULL = the legacy default stream); all work
- *     is enqueued on it.  Only rans_tables_prepare and rans_get_status
- *     synchronise.
+ *     is enqueued on it.  Only rans_tables_prepare, rans_alias_prepare and
+ *     rans_get_status synchronise.
  *   - Argument errors detectable on the host return immediately with a
  *     negative status.  Errors found on the device (bad index, zero-width
  *     bucket, raw value beyond 60 bits, a malformed or truncated stream, output
