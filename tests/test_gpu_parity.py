@@ -509,3 +509,24 @@ def test_encode_from_scales_reports_values_out_of_range():
                                           dev(np.asarray(w["scales"], np.float32)),
                                           w["scale_bound"], tables, ch, means=dev(w["means"]))
     assert rb.rans_get_status(ws.enc) == rb.ERR_RANGE
+
+
+def test_float_latents_take_the_64_bit_format_only():
+    """The float-latent entry points code the 64-bit format at W = 1 or 32;
+    rans32_16 or alias chunkings, and 2/4/8 interleaves, are refused."""
+    w, wi, (c, l, o) = _float_case(W=32)
+    tables = tables_from_numpy(c, l, o)
+    dev = lambda a: torch.from_numpy(np.ascontiguousarray(a).reshape(-1)).cuda()
+    y, sc, tab = dev(w["y"]), dev(w["fscales"]), dev(np.asarray(w["scales"], np.float32))
+    n = y.numel()
+    shape = w["chunking"]["shape"]
+    for ch in (rb.Chunking.tiled(shape, 4, 64, 64, 32, fmt="rans32_16"),
+               rb.Chunking.tiled(shape, 4, 64, 64, 4, alias=True),
+               rb.Chunking.tiled(shape, 4, 64, 64, 4)):
+        ws = rb.Workspaces(ch, n)
+        st = rb.rans_encode_from_scales(y, None, sc, n, tab, w["scale_bound"], tables, ch,
+                                        ws.out, ws.offsets, ws.enc)
+        assert st == rb.ERR_ARG
+        st = rb.rans_decode_to_values(ws.out, ws.offsets, sc, None, n, tab, w["scale_bound"],
+                                      tables, ch, torch.empty(n, device="cuda"), ws.dec)
+        assert st == rb.ERR_ARG
