@@ -413,9 +413,10 @@ def run_ours(args, world, rank, local):
         container = {"streams": int(sum(counts)), "bytes": int(gidx[-1].item()),
                      "rank0_base": base if rank == 0 else None}
 
-    tab_ms = float(np.mean([e[0].elapsed_time(e[1]) for e in ev]))
-    enc_ms = float(np.mean([e[1].elapsed_time(e[2]) for e in ev]))
-    dec_ms = float(np.mean([e[2].elapsed_time(e[3]) for e in ev]))
+    tab_t = [e[0].elapsed_time(e[1]) for e in ev]
+    enc_t = [e[1].elapsed_time(e[2]) for e in ev]
+    dec_t = [e[2].elapsed_time(e[3]) for e in ev]
+    tab_ms, enc_ms, dec_ms = (float(np.mean(t)) for t in (tab_t, enc_t, dec_t))
     comp = int(ws.offsets[-1].item())
     sym_b = sym.element_size()
     alg_enc = n * (sym_b + 4) + comp     # symbols + indexes read, bytes written
@@ -537,9 +538,13 @@ def run_ours(args, world, rank, local):
         workers = os.cpu_count() or 1
         ms = {"batch": 768, "sweep": 64, "r16": 256}.get(args.workload, S)
         ns, ts = oracle_sample(w, ms, workers)
+        ms1 = max(1, ms // workers)           # one thread: about the same wall time
+        ns1, ts1 = oracle_sample(w, ms1, 1)
         cpu = {"value": ns / ts / 1e9, "unit": UNIT, "cores": workers, "kind": "oracle",
                "sample": "oracle encode+decode of the first %d streams (%d symbols), "
-                         "one stream per call over %d threads" % (ms, ns, workers)}
+                         "one stream per call over %d threads" % (ms, ns, workers),
+               "single_thread": {"value": ns1 / ts1 / 1e9, "unit": UNIT,
+                                 "sample": "the first %d streams on one thread" % ms1}}
 
     launches_per_step = 1 + 1 + 3 + 1   # rows, table refresh, enc+scan+copy, dec
     if rank == 0:
@@ -556,11 +561,13 @@ def run_ours(args, world, rank, local):
                        "l2": ("inputs larger than L2 (%d MB read per encode)" %
                               (n * (sym_b + 4) // 2**20)) if flush is None else
                              "L2 flushed before every step (256 MB write, not timed)"},
-            "encode": {"ms": enc_ms, "gsym_s": n / enc_ms / 1e6, "GBps": enc_gbs,
-                       "frac_hbm": enc_gbs / peak, "alg_bytes": alg_enc},
-            "decode": {"ms": dec_ms, "gsym_s": n / dec_ms / 1e6, "GBps": dec_gbs,
-                       "frac_hbm": dec_gbs / peak, "alg_bytes": alg_dec},
-            "tables": {"ms": tab_ms},
+            "encode": {"ms": enc_ms, "ms_median": float(np.median(enc_t)),
+                       "ms_best": float(np.min(enc_t)), "gsym_s": n / enc_ms / 1e6,
+                       "GBps": enc_gbs, "frac_hbm": enc_gbs / peak, "alg_bytes": alg_enc},
+            "decode": {"ms": dec_ms, "ms_median": float(np.median(dec_t)),
+                       "ms_best": float(np.min(dec_t)), "gsym_s": n / dec_ms / 1e6,
+                       "GBps": dec_gbs, "frac_hbm": dec_gbs / peak, "alg_bytes": alg_dec},
+            "tables": {"ms": tab_ms, "ms_median": float(np.median(tab_t))},
             "compressed_bytes": comp, "bits_per_symbol": 8.0 * comp / n,
             "roofline": {"bound": "hbm", "achieved": ach, "peak": peak, "unit": "GB/s",
                          "frac": ach / peak, "traffic": traffic, "kernel": dominant,
