@@ -70,16 +70,23 @@ def parse():
     return ap.parse_args()
 
 
+# The sources the measured coders (encode_kernel, decode_kernel and the
+# compaction kernels) are compiled from.
+MEASURED_SOURCES = ("rans_entropy_coding_b200/csrc/encode.cu",
+                    "rans_entropy_coding_b200/csrc/decode.cu",
+                    "rans_entropy_coding_b200/csrc/rans_common.cuh",
+                    "rans_entropy_coding_b200/csrc/rans_internal.h",
+                    "include/rans_b200.h")
+
+
 def kernel_sources_digest():
-    """sha256 over the CUDA sources, so a DRAM-traffic figure taken with ncu
-    is only reported while the kernels it measured are unchanged."""
+    """sha256 over the coders' CUDA sources, so a DRAM-traffic figure taken
+    with ncu is only reported while the kernels it measured are unchanged."""
     import hashlib
     h = hashlib.sha256()
-    csrc = os.path.join(ROOT, "rans_entropy_coding_b200", "csrc")
-    for name in sorted(os.listdir(csrc)):
-        if name.endswith((".cu", ".cuh", ".h")):
-            h.update(name.encode())
-            h.update(open(os.path.join(csrc, name), "rb").read())
+    for rel in MEASURED_SOURCES:
+        h.update(os.path.basename(rel).encode())
+        h.update(open(os.path.join(ROOT, rel), "rb").read())
     return h.hexdigest()
 
 
