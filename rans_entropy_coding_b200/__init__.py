@@ -12,7 +12,7 @@ from ._lib import (  # noqa: F401
     check, decode_to_values, decode_with_indexes, encode_from_scales, encode_with_indexes, lib,
     rans_alias_bytes, rans_alias_prepare, rans_build_cdfs_from_pmfs, rans_build_indexes, rans_decode_to_values,
     rans_encode_from_scales,
-    rans_build_cdfs_from_scales, rans_chunking, rans_debug_divide, rans_decode_with_indexes,
+    rans_build_cdfs_from_scales, rans_chunking, rans_debug_divide, rans_debug_wait_timeout, rans_decode_with_indexes,
     rans_decode_workspace_bytes, rans_encode_with_indexes, rans_encode_with_indexes_noalloc,
     rans_encode_workspace_bytes,
     rans_gaussian_lengths, rans_get_status, rans_max_compressed_bytes, rans_num_streams,

@@ -96,6 +96,7 @@ SIGNATURES = [
      [_P, _U64, _P, _P, _P, _I64, _P, _I32, _F32, _TBP, _CHP, _P, _P, _U64, _P]),
     ("rans_get_status", ctypes.c_int, [_P, _P]),
     ("rans_debug_divide", ctypes.c_int, [_P, _P, _I64, _P, _P, _P]),
+    ("rans_debug_wait_timeout", ctypes.c_int, [_P, ctypes.c_uint32, _P]),
 ]
 
 _lib = None
@@ -267,6 +268,11 @@ def rans_decode_to_values(data, stream_offsets, scales, means, n, scale_table, s
 
 def rans_get_status(workspace, stream=None):
     return lib().rans_get_status(_ptr(workspace), _stream(stream))
+
+
+def rans_debug_wait_timeout(workspace, limit, stream=None):
+    _need_cuda(workspace)
+    return lib().rans_debug_wait_timeout(_ptr(workspace), limit, _stream(stream))
 
 
 def rans_debug_divide(x, f, q, r, stream=None):

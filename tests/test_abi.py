@@ -11,13 +11,15 @@ import rans_entropy_coding_b200 as rb
 from rans_entropy_coding_b200 import build as rbuild
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
-HEADER = os.path.join(ROOT, "include", "rans_b200.h")
+HEADERS = [os.path.join(ROOT, "include", h) for h in ("rans_b200.h", "rans_b200_debug.h")]
 
 
 def declared_functions():
-    src = open(HEADER).read()
-    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
-    return sorted(set(re.findall(r"\b(rans_[a-z0-9_]+)\s*\(", src)))
+    names = set()
+    for path in HEADERS:
+        src = re.sub(r"/\*.*?\*/", "", open(path).read(), flags=re.S)
+        names |= set(re.findall(r"\b(rans_[a-z0-9_]+)\s*\(", src))
+    return sorted(names)
 
 
 @pytest.fixture(scope="module")

@@ -530,3 +530,17 @@ def test_float_latents_take_the_64_bit_format_only():
         st = rb.rans_decode_to_values(ws.out, ws.offsets, sc, None, n, tab, w["scale_bound"],
                                       tables, ch, torch.empty(n, device="cuda"), ws.dec)
         assert st == rb.ERR_ARG
+
+
+def test_bounded_wait_gives_up_and_the_context_stays_usable():
+    """The table staging's bounded mbarrier wait, run on a barrier nothing
+    completes, records RANS_ERR_TIMEOUT and returns; the next coding call on
+    the same context works."""
+    import time
+    ws = rb.aligned_empty(256)
+    t = time.time()
+    rb.check(rb.rans_debug_wait_timeout(ws, 2000))
+    assert rb.rans_get_status(ws) == rb.ERR_TIMEOUT
+    assert time.time() - t < 30
+    assert rb.rans_debug_wait_timeout(ws, 0) == rb.ERR_ARG
+    _check_streams(_edge_tiny(32, seed=11))
