@@ -17,3 +17,4 @@ from ._lib import (  # noqa: F401
     rans_encode_workspace_bytes,
     rans_gaussian_lengths, rans_get_status, rans_max_compressed_bytes, rans_num_streams,
     rans_tables, rans_tables_bytes, rans_tables_prepare, rans_tables_refresh)
+from .interface import RansCoder, from_byte_strings, to_byte_strings  # noqa: F401,E402
