@@ -3,6 +3,8 @@
 // runs in the kernels of tables.cu, encode.cu and decode.cu.
 #include <cstring>
 
+#include <nvtx3/nvToolsExt.h>
+
 #include "rans_common.cuh"
 #include "rans_internal.h"
 
@@ -32,6 +34,13 @@ int smem_optin(int device) {
 namespace {
 
 using rb::Geom;
+
+// An NVTX range around an entry point, so that traces show the library's
+// calls (no cost beyond a call when no tool is attached).
+struct NvtxRange {
+  explicit NvtxRange(const char *name) { nvtxRangePushA(name); }
+  ~NvtxRange() { nvtxRangePop(); }
+};
 
 constexpr uint64_t kWsHeader = 256;
 
@@ -198,6 +207,7 @@ RANS_API int rans_gaussian_lengths(const float *scales, int32_t K, double tail_m
 RANS_API int rans_build_cdfs_from_scales(const float *scales, int32_t K, double tail_mass,
                                          int32_t precision, int32_t *cdfs, int32_t Lmax,
                                          int32_t *cdf_lengths, int32_t *offsets, void *stream) {
+  NvtxRange nvtx_("rans_build_cdfs_from_scales");
   if (K < 1 || Lmax < 3 || !scales || !cdfs || !cdf_lengths || !offsets) return RANS_ERR_ARG;
   if (!(tail_mass > 0.0) || !(tail_mass < 1.0)) return RANS_ERR_ARG;
   if (precision < 1 || precision > 16) return RANS_ERR_ARG;
@@ -209,6 +219,7 @@ RANS_API int rans_build_cdfs_from_pmfs(const float *pmfs, int32_t K, int32_t pmf
                                        const int32_t *pmf_lengths, const float *tail_mass,
                                        int32_t precision, int32_t *cdfs, int32_t Lmax,
                                        int32_t *cdf_lengths, void *stream) {
+  NvtxRange nvtx_("rans_build_cdfs_from_pmfs");
   if (K < 1 || pmf_stride < 1 || Lmax < 2 || !pmfs || !pmf_lengths || !tail_mass || !cdfs ||
       !cdf_lengths)
     return RANS_ERR_ARG;
@@ -225,6 +236,7 @@ RANS_API int rans_tables_prepare(const int32_t *cdfs, int32_t K, int32_t Lmax,
                                  const int32_t *cdf_lengths, const int32_t *offsets,
                                  int32_t precision, void *blob, uint64_t blob_bytes,
                                  rans_tables *out, void *stream) {
+  NvtxRange nvtx_("rans_tables_prepare");
   if (K < 1 || Lmax < 2 || Lmax > 65537 || !cdfs || !cdf_lengths || !offsets || !blob || !out)
     return RANS_ERR_ARG;
   if (precision < 1 || precision > 16) return RANS_ERR_ARG;
@@ -235,6 +247,7 @@ RANS_API int rans_tables_prepare(const int32_t *cdfs, int32_t K, int32_t Lmax,
 RANS_API int rans_tables_refresh(const int32_t *cdfs, int32_t K, int32_t Lmax,
                                  const int32_t *cdf_lengths, const int32_t *offsets,
                                  const rans_tables *tables, void *stream) {
+  NvtxRange nvtx_("rans_tables_refresh");
   if (!tables_usable(tables) || K != tables->K || Lmax < 2 || !cdfs || !cdf_lengths || !offsets)
     return RANS_ERR_ARG;
   return rb::refresh_tables(cdfs, K, Lmax, cdf_lengths, offsets, *tables, as_stream(stream));
@@ -249,6 +262,7 @@ RANS_API uint64_t rans_alias_bytes(const rans_tables *tables) {
 RANS_API int rans_alias_prepare(const int32_t *cdfs, int32_t K, int32_t Lmax,
                                 const int32_t *cdf_lengths, rans_tables *tables, void *alias,
                                 uint64_t alias_bytes, void *stream) {
+  NvtxRange nvtx_("rans_alias_prepare");
   if (!tables_usable(tables) || K != tables->K || Lmax < 2 || !cdfs || !cdf_lengths || !alias)
     return RANS_ERR_ARG;
   return rb::prepare_alias(cdfs, K, Lmax, cdf_lengths, *tables, alias, alias_bytes,
@@ -285,6 +299,7 @@ RANS_API int rans_encode_with_indexes(const void *symbols, int32_t sym_dtype,
                                       uint8_t *out, uint64_t out_capacity,
                                       uint64_t *stream_offsets, void *workspace,
                                       uint64_t workspace_bytes, void *stream) {
+  NvtxRange nvtx_("rans_encode_with_indexes");
   if (!tables_usable(tables)) return RANS_ERR_ARG;
   if (n > 0 && (!symbols || !indexes)) return RANS_ERR_ARG;
   if (!stream_offsets || !workspace || (out_capacity > 0 && !out)) return RANS_ERR_ARG;
@@ -316,6 +331,7 @@ RANS_API int rans_decode_with_indexes(const uint8_t *in, uint64_t in_bytes,
                                       const rans_chunking *chunking, void *symbols_out,
                                       int32_t sym_dtype, void *workspace,
                                       uint64_t workspace_bytes, void *stream) {
+  NvtxRange nvtx_("rans_decode_with_indexes");
   if (!tables_usable(tables)) return RANS_ERR_ARG;
   if (n > 0 && (!symbols_out || !indexes)) return RANS_ERR_ARG;
   if (!stream_offsets || !workspace || (in_bytes > 0 && !in)) return RANS_ERR_ARG;
@@ -340,6 +356,7 @@ RANS_API int rans_decode_with_indexes(const uint8_t *in, uint64_t in_bytes,
 
 RANS_API int rans_build_indexes(const float *scales, int64_t n, const float *scale_table,
                                 int32_t K, float scale_bound, int32_t *indexes, void *stream) {
+  NvtxRange nvtx_("rans_build_indexes");
   if (n < 0 || K < 1 || (n > 0 && (!scales || !scale_table || !indexes))) return RANS_ERR_ARG;
   return rb::launch_build_indexes(scales, n, scale_table, K, scale_bound, indexes,
                                   as_stream(stream));
@@ -362,6 +379,7 @@ RANS_API int rans_encode_from_scales(const float *y, const float *means, const f
                                      const rans_chunking *chunking, uint8_t *out,
                                      uint64_t out_capacity, uint64_t *stream_offsets,
                                      void *workspace, uint64_t workspace_bytes, void *stream) {
+  NvtxRange nvtx_("rans_encode_from_scales");
   int st = float_args(tables, chunking, table_len);
   if (st) return st;
   if (n > 0 && (!y || !scales || !scale_table)) return RANS_ERR_ARG;
@@ -393,6 +411,7 @@ RANS_API int rans_decode_to_values(const uint8_t *in, uint64_t in_bytes,
                                    const rans_tables *tables, const rans_chunking *chunking,
                                    float *values, void *workspace, uint64_t workspace_bytes,
                                    void *stream) {
+  NvtxRange nvtx_("rans_decode_to_values");
   int st = float_args(tables, chunking, table_len);
   if (st) return st;
   if (n > 0 && (!values || !scales || !scale_table)) return RANS_ERR_ARG;

@@ -188,3 +188,28 @@ def test_table_refresh_at_precision_15():
     assert offs.tolist() == woffs.tolist()
     assert np.array_equal(data, want)
     assert np.array_equal(dec, np.asarray(w["symbols"]).reshape(-1))
+
+
+@pytest.mark.parametrize("fmt,W", [("rans64", 1), ("rans64", 4), ("rans64", 32),
+                                   ("rans32_16", 8), ("rans32_16", 32)])
+def test_rows_of_two_and_three_entries(fmt, W):
+    """Rows with only the escape bucket, one symbol of width 2^p - 1 or of
+    width 1 beside the escape, and two halves; symbols in and far out of
+    each row's range."""
+    prec = 16 if fmt == "rans64" else 15
+    M = 1 << prec
+    c = np.array([[0, M, 0], [0, M - 1, M], [0, 1, M], [0, M // 2, M]], np.int32)
+    l = np.array([2, 3, 3, 3], np.int32)
+    o = np.array([0, -1, 5, 100], np.int32)
+    rng = np.random.Generator(np.random.PCG64(41))
+    n = 5000
+    idx = rng.integers(0, 4, size=n).astype(np.int32)
+    sym = (o[idx] + rng.integers(-2, 3, size=n)).astype(np.int64)
+    sym[::37] = rng.integers(-2**31, 2**31 - 1, size=sym[::37].size)
+    w = dict(symbols=sym.astype(np.int32), indexes=idx, W=W, index_block=1, fmt=fmt,
+             precision=prec, chunking=dict(kind="contig", n_streams=7))
+    tables = tables_from_numpy(c, l, o, precision=prec)
+    data, offs, dec, _, _ = gpu_encode_decode(w, tables)
+    want, woffs = oracle_encode(w, c, l, o)
+    assert offs.tolist() == woffs.tolist() and np.array_equal(data, want)
+    assert np.array_equal(dec, w["symbols"])
