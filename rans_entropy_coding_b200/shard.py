@@ -40,3 +40,38 @@ def global_index(local_offsets, group=None):
         out.append(offs[1:] + run)
         run += int(offs[counts[r]].item())
     return torch.cat(out), base, counts
+
+
+def gather_container(data, local_offsets, dst=0, group=None):
+    """The other exchange the sharded container allows: every rank's bytes
+    sent to rank ``dst`` (point to point, rank order), which returns
+    (data, global_offsets) of the whole container; the other ranks return
+    None.  data: this rank's uint8 tensor of at least local_offsets[-1]
+    bytes, on the device the process group moves."""
+    gidx, base, counts = global_index(local_offsets, group)
+    me, world = dist.get_rank(group), dist.get_world_size(group)
+    mine = int(local_offsets[-1].item())
+    if me != dst:
+        if mine:
+            dist.send(data[:mine].contiguous(), dst=dst, group=group)
+        return None
+    total = int(gidx[-1].item())
+    out = torch.empty(total, dtype=torch.uint8, device=data.device)
+    bounds, run = [], 0
+    ends = gidx.tolist()
+    first = 0
+    for r in range(world):
+        n_r = counts[r]
+        size = int(ends[first + n_r]) - int(ends[first])
+        bounds.append((run, size))
+        run += size
+        first += n_r
+    for r in range(world):
+        start, size = bounds[r]
+        if size == 0:
+            continue
+        if r == me:
+            out[start:start + size] = data[:size]
+        else:
+            dist.recv(out[start:start + size], src=r, group=group)
+    return out, gidx

@@ -44,8 +44,13 @@ def _rank(rank, world, port, out):
         offs = O.encode_with_indexes(sym, w["indexes"], c, l, o, w["chunking"], W=32,
                                      streams=list(range(8 + rank)))[1]
         gidx, base, counts = shard.global_index(torch.from_numpy(offs.astype(np.int64)))
+        streams_data = O.encode_with_indexes(sym, w["indexes"], c, l, o, w["chunking"], W=32,
+                                             streams=list(range(8 + rank)))[0]
+        got = shard.gather_container(torch.from_numpy(streams_data.copy()),
+                                     torch.from_numpy(offs.astype(np.int64)), dst=0)
+        whole = None if got is None else (got[0].numpy().tobytes(), got[1].numpy().tolist())
         out[rank] = (tmax, gathered, gidx.numpy().tolist(), base, counts,
-                     offs.astype(np.int64).tolist())
+                     offs.astype(np.int64).tolist(), whole, streams_data.tobytes())
     finally:
         dist.destroy_process_group()
 
@@ -83,4 +88,17 @@ def test_sharded_container_index():
     assert res[0][4] == [8, 9] and len(g0) == 8 + 9 + 1
     assert res[0][3] == 0 and res[1][3] == o0[-1]            # rank bases
     assert g0 == o0 + [v + o0[-1] for v in o1[1:]]
+
+
+def test_gathered_container_is_both_ranks_bytes_in_rank_order():
+    world = 2
+    port = _free_port()
+    with mp.Manager() as m:
+        out = m.dict()
+        mp.spawn(_rank, args=(world, port, out), nprocs=world, join=True)
+        res = dict(out)
+    assert res[1][6] is None                                 # only the destination gets it
+    data, offsets = res[0][6]
+    assert data == res[0][7] + res[1][7]
+    assert offsets == res[0][2]
 
