@@ -214,7 +214,7 @@ def load_inputs(rank, group, images=N_IMAGES, workload="batch", interleave=None)
         ids = shard_images(rank, images)
         w = WL.y_batch(n_images=len(ids), first_image=ids[0], cg=group)
         w["W"] = 32
-    if interleave is not None and workload not in ("batch", "sweep"):
+    if interleave is not None:
         w["W"] = interleave
     return w
 
@@ -234,7 +234,7 @@ def workload_name(w, args):
             workload_name(dict(w, fmt="rans64", alias=False), args), w["fmt"],
             " alias" if w.get("alias") else "", w["precision"])
     if args.workload == "batch":
-        return WORKLOAD
+        return WORKLOAD if w["W"] == 32 else WORKLOAD.replace("W=32", "W=%d" % w["W"])
     if args.workload == "float":
         return ("float_batch%d: %dx192x68x120 float32 y, means and scales per element, "
                 "64-entry scale table, tiles 64x64 x %d channels, W=32" %
