@@ -21,7 +21,8 @@ def _row_from(g):
 
 @pytest.mark.parametrize("name", ["e1_two_symbols.txt", "e2_escape_positive.txt",
                                   "e3_renorm_word.txt", "e6_escape_negative.txt",
-                                  "e7_two_pieces.txt", "e8_bypass_word.txt"])
+                                  "e7_two_pieces.txt", "e8_bypass_word.txt",
+                                  "e9_two_lanes.txt"])
 def test_hand_worked_streams(golden, name):
     g = golden(name)
     cdf, lengths, offsets = _row_from(g)
