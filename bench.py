@@ -196,7 +196,24 @@ def shard_images(rank, images=N_IMAGES):
     return list(range(images * rank, images * (rank + 1)))
 
 
-def load_inputs(rank, group, images=N_IMAGES, workload="batch", interleave=None):
+def shard_streams(w, world, rank):
+    """Rank ``rank``'s block of a contiguously chunked workload (the sweep):
+    a contiguous range of whole streams with its symbols and row indexes
+    (strong scaling: the ranks split one fixed workload; streams are
+    independent, so no exchange is needed).  Returns the rank's workload dict
+    with "stream_block" = (first stream, count, global symbol count, global
+    stream count)."""
+    from rans_entropy_coding_b200 import shard
+    sym = np.asarray(w["symbols"]).reshape(-1)
+    blk = int(w["index_block"])
+    b = shard.stream_block(sym.size, int(w["chunking"]["n_streams"]), world, rank, blk)
+    (a, e), (i0, i1) = b["elems"], b["index_range"]
+    return dict(w, symbols=sym[a:e], indexes=np.asarray(w["indexes"])[i0:i1],
+                chunking=b["chunking"],
+                stream_block=(b["first"], b["count"], sym.size, int(w["chunking"]["n_streams"])))
+
+
+def load_inputs(rank, group, images=N_IMAGES, workload="batch", interleave=None, world=1):
     if workload == "tiny":
         w = WL.tiny()
     elif workload == "z":
@@ -205,6 +222,8 @@ def load_inputs(rank, group, images=N_IMAGES, workload="batch", interleave=None)
         w = WL.y_latent(W=interleave or 32)
     elif workload == "sweep":
         w = WL.sweep(log2_n=28)
+        if world > 1:  # split by stream range
+            w = shard_streams(w, world, rank)
     elif workload == "r16":
         w = WL.r16_rows()
     elif workload == "float":
@@ -241,10 +260,15 @@ def workload_name(w, args):
                 (args.images, args.images, args.group))
     n = int(np.asarray(w["symbols"]).size)
     rows = len(w["scales"]) if "scales" in w else len(w["pmf_lengths"])
-    return "%s: %d %s symbols, %d %s rows, %s %d streams, W=%d, index block %d" % (
+    n_streams = w["chunking"].get("n_streams", 0)
+    split = w.get("stream_block")
+    if split:  # the whole workload, then the ranks' split
+        n, n_streams = split[2], split[3]
+    name = "%s: %d %s symbols, %d %s rows, %s %d streams, W=%d, index block %d" % (
         args.workload, n, np.asarray(w["symbols"]).dtype, rows,
-        "Gaussian" if "scales" in w else "pmf", w["chunking"]["kind"],
-        w["chunking"].get("n_streams", 0), w["W"], w["index_block"])
+        "Gaussian" if "scales" in w else "pmf", "contig" if split else w["chunking"]["kind"],
+        n_streams, w["W"], w["index_block"])
+    return name + (", split by stream range over the ranks" if split else "")
 
 
 # --------------------------------------------------------- CPU oracle leg --
@@ -324,8 +348,8 @@ def run_ours(args, world, rank, local):
     rb.lib()
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
-    w = apply_format(load_inputs(rank, args.group, args.images, args.workload, args.interleave),
-                     args.format, args.alias)
+    w = apply_format(load_inputs(rank, args.group, args.images, args.workload, args.interleave,
+                                 world), args.format, args.alias)
     fmt, prec = w["fmt"], w["precision"]
     sym_np = np.ascontiguousarray(np.asarray(w["symbols"]).reshape(-1))
     idx_np = np.ascontiguousarray(w["indexes"], dtype=np.int32)
@@ -442,7 +466,10 @@ def run_ours(args, world, rank, local):
                                 "images=%d group=%d" % (args.images, args.group))
                if args.workload == "batch" else None)
     ach = dec_gbs if dominant == "decode" else enc_gbs
-    total_syms = n * world
+    # strong scaling when the ranks split one workload's streams (the
+    # sweep), weak when each rank codes its own images
+    split = w.get("stream_block")
+    total_syms = split[2] if split else n * world
     ms_per_step = elapsed_ms / args.steps
     if flush is not None:  # the steps' coding time, without the L2 flushes
         ms_per_step = tab_ms + enc_ms + dec_ms
@@ -558,13 +585,15 @@ def run_ours(args, world, rank, local):
         line = {
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
-            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-            "dtype": "u64" if fmt == "rans64" else "u32",
+            "higher_is_better": True, "scaling": "strong" if split else "weak",
+            "vs_baseline": None, "dtype": "u64" if fmt == "rans64" else "u32",
             "data": "synthetic",
             "config": {"workload": workload_name(w, args), "symbols_per_gpu": n,
                        "streams_per_gpu": S, "channel_group": args.group,
                        "interleave": w["W"], "rows": K,
-                       "lmax": Lmax, "parallelism": "shard-by-image x%d" % world,
+                       "lmax": Lmax,
+                       "parallelism": ("shard-by-stream-range x%d" if split else
+                                       "shard-by-image x%d") % world,
                        "l2": ("inputs larger than L2 (%d MB read per encode)" %
                               (n * (sym_b + 4) // 2**20)) if flush is None else
                              "L2 flushed before every step (256 MB write, not timed)"},

@@ -366,8 +366,10 @@ int rans_decode_with_indexes(const uint8_t *in, uint64_t in_bytes,
  * library.
  *   The workspace is a 32 MiB array inside the library that every GPU loading
  *   it keeps until exit; inputs needing more (rans_encode_workspace_bytes)
- *   return RANS_ERR_CAPACITY.  The first call on a device looks the array's
- *   device address up (call it once before any stream capture).  All calls
+ *   return RANS_ERR_CAPACITY.  The first call in a device's CUDA context
+ *   looks the array's device address up (call it once before any stream
+ *   capture); after a device reset the new context's first call looks it up
+ *   again.  All calls
  *   share the array: calls that overlap on the GPU race, so serialise them.
  *   Device errors cannot be read with rans_get_status here; instead
  *   stream_offsets[S] is set to UINT64_MAX.  Other arguments, outputs and

@@ -256,8 +256,22 @@ def decode_stream(data, rows, cdfs, lengths, offsets, W=1, fmt="rans64", precisi
 
 
 # ---------------------------------------------------------------- chunking --
-def stream_positions(n, chunking):
-    """Flat element positions of every stream, in coding order.
+def num_streams(n, chunking):
+    """Number of streams of a chunking of n elements."""
+    kind = chunking["kind"]
+    if kind == "contig":
+        return int(chunking["n_streams"])
+    if kind == "explicit":
+        return len(chunking["starts"]) - 1
+    if kind == "tiled":
+        B, C, H, Wd = (int(v) for v in chunking["shape"])
+        cg, th, tw = int(chunking["cg"]), int(chunking["th"]), int(chunking["tw"])
+        return B * (-(-C // cg)) * (-(-H // th)) * (-(-Wd // tw))
+    raise ValueError("unknown chunking kind %r" % kind)
+
+
+def stream_position(n, chunking, k):
+    """Flat element positions of stream k, in coding order.
 
     ``chunking`` is a dict: {"kind": "contig", "n_streams": S} |
     {"kind": "explicit", "starts": [S+1 offsets]} |
@@ -267,32 +281,34 @@ def stream_positions(n, chunking):
     if kind == "contig":
         S = int(chunking["n_streams"])
         per = -(-n // S) if S > 0 else 0
-        out = []
-        for k in range(S):
-            a = min(k * per, n)
-            b = min((k + 1) * per, n)
-            out.append(np.arange(a, b, dtype=np.int64))
-        return out
+        a = min(k * per, n)
+        b = min((k + 1) * per, n)
+        return np.arange(a, b, dtype=np.int64)
     if kind == "explicit":
         st = np.asarray(chunking["starts"], dtype=np.int64)
-        return [np.arange(st[k], st[k + 1], dtype=np.int64) for k in range(st.size - 1)]
+        return np.arange(st[k], st[k + 1], dtype=np.int64)
     if kind == "tiled":
         B, C, H, Wd = (int(v) for v in chunking["shape"])
         cg, th, tw = int(chunking["cg"]), int(chunking["th"]), int(chunking["tw"])
         assert B * C * H * Wd == n
-        out = []
-        for b in range(B):
-            for c0 in range(0, C, cg):
-                for h0 in range(0, H, th):
-                    for w0 in range(0, Wd, tw):
-                        cs = np.arange(c0, min(c0 + cg, C), dtype=np.int64)
-                        hs = np.arange(h0, min(h0 + th, H), dtype=np.int64)
-                        ws = np.arange(w0, min(w0 + tw, Wd), dtype=np.int64)
-                        pos = ((b * C + cs[:, None, None]) * H + hs[None, :, None]) * Wd \
-                            + ws[None, None, :]
-                        out.append(pos.reshape(-1))
-        return out
+        ng, nty, ntx = -(-C // cg), -(-H // th), -(-Wd // tw)
+        # streams are numbered (b, channel group, tile row, tile column)
+        b, r = divmod(k, ng * nty * ntx)
+        g, r = divmod(r, nty * ntx)
+        ty, tx = divmod(r, ntx)
+        c0, h0, w0 = g * cg, ty * th, tx * tw
+        cs = np.arange(c0, min(c0 + cg, C), dtype=np.int64)
+        hs = np.arange(h0, min(h0 + th, H), dtype=np.int64)
+        ws = np.arange(w0, min(w0 + tw, Wd), dtype=np.int64)
+        pos = ((b * C + cs[:, None, None]) * H + hs[None, :, None]) * Wd + ws[None, None, :]
+        return pos.reshape(-1)
     raise ValueError("unknown chunking kind %r" % kind)
+
+
+def stream_positions(n, chunking):
+    """Flat element positions of every stream, in coding order (a list with
+    one array per stream)."""
+    return [stream_position(n, chunking, k) for k in range(num_streams(n, chunking))]
 
 
 def _rows_for(positions, indexes, index_block):

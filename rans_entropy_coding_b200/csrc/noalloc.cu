@@ -11,13 +11,18 @@
 // which every GPU that loads the library keeps until the process exits.
 //
 // Host code cannot use the array's name as a device address, so the first
-// call on each device looks the address up with cudaGetSymbolAddress (with
-// that device current) and caches it; that first call should therefore come
-// before any stream capture.  All calls share the array: calls whose work
-// overlaps on the GPU (concurrent streams, or several host threads on one
-// device) race on it and must be serialised by the caller.  Nothing here
-// allocates: no cudaMalloc, no cudaFree, no allocating library routine.
+// call in each CUDA context looks the address up with cudaGetSymbolAddress
+// (with that context's device current) and caches it beside the context's
+// ID; that first call should therefore come before any stream capture.  A
+// context that is destroyed and created again (a device reset) gets a new
+// ID, so the next call looks the address up again instead of using the old
+// one.  All calls share the array: calls whose work overlaps on the GPU
+// (concurrent streams, or several host threads on one device) race on it
+// and must be serialised by the caller.  Nothing here allocates: no
+// cudaMalloc, no cudaFree, no allocating library routine.
 #include <mutex>
+
+#include <cuda.h>  // CUcontext / CUresult types; the entry points are fetched at run time
 
 #include "rans_common.cuh"
 #include "rans_internal.h"
@@ -29,21 +34,67 @@ constexpr uint64_t kStaticWorkspaceBytes = 32ull << 20;  // 32 MiB
 __device__ __align__(256) unsigned char g_static_workspace[kStaticWorkspaceBytes];
 
 std::mutex g_setup_mutex;
-void *g_workspace_addr[128] = {nullptr};
 
-// Device address of the static workspace on the current device (looked up
-// once per device).
+// The context a lookup was made in, by the driver's context ID (unique for
+// the life of the process, unlike a context handle, which can be reused).
+struct CachedAddr {
+  unsigned long long ctx_id;
+  void *addr;
+};
+CachedAddr g_workspace_addr[128] = {};
+
+// Driver entry points, fetched through the runtime so that the library
+// needs no link against the driver library.
+typedef CUresult (*CtxGetCurrentFn)(CUcontext *);
+typedef CUresult (*CtxGetIdFn)(CUcontext, unsigned long long *);
+CtxGetCurrentFn g_ctx_get_current = nullptr;
+CtxGetIdFn g_ctx_get_id = nullptr;
+
+// ID of the context current on this thread; 0 when none is (yet) current.
+// Called with g_setup_mutex held.
+int current_context_id(unsigned long long *id) {
+  *id = 0;
+  if (g_ctx_get_current == nullptr || g_ctx_get_id == nullptr) {
+    cudaDriverEntryPointQueryResult q1, q2;
+    void *f1 = nullptr, *f2 = nullptr;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &f1, cudaEnableDefault, &q1) != cudaSuccess ||
+        q1 != cudaDriverEntryPointSuccess || f1 == nullptr ||
+        cudaGetDriverEntryPoint("cuCtxGetId", &f2, cudaEnableDefault, &q2) != cudaSuccess ||
+        q2 != cudaDriverEntryPointSuccess || f2 == nullptr)
+      return RANS_ERR_CUDA;
+    g_ctx_get_current = reinterpret_cast<CtxGetCurrentFn>(f1);
+    g_ctx_get_id = reinterpret_cast<CtxGetIdFn>(f2);
+  }
+  CUcontext ctx = nullptr;
+  if (g_ctx_get_current(&ctx) != CUDA_SUCCESS) return RANS_ERR_CUDA;
+  if (ctx == nullptr) return RANS_OK;
+  return g_ctx_get_id(ctx, id) == CUDA_SUCCESS ? RANS_OK : RANS_ERR_CUDA;
+}
+
+// Device address of the static workspace in the current device's context
+// (looked up once per context).
 int static_workspace(void **addr) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 128) return RANS_ERR_CUDA;
   std::lock_guard<std::mutex> lock(g_setup_mutex);
-  if (g_workspace_addr[dev] == nullptr) {
-    void *p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_static_workspace) != cudaSuccess || p == nullptr)
-      return RANS_ERR_CUDA;
-    g_workspace_addr[dev] = p;
+  unsigned long long id = 0;
+  int st = current_context_id(&id);
+  if (st) return st;
+  CachedAddr &e = g_workspace_addr[dev];
+  if (id != 0 && e.addr != nullptr && e.ctx_id == id) {
+    *addr = e.addr;
+    return RANS_OK;
   }
-  *addr = g_workspace_addr[dev];
+  // the lookup also makes the device's context current when none was
+  void *p = nullptr;
+  if (cudaGetSymbolAddress(&p, g_static_workspace) != cudaSuccess || p == nullptr)
+    return RANS_ERR_CUDA;
+  st = current_context_id(&id);
+  if (st) return st;
+  if (id == 0) return RANS_ERR_CUDA;
+  e.ctx_id = id;
+  e.addr = p;
+  *addr = p;
   return RANS_OK;
 }
 

@@ -75,3 +75,39 @@ def gather_container(data, local_offsets, dst=0, group=None):
         else:
             dist.recv(out[start:start + size], src=r, group=group)
     return out, gidx
+
+
+def stream_block(n, n_streams, world, rank, index_block=1):
+    """Rank ``rank``'s share of a contiguous chunking of n elements into
+    n_streams streams (stream k covers [k*per, min((k+1)*per, n)),
+    per = ceil(n / n_streams)): a contiguous block of whole streams, the
+    blocks of ranks 0 .. world-1 covering all streams in order, their sizes
+    differing by at most one stream.  Streams are independent ("kompressor"
+    README, Why), so each rank codes its block with no exchange and the
+    ranks' bytes in rank order are the single-GPU container.
+
+    Returns a dict: ``first`` and ``count`` (the rank's streams),
+    ``elems`` (the element range [a0, b) the rank reads: its streams' range
+    [a, b) widened down to the start of the index block holding a, so that
+    its row indexes are a plain slice), ``index_range`` ([a0 // index_block,
+    ceil(b / index_block))) and ``chunking`` (the rank's chunking of its
+    b - a0 elements: contiguous when that reproduces the global stream
+    boundaries, else explicit with those boundaries)."""
+    if n_streams < 1 or world < 1 or not 0 <= rank < world or index_block < 1:
+        raise ValueError("bad stream block request")
+    per = -(-n // n_streams) if n else 0
+    base, extra = divmod(n_streams, world)
+    first = rank * base + min(rank, extra)
+    count = base + (1 if rank < extra else 0)
+    a = min(first * per, n)
+    b = min((first + count) * per, n)
+    a0 = a - a % index_block
+    bounds = [min((first + k) * per, n) - a0 for k in range(count + 1)]
+    local_per = -(-(b - a0) // count) if count else 0
+    if count and a0 == a and all(min(k * local_per, b - a) == bounds[k]
+                                 for k in range(count + 1)):
+        chunking = dict(kind="contig", n_streams=count)
+    else:
+        chunking = dict(kind="explicit", starts=bounds)
+    return dict(first=first, count=count, elems=(a0, b),
+                index_range=(a0 // index_block, -(-b // index_block)), chunking=chunking)

@@ -79,3 +79,28 @@ def oracle_encode(w, c, l, o, streams=None):
     return O.encode_with_indexes(sym, w["indexes"], c, l, o, w["chunking"], W=w["W"],
                                  index_block=w["index_block"], streams=streams, fmt=fmt_of(w),
                                  precision=precision_of(w), alias=alias_of(w))
+
+
+def oracle_encode_parallel(w, c, l, o, workers=None):
+    """The oracle's container encode of every stream of the workload, one
+    stream per oracle call spread over host threads (the C oracle runs
+    without the GIL); returns (bytes, offsets uint64[S+1]) like
+    oracle_encode."""
+    import concurrent.futures as cf
+    import os
+    flat = np.asarray(w["symbols"]).reshape(-1)
+    idx = np.asarray(w["indexes"], dtype=np.int32)
+    blk = int(w["index_block"])
+    S = O.num_streams(flat.size, w["chunking"])
+
+    def one(k):
+        p = O.stream_position(flat.size, w["chunking"], k)
+        return O.encode_stream(flat[p].astype(np.int64), idx[p // blk], c, l, o, w["W"],
+                               fmt_of(w), precision_of(w), alias_of(w))
+
+    with cf.ThreadPoolExecutor(max_workers=workers or os.cpu_count() or 1) as ex:
+        parts = list(ex.map(one, range(S)))
+    offs = np.zeros(S + 1, dtype=np.uint64)
+    offs[1:] = np.cumsum([p.size for p in parts], dtype=np.uint64)
+    data = np.concatenate(parts) if parts else np.zeros(0, dtype=np.uint8)
+    return data, offs

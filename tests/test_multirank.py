@@ -102,3 +102,46 @@ def test_gathered_container_is_both_ranks_bytes_in_rank_order():
     assert data == res[0][7] + res[1][7]
     assert offsets == res[0][2]
 
+
+
+def _sweep_rank(rank, world, port, out):
+    """Rank ``rank`` codes its stream block of a small sweep with the oracle
+    and joins the container index."""
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank),
+                      WORLD_SIZE=str(world))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        w = bench.shard_streams(WL.sweep(log2_n=16, n_streams=7), world, rank)
+        c, l = O.build_cdfs_from_pmfs(w["pmfs"], w["pmf_lengths"], w["tail"])
+        data, offs = O.encode_with_indexes(w["symbols"], w["indexes"], c, l, w["offsets"],
+                                           w["chunking"], W=32, index_block=w["index_block"])
+        gidx, base, counts = shard.global_index(torch.from_numpy(offs.astype(np.int64)))
+        out[rank] = (w["stream_block"], w["chunking"]["kind"], gidx.numpy().tolist(), base,
+                     counts, data.tobytes())
+    finally:
+        dist.destroy_process_group()
+
+
+def test_two_ranks_split_the_sweep_by_stream_range():
+    """The sweep split by stream range: rank 0 codes streams 0-3 and rank 1
+    streams 4-6 (stream 4 starts inside an index block and the last stream
+    is short, so rank 1 reads from the block's start and needs explicit
+    boundaries); the all-gathered index and the ranks' bytes in rank order
+    are the container one process codes from the whole sweep."""
+    world = 2
+    port = _free_port()
+    with mp.Manager() as m:
+        out = m.dict()
+        mp.spawn(_sweep_rank, args=(world, port, out), nprocs=world, join=True)
+        res = dict(out)
+    n = 1 << 16
+    assert res[0][0] == (0, 4, n, 7) and res[1][0] == (4, 3, n, 7)
+    assert res[0][1] == "contig" and res[1][1] == "explicit"
+    assert res[0][2] == res[1][2] and res[0][4] == [4, 3]
+    w = WL.sweep(log2_n=16, n_streams=7)
+    c, l = O.build_cdfs_from_pmfs(w["pmfs"], w["pmf_lengths"], w["tail"])
+    data, offs = O.encode_with_indexes(w["symbols"], w["indexes"], c, l, w["offsets"],
+                                       w["chunking"], W=32, index_block=w["index_block"])
+    assert res[0][2] == offs.astype(np.int64).tolist()
+    assert res[1][3] == int(offs[4])
+    assert res[0][5] + res[1][5] == data.tobytes()

@@ -37,6 +37,30 @@ def test_noalloc_encode_matches_regular_encode():
         torch.cuda.synchronize()
         assert torch.equal(offs2, want_offs)
         assert torch.equal(out2[:total], want_bytes)
+    # device errors are marked in the outputs (stream_offsets[S] = UINT64_MAX,
+    # -1 read as int64); the next good call, which starts from a cleared
+    # status word in the shared array, gives the regular result again
+    bad = idx.clone()
+    bad[4321] = 64                                  # rows are 0..63
+    small = torch.zeros(total // 2, dtype=torch.uint8, device="cuda")
+    for case in ("index", "capacity"):
+        offs3 = torch.zeros_like(offs)
+        if case == "index":
+            st = rb.rans_encode_with_indexes_noalloc(sym, bad, sym.numel(), tables, ch, out2,
+                                                     offs3)
+        else:
+            st = rb.rans_encode_with_indexes_noalloc(sym, idx, sym.numel(), tables, ch, small,
+                                                     offs3)
+        rb.check(st, "noalloc encode (%s error)" % case)
+        torch.cuda.synchronize()
+        assert int(offs3[-1].item()) == -1, case
+        out4 = torch.zeros_like(out2)
+        offs4 = torch.zeros_like(offs)
+        rb.check(rb.rans_encode_with_indexes_noalloc(sym, idx, sym.numel(), tables, ch, out4,
+                                                     offs4), "noalloc encode after an error")
+        torch.cuda.synchronize()
+        assert torch.equal(offs4, want_offs), case
+        assert torch.equal(out4[:total], want_bytes), case
     # past the fixed workspace size: refused with a clear error, nothing launched
     big = rb.Chunking.contig(1, 32)
     st = rb.lib().rans_encode_with_indexes_noalloc(None, 0, None, 1 << 30, tables.c, big.c, None,
