@@ -33,6 +33,8 @@
 //  Tables are staged into shared memory with bulk copies when they fit.
 #include <type_traits>
 
+#include <cuda.h>  // CUtensorMap
+
 #include "rans_common.cuh"
 #include "rans_internal.h"
 
@@ -729,6 +731,566 @@ __host__ __device__ inline uint32_t dec_table_bytes(int mode, const DecCtx &c) {
                    : (mode == 2 ? c.meta_bytes + c.start_bytes : 0u);
 }
 
+// ---------------------------------------------- W = 32, tile-staged I/O ----
+// Tiled streams whose tile rows are whole 16-byte units go through a leaner
+// warp decoder: the row indexes of 4 tile rows of one channel (a chunk of
+// ww / 8 groups) arrive in a per-warp shared-memory ring with one
+// tensor-tile copy, each decoded value overwrites its row index in the ring,
+// and the chunk leaves with one tensor-tile store.  No thread computes an
+// element address; the copy engine walks the tile's rows and channels.
+// The ring has two halves of 4 rows x up to 64 int32: while chunk k decodes
+// from one half, chunk k + 1 lands in the other.  Its load is issued three
+// groups before the end of chunk k, when chunk k - 1's store has long read
+// that half, and finds the chunk in L2: every chunk is prefetched into L2
+// three chunks ahead.
+constexpr uint32_t kTileWaitTries = 1u << 22;  // bounded mbarrier waits (about 4 s)
+
+struct TileMaps {
+  CUtensorMap idx[2];  // row indexes: box (tile width, 4, 1); [1]: last tile column
+  CUtensorMap out[2];  // decoded symbols, same boxes
+};
+
+// One group of a full 32-lane group: lookup, state update, refill; returns
+// the decoded value (symbol + offset).  The escape ballot is taken beside the
+// refill; a group with an escape goes down the lane-serial path.
+template <class F, bool SEARCH>
+__device__ __forceinline__ int32_t dec_group_val(WarpDec<F> &st, const RowMeta &m,
+                                                 const uint16_t *starts, const uint32_t *slots,
+                                                 const typename F::Word *words, uint64_t nw,
+                                                 uint32_t sh) {
+  const int lane = threadIdx.x & 31;
+  const uint32_t cum = F::cum16(st.x, sh);
+  const uint32_t sym = lookup<SEARCH, true>(cum, m, starts, slots, true);
+  const uint32_t start = starts[m.bucket_base + sym];
+  const uint32_t freq = width_of(start, starts[m.bucket_base + sym + 1]);
+  const typename F::State x = F::dec_step(st.x, cum, start, freq, sh);
+  const bool esc = sym == m.maxv;
+  const bool need = x < F::kLow;
+  const uint32_t src = (uint32_t)lane >= st.off ? st.w0 : st.w1;
+  const uint32_t nm = __ballot_sync(kFull, need);
+  const bool any_esc = __any_sync(kFull, esc);
+  const uint32_t j = st.off + __popc(nm & lanemask_lt());
+  const uint32_t wv = __shfl_sync(kFull, src, j & 31);
+  int32_t val = (int32_t)sym + m.offset;
+  if (!any_esc) {
+    st.x = need ? ((x << F::kWordBits) | wv) : x;
+    st.off += __popc(nm);
+    if (st.off >= 32) {
+      st.w0 = st.w1;
+      st.w1 = st.w2;
+      st.cur += 32;
+      st.off -= 32;
+      st.w2 = word_at(words, nw, st.cur + 64 + lane);
+    }
+  } else {
+    const EscapeResult<F> er = escape_group<F>(x, true, esc, m.maxv, st.cur + st.off, words, nw);
+    st.x = er.x;
+    if (esc) val = (int32_t)(er.val + (int64_t)m.offset);
+    st.bad |= er.bad;
+    st.cur = er.cur;
+    st.off = 0;
+    load_window(st, words, nw);
+  }
+  return val;
+}
+
+// Where a tiled stream's chunks are: the tensor-tile coordinates (x = first
+// column, y = row, z = image * C + channel) of its next chunk, stepped 4 rows
+// at a time through the tile and then to the next channel.
+struct ChunkPos {
+  int32_t y, z, y0, y1;  // y1 = y0 + tile height
+  __device__ __forceinline__ void next() {
+    y += 4;
+    if (y == y1) {
+      y = y0;
+      ++z;
+    }
+  }
+};
+
+// Decodes stream s with tile staging; false when a bounded wait gave up (the
+// warp then stops, its copies drained).
+template <class F, bool SEARCH>
+__device__ __forceinline__ bool decode_tile_stream(const DecCtx &c, const TileMaps &maps,
+                                                   const RowMeta *meta, const uint16_t *starts,
+                                                   const uint32_t *slots, uint32_t ring,
+                                                   int32_t *ring_p, uint32_t bar0,
+                                                   uint32_t &par, int64_t s) {
+  using State = typename F::State;
+  using Word = typename F::Word;
+  const int lane = threadIdx.x & 31;
+  const Geom &g = c.g;
+  const StreamDesc d = stream_desc(g, s);
+  const Word *words = nullptr;
+  uint64_t nw = 0;
+  if (!d.ok || !stream_bounds<F>(c, s, 32, words, nw)) {
+    if (lane == 0) report(c.status, d.ok ? RANS_ERR_CORRUPT : RANS_ERR_ARG, s);
+    return true;
+  }
+  if (lane == 0)
+    bulk_prefetch_l2(reinterpret_cast<const char *>(c.in),
+                     reinterpret_cast<const char *>(c.in) + c.in_bytes,
+                     reinterpret_cast<const char *>(words + 64), sizeof(Word) * (nw - 64));
+  const uint32_t sh = F::shift(c.sh);
+  const uint32_t kmax = (uint32_t)c.K - 1u;
+  // the tile: image b, channel group gi, tile row ty, tile column tx
+  const int64_t per_img = g.ng * g.nty * g.ntx;
+  const int64_t b = s / per_img, r0 = s - b * per_img;
+  const int64_t gi = r0 / (g.nty * g.ntx), r1 = r0 - gi * (g.nty * g.ntx);
+  const int64_t ty = r1 / g.ntx, tx = r1 - ty * g.ntx;
+  const int32_t x0 = (int32_t)(tx * g.tw);
+  const int32_t ww = d.t.ww, hh = d.t.hh;
+  const int cls = ww == (int32_t)g.tw ? 0 : 1;
+  const void *imap = &maps.idx[cls];
+  const void *omap = &maps.out[cls];
+  const int32_t Gc = ww >> 3;              // groups per chunk: 4 rows x ww / 32
+  const uint32_t cbytes = 16u * (uint32_t)ww;
+  const int32_t M = (int32_t)(d.n / (4 * ww));
+  ChunkPos ld, sd;
+  ld.y0 = ld.y = (int32_t)(ty * g.th);
+  ld.y1 = ld.y0 + hh;
+  ld.z = (int32_t)(b * g.C + gi * g.cg);
+  sd = ld;
+  ChunkPos pf = ld;  // the next chunk to prefetch into L2
+  const uint32_t bar1 = bar0 + 8;
+  // chunk 0 into half 0, once earlier stores have read the ring; chunks 1
+  // and 2 into L2
+  __syncwarp();
+  if (lane == 0) {
+    tma::bulk_wait_read();
+    tma::fence_proxy_async();
+    tma::arrive_expect(bar0, cbytes);
+    tma::load_3d(ring, imap, x0, ld.y, ld.z, bar0);
+  }
+  ld.next();
+  pf.next();
+  for (int32_t q = 1; q < 3 && q < M; ++q) {
+    if (lane == 0) tma::prefetch_l2_3d(imap, x0, pf.y, pf.z);
+    pf.next();
+  }
+  const int32_t jload = Gc > 3 ? Gc - 3 : 0;  // the group after which chunk k + 1 loads
+
+  WarpDec<F> st;
+  st.x = (State)__ldg(words + 2 * lane) | ((State)__ldg(words + 2 * lane + 1) << F::kWordBits);
+  st.cur = 64;
+  st.off = 0;
+  load_window(st, words, nw);
+  st.rmax = 0;
+  st.bad = false;
+  auto meta_of = [&](uint32_t r) -> RowMeta {
+    st.rmax = max(st.rmax, r);
+    return row_meta(meta, min(r, kmax));
+  };
+  // loads in flight, by half (bit h)
+  uint32_t pending = 1u;
+  // a bounded wait for the chunk in half h; on giving up, a bounded wait for
+  // every load still in flight, and the warp stops
+  auto wait_half = [&](int h) -> bool {
+    const uint32_t bar = h ? bar1 : bar0;
+    const bool ok = tma::wait_bounded(bar, (par >> h) & 1u, kTileWaitTries);
+    if (__all_sync(kFull, ok)) {
+      par ^= 1u << h;
+      pending &= ~(1u << h);
+      return true;
+    }
+    if (lane == 0) report(c.status, RANS_ERR_TIMEOUT, s);
+    for (int q = 0; q < 2; ++q)
+      if (pending >> q & 1u) tma::wait_bounded(q ? bar1 : bar0, (par >> q) & 1u, kTileWaitTries);
+    return false;
+  };
+  if (!wait_half(0)) return false;
+  RowMeta m = meta_of((uint32_t)ring_p[lane]);
+#pragma unroll 1
+  for (int32_t k = 0; k < M; ++k) {
+    const int h = k & 1;
+    int32_t *rh = ring_p + h * (int32_t)(kTileRingHalf / 4);
+#pragma unroll 1
+    for (int32_t j = 0; j < Gc; ++j) {
+      uint32_t rn = 0;
+      if (j + 1 < Gc) {
+        rn = (uint32_t)rh[(j + 1) * 32 + lane];
+      } else if (k + 1 < M) {
+        if (!wait_half(h ^ 1)) return false;
+        rn = (uint32_t)ring_p[(h ^ 1) * (int32_t)(kTileRingHalf / 4) + lane];
+      }
+      const RowMeta mn = meta_of(rn);
+      rh[j * 32 + lane] = dec_group_val<F, SEARCH>(st, m, starts, slots, words, nw, sh);
+      if (j == 0 && k + 3 < M) {
+        if (lane == 0) tma::prefetch_l2_3d(imap, x0, pf.y, pf.z);
+        pf.next();
+      }
+      if (j == jload && k + 1 < M) {
+        // chunk k + 1 into the other half, once chunk k - 1's store has read
+        // it
+        __syncwarp();
+        if (lane == 0) {
+          const uint32_t bar = h ? bar0 : bar1;
+          tma::bulk_wait_read();
+          tma::fence_proxy_async();
+          tma::arrive_expect(bar, cbytes);
+          tma::load_3d(ring + (uint32_t)(h ^ 1) * kTileRingHalf, imap, x0, ld.y, ld.z, bar);
+        }
+        pending |= 1u << (h ^ 1);
+        ld.next();
+      }
+      m = mn;
+    }
+    // chunk k's decoded values go out
+    tma::fence_proxy_async();
+    __syncwarp();
+    if (lane == 0) {
+      tma::store_3d(omap, x0, sd.y, sd.z, ring + (uint32_t)h * kTileRingHalf);
+      tma::bulk_commit();
+    }
+    sd.next();
+  }
+  if (__any_sync(kFull, st.rmax > kmax)) {
+    if (lane == 0) report(c.status, RANS_ERR_INDEX, s);
+    return true;
+  }
+  const bool ok = !st.bad && st.x == F::kLow && st.cur + st.off == nw;
+  if (!__all_sync(kFull, ok) && lane == 0) report(c.status, RANS_ERR_CORRUPT, s);
+  return true;
+}
+
+// ------------------------------------------ unrolled chunks, no branches --
+// The decoder's time per group follows its instruction count: the state
+// chain leaves little independent work, and a group body cut into small
+// blocks by branches (the escape test, the window advance, the chunk
+// bookkeeping) keeps the compiler from overlapping what there is.  For tile
+// widths of 56 and 64 (7 and 8 groups per chunk) a chunk is therefore decoded
+// as one unrolled block: the copy-engine work is predicated on lane 0,
+// escapes are only recorded, and the only branch left is the window
+// advance (about once in seven groups).  A chunk in which any lane met an
+// escape is decoded again from its saved state on the lane-serial path (its
+// row indexes reloaded, since the fast pass overwrote them with values); the
+// fast pass after an escape runs on a wrong state but reads only inside the
+// tables, the register window and the stream's words.
+
+// Word i of the stream (clamped to its last word) where p is nonzero, else
+// `old`, with no branch.
+template <class F>
+__device__ __forceinline__ uint32_t window_word_if(uint32_t p, const typename F::Word *words,
+                                                   uint64_t nw, uint64_t i, uint32_t old) {
+  const typename F::Word *a = words + (i < nw ? i : nw - 1);
+  if constexpr (sizeof(typename F::Word) == 4) {
+    asm("{\n\t.reg .pred q;\n\tsetp.ne.u32 q, %1, 0;\n\t@q ld.global.nc.u32 %0, [%2];\n\t}"
+        : "+r"(old)
+        : "r"(p), "l"(a));
+  } else {
+    asm("{\n\t.reg .pred q;\n\t.reg .u16 h;\n\tsetp.ne.u32 q, %1, 0;\n\t"
+        "@q ld.global.nc.u16 h, [%2];\n\t@q cvt.u32.u16 %0, h;\n\t}"
+        : "+r"(old)
+        : "r"(p), "l"(a));
+  }
+  return old;
+}
+
+// One full group on the fast path: lookup, state update and refill with no
+// branch; a lane whose symbol is the escape bucket only sets `esc`.
+template <class F>
+__device__ __forceinline__ int32_t dec_group_fast(WarpDec<F> &st, const RowMeta &m,
+                                                  const uint16_t *starts, const uint32_t *slots,
+                                                  const typename F::Word *words, uint64_t nw,
+                                                  uint32_t sh, uint32_t &esc) {
+  const int lane = threadIdx.x & 31;
+  const uint32_t cum = F::cum16(st.x, sh);
+  const uint32_t sym = lookup<false, true>(cum, m, starts, slots, true);
+  const uint32_t start = starts[m.bucket_base + sym];
+  const uint32_t freq = width_of(start, starts[m.bucket_base + sym + 1]);
+  const typename F::State x = F::dec_step(st.x, cum, start, freq, sh);
+  esc |= sym == m.maxv ? 1u : 0u;
+  const bool need = x < F::kLow;
+  const uint32_t src = (uint32_t)lane >= st.off ? st.w0 : st.w1;
+  const uint32_t nm = __ballot_sync(kFull, need);
+  const uint32_t wv = __shfl_sync(kFull, src, st.off + __popc(nm & lanemask_lt()));
+  st.x = need ? ((x << F::kWordBits) | wv) : x;
+  st.off += __popc(nm);
+  // the window advances about once in seven groups: behind a branch, so that
+  // no instruction of the other groups reads the register whose load is
+  // still in flight
+  if (st.off >= 32) {
+    st.w0 = st.w1;
+    st.w1 = st.w2;
+    st.cur += 32;
+    st.off -= 32;
+    st.w2 = word_at(words, nw, st.cur + 64 + lane);
+  }
+  return (int32_t)sym + m.offset;
+}
+
+__device__ __forceinline__ void chunk_next_if(ChunkPos &p, bool on) {
+  const int32_t y = p.y + 4;
+  const bool wrap = y == p.y1;
+  p.y = on ? (wrap ? p.y0 : y) : p.y;
+  p.z += on && wrap ? 1 : 0;
+}
+
+template <class F, int GC>
+__device__ __forceinline__ bool decode_tile_stream_fast(const DecCtx &c, const TileMaps &maps,
+                                                        const RowMeta *meta,
+                                                        const uint16_t *starts,
+                                                        const uint32_t *slots, uint32_t ring,
+                                                        int32_t *ring_p, uint32_t bar0,
+                                                        uint32_t &par, int64_t s) {
+  using State = typename F::State;
+  using Word = typename F::Word;
+  constexpr int kJload = GC > 3 ? GC - 3 : 0;  // the group after which chunk k + 1 loads
+  constexpr int kHalfW = (int)(kTileRingHalf / 4);
+  const int lane = threadIdx.x & 31;
+  const Geom &g = c.g;
+  const StreamDesc d = stream_desc(g, s);
+  const Word *words = nullptr;
+  uint64_t nw = 0;
+  if (!d.ok || !stream_bounds<F>(c, s, 32, words, nw)) {
+    if (lane == 0) report(c.status, d.ok ? RANS_ERR_CORRUPT : RANS_ERR_ARG, s);
+    return true;
+  }
+  if (lane == 0)
+    bulk_prefetch_l2(reinterpret_cast<const char *>(c.in),
+                     reinterpret_cast<const char *>(c.in) + c.in_bytes,
+                     reinterpret_cast<const char *>(words + 64), sizeof(Word) * (nw - 64));
+  const uint32_t sh = F::shift(c.sh);
+  const uint32_t kmax = (uint32_t)c.K - 1u;
+  const int64_t per_img = g.ng * g.nty * g.ntx;
+  const int64_t b = s / per_img, t0 = s - b * per_img;
+  const int64_t gi = t0 / (g.nty * g.ntx), t1 = t0 - gi * (g.nty * g.ntx);
+  const int64_t ty = t1 / g.ntx, tx = t1 - ty * g.ntx;
+  const int32_t x0 = (int32_t)(tx * g.tw);
+  const int32_t hh = d.t.hh;
+  const int cls = d.t.ww == (int32_t)g.tw ? 0 : 1;
+  const void *imap = &maps.idx[cls];
+  const void *omap = &maps.out[cls];
+  const uint32_t cbytes = 128u * GC;
+  const int32_t M = (int32_t)(d.n / (32 * GC));
+  ChunkPos ld, sd;
+  ld.y0 = ld.y = (int32_t)(ty * g.th);
+  ld.y1 = ld.y0 + hh;
+  ld.z = (int32_t)(b * g.C + gi * g.cg);
+  sd = ld;
+  ChunkPos pf = ld;
+  const uint32_t bar1 = bar0 + 8;
+  const uint32_t l0 = lane == 0 ? 1u : 0u;
+  __syncwarp();
+  tma::bulk_wait_read_if(l0);
+  tma::fence_proxy_async();
+  tma::arrive_expect_if(l0, bar0, cbytes);
+  tma::load_3d_if(l0, ring, imap, x0, ld.y, ld.z, bar0);
+  ld.next();
+  pf.next();
+  for (int32_t q = 1; q < 3 && q < M; ++q) {
+    tma::prefetch_l2_3d_if(l0, imap, x0, pf.y, pf.z);
+    pf.next();
+  }
+  uint32_t pending = 1u;
+
+  WarpDec<F> st;
+  st.x = (State)__ldg(words + 2 * lane) | ((State)__ldg(words + 2 * lane + 1) << F::kWordBits);
+  st.cur = 64;
+  st.off = 0;
+  load_window(st, words, nw);
+  st.rmax = 0;
+  st.bad = false;
+  auto meta_of = [&](uint32_t r) -> RowMeta {
+    st.rmax = max(st.rmax, r);
+    return row_meta(meta, min(r, kmax));
+  };
+  auto wait_half = [&](int h) -> bool {
+    const uint32_t bar = h ? bar1 : bar0;
+    const bool ok = tma::wait_bounded(bar, (par >> h) & 1u, kTileWaitTries);
+    if (__all_sync(kFull, ok)) {
+      par ^= 1u << h;
+      pending &= ~(1u << h);
+      return true;
+    }
+    if (lane == 0) report(c.status, RANS_ERR_TIMEOUT, s);
+    for (int q = 0; q < 2; ++q)
+      if (pending >> q & 1u) tma::wait_bounded(q ? bar1 : bar0, (par >> q) & 1u, kTileWaitTries);
+    return false;
+  };
+#pragma unroll 1
+  for (int32_t k = 0; k < M; ++k) {
+    const int h = k & 1;
+    if (!wait_half(h)) return false;
+    int32_t *rh = ring_p + h * kHalfW;
+    const uint32_t more1 = k + 1 < M ? 1u : 0u, more3 = k + 3 < M ? 1u : 0u;
+    const WarpDec<F> st0 = st;
+    uint32_t esc = 0;
+    RowMeta m = meta_of((uint32_t)rh[lane]);
+#pragma unroll
+    for (int j = 0; j < GC; ++j) {
+      RowMeta mn = m;
+      if (j + 1 < GC) mn = meta_of((uint32_t)rh[(j + 1) * 32 + lane]);
+      rh[j * 32 + lane] = dec_group_fast<F>(st, m, starts, slots, words, nw, sh, esc);
+      if (j == 0) {
+        tma::prefetch_l2_3d_if(l0 & more3, imap, x0, pf.y, pf.z);
+        chunk_next_if(pf, more3 != 0);
+      }
+      if (j == kJload) {
+        // chunk k + 1 into the other half, once chunk k - 1's store has read it
+        __syncwarp();
+        const uint32_t bar = h ? bar0 : bar1;
+        tma::bulk_wait_read_if(l0 & more1);
+        tma::fence_proxy_async();
+        tma::arrive_expect_if(l0 & more1, bar, cbytes);
+        tma::load_3d_if(l0 & more1, ring + (uint32_t)(h ^ 1) * kTileRingHalf, imap, x0, ld.y,
+                        ld.z, bar);
+        pending |= more1 << (h ^ 1);
+        chunk_next_if(ld, more1 != 0);
+      }
+      m = mn;
+    }
+    if (__any_sync(kFull, esc != 0)) {
+      // an escape in this chunk: reload its row indexes and decode it again
+      // from its saved state on the lane-serial path
+      __syncwarp();
+      const uint32_t bar = h ? bar1 : bar0;
+      tma::fence_proxy_async();
+      tma::arrive_expect_if(l0, bar, cbytes);
+      tma::load_3d_if(l0, ring + (uint32_t)h * kTileRingHalf, imap, x0, sd.y, sd.z, bar);
+      pending |= 1u << h;
+      if (!wait_half(h)) return false;
+      st = st0;
+#pragma unroll 1
+      for (int j = 0; j < GC; ++j) {
+        const RowMeta mj = meta_of((uint32_t)rh[j * 32 + lane]);
+        rh[j * 32 + lane] = dec_group_val<F, false>(st, mj, starts, slots, words, nw, sh);
+      }
+    }
+    // chunk k's decoded values go out
+    tma::fence_proxy_async();
+    __syncwarp();
+    tma::store_3d_commit_if(l0, omap, x0, sd.y, sd.z, ring + (uint32_t)h * kTileRingHalf);
+    sd.next();
+  }
+  if (__any_sync(kFull, st.rmax > kmax)) {
+    if (lane == 0) report(c.status, RANS_ERR_INDEX, s);
+    return true;
+  }
+  const bool ok = !st.bad && st.x == F::kLow && st.cur + st.off == nw;
+  if (!__all_sync(kFull, ok) && lane == 0) report(c.status, RANS_ERR_CORRUPT, s);
+  return true;
+}
+
+template <class F>
+__global__ void __launch_bounds__(kDecMaxThreads32)
+    decode_tile_kernel(DecCtx c, const __grid_constant__ TileMaps maps) {
+  extern __shared__ __align__(16) unsigned char smem[];
+  __shared__ uint64_t bar;
+  __shared__ uint64_t ring_bar[kDecMaxWarps][2];
+  const char *gb = c.blob + kHeaderBytes;
+  if (!stage_to_smem(smem, gb, c.meta_bytes, &bar, c.status, smem + c.meta_bytes,
+                     gb + c.meta_bytes + c.bucket_bytes, c.start_bytes + c.slot_bytes))
+    return;
+  const RowMeta *meta = reinterpret_cast<const RowMeta *>(smem);
+  const uint16_t *starts = reinterpret_cast<const uint16_t *>(smem + c.meta_bytes);
+  const uint32_t *slots = reinterpret_cast<const uint32_t *>(smem + c.meta_bytes + c.start_bytes);
+  const uint32_t tab = c.meta_bytes + c.start_bytes + c.slot_bytes;
+  const int warp = threadIdx.x >> 5, nwarp = blockDim.x >> 5, lane = threadIdx.x & 31;
+  // each warp's ring: 128-byte aligned (tensor-tile copies)
+  const uint32_t sbase = smem_addr(smem);
+  const uint32_t ring = ((sbase + tab + 127u) & ~127u) + (uint32_t)warp * kTileRingBytes;
+  int32_t *ring_p = reinterpret_cast<int32_t *>(smem + (ring - sbase));
+  const uint32_t bar0 = smem_addr(&ring_bar[warp][0]);
+  if (lane == 0) {
+    tma::mbar_init(bar0, 1);
+    tma::mbar_init(bar0 + 8, 1);
+    tma::fence_mbar_init();
+  }
+  __syncwarp();
+  uint32_t par = 0;
+  // slots that ran out of bitmap room (flagged in the blob header) search
+  const bool search = reinterpret_cast<const uint32_t *>(c.blob)[kSearchFlagWord] != 0;
+  for (int64_t k = blockIdx.x + (int64_t)gridDim.x * warp; k < c.g.S;
+       k += (int64_t)gridDim.x * nwarp) {
+    const int64_t s = stream_of(c.g, k);
+    bool ok;
+    if (search) {
+      ok = decode_tile_stream<F, true>(c, maps, meta, starts, slots, ring, ring_p, bar0, par, s);
+    } else {
+      // unrolled chunks for tile widths 64 and 56 (8 and 7 groups), the general
+      // loop otherwise (fewer unrolled variants keep the hot code in the
+      // instruction cache)
+      const int64_t ww = c.g.tw * ((s % c.g.ntx) + 1) <= c.g.Wd ? c.g.tw
+                                                                   : c.g.Wd % c.g.tw;
+      switch (ww) {
+        case 64: ok = decode_tile_stream_fast<F, 8>(c, maps, meta, starts, slots, ring, ring_p, bar0, par, s); break;
+        case 56: ok = decode_tile_stream_fast<F, 7>(c, maps, meta, starts, slots, ring, ring_p, bar0, par, s); break;
+        default: ok = decode_tile_stream<F, false>(c, maps, meta, starts, slots, ring, ring_p, bar0, par, s);
+      }
+    }
+    if (!ok) break;
+  }
+  if (lane == 0) tma::bulk_wait_all();
+}
+
+// Whether a tiled W = 32 decode can take the tile-staged kernel: int32 rows
+// and symbols in 16-byte aligned tensors, one index per element, every tile
+// row a whole number of 16-byte units and of 8-symbol steps (so a chunk of 4
+// rows is a whole number of groups, at least 2), tile heights multiples of 4,
+// and the row metadata, starts, slots and rings in shared memory.
+bool tile_path_ok(const DecCtx &c, int mode, int sym_dtype, const void *indexes,
+                  const void *symbols) {
+  const Geom &g = c.g;
+  if (g.kind != RANS_CHUNK_TILED || g.W != 32 || g.alias || mode != 1 || g.ib_shift != 0 ||
+      sym_dtype != RANS_SYM_INT32)
+    return false;
+  if ((reinterpret_cast<uintptr_t>(indexes) & 15) || (reinterpret_cast<uintptr_t>(symbols) & 15))
+    return false;
+  const int64_t ww1 = g.Wd % g.tw, hh1 = g.H % g.th;
+  auto width_ok = [](int64_t w) { return w % 8 == 0 && w >= 16 && w <= 64; };
+  if (!width_ok(g.tw > g.Wd ? g.Wd : g.tw) || (ww1 != 0 && !width_ok(ww1))) return false;
+  if (g.th % 4 != 0 || hh1 % 4 != 0 || g.Wd % 4 != 0) return false;
+  return true;
+}
+
+// Launches the tile-staged decoder; kNotTaken when the tables and rings do
+// not fit in shared memory (the caller then takes the general kernel).
+constexpr int kNotTaken = 1;
+
+template <class F>
+int launch_decode_tile(const DecCtx &c, const int32_t *indexes, void *symbols, cudaStream_t st) {
+  const Geom &g = c.g;
+  int dev = 0;
+  cudaGetDevice(&dev);
+  const uint32_t tab = dec_table_bytes(1, c);
+  const int optin = smem_optin(dev);
+  const uint32_t lim = (uint32_t)optin - 64u - 2u * 8u * kDecMaxWarps;
+  if (tab + 128u + kTileRingBytes > lim) return kNotTaken;
+  TileMaps maps;
+  const int64_t per_img = g.ng * g.nty * g.ntx;
+  const int64_t depth = (g.S / per_img) * g.C;
+  const uint32_t w0 = (uint32_t)(g.tw > g.Wd ? g.Wd : g.tw);
+  const uint32_t w1 = g.Wd % g.tw ? (uint32_t)(g.Wd % g.tw) : w0;
+  for (int k = 0; k < 2; ++k) {
+    const uint32_t bw = k ? w1 : w0;
+    if (encode_tile_map(&maps.idx[k], indexes, g.Wd, g.H, depth, bw, 4) ||
+        encode_tile_map(&maps.out[k], symbols, g.Wd, g.H, depth, bw, 4))
+      return RANS_ERR_CUDA;
+  }
+  const int sms = num_sms(dev);
+  int64_t warps = (g.S + sms - 1) / sms;
+  if (warps > kDecMaxWarps) warps = kDecMaxWarps;
+  const int64_t room = ((int64_t)lim - tab - 128) / kTileRingBytes;
+  if (warps > room) warps = room;
+  if (warps < 1) warps = 1;
+  const uint32_t smem = tab + 128u + (uint32_t)warps * kTileRingBytes;
+  auto kern = decode_tile_kernel<F>;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
+      cudaSuccess)
+    return RANS_ERR_CUDA;
+  int fit = 0;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&fit, kern, (int)warps * 32, smem) !=
+          cudaSuccess ||
+      fit < 1)
+    return RANS_ERR_CUDA;
+  const int64_t need = (g.S + warps - 1) / warps;
+  const int64_t cap = (int64_t)fit * sms;
+  const int64_t blocks = need < cap ? need : cap;
+  kern<<<(unsigned)blocks, (unsigned)warps * 32, smem, st>>>(c, maps);
+  return cudaGetLastError() == cudaSuccess ? RANS_OK : RANS_ERR_CUDA;
+}
+
 template <class F, int W, typename SymT, int MODE, bool IB0>
 __global__ void __launch_bounds__(W == 32 ? kDecMaxThreads32 : kDecThreads1)
     decode_kernel(DecCtx c) {
@@ -984,6 +1546,11 @@ int launch_decode(const uint8_t *in, uint64_t in_bytes, const uint64_t *offsets,
   c.bound = 0.0f;
   c.stab_smem = 0;
   const int mode = t.dec_in_smem;
+  if (tile_path_ok(c, mode, sym_dtype, indexes, symbols)) {
+    const int r = g.fmt == RANS_FMT_RANS32_16 ? launch_decode_tile<Rans32>(c, indexes, symbols, st)
+                                              : launch_decode_tile<Rans64>(c, indexes, symbols, st);
+    if (r != kNotTaken) return r;
+  }
   switch (sym_dtype) {
     case RANS_SYM_INT32: return launch_decode_s<int32_t>(c, mode, st);
     case RANS_SYM_UINT8: return launch_decode_s<uint8_t>(c, mode, st);

@@ -23,6 +23,8 @@
 //    lanes places them, and the lane writes them.
 #include <type_traits>
 
+#include <cuda.h>  // CUtensorMap
+
 #include "rans_common.cuh"
 #include "rans_internal.h"
 
@@ -652,6 +654,312 @@ __host__ __device__ inline uint32_t enc_table_bytes(int mode, const EncCtx &c) {
                    : (mode == 2 ? c.meta_bytes + c.start_bytes : 0u);
 }
 
+// ---------------------------------------------- W = 32, tile-staged input --
+// Tiled streams whose tile rows are whole 16-byte units go through a leaner
+// warp encoder: the row indexes and symbols of 4 tile rows of one channel (a
+// chunk of ww / 8 groups) arrive in a per-warp shared-memory ring with two
+// tensor-tile copies on one mbarrier, the stream's chunks taken last to
+// first (the coder runs backwards).  Stream group g sits in ring slot
+// g mod 2 Gc; chunk c fills slots [(c mod 2) Gc, (c mod 2) Gc + Gc).  While
+// one chunk codes, the chunk before it lands in the other half, and the one
+// two before that is prefetched into L2.  As in the general coder, a group's
+// row index is read three groups ahead, its symbol and row metadata two
+// ahead and its bucket word and reciprocal one ahead of its state update.
+constexpr uint32_t kEncTileRingBytes = 4096;  // 16 groups of indexes + 16 of symbols
+constexpr uint32_t kEncTileWaitTries = 1u << 22;
+
+struct EncTileMaps {
+  CUtensorMap idx[2];  // row indexes: box (tile width, 4, 1); [1]: last tile column
+  CUtensorMap sym[2];  // int32 symbols, same boxes
+};
+
+template <class F, bool ST>
+__device__ __forceinline__ bool encode_tile_stream(const EncCtx &c, const EncTileMaps &maps,
+                                                   const RowMeta *meta, const uint32_t *buckets,
+                                                   uint32_t ring, const uint32_t *ring_p,
+                                                   uint32_t bar0, uint32_t &par, int64_t s) {
+  using Word = typename F::Word;
+  const int lane = threadIdx.x & 31;
+  const Geom &g = c.g;
+  const StreamDesc d = stream_desc(g, s);
+  if (!d.ok) {
+    if (lane == 0) report(c.status, RANS_ERR_ARG, s);
+    return true;
+  }
+  Word *end = reinterpret_cast<Word *>(c.scratch + slot_end(g, d, s));
+  const uint32_t sh = F::shift(c.sh);
+  const uint32_t kmax = (uint32_t)c.K - 1u;
+  const uint32_t above = 0xfffffffeu << lane;  // lanes > this lane
+  // the tile: image b, channel group gi, tile row ty, tile column tx
+  const int64_t per_img = g.ng * g.nty * g.ntx;
+  const int64_t b = s / per_img, t0 = s - b * per_img;
+  const int64_t gi = t0 / (g.nty * g.ntx), t1 = t0 - gi * (g.nty * g.ntx);
+  const int64_t ty = t1 / g.ntx, tx = t1 - ty * g.ntx;
+  const int32_t x0 = (int32_t)(tx * g.tw);
+  const int32_t ww = d.t.ww, hh = d.t.hh;
+  const int cls = ww == (int32_t)g.tw ? 0 : 1;
+  const void *imap = &maps.idx[cls];
+  const void *smap = &maps.sym[cls];
+  const int32_t Gc = ww >> 3;                    // groups per chunk (>= 4)
+  const int32_t M = (int32_t)(d.n / (4 * ww));   // chunks
+  const int32_t G = M * Gc;
+  const uint32_t cbytes = 16u * (uint32_t)ww;
+  const uint32_t half = (uint32_t)Gc * 128u;     // bytes of one half of either ring
+  const uint32_t sym_w = kEncTileRingBytes / 8;  // word offset of the symbol ring
+  // tensor-tile coordinates of chunks, stepped back 4 rows at a time from the
+  // last chunk: ld for the loads into shared memory, pf for the L2 prefetches
+  struct Back {
+    int32_t y, z, y0, ylast;
+    __device__ __forceinline__ void prev() {
+      y -= 4;
+      if (y < y0) {
+        y = ylast;
+        --z;
+      }
+    }
+  };
+  Back ld;
+  ld.y0 = (int32_t)(ty * g.th);
+  ld.ylast = ld.y = ld.y0 + hh - 4;
+  ld.z = (int32_t)(b * g.C + gi * g.cg) + (int32_t)(d.n / ((int64_t)hh * ww)) - 1;
+  Back pf = ld;
+  const uint32_t bar1 = bar0 + 8;
+  uint32_t pending = 0;  // loads in flight, by half
+  // the load of stream chunk ch (into half ch & 1); chunks are loaded in
+  // descending order
+  auto issue = [&](int32_t ch) {
+    const int h = ch & 1;
+    if (lane == 0) {
+      const uint32_t bar = h ? bar1 : bar0;
+      tma::fence_proxy_async();
+      tma::arrive_expect(bar, 2u * cbytes);
+      tma::load_3d(ring + (uint32_t)h * half, imap, x0, ld.y, ld.z, bar);
+      tma::load_3d(ring + 4u * sym_w + (uint32_t)h * half, smap, x0, ld.y, ld.z, bar);
+    }
+    pending |= 1u << h;
+    ld.prev();
+  };
+  auto prefetch = [&]() {
+    if (lane == 0) {
+      tma::prefetch_l2_3d(imap, x0, pf.y, pf.z);
+      tma::prefetch_l2_3d(smap, x0, pf.y, pf.z);
+    }
+    pf.prev();
+  };
+  auto wait_chunk = [&](int32_t ch) -> bool {
+    const int h = ch & 1;
+    const uint32_t bar = h ? bar1 : bar0;
+    const bool ok = tma::wait_bounded(bar, (par >> h) & 1u, kEncTileWaitTries);
+    if (__all_sync(kFull, ok)) {
+      par ^= 1u << h;
+      pending &= ~(1u << h);
+      return true;
+    }
+    if (lane == 0) report(c.status, RANS_ERR_TIMEOUT, s);
+    for (int q = 0; q < 2; ++q)
+      if (pending >> q & 1u) tma::wait_bounded(q ? bar1 : bar0, (par >> q) & 1u, kEncTileWaitTries);
+    return false;
+  };
+  __syncwarp();
+  issue(M - 1);
+  if (M > 1) issue(M - 2);
+  pf.prev();
+  if (M > 1) pf.prev();
+  for (int32_t q = 2; q < 4 && q < M; ++q) prefetch();
+
+  WarpEnc<F> st;
+  st.x = F::kLow;
+  st.cursor = 0;
+  st.rmax = 0;
+  st.range_err = false;
+  auto meta_of = [&](uint32_t r) -> RowMeta {
+    st.rmax = max(st.rmax, r);
+    return row_meta(meta, min(r, kmax));
+  };
+  // stream group gg sits in ring slot gg mod 2 Gc
+  const int32_t nslot = 2 * Gc;
+  auto dn = [&](int32_t sl) { return sl == 0 ? nslot - 1 : sl - 1; };
+  if (!wait_chunk(M - 1)) return false;
+  // groups G - 1 .. G - 3 are in the last chunk (Gc >= 4)
+  const int32_t sl_a = (G - 1) % nslot;
+  const int32_t sl_b = dn(sl_a), sl_c = dn(sl_b);
+  EncLook L = enc_look<F>(
+      enc_bucket<ST>((int32_t)ring_p[sym_w + sl_a * 32 + lane], meta_of(ring_p[sl_a * 32 + lane]),
+                     buckets),
+      true, sh);
+  int32_t s1 = (int32_t)ring_p[sym_w + sl_b * 32 + lane];
+  RowMeta m1 = meta_of(ring_p[sl_b * 32 + lane]);
+  uint32_t r2 = ring_p[sl_c * 32 + lane];
+  // reads ahead: the row index of group g3 = G - 4 - k and the symbol of
+  // g2 = G - 3 - k, each with its chunk and place in the chunk and ring slot
+  int32_t g3 = G - 4, c3 = g3 >= 0 ? g3 / Gc : -1, j3 = g3 >= 0 ? g3 - c3 * Gc : 0;
+  int32_t g2 = G - 3, c2 = g2 / Gc, j2 = g2 - c2 * Gc;
+  int32_t sl3 = dn(sl_c), sl2 = sl_c;
+#pragma unroll 1
+  for (int32_t k = 0; k < G; ++k) {
+    // group G - 1 - k codes, G - 2 - k is looked up
+    const EncBucket b1 = enc_bucket<ST>(s1, m1, buckets);
+    const typename F::State x0 = st.x;
+    const uint32_t c0 = st.cursor;
+    enc_group_fast<F, true>(st, L, true, above, end, sh);
+    const EncLook L1 = enc_look<F>(b1, true, sh);
+    uint32_t r3 = 0;
+    if (g3 >= 0) {
+      if (j3 == Gc - 1 && c3 < M - 1) {  // the first read of chunk c3
+        if (!wait_chunk(c3)) return false;
+      }
+      r3 = ring_p[sl3 * 32 + lane];
+    }
+    int32_t s2 = 0;
+    RowMeta m2 = m1;
+    if (g2 >= 0) {
+      s2 = (int32_t)ring_p[sym_w + sl2 * 32 + lane];
+      m2 = meta_of(r2);
+      // the last read of chunk c2: the chunk two before it may land in its
+      // half, and one four before it go to L2
+      if (j2 == 0 && c2 >= 2) {
+        __syncwarp();
+        issue(c2 - 2);
+        if (c2 >= 4) prefetch();
+      }
+    }
+    if (L.any_esc) enc_group_escape<F>(st, x0, c0, L, true, end, sh);
+    L = L1;
+    s1 = s2;
+    m1 = m2;
+    r2 = r3;
+    sl3 = dn(sl3);
+    sl2 = dn(sl2);
+    --g3;
+    if (--j3 < 0) {
+      j3 = Gc - 1;
+      --c3;
+    }
+    --g2;
+    if (--j2 < 0) {
+      j2 = Gc - 1;
+      --c2;
+    }
+  }
+  if (__any_sync(kFull, st.rmax > kmax)) {
+    if (lane == 0) report(c.status, RANS_ERR_INDEX, s);
+    return true;
+  }
+  if (__any_sync(kFull, st.range_err)) {
+    if (lane == 0) report(c.status, RANS_ERR_RANGE, s);
+    return true;
+  }
+  // flush: lanes 31..0 push high then low, so lane 0's low word comes first
+  const uint32_t kk = st.cursor + 2u * (31u - (uint32_t)lane);
+  st_global(end - 1 - kk, (Word)(st.x >> F::kWordBits));
+  st_global(end - 2 - kk, (Word)st.x);
+  if (lane == 0) c.lens[s] = sizeof(Word) * (uint64_t)(st.cursor + 64);
+  return true;
+}
+
+template <class F, bool ST>
+__global__ void __launch_bounds__(kEncThreads32)
+    encode_tile_kernel(EncCtx c, const __grid_constant__ EncTileMaps maps) {
+  extern __shared__ __align__(16) unsigned char smem[];
+  __shared__ uint64_t bar;
+  __shared__ uint64_t ring_bar[kEncMaxWarps][2];
+  const char *gb = c.blob + kHeaderBytes;
+  if (ST) {
+    if (!stage_to_smem(smem, gb, c.meta_bytes, &bar, c.status, smem + c.meta_bytes,
+                       gb + c.meta_bytes + c.bucket_bytes, c.start_bytes))
+      return;
+  } else {
+    if (!stage_to_smem(smem, gb, c.meta_bytes + c.bucket_bytes, &bar, c.status)) return;
+  }
+  const RowMeta *meta = reinterpret_cast<const RowMeta *>(smem);
+  const uint32_t *buckets = reinterpret_cast<const uint32_t *>(smem + c.meta_bytes);
+  const uint32_t tab = enc_table_bytes(ST ? 2 : 1, c);
+  const int warp = threadIdx.x >> 5, nwarp = blockDim.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t sbase = smem_addr(smem);
+  const uint32_t ring = ((sbase + tab + 127u) & ~127u) + (uint32_t)warp * kEncTileRingBytes;
+  const uint32_t *ring_p = reinterpret_cast<const uint32_t *>(smem + (ring - sbase));
+  const uint32_t bar0 = smem_addr(&ring_bar[warp][0]);
+  if (lane == 0) {
+    tma::mbar_init(bar0, 1);
+    tma::mbar_init(bar0 + 8, 1);
+    tma::fence_mbar_init();
+  }
+  __syncwarp();
+  uint32_t par = 0;
+  for (int64_t k = blockIdx.x + (int64_t)gridDim.x * warp; k < c.g.S;
+       k += (int64_t)gridDim.x * nwarp)
+    if (!encode_tile_stream<F, ST>(c, maps, meta, buckets, ring, ring_p, bar0, par,
+                                   stream_of(c.g, k)))
+      break;
+}
+
+// Whether a tiled W = 32 encode can take the tile-staged kernel (the
+// conditions of the decoder's tile path -- int32 rows and symbols in 16-byte
+// aligned tensors, one index per element, tile rows of whole 16-byte units
+// and 8-symbol steps, tile heights multiples of 4 -- with tile widths of at
+// least 32, so that a chunk holds the 4 groups the coder reads ahead) with
+// its tables in shared memory.
+bool enc_tile_path_ok(const EncCtx &c, int mode, int sym_dtype, const void *indexes,
+                      const void *symbols) {
+  const Geom &g = c.g;
+  if (g.kind != RANS_CHUNK_TILED || g.W != 32 || g.alias || (mode != 1 && mode != 2) ||
+      g.ib_shift != 0 || sym_dtype != RANS_SYM_INT32)
+    return false;
+  if ((reinterpret_cast<uintptr_t>(indexes) & 15) || (reinterpret_cast<uintptr_t>(symbols) & 15))
+    return false;
+  const int64_t ww1 = g.Wd % g.tw, hh1 = g.H % g.th;
+  auto width_ok = [](int64_t w) { return w % 8 == 0 && w >= 32 && w <= 64; };
+  if (!width_ok(g.tw > g.Wd ? g.Wd : g.tw) || (ww1 != 0 && !width_ok(ww1))) return false;
+  if (g.th % 4 != 0 || hh1 % 4 != 0 || g.Wd % 4 != 0) return false;
+  return true;
+}
+
+constexpr int kNotTaken = 1;
+
+template <class F>
+int launch_encode_tile(const EncCtx &c, int mode, const int32_t *indexes, const void *symbols,
+                       cudaStream_t st) {
+  const Geom &g = c.g;
+  int dev = 0;
+  cudaGetDevice(&dev);
+  const uint32_t tab = enc_table_bytes(mode, c);
+  const int optin = smem_optin(dev);
+  const uint32_t lim = (uint32_t)optin - 64u - 2u * 8u * kEncMaxWarps;
+  if (tab + 128u + kEncTileRingBytes > lim) return kNotTaken;
+  EncTileMaps maps;
+  const int64_t per_img = g.ng * g.nty * g.ntx;
+  const int64_t depth = (g.S / per_img) * g.C;
+  const uint32_t w0 = (uint32_t)(g.tw > g.Wd ? g.Wd : g.tw);
+  const uint32_t w1 = g.Wd % g.tw ? (uint32_t)(g.Wd % g.tw) : w0;
+  for (int k = 0; k < 2; ++k) {
+    const uint32_t bw = k ? w1 : w0;
+    if (encode_tile_map(&maps.idx[k], indexes, g.Wd, g.H, depth, bw, 4) ||
+        encode_tile_map(&maps.sym[k], symbols, g.Wd, g.H, depth, bw, 4))
+      return RANS_ERR_CUDA;
+  }
+  const int sms = num_sms(dev);
+  int64_t warps = (g.S + sms - 1) / sms;
+  if (warps > kEncMaxWarps) warps = kEncMaxWarps;
+  const int64_t room = ((int64_t)lim - tab - 128) / kEncTileRingBytes;
+  if (warps > room) warps = room;
+  if (warps < 1) warps = 1;
+  const uint32_t smem = tab + 128u + (uint32_t)warps * kEncTileRingBytes;
+  auto kern = mode == 2 ? encode_tile_kernel<F, true> : encode_tile_kernel<F, false>;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
+      cudaSuccess)
+    return RANS_ERR_CUDA;
+  int fit = 0;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&fit, kern, (int)warps * 32, smem) !=
+          cudaSuccess ||
+      fit < 1)
+    return RANS_ERR_CUDA;
+  const int64_t need = (g.S + warps - 1) / warps;
+  const int64_t cap = (int64_t)fit * sms;
+  const int64_t blocks = need < cap ? need : cap;
+  kern<<<(unsigned)blocks, (unsigned)warps * 32, smem, st>>>(c, maps);
+  return cudaGetLastError() == cudaSuccess ? RANS_OK : RANS_ERR_CUDA;
+}
+
 template <class F, int W, typename SymT, int MODE, bool IB0, bool FLT>
 __global__ void __launch_bounds__(W == 32 ? kEncThreads32 : kEncThreads1)
     encode_kernel(EncCtx c) {
@@ -954,6 +1262,12 @@ int launch_encode(const void *symbols, int sym_dtype, const int32_t *indexes,
   c.bound = 0.0f;
   c.stab_smem = 0;
   const int mode = t.enc_in_smem;
+  if (enc_tile_path_ok(c, mode, sym_dtype, indexes, symbols)) {
+    const int r = g.fmt == RANS_FMT_RANS32_16
+                      ? launch_encode_tile<Rans32>(c, mode, indexes, symbols, st)
+                      : launch_encode_tile<Rans64>(c, mode, indexes, symbols, st);
+    if (r != kNotTaken) return r;
+  }
   switch (sym_dtype) {
     case RANS_SYM_INT32: return launch_encode_s<int32_t>(c, mode, st);
     case RANS_SYM_UINT8: return launch_encode_s<uint8_t>(c, mode, st);

@@ -76,6 +76,13 @@ constexpr int kEncStage = 16;      // encoder ring: 16 groups of indexes + symbo
 constexpr int kDecMaxWarps = 24;   // decoder CTA: up to 768 threads
 constexpr int kEncMaxWarps = 24;   // encoder CTA: up to 768 threads
 constexpr uint32_t kDecStageBytes = kDecMaxWarps * kDecStage * 32 * 4;
+// Tile-staged warp decoder: per warp a ring of two halves of 4 tile rows of
+// up to 64 int32 each, 128-byte aligned.
+constexpr uint32_t kTileRingHalf = 1024;
+constexpr uint32_t kTileRingBytes = 2 * kTileRingHalf;
+// Shared memory the decoder's tables leave for its rings.
+constexpr uint32_t kDecRingRoom = kDecMaxWarps * kTileRingBytes + 128;
+static_assert(kDecRingRoom >= kDecStageBytes, "room for either decoder's rings");
 constexpr uint32_t kEncStageBytes = kEncMaxWarps * kEncStage * 32 * 4 * 2;
 
 __host__ __device__ inline uint64_t pad16(uint64_t b) { return (b + 15) & ~uint64_t(15); }
@@ -685,4 +692,115 @@ __device__ inline bool stage_to_smem(void *dst, const void *src, uint32_t bytes,
   return __syncthreads_and(done ? 1 : 0) != 0;
 }
 
+}  // namespace rb
+
+// ------------------------------------------- tensor-tile staging (TMA) ----
+// Tiles of an int32 tensor move between global and shared memory with
+// cp.async.bulk.tensor (no multicast): a load completes on an mbarrier with a
+// byte count, a store is tracked by the issuing thread's bulk groups.  The
+// tensor maps (CUtensorMap, built on the host) describe a 3-D int32 tensor
+// (x = width, y = height, z = image * channel) and a box of w x 4 rows x 1.
+namespace rb {
+namespace tma {
+
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
+}
+__device__ __forceinline__ void fence_mbar_init() {
+  asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+__device__ __forceinline__ void arrive_expect(uint32_t bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes)
+               : "memory");
+}
+// Orders this thread's generic-proxy shared-memory accesses before later
+// async-proxy (bulk copy) accesses of the same memory.
+__device__ __forceinline__ void fence_proxy_async() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+__device__ __forceinline__ void load_3d(uint32_t dst, const void *map, int32_t x, int32_t y,
+                                        int32_t z, uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3, %4}], [%5];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(z), "r"(bar)
+      : "memory");
+}
+__device__ __forceinline__ void store_3d(const void *map, int32_t x, int32_t y, int32_t z,
+                                         uint32_t src) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.global.shared::cta.tile.bulk_group [%0, {%1, %2, %3}], [%4];" ::
+          "l"(reinterpret_cast<uint64_t>(map)),
+      "r"(x), "r"(y), "r"(z), "r"(src)
+      : "memory");
+}
+// Brings a tensor tile into L2 ahead of its load (no completion to wait for).
+__device__ __forceinline__ void prefetch_l2_3d(const void *map, int32_t x, int32_t y, int32_t z) {
+  asm volatile("cp.async.bulk.prefetch.tensor.3d.L2.global.tile [%0, {%1, %2, %3}];" ::"l"(
+                   reinterpret_cast<uint64_t>(map)),
+               "r"(x), "r"(y), "r"(z)
+               : "memory");
+}
+__device__ __forceinline__ void bulk_commit() {
+  asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+}
+// Waits until this thread's committed bulk stores have read their source.
+__device__ __forceinline__ void bulk_wait_read() {
+  asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+}
+// Waits until this thread's committed bulk stores have completed.
+__device__ __forceinline__ void bulk_wait_all() {
+  asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
+}
+// Predicated forms (no branch around them): the operation runs only where p
+// is nonzero, so a warp-wide code block can issue it from one lane.
+__device__ __forceinline__ void arrive_expect_if(uint32_t p, uint32_t bar, uint32_t bytes) {
+  asm volatile(
+      "{\n\t.reg .pred q;\n\tsetp.ne.u32 q, %0, 0;\n\t"
+      "@q mbarrier.arrive.expect_tx.shared::cta.b64 _, [%1], %2;\n\t}" ::"r"(p),
+      "r"(bar), "r"(bytes)
+      : "memory");
+}
+__device__ __forceinline__ void load_3d_if(uint32_t p, uint32_t dst, const void *map, int32_t x,
+                                           int32_t y, int32_t z, uint32_t bar) {
+  asm volatile(
+      "{\n\t.reg .pred q;\n\tsetp.ne.u32 q, %0, 0;\n\t"
+      "@q cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      " [%1], [%2, {%3, %4, %5}], [%6];\n\t}" ::"r"(p),
+      "r"(dst), "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(z), "r"(bar)
+      : "memory");
+}
+__device__ __forceinline__ void prefetch_l2_3d_if(uint32_t p, const void *map, int32_t x,
+                                                  int32_t y, int32_t z) {
+  asm volatile(
+      "{\n\t.reg .pred q;\n\tsetp.ne.u32 q, %0, 0;\n\t"
+      "@q cp.async.bulk.prefetch.tensor.3d.L2.global.tile [%1, {%2, %3, %4}];\n\t}" ::"r"(p),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(z)
+      : "memory");
+}
+__device__ __forceinline__ void store_3d_commit_if(uint32_t p, const void *map, int32_t x,
+                                                   int32_t y, int32_t z, uint32_t src) {
+  asm volatile(
+      "{\n\t.reg .pred q;\n\tsetp.ne.u32 q, %0, 0;\n\t"
+      "@q cp.async.bulk.tensor.3d.global.shared::cta.tile.bulk_group [%1, {%2, %3, %4}], [%5];"
+      "\n\t@q cp.async.bulk.commit_group;\n\t}" ::"r"(p),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(z), "r"(src)
+      : "memory");
+}
+__device__ __forceinline__ void bulk_wait_read_if(uint32_t p) {
+  asm volatile(
+      "{\n\t.reg .pred q;\n\tsetp.ne.u32 q, %0, 0;\n\t"
+      "@q cp.async.bulk.wait_group.read 0;\n\t}" ::"r"(p)
+      : "memory");
+}
+
+// A bounded wait for phase `parity` of an mbarrier: true once it completed,
+// false after `tries` attempts (each suspending for up to about 1 us).
+__device__ __forceinline__ bool wait_bounded(uint32_t bar, uint32_t parity, uint32_t tries) {
+  for (uint32_t it = 0; it < tries; ++it)
+    if (mbar_try_wait(bar, parity)) return true;
+  return false;
+}
+
+}  // namespace tma
 }  // namespace rb

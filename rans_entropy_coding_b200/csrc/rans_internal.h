@@ -59,6 +59,12 @@ int launch_decode(const uint8_t *in, uint64_t in_bytes, const uint64_t *offsets,
 int launch_debug_divide(const uint64_t *x, const uint32_t *f, int64_t n, uint64_t *q,
                         uint32_t *r, cudaStream_t st);
 
+// A tensor map (CUtensorMap, 128 bytes, 64-byte aligned) for a 3-D int32
+// tensor of width x height x depth elements (row-major, width fastest) and a
+// box of box_w x box_h x 1; base 16-byte aligned, width * 4 a multiple of 16.
+int encode_tile_map(void *map, const void *base, uint64_t width, uint64_t height,
+                    uint64_t depth, uint32_t box_w, uint32_t box_h);
+
 // Device properties cached per device.
 int num_sms(int device);
 int smem_optin(int device);

@@ -733,6 +733,28 @@ int refresh_tables(const int32_t *cdfs, int K, int Lmax, const int32_t *lengths,
 // again, and 256 KB (shared-memory tables plan up to
 // a quarter of their slot room as bitmap words; tables read from global
 // memory as many words as slots).
+// The bitmap words a row's slots need at 2^q slots: max(1, w / 16) for each
+// slot of width w = 2^(16-q) with three or more bucket boundaries strictly
+// inside it (the rule of fill_slot_block), counted on the host from the row
+// (entries scaled to 16 bits by << sh; entries out of range are skipped, the
+// device rejects such rows).
+uint64_t bitmap_words_needed(const int32_t *row, int nb, int q, uint32_t sh) {
+  const int w = 1 << (16 - q);
+  const uint64_t nch = w > 16 ? (uint64_t)(w >> 4) : 1ull;
+  const int nslots = 1 << q;
+  std::vector<uint8_t> inner(nslots, 0);
+  for (int j = 1; j < nb; ++j) {
+    const int64_t v = (int64_t)row[j] << sh;
+    if (v <= 0 || v >= (int64_t)kTotal || v % w == 0) continue;
+    uint8_t &c = inner[v / w];
+    if (c < 3) ++c;
+  }
+  uint64_t n = 0;
+  for (int t = 0; t < nslots; ++t)
+    if (inner[t] >= 3) n += nch;
+  return n;
+}
+
 uint64_t tables_bytes_bound(int K, int Lmax) {
   if (K <= 0 || Lmax < 2) return 0;
   const int64_t nb = (int64_t)Lmax - 1;
@@ -811,17 +833,32 @@ int prepare_tables(const int32_t *cdfs, int K, int Lmax, const int32_t *lengths,
                                                                                           : 0);
   bool dec_smem = false;
   uint64_t chunk_words = 0;
-  if ((int64_t)meta_bytes + start_bytes + kDecStageBytes <= budget) {
-    const int64_t room = budget - meta_bytes - start_bytes - kDecStageBytes;
-    // About one slot per bucket; halve the largest row's lookup until the
-    // slots take at most three quarters of the room, the rest going to
-    // bitmap words.
-    while ((int64_t)pad16(4ull * slot_total()) > room - room / 4) {
+  if ((int64_t)meta_bytes + start_bytes + kDecRingRoom <= budget) {
+    const int64_t room = budget - meta_bytes - start_bytes - kDecRingRoom;
+    // About one slot per bucket; halve the largest row's lookup until its
+    // slots and the bitmap words they need (counted from the rows) fit the
+    // room.  Bitmap words get all the room the slots leave.
+    std::vector<int32_t> rows((size_t)K * (size_t)Lmax);
+    if (cudaMemcpyAsync(rows.data(), cdfs, sizeof(int32_t) * rows.size(), cudaMemcpyDeviceToHost,
+                        st) != cudaSuccess ||
+        cudaStreamSynchronize(st) != cudaSuccess)
+      return RANS_ERR_CUDA;
+    std::vector<uint64_t> words(K);
+    for (int r = 0; r < K; ++r)
+      words[r] = (1ull << q[r]) + bitmap_words_needed(&rows[(size_t)r * Lmax], len[r] - 1, q[r], sh);
+    auto total = [&]() {
+      uint64_t t = 0;
+      for (int r = 0; r < K; ++r) t += words[r];
+      return t;
+    };
+    while ((int64_t)pad16(4ull * total()) > room) {
       int best = -1;
       for (int r = 0; r < K; ++r)
         if (q[r] > kMinQ && (best < 0 || q[r] >= q[best])) best = r;
       if (best < 0) break;
       --q[best];
+      words[best] = (1ull << q[best]) +
+                    bitmap_words_needed(&rows[(size_t)best * Lmax], len[best] - 1, q[best], sh);
     }
     const int64_t left = room - (int64_t)pad16(4ull * slot_total());
     dec_smem = left >= 0;

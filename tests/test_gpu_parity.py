@@ -11,7 +11,7 @@ import oracle as O
 import rans_entropy_coding_b200 as rb
 import workloads as WL
 from harness import (chunking_of, gpu_encode_decode, gpu_rows, oracle_encode, oracle_tables,
-                     tables_from_numpy)
+                     precision_of, tables_from_numpy)
 
 pytestmark = pytest.mark.gpu
 
@@ -48,7 +48,7 @@ def _edge_tiny(W=1, seed=0, dtype=np.int32):
 
 def _check_streams(w, exact_tables=True):
     c, l, o = oracle_tables(w)
-    tables = tables_from_numpy(c, l, o)
+    tables = tables_from_numpy(c, l, o, precision=precision_of(w))
     data, offs, dec, _, _ = gpu_encode_decode(w, tables)
     want, woffs = oracle_encode(w, c, l, o)
     assert offs.tolist() == woffs.tolist()
@@ -544,3 +544,27 @@ def test_bounded_wait_gives_up_and_the_context_stays_usable():
     assert time.time() - t < 30
     assert rb.rans_debug_wait_timeout(ws, 0) == rb.ERR_ARG
     _check_streams(_edge_tiny(32, seed=11))
+
+
+@pytest.mark.parametrize("shape,cg,th,tw,fmt", [
+    ((1, 192, 68, 120), 4, 64, 64, "rans32_16"),   # the batch tiles in the 16-bit word format
+    ((2, 10, 12, 48), 3, 8, 16, "rans64"),         # narrowest tiles, a partial channel group
+    ((1, 6, 20, 96), 2, 4, 40, "rans64"),          # last column 16 wide, 4-row tiles
+    ((1, 4, 64, 256), 4, 64, 64, "rans64"),        # every tile full
+])
+def test_tile_staged_decoder_shapes(shape, cg, th, tw, fmt):
+    """Tiled streams whose rows are whole 16-byte units (the decoder stages
+    them 4 rows at a time): several tile shapes, both coder formats, and the
+    tiny workload's far escapes spread over the tensor."""
+    n = int(np.prod(shape))
+    w = WL.y_batch(n_images=1, cg=cg, th=th, tw=tw)
+    rng = np.random.Generator(np.random.PCG64(41))
+    sym = np.asarray(w["symbols"]).reshape(-1)[:n].copy() if n <= np.asarray(
+        w["symbols"]).size else np.resize(np.asarray(w["symbols"]).reshape(-1), n)
+    idx = np.resize(np.asarray(w["indexes"]), n).astype(np.int32)
+    far = rng.random(n) < 0.002
+    sym = np.where(far, rng.integers(-2**31, 2**31 - 1, size=n, dtype=np.int64), sym)
+    w = dict(w, symbols=sym.astype(np.int32).reshape(shape), indexes=idx,
+             chunking=dict(kind="tiled", shape=shape, cg=cg, th=th, tw=tw), W=32, fmt=fmt,
+             precision=16 if fmt == "rans64" else 15)
+    _check_streams(w)
