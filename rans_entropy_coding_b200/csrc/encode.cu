@@ -857,6 +857,161 @@ __device__ __forceinline__ bool encode_tile_stream(const EncCtx &c, const EncTil
   return true;
 }
 
+// ------------------------------------------ unrolled chunks, no branches --
+// The coders' time per group follows their instruction count and the
+// branches that cut a group into small blocks.  For 56- and 64-wide tiles (7
+// and 8 groups per chunk) a chunk is coded as one unrolled block: the
+// compiler is free to run the later groups' lookups (row metadata, bucket
+// word, reciprocal) under the earlier groups' state updates, the copy-engine
+// work is predicated on lane 0, and escapes are only recorded.  A chunk in
+// which a lane met an escape is coded again from its saved state and cursor
+// with the escape path; the fast pass before it writes at most one word per
+// lane and group, inside the stream's worst-case scratch slot, and the redo
+// writes every word the stream keeps.
+template <class F, bool ST, int GC>
+__device__ __forceinline__ bool encode_tile_stream_fast(const EncCtx &c, const EncTileMaps &maps,
+                                                        const RowMeta *meta,
+                                                        const uint32_t *buckets, uint32_t ring,
+                                                        const uint32_t *ring_p, uint32_t bar0,
+                                                        uint32_t &par, int64_t s) {
+  using Word = typename F::Word;
+  const int lane = threadIdx.x & 31;
+  const Geom &g = c.g;
+  const StreamDesc d = stream_desc(g, s);
+  if (!d.ok) {
+    if (lane == 0) report(c.status, RANS_ERR_ARG, s);
+    return true;
+  }
+  Word *end = reinterpret_cast<Word *>(c.scratch + slot_end(g, d, s));
+  const uint32_t sh = F::shift(c.sh);
+  const uint32_t kmax = (uint32_t)c.K - 1u;
+  const uint32_t above = 0xfffffffeu << lane;  // lanes > this lane
+  const int64_t per_img = g.ng * g.nty * g.ntx;
+  const int64_t b = s / per_img, t0 = s - b * per_img;
+  const int64_t gi = t0 / (g.nty * g.ntx), t1 = t0 - gi * (g.nty * g.ntx);
+  const int64_t ty = t1 / g.ntx, tx = t1 - ty * g.ntx;
+  const int32_t x0 = (int32_t)(tx * g.tw);
+  const int32_t hh = d.t.hh;
+  const int cls = d.t.ww == (int32_t)g.tw ? 0 : 1;
+  const void *imap = &maps.idx[cls];
+  const void *smap = &maps.sym[cls];
+  const int32_t M = (int32_t)(d.n / (32 * GC));
+  const uint32_t cbytes = 128u * GC;
+  constexpr uint32_t kHalf = 128u * GC;
+  constexpr int kSymW = (int)(kEncTileRingBytes / 8);  // word offset of the symbol ring
+  // chunk coordinates stepped back 4 rows at a time from the last chunk: ld
+  // for the loads into shared memory, pf for the L2 prefetches
+  const int32_t y0 = (int32_t)(ty * g.th), ylast = y0 + hh - 4;
+  int32_t ly = ylast, lz = (int32_t)(b * g.C + gi * g.cg) + (int32_t)(d.n / ((int64_t)hh * d.t.ww)) - 1;
+  int32_t py = ly, pz = lz;
+  auto back_if = [&](int32_t &y, int32_t &z, bool on) {
+    const int32_t yy = y - 4;
+    const bool wrap = yy < y0;
+    y = on ? (wrap ? ylast : yy) : y;
+    z -= on && wrap ? 1 : 0;
+  };
+  const uint32_t bar1 = bar0 + 8;
+  const uint32_t l0 = lane == 0 ? 1u : 0u;
+  uint32_t pending = 0;
+  // the load of stream chunk ch into half ch & 1 (chunks load in descending order)
+  auto issue_if = [&](int32_t ch, uint32_t on) {
+    const int h = ch & 1;
+    const uint32_t bar = h ? bar1 : bar0;
+    tma::fence_proxy_async();
+    tma::arrive_expect_if(l0 & on, bar, 2u * cbytes);
+    tma::load_3d_if(l0 & on, ring + (uint32_t)h * kHalf, imap, x0, ly, lz, bar);
+    tma::load_3d_if(l0 & on, ring + 4u * kSymW + (uint32_t)h * kHalf, smap, x0, ly, lz, bar);
+    pending |= on << h;
+    back_if(ly, lz, on != 0);
+  };
+  auto prefetch_if = [&](uint32_t on) {
+    tma::prefetch_l2_3d_if(l0 & on, imap, x0, py, pz);
+    tma::prefetch_l2_3d_if(l0 & on, smap, x0, py, pz);
+    back_if(py, pz, on != 0);
+  };
+  auto wait_chunk = [&](int32_t ch) -> bool {
+    const int h = ch & 1;
+    const uint32_t bar = h ? bar1 : bar0;
+    const bool ok = tma::wait_bounded(bar, (par >> h) & 1u, kEncTileWaitTries);
+    if (__all_sync(kFull, ok)) {
+      par ^= 1u << h;
+      pending &= ~(1u << h);
+      return true;
+    }
+    if (lane == 0) report(c.status, RANS_ERR_TIMEOUT, s);
+    for (int q = 0; q < 2; ++q)
+      if (pending >> q & 1u) tma::wait_bounded(q ? bar1 : bar0, (par >> q) & 1u, kEncTileWaitTries);
+    return false;
+  };
+  __syncwarp();
+  issue_if(M - 1, 1u);
+  back_if(py, pz, true);
+  for (int32_t q = 1; q < 3; ++q) prefetch_if(M - 1 - q >= 0 ? 1u : 0u);
+
+  WarpEnc<F> st;
+  st.x = F::kLow;
+  st.cursor = 0;
+  st.rmax = 0;
+  st.range_err = false;
+  auto meta_of = [&](uint32_t r) -> RowMeta {
+    st.rmax = max(st.rmax, r);
+    return row_meta(meta, min(r, kmax));
+  };
+#pragma unroll 1
+  for (int32_t ch = M - 1; ch >= 0; --ch) {
+    if (!wait_chunk(ch)) return false;
+    // the chunk before this one into the other half (consumed by the chunk
+    // after this one), and the one three before it into L2
+    __syncwarp();
+    issue_if(ch - 1, ch >= 1 ? 1u : 0u);
+    prefetch_if(ch >= 3 ? 1u : 0u);
+    const uint32_t *ri = ring_p + (ch & 1) * (int)(kHalf / 4);
+    const uint32_t *rs = ri + kSymW;
+    const typename F::State xs = st.x;
+    const uint32_t cs = st.cursor;
+    uint32_t esc = 0;
+#pragma unroll
+    for (int j = GC - 1; j >= 0; --j) {
+      const EncBucket bk =
+          enc_bucket<ST>((int32_t)rs[j * 32 + lane], meta_of(ri[j * 32 + lane]), buckets);
+      esc |= bk.in_range ? 0u : 1u;
+      EncLook L;
+      L.start = bucket_start(bk.e);
+      L.freq = bucket_freq(bk.e);
+      L.rcp = F::rcp(L.freq, sh);
+      enc_group_fast<F, true>(st, L, true, above, end, sh);
+    }
+    if (__any_sync(kFull, esc != 0)) {
+      // an escape in this chunk: code it again from its saved state
+      st.x = xs;
+      st.cursor = cs;
+#pragma unroll 1
+      for (int j = GC - 1; j >= 0; --j) {
+        const EncBucket bk =
+            enc_bucket<ST>((int32_t)rs[j * 32 + lane], meta_of(ri[j * 32 + lane]), buckets);
+        const EncLook L = enc_look<F>(bk, true, sh);
+        const typename F::State xg = st.x;
+        const uint32_t cg = st.cursor;
+        enc_group_fast<F, true>(st, L, true, above, end, sh);
+        if (L.any_esc) enc_group_escape<F>(st, xg, cg, L, true, end, sh);
+      }
+    }
+  }
+  if (__any_sync(kFull, st.rmax > kmax)) {
+    if (lane == 0) report(c.status, RANS_ERR_INDEX, s);
+    return true;
+  }
+  if (__any_sync(kFull, st.range_err)) {
+    if (lane == 0) report(c.status, RANS_ERR_RANGE, s);
+    return true;
+  }
+  const uint32_t kk = st.cursor + 2u * (31u - (uint32_t)lane);
+  st_global(end - 1 - kk, (Word)(st.x >> F::kWordBits));
+  st_global(end - 2 - kk, (Word)st.x);
+  if (lane == 0) c.lens[s] = sizeof(Word) * (uint64_t)(st.cursor + 64);
+  return true;
+}
+
 template <class F, bool ST>
 __global__ void __launch_bounds__(kEncThreads32)
     encode_tile_kernel(EncCtx c, const __grid_constant__ EncTileMaps maps) {
@@ -887,10 +1042,19 @@ __global__ void __launch_bounds__(kEncThreads32)
   __syncwarp();
   uint32_t par = 0;
   for (int64_t k = blockIdx.x + (int64_t)gridDim.x * warp; k < c.g.S;
-       k += (int64_t)gridDim.x * nwarp)
-    if (!encode_tile_stream<F, ST>(c, maps, meta, buckets, ring, ring_p, bar0, par,
-                                   stream_of(c.g, k)))
-      break;
+       k += (int64_t)gridDim.x * nwarp) {
+    const int64_t s = stream_of(c.g, k);
+    // unrolled chunks for tile widths 64 and 56 (8 and 7 groups), the general
+    // loop otherwise
+    const int64_t ww = c.g.tw * ((s % c.g.ntx) + 1) <= c.g.Wd ? c.g.tw : c.g.Wd % c.g.tw;
+    bool ok;
+    switch (ww) {
+      case 64: ok = encode_tile_stream_fast<F, ST, 8>(c, maps, meta, buckets, ring, ring_p, bar0, par, s); break;
+      case 56: ok = encode_tile_stream_fast<F, ST, 7>(c, maps, meta, buckets, ring, ring_p, bar0, par, s); break;
+      default: ok = encode_tile_stream<F, ST>(c, maps, meta, buckets, ring, ring_p, bar0, par, s);
+    }
+    if (!ok) break;
+  }
 }
 
 // Whether a tiled W = 32 encode can take the tile-staged kernel (the
