@@ -173,7 +173,7 @@ typedef struct rans_tables {
                                global */
     int32_t device;         /* CUDA device the blob lives on */
     int32_t precision;      /* the rows sum to 2^precision */
-    int32_t reserved;
+    int32_t max_slot_log2;  /* log2 of the largest row's decode lookup slot count */
     void *alias;            /* alias tables (rans_alias_prepare), or NULL */
     uint64_t alias_bytes;
     uint64_t alias_remap_offset;  /* byte offset of the remap entries in `alias` */

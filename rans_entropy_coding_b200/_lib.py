@@ -57,7 +57,7 @@ class rans_tables(ctypes.Structure):
                 ("start_bytes", ctypes.c_uint32), ("slot_bytes", ctypes.c_uint32),
                 ("enc_in_smem", ctypes.c_int32),
                 ("dec_in_smem", ctypes.c_int32), ("device", ctypes.c_int32),
-                ("precision", ctypes.c_int32), ("reserved", ctypes.c_int32),
+                ("precision", ctypes.c_int32), ("max_slot_log2", ctypes.c_int32),
                 ("alias", ctypes.c_void_p), ("alias_bytes", ctypes.c_uint64),
                 ("alias_remap_offset", ctypes.c_uint64)]
 

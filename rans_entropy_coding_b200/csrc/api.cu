@@ -2,6 +2,8 @@
 // chunking geometry, workspace layout and launch order.  Every coding step
 // runs in the kernels of tables.cu, encode.cu and decode.cu.
 #include <cstring>
+#include <mutex>
+#include <vector>
 
 #include <nvtx3/nvToolsExt.h>
 
@@ -24,9 +26,66 @@ int num_sms(int device) {
 }
 
 int smem_optin(int device) {
-  int v = 0;
-  cudaDeviceGetAttribute(&v, cudaDevAttrMaxSharedMemoryPerBlockOptin, device);
-  return v;
+  static int cache[128] = {0};
+  if (device < 0 || device >= 128) return 0;
+  if (cache[device] == 0) {
+    int v = 0;
+    cudaDeviceGetAttribute(&v, cudaDevAttrMaxSharedMemoryPerBlockOptin, device);
+    cache[device] = v;
+  }
+  return cache[device];
+}
+
+// Launch set-up answers cached per (kernel, device): the dynamic shared
+// memory limit already set, and resident blocks per SM for a (threads,
+// shared memory) pair, so a coding call repeats no runtime query.
+namespace {
+struct SmemEntry {
+  const void *fn;
+  int dev;
+  uint32_t bytes;
+};
+struct OccEntry {
+  const void *fn;
+  int dev, threads;
+  uint32_t smem;
+  int blocks;
+};
+std::mutex g_launch_mutex;
+std::vector<SmemEntry> g_smem_set;
+std::vector<OccEntry> g_occ;
+}  // namespace
+
+cudaError_t ensure_dyn_smem(const void *fn, uint32_t bytes) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  std::lock_guard<std::mutex> lock(g_launch_mutex);
+  for (SmemEntry &x : g_smem_set)
+    if (x.fn == fn && x.dev == dev) {
+      if (x.bytes >= bytes) return cudaSuccess;
+      e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+      if (e == cudaSuccess) x.bytes = bytes;
+      return e;
+    }
+  e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+  if (e == cudaSuccess) g_smem_set.push_back({fn, dev, bytes});
+  return e;
+}
+
+cudaError_t blocks_per_sm(int *out, const void *fn, int threads, uint32_t smem) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  std::lock_guard<std::mutex> lock(g_launch_mutex);
+  for (const OccEntry &x : g_occ)
+    if (x.fn == fn && x.dev == dev && x.threads == threads && x.smem == smem) {
+      *out = x.blocks;
+      return cudaSuccess;
+    }
+  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(out, fn, threads, (size_t)smem);
+  if (e == cudaSuccess && g_occ.size() < 4096) g_occ.push_back({fn, dev, threads, smem, *out});
+  return e;
 }
 
 }  // namespace rb

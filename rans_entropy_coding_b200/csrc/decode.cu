@@ -1276,11 +1276,11 @@ int launch_decode_tile(const DecCtx &c, const int32_t *indexes, void *symbols, c
   if (warps < 1) warps = 1;
   const uint32_t smem = tab + 128u + (uint32_t)warps * kTileRingBytes;
   auto kern = decode_tile_kernel<F>;
-  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
+  if (ensure_dyn_smem((const void *)kern, (uint32_t)(smem)) !=
       cudaSuccess)
     return RANS_ERR_CUDA;
   int fit = 0;
-  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&fit, kern, (int)warps * 32, smem) !=
+  if (blocks_per_sm(&fit, (const void *)kern, (int)warps * 32, (uint32_t)(smem)) !=
           cudaSuccess ||
       fit < 1)
     return RANS_ERR_CUDA;
@@ -1390,11 +1390,11 @@ int launch_decode_wn(const DecCtx &c, int mode, cudaStream_t st) {
   const uint32_t tab = dec_table_bytes(mode, c);
   int dev = 0;
   cudaGetDevice(&dev);
-  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)tab) !=
+  if (ensure_dyn_smem((const void *)kern, (uint32_t)(tab)) !=
       cudaSuccess)
     return RANS_ERR_CUDA;
   int fit = 0;
-  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&fit, kern, kSegThreads, tab) !=
+  if (blocks_per_sm(&fit, (const void *)kern, kSegThreads, (uint32_t)(tab)) !=
           cudaSuccess ||
       fit < 1)
     return RANS_ERR_CUDA;
@@ -1419,7 +1419,7 @@ int launch_decode_t(const DecCtx &c, cudaStream_t st) {
   const int optin = smem_optin(dev);
   const uint32_t lim = (uint32_t)optin - 64u;  // room for the kernel's static shared memory
   const uint32_t max_dyn = tab + kDecStageBytes + tbl <= lim ? tab + kDecStageBytes + tbl : lim;
-  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)max_dyn) !=
+  if (ensure_dyn_smem((const void *)kern, (uint32_t)(max_dyn)) !=
       cudaSuccess)
     return RANS_ERR_CUDA;
   const int sms = num_sms(dev);
@@ -1429,7 +1429,7 @@ int launch_decode_t(const DecCtx &c, cudaStream_t st) {
     // One or a few CTAs per SM (bounded by the staged tables); enough warps
     // for one stream each when possible.
     int per_sm = 0;
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, 32, tab + per_warp) !=
+    if (blocks_per_sm(&per_sm, (const void *)kern, 32, (uint32_t)(tab + per_warp)) !=
             cudaSuccess ||
         per_sm < 1)
       return RANS_ERR_CUDA;
@@ -1441,7 +1441,7 @@ int launch_decode_t(const DecCtx &c, cudaStream_t st) {
     threads = (int)warps * 32;
     smem = tab + (uint32_t)warps * per_warp;
     int fit = 0;
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&fit, kern, threads, smem) != cudaSuccess ||
+    if (blocks_per_sm(&fit, (const void *)kern, threads, (uint32_t)(smem)) != cudaSuccess ||
         fit < 1)
       return RANS_ERR_CUDA;
     int64_t need = (c.g.S + warps - 1) / warps;
@@ -1450,7 +1450,7 @@ int launch_decode_t(const DecCtx &c, cudaStream_t st) {
   } else {
     threads = kDecThreads1;
     int fit = 0;
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&fit, kern, threads, smem) != cudaSuccess ||
+    if (blocks_per_sm(&fit, (const void *)kern, threads, (uint32_t)(smem)) != cudaSuccess ||
         fit < 1)
       return RANS_ERR_CUDA;
     int64_t need = (c.g.S + threads - 1) / threads;

@@ -1109,11 +1109,11 @@ int launch_encode_tile(const EncCtx &c, int mode, const int32_t *indexes, const 
   if (warps < 1) warps = 1;
   const uint32_t smem = tab + 128u + (uint32_t)warps * kEncTileRingBytes;
   auto kern = mode == 2 ? encode_tile_kernel<F, true> : encode_tile_kernel<F, false>;
-  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
+  if (ensure_dyn_smem((const void *)kern, (uint32_t)(smem)) !=
       cudaSuccess)
     return RANS_ERR_CUDA;
   int fit = 0;
-  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&fit, kern, (int)warps * 32, smem) !=
+  if (blocks_per_sm(&fit, (const void *)kern, (int)warps * 32, (uint32_t)(smem)) !=
           cudaSuccess ||
       fit < 1)
     return RANS_ERR_CUDA;
@@ -1277,6 +1277,54 @@ __global__ void copy_streams_kernel(Geom g, const char *scratch, const uint64_t 
   }
 }
 
+// Scan and copy in one launch, for up to kFusedMaxStreams streams: block b
+// owns streams [b * kCompactWarps, (b + 1) * kCompactWarps), one warp each.
+// Its first stream's offset is the sum of every earlier stream's length
+// (read by the whole block from L2: at most kFusedMaxStreams lengths), the
+// block's own offsets follow from a warp scan, and each warp copies its
+// stream.  The last block writes the total and checks the capacity.
+constexpr int kCompactWarps = 8;
+constexpr int64_t kFusedMaxStreams = 65536;
+
+template <typename Word>
+__global__ void __launch_bounds__(kCompactWarps * 32)
+    compact_streams_kernel(Geom g, const char *scratch, const uint64_t *lens, uint64_t *offsets,
+                           uint8_t *out, uint64_t capacity, int32_t *status) {
+  __shared__ unsigned long long part[kCompactWarps];
+  __shared__ unsigned long long own[kCompactWarps];
+  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+  const int64_t s0 = (int64_t)blockIdx.x * kCompactWarps;
+  // the lengths of streams [0, s0)
+  unsigned long long before = 0;
+  for (int64_t i = threadIdx.x; i < s0; i += blockDim.x) before += lens[i];
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) before += __shfl_xor_sync(kFull, before, o);
+  if (lane == 0) part[wid] = before;
+  // this block's streams: lane 0 of warp w holds stream s0 + w's length
+  const int64_t s = s0 + wid;
+  const unsigned long long len = s < g.S ? lens[s] : 0ull;
+  if (lane == 0) own[wid] = len;
+  __syncthreads();
+  unsigned long long base = 0, ex = 0, tot = 0;
+  for (int w = 0; w < kCompactWarps; ++w) {
+    base += part[w];
+    ex += w < wid ? own[w] : 0ull;
+    tot += own[w];
+  }
+  const uint64_t off = base + ex;
+  if (s < g.S && lane == 0) offsets[s + 1] = off + len;
+  if (blockIdx.x == 0 && threadIdx.x == 0) offsets[0] = 0;
+  if (blockIdx.x == gridDim.x - 1 && threadIdx.x == 0 && base + tot > capacity)
+    report(status, RANS_ERR_CAPACITY, -1);
+  if (s >= g.S) return;
+  const StreamDesc d = stream_desc(g, s);
+  if (!d.ok || off + len > capacity) return;
+  const Word *src = reinterpret_cast<const Word *>(scratch + slot_end(g, d, s) - len);
+  Word *dst = reinterpret_cast<Word *>(out + off);
+  const uint64_t words = len / sizeof(Word);
+  for (uint64_t k = lane; k < words; k += 32) dst[k] = __ldg(src + k);
+}
+
 __global__ void debug_divide_kernel(const uint64_t *x, const uint32_t *f, int64_t n, uint64_t *q,
                                     uint32_t *r) {
   for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n;
@@ -1302,7 +1350,7 @@ int launch_encode_t(const EncCtx &c, cudaStream_t st) {
   const int optin = smem_optin(dev);
   const uint32_t lim = (uint32_t)optin - 64u;  // room for the kernel's static shared memory
   const uint32_t max_dyn = tab + kEncStageBytes + tbl <= lim ? tab + kEncStageBytes + tbl : lim;
-  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)max_dyn) !=
+  if (ensure_dyn_smem((const void *)kern, (uint32_t)(max_dyn)) !=
       cudaSuccess)
     return RANS_ERR_CUDA;
   const int sms = num_sms(dev);
@@ -1312,7 +1360,7 @@ int launch_encode_t(const EncCtx &c, cudaStream_t st) {
     // Spread the streams over every SM: as many CTAs as fit per SM, each with
     // enough warps for one stream per warp when possible.
     int per_sm = 0;
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, 32, tab + per_warp) !=
+    if (blocks_per_sm(&per_sm, (const void *)kern, 32, (uint32_t)(tab + per_warp)) !=
             cudaSuccess ||
         per_sm < 1)
       return RANS_ERR_CUDA;
@@ -1327,7 +1375,7 @@ int launch_encode_t(const EncCtx &c, cudaStream_t st) {
     threads = (int)warps * 32;
     smem = tab + (uint32_t)warps * per_warp;
     int fit = 0;
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&fit, kern, threads, smem) != cudaSuccess ||
+    if (blocks_per_sm(&fit, (const void *)kern, threads, (uint32_t)(smem)) != cudaSuccess ||
         fit < 1)
       return RANS_ERR_CUDA;
     const int64_t need = (c.g.S + warps - 1) / warps;
@@ -1336,7 +1384,7 @@ int launch_encode_t(const EncCtx &c, cudaStream_t st) {
   } else {
     threads = kEncThreads1;
     int fit = 0;
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&fit, kern, threads, smem) != cudaSuccess ||
+    if (blocks_per_sm(&fit, (const void *)kern, threads, (uint32_t)(smem)) != cudaSuccess ||
         fit < 1)
       return RANS_ERR_CUDA;
     const int64_t need = (c.g.S + threads - 1) / threads;
@@ -1357,11 +1405,11 @@ int launch_encode_wn(const EncCtx &c, int mode, cudaStream_t st) {
   const uint32_t tab = enc_table_bytes(mode, c);
   int dev = 0;
   cudaGetDevice(&dev);
-  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)tab) !=
+  if (ensure_dyn_smem((const void *)kern, (uint32_t)(tab)) !=
       cudaSuccess)
     return RANS_ERR_CUDA;
   int fit = 0;
-  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&fit, kern, kSegThreads, tab) !=
+  if (blocks_per_sm(&fit, (const void *)kern, kSegThreads, (uint32_t)(tab)) !=
           cudaSuccess ||
       fit < 1)
     return RANS_ERR_CUDA;
@@ -1477,6 +1525,16 @@ int launch_encode_float(const float *y, const float *means, const float *scales,
 int launch_compact(const Geom &g, const char *scratch, const uint64_t *lens, uint8_t *out,
                    uint64_t out_capacity, uint64_t *offsets, int32_t *status,
                    cudaStream_t st) {
+  if (g.S > 0 && g.S <= kFusedMaxStreams) {
+    const unsigned blocks = (unsigned)((g.S + kCompactWarps - 1) / kCompactWarps);
+    if (g.fmt == RANS_FMT_RANS32_16)
+      compact_streams_kernel<uint16_t><<<blocks, kCompactWarps * 32, 0, st>>>(
+          g, scratch, lens, offsets, out, out_capacity, status);
+    else
+      compact_streams_kernel<uint32_t><<<blocks, kCompactWarps * 32, 0, st>>>(
+          g, scratch, lens, offsets, out, out_capacity, status);
+    return cudaGetLastError() == cudaSuccess ? RANS_OK : RANS_ERR_CUDA;
+  }
   scan_lengths_kernel<<<1, kScanThreads, 0, st>>>(lens, g.S, offsets, out_capacity, status);
   if (g.S > 0) {
     int dev = 0;

@@ -68,5 +68,10 @@ int encode_tile_map(void *map, const void *base, uint64_t width, uint64_t height
 // Device properties cached per device.
 int num_sms(int device);
 int smem_optin(int device);
+// Kernel launch set-up, cached per (kernel, device): raise the kernel's
+// dynamic shared memory limit to at least `bytes`, and its resident blocks
+// per SM at `threads` threads and `smem` bytes of dynamic shared memory.
+cudaError_t ensure_dyn_smem(const void *fn, uint32_t bytes);
+cudaError_t blocks_per_sm(int *out, const void *fn, int threads, uint32_t smem);
 
 }  // namespace rb

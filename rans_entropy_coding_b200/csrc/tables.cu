@@ -28,9 +28,11 @@ namespace rb {
 namespace {
 
 constexpr int kRowThreads = 1024;
+static_assert(kRowThreads == 1024, "one lane per warp total in the block scan");
 
 // Block-wide exclusive scan of a 64-bit value over kRowThreads threads (warp
-// shuffles, then one thread over the warp totals); *total gets the block sum.
+// shuffles, then every warp scans the 32 warp totals); *total gets the block
+// sum.
 struct BlockScratch {
   unsigned long long warp[kRowThreads / 32];
   unsigned long long total;
@@ -48,18 +50,16 @@ __device__ unsigned long long block_excl_scan(unsigned long long v, BlockScratch
   }
   if (lane == 31) sh.warp[wid] = inc;
   __syncthreads();
-  if (threadIdx.x == 0) {
-    unsigned long long run = 0;
-    for (int i = 0; i < kRowThreads / 32; ++i) {
-      const unsigned long long w = sh.warp[i];
-      sh.warp[i] = run;
-      run += w;
-    }
-    sh.total = run;
+  // every warp scans the 32 warp totals itself and takes its own prefix
+  const unsigned long long w = sh.warp[lane];
+  unsigned long long wi = w;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const unsigned long long t = __shfl_up_sync(kFull, wi, o);
+    if (lane >= o) wi += t;
   }
-  __syncthreads();
-  *total = sh.total;
-  const unsigned long long ex = sh.warp[wid] + inc - v;
+  *total = __shfl_sync(kFull, wi, 31);
+  const unsigned long long ex = __shfl_sync(kFull, wi - w, wid) + inc - v;
   __syncthreads();  // every thread has read the scratch before anyone reuses it
   return ex;
 }
@@ -394,7 +394,7 @@ struct ChunkArea {
 // covers kSlotsPerBlock slots of one row and stages the row in shared
 // memory when it has at most kRowSmem entries.
 constexpr int kSlotThreads = 256;
-constexpr int kSlotsPerThread = 4;
+constexpr int kSlotsPerThread = 1;
 constexpr int kSlotsPerBlock = kSlotThreads * kSlotsPerThread;
 constexpr int kRowSmem = 8192;
 constexpr uint32_t kSlotSmemBytes = 4u * kRowSmem;
@@ -719,9 +719,10 @@ int refresh_tables(const int32_t *cdfs, int K, int Lmax, const int32_t *lengths,
   ca.used = reinterpret_cast<uint32_t *>(b) + kChunkUsedWord;
   ca.search = reinterpret_cast<uint32_t *>(b) + kSearchFlagWord;
   if (cudaMemsetAsync(ca.used, 0, 8, st) != cudaSuccess) return RANS_ERR_CUDA;
-  // blocks of kSlotsPerBlock slots, enough for the largest possible row
-  // (2^kMaxQ slots); blocks past a smaller row's slots return at once
-  dim3 grid((unsigned)((1 << kMaxQ) / kSlotsPerBlock), (unsigned)K);
+  // blocks of kSlotsPerBlock slots, enough for the table's largest row
+  // (blocks past a smaller row's slots return at once)
+  const int qmax = t.max_slot_log2 >= kMinQ && t.max_slot_log2 <= kMaxQ ? t.max_slot_log2 : kMaxQ;
+  dim3 grid((unsigned)(((1 << qmax) + kSlotsPerBlock - 1) / kSlotsPerBlock), (unsigned)K);
   refresh_kernel<<<grid, kSlotThreads, kSlotSmemBytes, st>>>(
       cdfs, Lmax, lengths, offsets, (uint32_t)(kPrec - t.precision), dmeta, dbuckets, dstarts,
       dslots, ca, status);
@@ -933,6 +934,9 @@ int prepare_tables(const int32_t *cdfs, int K, int Lmax, const int32_t *lengths,
       dec_smem ? 1 : ((int64_t)meta_bytes + start_bytes + kDecStageBytes <= budget ? 2 : 0);
   out->device = dev;
   out->precision = prec;
+  int qmax = kMinQ;
+  for (int r = 0; r < K; ++r) qmax = q[r] > qmax ? q[r] : qmax;
+  out->max_slot_log2 = qmax;
   return RANS_OK;
 }
 
@@ -960,8 +964,7 @@ int prepare_alias(const int32_t *cdfs, int K, int Lmax, const int32_t *lengths,
   uint2 *aslots = reinterpret_cast<uint2 *>(alias);
   uint16_t *remap = reinterpret_cast<uint16_t *>(reinterpret_cast<char *>(alias) + slot_bytes);
   const uint32_t smem = 6u * 4u * (uint32_t)nmax;
-  if (cudaFuncSetAttribute(alias_build_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           (int)smem) != cudaSuccess)
+  if (ensure_dyn_smem((const void *)alias_build_kernel, (uint32_t)(smem)) != cudaSuccess)
     return RANS_ERR_CUDA;
   if (cudaMemsetAsync(alias, 0, slot_bytes, st) != cudaSuccess) return RANS_ERR_CUDA;
   alias_build_kernel<<<K, 256, smem, st>>>(cdfs, Lmax, lengths, dmeta, t.precision, nmax, aslots,
