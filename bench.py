@@ -63,6 +63,9 @@ def parse():
     ap.add_argument("--workload", choices=["batch", "tiny", "z", "y", "sweep", "float", "r16"],
                     default="batch")
     ap.add_argument("--interleave", type=int, default=None, help="W for --workload y")
+    ap.add_argument("--log2n", type=int, default=28,
+                    help="--workload sweep: 2^log2n symbols (28 is the configuration; smaller "
+                         "sizes serve profiling)")
     ap.add_argument("--format", choices=["rans64", "rans32_16"], default=None,
                     help="coder format (default: rans32_16 for --workload r16, else rans64)")
     ap.add_argument("--alias", action="store_true",
@@ -216,7 +219,8 @@ def shard_streams(w, world, rank):
                 stream_block=(b["first"], b["count"], sym.size, int(w["chunking"]["n_streams"])))
 
 
-def load_inputs(rank, group, images=N_IMAGES, workload="batch", interleave=None, world=1):
+def load_inputs(rank, group, images=N_IMAGES, workload="batch", interleave=None, world=1,
+                log2n=28):
     if workload == "tiny":
         w = WL.tiny()
     elif workload == "z":
@@ -224,7 +228,7 @@ def load_inputs(rank, group, images=N_IMAGES, workload="batch", interleave=None,
     elif workload == "y":
         w = WL.y_latent(W=interleave or 32)
     elif workload == "sweep":
-        w = WL.sweep(log2_n=28)
+        w = WL.sweep(log2_n=log2n)
         if world > 1:  # split by stream range
             w = shard_streams(w, world, rank)
     elif workload == "r16":
@@ -311,7 +315,8 @@ def run_reference(args, world, rank):
     if rank != 0:
         return
     w = apply_format(load_inputs(0, args.group, workload=args.workload,
-                                 interleave=args.interleave), args.format, args.alias)
+                                 interleave=args.interleave, log2n=args.log2n), args.format,
+                     args.alias)
     if args.workload == "float":  # the oracle codes rows and symbols computed first
         import oracle as O
         w = dict(w, symbols=O.quantize(w["y"], w["means"]), W=32,
@@ -352,7 +357,7 @@ def run_ours(args, world, rank, local):
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
     w = apply_format(load_inputs(rank, args.group, args.images, args.workload, args.interleave,
-                                 world), args.format, args.alias)
+                                 world, args.log2n), args.format, args.alias)
     fmt, prec = w["fmt"], w["precision"]
     sym_np = np.ascontiguousarray(np.asarray(w["symbols"]).reshape(-1))
     idx_np = np.ascontiguousarray(w["indexes"], dtype=np.int32)

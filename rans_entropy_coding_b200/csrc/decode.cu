@@ -1019,6 +1019,53 @@ __device__ __forceinline__ int32_t dec_group_fast(WarpDec<F> &st, const RowMeta 
   return (int32_t)sym + m.offset;
 }
 
+
+// The fast group of the 64-bit format with every step in 32-bit halves (the
+// window cursor too: the caller takes this path for streams of fewer than
+// 2^31 words).
+__device__ __forceinline__ int32_t dec_group_lean64(WarpDec<Rans64> &st, const RowMeta &m,
+                                                    const uint16_t *starts, const uint32_t *slots,
+                                                    const uint32_t *words, uint32_t nw32,
+                                                    uint32_t &esc) {
+  const uint32_t lane = threadIdx.x & 31;
+  const uint32_t xl = (uint32_t)st.x, xh = (uint32_t)(st.x >> 32);
+  const uint32_t cum = xl & 0xffffu;
+  const uint32_t sh = m.slot >> 27;
+  const uint32_t i1 = (m.slot & 0x07ffffffu) + (cum >> sh);
+  const uint32_t se = slots[i1];
+  const uint32_t c = cum & ((1u << sh) - 1u);
+  const uint32_t lo = se & 0xffffu;
+  const uint32_t e1 = __byte_perm(se, 0u, 0x4442u), e2 = se >> 24;
+  uint32_t sym = lo + (c > e1 ? 1u : 0u) + (c > e2 ? 1u : 0u);
+  const bool bm = e1 == 0xffu && e2 != 0xffu;
+  const uint32_t i2 = bm ? (lo | ((se >> 8) & 0xff0000u)) + (c >> 4) : i1;
+  const uint32_t ce = slots[i2];
+  const uint32_t sym2 = (ce >> 16) + __popc(ce & ((2u << (c & 15u)) - 1u));
+  sym = min(bm ? sym2 : sym, m.maxv);
+  esc |= sym == m.maxv ? 1u : 0u;
+  const uint32_t a = m.bucket_base + sym;
+  const uint32_t s0 = starts[a], s1 = starts[a + 1];
+  const uint32_t f = (s1 - s0) + (s1 == 0u ? 65536u : 0u);
+  const uint32_t tl = __funnelshift_r(xl, xh, 16), th = xh >> 16;
+  const uint64_t p = (uint64_t)f * tl + (uint64_t)(cum - s0);
+  const uint32_t nl = (uint32_t)p, nh = (uint32_t)(p >> 32) + f * th;
+  const bool need = __funnelshift_r(nl, nh, 31) == 0u;
+  const uint32_t src = lane >= st.off ? st.w0 : st.w1;
+  const uint32_t bal = __ballot_sync(kFull, need);
+  const uint32_t wv = __shfl_sync(kFull, src, st.off + __popc(bal & lanemask_lt()));
+  st.x = ((uint64_t)(need ? nl : nh) << 32) | (need ? wv : nl);
+  st.off += __popc(bal);
+  if (st.off >= 32) {
+    st.w0 = st.w1;
+    st.w1 = st.w2;
+    st.cur += 32;
+    st.off -= 32;
+    const uint32_t wi = (uint32_t)st.cur + 64u + lane;
+    st.w2 = __ldg(words + (wi < nw32 ? wi : nw32 - 1u));
+  }
+  return (int32_t)sym + m.offset;
+}
+
 __device__ __forceinline__ void chunk_next_if(ChunkPos &p, bool on) {
   const int32_t y = p.y + 4;
   const bool wrap = y == p.y1;
@@ -1035,7 +1082,7 @@ __device__ __forceinline__ bool decode_tile_stream_fast(const DecCtx &c, const T
                                                         uint32_t &par, int64_t s) {
   using State = typename F::State;
   using Word = typename F::Word;
-  constexpr int kJload = GC > 3 ? GC - 3 : 0;  // the group after which chunk k + 1 loads
+  constexpr int kJload = 0;  // chunk k + 1 loads right after chunk k's first group
   constexpr int kHalfW = (int)(kTileRingHalf / 4);
   const int lane = threadIdx.x & 31;
   const Geom &g = c.g;
@@ -1121,7 +1168,10 @@ __device__ __forceinline__ bool decode_tile_stream_fast(const DecCtx &c, const T
     for (int j = 0; j < GC; ++j) {
       RowMeta mn = m;
       if (j + 1 < GC) mn = meta_of((uint32_t)rh[(j + 1) * 32 + lane]);
-      rh[j * 32 + lane] = dec_group_fast<F>(st, m, starts, slots, words, nw, sh, esc);
+      if constexpr (std::is_same<F, Rans64>::value)
+        rh[j * 32 + lane] = dec_group_lean64(st, m, starts, slots, words, (uint32_t)nw, esc);
+      else
+        rh[j * 32 + lane] = dec_group_fast<F>(st, m, starts, slots, words, nw, sh, esc);
       if (j == 0) {
         tma::prefetch_l2_3d_if(l0 & more3, imap, x0, pf.y, pf.z);
         chunk_next_if(pf, more3 != 0);
@@ -1211,8 +1261,10 @@ __global__ void __launch_bounds__(kDecMaxThreads32)
       // unrolled chunks for tile widths 64 and 56 (8 and 7 groups), the general
       // loop otherwise (fewer unrolled variants keep the hot code in the
       // instruction cache)
-      const int64_t ww = c.g.tw * ((s % c.g.ntx) + 1) <= c.g.Wd ? c.g.tw
-                                                                   : c.g.Wd % c.g.tw;
+      int64_t ww = c.g.tw * ((s % c.g.ntx) + 1) <= c.g.Wd ? c.g.tw : c.g.Wd % c.g.tw;
+      // (the fast chunks keep 32-bit word cursors: streams of fewer than 2^31 words)
+      const uint64_t wbytes = c.offs[s + 1] - c.offs[s];
+      if (wbytes >= (sizeof(typename F::Word) << 31)) ww = 0;
       switch (ww) {
         case 64: ok = decode_tile_stream_fast<F, 8>(c, maps, meta, starts, slots, ring, ring_p, bar0, par, s); break;
         case 56: ok = decode_tile_stream_fast<F, 7>(c, maps, meta, starts, slots, ring, ring_p, bar0, par, s); break;
