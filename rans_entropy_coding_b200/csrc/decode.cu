@@ -961,30 +961,12 @@ __device__ __forceinline__ bool decode_tile_stream(const DecCtx &c, const TileMa
 // widths of 56 and 64 (7 and 8 groups per chunk) a chunk is therefore decoded
 // as one unrolled block: the copy-engine work is predicated on lane 0,
 // escapes are only recorded, and the only branch left is the window
-// advance (about once in seven groups).  A chunk in which any lane met an
-// escape is decoded again from its saved state on the lane-serial path (its
-// row indexes reloaded, since the fast pass overwrote them with values); the
-// fast pass after an escape runs on a wrong state but reads only inside the
-// tables, the register window and the stream's words.
-
-// Word i of the stream (clamped to its last word) where p is nonzero, else
-// `old`, with no branch.
-template <class F>
-__device__ __forceinline__ uint32_t window_word_if(uint32_t p, const typename F::Word *words,
-                                                   uint64_t nw, uint64_t i, uint32_t old) {
-  const typename F::Word *a = words + (i < nw ? i : nw - 1);
-  if constexpr (sizeof(typename F::Word) == 4) {
-    asm("{\n\t.reg .pred q;\n\tsetp.ne.u32 q, %1, 0;\n\t@q ld.global.nc.u32 %0, [%2];\n\t}"
-        : "+r"(old)
-        : "r"(p), "l"(a));
-  } else {
-    asm("{\n\t.reg .pred q;\n\t.reg .u16 h;\n\tsetp.ne.u32 q, %1, 0;\n\t"
-        "@q ld.global.nc.u16 h, [%2];\n\t@q cvt.u32.u16 %0, h;\n\t}"
-        : "+r"(old)
-        : "r"(p), "l"(a));
-  }
-  return old;
-}
+// advance (about once in seven groups; the 64-bit format's variant below
+// reads its words from a shared-memory window and has none).  A chunk in
+// which any lane met an escape is decoded again from its saved state on the
+// lane-serial path (its row indexes reloaded, since the fast pass overwrote
+// them with values); the fast pass after an escape runs on a wrong state but
+// reads only inside the tables, the register window and the stream's words.
 
 // One full group on the fast path: lookup, state update and refill with no
 // branch; a lane whose symbol is the escape bucket only sets `esc`.
@@ -1019,52 +1001,6 @@ __device__ __forceinline__ int32_t dec_group_fast(WarpDec<F> &st, const RowMeta 
   return (int32_t)sym + m.offset;
 }
 
-
-// The fast group of the 64-bit format with every step in 32-bit halves (the
-// window cursor too: the caller takes this path for streams of fewer than
-// 2^31 words).
-__device__ __forceinline__ int32_t dec_group_lean64(WarpDec<Rans64> &st, const RowMeta &m,
-                                                    const uint16_t *starts, const uint32_t *slots,
-                                                    const uint32_t *words, uint32_t nw32,
-                                                    uint32_t &esc) {
-  const uint32_t lane = threadIdx.x & 31;
-  const uint32_t xl = (uint32_t)st.x, xh = (uint32_t)(st.x >> 32);
-  const uint32_t cum = xl & 0xffffu;
-  const uint32_t sh = m.slot >> 27;
-  const uint32_t i1 = (m.slot & 0x07ffffffu) + (cum >> sh);
-  const uint32_t se = slots[i1];
-  const uint32_t c = cum & ((1u << sh) - 1u);
-  const uint32_t lo = se & 0xffffu;
-  const uint32_t e1 = __byte_perm(se, 0u, 0x4442u), e2 = se >> 24;
-  uint32_t sym = lo + (c > e1 ? 1u : 0u) + (c > e2 ? 1u : 0u);
-  const bool bm = e1 == 0xffu && e2 != 0xffu;
-  const uint32_t i2 = bm ? (lo | ((se >> 8) & 0xff0000u)) + (c >> 4) : i1;
-  const uint32_t ce = slots[i2];
-  const uint32_t sym2 = (ce >> 16) + __popc(ce & ((2u << (c & 15u)) - 1u));
-  sym = min(bm ? sym2 : sym, m.maxv);
-  esc |= sym == m.maxv ? 1u : 0u;
-  const uint32_t a = m.bucket_base + sym;
-  const uint32_t s0 = starts[a], s1 = starts[a + 1];
-  const uint32_t f = (s1 - s0) + (s1 == 0u ? 65536u : 0u);
-  const uint32_t tl = __funnelshift_r(xl, xh, 16), th = xh >> 16;
-  const uint64_t p = (uint64_t)f * tl + (uint64_t)(cum - s0);
-  const uint32_t nl = (uint32_t)p, nh = (uint32_t)(p >> 32) + f * th;
-  const bool need = __funnelshift_r(nl, nh, 31) == 0u;
-  const uint32_t src = lane >= st.off ? st.w0 : st.w1;
-  const uint32_t bal = __ballot_sync(kFull, need);
-  const uint32_t wv = __shfl_sync(kFull, src, st.off + __popc(bal & lanemask_lt()));
-  st.x = ((uint64_t)(need ? nl : nh) << 32) | (need ? wv : nl);
-  st.off += __popc(bal);
-  if (st.off >= 32) {
-    st.w0 = st.w1;
-    st.w1 = st.w2;
-    st.cur += 32;
-    st.off -= 32;
-    const uint32_t wi = (uint32_t)st.cur + 64u + lane;
-    st.w2 = __ldg(words + (wi < nw32 ? wi : nw32 - 1u));
-  }
-  return (int32_t)sym + m.offset;
-}
 
 __device__ __forceinline__ void chunk_next_if(ChunkPos &p, bool on) {
   const int32_t y = p.y + 4;
@@ -1168,10 +1104,7 @@ __device__ __forceinline__ bool decode_tile_stream_fast(const DecCtx &c, const T
     for (int j = 0; j < GC; ++j) {
       RowMeta mn = m;
       if (j + 1 < GC) mn = meta_of((uint32_t)rh[(j + 1) * 32 + lane]);
-      if constexpr (std::is_same<F, Rans64>::value)
-        rh[j * 32 + lane] = dec_group_lean64(st, m, starts, slots, words, (uint32_t)nw, esc);
-      else
-        rh[j * 32 + lane] = dec_group_fast<F>(st, m, starts, slots, words, nw, sh, esc);
+      rh[j * 32 + lane] = dec_group_fast<F>(st, m, starts, slots, words, nw, sh, esc);
       if (j == 0) {
         tma::prefetch_l2_3d_if(l0 & more3, imap, x0, pf.y, pf.z);
         chunk_next_if(pf, more3 != 0);
@@ -1222,12 +1155,275 @@ __device__ __forceinline__ bool decode_tile_stream_fast(const DecCtx &c, const T
   return true;
 }
 
+// ------------------------------------------ 64-bit format, word window --
+// The 64-bit format's unrolled chunks keep the stream's words in a ring of
+// kWinWords words in shared memory, refilled with cp.async once per chunk
+// in blocks of 32 (the blocks the reads have passed).  A group reads its
+// refill word from the ring (one shared load at the lane's rank among the
+// lanes that refill) and takes no branch, so a chunk of 7 or 8 groups is
+// one block of straight-line code.  The decoded values stay in registers
+// until the chunk ends, so no store to the ring orders the groups' table
+// reads.
+constexpr uint32_t kWinWords = 512;
+constexpr uint32_t kWinBytes = 4 * kWinWords;
+static_assert(kTileStreamBytes == kTileRingBytes + kWinBytes, "index ring + word window");
+
+// The tile origin of stream s: first column x0 and the chunk position of
+// its first chunk.
+__device__ __forceinline__ void tile_origin(const Geom &g, const StreamDesc &d, int64_t s,
+                                            int32_t &x0, ChunkPos &p) {
+  const int64_t per_img = g.ng * g.nty * g.ntx;
+  const int64_t b = s / per_img, t0 = s - b * per_img;
+  const int64_t gi = t0 / (g.nty * g.ntx), t1 = t0 - gi * (g.nty * g.ntx);
+  const int64_t ty = t1 / g.ntx, tx = t1 - ty * g.ntx;
+  x0 = (int32_t)(tx * g.tw);
+  p.y0 = p.y = (int32_t)(ty * g.th);
+  p.y1 = p.y0 + d.t.hh;
+  p.z = (int32_t)(b * g.C + gi * g.cg);
+}
+
+// One group: lookup, state update and refill, no branch; a lane whose
+// symbol is the escape bucket only sets `esc`.  win: the stream's word
+// ring (word i at win[i mod kWinWords]), rd: the next word to read.
+__device__ __forceinline__ int32_t dec_group_win64(uint64_t &x, uint32_t &rd, const RowMeta &m,
+                                                   const uint16_t *starts, const uint32_t *slots,
+                                                   const uint32_t *win, uint32_t &esc) {
+  const uint32_t xl = (uint32_t)x, xh = (uint32_t)(x >> 32);
+  const uint32_t cum = xl & 0xffffu;
+  const uint32_t sh = m.slot >> 27;
+  const uint32_t i1 = (m.slot & 0x07ffffffu) + (cum >> sh);
+  const uint32_t se = slots[i1];
+  const uint32_t c = cum & ((1u << sh) - 1u);
+  const uint32_t lo = se & 0xffffu;
+  const uint32_t e1 = __byte_perm(se, 0u, 0x4442u), e2 = se >> 24;
+  uint32_t sym = lo + (c > e1 ? 1u : 0u) + (c > e2 ? 1u : 0u);
+  const bool bm = e1 == 0xffu && e2 != 0xffu;
+  const uint32_t i2 = bm ? (lo | ((se >> 8) & 0xff0000u)) + (c >> 4) : i1;
+  const uint32_t ce = slots[i2];
+  const uint32_t sym2 = (ce >> 16) + __popc(ce & ((2u << (c & 15u)) - 1u));
+  sym = min(bm ? sym2 : sym, m.maxv);
+  esc |= sym == m.maxv ? 1u : 0u;
+  const uint32_t a = m.bucket_base + sym;
+  const uint32_t s0 = starts[a], s1 = starts[a + 1];
+  const uint32_t f = (s1 - s0) + (s1 == 0u ? 65536u : 0u);
+  // x' = f (x >> 16) + cum - start in 32-bit halves; refill when x' < 2^31
+  const uint32_t tl = __funnelshift_r(xl, xh, 16), th = xh >> 16;
+  const uint64_t p = (uint64_t)f * tl + (uint64_t)(cum - s0);
+  const uint32_t nl = (uint32_t)p, nh = (uint32_t)(p >> 32) + f * th;
+  const bool need = __funnelshift_r(nl, nh, 31) == 0u;
+  const uint32_t bal = __ballot_sync(kFull, need);
+  const uint32_t wv = win[(rd + __popc(bal & lanemask_lt())) & (kWinWords - 1u)];
+  x = ((uint64_t)(need ? nl : nh) << 32) | (need ? wv : nl);
+  rd += __popc(bal);
+  return (int32_t)sym + m.offset;
+}
+
+// Loads the blocks of 32 words the reads have passed (once they land, the
+// ring holds words [ldn - kWinWords, ldn)) with the words that follow; one
+// cp.async commit group per call, possibly empty.  Word indexes past the
+// stream read its last word.
+__device__ __forceinline__ void win_refill(uint32_t *win, const uint32_t *words, uint32_t nw,
+                                           uint32_t rd, uint32_t &ldn) {
+  const uint32_t lane = threadIdx.x & 31;
+  const uint32_t end = (rd & ~31u) + kWinWords;
+#pragma unroll 1
+  for (; ldn < end; ldn += 32) {
+    const uint32_t wi = ldn + lane;
+    cp_async4(win + (wi & (kWinWords - 1u)), words + (wi < nw ? wi : nw - 1u));
+  }
+  cp_async_commit();
+}
+
+// Stream s (64-bit format, tile width 56 or 64: GC = 7 or 8 groups a chunk,
+// fewer than 2^31 words) on the unrolled path.
+template <int GC>
+__device__ __forceinline__ bool decode_tile_win64(const DecCtx &c, const TileMaps &maps,
+                                                  const RowMeta *meta, const uint16_t *starts,
+                                                  const uint32_t *slots, uint32_t ring,
+                                                  int32_t *ring_p, uint32_t bar0, uint32_t &par,
+                                                  int64_t s, const StreamDesc &d,
+                                                  const uint32_t *words, uint32_t nw) {
+  constexpr int kHalfW = (int)(kTileRingHalf / 4);
+  constexpr uint32_t cbytes = 128u * GC;
+  const int lane = threadIdx.x & 31;
+  const Geom &g = c.g;
+  const uint32_t kmax = (uint32_t)c.K - 1u;
+  const int cls = d.t.ww == (int32_t)g.tw ? 0 : 1;
+  const void *imap = &maps.idx[cls];
+  const void *omap = &maps.out[cls];
+  const int32_t M = (int32_t)(d.n / (32 * GC));
+  const uint32_t l0 = lane == 0 ? 1u : 0u;
+  const uint32_t bar1 = bar0 + 8;
+  uint32_t *win = reinterpret_cast<uint32_t *>(ring_p + kTileRingBytes / 4);
+  int32_t x0;
+  ChunkPos ld;
+  tile_origin(g, d, s, x0, ld);
+  ChunkPos sd = ld, pf = ld;
+  if (lane == 0)
+    bulk_prefetch_l2(reinterpret_cast<const char *>(c.in),
+                     reinterpret_cast<const char *>(c.in) + c.in_bytes,
+                     reinterpret_cast<const char *>(words + 64), sizeof(uint32_t) * (nw - 64));
+  // chunk 0 into half 0, once earlier stores have read the ring; chunks 1
+  // and 2 into L2
+  __syncwarp();
+  tma::bulk_wait_read_if(l0);
+  tma::fence_proxy_async();
+  tma::arrive_expect_if(l0, bar0, cbytes);
+  tma::load_3d_if(l0, ring, imap, x0, ld.y, ld.z, bar0);
+  ld.next();
+  pf.next();
+  for (int32_t q = 1; q < 3 && q < M; ++q) {
+    tma::prefetch_l2_3d_if(l0, imap, x0, pf.y, pf.z);
+    pf.next();
+  }
+  uint32_t pending = 1u;
+
+  uint64_t x = (uint64_t)__ldg(words + 2 * lane) | ((uint64_t)__ldg(words + 2 * lane + 1) << 32);
+  uint32_t rd = 64, ldn = 64, rmax = 0;
+  bool bad = false;
+  auto meta_of = [&](uint32_t r) -> RowMeta {
+    rmax = max(rmax, r);
+    return row_meta(meta, min(r, kmax));
+  };
+  // a bounded wait for the chunk in half h; on giving up, a bounded wait for
+  // every load still in flight, and the warp stops
+  auto wait_half = [&](int h) -> bool {
+    const uint32_t bar = h ? bar1 : bar0;
+    const bool ok = tma::wait_bounded(bar, (par >> h) & 1u, kTileWaitTries);
+    if (__all_sync(kFull, ok)) {
+      par ^= 1u << h;
+      pending &= ~(1u << h);
+      return true;
+    }
+    if (lane == 0) report(c.status, RANS_ERR_TIMEOUT, s);
+    for (int q = 0; q < 2; ++q)
+      if (pending >> q & 1u) tma::wait_bounded(q ? bar1 : bar0, (par >> q) & 1u, kTileWaitTries);
+    cp_async_wait<0>();
+    return false;
+  };
+#pragma unroll 1
+  for (int32_t k = 0; k < M; ++k) {
+    const int h = k & 1;
+    // the word window: top up, then wait for the words this chunk can read
+    // (at most 32 a group): the blocks loaded before this chunk hold them
+    // unless the window was just restarted
+    const bool ahead = rd + 32u * GC <= ldn;
+    win_refill(win, words, nw, rd, ldn);
+    if (ahead) cp_async_wait<1>(); else cp_async_wait<0>();
+    if (!wait_half(h)) return false;
+    __syncwarp();  // every lane's window words, before any lane reads them
+    const uint32_t more1 = k + 1 < M ? 1u : 0u, more3 = k + 3 < M ? 1u : 0u;
+    int32_t *rh = ring_p + h * kHalfW;
+    const uint64_t xs = x;
+    const uint32_t rds = rd;
+    uint32_t esc = 0;
+    int32_t val[GC];
+#pragma unroll
+    for (int j = 0; j < GC; ++j) {
+      const RowMeta m = meta_of((uint32_t)rh[j * 32 + lane]);
+      val[j] = dec_group_win64(x, rd, m, starts, slots, win, esc);
+      if (j == 0) {
+        // chunk k + 3 into L2; chunk k + 1 into the other half, once chunk
+        // k - 1's store has read it
+        tma::prefetch_l2_3d_if(l0 & more3, imap, x0, pf.y, pf.z);
+        chunk_next_if(pf, more3 != 0);
+        __syncwarp();
+        const uint32_t bar = h ? bar0 : bar1;
+        tma::bulk_wait_read_if(l0 & more1);
+        tma::fence_proxy_async();
+        tma::arrive_expect_if(l0 & more1, bar, cbytes);
+        tma::load_3d_if(l0 & more1, ring + (uint32_t)(h ^ 1) * kTileRingHalf, imap, x0, ld.y,
+                        ld.z, bar);
+        pending |= more1 << (h ^ 1);
+        chunk_next_if(ld, more1 != 0);
+      }
+    }
+    if (!__any_sync(kFull, esc != 0)) {
+#pragma unroll
+      for (int j = 0; j < GC; ++j) rh[j * 32 + lane] = val[j];
+    } else {
+      // an escape in this chunk: decode it again from its saved state on
+      // the lane-serial path (its row indexes are still in the ring), then
+      // restart the word window where that left off
+      WarpDec<Rans64> w;
+      w.x = xs;
+      w.cur = rds;
+      w.off = 0;
+      w.rmax = 0;
+      w.bad = false;
+      load_window(w, words, nw);
+#pragma unroll 1
+      for (int j = 0; j < GC; ++j) {
+        const RowMeta mj = meta_of((uint32_t)rh[j * 32 + lane]);
+        rh[j * 32 + lane] =
+            dec_group_val<Rans64, false>(w, mj, starts, slots, words, nw, Rans64::shift(c.sh));
+      }
+      bad = bad || w.bad;
+      x = w.x;
+      rd = (uint32_t)(w.cur + w.off);
+      cp_async_wait<0>();
+      __syncwarp();
+      ldn = rd & ~31u;
+    }
+    // chunk k's decoded values go out
+    tma::fence_proxy_async();
+    __syncwarp();
+    tma::store_3d_commit_if(l0, omap, x0, sd.y, sd.z, ring + (uint32_t)h * kTileRingHalf);
+    sd.next();
+  }
+  cp_async_wait<0>();
+  if (__any_sync(kFull, rmax > kmax)) {
+    if (lane == 0) report(c.status, RANS_ERR_INDEX, s);
+    return true;
+  }
+  const bool ok = !bad && x == Rans64::kLow && rd == nw;
+  if (!__all_sync(kFull, ok) && lane == 0) report(c.status, RANS_ERR_CORRUPT, s);
+  return true;
+}
+
+// Stream s with the warp's ring and barriers: the unrolled chunks for tile
+// widths 64 and 56 (8 and 7 groups) when its words are well formed and
+// fewer than 2^31 (32-bit word cursors), the general loop otherwise or when
+// the table has slots that search.
 template <class F>
-__global__ void __launch_bounds__(kDecMaxThreads32)
+__device__ __forceinline__ bool decode_tile_one(const DecCtx &c, const TileMaps &maps,
+                                                const RowMeta *meta, const uint16_t *starts,
+                                                const uint32_t *slots, uint32_t ring,
+                                                int32_t *ring_p, uint32_t bar0, uint32_t &par,
+                                                int64_t s, bool search) {
+  if (search)
+    return decode_tile_stream<F, true>(c, maps, meta, starts, slots, ring, ring_p, bar0, par, s);
+  const StreamDesc d = stream_desc(c.g, s);
+  const typename F::Word *words = nullptr;
+  uint64_t nw = 0;
+  const bool fast = d.ok && (d.t.ww == 64 || d.t.ww == 56) &&
+                    stream_bounds<F>(c, s, 32, words, nw) && nw < (uint64_t(1) << 31);
+  if (fast) {
+    if constexpr (std::is_same<F, Rans64>::value) {
+      if (d.t.ww == 64)
+        return decode_tile_win64<8>(c, maps, meta, starts, slots, ring, ring_p, bar0, par, s, d,
+                                    words, (uint32_t)nw);
+      return decode_tile_win64<7>(c, maps, meta, starts, slots, ring, ring_p, bar0, par, s, d,
+                                  words, (uint32_t)nw);
+    } else {
+      if (d.t.ww == 64)
+        return decode_tile_stream_fast<F, 8>(c, maps, meta, starts, slots, ring, ring_p, bar0,
+                                             par, s);
+      return decode_tile_stream_fast<F, 7>(c, maps, meta, starts, slots, ring, ring_p, bar0, par,
+                                           s);
+    }
+  }
+  return decode_tile_stream<F, false>(c, maps, meta, starts, slots, ring, ring_p, bar0, par, s);
+}
+
+// The tile-staged decoder: one stream per warp at a time, in scheduling
+// order (largest tiles first).
+template <class F>
+__global__ void __launch_bounds__(kTileMaxStreams * 32, 1)
     decode_tile_kernel(DecCtx c, const __grid_constant__ TileMaps maps) {
   extern __shared__ __align__(16) unsigned char smem[];
   __shared__ uint64_t bar;
-  __shared__ uint64_t ring_bar[kDecMaxWarps][2];
+  __shared__ uint64_t ring_bar[kTileMaxStreams][2];
   const char *gb = c.blob + kHeaderBytes;
   if (!stage_to_smem(smem, gb, c.meta_bytes, &bar, c.status, smem + c.meta_bytes,
                      gb + c.meta_bytes + c.bucket_bytes, c.start_bytes + c.slot_bytes))
@@ -1237,9 +1433,10 @@ __global__ void __launch_bounds__(kDecMaxThreads32)
   const uint32_t *slots = reinterpret_cast<const uint32_t *>(smem + c.meta_bytes + c.start_bytes);
   const uint32_t tab = c.meta_bytes + c.start_bytes + c.slot_bytes;
   const int warp = threadIdx.x >> 5, nwarp = blockDim.x >> 5, lane = threadIdx.x & 31;
-  // each warp's ring: 128-byte aligned (tensor-tile copies)
+  // each warp's index ring and word window: 128-byte aligned (tensor-tile
+  // copies)
   const uint32_t sbase = smem_addr(smem);
-  const uint32_t ring = ((sbase + tab + 127u) & ~127u) + (uint32_t)warp * kTileRingBytes;
+  const uint32_t ring = ((sbase + tab + 127u) & ~127u) + (uint32_t)warp * kTileStreamBytes;
   int32_t *ring_p = reinterpret_cast<int32_t *>(smem + (ring - sbase));
   const uint32_t bar0 = smem_addr(&ring_bar[warp][0]);
   if (lane == 0) {
@@ -1253,25 +1450,9 @@ __global__ void __launch_bounds__(kDecMaxThreads32)
   const bool search = reinterpret_cast<const uint32_t *>(c.blob)[kSearchFlagWord] != 0;
   for (int64_t k = blockIdx.x + (int64_t)gridDim.x * warp; k < c.g.S;
        k += (int64_t)gridDim.x * nwarp) {
-    const int64_t s = stream_of(c.g, k);
-    bool ok;
-    if (search) {
-      ok = decode_tile_stream<F, true>(c, maps, meta, starts, slots, ring, ring_p, bar0, par, s);
-    } else {
-      // unrolled chunks for tile widths 64 and 56 (8 and 7 groups), the general
-      // loop otherwise (fewer unrolled variants keep the hot code in the
-      // instruction cache)
-      int64_t ww = c.g.tw * ((s % c.g.ntx) + 1) <= c.g.Wd ? c.g.tw : c.g.Wd % c.g.tw;
-      // (the fast chunks keep 32-bit word cursors: streams of fewer than 2^31 words)
-      const uint64_t wbytes = c.offs[s + 1] - c.offs[s];
-      if (wbytes >= (sizeof(typename F::Word) << 31)) ww = 0;
-      switch (ww) {
-        case 64: ok = decode_tile_stream_fast<F, 8>(c, maps, meta, starts, slots, ring, ring_p, bar0, par, s); break;
-        case 56: ok = decode_tile_stream_fast<F, 7>(c, maps, meta, starts, slots, ring, ring_p, bar0, par, s); break;
-        default: ok = decode_tile_stream<F, false>(c, maps, meta, starts, slots, ring, ring_p, bar0, par, s);
-      }
-    }
-    if (!ok) break;
+    if (!decode_tile_one<F>(c, maps, meta, starts, slots, ring, ring_p, bar0, par,
+                            stream_of(c.g, k), search))
+      break;
   }
   if (lane == 0) tma::bulk_wait_all();
 }
@@ -1307,8 +1488,8 @@ int launch_decode_tile(const DecCtx &c, const int32_t *indexes, void *symbols, c
   cudaGetDevice(&dev);
   const uint32_t tab = dec_table_bytes(1, c);
   const int optin = smem_optin(dev);
-  const uint32_t lim = (uint32_t)optin - 64u - 2u * 8u * kDecMaxWarps;
-  if (tab + 128u + kTileRingBytes > lim) return kNotTaken;
+  const uint32_t lim = (uint32_t)optin - 64u - 2u * 8u * kTileMaxStreams;
+  if (tab + 128u + kTileStreamBytes > lim) return kNotTaken;
   TileMaps maps;
   const int64_t per_img = g.ng * g.nty * g.ntx;
   const int64_t depth = (g.S / per_img) * g.C;
@@ -1322,19 +1503,15 @@ int launch_decode_tile(const DecCtx &c, const int32_t *indexes, void *symbols, c
   }
   const int sms = num_sms(dev);
   int64_t warps = (g.S + sms - 1) / sms;
-  if (warps > kDecMaxWarps) warps = kDecMaxWarps;
-  const int64_t room = ((int64_t)lim - tab - 128) / kTileRingBytes;
+  if (warps > kTileMaxStreams) warps = kTileMaxStreams;
+  const int64_t room = ((int64_t)lim - tab - 128) / kTileStreamBytes;
   if (warps > room) warps = room;
   if (warps < 1) warps = 1;
-  const uint32_t smem = tab + 128u + (uint32_t)warps * kTileRingBytes;
+  const uint32_t smem = tab + 128u + (uint32_t)warps * kTileStreamBytes;
   auto kern = decode_tile_kernel<F>;
-  if (ensure_dyn_smem((const void *)kern, (uint32_t)(smem)) !=
-      cudaSuccess)
-    return RANS_ERR_CUDA;
+  if (ensure_dyn_smem((const void *)kern, smem) != cudaSuccess) return RANS_ERR_CUDA;
   int fit = 0;
-  if (blocks_per_sm(&fit, (const void *)kern, (int)warps * 32, (uint32_t)(smem)) !=
-          cudaSuccess ||
-      fit < 1)
+  if (blocks_per_sm(&fit, (const void *)kern, (int)warps * 32, smem) != cudaSuccess || fit < 1)
     return RANS_ERR_CUDA;
   const int64_t need = (g.S + warps - 1) / warps;
   const int64_t cap = (int64_t)fit * sms;

@@ -80,9 +80,14 @@ constexpr uint32_t kDecStageBytes = kDecMaxWarps * kDecStage * 32 * 4;
 // up to 64 int32 each, 128-byte aligned.
 constexpr uint32_t kTileRingHalf = 1024;
 constexpr uint32_t kTileRingBytes = 2 * kTileRingHalf;
+// The tile decoder's shared memory per stream: its index ring and a word
+// window of the same size.
+constexpr uint32_t kTileStreamBytes = 2 * kTileRingBytes;
 // Shared memory the decoder's tables leave for its rings.
 constexpr uint32_t kDecRingRoom = kDecMaxWarps * kTileRingBytes + 128;
 static_assert(kDecRingRoom >= kDecStageBytes, "room for either decoder's rings");
+// Streams a tile decoder CTA holds at once.
+constexpr int kTileMaxStreams = (int)((kDecRingRoom - 128) / kTileStreamBytes);
 constexpr uint32_t kEncStageBytes = kEncMaxWarps * kEncStage * 32 * 4 * 2;
 
 __host__ __device__ inline uint64_t pad16(uint64_t b) { return (b + 15) & ~uint64_t(15); }
