@@ -378,6 +378,10 @@ def run_ours(args, world, rank, local):
         def build_rows():
             rb.check(rb.rans_build_cdfs_from_scales(scales, tail, cdfs, lengths, offsets,
                                                     precision=prec), "cdfs")
+
+        def rebuild_tables():  # the rows and the prepared tables in one launch
+            rb.check(rb.rans_tables_refresh_from_scales(scales, tail, cdfs, lengths, offsets,
+                                                        tables), "tables")
     else:
         pmfs = torch.from_numpy(np.ascontiguousarray(w["pmfs"])).to(dev)
         plen = torch.from_numpy(np.asarray(w["pmf_lengths"], np.int32)).to(dev)
@@ -388,6 +392,10 @@ def run_ours(args, world, rank, local):
         def build_rows():
             rb.check(rb.rans_build_cdfs_from_pmfs(pmfs, plen, ptail, cdfs, lengths,
                                                   precision=prec), "cdfs")
+
+        def rebuild_tables():
+            build_rows()
+            rb.check(rb.rans_tables_refresh(cdfs, lengths, offsets, tables), "refresh")
     K, Lmax = cdfs.shape
     tables = rb.Tables(cdfs, lengths, offsets, precision=prec)
     if w["alias"]:  # built once, before timing: the rows do not change between steps
@@ -405,8 +413,7 @@ def run_ours(args, world, rank, local):
     ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
 
     def phase_tables():
-        build_rows()
-        rb.check(rb.rans_tables_refresh(cdfs, lengths, offsets, tables), "refresh")
+        rebuild_tables()
 
     def phase_encode():
         rb.check(rb.rans_encode_with_indexes(sym, idx, n, tables, ch, ws.out, ws.offsets,
@@ -679,8 +686,8 @@ def run_float(args, world, rank, local):
 
     def step(e=None):
         if e: e[0].record(stream)
-        rb.check(rb.rans_build_cdfs_from_scales(table, tail, cdfs, lengths, offsets), "cdfs")
-        rb.check(rb.rans_tables_refresh(cdfs, lengths, offsets, tables), "refresh")
+        rb.check(rb.rans_tables_refresh_from_scales(table, tail, cdfs, lengths, offsets, tables),
+                 "tables")
         if e: e[1].record(stream)
         rb.check(rb.rans_encode_from_scales(y, mu, sc, n, table, bound, tables, ch, ws.out,
                                             ws.offsets, ws.enc), "encode")

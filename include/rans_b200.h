@@ -276,6 +276,23 @@ int rans_tables_refresh(const int32_t *cdfs, int32_t K, int32_t Lmax,
                         const int32_t *cdf_lengths, const int32_t *offsets,
                         const rans_tables *tables, void *stream);
 
+/*
+ * rans_build_cdfs_from_scales (at the table set's precision) and
+ * rans_tables_refresh from those rows, in one kernel launch: one CTA per row
+ * quantises the row and rewrites its offset, packed buckets and lookup slots
+ * from it.  Same outputs as the two calls: cdfs, cdf_lengths and offsets as
+ * rans_build_cdfs_from_scales writes them, the table set as
+ * rans_tables_refresh leaves it.  A row that cannot be built, or whose
+ * length differs from the prepared layout, records RANS_ERR_TABLE in the
+ * blob's status word (and its negative status as its length).  Asynchronous.
+ *   scales: device float[K]; cdfs: device int32[K][Lmax] out;
+ *   cdf_lengths, offsets: device int32[K] out;
+ *   tables: prepared for the same K from Gaussian rows of the same lengths.
+ */
+int rans_tables_refresh_from_scales(const float *scales, int32_t K, double tail_mass,
+                                    int32_t *cdfs, int32_t Lmax, int32_t *cdf_lengths,
+                                    int32_t *offsets, const rans_tables *tables, void *stream);
+
 /* Bytes of the alias tables of a prepared table set: 8 bytes per bucket
  * (slot words) and 2^precision 16-bit remap entries per row. */
 uint64_t rans_alias_bytes(const rans_tables *tables);

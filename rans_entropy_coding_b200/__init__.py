@@ -16,5 +16,6 @@ from ._lib import (  # noqa: F401
     rans_decode_workspace_bytes, rans_encode_with_indexes, rans_encode_with_indexes_noalloc,
     rans_encode_workspace_bytes,
     rans_gaussian_lengths, rans_get_status, rans_max_compressed_bytes, rans_num_streams,
-    rans_tables, rans_tables_bytes, rans_tables_prepare, rans_tables_refresh)
+    rans_tables, rans_tables_bytes, rans_tables_prepare, rans_tables_refresh,
+    rans_tables_refresh_from_scales)
 from .interface import RansCoder, from_byte_strings, to_byte_strings  # noqa: F401,E402

@@ -77,6 +77,8 @@ SIGNATURES = [
     ("rans_tables_bytes", _U64, [_I32, _I32]),
     ("rans_tables_prepare", ctypes.c_int, [_P, _I32, _I32, _P, _P, _I32, _P, _U64, _TBP, _P]),
     ("rans_tables_refresh", ctypes.c_int, [_P, _I32, _I32, _P, _P, _TBP, _P]),
+    ("rans_tables_refresh_from_scales", ctypes.c_int,
+     [_P, _I32, _F64, _P, _I32, _P, _P, _TBP, _P]),
     ("rans_alias_bytes", _U64, [_TBP]),
     ("rans_alias_prepare", ctypes.c_int, [_P, _I32, _I32, _P, _TBP, _P, _U64, _P]),
     ("rans_num_streams", _I64, [_CHP, _I64]),
@@ -185,6 +187,15 @@ def rans_tables_refresh(cdfs, cdf_lengths, offsets, tables, stream=None):
     _need_cuda(cdfs, cdf_lengths, offsets)
     return lib().rans_tables_refresh(_ptr(cdfs), cdfs.shape[0], cdfs.shape[1], _ptr(cdf_lengths),
                                      _ptr(offsets), ctypes.byref(tables.c), _stream(stream))
+
+
+def rans_tables_refresh_from_scales(scales, tail_mass, cdfs, cdf_lengths, offsets, tables,
+                                    stream=None):
+    _need_cuda(scales, cdfs, cdf_lengths, offsets)
+    return lib().rans_tables_refresh_from_scales(_ptr(scales), scales.numel(), tail_mass,
+                                                 _ptr(cdfs), cdfs.shape[1], _ptr(cdf_lengths),
+                                                 _ptr(offsets), ctypes.byref(tables.c),
+                                                 _stream(stream))
 
 
 def rans_alias_bytes(tables):

@@ -312,6 +312,19 @@ RANS_API int rans_tables_refresh(const int32_t *cdfs, int32_t K, int32_t Lmax,
   return rb::refresh_tables(cdfs, K, Lmax, cdf_lengths, offsets, *tables, as_stream(stream));
 }
 
+RANS_API int rans_tables_refresh_from_scales(const float *scales, int32_t K, double tail_mass,
+                                             int32_t *cdfs, int32_t Lmax, int32_t *cdf_lengths,
+                                             int32_t *offsets, const rans_tables *tables,
+                                             void *stream) {
+  NvtxRange nvtx_("rans_tables_refresh_from_scales");
+  if (!tables_usable(tables) || K != tables->K || Lmax < 3 || !scales || !cdfs ||
+      !cdf_lengths || !offsets)
+    return RANS_ERR_ARG;
+  if (!(tail_mass > 0.0) || !(tail_mass < 1.0)) return RANS_ERR_ARG;
+  return rb::refresh_tables_from_scales(scales, K, tail_mass, cdfs, Lmax, cdf_lengths, offsets,
+                                        *tables, as_stream(stream));
+}
+
 RANS_API uint64_t rans_alias_bytes(const rans_tables *tables) {
   if (!tables || tables->K < 1 || tables->precision < 1 || tables->precision > 16) return 0;
   return ((8ull * (uint64_t)tables->n_buckets + 255) & ~255ull) +

@@ -25,6 +25,11 @@ int prepare_alias(const int32_t *cdfs, int K, int Lmax, const int32_t *lengths,
                   rans_tables &t, void *alias, uint64_t alias_bytes, cudaStream_t st);
 int refresh_tables(const int32_t *cdfs, int K, int Lmax, const int32_t *lengths,
                    const int32_t *offsets, const rans_tables &t, cudaStream_t st);
+// Gaussian rows (precision t.precision) into cdfs, lengths and offsets, and
+// the prepared table set t rebuilt from them, in one launch.
+int refresh_tables_from_scales(const float *scales, int K, double tail, int32_t *cdfs, int Lmax,
+                               int32_t *lengths, int32_t *offsets, const rans_tables &t,
+                               cudaStream_t st);
 // Rows summing to 2^prec, stored scaled to 16 bits.
 int prepare_tables(const int32_t *cdfs, int K, int Lmax, const int32_t *lengths,
                    const int32_t *offsets, int prec, void *blob, uint64_t blob_bytes,

@@ -104,6 +104,19 @@ struct QuantScratch {
   unsigned int nbig;
 };
 
+// floor(a / T) for T >= 1 and a / T < 2^32 (a = total * c with c <= T):
+// the double product a * (1 / T) is within one of the quotient (its
+// relative error is a few units of 2^-53 and the quotient is below 2^32),
+// and one exact integer step corrects it.
+__device__ __forceinline__ unsigned long long div_floor(unsigned long long a,
+                                                        unsigned long long T, double rT) {
+  unsigned long long q = (unsigned long long)((double)a * rT);
+  const long long r = (long long)(a - q * T);
+  if (r < 0) --q;
+  else if ((unsigned long long)r >= T) ++q;
+  return q;
+}
+
 template <class PF>
 __device__ int quantise_row(const PF &pf, int n, int32_t *row, BlockScratch &sh,
                             QuantScratch &q, uint32_t total) {
@@ -123,11 +136,12 @@ __device__ int quantise_row(const PF &pf, int n, int32_t *row, BlockScratch &sh,
   // empty buckets and the widths of the others
   unsigned long long zl = 0;
   {
+    const double rT = 1.0 / (double)T;
     unsigned long long c = before;
-    unsigned long long b0 = ((unsigned long long)total * c) / T;
+    unsigned long long b0 = div_floor((unsigned long long)total * c, T, rT);
     for (int i = i0; i < i1; ++i) {
       c += (uint32_t)row[i + 1];
-      const unsigned long long b1 = ((unsigned long long)total * c) / T;
+      const unsigned long long b1 = div_floor((unsigned long long)total * c, T, rT);
       const uint32_t w = (uint32_t)(b1 - b0);
       b0 = b1;
       row[i + 1] = (int32_t)w;
@@ -511,6 +525,24 @@ __device__ void fill_row_slots(const int32_t *grow, int nb, uint32_t slot0, int 
     fill_slot_block(row, nb, slot0, w, nslots, tb, slots, ca, sh);
 }
 
+// Row r's packed buckets and 16-bit starts from its len entries (row[0] = 0
+// and row[len - 1] << sh = 65536 checked by the caller); a bucket that is
+// not strictly increasing or out of range records RANS_ERR_TABLE.
+__device__ __forceinline__ void pack_row(const int32_t *row, int len, uint32_t base,
+                                         uint32_t sh, uint32_t *buckets, uint16_t *starts,
+                                         int32_t *status, int r) {
+  const int32_t top = (int32_t)(kTotal >> sh);
+  for (int j = threadIdx.x; j < len - 1; j += blockDim.x) {
+    const int32_t a = row[j], b = row[j + 1];
+    if (!(b > a) || a < 0 || b > top) {
+      report(status, RANS_ERR_TABLE, r);
+      continue;
+    }
+    buckets[base + j] = bucket_word(a, b, sh);
+  }
+  for (int j = threadIdx.x; j < len; j += blockDim.x) starts[base + j] = (uint16_t)(row[j] << sh);
+}
+
 // Rebuilds a prepared table set from new CDF rows with the same lengths:
 // block (x, r) fills slot block x of row r; block (0, r) also checks the
 // row's length against the layout, refreshes its offset and packs its
@@ -541,16 +573,7 @@ __global__ void __launch_bounds__(kSlotThreads)
       prow = srow;
     }
     if (threadIdx.x < kMetaCopies) meta[r * kMetaCopies + threadIdx.x].offset = offsets[r];
-    for (int j = threadIdx.x; j < nb; j += blockDim.x) {
-      const int32_t a = prow[j], b = prow[j + 1];
-      if (!(b > a) || a < 0 || b > top) {
-        report(status, RANS_ERR_TABLE, r);
-        continue;
-      }
-      buckets[m.bucket_base + j] = bucket_word(a, b, sh);
-    }
-    for (int j = threadIdx.x; j < len; j += blockDim.x)
-      starts[m.bucket_base + j] = (uint16_t)(prow[j] << sh);
+    pack_row(prow, len, m.bucket_base, sh, buckets, starts, status, r);
     __syncthreads();  // the staged row is staged again below
   }
   fill_row_slots(row, nb, slot_base(m.slot), (int)slot_shift(m.slot), slots, ca, srow, sh);
@@ -568,6 +591,54 @@ __global__ void __launch_bounds__(kSlotThreads)
   const int len = lengths[r];
   if (len < 2 || row[0] != 0 || row[len - 1] != (int32_t)(kTotal >> sh)) return;
   fill_row_slots(row, len - 1, slot_base(m.slot), (int)slot_shift(m.slot), slots, ca, srow, sh);
+}
+
+// rans_build_cdfs_from_scales and rans_tables_refresh in one launch: block r
+// quantises Gaussian row r as gaussian_rows_kernel does, then rewrites the
+// row's offset, packed buckets, starts and every lookup slot of the row as
+// refresh_kernel does, from the row it has just written (staged in shared
+// memory).  A row that cannot be built, or whose length differs from the
+// prepared layout, records RANS_ERR_TABLE in the blob's status word.
+__global__ void __launch_bounds__(kRowThreads)
+    gaussian_refresh_kernel(const float *scales, double tail, int prec, int32_t *cdfs, int Lmax,
+                            int32_t *lengths, int32_t *offsets, RowMeta *meta, uint32_t *buckets,
+                            uint16_t *starts, uint32_t *slots, ChunkArea ca, int32_t *status) {
+  extern __shared__ int32_t srow[];
+  __shared__ BlockScratch sh;
+  __shared__ QuantScratch qs;
+  const int r = blockIdx.x;
+  int32_t *row = cdfs + (size_t)r * (size_t)Lmax;
+  int32_t c = 0;
+  int st = gaussian_center(scales[r], tail, &c);
+  const int len = 2 * c + 3;
+  if (st == RANS_OK && len > Lmax) st = RANS_ERR_CAPACITY;
+  if (st == RANS_OK) {
+    GaussPmf pf{c, 2 * c + 1, (double)scales[r], 1u << prec};
+    st = quantise_row(pf, 2 * c + 2, row, sh, qs, 1u << prec);
+  }
+  for (int j = (st == RANS_OK ? len : 0) + threadIdx.x; j < Lmax; j += kRowThreads) row[j] = 0;
+  if (threadIdx.x == 0) {
+    lengths[r] = st ? st : len;
+    offsets[r] = st ? 0 : -c;
+  }
+  // (st is the same on every thread)
+  const RowMeta m = meta[r * kMetaCopies];
+  if (st != RANS_OK || len != (int)m.maxv + 2) {
+    if (threadIdx.x == 0) report(status, RANS_ERR_TABLE, r);
+    return;
+  }
+  const uint32_t ssh = (uint32_t)(kPrec - prec);
+  const int32_t *prow = row;  // (quantise_row ends on a barrier: the row is written)
+  if (len <= kRowSmem) {
+    stage_row(srow, row, len);
+    prow = srow;
+  }
+  if (threadIdx.x < kMetaCopies) meta[r * kMetaCopies + threadIdx.x].offset = -c;
+  pack_row(prow, len, m.bucket_base, ssh, buckets, starts, status, r);
+  const int shift = (int)slot_shift(m.slot);
+  const int nslots = 1 << (16 - shift);
+  for (int tb = 0; tb < nslots; tb += kRowThreads * kSlotsPerThread)
+    fill_slot_block(prow, len - 1, slot_base(m.slot), 1 << shift, nslots, tb, slots, ca, ssh);
 }
 
 // Alias tables, one row per block (the reading of the alias method given
@@ -726,6 +797,30 @@ int refresh_tables(const int32_t *cdfs, int K, int Lmax, const int32_t *lengths,
   refresh_kernel<<<grid, kSlotThreads, kSlotSmemBytes, st>>>(
       cdfs, Lmax, lengths, offsets, (uint32_t)(kPrec - t.precision), dmeta, dbuckets, dstarts,
       dslots, ca, status);
+  return cudaGetLastError() == cudaSuccess ? RANS_OK : RANS_ERR_CUDA;
+}
+
+int refresh_tables_from_scales(const float *scales, int K, double tail, int32_t *cdfs, int Lmax,
+                               int32_t *lengths, int32_t *offsets, const rans_tables &t,
+                               cudaStream_t st) {
+  if (K != t.K) return RANS_ERR_ARG;
+  char *b = reinterpret_cast<char *>(t.blob);
+  int32_t *status = reinterpret_cast<int32_t *>(b);
+  RowMeta *dmeta = reinterpret_cast<RowMeta *>(b + kHeaderBytes);
+  uint32_t *dbuckets = reinterpret_cast<uint32_t *>(b + kHeaderBytes + t.meta_bytes);
+  uint16_t *dstarts =
+      reinterpret_cast<uint16_t *>(b + kHeaderBytes + t.meta_bytes + t.bucket_bytes);
+  uint32_t *dslots = reinterpret_cast<uint32_t *>(b + kHeaderBytes + t.meta_bytes +
+                                                  t.bucket_bytes + t.start_bytes);
+  ChunkArea ca;
+  ca.base = (uint32_t)t.n_slots;
+  ca.cap = t.slot_bytes / 4 - (uint32_t)t.n_slots;
+  ca.used = reinterpret_cast<uint32_t *>(b) + kChunkUsedWord;
+  ca.search = reinterpret_cast<uint32_t *>(b) + kSearchFlagWord;
+  if (cudaMemsetAsync(ca.used, 0, 8, st) != cudaSuccess) return RANS_ERR_CUDA;
+  gaussian_refresh_kernel<<<K, kRowThreads, kSlotSmemBytes, st>>>(
+      scales, tail, t.precision, cdfs, Lmax, lengths, offsets, dmeta, dbuckets, dstarts, dslots,
+      ca, status);
   return cudaGetLastError() == cudaSuccess ? RANS_OK : RANS_ERR_CUDA;
 }
 

@@ -568,3 +568,41 @@ def test_tile_staged_decoder_shapes(shape, cg, th, tw, fmt):
              chunking=dict(kind="tiled", shape=shape, cg=cg, th=th, tw=tw), W=32, fmt=fmt,
              precision=16 if fmt == "rans64" else 15)
     _check_streams(w)
+
+
+def test_fused_gaussian_refresh_matches_oracle_rows():
+    """rans_tables_refresh_from_scales: the Gaussian rows, lengths and offsets
+    of a nudged scale table equal the oracle's, and the refreshed table set
+    codes exactly like the oracle on those rows; a scale whose row changes
+    length is refused on the device."""
+    w = WL.y_latent(W=32)
+    scales = np.asarray(w["scales"], np.float32)
+    tail = w["tail_mass"]
+    c, l, o = O.build_cdfs_from_scales(scales, tail)
+    tables = tables_from_numpy(c, l, o)
+    # every scale nudged up where its row keeps its length
+    s2 = (scales * np.float32(1.0005)).astype(np.float32)
+    c2, l2, o2 = O.build_cdfs_from_scales(s2, tail)
+    keep = l2 != l
+    s2[keep] = scales[keep]
+    c2, l2, o2 = O.build_cdfs_from_scales(s2, tail)
+    assert np.array_equal(l2, l) and not np.array_equal(c2, c)
+    K, Lmax = c.shape
+    dcd = torch.full((K, Lmax), -7, dtype=torch.int32, device="cuda")
+    dl = torch.zeros(K, dtype=torch.int32, device="cuda")
+    do = torch.zeros(K, dtype=torch.int32, device="cuda")
+    rb.check(rb.rans_tables_refresh_from_scales(torch.from_numpy(s2).cuda(), tail, dcd, dl, do,
+                                                tables))
+    assert rb.rans_get_status(tables.blob) == rb.OK
+    assert np.array_equal(dcd.cpu().numpy(), c2)
+    assert np.array_equal(dl.cpu().numpy(), l2) and np.array_equal(do.cpu().numpy(), o2)
+    data, offs, dec, _, _ = gpu_encode_decode(w, tables)
+    want, woffs = oracle_encode(w, c2, l2, o2)
+    assert offs.tolist() == woffs.tolist() and np.array_equal(data, want)
+    assert np.array_equal(dec, np.asarray(w["symbols"]).reshape(-1))
+    # a row whose length changes
+    s3 = s2.copy()
+    s3[5] *= np.float32(2.0)
+    rb.check(rb.rans_tables_refresh_from_scales(torch.from_numpy(s3).cuda(), tail, dcd, dl, do,
+                                                tables))
+    assert rb.rans_get_status(tables.blob) == rb.ERR_TABLE
