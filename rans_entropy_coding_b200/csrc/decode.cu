@@ -1185,23 +1185,31 @@ __device__ __forceinline__ void tile_origin(const Geom &g, const StreamDesc &d, 
 // One group: lookup, state update and refill, no branch; a lane whose
 // symbol is the escape bucket only sets `esc`.  win: the stream's word
 // ring (word i at win[i mod kWinWords]), rd: the next word to read.
+// SEARCH: a table with slots that ran out of bitmap room; those slots take
+// the general lookup's binary search (a branch, entered once per warp).
+template <bool SEARCH>
 __device__ __forceinline__ int32_t dec_group_win64(uint64_t &x, uint32_t &rd, const RowMeta &m,
                                                    const uint16_t *starts, const uint32_t *slots,
                                                    const uint32_t *win, uint32_t &esc) {
   const uint32_t xl = (uint32_t)x, xh = (uint32_t)(x >> 32);
   const uint32_t cum = xl & 0xffffu;
-  const uint32_t sh = m.slot >> 27;
-  const uint32_t i1 = (m.slot & 0x07ffffffu) + (cum >> sh);
-  const uint32_t se = slots[i1];
-  const uint32_t c = cum & ((1u << sh) - 1u);
-  const uint32_t lo = se & 0xffffu;
-  const uint32_t e1 = __byte_perm(se, 0u, 0x4442u), e2 = se >> 24;
-  uint32_t sym = lo + (c > e1 ? 1u : 0u) + (c > e2 ? 1u : 0u);
-  const bool bm = e1 == 0xffu && e2 != 0xffu;
-  const uint32_t i2 = bm ? (lo | ((se >> 8) & 0xff0000u)) + (c >> 4) : i1;
-  const uint32_t ce = slots[i2];
-  const uint32_t sym2 = (ce >> 16) + __popc(ce & ((2u << (c & 15u)) - 1u));
-  sym = min(bm ? sym2 : sym, m.maxv);
+  uint32_t sym;
+  if constexpr (SEARCH) {
+    sym = lookup<true, true>(cum, m, starts, slots, true);
+  } else {
+    const uint32_t sh = m.slot >> 27;
+    const uint32_t i1 = (m.slot & 0x07ffffffu) + (cum >> sh);
+    const uint32_t se = slots[i1];
+    const uint32_t c = cum & ((1u << sh) - 1u);
+    const uint32_t lo = se & 0xffffu;
+    const uint32_t e1 = __byte_perm(se, 0u, 0x4442u), e2 = se >> 24;
+    sym = lo + (c > e1 ? 1u : 0u) + (c > e2 ? 1u : 0u);
+    const bool bm = e1 == 0xffu && e2 != 0xffu;
+    const uint32_t i2 = bm ? (lo | ((se >> 8) & 0xff0000u)) + (c >> 4) : i1;
+    const uint32_t ce = slots[i2];
+    const uint32_t sym2 = (ce >> 16) + __popc(ce & ((2u << (c & 15u)) - 1u));
+    sym = min(bm ? sym2 : sym, m.maxv);
+  }
   esc |= sym == m.maxv ? 1u : 0u;
   const uint32_t a = m.bucket_base + sym;
   const uint32_t s0 = starts[a], s1 = starts[a + 1];
@@ -1235,14 +1243,22 @@ __device__ __forceinline__ void win_refill(uint32_t *win, const uint32_t *words,
 }
 
 // Stream s (64-bit format, tile width 56 or 64: GC = 7 or 8 groups a chunk,
-// fewer than 2^31 words) on the unrolled path.
-template <int GC>
+// fewer than 2^31 words) on the unrolled path.  FLT: float latents: the
+// index tile holds the scales (each group's row is its scale's table row,
+// from the scale table `stab` in shared memory) and the output tile the
+// values float(symbol) + mean, the means read from global memory at the
+// chunk's start (0 without means).
+// FM: 0 int32 rows, 1 float latents with the scale table searched, 2 float
+// latents with its rows read through `keys`.
+template <int GC, int FM, bool SEARCH>
 __device__ __forceinline__ bool decode_tile_win64(const DecCtx &c, const TileMaps &maps,
                                                   const RowMeta *meta, const uint16_t *starts,
                                                   const uint32_t *slots, uint32_t ring,
                                                   int32_t *ring_p, uint32_t bar0, uint32_t &par,
                                                   int64_t s, const StreamDesc &d,
-                                                  const uint32_t *words, uint32_t nw) {
+                                                  const uint32_t *words, uint32_t nw,
+                                                  const float *stab, const ScaleKeys &keys) {
+  constexpr bool FLT = FM != 0;
   constexpr int kHalfW = (int)(kTileRingHalf / 4);
   constexpr uint32_t cbytes = 128u * GC;
   const int lane = threadIdx.x & 31;
@@ -1282,9 +1298,25 @@ __device__ __forceinline__ bool decode_tile_win64(const DecCtx &c, const TileMap
   uint32_t rd = 64, ldn = 64, rmax = 0;
   bool bad = false;
   auto meta_of = [&](uint32_t r) -> RowMeta {
+    if (FM == 1) r = scale_row(bound_scale(__uint_as_float(r), c.bound), stab, c.K);
+    if (FM == 2) r = keys.row(bound_scale(__uint_as_float(r), c.bound));
     rmax = max(rmax, r);
     return row_meta(meta, min(r, kmax));
   };
+  // FLT: a decoded value out (float(v) + mean as its bits), else v
+  auto out_of = [&](int32_t v, float mean) -> int32_t {
+    return FLT ? __float_as_int((float)v + mean) : v;
+  };
+  // FLT: group j's lane reads the mean of element e = 32 j + lane of the
+  // chunk, row e / ww, column e mod ww
+  int32_t moff[GC];
+  if (FLT) {
+#pragma unroll
+    for (int j = 0; j < GC; ++j) {
+      const int e = j * 32 + lane, r = e / (8 * GC);
+      moff[j] = r * (int32_t)g.Wd + (e - r * 8 * GC);
+    }
+  }
   // a bounded wait for the chunk in half h; on giving up, a bounded wait for
   // every load still in flight, and the warp stops
   auto wait_half = [&](int h) -> bool {
@@ -1318,10 +1350,20 @@ __device__ __forceinline__ bool decode_tile_win64(const DecCtx &c, const TileMap
     const uint32_t rds = rd;
     uint32_t esc = 0;
     int32_t val[GC];
+    float mu[GC];
+    if (FLT) {
+#pragma unroll
+      for (int j = 0; j < GC; ++j) mu[j] = 0.0f;
+      if (c.fmean) {
+        const float *mp = c.fmean + (((int64_t)sd.z * g.H + sd.y) * g.Wd + x0);
+#pragma unroll
+        for (int j = 0; j < GC; ++j) mu[j] = __ldg(mp + moff[j]);
+      }
+    }
 #pragma unroll
     for (int j = 0; j < GC; ++j) {
       const RowMeta m = meta_of((uint32_t)rh[j * 32 + lane]);
-      val[j] = dec_group_win64(x, rd, m, starts, slots, win, esc);
+      val[j] = dec_group_win64<SEARCH>(x, rd, m, starts, slots, win, esc);
       if (j == 0) {
         // chunk k + 3 into L2; chunk k + 1 into the other half, once chunk
         // k - 1's store has read it
@@ -1340,7 +1382,7 @@ __device__ __forceinline__ bool decode_tile_win64(const DecCtx &c, const TileMap
     }
     if (!__any_sync(kFull, esc != 0)) {
 #pragma unroll
-      for (int j = 0; j < GC; ++j) rh[j * 32 + lane] = val[j];
+      for (int j = 0; j < GC; ++j) rh[j * 32 + lane] = out_of(val[j], FLT ? mu[j] : 0.0f);
     } else {
       // an escape in this chunk: decode it again from its saved state on
       // the lane-serial path (its row indexes are still in the ring), then
@@ -1355,8 +1397,14 @@ __device__ __forceinline__ bool decode_tile_win64(const DecCtx &c, const TileMap
 #pragma unroll 1
       for (int j = 0; j < GC; ++j) {
         const RowMeta mj = meta_of((uint32_t)rh[j * 32 + lane]);
-        rh[j * 32 + lane] =
-            dec_group_val<Rans64, false>(w, mj, starts, slots, words, nw, Rans64::shift(c.sh));
+        float mean = 0.0f;
+        if (FLT) {
+#pragma unroll
+          for (int q = 0; q < GC; ++q) mean = q == j ? mu[q] : mean;
+        }
+        rh[j * 32 + lane] = out_of(
+            dec_group_val<Rans64, SEARCH>(w, mj, starts, slots, words, nw, Rans64::shift(c.sh)),
+            mean);
       }
       bad = bad || w.bad;
       x = w.x;
@@ -1385,26 +1433,57 @@ __device__ __forceinline__ bool decode_tile_win64(const DecCtx &c, const TileMap
 // widths 64 and 56 (8 and 7 groups) when its words are well formed and
 // fewer than 2^31 (32-bit word cursors), the general loop otherwise or when
 // the table has slots that search.
-template <class F>
+// FLT (float latents, 64-bit format): the unrolled path only (with the
+// searching lookup when the table has slots that search); the host takes the
+// tile kernel for them only when every tile is 64 or 56 wide, and a stream
+// that is not well formed is reported here.
+template <class F, bool FLT>
 __device__ __forceinline__ bool decode_tile_one(const DecCtx &c, const TileMaps &maps,
                                                 const RowMeta *meta, const uint16_t *starts,
                                                 const uint32_t *slots, uint32_t ring,
                                                 int32_t *ring_p, uint32_t bar0, uint32_t &par,
-                                                int64_t s, bool search) {
-  if (search)
-    return decode_tile_stream<F, true>(c, maps, meta, starts, slots, ring, ring_p, bar0, par, s);
+                                                int64_t s, bool search, const float *stab,
+                                                const ScaleKeys &keys, bool use_keys) {
+  const int lane = threadIdx.x & 31;
+  if constexpr (!FLT) {
+    if (search)
+      return decode_tile_stream<F, true>(c, maps, meta, starts, slots, ring, ring_p, bar0, par,
+                                         s);
+  }
   const StreamDesc d = stream_desc(c.g, s);
   const typename F::Word *words = nullptr;
   uint64_t nw = 0;
   const bool fast = d.ok && (d.t.ww == 64 || d.t.ww == 56) &&
                     stream_bounds<F>(c, s, 32, words, nw) && nw < (uint64_t(1) << 31);
+  if constexpr (FLT) {
+    if (!fast) {
+      if (lane == 0) report(c.status, d.ok ? RANS_ERR_CORRUPT : RANS_ERR_ARG, s);
+      return true;
+    }
+  }
   if (fast) {
     if constexpr (std::is_same<F, Rans64>::value) {
-      if (d.t.ww == 64)
-        return decode_tile_win64<8>(c, maps, meta, starts, slots, ring, ring_p, bar0, par, s, d,
-                                    words, (uint32_t)nw);
-      return decode_tile_win64<7>(c, maps, meta, starts, slots, ring, ring_p, bar0, par, s, d,
-                                  words, (uint32_t)nw);
+      const uint32_t n32 = (uint32_t)nw;
+      if constexpr (FLT) {
+        const bool w64 = d.t.ww == 64;
+        if (search && use_keys)
+          return w64 ? decode_tile_win64<8, 2, true>(c, maps, meta, starts, slots, ring, ring_p, bar0, par, s, d, words, n32, stab, keys)
+                     : decode_tile_win64<7, 2, true>(c, maps, meta, starts, slots, ring, ring_p, bar0, par, s, d, words, n32, stab, keys);
+        if (search)
+          return w64 ? decode_tile_win64<8, 1, true>(c, maps, meta, starts, slots, ring, ring_p, bar0, par, s, d, words, n32, stab, keys)
+                     : decode_tile_win64<7, 1, true>(c, maps, meta, starts, slots, ring, ring_p, bar0, par, s, d, words, n32, stab, keys);
+        if (use_keys)
+          return w64 ? decode_tile_win64<8, 2, false>(c, maps, meta, starts, slots, ring, ring_p, bar0, par, s, d, words, n32, stab, keys)
+                     : decode_tile_win64<7, 2, false>(c, maps, meta, starts, slots, ring, ring_p, bar0, par, s, d, words, n32, stab, keys);
+        return w64 ? decode_tile_win64<8, 1, false>(c, maps, meta, starts, slots, ring, ring_p, bar0, par, s, d, words, n32, stab, keys)
+                   : decode_tile_win64<7, 1, false>(c, maps, meta, starts, slots, ring, ring_p, bar0, par, s, d, words, n32, stab, keys);
+      } else {
+        if (d.t.ww == 64)
+          return decode_tile_win64<8, 0, false>(c, maps, meta, starts, slots, ring, ring_p, bar0,
+                                                par, s, d, words, n32, stab, keys);
+        return decode_tile_win64<7, 0, false>(c, maps, meta, starts, slots, ring, ring_p, bar0,
+                                              par, s, d, words, n32, stab, keys);
+      }
     } else {
       if (d.t.ww == 64)
         return decode_tile_stream_fast<F, 8>(c, maps, meta, starts, slots, ring, ring_p, bar0,
@@ -1413,12 +1492,14 @@ __device__ __forceinline__ bool decode_tile_one(const DecCtx &c, const TileMaps 
                                            s);
     }
   }
-  return decode_tile_stream<F, false>(c, maps, meta, starts, slots, ring, ring_p, bar0, par, s);
+  if constexpr (!FLT)
+    return decode_tile_stream<F, false>(c, maps, meta, starts, slots, ring, ring_p, bar0, par, s);
+  return true;
 }
 
 // The tile-staged decoder: one stream per warp at a time, in scheduling
-// order (largest tiles first).
-template <class F>
+// order (largest tiles first).  FLT: float latents (scales in, values out).
+template <class F, bool FLT>
 __global__ void __launch_bounds__(kTileMaxStreams * 32, 1)
     decode_tile_kernel(DecCtx c, const __grid_constant__ TileMaps maps) {
   extern __shared__ __align__(16) unsigned char smem[];
@@ -1439,6 +1520,18 @@ __global__ void __launch_bounds__(kTileMaxStreams * 32, 1)
   const uint32_t ring = ((sbase + tab + 127u) & ~127u) + (uint32_t)warp * kTileStreamBytes;
   int32_t *ring_p = reinterpret_cast<int32_t *>(smem + (ring - sbase));
   const uint32_t bar0 = smem_addr(&ring_bar[warp][0]);
+  // FLT: the scale table after every warp's ring, then its key counts
+  float *stab = nullptr;
+  ScaleKeys keys{};
+  bool use_keys = false;
+  if (FLT) {
+    stab = reinterpret_cast<float *>(smem + (((sbase + tab + 127u) & ~127u) - sbase) +
+                                     (uint32_t)nwarp * kTileStreamBytes);
+    for (int i = threadIdx.x; i < c.K; i += blockDim.x) stab[i] = c.stab[i];
+    __syncthreads();
+    use_keys = build_scale_keys(stab, c.K, reinterpret_cast<uint8_t *>(stab) + pad16(4ull * c.K),
+                                keys);
+  }
   if (lane == 0) {
     tma::mbar_init(bar0, 1);
     tma::mbar_init(bar0 + 8, 1);
@@ -1450,8 +1543,8 @@ __global__ void __launch_bounds__(kTileMaxStreams * 32, 1)
   const bool search = reinterpret_cast<const uint32_t *>(c.blob)[kSearchFlagWord] != 0;
   for (int64_t k = blockIdx.x + (int64_t)gridDim.x * warp; k < c.g.S;
        k += (int64_t)gridDim.x * nwarp) {
-    if (!decode_tile_one<F>(c, maps, meta, starts, slots, ring, ring_p, bar0, par,
-                            stream_of(c.g, k), search))
+    if (!decode_tile_one<F, FLT>(c, maps, meta, starts, slots, ring, ring_p, bar0, par,
+                                 stream_of(c.g, k), search, stab, keys, use_keys))
       break;
   }
   if (lane == 0) tma::bulk_wait_all();
@@ -1481,14 +1574,16 @@ bool tile_path_ok(const DecCtx &c, int mode, int sym_dtype, const void *indexes,
 // not fit in shared memory (the caller then takes the general kernel).
 constexpr int kNotTaken = 1;
 
-template <class F>
-int launch_decode_tile(const DecCtx &c, const int32_t *indexes, void *symbols, cudaStream_t st) {
+template <class F, bool FLT = false>
+int launch_decode_tile(const DecCtx &c, const void *indexes, void *symbols, cudaStream_t st) {
   const Geom &g = c.g;
   int dev = 0;
   cudaGetDevice(&dev);
   const uint32_t tab = dec_table_bytes(1, c);
+  const uint32_t stab_bytes =
+      FLT ? (uint32_t)pad16(4ull * (uint64_t)c.K) + kScaleKeyBytes : 0u;
   const int optin = smem_optin(dev);
-  const uint32_t lim = (uint32_t)optin - 64u - 2u * 8u * kTileMaxStreams;
+  const uint32_t lim = (uint32_t)optin - 64u - 2u * 8u * kTileMaxStreams - stab_bytes;
   if (tab + 128u + kTileStreamBytes > lim) return kNotTaken;
   TileMaps maps;
   const int64_t per_img = g.ng * g.nty * g.ntx;
@@ -1507,8 +1602,8 @@ int launch_decode_tile(const DecCtx &c, const int32_t *indexes, void *symbols, c
   const int64_t room = ((int64_t)lim - tab - 128) / kTileStreamBytes;
   if (warps > room) warps = room;
   if (warps < 1) warps = 1;
-  const uint32_t smem = tab + 128u + (uint32_t)warps * kTileStreamBytes;
-  auto kern = decode_tile_kernel<F>;
+  const uint32_t smem = tab + 128u + (uint32_t)warps * kTileStreamBytes + stab_bytes;
+  auto kern = decode_tile_kernel<F, FLT>;
   if (ensure_dyn_smem((const void *)kern, smem) != cudaSuccess) return RANS_ERR_CUDA;
   int fit = 0;
   if (blocks_per_sm(&fit, (const void *)kern, (int)warps * 32, smem) != cudaSuccess || fit < 1)
@@ -1747,7 +1842,13 @@ int launch_decode_float(const uint8_t *in, uint64_t in_bytes, const uint64_t *of
   c.fmean = means;
   c.stab = scale_table;
   c.bound = scale_bound;
-  // float values decode the 64-bit format only (the caller checks)
+  // float values decode the 64-bit format only (the caller checks); tiled
+  // streams of 64- and 56-wide tiles take the tile-staged kernel (scales in
+  // as the index tiles, values out as the symbol tiles)
+  if (t.dec_in_smem == 1 && flt_tile_shape_ok(g, scales, values)) {
+    const int r = launch_decode_tile<Rans64, true>(c, scales, values, st);
+    if (r != kNotTaken) return r;
+  }
   return g.W == 32 ? launch_decode_w<Rans64, 32, float>(c, t.dec_in_smem, st)
                    : launch_decode_w<Rans64, 1, float>(c, t.dec_in_smem, st);
 }

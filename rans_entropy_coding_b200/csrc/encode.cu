@@ -868,12 +868,21 @@ __device__ __forceinline__ bool encode_tile_stream(const EncCtx &c, const EncTil
 // with the escape path; the fast pass before it writes at most one word per
 // lane and group, inside the stream's worst-case scratch slot, and the redo
 // writes every word the stream keeps.
-template <class F, bool ST, int GC>
+// FLT: the tiles hold float latents: the index tile is the scales (each
+// group's row is its scale's table row, from the scale table `stab` in
+// shared memory) and the symbol tile y, coded as rint(y - mean) with the
+// means read from global memory at the chunk's start (an out-of-range value
+// is recorded and coded as 0).
+// FM: 0 int32 rows and symbols, 1 float latents with the scale table
+// searched, 2 float latents with its rows read through `keys`.
+template <class F, bool ST, int GC, int FM>
 __device__ __forceinline__ bool encode_tile_stream_fast(const EncCtx &c, const EncTileMaps &maps,
                                                         const RowMeta *meta,
                                                         const uint32_t *buckets, uint32_t ring,
                                                         const uint32_t *ring_p, uint32_t bar0,
-                                                        uint32_t &par, int64_t s) {
+                                                        uint32_t &par, int64_t s,
+                                                        const float *stab, const ScaleKeys &keys) {
+  constexpr bool FLT = FM != 0;
   using Word = typename F::Word;
   const int lane = threadIdx.x & 31;
   const Geom &g = c.g;
@@ -902,7 +911,9 @@ __device__ __forceinline__ bool encode_tile_stream_fast(const EncCtx &c, const E
   // chunk coordinates stepped back 4 rows at a time from the last chunk: ld
   // for the loads into shared memory, pf for the L2 prefetches
   const int32_t y0 = (int32_t)(ty * g.th), ylast = y0 + hh - 4;
-  int32_t ly = ylast, lz = (int32_t)(b * g.C + gi * g.cg) + (int32_t)(d.n / ((int64_t)hh * d.t.ww)) - 1;
+  const int32_t zlast =
+      (int32_t)(b * g.C + gi * g.cg) + (int32_t)(d.n / ((int64_t)hh * d.t.ww)) - 1;
+  int32_t ly = ylast, lz = zlast;
   int32_t py = ly, pz = lz;
   auto back_if = [&](int32_t &y, int32_t &z, bool on) {
     const int32_t yy = y - 4;
@@ -954,11 +965,50 @@ __device__ __forceinline__ bool encode_tile_stream_fast(const EncCtx &c, const E
   st.rmax = 0;
   st.range_err = false;
   auto meta_of = [&](uint32_t r) -> RowMeta {
+    if (FM == 1) r = scale_row(bound_scale(__uint_as_float(r), c.bound), stab, c.K);
+    if (FM == 2) r = keys.row(bound_scale(__uint_as_float(r), c.bound));
     st.rmax = max(st.rmax, r);
     return row_meta(meta, min(r, kmax));
   };
+  // FLT: the chunk's means (0 without means), read one chunk ahead (my, mz:
+  // the next chunk's position), and the symbol of a staged y.  Group j's
+  // lane reads element e = 32 j + lane of the chunk: row e / ww, column
+  // e mod ww.
+  float mu[GC], mu_n[GC];
+  int32_t moff[GC];
+  int32_t my = ylast, mz = zlast;  // the last chunk's position
+  if (FLT) {
+#pragma unroll
+    for (int j = 0; j < GC; ++j) {
+      const int e = j * 32 + lane, r = e / (8 * GC);
+      moff[j] = r * (int32_t)g.Wd + (e - r * 8 * GC);
+    }
+  }
+  auto load_means = [&](bool on, float (&m)[GC]) {
+#pragma unroll
+    for (int j = 0; j < GC; ++j) m[j] = 0.0f;
+    if (c.fmean && on) {
+      const float *mp = c.fmean + (((int64_t)mz * g.H + my) * g.Wd + x0);
+#pragma unroll
+      for (int j = 0; j < GC; ++j) m[j] = __ldg(mp + moff[j]);
+    }
+    back_if(my, mz, on);
+  };
+  if (FLT) load_means(true, mu_n);
+  auto sym_of = [&](uint32_t v, float mean) -> int32_t {
+    if (!FLT) return (int32_t)v;
+    bool ok;
+    const int32_t q = quantize(__uint_as_float(v), mean, ok);
+    st.range_err |= !ok;
+    return q;
+  };
 #pragma unroll 1
   for (int32_t ch = M - 1; ch >= 0; --ch) {
+    if (FLT) {
+#pragma unroll
+      for (int j = 0; j < GC; ++j) mu[j] = mu_n[j];
+      load_means(ch >= 1, mu_n);
+    }
     if (!wait_chunk(ch)) return false;
     // the chunk before this one into the other half (consumed by the chunk
     // after this one), and the one three before it into L2
@@ -973,7 +1023,7 @@ __device__ __forceinline__ bool encode_tile_stream_fast(const EncCtx &c, const E
 #pragma unroll
     for (int j = GC - 1; j >= 0; --j) {
       const EncBucket bk =
-          enc_bucket<ST>((int32_t)rs[j * 32 + lane], meta_of(ri[j * 32 + lane]), buckets);
+          enc_bucket<ST>(sym_of(rs[j * 32 + lane], mu[j]), meta_of(ri[j * 32 + lane]), buckets);
       esc |= bk.in_range ? 0u : 1u;
       EncLook L;
       L.start = bucket_start(bk.e);
@@ -987,8 +1037,11 @@ __device__ __forceinline__ bool encode_tile_stream_fast(const EncCtx &c, const E
       st.cursor = cs;
 #pragma unroll 1
       for (int j = GC - 1; j >= 0; --j) {
-        const EncBucket bk =
-            enc_bucket<ST>((int32_t)rs[j * 32 + lane], meta_of(ri[j * 32 + lane]), buckets);
+        float mj = 0.0f;
+#pragma unroll
+        for (int q = 0; q < GC; ++q) mj = q == j ? mu[q] : mj;
+        const EncBucket bk = enc_bucket<ST>(sym_of(rs[j * 32 + lane], mj),
+                                            meta_of(ri[j * 32 + lane]), buckets);
         const EncLook L = enc_look<F>(bk, true, sh);
         const typename F::State xg = st.x;
         const uint32_t cg = st.cursor;
@@ -1012,7 +1065,7 @@ __device__ __forceinline__ bool encode_tile_stream_fast(const EncCtx &c, const E
   return true;
 }
 
-template <class F, bool ST>
+template <class F, bool ST, bool FLT>
 __global__ void __launch_bounds__(kEncThreads32)
     encode_tile_kernel(EncCtx c, const __grid_constant__ EncTileMaps maps) {
   extern __shared__ __align__(16) unsigned char smem[];
@@ -1034,6 +1087,18 @@ __global__ void __launch_bounds__(kEncThreads32)
   const uint32_t ring = ((sbase + tab + 127u) & ~127u) + (uint32_t)warp * kEncTileRingBytes;
   const uint32_t *ring_p = reinterpret_cast<const uint32_t *>(smem + (ring - sbase));
   const uint32_t bar0 = smem_addr(&ring_bar[warp][0]);
+  // FLT: the scale table after every warp's ring, then its key counts
+  float *stab = nullptr;
+  ScaleKeys keys{};
+  bool use_keys = false;
+  if (FLT) {
+    stab = reinterpret_cast<float *>(smem + (((sbase + tab + 127u) & ~127u) - sbase) +
+                                     (uint32_t)nwarp * kEncTileRingBytes);
+    for (int i = threadIdx.x; i < c.K; i += blockDim.x) stab[i] = c.stab[i];
+    __syncthreads();
+    use_keys = build_scale_keys(stab, c.K, reinterpret_cast<uint8_t *>(stab) + pad16(4ull * c.K),
+                                keys);
+  }
   if (lane == 0) {
     tma::mbar_init(bar0, 1);
     tma::mbar_init(bar0 + 8, 1);
@@ -1045,13 +1110,29 @@ __global__ void __launch_bounds__(kEncThreads32)
        k += (int64_t)gridDim.x * nwarp) {
     const int64_t s = stream_of(c.g, k);
     // unrolled chunks for tile widths 64 and 56 (8 and 7 groups), the general
-    // loop otherwise
+    // loop otherwise (float latents take the tile kernel only when every tile
+    // is 64 or 56 wide)
     const int64_t ww = c.g.tw * ((s % c.g.ntx) + 1) <= c.g.Wd ? c.g.tw : c.g.Wd % c.g.tw;
-    bool ok;
+    bool ok = true;
     switch (ww) {
-      case 64: ok = encode_tile_stream_fast<F, ST, 8>(c, maps, meta, buckets, ring, ring_p, bar0, par, s); break;
-      case 56: ok = encode_tile_stream_fast<F, ST, 7>(c, maps, meta, buckets, ring, ring_p, bar0, par, s); break;
-      default: ok = encode_tile_stream<F, ST>(c, maps, meta, buckets, ring, ring_p, bar0, par, s);
+      case 64:
+        if (FLT && use_keys)
+          ok = encode_tile_stream_fast<F, ST, 8, 2>(c, maps, meta, buckets, ring, ring_p, bar0, par, s, stab, keys);
+        else
+          ok = encode_tile_stream_fast<F, ST, 8, FLT ? 1 : 0>(c, maps, meta, buckets, ring, ring_p, bar0, par, s, stab, keys);
+        break;
+      case 56:
+        if (FLT && use_keys)
+          ok = encode_tile_stream_fast<F, ST, 7, 2>(c, maps, meta, buckets, ring, ring_p, bar0, par, s, stab, keys);
+        else
+          ok = encode_tile_stream_fast<F, ST, 7, FLT ? 1 : 0>(c, maps, meta, buckets, ring, ring_p, bar0, par, s, stab, keys);
+        break;
+      default:
+        if constexpr (FLT) {
+          if (lane == 0) report(c.status, RANS_ERR_ARG, s);
+        } else {
+          ok = encode_tile_stream<F, ST>(c, maps, meta, buckets, ring, ring_p, bar0, par, s);
+        }
     }
     if (!ok) break;
   }
@@ -1080,15 +1161,18 @@ bool enc_tile_path_ok(const EncCtx &c, int mode, int sym_dtype, const void *inde
 
 constexpr int kNotTaken = 1;
 
-template <class F>
+template <class F, bool FLT = false>
 int launch_encode_tile(const EncCtx &c, int mode, const int32_t *indexes, const void *symbols,
                        cudaStream_t st) {
   const Geom &g = c.g;
   int dev = 0;
   cudaGetDevice(&dev);
   const uint32_t tab = enc_table_bytes(mode, c);
+  const uint32_t stab_bytes =
+      FLT ? (uint32_t)pad16(4ull * (uint64_t)c.K) + kScaleKeyBytes : 0u;
   const int optin = smem_optin(dev);
-  const uint32_t lim = (uint32_t)optin - 64u - 2u * 8u * kEncMaxWarps;
+  const uint32_t lim = (uint32_t)optin - 64u - 2u * 8u * kEncMaxWarps - stab_bytes;
+  if (FLT && c.K > 65536) return kNotTaken;
   if (tab + 128u + kEncTileRingBytes > lim) return kNotTaken;
   EncTileMaps maps;
   const int64_t per_img = g.ng * g.nty * g.ntx;
@@ -1107,8 +1191,8 @@ int launch_encode_tile(const EncCtx &c, int mode, const int32_t *indexes, const 
   const int64_t room = ((int64_t)lim - tab - 128) / kEncTileRingBytes;
   if (warps > room) warps = room;
   if (warps < 1) warps = 1;
-  const uint32_t smem = tab + 128u + (uint32_t)warps * kEncTileRingBytes;
-  auto kern = mode == 2 ? encode_tile_kernel<F, true> : encode_tile_kernel<F, false>;
+  const uint32_t smem = tab + 128u + (uint32_t)warps * kEncTileRingBytes + stab_bytes;
+  auto kern = mode == 2 ? encode_tile_kernel<F, true, FLT> : encode_tile_kernel<F, false, FLT>;
   if (ensure_dyn_smem((const void *)kern, (uint32_t)(smem)) !=
       cudaSuccess)
     return RANS_ERR_CUDA;
@@ -1511,9 +1595,15 @@ int launch_encode_float(const float *y, const float *means, const float *scales,
   c.scratch = scratch;
   c.lens = lens;
   c.status = status;
-  // float latents code the 64-bit format only (the caller checks); tables
-  // too large for the bucket words in shared memory are read from global
-  // memory here
+  // float latents code the 64-bit format only (the caller checks); tiled
+  // streams of 64- and 56-wide tiles take the tile-staged kernel (scales and
+  // y staged as the index and symbol tiles)
+  if ((t.enc_in_smem == 1 || t.enc_in_smem == 2) && flt_tile_shape_ok(g, y, scales)) {
+    const int r = launch_encode_tile<Rans64, true>(c, t.enc_in_smem, reinterpret_cast<const int32_t *>(scales), y, st);
+    if (r != kNotTaken) return r;
+  }
+  // tables too large for the bucket words in shared memory are read from
+  // global memory here
   const bool smem = t.enc_in_smem == 1;
   if (g.W == 32)
     return smem ? launch_encode_t<Rans64, 32, int32_t, 1, true, true>(c, st)

@@ -70,6 +70,9 @@ int launch_debug_divide(const uint64_t *x, const uint32_t *f, int64_t n, uint64_
 int encode_tile_map(void *map, const void *base, uint64_t width, uint64_t height,
                     uint64_t depth, uint32_t box_w, uint32_t box_h);
 
+// Whether float latents (staged tensors a and b) can take the tile kernels.
+bool flt_tile_shape_ok(const Geom &g, const void *a, const void *b);
+
 // Device properties cached per device.
 int num_sms(int device);
 int smem_optin(int device);

@@ -721,12 +721,24 @@ __global__ void __launch_bounds__(256)
   }
 }
 
-// Row index of every scale (scale_row in rans_common.cuh).
+// Row index of every scale: through the key counts (ScaleKeys in
+// rans_common.cuh) when the table qualifies, else by the search (scale_row).
 __global__ void build_indexes_kernel(const float *scales, int64_t n, const float *table, int K,
                                      float bound, int32_t *indexes) {
+  __shared__ float stab[64];
+  __shared__ uint8_t cnt[kScaleKeyBytes];
+  ScaleKeys keys{};
+  bool use_keys = false;
+  if (K <= 64) {  // (uniform: every thread takes the same branch)
+    for (int i = threadIdx.x; i < K; i += blockDim.x) stab[i] = table[i];
+    __syncthreads();
+    use_keys = build_scale_keys(stab, K, cnt, keys);
+  }
   for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n;
-       i += (int64_t)gridDim.x * blockDim.x)
-    indexes[i] = (int32_t)scale_row(bound_scale(__ldg(scales + i), bound), table, K);
+       i += (int64_t)gridDim.x * blockDim.x) {
+    const float s = bound_scale(__ldg(scales + i), bound);
+    indexes[i] = (int32_t)(use_keys ? keys.row(s) : scale_row(s, table, K));
+  }
 }
 
 int ceil_log2(int64_t v) {

@@ -10,6 +10,7 @@
 
 #include <cuda.h>
 
+#include "rans_common.cuh"
 #include "rans_internal.h"
 
 namespace rb {
@@ -56,6 +57,18 @@ int encode_tile_map(void *map, const void *base, uint64_t width, uint64_t height
                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
                        CU_TENSOR_MAP_L2_PROMOTION_L2_128B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS ? RANS_OK : RANS_ERR_CUDA;
+}
+
+// Float latents on the tile kernels: tiled W = 32 streams (64-bit format,
+// no alias, one scale per element) whose tiles are all 64 or 56 wide and a
+// multiple of 4 rows high, the two staged tensors 16-byte aligned.
+bool flt_tile_shape_ok(const Geom &g, const void *a, const void *b) {
+  if (g.kind != RANS_CHUNK_TILED || g.W != 32 || g.alias || g.ib_shift != 0) return false;
+  if ((reinterpret_cast<uintptr_t>(a) & 15) || (reinterpret_cast<uintptr_t>(b) & 15)) return false;
+  auto width_ok = [](int64_t w) { return w == 64 || w == 56; };
+  const int64_t ww1 = g.Wd % g.tw, hh1 = g.H % g.th;
+  if (!width_ok(g.tw > g.Wd ? g.Wd : g.tw) || (ww1 != 0 && !width_ok(ww1))) return false;
+  return g.th % 4 == 0 && hh1 % 4 == 0 && g.Wd % 4 == 0;
 }
 
 }  // namespace rb

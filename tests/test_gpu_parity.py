@@ -471,6 +471,30 @@ def test_build_indexes_matches_oracle(K):
     assert np.array_equal(got.cpu().numpy(), O.build_indexes(s, t, WL.SCALE_MIN))
 
 
+@pytest.mark.parametrize("kind", ["dense", "repeated", "wide"])
+def test_build_indexes_unusual_tables(kind):
+    """Tables the key-count lookup must hand back to the search (a repeated
+    entry) or index at fine or coarse key widths (64 entries within 0.1%, or
+    spread over 2^-100 .. 2^100): rows equal the oracle's."""
+    rng = np.random.Generator(np.random.PCG64(32))
+    if kind == "dense":
+        t = np.float32(1.0) + np.arange(64, dtype=np.float32) * np.float32(1.6e-5)
+    elif kind == "repeated":
+        t = WL.log_spaced_scales(WL.SCALE_MIN, WL.SCALE_MAX_Y, 64).astype(np.float32)
+        t[20] = t[21]
+    else:
+        t = np.exp2(np.linspace(-100, 100, 64)).astype(np.float32)
+    lo, hi = float(t.min()) / 2, float(t.max()) * 2
+    s = np.concatenate([np.exp(rng.uniform(np.log(lo), np.log(hi), 50000)), t,
+                        np.nextafter(t, np.float32(0)), np.nextafter(t, np.float32(np.inf)),
+                        [0.0, -1.0, np.inf, np.nan]]).astype(np.float32)
+    got = torch.empty(s.size, dtype=torch.int32, device="cuda")
+    bound = float(t.min()) / 4
+    rb.check(rb.rans_build_indexes(torch.from_numpy(s).cuda(), torch.from_numpy(t).cuda(),
+                                   bound, got))
+    assert np.array_equal(got.cpu().numpy(), O.build_indexes(s, t, bound))
+
+
 @pytest.mark.parametrize("W,with_means,n_rows", [(32, True, 64), (32, False, 64), (1, True, 64),
                                                 (32, True, 256), (32, True, 128)])
 def test_encode_from_scales_matches_oracle(W, with_means, n_rows):
@@ -495,6 +519,41 @@ def test_encode_from_scales_matches_oracle(W, with_means, n_rows):
                                     w["scale_bound"], tables, ch, means=dev(w["means"]))
     assert rb.rans_get_status(wsd) == rb.OK
     ref = O.dequantize(wi["symbols"], None if w["means"] is None else w["means"].reshape(-1))
+    assert np.array_equal(vals.cpu().numpy(), ref)
+
+
+@pytest.mark.parametrize("with_means", [True, False])
+def test_float_tiles_with_far_values(with_means):
+    """Float latents on the tile-staged coders (64- and 56-wide tiles): 0.1%
+    of the values pushed far outside their rows, so chunks with escapes are
+    coded and decoded again on the escape path; streams and values equal the
+    oracle's."""
+    w = WL.y_float(n_images=2, W=32, with_means=with_means)
+    rng = np.random.Generator(np.random.PCG64(77))
+    y = np.array(w["y"], copy=True).reshape(-1)
+    far = rng.choice(y.size, y.size // 1000, replace=False)
+    y[far] += rng.choice(np.float32([-1, 1]), far.size) * rng.uniform(3e3, 3e6, far.size).astype(np.float32)
+    w["y"] = y.reshape(w["y"].shape)
+    c, l, o = O.build_cdfs_from_scales(w["scales"], w["tail_mass"])
+    rows = O.build_indexes(w["fscales"], w["scales"], w["scale_bound"]).reshape(-1)
+    sym = O.quantize(w["y"], w["means"]).reshape(-1)
+    wi = dict(w, symbols=sym, indexes=rows)
+    want, woffs = oracle_encode(wi, c, l, o)
+    dev = lambda a: None if a is None else torch.from_numpy(np.ascontiguousarray(a).reshape(-1)).cuda()
+    tables = tables_from_numpy(c, l, o)
+    assert tables.c.enc_in_smem == 1 and tables.c.dec_in_smem == 1
+    ch = chunking_of(w)
+    table = dev(np.asarray(w["scales"], np.float32))
+    out, offs, ws = rb.encode_from_scales(dev(w["y"]), dev(w["fscales"]), table,
+                                          w["scale_bound"], tables, ch, means=dev(w["means"]))
+    assert rb.rans_get_status(ws.enc) == rb.OK
+    total = int(offs[-1].item())
+    assert offs.cpu().numpy().astype(np.uint64).tolist() == woffs.tolist()
+    assert np.array_equal(out[:total].cpu().numpy(), want)
+    vals, wsd = rb.decode_to_values(out[:total], offs, dev(w["fscales"]), table,
+                                    w["scale_bound"], tables, ch, means=dev(w["means"]))
+    assert rb.rans_get_status(wsd) == rb.OK
+    ref = O.dequantize(sym, None if w["means"] is None else w["means"].reshape(-1))
     assert np.array_equal(vals.cpu().numpy(), ref)
 
 
