@@ -253,8 +253,26 @@ struct GaussPmf {
   int center, npmf;
   double s;
   uint32_t total;  // 2^precision
+  const double *U;  // u(0 .. center + 1) in shared memory, or null
   __device__ unsigned long long eval(int i0, int i1, int32_t *f, int &bad) const {
     unsigned long long sum = 0;
+    if (U) {
+      // the row is symmetric about its centre: entry i takes u(d) - u(d + 1),
+      // d = |i - centre|, and the tail 2 u(centre + 1) (the same double
+      // argument as 2 Phi((-0.5 - centre) / s))
+      for (int i = i0; i < i1; ++i) {
+        const int d = abs(i - center);
+        const float p = i == npmf ? (float)(2.0 * U[center + 1]) : (float)(U[d] - U[d + 1]);
+        long long q = scaled_freq(p, total);
+        if (q < 0) {
+          bad = 1;
+          q = 0;
+        }
+        f[i] = (int32_t)(uint32_t)q;
+        sum += (unsigned long long)q;
+      }
+      return sum;
+    }
     int da = -1, db = -1;  // the two most recent u values
     double ua = 0.0, ub = 0.0;
     auto u = [&](int d) -> double {
@@ -309,9 +327,23 @@ struct GivenPmf {
   }
 };
 
+// u(d) = Phi((0.5 - d) / s) for d = 0 .. c + 1 into U (shared memory, c + 2
+// doubles), spread over the block; null when they do not fit in cap doubles
+// (the row's threads then evaluate their own).
+__device__ __forceinline__ const double *gauss_u_table(double *U, int cap, int c, double s) {
+  if (c + 2 > cap) return nullptr;  // (uniform)
+  for (int d = threadIdx.x; d <= c + 1; d += blockDim.x)
+    U[d] = std_normal_cdf((0.5 - (double)d) / s);
+  __syncthreads();
+  return U;
+}
+
+constexpr uint32_t kGaussSmemBytes = 32768;  // u table (and the fused kernel's row)
+
 __global__ void __launch_bounds__(kRowThreads)
     gaussian_rows_kernel(const float *scales, double tail, int prec, int32_t *cdfs, int Lmax,
                          int32_t *lengths, int32_t *offsets) {
+  extern __shared__ double utab[];
   __shared__ BlockScratch sh;
   __shared__ QuantScratch qs;
   const int r = blockIdx.x;
@@ -321,7 +353,9 @@ __global__ void __launch_bounds__(kRowThreads)
   int len = 2 * c + 3;
   if (st == RANS_OK && len > Lmax) st = RANS_ERR_CAPACITY;
   if (st == RANS_OK) {
-    GaussPmf pf{c, 2 * c + 1, (double)scales[r], 1u << prec};
+    const double sd = (double)scales[r];
+    const double *U = gauss_u_table(utab, (int)(kGaussSmemBytes / 8), c, sd);
+    GaussPmf pf{c, 2 * c + 1, sd, 1u << prec, U};
     st = quantise_row(pf, 2 * c + 2, row, sh, qs, 1u << prec);
   }
   for (int j = (st == RANS_OK ? len : 0) + threadIdx.x; j < Lmax; j += kRowThreads) row[j] = 0;
@@ -431,16 +465,19 @@ __device__ __forceinline__ uint32_t boundary_bits(const int32_t *row, int nb, in
 
 // The slots [tb, tb + kSlotsPerBlock) of a row (row in shared or global
 // memory, entries scaled by << sh).
+// SPT slots per thread, blockDim.x apart (so that a warp's stores stay
+// coalesced), their searches independent of one another.
+template <int SPT = kSlotsPerThread>
 __device__ void fill_slot_block(const int32_t *row, int nb, uint32_t slot0, int w, int nslots,
                                 int tb, uint32_t *slots, const ChunkArea &ca, uint32_t sh) {
   const int lane = threadIdx.x & 31;
-  const int t0 = tb + (int)threadIdx.x * kSlotsPerThread;
+  const int t0 = tb + (int)threadIdx.x;
   const uint32_t nch = w > 16 ? (uint32_t)(w >> 4) : 1u;  // bitmap words of a slot
-  int lo[kSlotsPerThread], hi[kSlotsPerThread];
+  int lo[SPT], hi[SPT];
   uint32_t need = 0;
 #pragma unroll
-  for (int u = 0; u < kSlotsPerThread; ++u) {
-    const int t = t0 + u;
+  for (int u = 0; u < SPT; ++u) {
+    const int t = t0 + u * (int)blockDim.x;
     lo[u] = hi[u] = 0;
     if (t < nslots) {
       lo[u] = bucket_of(row, nb, t * w, sh);
@@ -460,8 +497,8 @@ __device__ void fill_slot_block(const int32_t *row, int nb, uint32_t slot0, int 
   if (lane == 31 && wtot > 0) wbase = atomicAdd(ca.used, wtot);
   uint32_t at = __shfl_sync(kFull, wbase, 31) + incl - need;
 #pragma unroll
-  for (int u = 0; u < kSlotsPerThread; ++u) {
-    const int t = t0 + u;
+  for (int u = 0; u < SPT; ++u) {
+    const int t = t0 + u * (int)blockDim.x;
     if (t >= nslots) continue;
     const int a = t * w;
     const int inside = hi[u] - lo[u];
@@ -603,7 +640,7 @@ __global__ void __launch_bounds__(kRowThreads)
     gaussian_refresh_kernel(const float *scales, double tail, int prec, int32_t *cdfs, int Lmax,
                             int32_t *lengths, int32_t *offsets, RowMeta *meta, uint32_t *buckets,
                             uint16_t *starts, uint32_t *slots, ChunkArea ca, int32_t *status) {
-  extern __shared__ int32_t srow[];
+  extern __shared__ __align__(16) int32_t srow[];
   __shared__ BlockScratch sh;
   __shared__ QuantScratch qs;
   const int r = blockIdx.x;
@@ -613,7 +650,11 @@ __global__ void __launch_bounds__(kRowThreads)
   const int len = 2 * c + 3;
   if (st == RANS_OK && len > Lmax) st = RANS_ERR_CAPACITY;
   if (st == RANS_OK) {
-    GaussPmf pf{c, 2 * c + 1, (double)scales[r], 1u << prec};
+    // the u table in the space the row is staged in below
+    const double sd = (double)scales[r];
+    const double *U = gauss_u_table(reinterpret_cast<double *>(srow),
+                                    (int)(kSlotSmemBytes / 8), c, sd);
+    GaussPmf pf{c, 2 * c + 1, sd, 1u << prec, U};
     st = quantise_row(pf, 2 * c + 2, row, sh, qs, 1u << prec);
   }
   for (int j = (st == RANS_OK ? len : 0) + threadIdx.x; j < Lmax; j += kRowThreads) row[j] = 0;
@@ -637,8 +678,8 @@ __global__ void __launch_bounds__(kRowThreads)
   pack_row(prow, len, m.bucket_base, ssh, buckets, starts, status, r);
   const int shift = (int)slot_shift(m.slot);
   const int nslots = 1 << (16 - shift);
-  for (int tb = 0; tb < nslots; tb += kRowThreads * kSlotsPerThread)
-    fill_slot_block(prow, len - 1, slot_base(m.slot), 1 << shift, nslots, tb, slots, ca, ssh);
+  for (int tb = 0; tb < nslots; tb += kRowThreads * 4)
+    fill_slot_block<4>(prow, len - 1, slot_base(m.slot), 1 << shift, nslots, tb, slots, ca, ssh);
 }
 
 // Alias tables, one row per block (the reading of the alias method given
@@ -759,8 +800,8 @@ int launch_gaussian_lengths(const float *scales, int K, double tail, int32_t *le
 
 int launch_gaussian_rows(const float *scales, int K, double tail, int prec, int32_t *cdfs,
                          int Lmax, int32_t *lengths, int32_t *offsets, cudaStream_t st) {
-  gaussian_rows_kernel<<<K, kRowThreads, 0, st>>>(scales, tail, prec, cdfs, Lmax, lengths,
-                                                  offsets);
+  gaussian_rows_kernel<<<K, kRowThreads, kGaussSmemBytes, st>>>(scales, tail, prec, cdfs, Lmax,
+                                                                lengths, offsets);
   return cudaGetLastError() == cudaSuccess ? RANS_OK : RANS_ERR_CUDA;
 }
 
