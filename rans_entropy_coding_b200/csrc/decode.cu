@@ -1550,6 +1550,140 @@ __global__ void __launch_bounds__(kTileMaxStreams * 32, 1)
   if (lane == 0) tma::bulk_wait_all();
 }
 
+// --------------------------------------------- contiguous chunked streams --
+// Contiguous streams (64-bit format, W = 32) made of whole chunks of 256
+// symbols whose row changes at most once per chunk (an index block of 256
+// symbols or more; the byte sweep's shape): a chunk's row index is one load,
+// read a chunk ahead, and its metadata one shared load; its 8 groups decode
+// as one block of straight-line code on the shared-memory word window; its
+// values go to a two-half ring in shared memory and out with one bulk store.
+constexpr int kChunkSyms = 256;
+
+template <typename SymT>
+__host__ __device__ constexpr uint32_t chunk_warp_bytes() {
+  return kWinBytes + 2u * (uint32_t)kChunkSyms * (uint32_t)sizeof(SymT);
+}
+
+template <typename SymT, bool SEARCH>
+__device__ __forceinline__ void decode_chunk_stream(const DecCtx &c, const RowMeta *meta,
+                                                    const uint16_t *starts,
+                                                    const uint32_t *slots, uint32_t *win,
+                                                    SymT *oring, int64_t s) {
+  constexpr int GC = kChunkSyms / 32;
+  const int lane = threadIdx.x & 31;
+  const Geom &g = c.g;
+  const StreamDesc d = stream_desc(g, s);
+  const uint32_t *words = nullptr;
+  uint64_t nw64 = 0;
+  if (!d.ok || !stream_bounds<Rans64>(c, s, 32, words, nw64) || nw64 >= (uint64_t(1) << 31)) {
+    if (lane == 0) report(c.status, d.ok ? RANS_ERR_CORRUPT : RANS_ERR_ARG, s);
+    return;
+  }
+  const uint32_t nw = (uint32_t)nw64;
+  const uint32_t kmax = (uint32_t)c.K - 1u;
+  const int32_t M = (int32_t)(d.n / kChunkSyms);
+  const int ib = g.ib_shift;
+  const uint32_t l0 = lane == 0 ? 1u : 0u;
+  SymT *out = reinterpret_cast<SymT *>(c.out) + d.base;
+  if (lane == 0)
+    bulk_prefetch_l2(reinterpret_cast<const char *>(c.in),
+                     reinterpret_cast<const char *>(c.in) + c.in_bytes,
+                     reinterpret_cast<const char *>(words + 64), sizeof(uint32_t) * (nw - 64));
+  uint64_t x = (uint64_t)__ldg(words + 2 * lane) | ((uint64_t)__ldg(words + 2 * lane + 1) << 32);
+  uint32_t rd = 64, ldn = 64, rmax = 0;
+  bool bad = false;
+  uint32_t r_next = (uint32_t)__ldg(c.idx + (d.base >> ib));
+#pragma unroll 1
+  for (int32_t k = 0; k < M; ++k) {
+    const int h = k & 1;
+    const uint32_t r = r_next;
+    if (k + 1 < M) r_next = (uint32_t)__ldg(c.idx + ((d.base + (int64_t)(k + 1) * kChunkSyms) >> ib));
+    rmax = max(rmax, r);
+    const RowMeta m = row_meta(meta, min(r, kmax));
+    // the word window (as the tile decoder's); the ring half of this chunk's
+    // values, once chunk k - 2's store has read it
+    const bool ahead = rd + 32u * GC <= ldn;
+    win_refill(win, words, nw, rd, ldn);
+    if (ahead) cp_async_wait<1>(); else cp_async_wait<0>();
+    tma::bulk_wait_read1_if(l0);
+    __syncwarp();
+    const uint64_t xs = x;
+    const uint32_t rds = rd;
+    uint32_t esc = 0;
+    int32_t val[GC];
+#pragma unroll
+    for (int j = 0; j < GC; ++j) val[j] = dec_group_win64<SEARCH>(x, rd, m, starts, slots, win, esc);
+    SymT *oh = oring + h * kChunkSyms;
+    if (!__any_sync(kFull, esc != 0)) {
+#pragma unroll
+      for (int j = 0; j < GC; ++j) oh[j * 32 + lane] = (SymT)val[j];
+    } else {
+      // an escape in this chunk: decode it again from its saved state on
+      // the lane-serial path, then restart the word window there
+      WarpDec<Rans64> w;
+      w.x = xs;
+      w.cur = rds;
+      w.off = 0;
+      w.rmax = 0;
+      w.bad = false;
+      load_window(w, words, nw);
+#pragma unroll 1
+      for (int j = 0; j < GC; ++j)
+        oh[j * 32 + lane] =
+            (SymT)dec_group_val<Rans64, SEARCH>(w, m, starts, slots, words, nw, 0u);
+      bad = bad || w.bad;
+      x = w.x;
+      rd = (uint32_t)(w.cur + w.off);
+      cp_async_wait<0>();
+      __syncwarp();
+      ldn = rd & ~31u;
+    }
+    // the chunk's values go out
+    tma::fence_proxy_async();
+    __syncwarp();
+    tma::store_1d_commit_if(l0, out + (int64_t)k * kChunkSyms, smem_addr(oh),
+                            (uint32_t)(kChunkSyms * sizeof(SymT)));
+  }
+  cp_async_wait<0>();
+  if (__any_sync(kFull, rmax > kmax)) {
+    if (lane == 0) report(c.status, RANS_ERR_INDEX, s);
+    return;
+  }
+  const bool ok = !bad && x == Rans64::kLow && rd == nw;
+  if (!__all_sync(kFull, ok) && lane == 0) report(c.status, RANS_ERR_CORRUPT, s);
+}
+
+template <typename SymT>
+__global__ void __launch_bounds__(kDecMaxWarps * 32, 1) decode_chunk_kernel(DecCtx c) {
+  extern __shared__ __align__(16) unsigned char smem[];
+  __shared__ uint64_t bar;
+  const char *gb = c.blob + kHeaderBytes;
+  if (!stage_to_smem(smem, gb, c.meta_bytes, &bar, c.status, smem + c.meta_bytes,
+                     gb + c.meta_bytes + c.bucket_bytes, c.start_bytes + c.slot_bytes))
+    return;
+  const RowMeta *meta = reinterpret_cast<const RowMeta *>(smem);
+  const uint16_t *starts = reinterpret_cast<const uint16_t *>(smem + c.meta_bytes);
+  const uint32_t *slots = reinterpret_cast<const uint32_t *>(smem + c.meta_bytes + c.start_bytes);
+  const uint32_t tab = c.meta_bytes + c.start_bytes + c.slot_bytes;
+  const int warp = threadIdx.x >> 5, nwarp = blockDim.x >> 5, lane = threadIdx.x & 31;
+  // each warp's word window and value ring, 128-byte aligned
+  const uint32_t sbase = smem_addr(smem);
+  const uint32_t wbase = ((sbase + tab + 127u) & ~127u) + (uint32_t)warp * chunk_warp_bytes<SymT>();
+  uint32_t *win = reinterpret_cast<uint32_t *>(smem + (wbase - sbase));
+  SymT *oring = reinterpret_cast<SymT *>(smem + (wbase - sbase) + kWinBytes);
+  // slots that ran out of bitmap room (flagged in the blob header) search
+  const bool search = reinterpret_cast<const uint32_t *>(c.blob)[kSearchFlagWord] != 0;
+  for (int64_t k = blockIdx.x + (int64_t)gridDim.x * warp; k < c.g.S;
+       k += (int64_t)gridDim.x * nwarp) {
+    if (search)
+      decode_chunk_stream<SymT, true>(c, meta, starts, slots, win, oring, k);
+    else
+      decode_chunk_stream<SymT, false>(c, meta, starts, slots, win, oring, k);
+  }
+  (void)lane;
+  if ((threadIdx.x & 31) == 0) tma::bulk_wait_all();
+}
+
 // Whether a tiled W = 32 decode can take the tile-staged kernel: int32 rows
 // and symbols in 16-byte aligned tensors, one index per element, every tile
 // row a whole number of 16-byte units and of 8-symbol steps (so a chunk of 4
@@ -1612,6 +1746,51 @@ int launch_decode_tile(const DecCtx &c, const void *indexes, void *symbols, cuda
   const int64_t cap = (int64_t)fit * sms;
   const int64_t blocks = need < cap ? need : cap;
   kern<<<(unsigned)blocks, (unsigned)warps * 32, smem, st>>>(c, maps);
+  return cudaGetLastError() == cudaSuccess ? RANS_OK : RANS_ERR_CUDA;
+}
+
+// Whether a decode can take the chunked kernel: contiguous W = 32 streams of
+// the 64-bit format, every stream a whole number of 256-symbol chunks, an
+// index block of at least 256 symbols, the tables' lookup slots in shared
+// memory, and a 16-byte aligned output of 1-, 2- or 4-byte symbols.
+bool chunk_path_ok(const DecCtx &c, int mode, int sym_dtype, const void *symbols) {
+  const Geom &g = c.g;
+  if (g.kind != RANS_CHUNK_CONTIG || g.W != 32 || g.alias || g.fmt != RANS_FMT_RANS64 ||
+      mode != 1 || g.ib_shift < 8)
+    return false;
+  if (sym_dtype != RANS_SYM_UINT8 && sym_dtype != RANS_SYM_INT16 && sym_dtype != RANS_SYM_INT32)
+    return false;
+  if (g.per < kChunkSyms || g.per % kChunkSyms != 0 || g.per > (int64_t(1) << 28) ||
+      g.n != g.S * g.per)
+    return false;
+  return (reinterpret_cast<uintptr_t>(symbols) & 15) == 0;
+}
+
+template <typename SymT>
+int launch_decode_chunk(const DecCtx &c, cudaStream_t st) {
+  const Geom &g = c.g;
+  int dev = 0;
+  cudaGetDevice(&dev);
+  const uint32_t tab = dec_table_bytes(1, c);
+  const uint32_t per_warp = chunk_warp_bytes<SymT>();
+  const uint32_t lim = (uint32_t)smem_optin(dev) - 64u;
+  if (tab + 128u + per_warp > lim) return kNotTaken;
+  const int sms = num_sms(dev);
+  int64_t warps = (g.S + sms - 1) / sms;
+  if (warps > kDecMaxWarps) warps = kDecMaxWarps;
+  const int64_t room = ((int64_t)lim - tab - 128) / per_warp;
+  if (warps > room) warps = room;
+  if (warps < 1) warps = 1;
+  const uint32_t smem = tab + 128u + (uint32_t)warps * per_warp;
+  auto kern = decode_chunk_kernel<SymT>;
+  if (ensure_dyn_smem((const void *)kern, smem) != cudaSuccess) return RANS_ERR_CUDA;
+  int fit = 0;
+  if (blocks_per_sm(&fit, (const void *)kern, (int)warps * 32, smem) != cudaSuccess || fit < 1)
+    return RANS_ERR_CUDA;
+  const int64_t need = (g.S + warps - 1) / warps;
+  const int64_t cap = (int64_t)fit * sms;
+  const int64_t blocks = need < cap ? need : cap;
+  kern<<<(unsigned)blocks, (unsigned)warps * 32, smem, st>>>(c);
   return cudaGetLastError() == cudaSuccess ? RANS_OK : RANS_ERR_CUDA;
 }
 
@@ -1876,6 +2055,12 @@ int launch_decode(const uint8_t *in, uint64_t in_bytes, const uint64_t *offsets,
   c.bound = 0.0f;
   c.stab_smem = 0;
   const int mode = t.dec_in_smem;
+  if (chunk_path_ok(c, mode, sym_dtype, symbols)) {
+    const int r = sym_dtype == RANS_SYM_UINT8   ? launch_decode_chunk<uint8_t>(c, st)
+                  : sym_dtype == RANS_SYM_INT16 ? launch_decode_chunk<int16_t>(c, st)
+                                                : launch_decode_chunk<int32_t>(c, st);
+    if (r != kNotTaken) return r;
+  }
   if (tile_path_ok(c, mode, sym_dtype, indexes, symbols)) {
     const int r = g.fmt == RANS_FMT_RANS32_16 ? launch_decode_tile<Rans32>(c, indexes, symbols, st)
                                               : launch_decode_tile<Rans64>(c, indexes, symbols, st);

@@ -1138,6 +1138,143 @@ __global__ void __launch_bounds__(kEncThreads32)
   }
 }
 
+// --------------------------------------------- contiguous chunked streams --
+// Contiguous streams (64-bit format, W = 32) made of whole chunks of 256
+// symbols whose row changes at most once per chunk (an index block of 256
+// symbols or more; the byte sweep's shape): a chunk's row index is one load,
+// read a chunk ahead, and its row metadata one shared load; its symbols come
+// into a two-half ring in shared memory with 16-byte cp.async copies, a
+// chunk ahead; its 8 groups are coded as one unrolled block (escapes only
+// recorded, the chunk coded again from its saved state when one occurs), in
+// the same order as the general coder, so the streams are the same.
+constexpr int kEncChunkSyms = 256;
+
+template <typename SymT, bool ST>
+__device__ __forceinline__ void encode_chunk_stream(const EncCtx &c, const RowMeta *meta,
+                                                    const uint32_t *buckets, SymT *ring,
+                                                    int64_t s) {
+  using F = Rans64;
+  using Word = typename F::Word;
+  constexpr int GC = kEncChunkSyms / 32;
+  constexpr int kChunkBytes = kEncChunkSyms * (int)sizeof(SymT);
+  const int lane = threadIdx.x & 31;
+  const Geom &g = c.g;
+  const StreamDesc d = stream_desc(g, s);
+  if (!d.ok) {
+    if (lane == 0) report(c.status, RANS_ERR_ARG, s);
+    return;
+  }
+  Word *end = reinterpret_cast<Word *>(c.scratch + slot_end(g, d, s));
+  const uint32_t sh = 0;
+  const uint32_t kmax = (uint32_t)c.K - 1u;
+  const uint32_t above = 0xfffffffeu << lane;  // lanes > this lane
+  const SymT *src = reinterpret_cast<const SymT *>(c.sym) + d.base;
+  const int32_t M = (int32_t)(d.n / kEncChunkSyms);
+  const int ib = g.ib_shift;
+  // chunk ch's symbols into ring half ch & 1 (one commit group per call)
+  auto issue = [&](int32_t ch) {
+    const char *gs = reinterpret_cast<const char *>(src + (int64_t)ch * kEncChunkSyms);
+    char *ds = reinterpret_cast<char *>(ring + (ch & 1) * kEncChunkSyms);
+#pragma unroll
+    for (int o = lane * 16; o < kChunkBytes; o += 32 * 16) cp_async16(ds + o, gs + o);
+    cp_async_commit();
+  };
+  auto row_at = [&](int32_t ch) -> uint32_t {
+    return (uint32_t)__ldg(c.idx + ((d.base + (int64_t)ch * kEncChunkSyms) >> ib));
+  };
+  WarpEnc<F> st;
+  st.x = F::kLow;
+  st.cursor = 0;
+  st.rmax = 0;
+  st.range_err = false;
+  issue(M - 1);
+  uint32_t r_next = row_at(M - 1);
+#pragma unroll 1
+  for (int32_t ch = M - 1; ch >= 0; --ch) {
+    const uint32_t r = r_next;
+    // the chunk before this one into the other half (read two chunks ago),
+    // then this chunk's symbols landed
+    __syncwarp();
+    if (ch >= 1) {
+      issue(ch - 1);
+      r_next = row_at(ch - 1);
+    } else {
+      cp_async_commit();
+    }
+    cp_async_wait<1>();
+    __syncwarp();
+    st.rmax = max(st.rmax, r);
+    const RowMeta m = row_meta(meta, min(r, kmax));
+    const SymT *rs = ring + (ch & 1) * kEncChunkSyms;
+    const typename F::State xs = st.x;
+    const uint32_t cs = st.cursor;
+    uint32_t esc = 0;
+#pragma unroll
+    for (int j = GC - 1; j >= 0; --j) {
+      const EncBucket bk = enc_bucket<ST>((int32_t)rs[j * 32 + lane], m, buckets);
+      esc |= bk.in_range ? 0u : 1u;
+      EncLook L;
+      L.start = bucket_start(bk.e);
+      L.freq = bucket_freq(bk.e);
+      L.rcp = F::rcp(L.freq, sh);
+      enc_group_fast<F, true>(st, L, true, above, end, sh);
+    }
+    if (__any_sync(kFull, esc != 0)) {
+      // an escape in this chunk: code it again from its saved state
+      st.x = xs;
+      st.cursor = cs;
+#pragma unroll 1
+      for (int j = GC - 1; j >= 0; --j) {
+        const EncBucket bk = enc_bucket<ST>((int32_t)rs[j * 32 + lane], m, buckets);
+        const EncLook L = enc_look<F>(bk, true, sh);
+        const typename F::State xg = st.x;
+        const uint32_t cg = st.cursor;
+        enc_group_fast<F, true>(st, L, true, above, end, sh);
+        if (L.any_esc) enc_group_escape<F>(st, xg, cg, L, true, end, sh);
+      }
+    }
+  }
+  cp_async_wait<0>();
+  if (__any_sync(kFull, st.rmax > kmax)) {
+    if (lane == 0) report(c.status, RANS_ERR_INDEX, s);
+    return;
+  }
+  if (__any_sync(kFull, st.range_err)) {
+    if (lane == 0) report(c.status, RANS_ERR_RANGE, s);
+    return;
+  }
+  // flush: lanes 31..0 push high then low, so lane 0's low word comes first
+  const uint32_t kk = st.cursor + 2u * (31u - (uint32_t)lane);
+  st_global(end - 1 - kk, (Word)(st.x >> F::kWordBits));
+  st_global(end - 2 - kk, (Word)st.x);
+  if (lane == 0) c.lens[s] = sizeof(Word) * (uint64_t)(st.cursor + 64);
+}
+
+template <typename SymT, bool ST>
+__global__ void __launch_bounds__(kEncThreads32) encode_chunk_kernel(EncCtx c) {
+  extern __shared__ __align__(16) unsigned char smem[];
+  __shared__ uint64_t bar;
+  const char *gb = c.blob + kHeaderBytes;
+  if (ST) {
+    if (!stage_to_smem(smem, gb, c.meta_bytes, &bar, c.status, smem + c.meta_bytes,
+                       gb + c.meta_bytes + c.bucket_bytes, c.start_bytes))
+      return;
+  } else {
+    if (!stage_to_smem(smem, gb, c.meta_bytes + c.bucket_bytes, &bar, c.status)) return;
+  }
+  const RowMeta *meta = reinterpret_cast<const RowMeta *>(smem);
+  const uint32_t *buckets = reinterpret_cast<const uint32_t *>(smem + c.meta_bytes);
+  const uint32_t tab = enc_table_bytes(ST ? 2 : 1, c);
+  const int warp = threadIdx.x >> 5, nwarp = blockDim.x >> 5;
+  const uint32_t sbase = smem_addr(smem);
+  const uint32_t rbase = ((sbase + tab + 127u) & ~127u) +
+                         (uint32_t)warp * (2u * kEncChunkSyms * (uint32_t)sizeof(SymT));
+  SymT *ring = reinterpret_cast<SymT *>(smem + (rbase - sbase));
+  for (int64_t k = blockIdx.x + (int64_t)gridDim.x * warp; k < c.g.S;
+       k += (int64_t)gridDim.x * nwarp)
+    encode_chunk_stream<SymT, ST>(c, meta, buckets, ring, k);
+}
+
 // Whether a tiled W = 32 encode can take the tile-staged kernel (the
 // conditions of the decoder's tile path -- int32 rows and symbols in 16-byte
 // aligned tensors, one index per element, tile rows of whole 16-byte units
@@ -1205,6 +1342,49 @@ int launch_encode_tile(const EncCtx &c, int mode, const int32_t *indexes, const 
   const int64_t cap = (int64_t)fit * sms;
   const int64_t blocks = need < cap ? need : cap;
   kern<<<(unsigned)blocks, (unsigned)warps * 32, smem, st>>>(c, maps);
+  return cudaGetLastError() == cudaSuccess ? RANS_OK : RANS_ERR_CUDA;
+}
+
+// Whether an encode can take the chunked kernel: contiguous W = 32 streams
+// of the 64-bit format, every stream a whole number of 256-symbol chunks, an
+// index block of at least 256 symbols, the tables in shared memory, and
+// 16-byte aligned 1-, 2- or 4-byte symbols.
+bool enc_chunk_path_ok(const EncCtx &c, int mode, int sym_dtype, const void *symbols) {
+  const Geom &g = c.g;
+  if (g.kind != RANS_CHUNK_CONTIG || g.W != 32 || g.alias || g.fmt != RANS_FMT_RANS64 ||
+      (mode != 1 && mode != 2) || g.ib_shift < 8)
+    return false;
+  if (sym_dtype != RANS_SYM_UINT8 && sym_dtype != RANS_SYM_INT16 && sym_dtype != RANS_SYM_INT32)
+    return false;
+  if (g.per < kEncChunkSyms || g.per % kEncChunkSyms != 0 || g.n != g.S * g.per) return false;
+  return (reinterpret_cast<uintptr_t>(symbols) & 15) == 0;
+}
+
+template <typename SymT>
+int launch_encode_chunk(const EncCtx &c, int mode, cudaStream_t st) {
+  const Geom &g = c.g;
+  int dev = 0;
+  cudaGetDevice(&dev);
+  const uint32_t tab = enc_table_bytes(mode, c);
+  const uint32_t per_warp = 2u * kEncChunkSyms * (uint32_t)sizeof(SymT);
+  const uint32_t lim = (uint32_t)smem_optin(dev) - 64u;
+  if (tab + 128u + per_warp > lim) return kNotTaken;
+  const int sms = num_sms(dev);
+  int64_t warps = (g.S + sms - 1) / sms;
+  if (warps > kEncMaxWarps) warps = kEncMaxWarps;
+  const int64_t room = ((int64_t)lim - tab - 128) / per_warp;
+  if (warps > room) warps = room;
+  if (warps < 1) warps = 1;
+  const uint32_t smem = tab + 128u + (uint32_t)warps * per_warp;
+  auto kern = mode == 2 ? encode_chunk_kernel<SymT, true> : encode_chunk_kernel<SymT, false>;
+  if (ensure_dyn_smem((const void *)kern, smem) != cudaSuccess) return RANS_ERR_CUDA;
+  int fit = 0;
+  if (blocks_per_sm(&fit, (const void *)kern, (int)warps * 32, smem) != cudaSuccess || fit < 1)
+    return RANS_ERR_CUDA;
+  const int64_t need = (g.S + warps - 1) / warps;
+  const int64_t cap = (int64_t)fit * sms;
+  const int64_t blocks = need < cap ? need : cap;
+  kern<<<(unsigned)blocks, (unsigned)warps * 32, smem, st>>>(c);
   return cudaGetLastError() == cudaSuccess ? RANS_OK : RANS_ERR_CUDA;
 }
 
@@ -1558,6 +1738,12 @@ int launch_encode(const void *symbols, int sym_dtype, const int32_t *indexes,
   c.bound = 0.0f;
   c.stab_smem = 0;
   const int mode = t.enc_in_smem;
+  if (enc_chunk_path_ok(c, mode, sym_dtype, symbols)) {
+    const int r = sym_dtype == RANS_SYM_UINT8   ? launch_encode_chunk<uint8_t>(c, mode, st)
+                  : sym_dtype == RANS_SYM_INT16 ? launch_encode_chunk<int16_t>(c, mode, st)
+                                                : launch_encode_chunk<int32_t>(c, mode, st);
+    if (r != kNotTaken) return r;
+  }
   if (enc_tile_path_ok(c, mode, sym_dtype, indexes, symbols)) {
     const int r = g.fmt == RANS_FMT_RANS32_16
                       ? launch_encode_tile<Rans32>(c, mode, indexes, symbols, st)

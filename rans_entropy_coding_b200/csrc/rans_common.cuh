@@ -497,6 +497,13 @@ __device__ __forceinline__ void cp_async4(void *smem_dst, const void *gsrc) {
                "l"(gsrc)
                : "memory");
 }
+// 16 bytes, both addresses 16-byte aligned, bypassing L1.
+__device__ __forceinline__ void cp_async16(void *smem_dst, const void *gsrc) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(
+                   (uint32_t)__cvta_generic_to_shared(smem_dst)),
+               "l"(gsrc)
+               : "memory");
+}
 __device__ __forceinline__ void cp_async_commit() {
   asm volatile("cp.async.commit_group;" ::: "memory");
 }
@@ -855,6 +862,27 @@ __device__ __forceinline__ void bulk_wait_read_if(uint32_t p) {
   asm volatile(
       "{\n\t.reg .pred q;\n\tsetp.ne.u32 q, %0, 0;\n\t"
       "@q cp.async.bulk.wait_group.read 0;\n\t}" ::"r"(p)
+      : "memory");
+}
+
+// A plain (1-D) bulk store of `bytes` bytes (a multiple of 16, both
+// addresses 16-byte aligned) from shared to global memory, committed as one
+// bulk group, where p is nonzero.
+__device__ __forceinline__ void store_1d_commit_if(uint32_t p, void *dst, uint32_t src,
+                                                   uint32_t bytes) {
+  asm volatile(
+      "{\n\t.reg .pred q;\n\tsetp.ne.u32 q, %0, 0;\n\t"
+      "@q cp.async.bulk.global.shared::cta.bulk_group [%1], [%2], %3;"
+      "\n\t@q cp.async.bulk.commit_group;\n\t}" ::"r"(p),
+      "l"(reinterpret_cast<uint64_t>(dst)), "r"(src), "r"(bytes)
+      : "memory");
+}
+// Waits, where p is nonzero, until every bulk group but the most recent one
+// has read its shared-memory source.
+__device__ __forceinline__ void bulk_wait_read1_if(uint32_t p) {
+  asm volatile(
+      "{\n\t.reg .pred q;\n\tsetp.ne.u32 q, %0, 0;\n\t"
+      "@q cp.async.bulk.wait_group.read 1;\n\t}" ::"r"(p)
       : "memory");
 }
 

@@ -211,6 +211,24 @@ def test_sweep_uint8_blocks():
     _check_streams(WL.sweep(log2_n=20, n_streams=32))
 
 
+@pytest.mark.parametrize("dtype", [np.uint8, np.int16, np.int32])
+def test_chunked_contiguous_streams(dtype):
+    """Contiguous streams of whole 256-symbol chunks with one row per 256
+    symbols (the chunked coders): uint8, int16 and int32 symbols on rows
+    shorter than the alphabet, and far values, so that chunks with escapes
+    are coded again on the escape path."""
+    w = WL.sweep(log2_n=16, n_streams=8, block=256)
+    w["pmf_lengths"] = np.full(16, 200, dtype=np.int32)
+    sym = np.asarray(w["symbols"]).astype(dtype)
+    if dtype != np.uint8:
+        rng = np.random.Generator(np.random.PCG64(5))
+        far = rng.choice(sym.size, sym.size // 200, replace=False)
+        big = 30000 if dtype == np.int16 else 1 << 30
+        sym[far] = rng.integers(-big, big, far.size).astype(dtype)
+    w["symbols"] = sym
+    _check_streams(w)
+
+
 @pytest.mark.parametrize("W", [2, 4, 8])
 def test_few_state_interleaves(W):
     """2, 4 and 8 interleaved states per stream, one thread per stream:
