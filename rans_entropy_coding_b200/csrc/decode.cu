@@ -1653,8 +1653,10 @@ __device__ __forceinline__ void decode_chunk_stream(const DecCtx &c, const RowMe
   if (!__all_sync(kFull, ok) && lane == 0) report(c.status, RANS_ERR_CORRUPT, s);
 }
 
+constexpr int kChunkMaxWarps = 32;  // a 2^28-symbol sweep's 8,192 streams in two rounds
+
 template <typename SymT>
-__global__ void __launch_bounds__(kDecMaxWarps * 32, 1) decode_chunk_kernel(DecCtx c) {
+__global__ void __launch_bounds__(kChunkMaxWarps * 32, 1) decode_chunk_kernel(DecCtx c) {
   extern __shared__ __align__(16) unsigned char smem[];
   __shared__ uint64_t bar;
   const char *gb = c.blob + kHeaderBytes;
@@ -1777,7 +1779,7 @@ int launch_decode_chunk(const DecCtx &c, cudaStream_t st) {
   if (tab + 128u + per_warp > lim) return kNotTaken;
   const int sms = num_sms(dev);
   int64_t warps = (g.S + sms - 1) / sms;
-  if (warps > kDecMaxWarps) warps = kDecMaxWarps;
+  if (warps > kChunkMaxWarps) warps = kChunkMaxWarps;
   const int64_t room = ((int64_t)lim - tab - 128) / per_warp;
   if (warps > room) warps = room;
   if (warps < 1) warps = 1;

@@ -1250,8 +1250,10 @@ __device__ __forceinline__ void encode_chunk_stream(const EncCtx &c, const RowMe
   if (lane == 0) c.lens[s] = sizeof(Word) * (uint64_t)(st.cursor + 64);
 }
 
+constexpr int kEncChunkMaxWarps = 32;  // a 2^28-symbol sweep's 8,192 streams in two rounds
+
 template <typename SymT, bool ST>
-__global__ void __launch_bounds__(kEncThreads32) encode_chunk_kernel(EncCtx c) {
+__global__ void __launch_bounds__(kEncChunkMaxWarps * 32, 1) encode_chunk_kernel(EncCtx c) {
   extern __shared__ __align__(16) unsigned char smem[];
   __shared__ uint64_t bar;
   const char *gb = c.blob + kHeaderBytes;
@@ -1371,7 +1373,7 @@ int launch_encode_chunk(const EncCtx &c, int mode, cudaStream_t st) {
   if (tab + 128u + per_warp > lim) return kNotTaken;
   const int sms = num_sms(dev);
   int64_t warps = (g.S + sms - 1) / sms;
-  if (warps > kEncMaxWarps) warps = kEncMaxWarps;
+  if (warps > kEncChunkMaxWarps) warps = kEncChunkMaxWarps;
   const int64_t room = ((int64_t)lim - tab - 128) / per_warp;
   if (warps > room) warps = room;
   if (warps < 1) warps = 1;
