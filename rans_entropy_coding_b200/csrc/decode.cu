@@ -1360,10 +1360,13 @@ __device__ __forceinline__ bool decode_tile_win64(const DecCtx &c, const TileMap
         for (int j = 0; j < GC; ++j) mu[j] = __ldg(mp + moff[j]);
       }
     }
+    // every group's row metadata first: they do not depend on the state
+    RowMeta ms[GC];
+#pragma unroll
+    for (int j = 0; j < GC; ++j) ms[j] = meta_of((uint32_t)rh[j * 32 + lane]);
 #pragma unroll
     for (int j = 0; j < GC; ++j) {
-      const RowMeta m = meta_of((uint32_t)rh[j * 32 + lane]);
-      val[j] = dec_group_win64<SEARCH>(x, rd, m, starts, slots, win, esc);
+      val[j] = dec_group_win64<SEARCH>(x, rd, ms[j], starts, slots, win, esc);
       if (j == 0) {
         // chunk k + 3 into L2; chunk k + 1 into the other half, once chunk
         // k - 1's store has read it

@@ -1020,14 +1020,30 @@ __device__ __forceinline__ bool encode_tile_stream_fast(const EncCtx &c, const E
     const typename F::State xs = st.x;
     const uint32_t cs = st.cursor;
     uint32_t esc = 0;
+    // integer rows and symbols: every group's bucket first, since the
+    // lookups do not depend on the state (float latents keep them beside
+    // each group: their extra registers would spill)
+    uint32_t be[GC];
+    if constexpr (!FLT) {
+#pragma unroll
+      for (int j = GC - 1; j >= 0; --j) {
+        const EncBucket bk =
+            enc_bucket<ST>((int32_t)rs[j * 32 + lane], meta_of(ri[j * 32 + lane]), buckets);
+        esc |= bk.in_range ? 0u : 1u;
+        be[j] = bk.e;
+      }
+    }
 #pragma unroll
     for (int j = GC - 1; j >= 0; --j) {
-      const EncBucket bk =
-          enc_bucket<ST>(sym_of(rs[j * 32 + lane], mu[j]), meta_of(ri[j * 32 + lane]), buckets);
-      esc |= bk.in_range ? 0u : 1u;
+      if constexpr (FLT) {
+        const EncBucket bk = enc_bucket<ST>(sym_of(rs[j * 32 + lane], mu[j]),
+                                            meta_of(ri[j * 32 + lane]), buckets);
+        esc |= bk.in_range ? 0u : 1u;
+        be[j] = bk.e;
+      }
       EncLook L;
-      L.start = bucket_start(bk.e);
-      L.freq = bucket_freq(bk.e);
+      L.start = bucket_start(be[j]);
+      L.freq = bucket_freq(be[j]);
       L.rcp = F::rcp(L.freq, sh);
       enc_group_fast<F, true>(st, L, true, above, end, sh);
     }
@@ -1209,13 +1225,18 @@ __device__ __forceinline__ void encode_chunk_stream(const EncCtx &c, const RowMe
     const typename F::State xs = st.x;
     const uint32_t cs = st.cursor;
     uint32_t esc = 0;
+    uint32_t be[GC];
 #pragma unroll
     for (int j = GC - 1; j >= 0; --j) {
       const EncBucket bk = enc_bucket<ST>((int32_t)rs[j * 32 + lane], m, buckets);
       esc |= bk.in_range ? 0u : 1u;
+      be[j] = bk.e;
+    }
+#pragma unroll
+    for (int j = GC - 1; j >= 0; --j) {
       EncLook L;
-      L.start = bucket_start(bk.e);
-      L.freq = bucket_freq(bk.e);
+      L.start = bucket_start(be[j]);
+      L.freq = bucket_freq(be[j]);
       L.rcp = F::rcp(L.freq, sh);
       enc_group_fast<F, true>(st, L, true, above, end, sh);
     }
