@@ -975,6 +975,8 @@ __device__ __forceinline__ bool encode_tile_stream_fast(const EncCtx &c, const E
   // lane reads element e = 32 j + lane of the chunk: row e / ww, column
   // e mod ww.
   float mu[GC], mu_n[GC];
+#pragma unroll
+  for (int j = 0; j < GC; ++j) mu[j] = mu_n[j] = 0.0f;
   int32_t moff[GC];
   int32_t my = ylast, mz = zlast;  // the last chunk's position
   if (FLT) {
@@ -1020,22 +1022,23 @@ __device__ __forceinline__ bool encode_tile_stream_fast(const EncCtx &c, const E
     const typename F::State xs = st.x;
     const uint32_t cs = st.cursor;
     uint32_t esc = 0;
-    // integer rows and symbols: every group's bucket first, since the
-    // lookups do not depend on the state (float latents keep them beside
-    // each group: their extra registers would spill)
+    // every group's bucket first, since the lookups do not depend on the
+    // state (float latents with starts tables keep them beside each group:
+    // their extra registers would spill)
+    constexpr bool kFirst = !(FLT && ST);
     uint32_t be[GC];
-    if constexpr (!FLT) {
+    if constexpr (kFirst) {
 #pragma unroll
       for (int j = GC - 1; j >= 0; --j) {
-        const EncBucket bk =
-            enc_bucket<ST>((int32_t)rs[j * 32 + lane], meta_of(ri[j * 32 + lane]), buckets);
+        const EncBucket bk = enc_bucket<ST>(sym_of(rs[j * 32 + lane], mu[j]),
+                                            meta_of(ri[j * 32 + lane]), buckets);
         esc |= bk.in_range ? 0u : 1u;
         be[j] = bk.e;
       }
     }
 #pragma unroll
     for (int j = GC - 1; j >= 0; --j) {
-      if constexpr (FLT) {
+      if constexpr (!kFirst) {
         const EncBucket bk = enc_bucket<ST>(sym_of(rs[j * 32 + lane], mu[j]),
                                             meta_of(ri[j * 32 + lane]), buckets);
         esc |= bk.in_range ? 0u : 1u;
@@ -1543,6 +1546,22 @@ __global__ void __launch_bounds__(kScanThreads)
   if (threadIdx.x == 0 && carry_sh > capacity) report(status, RANS_ERR_CAPACITY, -1);
 }
 
+// A warp copies `words` words from src to dst with eight loads in flight
+// per lane.
+template <typename Word>
+__device__ __forceinline__ void warp_copy_words(Word *dst, const Word *src, uint64_t words) {
+  const int lane = threadIdx.x & 31;
+  uint64_t k = 0;
+  for (; k + 256 <= words; k += 256) {
+    Word v[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) v[u] = __ldg(src + k + u * 32 + lane);
+#pragma unroll
+    for (int u = 0; u < 8; ++u) dst[k + u * 32 + lane] = v[u];
+  }
+  for (uint64_t q = k + lane; q < words; q += 32) dst[q] = __ldg(src + q);
+}
+
 // Word: the format's stream word (stream lengths and offsets are multiples
 // of its size).
 template <typename Word>
@@ -1560,7 +1579,7 @@ __global__ void copy_streams_kernel(Geom g, const char *scratch, const uint64_t 
     const Word *src = reinterpret_cast<const Word *>(scratch + slot_end(g, d, s) - len);
     Word *dst = reinterpret_cast<Word *>(out + off);
     const uint64_t words = len / sizeof(Word);
-    for (uint64_t k = lane; k < words; k += 32) dst[k] = __ldg(src + k);
+    warp_copy_words(dst, src, words);
   }
 }
 
@@ -1609,7 +1628,7 @@ __global__ void __launch_bounds__(kCompactWarps * 32)
   const Word *src = reinterpret_cast<const Word *>(scratch + slot_end(g, d, s) - len);
   Word *dst = reinterpret_cast<Word *>(out + off);
   const uint64_t words = len / sizeof(Word);
-  for (uint64_t k = lane; k < words; k += 32) dst[k] = __ldg(src + k);
+  warp_copy_words(dst, src, words);
 }
 
 __global__ void debug_divide_kernel(const uint64_t *x, const uint32_t *f, int64_t n, uint64_t *q,
