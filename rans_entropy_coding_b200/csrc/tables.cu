@@ -16,6 +16,7 @@
 // buckets in (width, index) order, each drained to width 1 before the next is
 // touched, so a threshold width t and a rank among the width-t buckets decide
 // every bucket's final width.
+#include <algorithm>
 #include <cmath>
 #include <cstring>
 #include <vector>
@@ -1011,7 +1012,16 @@ int prepare_tables(const int32_t *cdfs, int K, int Lmax, const int32_t *lengths,
     }
     const int64_t left = room - (int64_t)pad16(4ull * slot_total());
     dec_smem = left >= 0;
-    if (dec_smem) chunk_words = (uint64_t)(left / 16) * 4;
+    if (dec_smem) {
+      // bitmap words: twice what these rows need (a refresh from other rows
+      // of the same lengths may need more; slots that find none left
+      // search) and at most the room left, so that small tables leave
+      // shared memory to the decoders' per-warp rings
+      uint64_t bits = 0;
+      for (int r = 0; r < K; ++r) bits += words[r] - (1ull << q[r]);
+      const uint64_t want = ((2 * bits + 256 + 3) / 4) * 4;
+      chunk_words = std::min<uint64_t>((uint64_t)(left / 16) * 4, want);
+    }
   }
   uint64_t sbase = 0;
   for (int r = 0; r < K; ++r) {
