@@ -448,11 +448,22 @@ __device__ void decode_stream_w1(const DecCtx &c, const RowMeta *meta, const uin
   const int ib = c.g.ib_shift;
   const Tile t = d.t;
   State x = (State)__ldg(words) | ((State)__ldg(words + 1) << F::kWordBits);
-  uint64_t pw = 2;
+  uint64_t pw = 2;  // words consumed
   bool bad = false;
+  // the next four words wait in registers, each loaded four refills before
+  // it is used, so that a refill does not wait on memory (loads past the
+  // stream's end read its last word; consuming past it is an error)
+  uint32_t wq[4];
+#pragma unroll
+  for (int u = 0; u < 4; ++u) wq[u] = __ldg(words + (2 + u < nw ? 2 + u : nw - 1));
   auto rd = [&]() -> uint32_t {
-    uint32_t v = 0;
-    if (pw < nw) v = __ldg(words + pw); else bad = true;
+    const uint32_t v = wq[0];
+    bad |= pw >= nw;
+    wq[0] = wq[1];
+    wq[1] = wq[2];
+    wq[2] = wq[3];
+    const uint64_t q = pw + 4;
+    wq[3] = __ldg(words + (q < nw ? q : nw - 1));
     ++pw;
     return v;
   };
@@ -490,6 +501,10 @@ __device__ void decode_stream_w1(const DecCtx &c, const RowMeta *meta, const uin
     rmean[u] = 0.0f;
     if (u < n) fetch(rrow[u], rmean[u]);
   }
+  // the row metadata of the next symbol, read one symbol ahead (clamped to
+  // the table; an out-of-range row is reported when its symbol comes)
+  const uint32_t kmax = (uint32_t)c.K - 1u;
+  RowMeta m_next = row_meta(meta, min((uint32_t)rrow[0], kmax));
   for (int32_t i = 0; i < n; ++i) {
     const int64_t p = d.base + pl.rel(t);
     pl.fwd(t, 1);
@@ -509,7 +524,8 @@ __device__ void decode_stream_w1(const DecCtx &c, const RowMeta *meta, const uin
       report(c.status, RANS_ERR_INDEX, s);
       return;
     }
-    const RowMeta m = row_meta(meta, (uint32_t)r);
+    const RowMeta m = m_next;
+    m_next = row_meta(meta, min((uint32_t)rrow[0], kmax));
     const uint32_t cum = F::cum16(x, sh);
     const uint32_t sym =
         ROWS ? search_row(cum, m, buckets) : lookup<true, false>(cum, m, buckets, slots, true);
