@@ -565,6 +565,108 @@ __device__ void decode_stream_w1(const DecCtx &c, const RowMeta *meta, const uin
   if (bad || x != F::kLow || pw != nw) report(c.status, RANS_ERR_CORRUPT, s);
 }
 
+// One state on a contiguous stream (symbol i of the stream at base + i):
+// four symbols a step, their row indexes read a step ahead and their row
+// metadata before the first of them is decoded, the stream's next words in
+// registers; the symbol step is decode_stream_w1's.
+template <class F, typename SymT, bool ROWS>
+__device__ void decode_stream_w1c(const DecCtx &c, const RowMeta *meta, const uint16_t *buckets,
+                                  const uint32_t *slots, int64_t s) {
+  using State = typename F::State;
+  using Word = typename F::Word;
+  const StreamDesc d = stream_desc(c.g, s);
+  const Word *words = nullptr;
+  uint64_t nw = 0;
+  if (!d.ok || !stream_bounds<F>(c, s, 1, words, nw)) {
+    report(c.status, d.ok ? RANS_ERR_CORRUPT : RANS_ERR_ARG, s);
+    return;
+  }
+  bulk_prefetch_l2(reinterpret_cast<const char *>(c.in),
+                   reinterpret_cast<const char *>(c.in) + c.in_bytes,
+                   reinterpret_cast<const char *>(words), sizeof(Word) * nw);
+  const uint32_t sh = F::shift(c.sh);
+  const int ib = c.g.ib_shift;
+  const int32_t n = (int32_t)d.n;
+  const int32_t *idx = c.idx;
+  const int64_t base = d.base;
+  const uint32_t kmax = (uint32_t)c.K - 1u;
+  State x = (State)__ldg(words) | ((State)__ldg(words + 1) << F::kWordBits);
+  uint64_t pw = 2;  // words consumed
+  bool bad = false;
+  uint32_t wq[4];
+#pragma unroll
+  for (int u = 0; u < 4; ++u) wq[u] = __ldg(words + (2 + u < nw ? 2 + u : nw - 1));
+  auto rd = [&]() -> uint32_t {
+    const uint32_t v = wq[0];
+    bad |= pw >= nw;
+    wq[0] = wq[1];
+    wq[1] = wq[2];
+    wq[2] = wq[3];
+    const uint64_t q = pw + 4;
+    wq[3] = __ldg(words + (q < nw ? q : nw - 1));
+    ++pw;
+    return v;
+  };
+  auto rows4 = [&](int32_t i, int32_t (&r)[4]) {
+#pragma unroll
+    for (int u = 0; u < 4; ++u) r[u] = i + u < n ? __ldg(idx + ((base + i + u) >> ib)) : 0;
+  };
+  for (int32_t q = 0; q < 64 && q < n; q += 16) prefetch_l2(idx + ((base + q) >> ib));
+  int32_t ra[4], rn[4];
+  rows4(0, ra);
+  rows4(4, rn);
+#pragma unroll 1
+  for (int32_t i = 0; i < n; i += 4) {
+    RowMeta m[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) m[u] = row_meta(meta, min((uint32_t)ra[u], kmax));
+    if ((i & 15) == 0 && i + 64 < n) prefetch_l2(idx + ((base + i + 64) >> ib));
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      if (i + u >= n) break;
+      if ((uint32_t)ra[u] >= (uint32_t)c.K) {
+        report(c.status, RANS_ERR_INDEX, s);
+        return;
+      }
+      const uint32_t cum = F::cum16(x, sh);
+      const uint32_t sym = ROWS ? search_row(cum, m[u], buckets)
+                                : lookup<true, false>(cum, m[u], buckets, slots, true);
+      const uint32_t start = buckets[m[u].bucket_base + sym];
+      const uint32_t freq = width_of(start, buckets[m[u].bucket_base + sym + 1]);
+      x = F::dec_step(x, cum, start, freq, sh);
+      if (x < F::kLow) x = (x << F::kWordBits) | rd();
+      int64_t val = (int64_t)sym;
+      if (sym == m[u].maxv) {
+        auto getbits = [&]() -> uint32_t {
+          const uint32_t v = (uint32_t)x & kBypassMax;
+          x >>= kBypassBits;
+          if (x < F::kLow) x = (x << F::kWordBits) | rd();
+          return v;
+        };
+        uint32_t v4 = getbits();
+        uint32_t nb = v4;
+        while (v4 == kBypassMax && nb <= 15) {
+          v4 = getbits();
+          nb += v4;
+        }
+        if (nb > 15) {
+          bad = true;
+          nb = 0;
+        }
+        uint64_t raw = 0;
+        for (uint32_t k = 0; k < nb; ++k) raw |= (uint64_t)getbits() << (kBypassBits * k);
+        const int64_t half = (int64_t)(raw >> 1);
+        val = (raw & 1) ? (-half - 1) : ((int64_t)m[u].maxv + half);
+      }
+      SymIO<SymT>::store(c.out, base + i + u, val + (int64_t)m[u].offset);
+    }
+#pragma unroll
+    for (int u = 0; u < 4; ++u) ra[u] = rn[u];
+    rows4(i + 8, rn);
+  }
+  if (bad || x != F::kLow || pw != nw) report(c.status, RANS_ERR_CORRUPT, s);
+}
+
 // W = 2, 4 or 8 interleaved states on W consecutive lanes of a warp, 32 / W
 // streams per warp ("torch_ans 0.3.0", Usage legend: num_interleaves 2, 4
 // and 8 map to that many consecutive lanes, sub-warp groups).  Lane l of a
@@ -1865,9 +1967,19 @@ __global__ void __launch_bounds__(W == 32 ? kDecMaxThreads32 : kDecThreads1)
                                                            stream_of(c.g, k), stab);
     }
   } else {
+    // contiguous or explicit streams of integer symbols take the four-symbol
+    // loop, tiled streams and float values the general one
+    const bool flat = !std::is_same<SymT, float>::value && c.g.kind != RANS_CHUNK_TILED;
     for (int64_t k = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; k < c.g.S;
-         k += (int64_t)gridDim.x * blockDim.x)
+         k += (int64_t)gridDim.x * blockDim.x) {
+      if constexpr (!std::is_same<SymT, float>::value) {
+        if (flat) {
+          decode_stream_w1c<F, SymT, ROWS>(c, meta, buckets, slots, stream_of(c.g, k));
+          continue;
+        }
+      }
       decode_stream_w1<F, SymT, ROWS>(c, meta, buckets, slots, stream_of(c.g, k), stab);
+    }
   }
 }
 

@@ -529,6 +529,85 @@ __device__ void encode_stream_w1(const EncCtx &c, const RowMeta *meta, const uin
   c.lens[s] = sizeof(Word) * (uint64_t)cursor;
 }
 
+// One state on a contiguous stream (symbol i at base + i), coded last to
+// first four symbols a step: the step's symbols and rows are read a step
+// ahead, and its four buckets, reciprocals and escapes are looked up before
+// the first state update (they do not depend on the state); the symbol
+// step is encode_stream_w1's.
+template <class F, typename SymT, bool ST>
+__device__ void encode_stream_w1c(const EncCtx &c, const RowMeta *meta, const uint32_t *buckets,
+                                  int64_t s) {
+  using Word = typename F::Word;
+  const StreamDesc d = stream_desc(c.g, s);
+  if (!d.ok) {
+    report(c.status, RANS_ERR_ARG, s);
+    return;
+  }
+  Word *end = reinterpret_cast<Word *>(c.scratch + slot_end(c.g, d, s));
+  const uint32_t sh = F::shift(c.sh);
+  const int ib = c.g.ib_shift;
+  const int32_t n = (int32_t)d.n;
+  const int64_t base = d.base;
+  const uint32_t kmax = (uint32_t)c.K - 1u;
+  typename F::State x = F::kLow;
+  uint32_t cursor = 0;
+  // the step that codes j, j - 1, j - 2, j - 3
+  auto load4 = [&](int32_t j, int32_t (&sv)[4], int32_t (&r)[4]) {
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int32_t p = j - u;
+      sv[u] = p >= 0 ? SymIO<SymT>::load(c.sym, base + p) : 0;
+      r[u] = p >= 0 ? __ldg(c.idx + ((base + p) >> ib)) : 0;
+    }
+  };
+  auto prefetch_at = [&](int32_t p) {
+    prefetch_l2(reinterpret_cast<const SymT *>(c.sym) + base + p);
+    prefetch_l2(c.idx + ((base + p) >> ib));
+  };
+  for (int32_t q = n - 1; q >= 0 && q >= n - 64; q -= 16) prefetch_at(q);
+  int32_t sa[4], ra[4], sn[4], rn[4];
+  load4(n - 1, sa, ra);
+  load4(n - 5, sn, rn);
+#pragma unroll 1
+  for (int32_t j = n - 1; j >= 0; j -= 4) {
+    uint32_t st4[4], fr4[4];
+    uint64_t raw4[4];
+    bool esc4[4];
+    double rcp4[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      map_symbol<ST>(sa[u], row_meta(meta, min((uint32_t)ra[u], kmax)), buckets, st4[u], fr4[u],
+                     raw4[u], esc4[u]);
+      rcp4[u] = F::rcp(fr4[u], sh);
+    }
+    if (((n - 1 - j) & 15) == 0 && j - 64 >= 0) prefetch_at(j - 64);
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      if (j - u < 0) break;
+      if ((uint32_t)ra[u] >= (uint32_t)c.K) {
+        report(c.status, RANS_ERR_INDEX, s);
+        return;
+      }
+      if (esc4[u] && (raw4[u] >> 60) != 0) {
+        report(c.status, RANS_ERR_RANGE, s);
+        return;
+      }
+      cursor +=
+          symbol_ops<F, true>(x, st4[u], fr4[u], rcp4[u], raw4[u], esc4[u], end, cursor, sh);
+    }
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      sa[u] = sn[u];
+      ra[u] = rn[u];
+    }
+    load4(j - 8, sn, rn);
+  }
+  end[-1 - (int64_t)cursor] = (Word)(x >> F::kWordBits);
+  end[-2 - (int64_t)cursor] = (Word)x;
+  cursor += 2;
+  c.lens[s] = sizeof(Word) * (uint64_t)cursor;
+}
+
 // W = 2, 4 or 8 interleaved states on W consecutive lanes of a warp, 32 / W
 // streams per warp (the sub-warp groups of "torch_ans 0.3.0", Usage legend).
 // Lane l of a segment holds state l and codes symbols l, l + W, ... in
@@ -1456,9 +1535,19 @@ __global__ void __launch_bounds__(W == 32 ? kEncThreads32 : kEncThreads1)
       encode_stream_w32_entry<F, SymT, IB0, FLT, ST>(c, meta, buckets, stg, stream_of(c.g, k),
                                                      stab);
   } else {
+    // contiguous or explicit streams of integer symbols take the four-symbol
+    // loop, tiled streams and float latents the general one
+    const bool flat = !FLT && c.g.kind != RANS_CHUNK_TILED;
     for (int64_t k = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; k < c.g.S;
-         k += (int64_t)gridDim.x * blockDim.x)
+         k += (int64_t)gridDim.x * blockDim.x) {
+      if constexpr (!FLT) {
+        if (flat) {
+          encode_stream_w1c<F, SymT, ST>(c, meta, buckets, stream_of(c.g, k));
+          continue;
+        }
+      }
       encode_stream_w1<F, SymT, FLT, ST>(c, meta, buckets, stream_of(c.g, k), stab);
+    }
   }
 }
 
