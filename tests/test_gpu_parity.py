@@ -346,6 +346,35 @@ def test_decoder_reports_corrupt_streams(W):
     assert _decode_status(w, tables, data, offs, bad) == rb.ERR_INDEX
 
 
+@pytest.mark.parametrize("kind", ["tile", "chunk"])
+def test_staged_coders_report_errors(kind):
+    """The tile-staged coders (tiled streams) and the chunked coders
+    (contiguous streams of whole 256-symbol chunks) record a row index out of
+    range (encoder and decoder) and corrupt streams, like the general ones."""
+    if kind == "tile":
+        w = WL.y_batch(n_images=1)
+        w["W"] = 32
+    else:
+        w = WL.sweep(log2_n=16, n_streams=8, block=256)
+        w["symbols"] = np.asarray(w["symbols"]).astype(np.int32)
+    tables, data, offs = _coded(w)
+    assert _decode_status(w, tables, data, offs) == rb.OK
+    o2 = offs.copy()
+    o2[4:] -= 4
+    d2 = np.concatenate([data[:int(offs[4]) - 4], data[int(offs[4]):]])
+    assert _decode_status(w, tables, d2, o2) == rb.ERR_CORRUPT
+    d3 = data.copy()
+    d3[int(offs[5]) + 300] ^= 0x5A
+    assert _decode_status(w, tables, d3, offs) == rb.ERR_CORRUPT
+    bad = np.asarray(w["indexes"]).copy()
+    bad[min(777, bad.size - 1)] = 1000
+    assert _decode_status(w, tables, data, offs, bad) == rb.ERR_INDEX
+    sym = torch.from_numpy(np.ascontiguousarray(w["symbols"]).reshape(-1)).cuda()
+    _, _, ws = rb.encode_with_indexes(sym, torch.from_numpy(bad.astype(np.int32)).cuda(), tables,
+                                      chunking_of(w))
+    assert rb.rans_get_status(ws.enc) == rb.ERR_INDEX
+
+
 def test_encoder_reports_bad_index_and_capacity():
     w = WL.y_latent(W=32)
     c, l, o = oracle_tables(w)
