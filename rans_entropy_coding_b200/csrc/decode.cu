@@ -1788,7 +1788,7 @@ __global__ void __launch_bounds__(kChunkMaxWarps * 32, 1) decode_chunk_kernel(De
   const uint16_t *starts = reinterpret_cast<const uint16_t *>(smem + c.meta_bytes);
   const uint32_t *slots = reinterpret_cast<const uint32_t *>(smem + c.meta_bytes + c.start_bytes);
   const uint32_t tab = c.meta_bytes + c.start_bytes + c.slot_bytes;
-  const int warp = threadIdx.x >> 5, nwarp = blockDim.x >> 5, lane = threadIdx.x & 31;
+  const int warp = threadIdx.x >> 5, nwarp = blockDim.x >> 5;
   // each warp's word window and value ring, 128-byte aligned
   const uint32_t sbase = smem_addr(smem);
   const uint32_t wbase = ((sbase + tab + 127u) & ~127u) + (uint32_t)warp * chunk_warp_bytes<SymT>();
@@ -1803,7 +1803,6 @@ __global__ void __launch_bounds__(kChunkMaxWarps * 32, 1) decode_chunk_kernel(De
     else
       decode_chunk_stream<SymT, false>(c, meta, starts, slots, win, oring, k);
   }
-  (void)lane;
   if ((threadIdx.x & 31) == 0) tma::bulk_wait_all();
 }
 
