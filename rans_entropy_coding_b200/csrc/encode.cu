@@ -1102,27 +1102,17 @@ __device__ __forceinline__ bool encode_tile_stream_fast(const EncCtx &c, const E
     const uint32_t cs = st.cursor;
     uint32_t esc = 0;
     // every group's bucket first, since the lookups do not depend on the
-    // state (float latents with starts tables keep them beside each group:
-    // their extra registers would spill)
-    constexpr bool kFirst = !(FLT && ST);
+    // state
     uint32_t be[GC];
-    if constexpr (kFirst) {
 #pragma unroll
-      for (int j = GC - 1; j >= 0; --j) {
-        const EncBucket bk = enc_bucket<ST>(sym_of(rs[j * 32 + lane], mu[j]),
-                                            meta_of(ri[j * 32 + lane]), buckets);
-        esc |= bk.in_range ? 0u : 1u;
-        be[j] = bk.e;
-      }
+    for (int j = GC - 1; j >= 0; --j) {
+      const EncBucket bk = enc_bucket<ST>(sym_of(rs[j * 32 + lane], mu[j]),
+                                          meta_of(ri[j * 32 + lane]), buckets);
+      esc |= bk.in_range ? 0u : 1u;
+      be[j] = bk.e;
     }
 #pragma unroll
     for (int j = GC - 1; j >= 0; --j) {
-      if constexpr (!kFirst) {
-        const EncBucket bk = enc_bucket<ST>(sym_of(rs[j * 32 + lane], mu[j]),
-                                            meta_of(ri[j * 32 + lane]), buckets);
-        esc |= bk.in_range ? 0u : 1u;
-        be[j] = bk.e;
-      }
       EncLook L;
       L.start = bucket_start(be[j]);
       L.freq = bucket_freq(be[j]);
@@ -1163,8 +1153,12 @@ __device__ __forceinline__ bool encode_tile_stream_fast(const EncCtx &c, const E
   return true;
 }
 
+// Float latents: at most 16 warps a CTA, so that the extra per-element work
+// (the row and the symbol of each scale and y) has registers to spare.
+constexpr int kEncFltMaxWarps = 16;
+
 template <class F, bool ST, bool FLT>
-__global__ void __launch_bounds__(kEncThreads32)
+__global__ void __launch_bounds__(FLT ? kEncFltMaxWarps * 32 : kEncThreads32, 1)
     encode_tile_kernel(EncCtx c, const __grid_constant__ EncTileMaps maps) {
   extern __shared__ __align__(16) unsigned char smem[];
   __shared__ uint64_t bar;
@@ -1429,7 +1423,8 @@ int launch_encode_tile(const EncCtx &c, int mode, const int32_t *indexes, const 
   }
   const int sms = num_sms(dev);
   int64_t warps = (g.S + sms - 1) / sms;
-  if (warps > kEncMaxWarps) warps = kEncMaxWarps;
+  const int64_t max_warps = FLT ? kEncFltMaxWarps : kEncMaxWarps;
+  if (warps > max_warps) warps = max_warps;
   const int64_t room = ((int64_t)lim - tab - 128) / kEncTileRingBytes;
   if (warps > room) warps = room;
   if (warps < 1) warps = 1;
