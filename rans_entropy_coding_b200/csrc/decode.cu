@@ -1650,8 +1650,9 @@ __global__ void __launch_bounds__(kTileMaxStreams * 32, 1)
                                      (uint32_t)nwarp * kTileStreamBytes);
     for (int i = threadIdx.x; i < c.K; i += blockDim.x) stab[i] = c.stab[i];
     __syncthreads();
-    use_keys = build_scale_keys(stab, c.K, reinterpret_cast<uint8_t *>(stab) + pad16(4ull * c.K),
-                                keys);
+    use_keys = build_scale_keys(
+        stab, c.K, c.bound,
+        reinterpret_cast<uint16_t *>(reinterpret_cast<char *>(stab) + pad16(4ull * c.K)), keys);
   }
   if (lane == 0) {
     tma::mbar_init(bar0, 1);

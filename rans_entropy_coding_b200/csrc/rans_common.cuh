@@ -396,41 +396,45 @@ __device__ __forceinline__ float bound_scale(float s, float bound) {
 }
 
 // The same rows without a search, for tables of 2 to 64 strictly increasing,
-// positive, finite entries (the first K - 1 counted): positive floats order
-// like their bit patterns, so key(s) = bits(s) >> shift is monotone, and
-// with the shift chosen so that no two counted entries share a key, the
-// entries below s are cnt[key(s)] (those of smaller keys) plus the one entry
-// of s's own key if it is below s.  cnt, one byte per key from the first
-// entry's key to one past the last one's, lives in shared memory; a scale
-// that is not positive (or NaN) has row 0, as in the search.
-constexpr uint32_t kScaleKeyBytes = 1024;
+// positive, finite entries (the first K - 1 counted) and a positive bound:
+// positive floats order like their bit patterns, so key(s) = bits(s) >>
+// shift is monotone, and with the shift chosen so that no two counted
+// entries share a key, the entries below s are cnt[key(s)] (those of smaller
+// keys) plus the one entry of s's own key if it is below s.  The counts of
+// key k and k + 1 sit side by side in one 16-bit word (cnt2[k]), one word per
+// key from the first entry's key to one past the last one's, in shared
+// memory.  With a positive bound every scale the coders look up is positive
+// (NaN counts as the bound).
+constexpr uint32_t kScaleKeyWords = 1024;
+constexpr uint32_t kScaleKeyBytes = 2 * kScaleKeyWords;
 
 struct ScaleKeys {
-  const uint8_t *cnt;
+  const uint16_t *cnt2;
   const float *tab;
   uint32_t shift, kmin;
   int32_t nk1;  // last valid key index
+  // s > 0 (a scale raised to the positive bound)
   __device__ __forceinline__ uint32_t row(float s) const {
     int32_t k = (int32_t)(__float_as_uint(s) >> shift) - (int32_t)kmin;
     k = min(max(k, 0), nk1);
-    const uint32_t c = cnt[k], c1 = cnt[k + 1];
-    const uint32_t r = c + ((c1 > c && tab[c] < s) ? 1u : 0u);
-    return s > 0.0f ? r : 0u;
+    const uint32_t w = cnt2[k];
+    const uint32_t c = w & 0xffu, c1 = w >> 8;
+    return c + ((c1 > c && tab[c] < s) ? 1u : 0u);
   }
 };
 
-// Builds the key counts for the K-entry table tab (shared memory) into cnt
+// Builds the key counts for the K-entry table tab (shared memory) into cnt2
 // (kScaleKeyBytes of shared memory); every thread of the block calls it
-// (two barriers) and gets the same answer: false when the table does not
-// qualify, and the coder then searches.
-__device__ __forceinline__ bool build_scale_keys(const float *tab, int K, uint8_t *cnt,
-                                                 ScaleKeys &keys) {
-  bool ok = K >= 2 && K <= 64;
+// (two barriers) and gets the same answer: false when the table or the
+// bound does not qualify, and the coder then searches.
+__device__ __forceinline__ bool build_scale_keys(const float *tab, int K, float bound,
+                                                 uint16_t *cnt2, ScaleKeys &keys) {
+  bool ok = K >= 2 && K <= 64 && bound > 0.0f;
   const float t0 = ok ? tab[0] : 1.0f, tl = ok ? tab[K - 2] : 1.0f;
   ok = ok && t0 > 0.0f && tl < INFINITY;
   const uint32_t b0 = __float_as_uint(t0), bl = __float_as_uint(tl);
   uint32_t shift = 0;
-  while (shift < 31 && ((bl - b0) >> shift) + 2u > kScaleKeyBytes - 1u) ++shift;
+  while (shift < 31 && ((bl - b0) >> shift) + 2u > kScaleKeyWords - 1u) ++shift;
   const uint32_t kmin = b0 >> shift;
   const uint32_t nkeys = ok ? (bl >> shift) - kmin + 2u : 0u;
   for (int i = threadIdx.x; ok && i < K - 2; i += blockDim.x) {
@@ -439,14 +443,18 @@ __device__ __forceinline__ bool build_scale_keys(const float *tab, int K, uint8_
   }
   ok = __syncthreads_and(ok) != 0;
   if (ok) {
-    for (uint32_t k = threadIdx.x; k <= nkeys; k += blockDim.x) {
-      uint32_t n = 0;
-      for (int i = 0; i <= K - 2; ++i) n += (__float_as_uint(tab[i]) >> shift) < kmin + k;
-      cnt[k] = (uint8_t)n;
+    for (uint32_t k = threadIdx.x; k < nkeys; k += blockDim.x) {
+      uint32_t n0 = 0, n1 = 0;
+      for (int i = 0; i <= K - 2; ++i) {
+        const uint32_t ki = __float_as_uint(tab[i]) >> shift;
+        n0 += ki < kmin + k;
+        n1 += ki < kmin + k + 1;
+      }
+      cnt2[k] = (uint16_t)(n0 | (n1 << 8));
     }
   }
   __syncthreads();
-  keys.cnt = cnt;
+  keys.cnt2 = cnt2;
   keys.tab = tab;
   keys.shift = shift;
   keys.kmin = kmin;

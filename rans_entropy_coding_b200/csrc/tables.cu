@@ -768,13 +768,13 @@ __global__ void __launch_bounds__(256)
 __global__ void build_indexes_kernel(const float *scales, int64_t n, const float *table, int K,
                                      float bound, int32_t *indexes) {
   __shared__ float stab[64];
-  __shared__ uint8_t cnt[kScaleKeyBytes];
+  __shared__ uint16_t cnt[kScaleKeyWords];
   ScaleKeys keys{};
   bool use_keys = false;
   if (K <= 64) {  // (uniform: every thread takes the same branch)
     for (int i = threadIdx.x; i < K; i += blockDim.x) stab[i] = table[i];
     __syncthreads();
-    use_keys = build_scale_keys(stab, K, cnt, keys);
+    use_keys = build_scale_keys(stab, K, bound, cnt, keys);
   }
   for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n;
        i += (int64_t)gridDim.x * blockDim.x) {
