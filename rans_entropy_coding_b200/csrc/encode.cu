@@ -1631,20 +1631,31 @@ __global__ void __launch_bounds__(kScanThreads)
   if (threadIdx.x == 0 && carry_sh > capacity) report(status, RANS_ERR_CAPACITY, -1);
 }
 
-// A warp copies `words` words from src to dst with eight loads in flight
+// A warp copies `words` words from src to dst with sixteen loads in flight
 // per lane.
 template <typename Word>
 __device__ __forceinline__ void warp_copy_words(Word *dst, const Word *src, uint64_t words) {
   const int lane = threadIdx.x & 31;
   uint64_t k = 0;
-  for (; k + 256 <= words; k += 256) {
-    Word v[8];
+  for (; k + 512 <= words; k += 512) {
+    Word v[16];
 #pragma unroll
-    for (int u = 0; u < 8; ++u) v[u] = __ldg(src + k + u * 32 + lane);
+    for (int u = 0; u < 16; ++u) v[u] = __ldg(src + k + u * 32 + lane);
 #pragma unroll
-    for (int u = 0; u < 8; ++u) dst[k + u * 32 + lane] = v[u];
+    for (int u = 0; u < 16; ++u) dst[k + u * 32 + lane] = v[u];
   }
-  for (uint64_t q = k + lane; q < words; q += 32) dst[q] = __ldg(src + q);
+  // the tail: every load first, then every store
+  Word v[16];
+#pragma unroll
+  for (int u = 0; u < 16; ++u) {
+    const uint64_t q = k + u * 32 + lane;
+    v[u] = q < words ? __ldg(src + q) : Word(0);
+  }
+#pragma unroll
+  for (int u = 0; u < 16; ++u) {
+    const uint64_t q = k + u * 32 + lane;
+    if (q < words) dst[q] = v[u];
+  }
 }
 
 // Word: the format's stream word (stream lengths and offsets are multiples
@@ -1685,9 +1696,13 @@ __global__ void __launch_bounds__(kCompactWarps * 32)
   __shared__ unsigned long long own[kCompactWarps];
   const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
   const int64_t s0 = (int64_t)blockIdx.x * kCompactWarps;
-  // the lengths of streams [0, s0)
+  // the lengths of streams [0, s0), four loads in flight per thread
   unsigned long long before = 0;
-  for (int64_t i = threadIdx.x; i < s0; i += blockDim.x) before += lens[i];
+  int64_t i = threadIdx.x;
+  for (; i + 3 * (int64_t)blockDim.x < s0; i += 4 * (int64_t)blockDim.x)
+    before += __ldg(lens + i) + __ldg(lens + i + blockDim.x) + __ldg(lens + i + 2 * blockDim.x) +
+              __ldg(lens + i + 3 * blockDim.x);
+  for (; i < s0; i += blockDim.x) before += __ldg(lens + i);
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) before += __shfl_xor_sync(kFull, before, o);
   if (lane == 0) part[wid] = before;
