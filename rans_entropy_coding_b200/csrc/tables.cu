@@ -476,13 +476,22 @@ __device__ void fill_slot_block(const int32_t *row, int nb, uint32_t slot0, int 
   const uint32_t nch = w > 16 ? (uint32_t)(w >> 4) : 1u;  // bitmap words of a slot
   int lo[SPT], hi[SPT];
   uint32_t need = 0;
+  // lo: the bucket holding the slot's first value, one search per slot;
+  // hi, the bucket holding its last value, is the next slot's lo (the next
+  // lane's), less one when a bucket starts exactly at the next slot
 #pragma unroll
   for (int u = 0; u < SPT; ++u) {
     const int t = t0 + u * (int)blockDim.x;
-    lo[u] = hi[u] = 0;
+    lo[u] = t < nslots ? bucket_of(row, nb, t * w, sh) : 0;
+  }
+#pragma unroll
+  for (int u = 0; u < SPT; ++u) {
+    const int t = t0 + u * (int)blockDim.x;
+    int next = __shfl_down_sync(kFull, lo[u], 1);
+    if (lane == 31 && t + 1 < nslots) next = bucket_of(row, nb, (t + 1) * w, sh);
+    hi[u] = 0;
     if (t < nslots) {
-      lo[u] = bucket_of(row, nb, t * w, sh);
-      hi[u] = bucket_of(row, nb, t * w + w - 1, sh);
+      hi[u] = t + 1 >= nslots ? nb - 1 : ((row[next] << sh) == (t + 1) * w ? next - 1 : next);
       if (hi[u] - lo[u] >= 3) need += nch;
     }
   }
