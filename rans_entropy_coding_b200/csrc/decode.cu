@@ -16,21 +16,25 @@
 //    x < 2^16 (the F template parameter: Rans64 / Rans32 in rans_common.cuh;
 //    the tables hold 16-bit-scaled entries, so the lookup takes cum << sh);
 //  * W = 32: one warp per stream, lane = symbol index mod 32; refills take
-//    the next words of the shared stream in lane order (ballot + popc),
-//    served from a two-window register buffer of 64 prefetched words
+//    the next words of the shared stream in lane order (ballot + popc)
 //    ("torch_ans 0.3.0", Usage legend: warp renormalisation with one shared
-//    cursor);
+//    cursor), served from a 512-word ring in shared memory refilled by
+//    cp.async (the 64-bit format's tile and chunk decoders) or from a
+//    register buffer of 64 prefetched words (the others);
 //  * escapes run off the fast path: lanes proceed one by one in ascending
 //    order, reading their bypass pieces, since how many words a lane takes
 //    depends on what it reads ("torch_ans 0.3.0", Performance Tuning, GPU
 //    item 5: the bypass phase is sequential across the lanes and skipped by a
 //    group ballot).  The group is first decoded as if nothing escaped; the
 //    ballot, taken beside the refill, sends it down the slow path.
-//  Latency: row indexes stream through a per-warp shared-memory ring filled
-//  with cp.async kDecStage - 1 groups ahead, the next group's row metadata
-//  is read while this group decodes, and each stream's words are bulk
-//  prefetched into L2 when the warp starts it.
-//  Tables are staged into shared memory with bulk copies when they fit.
+//  Staging: tiled streams move their row indexes in and their values out as
+//  tensor-tile copies (decode_tile_kernel), contiguous streams of whole
+//  256-symbol chunks with a row per chunk their values out as bulk copies
+//  (decode_chunk_kernel); the general kernel streams row indexes through a
+//  per-warp shared-memory ring filled with cp.async kDecStage - 1 groups
+//  ahead.  Each stream's words are bulk prefetched into L2 when the warp
+//  starts it, and tables are staged into shared memory with bulk copies
+//  when they fit.
 #include <type_traits>
 
 #include <cuda.h>  // CUtensorMap

@@ -1,7 +1,11 @@
 // encode.cu -- encode_with_indexes: every stream is coded in reverse symbol
 // order into a worst-case scratch slot (words written downward, the way a
 // ryg_rans encoder fills its buffer from the end), then the streams are
-// compacted behind a device prefix scan.
+// compacted behind a device prefix scan.  Tiled streams take their row
+// indexes and symbols in as tensor-tile copies (encode_tile_kernel),
+// contiguous streams of whole 256-symbol chunks with a row per chunk their
+// symbols as 16-byte cp.async copies (encode_chunk_kernel); the general
+// kernel streams both through a per-warp cp.async ring.
 //
 //  * value mapping and escape ("torch_ans 0.3.0", Low-level API, rans_push:
 //    coded range [offset, offset + cdf_size - 2), zig-zag raw value, bypass
