@@ -617,7 +617,10 @@ def run_ours(args, world, rank, local):
                "single_thread": {"value": ns1 / ts1 / 1e9, "unit": UNIT,
                                  "sample": "the first %d streams on one thread" % ms1}}
 
-    launches_per_step = 1 + 1 + 3 + 1   # rows, table refresh, enc+scan+copy, dec
+    # our kernels per step: the table rebuild (one fused kernel for a scale
+    # table; rows + refresh for pmfs), the coder and its compaction (one
+    # kernel up to 65,536 streams, scan + copy above), the decoder
+    launches_per_step = (1 if "scales" in w else 2) + (2 if S <= 65536 else 3) + 1
     if rank == 0:
         line = {
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
@@ -759,7 +762,7 @@ def run_float(args, world, rank, local):
             "roofline": {"bound": "hbm", "achieved": ach, "peak": peak, "unit": "GB/s",
                          "frac": ach / peak, "traffic": None, "kernel": dominant},
             "cpu_baseline": cpu, "e2e": None, "clocks": clk.summary(),
-            "gpu_launches": 6 * args.steps,
+            "gpu_launches": (1 + (2 if S <= 65536 else 3) + 1) * args.steps,
         }), flush=True)
 
 
