@@ -1685,16 +1685,19 @@ __global__ void __launch_bounds__(kTileMaxStreams * 32, 1)
 // values go to a two-half ring in shared memory and out with one bulk store.
 constexpr int kChunkSyms = 256;
 
-template <typename SymT>
+// PER: one row index per symbol, staged through a two-half ring with the
+// chunk's values (else one per chunk, read directly).
+template <typename SymT, bool PER>
 __host__ __device__ constexpr uint32_t chunk_warp_bytes() {
-  return kWinBytes + 2u * (uint32_t)kChunkSyms * (uint32_t)sizeof(SymT);
+  return kWinBytes + 2u * (uint32_t)kChunkSyms * (uint32_t)sizeof(SymT) +
+         (PER ? 2u * (uint32_t)kChunkSyms * 4u : 0u);
 }
 
-template <typename SymT, bool SEARCH>
+template <typename SymT, bool SEARCH, bool PER>
 __device__ __forceinline__ void decode_chunk_stream(const DecCtx &c, const RowMeta *meta,
                                                     const uint16_t *starts,
                                                     const uint32_t *slots, uint32_t *win,
-                                                    SymT *oring, int64_t s) {
+                                                    SymT *oring, int32_t *iring, int64_t s) {
   constexpr int GC = kChunkSyms / 32;
   const int lane = threadIdx.x & 31;
   const Geom &g = c.g;
@@ -1718,27 +1721,63 @@ __device__ __forceinline__ void decode_chunk_stream(const DecCtx &c, const RowMe
   uint64_t x = (uint64_t)__ldg(words + 2 * lane) | ((uint64_t)__ldg(words + 2 * lane + 1) << 32);
   uint32_t rd = 64, ldn = 64, rmax = 0;
   bool bad = false;
-  uint32_t r_next = (uint32_t)__ldg(c.idx + (d.base >> ib));
+  // PER: chunk k's row indexes into index ring half k & 1 (16-byte copies,
+  // one commit group per call, possibly empty)
+  auto rows_in = [&](int32_t k) {
+    if (k < M) {
+      const int32_t *src = c.idx + d.base + (int64_t)k * kChunkSyms;
+      int32_t *dst = iring + (k & 1) * kChunkSyms;
+#pragma unroll
+      for (int o = lane * 4; o < kChunkSyms; o += 128) cp_async16(dst + o, src + o);
+    }
+    cp_async_commit();
+  };
+  if (PER) rows_in(0);
+  uint32_t r_next = PER ? 0u : (uint32_t)__ldg(c.idx + (d.base >> ib));
 #pragma unroll 1
   for (int32_t k = 0; k < M; ++k) {
     const int h = k & 1;
-    const uint32_t r = r_next;
-    if (k + 1 < M) r_next = (uint32_t)__ldg(c.idx + ((d.base + (int64_t)(k + 1) * kChunkSyms) >> ib));
-    rmax = max(rmax, r);
-    const RowMeta m = row_meta(meta, min(r, kmax));
-    // the word window (as the tile decoder's); the ring half of this chunk's
-    // values, once chunk k - 2's store has read it
+    RowMeta ms[GC];
+    if (!PER) {
+      const uint32_t r = r_next;
+      if (k + 1 < M)
+        r_next = (uint32_t)__ldg(c.idx + ((d.base + (int64_t)(k + 1) * kChunkSyms) >> ib));
+      rmax = max(rmax, r);
+      const RowMeta m = row_meta(meta, min(r, kmax));
+#pragma unroll
+      for (int j = 0; j < GC; ++j) ms[j] = m;
+    }
+    // PER: chunk k + 1's rows on their way; the word window (as the tile
+    // decoder's); then the rows of chunk k and the blocks read before this
+    // chunk have landed (the two newest commit groups may still be in flight)
+    if (PER) rows_in(k + 1);
     const bool ahead = rd + 32u * GC <= ldn;
     win_refill(win, words, nw, rd, ldn);
-    if (ahead) cp_async_wait<1>(); else cp_async_wait<0>();
+    if (ahead) {
+      if (PER) cp_async_wait<2>(); else cp_async_wait<1>();
+    } else {
+      cp_async_wait<0>();
+    }
+    // the ring half of this chunk's values, once chunk k - 2's store has read
+    // it
     tma::bulk_wait_read1_if(l0);
     __syncwarp();
+    if (PER) {
+      const int32_t *rk = iring + h * kChunkSyms;
+#pragma unroll
+      for (int j = 0; j < GC; ++j) {
+        const uint32_t r = (uint32_t)rk[j * 32 + lane];
+        rmax = max(rmax, r);
+        ms[j] = row_meta(meta, min(r, kmax));
+      }
+    }
     const uint64_t xs = x;
     const uint32_t rds = rd;
     uint32_t esc = 0;
     int32_t val[GC];
 #pragma unroll
-    for (int j = 0; j < GC; ++j) val[j] = dec_group_win64<SEARCH>(x, rd, m, starts, slots, win, esc);
+    for (int j = 0; j < GC; ++j)
+      val[j] = dec_group_win64<SEARCH>(x, rd, ms[j], starts, slots, win, esc);
     SymT *oh = oring + h * kChunkSyms;
     if (!__any_sync(kFull, esc != 0)) {
 #pragma unroll
@@ -1754,9 +1793,13 @@ __device__ __forceinline__ void decode_chunk_stream(const DecCtx &c, const RowMe
       w.bad = false;
       load_window(w, words, nw);
 #pragma unroll 1
-      for (int j = 0; j < GC; ++j)
+      for (int j = 0; j < GC; ++j) {
+        RowMeta mj = ms[0];
+#pragma unroll
+        for (int q = 1; q < GC; ++q) mj = q == j ? ms[q] : mj;
         oh[j * 32 + lane] =
-            (SymT)dec_group_val<Rans64, SEARCH>(w, m, starts, slots, words, nw, 0u);
+            (SymT)dec_group_val<Rans64, SEARCH>(w, mj, starts, slots, words, nw, 0u);
+      }
       bad = bad || w.bad;
       x = w.x;
       rd = (uint32_t)(w.cur + w.off);
@@ -1781,8 +1824,13 @@ __device__ __forceinline__ void decode_chunk_stream(const DecCtx &c, const RowMe
 
 constexpr int kChunkMaxWarps = 32;  // a 2^28-symbol sweep's 8,192 streams in two rounds
 
-template <typename SymT>
-__global__ void __launch_bounds__(kChunkMaxWarps * 32, 1) decode_chunk_kernel(DecCtx c) {
+// (per-symbol rows: at most 16 warps, so that the chunk's eight row
+// metadata fit in registers)
+constexpr int kChunkPerMaxWarps = 16;
+
+template <typename SymT, bool PER>
+__global__ void __launch_bounds__((PER ? kChunkPerMaxWarps : kChunkMaxWarps) * 32, 1)
+    decode_chunk_kernel(DecCtx c) {
   extern __shared__ __align__(16) unsigned char smem[];
   __shared__ uint64_t bar;
   const char *gb = c.blob + kHeaderBytes;
@@ -1796,17 +1844,20 @@ __global__ void __launch_bounds__(kChunkMaxWarps * 32, 1) decode_chunk_kernel(De
   const int warp = threadIdx.x >> 5, nwarp = blockDim.x >> 5;
   // each warp's word window and value ring, 128-byte aligned
   const uint32_t sbase = smem_addr(smem);
-  const uint32_t wbase = ((sbase + tab + 127u) & ~127u) + (uint32_t)warp * chunk_warp_bytes<SymT>();
+  const uint32_t wbase =
+      ((sbase + tab + 127u) & ~127u) + (uint32_t)warp * chunk_warp_bytes<SymT, PER>();
   uint32_t *win = reinterpret_cast<uint32_t *>(smem + (wbase - sbase));
   SymT *oring = reinterpret_cast<SymT *>(smem + (wbase - sbase) + kWinBytes);
+  int32_t *iring = reinterpret_cast<int32_t *>(smem + (wbase - sbase) + kWinBytes +
+                                               2u * kChunkSyms * sizeof(SymT));
   // slots that ran out of bitmap room (flagged in the blob header) search
   const bool search = reinterpret_cast<const uint32_t *>(c.blob)[kSearchFlagWord] != 0;
   for (int64_t k = blockIdx.x + (int64_t)gridDim.x * warp; k < c.g.S;
        k += (int64_t)gridDim.x * nwarp) {
     if (search)
-      decode_chunk_stream<SymT, true>(c, meta, starts, slots, win, oring, k);
+      decode_chunk_stream<SymT, true, PER>(c, meta, starts, slots, win, oring, iring, k);
     else
-      decode_chunk_stream<SymT, false>(c, meta, starts, slots, win, oring, k);
+      decode_chunk_stream<SymT, false, PER>(c, meta, starts, slots, win, oring, iring, k);
   }
   if ((threadIdx.x & 31) == 0) tma::bulk_wait_all();
 }
@@ -1883,8 +1934,9 @@ int launch_decode_tile(const DecCtx &c, const void *indexes, void *symbols, cuda
 bool chunk_path_ok(const DecCtx &c, int mode, int sym_dtype, const void *symbols) {
   const Geom &g = c.g;
   if (g.kind != RANS_CHUNK_CONTIG || g.W != 32 || g.alias || g.fmt != RANS_FMT_RANS64 ||
-      mode != 1 || g.ib_shift < 8)
+      mode != 1 || (g.ib_shift != 0 && g.ib_shift < 8))
     return false;
+  if (g.ib_shift == 0 && (reinterpret_cast<uintptr_t>(c.idx) & 15) != 0) return false;
   if (sym_dtype != RANS_SYM_UINT8 && sym_dtype != RANS_SYM_INT16 && sym_dtype != RANS_SYM_INT32)
     return false;
   if (g.per < kChunkSyms || g.per % kChunkSyms != 0 || g.per > (int64_t(1) << 28) ||
@@ -1893,23 +1945,24 @@ bool chunk_path_ok(const DecCtx &c, int mode, int sym_dtype, const void *symbols
   return (reinterpret_cast<uintptr_t>(symbols) & 15) == 0;
 }
 
-template <typename SymT>
+template <typename SymT, bool PER>
 int launch_decode_chunk(const DecCtx &c, cudaStream_t st) {
   const Geom &g = c.g;
   int dev = 0;
   cudaGetDevice(&dev);
   const uint32_t tab = dec_table_bytes(1, c);
-  const uint32_t per_warp = chunk_warp_bytes<SymT>();
+  const uint32_t per_warp = chunk_warp_bytes<SymT, PER>();
   const uint32_t lim = (uint32_t)smem_optin(dev) - 64u;
   if (tab + 128u + per_warp > lim) return kNotTaken;
   const int sms = num_sms(dev);
   int64_t warps = (g.S + sms - 1) / sms;
-  if (warps > kChunkMaxWarps) warps = kChunkMaxWarps;
+  const int64_t max_warps = PER ? kChunkPerMaxWarps : kChunkMaxWarps;
+  if (warps > max_warps) warps = max_warps;
   const int64_t room = ((int64_t)lim - tab - 128) / per_warp;
   if (warps > room) warps = room;
   if (warps < 1) warps = 1;
   const uint32_t smem = tab + 128u + (uint32_t)warps * per_warp;
-  auto kern = decode_chunk_kernel<SymT>;
+  auto kern = decode_chunk_kernel<SymT, PER>;
   if (ensure_dyn_smem((const void *)kern, smem) != cudaSuccess) return RANS_ERR_CUDA;
   int fit = 0;
   if (blocks_per_sm(&fit, (const void *)kern, (int)warps * 32, smem) != cudaSuccess || fit < 1)
@@ -2193,9 +2246,15 @@ int launch_decode(const uint8_t *in, uint64_t in_bytes, const uint64_t *offsets,
   c.stab_smem = 0;
   const int mode = t.dec_in_smem;
   if (chunk_path_ok(c, mode, sym_dtype, symbols)) {
-    const int r = sym_dtype == RANS_SYM_UINT8   ? launch_decode_chunk<uint8_t>(c, st)
-                  : sym_dtype == RANS_SYM_INT16 ? launch_decode_chunk<int16_t>(c, st)
-                                                : launch_decode_chunk<int32_t>(c, st);
+    const bool per = g.ib_shift == 0;
+    const int r = sym_dtype == RANS_SYM_UINT8
+                      ? (per ? launch_decode_chunk<uint8_t, true>(c, st)
+                             : launch_decode_chunk<uint8_t, false>(c, st))
+                  : sym_dtype == RANS_SYM_INT16
+                      ? (per ? launch_decode_chunk<int16_t, true>(c, st)
+                             : launch_decode_chunk<int16_t, false>(c, st))
+                      : (per ? launch_decode_chunk<int32_t, true>(c, st)
+                             : launch_decode_chunk<int32_t, false>(c, st));
     if (r != kNotTaken) return r;
   }
   if (tile_path_ok(c, mode, sym_dtype, indexes, symbols)) {

@@ -1246,10 +1246,12 @@ __global__ void __launch_bounds__(FLT ? kEncFltMaxWarps * 32 : kEncThreads32, 1)
 // the same order as the general coder, so the streams are the same.
 constexpr int kEncChunkSyms = 256;
 
-template <typename SymT, bool ST>
+// PER: one row index per symbol, copied with the symbols into an index
+// ring (else one per chunk, read directly).
+template <typename SymT, bool ST, bool PER>
 __device__ __forceinline__ void encode_chunk_stream(const EncCtx &c, const RowMeta *meta,
                                                     const uint32_t *buckets, SymT *ring,
-                                                    int64_t s) {
+                                                    int32_t *iring, int64_t s) {
   using F = Rans64;
   using Word = typename F::Word;
   constexpr int GC = kEncChunkSyms / 32;
@@ -1268,16 +1270,23 @@ __device__ __forceinline__ void encode_chunk_stream(const EncCtx &c, const RowMe
   const SymT *src = reinterpret_cast<const SymT *>(c.sym) + d.base;
   const int32_t M = (int32_t)(d.n / kEncChunkSyms);
   const int ib = g.ib_shift;
-  // chunk ch's symbols into ring half ch & 1 (one commit group per call)
+  // chunk ch's symbols (PER: and rows) into ring half ch & 1 (one commit
+  // group per call)
   auto issue = [&](int32_t ch) {
     const char *gs = reinterpret_cast<const char *>(src + (int64_t)ch * kEncChunkSyms);
     char *ds = reinterpret_cast<char *>(ring + (ch & 1) * kEncChunkSyms);
 #pragma unroll
     for (int o = lane * 16; o < kChunkBytes; o += 32 * 16) cp_async16(ds + o, gs + o);
+    if (PER) {
+      const int32_t *gi = c.idx + d.base + (int64_t)ch * kEncChunkSyms;
+      int32_t *di = iring + (ch & 1) * kEncChunkSyms;
+#pragma unroll
+      for (int o = lane * 4; o < kEncChunkSyms; o += 128) cp_async16(di + o, gi + o);
+    }
     cp_async_commit();
   };
   auto row_at = [&](int32_t ch) -> uint32_t {
-    return (uint32_t)__ldg(c.idx + ((d.base + (int64_t)ch * kEncChunkSyms) >> ib));
+    return PER ? 0u : (uint32_t)__ldg(c.idx + ((d.base + (int64_t)ch * kEncChunkSyms) >> ib));
   };
   WarpEnc<F> st;
   st.x = F::kLow;
@@ -1300,16 +1309,21 @@ __device__ __forceinline__ void encode_chunk_stream(const EncCtx &c, const RowMe
     }
     cp_async_wait<1>();
     __syncwarp();
-    st.rmax = max(st.rmax, r);
-    const RowMeta m = row_meta(meta, min(r, kmax));
     const SymT *rs = ring + (ch & 1) * kEncChunkSyms;
+    const int32_t *ri = iring + (ch & 1) * kEncChunkSyms;
+    // group j's row metadata: the chunk's, or (PER) each lane's own
+    auto meta_j = [&](int j) -> RowMeta {
+      const uint32_t rj = PER ? (uint32_t)ri[j * 32 + lane] : r;
+      st.rmax = max(st.rmax, rj);
+      return row_meta(meta, min(rj, kmax));
+    };
     const typename F::State xs = st.x;
     const uint32_t cs = st.cursor;
     uint32_t esc = 0;
     uint32_t be[GC];
 #pragma unroll
     for (int j = GC - 1; j >= 0; --j) {
-      const EncBucket bk = enc_bucket<ST>((int32_t)rs[j * 32 + lane], m, buckets);
+      const EncBucket bk = enc_bucket<ST>((int32_t)rs[j * 32 + lane], meta_j(j), buckets);
       esc |= bk.in_range ? 0u : 1u;
       be[j] = bk.e;
     }
@@ -1327,7 +1341,7 @@ __device__ __forceinline__ void encode_chunk_stream(const EncCtx &c, const RowMe
       st.cursor = cs;
 #pragma unroll 1
       for (int j = GC - 1; j >= 0; --j) {
-        const EncBucket bk = enc_bucket<ST>((int32_t)rs[j * 32 + lane], m, buckets);
+        const EncBucket bk = enc_bucket<ST>((int32_t)rs[j * 32 + lane], meta_j(j), buckets);
         const EncLook L = enc_look<F>(bk, true, sh);
         const typename F::State xg = st.x;
         const uint32_t cg = st.cursor;
@@ -1354,7 +1368,14 @@ __device__ __forceinline__ void encode_chunk_stream(const EncCtx &c, const RowMe
 
 constexpr int kEncChunkMaxWarps = 32;  // a 2^28-symbol sweep's 8,192 streams in two rounds
 
-template <typename SymT, bool ST>
+// Shared memory per warp: the two-half symbol ring, and (PER) the two-half
+// index ring.
+template <typename SymT, bool PER>
+__host__ __device__ constexpr uint32_t enc_chunk_warp_bytes() {
+  return 2u * kEncChunkSyms * (uint32_t)sizeof(SymT) + (PER ? 2u * kEncChunkSyms * 4u : 0u);
+}
+
+template <typename SymT, bool ST, bool PER>
 __global__ void __launch_bounds__(kEncChunkMaxWarps * 32, 1) encode_chunk_kernel(EncCtx c) {
   extern __shared__ __align__(16) unsigned char smem[];
   __shared__ uint64_t bar;
@@ -1371,12 +1392,13 @@ __global__ void __launch_bounds__(kEncChunkMaxWarps * 32, 1) encode_chunk_kernel
   const uint32_t tab = enc_table_bytes(ST ? 2 : 1, c);
   const int warp = threadIdx.x >> 5, nwarp = blockDim.x >> 5;
   const uint32_t sbase = smem_addr(smem);
-  const uint32_t rbase = ((sbase + tab + 127u) & ~127u) +
-                         (uint32_t)warp * (2u * kEncChunkSyms * (uint32_t)sizeof(SymT));
+  const uint32_t rbase = ((sbase + tab + 127u) & ~127u) + (uint32_t)warp * enc_chunk_warp_bytes<SymT, PER>();
   SymT *ring = reinterpret_cast<SymT *>(smem + (rbase - sbase));
+  int32_t *iring = reinterpret_cast<int32_t *>(smem + (rbase - sbase) +
+                                               2u * kEncChunkSyms * (uint32_t)sizeof(SymT));
   for (int64_t k = blockIdx.x + (int64_t)gridDim.x * warp; k < c.g.S;
        k += (int64_t)gridDim.x * nwarp)
-    encode_chunk_stream<SymT, ST>(c, meta, buckets, ring, k);
+    encode_chunk_stream<SymT, ST, PER>(c, meta, buckets, ring, iring, k);
 }
 
 // Whether a tiled W = 32 encode can take the tile-staged kernel (the
@@ -1457,21 +1479,22 @@ int launch_encode_tile(const EncCtx &c, int mode, const int32_t *indexes, const 
 bool enc_chunk_path_ok(const EncCtx &c, int mode, int sym_dtype, const void *symbols) {
   const Geom &g = c.g;
   if (g.kind != RANS_CHUNK_CONTIG || g.W != 32 || g.alias || g.fmt != RANS_FMT_RANS64 ||
-      (mode != 1 && mode != 2) || g.ib_shift < 8)
+      (mode != 1 && mode != 2) || (g.ib_shift != 0 && g.ib_shift < 8))
     return false;
+  if (g.ib_shift == 0 && (reinterpret_cast<uintptr_t>(c.idx) & 15) != 0) return false;
   if (sym_dtype != RANS_SYM_UINT8 && sym_dtype != RANS_SYM_INT16 && sym_dtype != RANS_SYM_INT32)
     return false;
   if (g.per < kEncChunkSyms || g.per % kEncChunkSyms != 0 || g.n != g.S * g.per) return false;
   return (reinterpret_cast<uintptr_t>(symbols) & 15) == 0;
 }
 
-template <typename SymT>
+template <typename SymT, bool PER>
 int launch_encode_chunk(const EncCtx &c, int mode, cudaStream_t st) {
   const Geom &g = c.g;
   int dev = 0;
   cudaGetDevice(&dev);
   const uint32_t tab = enc_table_bytes(mode, c);
-  const uint32_t per_warp = 2u * kEncChunkSyms * (uint32_t)sizeof(SymT);
+  const uint32_t per_warp = enc_chunk_warp_bytes<SymT, PER>();
   const uint32_t lim = (uint32_t)smem_optin(dev) - 64u;
   if (tab + 128u + per_warp > lim) return kNotTaken;
   const int sms = num_sms(dev);
@@ -1481,7 +1504,7 @@ int launch_encode_chunk(const EncCtx &c, int mode, cudaStream_t st) {
   if (warps > room) warps = room;
   if (warps < 1) warps = 1;
   const uint32_t smem = tab + 128u + (uint32_t)warps * per_warp;
-  auto kern = mode == 2 ? encode_chunk_kernel<SymT, true> : encode_chunk_kernel<SymT, false>;
+  auto kern = mode == 2 ? encode_chunk_kernel<SymT, true, PER> : encode_chunk_kernel<SymT, false, PER>;
   if (ensure_dyn_smem((const void *)kern, smem) != cudaSuccess) return RANS_ERR_CUDA;
   int fit = 0;
   if (blocks_per_sm(&fit, (const void *)kern, (int)warps * 32, smem) != cudaSuccess || fit < 1)
@@ -1885,9 +1908,15 @@ int launch_encode(const void *symbols, int sym_dtype, const int32_t *indexes,
   c.stab_smem = 0;
   const int mode = t.enc_in_smem;
   if (enc_chunk_path_ok(c, mode, sym_dtype, symbols)) {
-    const int r = sym_dtype == RANS_SYM_UINT8   ? launch_encode_chunk<uint8_t>(c, mode, st)
-                  : sym_dtype == RANS_SYM_INT16 ? launch_encode_chunk<int16_t>(c, mode, st)
-                                                : launch_encode_chunk<int32_t>(c, mode, st);
+    const bool per = g.ib_shift == 0;
+    const int r = sym_dtype == RANS_SYM_UINT8
+                      ? (per ? launch_encode_chunk<uint8_t, true>(c, mode, st)
+                             : launch_encode_chunk<uint8_t, false>(c, mode, st))
+                  : sym_dtype == RANS_SYM_INT16
+                      ? (per ? launch_encode_chunk<int16_t, true>(c, mode, st)
+                             : launch_encode_chunk<int16_t, false>(c, mode, st))
+                      : (per ? launch_encode_chunk<int32_t, true>(c, mode, st)
+                             : launch_encode_chunk<int32_t, false>(c, mode, st));
     if (r != kNotTaken) return r;
   }
   if (enc_tile_path_ok(c, mode, sym_dtype, indexes, symbols)) {
