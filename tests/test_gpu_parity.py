@@ -211,13 +211,14 @@ def test_sweep_uint8_blocks():
     _check_streams(WL.sweep(log2_n=20, n_streams=32))
 
 
+@pytest.mark.parametrize("block", [256, 1])
 @pytest.mark.parametrize("dtype", [np.uint8, np.int16, np.int32])
-def test_chunked_contiguous_streams(dtype):
+def test_chunked_contiguous_streams(dtype, block):
     """Contiguous streams of whole 256-symbol chunks with one row per 256
-    symbols (the chunked coders): uint8, int16 and int32 symbols on rows
-    shorter than the alphabet, and far values, so that chunks with escapes
-    are coded again on the escape path."""
-    w = WL.sweep(log2_n=16, n_streams=8, block=256)
+    symbols or one per symbol (the chunked coders): uint8, int16 and int32
+    symbols on rows shorter than the alphabet, and far values, so that
+    chunks with escapes are coded again on the escape path."""
+    w = WL.sweep(log2_n=16, n_streams=8, block=block)
     w["pmf_lengths"] = np.full(16, 200, dtype=np.int32)
     sym = np.asarray(w["symbols"]).astype(dtype)
     if dtype != np.uint8:
