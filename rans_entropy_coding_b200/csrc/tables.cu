@@ -339,14 +339,27 @@ __device__ __forceinline__ const double *gauss_u_table(double *U, int cap, int c
   return U;
 }
 
-constexpr uint32_t kGaussSmemBytes = 32768;  // u table (and the fused kernel's row)
+// Dynamic shared memory of the row kernels: the u table (kUTabBytes, Gaussian
+// rows only), then the row being quantised (kRowBufEntries entries; longer
+// rows are quantised in place in global memory).
+constexpr uint32_t kUTabBytes = 32768;
+constexpr int kRowBufEntries = 8192;
+constexpr uint32_t kRowBufBytes = 4u * kRowBufEntries;
+constexpr uint32_t kGaussSmemBytes = kUTabBytes + kRowBufBytes;
+static_assert((2u << kMaxQ) <= kUTabBytes, "a row's slot buckets (16-bit) fit in the u table");
+
+// Copies a row quantised in shared memory out to its global row.
+__device__ __forceinline__ void write_row(int32_t *row, const int32_t *work, int len) {
+  for (int j = threadIdx.x; j < len; j += blockDim.x) row[j] = work[j];
+}
 
 __global__ void __launch_bounds__(kRowThreads)
     gaussian_rows_kernel(const float *scales, double tail, int prec, int32_t *cdfs, int Lmax,
                          int32_t *lengths, int32_t *offsets) {
-  extern __shared__ double utab[];
+  extern __shared__ __align__(16) double utab[];
   __shared__ BlockScratch sh;
   __shared__ QuantScratch qs;
+  int32_t *rbuf = reinterpret_cast<int32_t *>(utab + kUTabBytes / 8);
   const int r = blockIdx.x;
   int32_t *row = cdfs + (size_t)r * (size_t)Lmax;
   int32_t c = 0;
@@ -355,9 +368,11 @@ __global__ void __launch_bounds__(kRowThreads)
   if (st == RANS_OK && len > Lmax) st = RANS_ERR_CAPACITY;
   if (st == RANS_OK) {
     const double sd = (double)scales[r];
-    const double *U = gauss_u_table(utab, (int)(kGaussSmemBytes / 8), c, sd);
+    const double *U = gauss_u_table(utab, (int)(kUTabBytes / 8), c, sd);
     GaussPmf pf{c, 2 * c + 1, sd, 1u << prec, U};
-    st = quantise_row(pf, 2 * c + 2, row, sh, qs, 1u << prec);
+    int32_t *work = len <= kRowBufEntries ? rbuf : row;
+    st = quantise_row(pf, 2 * c + 2, work, sh, qs, 1u << prec);
+    if (st == RANS_OK && work != row) write_row(row, work, len);
   }
   for (int j = (st == RANS_OK ? len : 0) + threadIdx.x; j < Lmax; j += kRowThreads) row[j] = 0;
   if (threadIdx.x == 0) {
@@ -369,6 +384,7 @@ __global__ void __launch_bounds__(kRowThreads)
 __global__ void __launch_bounds__(kRowThreads)
     pmf_rows_kernel(const float *pmfs, int stride, const int32_t *pmf_lengths,
                     const float *tail, int prec, int32_t *cdfs, int Lmax, int32_t *lengths) {
+  extern __shared__ __align__(16) int32_t rbuf[];
   __shared__ BlockScratch sh;
   __shared__ QuantScratch qs;
   const int r = blockIdx.x;
@@ -379,7 +395,9 @@ __global__ void __launch_bounds__(kRowThreads)
   else if (n + 2 > Lmax) st = RANS_ERR_CAPACITY;
   if (st == RANS_OK) {
     GivenPmf pf{pmfs + (size_t)r * (size_t)stride, n, tail[r], 1u << prec};
-    st = quantise_row(pf, n + 1, row, sh, qs, 1u << prec);
+    int32_t *work = n + 2 <= kRowBufEntries ? rbuf : row;
+    st = quantise_row(pf, n + 1, work, sh, qs, 1u << prec);
+    if (st == RANS_OK && work != row) write_row(row, work, n + 2);
   }
   for (int j = (st == RANS_OK ? n + 2 : 0) + threadIdx.x; j < Lmax; j += kRowThreads) row[j] = 0;
   if (threadIdx.x == 0) lengths[r] = st ? st : n + 2;
@@ -429,13 +447,45 @@ __device__ __forceinline__ int bucket_of(const int32_t *row, int nb, int v, uint
   return lo;
 }
 
+// A slot-filling launch counts its bitmap words and search flag in the
+// build words of the table set's header (zero between launches); its last
+// block to finish publishes them in the words the coders read
+// (kChunkUsedWord, kSearchFlagWord) and clears the build words, so no launch
+// needs a reset before it.
+constexpr uint32_t kBuildUsedWord = 18;    // bitmap words handed out so far
+constexpr uint32_t kBuildSearchWord = 19;  // 1 once a slot of the launch searches
+constexpr uint32_t kBuildDoneWord = 20;    // blocks of the launch that have finished
+
 // Where a table set's bitmap words go: they follow the slots of all rows.
 struct ChunkArea {
-  uint32_t base;      // slot-word index of the first bitmap word
-  uint32_t cap;       // bitmap words available
-  uint32_t *used;     // header counter of words handed out
-  uint32_t *search;   // header flag: some slot fell back to searching
+  uint32_t base;  // slot-word index of the first bitmap word
+  uint32_t cap;   // bitmap words available
+  uint32_t *hdr;  // the table set's header words (the build words)
 };
+
+// Ends a slot-filling launch: every thread of every block calls it once,
+// after its last bitmap allocation.  The last block to arrive publishes the
+// build's bitmap count and search flag and clears the build words for the
+// next launch.
+__device__ void finish_build(const ChunkArea &ca) {
+  __threadfence();
+  __syncthreads();
+  if (threadIdx.x != 0) return;
+  const uint32_t blocks = gridDim.x * gridDim.y * gridDim.z;
+  if (atomicAdd(ca.hdr + kBuildDoneWord, 1u) != blocks - 1) return;
+  __threadfence();
+  // both build words read and cleared in one round trip
+  uint32_t used, search;
+  asm volatile(
+      "atom.relaxed.gpu.global.exch.b32 %0, [%2], 0;\n\t"
+      "atom.relaxed.gpu.global.exch.b32 %1, [%3], 0;"
+      : "=r"(used), "=r"(search)
+      : "l"(ca.hdr + kBuildUsedWord), "l"(ca.hdr + kBuildSearchWord)
+      : "memory");
+  ca.hdr[kChunkUsedWord] = used;
+  ca.hdr[kSearchFlagWord] = search;
+  ca.hdr[kBuildDoneWord] = 0u;
+}
 
 // Slots are filled kSlotsPerThread consecutive ones per thread, each from
 // two binary searches (the buckets holding its first and last cumulative
@@ -468,9 +518,12 @@ __device__ __forceinline__ uint32_t boundary_bits(const int32_t *row, int nb, in
 // memory, entries scaled by << sh).
 // SPT slots per thread, blockDim.x apart (so that a warp's stores stay
 // coalesced), their searches independent of one another.
-template <int SPT = kSlotsPerThread>
+// LO: lo_tab holds the bucket of every slot's first value (slot_lo_table),
+// else each slot searches the row for it.
+template <int SPT = kSlotsPerThread, bool LO = false>
 __device__ void fill_slot_block(const int32_t *row, int nb, uint32_t slot0, int w, int nslots,
-                                int tb, uint32_t *slots, const ChunkArea &ca, uint32_t sh) {
+                                int tb, uint32_t *slots, const ChunkArea &ca, uint32_t sh,
+                                const uint16_t *lo_tab = nullptr) {
   const int lane = threadIdx.x & 31;
   const int t0 = tb + (int)threadIdx.x;
   const uint32_t nch = w > 16 ? (uint32_t)(w >> 4) : 1u;  // bitmap words of a slot
@@ -482,13 +535,14 @@ __device__ void fill_slot_block(const int32_t *row, int nb, uint32_t slot0, int 
 #pragma unroll
   for (int u = 0; u < SPT; ++u) {
     const int t = t0 + u * (int)blockDim.x;
-    lo[u] = t < nslots ? bucket_of(row, nb, t * w, sh) : 0;
+    lo[u] = t < nslots ? (LO ? (int)lo_tab[t] : bucket_of(row, nb, t * w, sh)) : 0;
   }
 #pragma unroll
   for (int u = 0; u < SPT; ++u) {
     const int t = t0 + u * (int)blockDim.x;
     int next = __shfl_down_sync(kFull, lo[u], 1);
-    if (lane == 31 && t + 1 < nslots) next = bucket_of(row, nb, (t + 1) * w, sh);
+    if (lane == 31 && t + 1 < nslots)
+      next = LO ? (int)lo_tab[t + 1] : bucket_of(row, nb, (t + 1) * w, sh);
     hi[u] = 0;
     if (t < nslots) {
       hi[u] = t + 1 >= nslots ? nb - 1 : ((row[next] << sh) == (t + 1) * w ? next - 1 : next);
@@ -504,7 +558,7 @@ __device__ void fill_slot_block(const int32_t *row, int nb, uint32_t slot0, int 
   }
   const uint32_t wtot = __shfl_sync(kFull, incl, 31);
   uint32_t wbase = 0;
-  if (lane == 31 && wtot > 0) wbase = atomicAdd(ca.used, wtot);
+  if (lane == 31 && wtot > 0) wbase = atomicAdd(ca.hdr + kBuildUsedWord, wtot);
   uint32_t at = __shfl_sync(kFull, wbase, 31) + incl - need;
 #pragma unroll
   for (int u = 0; u < SPT; ++u) {
@@ -534,7 +588,7 @@ __device__ void fill_slot_block(const int32_t *row, int nb, uint32_t slot0, int 
         }
         word = (p & 0xffffu) | (255u << 16) | ((p >> 16) << 24);
       } else {
-        *ca.search = 1u;
+        ca.hdr[kBuildSearchWord] = 1u;
         const uint32_t e2 = (uint32_t)(inside - 3);
         word = (uint32_t)lo[u] | ((e2 + 1u) << 16) | (e2 << 24);
       }
@@ -542,6 +596,21 @@ __device__ void fill_slot_block(const int32_t *row, int nb, uint32_t slot0, int 
     }
     slots[slot0 + t] = word;
   }
+}
+
+// The bucket holding each slot's first value, for all 2^(16 - shift) slots of
+// a row with nb buckets (entries scaled by << sh, strictly increasing, row[0]
+// = 0 and row[nb] << sh = 65536), into lo_tab: bucket j holds the slots t
+// with row[j] <= t * 2^shift < row[j + 1], so the buckets hand out every slot
+// exactly once.  Every thread of the block calls it (it ends on a barrier).
+__device__ __forceinline__ void slot_lo_table(const int32_t *row, int nb, int shift,
+                                              uint16_t *lo_tab, uint32_t sh) {
+  const int w1 = (1 << shift) - 1;
+  for (int j = threadIdx.x; j < nb; j += blockDim.x) {
+    const int te = ((row[j + 1] << sh) + w1) >> shift;
+    for (int t = ((row[j] << sh) + w1) >> shift; t < te; ++t) lo_tab[t] = (uint16_t)j;
+  }
+  __syncthreads();
 }
 
 // Copies n row entries into shared memory with cp.async (every copy in
@@ -602,28 +671,25 @@ __global__ void __launch_bounds__(kSlotThreads)
   const int r = blockIdx.y;
   const RowMeta m = meta[r * kMetaCopies];
   const int len = lengths[r];
-  if (len != (int)m.maxv + 2) {
-    if (threadIdx.x == 0 && blockIdx.x == 0) report(status, RANS_ERR_TABLE, r);
-    return;
-  }
   const int32_t *row = cdfs + (size_t)r * (size_t)Lmax;
-  const int nb = len - 1;
   const int32_t top = (int32_t)(kTotal >> sh);
-  if (row[0] != 0 || row[len - 1] != top) {
+  // (the conditions are the same on every thread of the block)
+  if (len != (int)m.maxv + 2 || row[0] != 0 || row[len - 1] != top) {
     if (threadIdx.x == 0 && blockIdx.x == 0) report(status, RANS_ERR_TABLE, r);
-    return;
-  }
-  if (blockIdx.x == 0) {
-    const int32_t *prow = row;
-    if (len <= kRowSmem) {
-      stage_row(srow, row, len);
-      prow = srow;
+  } else {
+    if (blockIdx.x == 0) {
+      const int32_t *prow = row;
+      if (len <= kRowSmem) {
+        stage_row(srow, row, len);
+        prow = srow;
+      }
+      if (threadIdx.x < kMetaCopies) meta[r * kMetaCopies + threadIdx.x].offset = offsets[r];
+      pack_row(prow, len, m.bucket_base, sh, buckets, starts, status, r);
+      __syncthreads();  // the staged row is staged again below
     }
-    if (threadIdx.x < kMetaCopies) meta[r * kMetaCopies + threadIdx.x].offset = offsets[r];
-    pack_row(prow, len, m.bucket_base, sh, buckets, starts, status, r);
-    __syncthreads();  // the staged row is staged again below
+    fill_row_slots(row, len - 1, slot_base(m.slot), (int)slot_shift(m.slot), slots, ca, srow, sh);
   }
-  fill_row_slots(row, nb, slot_base(m.slot), (int)slot_shift(m.slot), slots, ca, srow, sh);
+  finish_build(ca);
 }
 
 // The slot fill of rans_tables_prepare (rows already validated by
@@ -636,36 +702,40 @@ __global__ void __launch_bounds__(kSlotThreads)
   const RowMeta m = meta[r * kMetaCopies];
   const int32_t *row = cdfs + (size_t)r * (size_t)Lmax;
   const int len = lengths[r];
-  if (len < 2 || row[0] != 0 || row[len - 1] != (int32_t)(kTotal >> sh)) return;
-  fill_row_slots(row, len - 1, slot_base(m.slot), (int)slot_shift(m.slot), slots, ca, srow, sh);
+  if (len >= 2 && row[0] == 0 && row[len - 1] == (int32_t)(kTotal >> sh))
+    fill_row_slots(row, len - 1, slot_base(m.slot), (int)slot_shift(m.slot), slots, ca, srow, sh);
+  finish_build(ca);
 }
 
 // rans_build_cdfs_from_scales and rans_tables_refresh in one launch: block r
 // quantises Gaussian row r as gaussian_rows_kernel does, then rewrites the
 // row's offset, packed buckets, starts and every lookup slot of the row as
-// refresh_kernel does, from the row it has just written (staged in shared
-// memory).  A row that cannot be built, or whose length differs from the
+// refresh_kernel does, from the row it has just written (in shared memory
+// when it fits).  A row that cannot be built, or whose length differs from the
 // prepared layout, records RANS_ERR_TABLE in the blob's status word.
 __global__ void __launch_bounds__(kRowThreads)
     gaussian_refresh_kernel(const float *scales, double tail, int prec, int32_t *cdfs, int Lmax,
                             int32_t *lengths, int32_t *offsets, RowMeta *meta, uint32_t *buckets,
                             uint16_t *starts, uint32_t *slots, ChunkArea ca, int32_t *status) {
-  extern __shared__ __align__(16) int32_t srow[];
+  extern __shared__ __align__(16) double utab[];
   __shared__ BlockScratch sh;
   __shared__ QuantScratch qs;
+  int32_t *rbuf = reinterpret_cast<int32_t *>(utab + kUTabBytes / 8);
   const int r = blockIdx.x;
   int32_t *row = cdfs + (size_t)r * (size_t)Lmax;
   int32_t c = 0;
   int st = gaussian_center(scales[r], tail, &c);
   const int len = 2 * c + 3;
   if (st == RANS_OK && len > Lmax) st = RANS_ERR_CAPACITY;
+  // the row is quantised in shared memory when it fits, and packed and
+  // sliced from there
+  int32_t *work = len <= kRowBufEntries ? rbuf : row;
   if (st == RANS_OK) {
-    // the u table in the space the row is staged in below
     const double sd = (double)scales[r];
-    const double *U = gauss_u_table(reinterpret_cast<double *>(srow),
-                                    (int)(kSlotSmemBytes / 8), c, sd);
+    const double *U = gauss_u_table(utab, (int)(kUTabBytes / 8), c, sd);
     GaussPmf pf{c, 2 * c + 1, sd, 1u << prec, U};
-    st = quantise_row(pf, 2 * c + 2, row, sh, qs, 1u << prec);
+    st = quantise_row(pf, 2 * c + 2, work, sh, qs, 1u << prec);
+    if (st == RANS_OK && work != row) write_row(row, work, len);
   }
   for (int j = (st == RANS_OK ? len : 0) + threadIdx.x; j < Lmax; j += kRowThreads) row[j] = 0;
   if (threadIdx.x == 0) {
@@ -676,20 +746,28 @@ __global__ void __launch_bounds__(kRowThreads)
   const RowMeta m = meta[r * kMetaCopies];
   if (st != RANS_OK || len != (int)m.maxv + 2) {
     if (threadIdx.x == 0) report(status, RANS_ERR_TABLE, r);
-    return;
+  } else {
+    const uint32_t ssh = (uint32_t)(kPrec - prec);
+    // (quantise_row ends on a barrier: the row is complete)
+    if (threadIdx.x < kMetaCopies) meta[r * kMetaCopies + threadIdx.x].offset = -c;
+    pack_row(work, len, m.bucket_base, ssh, buckets, starts, status, r);
+    const int shift = (int)slot_shift(m.slot);
+    const int nslots = 1 << (16 - shift);
+    if (work == rbuf) {
+      // the slots' first buckets from the row's buckets, in the space of the
+      // u table (2^14 slots at most)
+      uint16_t *lo_tab = reinterpret_cast<uint16_t *>(utab);
+      slot_lo_table(work, len - 1, shift, lo_tab, ssh);
+      for (int tb = 0; tb < nslots; tb += kRowThreads * 4)
+        fill_slot_block<4, true>(work, len - 1, slot_base(m.slot), 1 << shift, nslots, tb, slots,
+                                 ca, ssh, lo_tab);
+    } else {
+      for (int tb = 0; tb < nslots; tb += kRowThreads * 4)
+        fill_slot_block<4>(work, len - 1, slot_base(m.slot), 1 << shift, nslots, tb, slots, ca,
+                           ssh);
+    }
   }
-  const uint32_t ssh = (uint32_t)(kPrec - prec);
-  const int32_t *prow = row;  // (quantise_row ends on a barrier: the row is written)
-  if (len <= kRowSmem) {
-    stage_row(srow, row, len);
-    prow = srow;
-  }
-  if (threadIdx.x < kMetaCopies) meta[r * kMetaCopies + threadIdx.x].offset = -c;
-  pack_row(prow, len, m.bucket_base, ssh, buckets, starts, status, r);
-  const int shift = (int)slot_shift(m.slot);
-  const int nslots = 1 << (16 - shift);
-  for (int tb = 0; tb < nslots; tb += kRowThreads * 4)
-    fill_slot_block<4>(prow, len - 1, slot_base(m.slot), 1 << shift, nslots, tb, slots, ca, ssh);
+  finish_build(ca);
 }
 
 // Alias tables, one row per block (the reading of the alias method given
@@ -810,6 +888,8 @@ int launch_gaussian_lengths(const float *scales, int K, double tail, int32_t *le
 
 int launch_gaussian_rows(const float *scales, int K, double tail, int prec, int32_t *cdfs,
                          int Lmax, int32_t *lengths, int32_t *offsets, cudaStream_t st) {
+  if (ensure_dyn_smem((const void *)gaussian_rows_kernel, kGaussSmemBytes) != cudaSuccess)
+    return RANS_ERR_CUDA;
   gaussian_rows_kernel<<<K, kRowThreads, kGaussSmemBytes, st>>>(scales, tail, prec, cdfs, Lmax,
                                                                 lengths, offsets);
   return cudaGetLastError() == cudaSuccess ? RANS_OK : RANS_ERR_CUDA;
@@ -818,7 +898,7 @@ int launch_gaussian_rows(const float *scales, int K, double tail, int prec, int3
 int launch_pmf_rows(const float *pmfs, int K, int stride, const int32_t *pmf_lengths,
                     const float *tail, int prec, int32_t *cdfs, int Lmax, int32_t *lengths,
                     cudaStream_t st) {
-  pmf_rows_kernel<<<K, kRowThreads, 0, st>>>(pmfs, stride, pmf_lengths, tail, prec, cdfs, Lmax,
+  pmf_rows_kernel<<<K, kRowThreads, kRowBufBytes, st>>>(pmfs, stride, pmf_lengths, tail, prec, cdfs, Lmax,
                                               lengths);
   return cudaGetLastError() == cudaSuccess ? RANS_OK : RANS_ERR_CUDA;
 }
@@ -850,9 +930,7 @@ int refresh_tables(const int32_t *cdfs, int K, int Lmax, const int32_t *lengths,
   ChunkArea ca;
   ca.base = (uint32_t)t.n_slots;
   ca.cap = t.slot_bytes / 4 - (uint32_t)t.n_slots;
-  ca.used = reinterpret_cast<uint32_t *>(b) + kChunkUsedWord;
-  ca.search = reinterpret_cast<uint32_t *>(b) + kSearchFlagWord;
-  if (cudaMemsetAsync(ca.used, 0, 8, st) != cudaSuccess) return RANS_ERR_CUDA;
+  ca.hdr = reinterpret_cast<uint32_t *>(b);
   // blocks of kSlotsPerBlock slots, enough for the table's largest row
   // (blocks past a smaller row's slots return at once)
   const int qmax = t.max_slot_log2 >= kMinQ && t.max_slot_log2 <= kMaxQ ? t.max_slot_log2 : kMaxQ;
@@ -878,10 +956,10 @@ int refresh_tables_from_scales(const float *scales, int K, double tail, int32_t 
   ChunkArea ca;
   ca.base = (uint32_t)t.n_slots;
   ca.cap = t.slot_bytes / 4 - (uint32_t)t.n_slots;
-  ca.used = reinterpret_cast<uint32_t *>(b) + kChunkUsedWord;
-  ca.search = reinterpret_cast<uint32_t *>(b) + kSearchFlagWord;
-  if (cudaMemsetAsync(ca.used, 0, 8, st) != cudaSuccess) return RANS_ERR_CUDA;
-  gaussian_refresh_kernel<<<K, kRowThreads, kSlotSmemBytes, st>>>(
+  ca.hdr = reinterpret_cast<uint32_t *>(b);
+  if (ensure_dyn_smem((const void *)gaussian_refresh_kernel, kGaussSmemBytes) != cudaSuccess)
+    return RANS_ERR_CUDA;
+  gaussian_refresh_kernel<<<K, kRowThreads, kGaussSmemBytes, st>>>(
       scales, tail, t.precision, cdfs, Lmax, lengths, offsets, dmeta, dbuckets, dstarts, dslots,
       ca, status);
   return cudaGetLastError() == cudaSuccess ? RANS_OK : RANS_ERR_CUDA;
@@ -1073,8 +1151,7 @@ int prepare_tables(const int32_t *cdfs, int K, int Lmax, const int32_t *lengths,
   ChunkArea ca;
   ca.base = (uint32_t)sbase;
   ca.cap = (uint32_t)(slot_bytes / 4 - sbase);
-  ca.used = reinterpret_cast<uint32_t *>(b) + kChunkUsedWord;
-  ca.search = reinterpret_cast<uint32_t *>(b) + kSearchFlagWord;
+  ca.hdr = reinterpret_cast<uint32_t *>(b);
   fill_slots_kernel<<<grid, kSlotThreads, kSlotSmemBytes, st>>>(cdfs, Lmax, dmeta, lengths, sh,
                                                                  dslots, ca);
   if (cudaGetLastError() != cudaSuccess) return RANS_ERR_CUDA;
