@@ -71,8 +71,8 @@ def parse():
     ap.add_argument("--alias", action="store_true",
                     help="alias-coded streams (rows of power-of-two bucket counts, W <= 8)")
     ap.add_argument("--eager", action="store_true",
-                    help="call the entry points every step instead of replaying each phase "
-                         "from a CUDA graph captured once")
+                    help="call the entry points every step instead of replaying the step "
+                         "(its phases and their timing events) from a CUDA graph")
     return ap.parse_args()
 
 
@@ -425,30 +425,39 @@ def run_ours(args, world, rank, local):
 
     phases = [phase_tables, phase_encode, phase_decode]
 
-    def step(e=None):
+    def step_body(e=None):
+        cur = torch.cuda.current_stream()
         if flush is not None:
             flush.fill_(1)
         for k, ph in enumerate(phases):
-            if e: e[k].record(stream)
+            if e: e[k].record(cur)
             ph()
-        if e: e[3].record(stream)
+        if e: e[3].record(cur)
 
     for _ in range(max(args.warmup, 0)):
-        step()
+        step_body()
     torch.cuda.synchronize()
+    steps = [lambda e=e: step_body(e) for e in ev]
     if not args.eager:
-        # every phase captured once into a CUDA graph (the same kernels on the
-        # same buffers), then replayed each step: one host launch per phase
+        # a step (the L2 flush if any, then the three phases) captured into
+        # one CUDA graph, its phase events recorded as graph nodes between
+        # them; one graph per timed step, so that each keeps its own events:
+        # a step is one host launch
+        ev = [[torch.cuda.Event(enable_timing=True, external=True) for _ in range(4)]
+              for _ in range(args.steps)]
         cap = torch.cuda.Stream(dev)
-        graphs = []
-        for ph in list(phases):
+
+        def capture(e):
             gr = torch.cuda.CUDAGraph()
             with torch.cuda.graph(gr, stream=cap):
-                ph()
-            graphs.append(gr)
-        phases = [gr.replay for gr in graphs]
+                step_body(e)
+            return gr
+
+        warm = capture(None)
+        graphs = [capture(e) for e in ev]
+        steps = [gr.replay for gr in graphs]
         for _ in range(max(args.warmup, 0)):
-            step()
+            warm.replay()
         torch.cuda.synchronize()
     rb.check(rb.rans_get_status(ws.enc), "encode status")
     rb.check(rb.rans_get_status(ws.dec), "decode status")
@@ -463,7 +472,7 @@ def run_ours(args, world, rank, local):
         barrier(world)
         t0.record(stream)
         for i in range(args.steps):
-            step(ev[i])
+            steps[i]()
         t1.record(stream)
         torch.cuda.synchronize()
         barrier(world)
@@ -633,7 +642,7 @@ def run_ours(args, world, rank, local):
                        "interleave": w["W"], "rows": K,
                        "lmax": Lmax,
                        "launch": "eager calls" if args.eager else
-                                 "each phase replayed from a CUDA graph captured once",
+                                 "each step one CUDA graph (its phases and their events)",
                        "parallelism": ("shard-by-stream-range x%d" if split else
                                        "shard-by-image x%d") % world,
                        "l2": ("inputs larger than L2 (%d MB read per encode)" %
@@ -687,21 +696,42 @@ def run_float(args, world, rank, local):
     stream = torch.cuda.current_stream()
     ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
 
-    def step(e=None):
-        if e: e[0].record(stream)
+    def step_body(e=None):
+        cur = torch.cuda.current_stream()
+        if e: e[0].record(cur)
         rb.check(rb.rans_tables_refresh_from_scales(table, tail, cdfs, lengths, offsets, tables),
                  "tables")
-        if e: e[1].record(stream)
+        if e: e[1].record(cur)
         rb.check(rb.rans_encode_from_scales(y, mu, sc, n, table, bound, tables, ch, ws.out,
                                             ws.offsets, ws.enc), "encode")
-        if e: e[2].record(stream)
+        if e: e[2].record(cur)
         rb.check(rb.rans_decode_to_values(ws.out, ws.offsets, sc, mu, n, table, bound, tables,
                                           ch, vals, ws.dec), "decode")
-        if e: e[3].record(stream)
+        if e: e[3].record(cur)
 
     for _ in range(max(args.warmup, 0)):
-        step()
+        step_body()
     torch.cuda.synchronize()
+    steps = [lambda e=e: step_body(e) for e in ev]
+    if not args.eager:
+        # one CUDA graph per timed step, its phase events graph nodes (as the
+        # integer workloads)
+        ev = [[torch.cuda.Event(enable_timing=True, external=True) for _ in range(4)]
+              for _ in range(args.steps)]
+        cap = torch.cuda.Stream(dev)
+
+        def capture(e):
+            gr = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(gr, stream=cap):
+                step_body(e)
+            return gr
+
+        warm = capture(None)
+        graphs = [capture(e) for e in ev]
+        steps = [gr.replay for gr in graphs]
+        for _ in range(max(args.warmup, 0)):
+            warm.replay()
+        torch.cuda.synchronize()
     for what, b in (("encode", ws.enc), ("decode", ws.dec), ("tables", tables.blob)):
         rb.check(rb.rans_get_status(b), what + " status")
     assert torch.equal(vals, want), "round trip failed"
@@ -713,7 +743,7 @@ def run_float(args, world, rank, local):
         barrier(world)
         t0.record(stream)
         for i in range(args.steps):
-            step(ev[i])
+            steps[i]()
         t1.record(stream)
         torch.cuda.synchronize()
         barrier(world)
@@ -752,6 +782,8 @@ def run_float(args, world, rank, local):
             "config": {"workload": workload_name(w, args), "symbols_per_gpu": n,
                        "streams_per_gpu": S, "channel_group": args.group, "interleave": 32,
                        "rows": K, "lmax": Lmax, "parallelism": "shard-by-image x%d" % world,
+                       "launch": "eager calls" if args.eager else
+                                 "each step one CUDA graph (its phases and their events)",
                        "l2": "inputs larger than L2 (%d MB read per encode)" % (n * 12 >> 20)},
             "encode": {"ms": enc_ms, "gsym_s": n / enc_ms / 1e6, "GBps": enc_gbs,
                        "frac_hbm": enc_gbs / peak, "alg_bytes": alg_enc},

@@ -464,16 +464,23 @@ struct ChunkArea {
 };
 
 // Ends a slot-filling launch: every thread of every block calls it once,
-// after its last bitmap allocation.  The last block to arrive publishes the
-// build's bitmap count and search flag and clears the build words for the
-// next launch.
+// after its last bitmap allocation.  The build words are only touched by
+// atomics; the block barrier puts every thread's before thread 0's
+// increment of the done counter, whose release (with the barrier) makes them
+// visible to the block that acquires the last increment.  That block
+// publishes the build's bitmap count and search flag and clears the build
+// words for the next launch.  (No thread waits for its slot stores here:
+// only the next launch reads them.)
 __device__ void finish_build(const ChunkArea &ca) {
-  __threadfence();
   __syncthreads();
   if (threadIdx.x != 0) return;
   const uint32_t blocks = gridDim.x * gridDim.y * gridDim.z;
-  if (atomicAdd(ca.hdr + kBuildDoneWord, 1u) != blocks - 1) return;
-  __threadfence();
+  uint32_t done;
+  asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], 1;"
+               : "=r"(done)
+               : "l"(ca.hdr + kBuildDoneWord)
+               : "memory");
+  if (done != blocks - 1) return;
   // both build words read and cleared in one round trip
   uint32_t used, search;
   asm volatile(
@@ -588,7 +595,7 @@ __device__ void fill_slot_block(const int32_t *row, int nb, uint32_t slot0, int 
         }
         word = (p & 0xffffu) | (255u << 16) | ((p >> 16) << 24);
       } else {
-        ca.hdr[kBuildSearchWord] = 1u;
+        atomicExch(ca.hdr + kBuildSearchWord, 1u);
         const uint32_t e2 = (uint32_t)(inside - 3);
         word = (uint32_t)lo[u] | ((e2 + 1u) << 16) | (e2 << 24);
       }
