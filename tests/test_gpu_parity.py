@@ -401,8 +401,43 @@ def test_encoder_reports_bad_index_and_capacity():
 
 def _header(tables):
     """The blob header's words (an internal layout: word 16 counts the bitmap
-    words handed out, word 17 flags slots that search)."""
+    words the last slot fill handed out, word 17 flags slots that search,
+    words 18-20 are a slot fill's own counters, zero between launches)."""
     return tables.blob[:256].view(torch.int32).cpu().numpy()
+
+
+def test_refreshes_publish_and_clear_build_words():
+    """Slot-filling launches count their bitmap words and search flag in build
+    words (header words 18, 19; word 20 counts finished blocks) that the last
+    block publishes in words 16 and 17 and clears, with no reset between
+    launches: repeated refreshes, fused or from rows, report the count of a
+    fresh prepare and leave the build words at zero, and the tables still
+    code like the oracle."""
+    w = WL.y_latent(W=32)
+    scales = np.asarray(w["scales"], np.float32)
+    tail = w["tail_mass"]
+    c, l, o = O.build_cdfs_from_scales(scales, tail)
+    tables = tables_from_numpy(c, l, o)
+    h0 = _header(tables)
+    assert h0[16] > 0 and h0[17] == 0 and not h0[18:21].any()
+    K, Lmax = c.shape
+    dcd = torch.zeros((K, Lmax), dtype=torch.int32, device="cuda")
+    dl = torch.zeros(K, dtype=torch.int32, device="cuda")
+    do = torch.zeros(K, dtype=torch.int32, device="cuda")
+    dsc = torch.from_numpy(scales).cuda()
+    for k in range(6):
+        if k % 2 == 0:
+            rb.check(rb.rans_tables_refresh_from_scales(dsc, tail, dcd, dl, do, tables))
+        else:
+            rb.check(rb.rans_tables_refresh(dcd, dl, do, tables))
+        h = _header(tables)
+        assert rb.rans_get_status(tables.blob) == rb.OK
+        assert h[16] == h0[16] and h[17] == 0 and not h[18:21].any(), (k, h[16:21])
+    assert np.array_equal(dcd.cpu().numpy(), c)
+    data, offs, dec, _, _ = gpu_encode_decode(w, tables)
+    want, woffs = oracle_encode(w, c, l, o)
+    assert offs.tolist() == woffs.tolist() and np.array_equal(data, want)
+    assert np.array_equal(dec, np.asarray(w["symbols"]).reshape(-1))
 
 
 @pytest.mark.parametrize("W", [1, 32])
