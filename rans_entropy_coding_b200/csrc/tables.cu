@@ -465,9 +465,9 @@ struct ChunkArea {
 
 // Ends a slot-filling launch: every thread of every block calls it once,
 // after its last bitmap allocation.  The build words are only touched by
-// atomics; the block barrier puts every thread's before thread 0's
-// increment of the done counter, whose release (with the barrier) makes them
-// visible to the block that acquires the last increment.  That block
+// atomics; the block barrier orders every thread's build-word atomics before
+// thread 0's increment of the done counter, whose release (with the barrier)
+// makes them visible to the block that acquires the last increment.  That block
 // publishes the build's bitmap count and search flag and clears the build
 // words for the next launch.  (No thread waits for its slot stores here:
 // only the next launch reads them.)
