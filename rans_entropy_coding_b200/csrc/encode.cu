@@ -1247,11 +1247,14 @@ __global__ void __launch_bounds__(FLT ? kEncFltMaxWarps * 32 : kEncThreads32, 1)
 constexpr int kEncChunkSyms = 256;
 
 // PER: one row index per symbol, copied with the symbols into an index
-// ring (else one per chunk, read directly).
-template <typename SymT, bool ST, bool PER>
+// ring (else one per chunk, read directly).  RCP: rtab holds every bucket's
+// divisor reciprocal (F::rcp of its width, the same double), read beside
+// its bucket word instead of computed per group.
+template <typename SymT, bool ST, bool PER, bool RCP = false>
 __device__ __forceinline__ void encode_chunk_stream(const EncCtx &c, const RowMeta *meta,
                                                     const uint32_t *buckets, SymT *ring,
-                                                    int32_t *iring, int64_t s) {
+                                                    int32_t *iring, int64_t s,
+                                                    const double *rtab = nullptr) {
   using F = Rans64;
   using Word = typename F::Word;
   constexpr int GC = kEncChunkSyms / 32;
@@ -1320,19 +1323,28 @@ __device__ __forceinline__ void encode_chunk_stream(const EncCtx &c, const RowMe
     const typename F::State xs = st.x;
     const uint32_t cs = st.cursor;
     uint32_t esc = 0;
-    uint32_t be[GC];
+    uint32_t be[GC];  // bucket words, or (RCP) bucket indexes
 #pragma unroll
     for (int j = GC - 1; j >= 0; --j) {
-      const EncBucket bk = enc_bucket<ST>((int32_t)rs[j * 32 + lane], meta_j(j), buckets);
-      esc |= bk.in_range ? 0u : 1u;
-      be[j] = bk.e;
+      if constexpr (RCP) {
+        const RowMeta m = meta_j(j);
+        const int64_t v = (int64_t)rs[j * 32 + lane] - (int64_t)m.offset;
+        const bool in = (uint64_t)v < (uint64_t)m.maxv;
+        esc |= in ? 0u : 1u;
+        be[j] = m.bucket_base + (in ? (uint32_t)v : m.maxv);
+      } else {
+        const EncBucket bk = enc_bucket<ST>((int32_t)rs[j * 32 + lane], meta_j(j), buckets);
+        esc |= bk.in_range ? 0u : 1u;
+        be[j] = bk.e;
+      }
     }
 #pragma unroll
     for (int j = GC - 1; j >= 0; --j) {
       EncLook L;
-      L.start = bucket_start(be[j]);
-      L.freq = bucket_freq(be[j]);
-      L.rcp = F::rcp(L.freq, sh);
+      const uint32_t e = RCP ? buckets[be[j]] : be[j];
+      L.start = bucket_start(e);
+      L.freq = bucket_freq(e);
+      L.rcp = RCP ? rtab[be[j]] : F::rcp(L.freq, sh);
       enc_group_fast<F, true>(st, L, true, above, end, sh);
     }
     if (__any_sync(kFull, esc != 0)) {
@@ -1375,8 +1387,14 @@ __host__ __device__ constexpr uint32_t enc_chunk_warp_bytes() {
   return 2u * kEncChunkSyms * (uint32_t)sizeof(SymT) + (PER ? 2u * kEncChunkSyms * 4u : 0u);
 }
 
-template <typename SymT, bool ST, bool PER>
+// Bytes of the bucket reciprocal table (RCP): one double per bucket word.
+__host__ __device__ inline uint32_t enc_rcp_bytes(const EncCtx &c) {
+  return 2u * c.bucket_bytes;
+}
+
+template <typename SymT, bool ST, bool PER, bool RCP = false>
 __global__ void __launch_bounds__(kEncChunkMaxWarps * 32, 1) encode_chunk_kernel(EncCtx c) {
+  static_assert(!RCP || !ST, "reciprocals beside bucket words");
   extern __shared__ __align__(16) unsigned char smem[];
   __shared__ uint64_t bar;
   const char *gb = c.blob + kHeaderBytes;
@@ -1389,7 +1407,17 @@ __global__ void __launch_bounds__(kEncChunkMaxWarps * 32, 1) encode_chunk_kernel
   }
   const RowMeta *meta = reinterpret_cast<const RowMeta *>(smem);
   const uint32_t *buckets = reinterpret_cast<const uint32_t *>(smem + c.meta_bytes);
-  const uint32_t tab = enc_table_bytes(ST ? 2 : 1, c);
+  uint32_t tab = enc_table_bytes(ST ? 2 : 1, c);
+  double *rtab = nullptr;
+  if constexpr (RCP) {
+    // every bucket's reciprocal, after the tables (16-byte aligned: the
+    // tables' sizes are multiples of 16)
+    rtab = reinterpret_cast<double *>(smem + tab);
+    for (uint32_t j = threadIdx.x; j < c.bucket_bytes / 4u; j += blockDim.x)
+      rtab[j] = Rans64::rcp(bucket_freq(buckets[j]), 0u);
+    __syncthreads();
+    tab += enc_rcp_bytes(c);
+  }
   const int warp = threadIdx.x >> 5, nwarp = blockDim.x >> 5;
   const uint32_t sbase = smem_addr(smem);
   const uint32_t rbase = ((sbase + tab + 127u) & ~127u) + (uint32_t)warp * enc_chunk_warp_bytes<SymT, PER>();
@@ -1398,7 +1426,7 @@ __global__ void __launch_bounds__(kEncChunkMaxWarps * 32, 1) encode_chunk_kernel
                                                2u * kEncChunkSyms * (uint32_t)sizeof(SymT));
   for (int64_t k = blockIdx.x + (int64_t)gridDim.x * warp; k < c.g.S;
        k += (int64_t)gridDim.x * nwarp)
-    encode_chunk_stream<SymT, ST, PER>(c, meta, buckets, ring, iring, k);
+    encode_chunk_stream<SymT, ST, PER, RCP>(c, meta, buckets, ring, iring, k, rtab);
 }
 
 // Whether a tiled W = 32 encode can take the tile-staged kernel (the
@@ -1500,11 +1528,19 @@ int launch_encode_chunk(const EncCtx &c, int mode, cudaStream_t st) {
   const int sms = num_sms(dev);
   int64_t warps = (g.S + sms - 1) / sms;
   if (warps > kEncChunkMaxWarps) warps = kEncChunkMaxWarps;
-  const int64_t room = ((int64_t)lim - tab - 128) / per_warp;
+  // every bucket's reciprocal in shared memory too (chunk rows, bucket
+  // words) when it costs no warps
+  const uint32_t rcp = enc_rcp_bytes(c);
+  const bool use_rcp = !PER && mode == 1 && tab % 16u == 0 &&
+                       (int64_t)tab + rcp + 128 + warps * per_warp <= (int64_t)lim;
+  const uint32_t tabr = tab + (use_rcp ? rcp : 0u);
+  const int64_t room = ((int64_t)lim - tabr - 128) / per_warp;
   if (warps > room) warps = room;
   if (warps < 1) warps = 1;
-  const uint32_t smem = tab + 128u + (uint32_t)warps * per_warp;
-  auto kern = mode == 2 ? encode_chunk_kernel<SymT, true, PER> : encode_chunk_kernel<SymT, false, PER>;
+  const uint32_t smem = tabr + 128u + (uint32_t)warps * per_warp;
+  auto kern = mode == 2 ? encode_chunk_kernel<SymT, true, PER>
+                        : (use_rcp ? encode_chunk_kernel<SymT, false, PER, !PER>
+                                   : encode_chunk_kernel<SymT, false, PER>);
   if (ensure_dyn_smem((const void *)kern, smem) != cudaSuccess) return RANS_ERR_CUDA;
   int fit = 0;
   if (blocks_per_sm(&fit, (const void *)kern, (int)warps * 32, smem) != cudaSuccess || fit < 1)
