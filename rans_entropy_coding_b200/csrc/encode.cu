@@ -1529,10 +1529,12 @@ int launch_encode_chunk(const EncCtx &c, int mode, cudaStream_t st) {
   int64_t warps = (g.S + sms - 1) / sms;
   if (warps > kEncChunkMaxWarps) warps = kEncChunkMaxWarps;
   // every bucket's reciprocal in shared memory too (chunk rows, bucket
-  // words) when it costs no warps
+  // words) when it costs no warps and the CTA is wide enough to build it
+  // quickly (at most 16 reciprocals a thread)
   const uint32_t rcp = enc_rcp_bytes(c);
   const bool use_rcp = !PER && mode == 1 && tab % 16u == 0 &&
-                       (int64_t)tab + rcp + 128 + warps * per_warp <= (int64_t)lim;
+                       (int64_t)tab + rcp + 128 + warps * per_warp <= (int64_t)lim &&
+                       (int64_t)(c.bucket_bytes / 4u) <= 16 * 32 * warps;
   const uint32_t tabr = tab + (use_rcp ? rcp : 0u);
   const int64_t room = ((int64_t)lim - tabr - 128) / per_warp;
   if (warps > room) warps = room;
