@@ -1309,10 +1309,13 @@ __device__ __forceinline__ void tile_origin(const Geom &g, const StreamDesc &d, 
 // ring (word i at win[i mod kWinWords]), rd: the next word to read.
 // SEARCH: a table with slots that ran out of bitmap room; those slots take
 // the general lookup's binary search (a branch, entered once per warp).
-template <bool SEARCH>
+// BW: the bucket's start and width from its bucket word (start | (width -
+// 1) << 16, one load) instead of two 16-bit starts.
+template <bool SEARCH, bool BW = false>
 __device__ __forceinline__ int32_t dec_group_win64(uint64_t &x, uint32_t &rd, const RowMeta &m,
                                                    const uint16_t *starts, const uint32_t *slots,
-                                                   const uint32_t *win, uint32_t &esc) {
+                                                   const uint32_t *win, uint32_t &esc,
+                                                   const uint32_t *bwords = nullptr) {
   const uint32_t xl = (uint32_t)x, xh = (uint32_t)(x >> 32);
   const uint32_t cum = xl & 0xffffu;
   uint32_t sym;
@@ -1334,8 +1337,16 @@ __device__ __forceinline__ int32_t dec_group_win64(uint64_t &x, uint32_t &rd, co
   }
   esc |= sym == m.maxv ? 1u : 0u;
   const uint32_t a = m.bucket_base + sym;
-  const uint32_t s0 = starts[a], s1 = starts[a + 1];
-  const uint32_t f = (s1 - s0) + (s1 == 0u ? 65536u : 0u);
+  uint32_t s0, f;
+  if constexpr (BW) {
+    const uint32_t e = bwords[a];
+    s0 = e & 0xffffu;
+    f = (e >> 16) + 1u;
+  } else {
+    const uint32_t s1 = starts[a + 1];
+    s0 = starts[a];
+    f = (s1 - s0) + (s1 == 0u ? 65536u : 0u);
+  }
   // x' = f (x >> 16) + cum - start in 32-bit halves; refill when x' < 2^31
   const uint32_t tl = __funnelshift_r(xl, xh, 16), th = xh >> 16;
   const uint64_t p = (uint64_t)f * tl + (uint64_t)(cum - s0);
@@ -1693,11 +1704,12 @@ __host__ __device__ constexpr uint32_t chunk_warp_bytes() {
          (PER ? 2u * (uint32_t)kChunkSyms * 4u : 0u);
 }
 
-template <typename SymT, bool SEARCH, bool PER>
+template <typename SymT, bool SEARCH, bool PER, bool BW = false>
 __device__ __forceinline__ void decode_chunk_stream(const DecCtx &c, const RowMeta *meta,
                                                     const uint16_t *starts,
                                                     const uint32_t *slots, uint32_t *win,
-                                                    SymT *oring, int32_t *iring, int64_t s) {
+                                                    SymT *oring, int32_t *iring, int64_t s,
+                                                    const uint32_t *bwords = nullptr) {
   constexpr int GC = kChunkSyms / 32;
   const int lane = threadIdx.x & 31;
   const Geom &g = c.g;
@@ -1777,7 +1789,7 @@ __device__ __forceinline__ void decode_chunk_stream(const DecCtx &c, const RowMe
     int32_t val[GC];
 #pragma unroll
     for (int j = 0; j < GC; ++j)
-      val[j] = dec_group_win64<SEARCH>(x, rd, ms[j], starts, slots, win, esc);
+      val[j] = dec_group_win64<SEARCH, BW>(x, rd, ms[j], starts, slots, win, esc, bwords);
     SymT *oh = oring + h * kChunkSyms;
     if (!__any_sync(kFull, esc != 0)) {
 #pragma unroll
@@ -1828,19 +1840,30 @@ constexpr int kChunkMaxWarps = 32;  // a 2^28-symbol sweep's 8,192 streams in tw
 // metadata fit in registers)
 constexpr int kChunkPerMaxWarps = 16;
 
-template <typename SymT, bool PER>
+// BW: the bucket words are staged too (the blob's meta, bucket words,
+// starts and slots in one range) and the fast path reads them.
+template <typename SymT, bool PER, bool BW = false>
 __global__ void __launch_bounds__((PER ? kChunkPerMaxWarps : kChunkMaxWarps) * 32, 1)
     decode_chunk_kernel(DecCtx c) {
   extern __shared__ __align__(16) unsigned char smem[];
   __shared__ uint64_t bar;
   const char *gb = c.blob + kHeaderBytes;
-  if (!stage_to_smem(smem, gb, c.meta_bytes, &bar, c.status, smem + c.meta_bytes,
-                     gb + c.meta_bytes + c.bucket_bytes, c.start_bytes + c.slot_bytes))
-    return;
+  const uint32_t bwb = BW ? c.bucket_bytes : 0u;  // staged bucket-word bytes
+  if (BW) {
+    if (!stage_to_smem(smem, gb, c.meta_bytes + c.bucket_bytes + c.start_bytes + c.slot_bytes,
+                       &bar, c.status))
+      return;
+  } else {
+    if (!stage_to_smem(smem, gb, c.meta_bytes, &bar, c.status, smem + c.meta_bytes,
+                       gb + c.meta_bytes + c.bucket_bytes, c.start_bytes + c.slot_bytes))
+      return;
+  }
   const RowMeta *meta = reinterpret_cast<const RowMeta *>(smem);
-  const uint16_t *starts = reinterpret_cast<const uint16_t *>(smem + c.meta_bytes);
-  const uint32_t *slots = reinterpret_cast<const uint32_t *>(smem + c.meta_bytes + c.start_bytes);
-  const uint32_t tab = c.meta_bytes + c.start_bytes + c.slot_bytes;
+  const uint32_t *bwords = BW ? reinterpret_cast<const uint32_t *>(smem + c.meta_bytes) : nullptr;
+  const uint16_t *starts = reinterpret_cast<const uint16_t *>(smem + c.meta_bytes + bwb);
+  const uint32_t *slots =
+      reinterpret_cast<const uint32_t *>(smem + c.meta_bytes + bwb + c.start_bytes);
+  const uint32_t tab = c.meta_bytes + bwb + c.start_bytes + c.slot_bytes;
   const int warp = threadIdx.x >> 5, nwarp = blockDim.x >> 5;
   // each warp's word window and value ring, 128-byte aligned
   const uint32_t sbase = smem_addr(smem);
@@ -1855,9 +1878,11 @@ __global__ void __launch_bounds__((PER ? kChunkPerMaxWarps : kChunkMaxWarps) * 3
   for (int64_t k = blockIdx.x + (int64_t)gridDim.x * warp; k < c.g.S;
        k += (int64_t)gridDim.x * nwarp) {
     if (search)
-      decode_chunk_stream<SymT, true, PER>(c, meta, starts, slots, win, oring, iring, k);
+      decode_chunk_stream<SymT, true, PER, BW>(c, meta, starts, slots, win, oring, iring, k,
+                                               bwords);
     else
-      decode_chunk_stream<SymT, false, PER>(c, meta, starts, slots, win, oring, iring, k);
+      decode_chunk_stream<SymT, false, PER, BW>(c, meta, starts, slots, win, oring, iring, k,
+                                                bwords);
   }
   if ((threadIdx.x & 31) == 0) tma::bulk_wait_all();
 }
@@ -1958,11 +1983,14 @@ int launch_decode_chunk(const DecCtx &c, cudaStream_t st) {
   int64_t warps = (g.S + sms - 1) / sms;
   const int64_t max_warps = PER ? kChunkPerMaxWarps : kChunkMaxWarps;
   if (warps > max_warps) warps = max_warps;
-  const int64_t room = ((int64_t)lim - tab - 128) / per_warp;
+  // the bucket words staged as well when that costs no warps
+  const bool bw = (int64_t)tab + c.bucket_bytes + 128 + warps * per_warp <= (int64_t)lim;
+  const uint32_t tabw = tab + (bw ? c.bucket_bytes : 0u);
+  const int64_t room = ((int64_t)lim - tabw - 128) / per_warp;
   if (warps > room) warps = room;
   if (warps < 1) warps = 1;
-  const uint32_t smem = tab + 128u + (uint32_t)warps * per_warp;
-  auto kern = decode_chunk_kernel<SymT, PER>;
+  const uint32_t smem = tabw + 128u + (uint32_t)warps * per_warp;
+  auto kern = bw ? decode_chunk_kernel<SymT, PER, true> : decode_chunk_kernel<SymT, PER>;
   if (ensure_dyn_smem((const void *)kern, smem) != cudaSuccess) return RANS_ERR_CUDA;
   int fit = 0;
   if (blocks_per_sm(&fit, (const void *)kern, (int)warps * 32, smem) != cudaSuccess || fit < 1)
