@@ -187,33 +187,47 @@ __device__ int quantise_row(const PF &pf, int n, int32_t *row, BlockScratch &sh,
     const unsigned long long R = Z - below;
     const unsigned long long full = R / (unsigned long long)(t - 1);
     const unsigned long long part = R % (unsigned long long)(t - 1);
-    // rank of each width-t bucket among the width-t buckets, in index order
-    unsigned long long nt = 0;
-    for (int i = i0; i < i1; ++i) nt += row[i + 1] == t;
+    // the final widths and the CDF in one scan: each thread counts its
+    // width-t buckets (nt) and adds up its other buckets' final widths (a:
+    // 1 below t, their own above); the width-t buckets before it (rank r <
+    // rk0, in index order) end at 1 below rank `full`, t - part at it and t
+    // above, which sums to g(rk0) in closed form.  (Both counts stay below
+    // 2^32, so one 64-bit scan carries them as two halves.)
+    unsigned long long nt = 0, a = 0;
+    for (int i = i0; i < i1; ++i) {
+      const long long w = row[i + 1];
+      nt += w == t;
+      a += w == t ? 0ull : (w < t ? 1ull : (unsigned long long)w);
+    }
     unsigned long long tot;
-    unsigned long long rk = block_excl_scan(nt, sh, &tot);
+    const unsigned long long ex = block_excl_scan((a << 32) | nt, sh, &tot);
+    unsigned long long rk = ex & 0xffffffffull;
+    const unsigned long long g =
+        (rk < full ? rk : full) +
+        (rk > full ? (unsigned long long)t - part + (rk - full - 1) * (unsigned long long)t : 0ull);
+    unsigned long long run = (ex >> 32) + g;
     for (int i = i0; i < i1; ++i) {
       long long w = row[i + 1];
-      if (w > 1 && w < t) {
-        w = 1;
-      } else if (w == t) {
+      if (w == t) {
         if (rk < full) w = 1;
         else if (rk == full) w -= (long long)part;
         ++rk;
+      } else if (w < t) {
+        w = 1;
       }
-      if (w == 0) w = 1;
-      row[i + 1] = (int32_t)w;
+      run += (unsigned long long)w;
+      row[i + 1] = (int32_t)run;
     }
-  }
-
-  // widths -> CDF in place
-  unsigned long long wl = 0;
-  for (int i = i0; i < i1; ++i) wl += (uint32_t)row[i + 1];
-  unsigned long long tot;
-  unsigned long long run = block_excl_scan(wl, sh, &tot);
-  for (int i = i0; i < i1; ++i) {
-    run += (uint32_t)row[i + 1];
-    row[i + 1] = (int32_t)run;
+  } else {
+    // widths -> CDF in place
+    unsigned long long wl = 0;
+    for (int i = i0; i < i1; ++i) wl += (uint32_t)row[i + 1];
+    unsigned long long tot;
+    unsigned long long run = block_excl_scan(wl, sh, &tot);
+    for (int i = i0; i < i1; ++i) {
+      run += (uint32_t)row[i + 1];
+      row[i + 1] = (int32_t)run;
+    }
   }
   if (threadIdx.x == 0) row[0] = 0;
   __syncthreads();
