@@ -65,12 +65,6 @@ __device__ unsigned long long block_excl_scan(unsigned long long v, BlockScratch
   return ex;
 }
 
-__device__ unsigned long long block_sum(unsigned long long v, BlockScratch &sh) {
-  unsigned long long t;
-  block_excl_scan(v, sh, &t);
-  return t;
-}
-
 // Scaled and rounded probability: round(p * total) half away from zero
 // (total = 2^precision), or -1 when p is negative, not finite or too large.
 __device__ __forceinline__ long long scaled_freq(float p, uint32_t total) {
@@ -127,11 +121,17 @@ __device__ int quantise_row(const PF &pf, int n, int32_t *row, BlockScratch &sh,
   int bad = 0;
   const unsigned long long local = pf.eval(i0, i1, row + 1, bad);
   q.hist[threadIdx.x] = 0;
-  if (threadIdx.x == 0) q.nbig = 0;
+  if (threadIdx.x == 0) {
+    q.nbig = 0;
+    sh.total = 0;  // (no threshold found yet; nothing else writes it before)
+  }
+  // a thread with a bad value adds 2^52 to the total: the rounded values are
+  // below 2^32 and at most 2^16 of them, so a good total stays below 2^48,
+  // and 1024 flags add up below 2^63
   unsigned long long T;
-  const unsigned long long before = block_excl_scan(local, sh, &T);
-  bad = __syncthreads_or(bad);
-  if (bad || T == 0) return RANS_ERR_TABLE;
+  const unsigned long long before =
+      block_excl_scan(local + (bad ? 1ull << 52 : 0ull), sh, &T);
+  if (T == 0 || (T >> 52) != 0) return RANS_ERR_TABLE;
 
   // pass 2: widths of the rescaled running sum floor(total c / T); count the
   // empty buckets and the widths of the others
@@ -151,15 +151,19 @@ __device__ int quantise_row(const PF &pf, int n, int32_t *row, BlockScratch &sh,
       else if (w >= (uint32_t)kBins) q.big[atomicAdd(&q.nbig, 1u)] = w;
     }
   }
-  const unsigned long long Z = block_sum(zl, sh);  // (its barriers also publish q)
+  __syncthreads();  // every thread's bins and wide buckets are in
+  // one scan gives Z (the empty buckets, high half) and, over the bins
+  // (thread b = width b), S(b - 1) and S(kBins - 1) (low half): both sums
+  // stay below 2^32
+  const unsigned int b = threadIdx.x;
+  const unsigned long long vb = b >= 2 ? (unsigned long long)(b - 1) * q.hist[b] : 0ull;
+  unsigned long long zs;
+  const unsigned long long exz = block_excl_scan((zl << 32) | vb, sh, &zs);
+  const unsigned long long Z = zs >> 32;
   if (Z > 0) {
     // t below kBins: the bin whose running S(t) first reaches Z
-    const unsigned int b = threadIdx.x;
-    const unsigned long long vb = b >= 2 ? (unsigned long long)(b - 1) * q.hist[b] : 0ull;
-    unsigned long long s_all;
-    const unsigned long long sb = block_excl_scan(vb, sh, &s_all);  // S(b - 1)
-    if (threadIdx.x == 0) sh.total = 0;
-    __syncthreads();
+    const unsigned long long sb = exz & 0xffffffffull;     // S(b - 1)
+    const unsigned long long s_all = zs & 0xffffffffull;   // S(kBins - 1)
     if (vb > 0 && sb < Z && sb + vb >= Z) {
       sh.total = b;
       sh.aux = sb;
@@ -180,9 +184,8 @@ __device__ int quantise_row(const PF &pf, int n, int32_t *row, BlockScratch &sh,
       }
     }
     __syncthreads();
-    const long long t = (long long)sh.total;
+    const long long t = (long long)sh.total;  // (not written again: no barrier after)
     const unsigned long long below = sh.aux;
-    __syncthreads();
     if (t == 0) return RANS_ERR_TABLE;  // nothing left to steal from
     const unsigned long long R = Z - below;
     const unsigned long long full = R / (unsigned long long)(t - 1);
