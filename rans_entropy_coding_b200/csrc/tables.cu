@@ -242,14 +242,24 @@ __device__ __forceinline__ double std_normal_cdf(double z) {
   return 0.5 * erfc(-z / sqrt(2.0));
 }
 
-__device__ __forceinline__ int gaussian_center(float scale, double tail, int32_t *center) {
+// The centre ceil(scale m) of a Gaussian row, m = -Phi^-1(tail / 2) (m given:
+// gaussian_multiplier(tail)).
+__device__ __forceinline__ double gaussian_multiplier(double tail) {
+  return -normcdfinv(tail / 2.0);
+}
+
+__device__ __forceinline__ int gaussian_center_m(float scale, double tail, double m,
+                                                 int32_t *center) {
   if (!(scale > 0.0f) || !isfinite(scale) || !(tail > 0.0) || !(tail < 1.0))
     return RANS_ERR_ARG;
-  double m = -normcdfinv(tail / 2.0);
   double c = ceil((double)scale * m);
   if (!(c >= 0.0) || c > 32766.0) return RANS_ERR_ARG;
   *center = (int32_t)c;
   return RANS_OK;
+}
+
+__device__ __forceinline__ int gaussian_center(float scale, double tail, int32_t *center) {
+  return gaussian_center_m(scale, tail, gaussian_multiplier(tail), center);
 }
 
 __global__ void gaussian_lengths_kernel(const float *scales, int K, double tail,
@@ -472,6 +482,12 @@ __device__ __forceinline__ int bucket_of(const int32_t *row, int nb, int v, uint
 constexpr uint32_t kBuildUsedWord = 18;    // bitmap words handed out so far
 constexpr uint32_t kBuildSearchWord = 19;  // 1 once a slot of the launch searches
 constexpr uint32_t kBuildDoneWord = 20;    // blocks of the launch that have finished
+// The Gaussian multiplier m = -Phi^-1(tail / 2) of the last scale-table
+// refresh and its tail, two doubles (words 22-23 and 24-25; zero after
+// prepare, which no valid tail matches): the next refresh with the same tail
+// reads m instead of evaluating the inverse CDF in every block.
+constexpr uint32_t kTailKeyWord = 22;
+constexpr uint32_t kMultWord = 24;
 
 // Where a table set's bitmap words go: they follow the slots of all rows.
 struct ChunkArea {
@@ -488,7 +504,9 @@ struct ChunkArea {
 // publishes the build's bitmap count and search flag and clears the build
 // words for the next launch.  (No thread waits for its slot stores here:
 // only the next launch reads them.)
-__device__ void finish_build(const ChunkArea &ca) {
+// With `tail` in (0, 1) the last block also caches the multiplier `mult` of
+// that tail (every block has read the cache before it arrives).
+__device__ void finish_build(const ChunkArea &ca, double tail = 0.0, double mult = 0.0) {
   __syncthreads();
   if (threadIdx.x != 0) return;
   const uint32_t blocks = gridDim.x * gridDim.y * gridDim.z;
@@ -498,6 +516,11 @@ __device__ void finish_build(const ChunkArea &ca) {
                : "l"(ca.hdr + kBuildDoneWord)
                : "memory");
   if (done != blocks - 1) return;
+  if (tail > 0.0 && tail < 1.0) {
+    double *hd = reinterpret_cast<double *>(ca.hdr);
+    hd[kTailKeyWord / 2] = tail;
+    hd[kMultWord / 2] = mult;
+  }
   // both build words read and cleared in one round trip
   uint32_t used, search;
   asm volatile(
@@ -668,9 +691,10 @@ __device__ void fill_row_slots(const int32_t *grow, int nb, uint32_t slot0, int 
 // Row r's packed buckets and 16-bit starts from its len entries (row[0] = 0
 // and row[len - 1] << sh = 65536 checked by the caller); a bucket that is
 // not strictly increasing or out of range records RANS_ERR_TABLE.
+// With row_out, the row's entries are also copied there.
 __device__ __forceinline__ void pack_row(const int32_t *row, int len, uint32_t base,
                                          uint32_t sh, uint32_t *buckets, uint16_t *starts,
-                                         int32_t *status, int r) {
+                                         int32_t *status, int r, int32_t *row_out = nullptr) {
   const int32_t top = (int32_t)(kTotal >> sh);
   for (int j = threadIdx.x; j < len - 1; j += blockDim.x) {
     const int32_t a = row[j], b = row[j + 1];
@@ -680,7 +704,11 @@ __device__ __forceinline__ void pack_row(const int32_t *row, int len, uint32_t b
     }
     buckets[base + j] = bucket_word(a, b, sh);
   }
-  for (int j = threadIdx.x; j < len; j += blockDim.x) starts[base + j] = (uint16_t)(row[j] << sh);
+  for (int j = threadIdx.x; j < len; j += blockDim.x) {
+    const int32_t v = row[j];
+    starts[base + j] = (uint16_t)(v << sh);
+    if (row_out) row_out[j] = v;
+  }
 }
 
 // Rebuilds a prepared table set from new CDF rows with the same lengths:
@@ -747,19 +775,21 @@ __global__ void __launch_bounds__(kRowThreads)
   int32_t *rbuf = reinterpret_cast<int32_t *>(utab + kUTabBytes / 8);
   const int r = blockIdx.x;
   int32_t *row = cdfs + (size_t)r * (size_t)Lmax;
+  // the multiplier cached by the last refresh, when it had this tail
+  const double *hd = reinterpret_cast<const double *>(ca.hdr);
+  const double mult = hd[kTailKeyWord / 2] == tail ? hd[kMultWord / 2] : gaussian_multiplier(tail);
   int32_t c = 0;
-  int st = gaussian_center(scales[r], tail, &c);
+  int st = gaussian_center_m(scales[r], tail, mult, &c);
   const int len = 2 * c + 3;
   if (st == RANS_OK && len > Lmax) st = RANS_ERR_CAPACITY;
-  // the row is quantised in shared memory when it fits, and packed and
-  // sliced from there
+  // the row is quantised in shared memory when it fits, and packed, written
+  // out and sliced from there
   int32_t *work = len <= kRowBufEntries ? rbuf : row;
   if (st == RANS_OK) {
     const double sd = (double)scales[r];
     const double *U = gauss_u_table(utab, (int)(kUTabBytes / 8), c, sd);
     GaussPmf pf{c, 2 * c + 1, sd, 1u << prec, U};
     st = quantise_row(pf, 2 * c + 2, work, sh, qs, 1u << prec);
-    if (st == RANS_OK && work != row) write_row(row, work, len);
   }
   for (int j = (st == RANS_OK ? len : 0) + threadIdx.x; j < Lmax; j += kRowThreads) row[j] = 0;
   if (threadIdx.x == 0) {
@@ -769,12 +799,14 @@ __global__ void __launch_bounds__(kRowThreads)
   // (st is the same on every thread)
   const RowMeta m = meta[r * kMetaCopies];
   if (st != RANS_OK || len != (int)m.maxv + 2) {
+    if (st == RANS_OK && work != row) write_row(row, work, len);
     if (threadIdx.x == 0) report(status, RANS_ERR_TABLE, r);
   } else {
     const uint32_t ssh = (uint32_t)(kPrec - prec);
     // (quantise_row ends on a barrier: the row is complete)
     if (threadIdx.x < kMetaCopies) meta[r * kMetaCopies + threadIdx.x].offset = -c;
-    pack_row(work, len, m.bucket_base, ssh, buckets, starts, status, r);
+    pack_row(work, len, m.bucket_base, ssh, buckets, starts, status, r,
+             work != row ? row : nullptr);
     const int shift = (int)slot_shift(m.slot);
     const int nslots = 1 << (16 - shift);
     if (work == rbuf) {
@@ -791,7 +823,7 @@ __global__ void __launch_bounds__(kRowThreads)
                            ssh);
     }
   }
-  finish_build(ca);
+  finish_build(ca, tail, mult);
 }
 
 // Alias tables, one row per block (the reading of the alias method given
