@@ -440,6 +440,32 @@ def test_refreshes_publish_and_clear_build_words():
     assert np.array_equal(dec, np.asarray(w["symbols"]).reshape(-1))
 
 
+def test_refresh_multiplier_cache_follows_the_tail():
+    """The fused refresh keeps the Gaussian multiplier of its tail in the
+    table header and reuses it only for the same tail: refreshes of one
+    table set with alternating tail masses give the oracle's rows, lengths
+    and offsets for each tail."""
+    w = WL.y_latent(W=32)
+    scales = np.asarray(w["scales"], np.float32)
+    t0 = w["tail_mass"]
+    c, l, o = O.build_cdfs_from_scales(scales, t0)
+    tables = tables_from_numpy(c, l, o)
+    K, Lmax = c.shape
+    dcd = torch.zeros((K, Lmax), dtype=torch.int32, device="cuda")
+    dl = torch.zeros(K, dtype=torch.int32, device="cuda")
+    do = torch.zeros(K, dtype=torch.int32, device="cuda")
+    dsc = torch.from_numpy(scales).cuda()
+    for tail in (t0, 1e-6, 1e-6, 1e-4, t0, t0):
+        # (a tail other than t0 changes the row lengths: the table set
+        # refuses the layout, the rows are still written)
+        rb.check(rb.rans_tables_refresh_from_scales(dsc, tail, dcd, dl, do, tables))
+        c2, l2, o2 = O.build_cdfs_from_scales(scales, tail)
+        gc, gl, go = dcd.cpu().numpy(), dl.cpu().numpy(), do.cpu().numpy()
+        assert gl.tolist() == l2.tolist() and go.tolist() == o2.tolist(), tail
+        for r in range(K):
+            assert gc[r, :l2[r]].tolist() == c2[r, :l2[r]].tolist(), (tail, r)
+
+
 @pytest.mark.parametrize("W", [1, 32])
 def test_slots_without_bitmap_room_search(W):
     """Prepared in a blob with no room for boundary bitmaps, the slots that
